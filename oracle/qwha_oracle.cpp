@@ -1,0 +1,446 @@
+// TEST INFRASTRUCTURE -- not part of the product.
+//
+// A plain, slow, double-precision CPU statement of the Walsh-Hadamard adapter
+// (WHA) layer of "QWHA: Quantization-Aware Walsh-Hadamard Adaptation for
+// Parameter-Efficient Fine-Tuning on Large Language Models". Only the test
+// suite, the package smoke check and the benchmark's CPU-baseline leg load it.
+// It shares no code, header, table or helper with the CUDA library; the two are
+// compared on the same seeded inputs.
+//
+// Sources (page title, then section):
+//   [P1] papernotes.org "QWHA ...", 整体框架 (framework), 关键设计 1/2/3,
+//        损失函数 / 训练策略
+//   [P2] gist.science "Technical Summary: QWHA ...", 2.1 Adapter Design,
+//        2.2 Quantization-Aware Initialization
+//
+// Readings taken where the pages are silent (each also listed in the design
+// notes of the repository):
+//   * H is the Sylvester-ordered Walsh-Hadamard matrix, normalised to be
+//     orthonormal: H_n[i][j] = (-1)^popcount(i & j) / sqrt(n). Then H is
+//     symmetric and its own inverse, so the adapter update dW = F H^-1 [P1 设计1,
+//     P2 2.1] equals F H.
+//   * A layer whose d_in is not a power of two uses the block-diagonal matrix
+//     of d_in/n equal blocks H_n.
+//   * Forward Y = X W_Q^T + alpha X dW^T, with alpha the adapter scale
+//     [P1 训练策略: alpha ~ 1].
+//   * Backward, only c trainable [P1 整体框架]: dc_j = dL/dc_j and dX = dL/dX
+//     for L = <Y, dY>.
+//   * AdaAlloc [P1 设计2, P2 2.2]: the per-channel budget formula is lost from
+//     the page, so the budget is proportional to the error norm of the
+//     channel, ||dW_Q[i,:]||_2 (no calibration activations: X = I), after a
+//     floor of min_per_row per channel; rounding remainder to the channels
+//     chosen by `mode`; per-channel cap d_in with the surplus re-shared.
+//     Within a channel the largest |(dW_Q H)[i,k]| win, ties to the lower k;
+//     the values are the dense solution (dW_Q H)[i,k] [P1 设计3, x0].
+//   * Sums that decide an integer (the budgets) use a fixed pairwise tree in
+//     index order over the zero-padded power-of-two length, and the transform
+//     used for ranking runs its butterfly stages in the textbook order
+//     h = 1, 2, 4, ..., n/2 in double, unnormalised. This fixes every rounding
+//     so that a GPU implementation can reproduce E and the budgets bit for bit.
+//
+// Build: g++ -O2 -std=c++17 -ffp-contract=off -fPIC -shared -pthread
+// (never -ffast-math).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <numeric>
+#include <thread>
+#include <vector>
+
+namespace {
+
+int g_threads = 0;
+
+int thread_count() {
+  if (g_threads > 0) return g_threads;
+  const char *env = std::getenv("QWHA_ORACLE_THREADS");
+  int n = env ? std::atoi(env) : 0;
+  if (n <= 0) n = (int)std::thread::hardware_concurrency();
+  if (n <= 0) n = 1;
+  return n;
+}
+
+// Run f(i) for i in [0, n), split into contiguous static ranges.
+template <class F>
+void parallel_for(int64_t n, F f) {
+  int nt = thread_count();
+  if (n < 2 || nt == 1) {
+    for (int64_t i = 0; i < n; ++i) f(i);
+    return;
+  }
+  if ((int64_t)nt > n) nt = (int)n;
+  std::vector<std::thread> pool;
+  pool.reserve(nt);
+  for (int t = 0; t < nt; ++t) {
+    int64_t lo = n * t / nt, hi = n * (t + 1) / nt;
+    pool.emplace_back([lo, hi, &f] {
+      for (int64_t i = lo; i < hi; ++i) f(i);
+    });
+  }
+  for (auto &th : pool) th.join();
+}
+
+bool is_pow2(int64_t n) { return n > 0 && (n & (n - 1)) == 0; }
+
+// Entry (a, b) of the orthonormal Sylvester matrix H_n; inv = 1/sqrt(n).
+double hadamard_entry(double inv, int a, int b) {
+  int parity = __builtin_popcount((unsigned)(a & b)) & 1;
+  return parity ? -inv : inv;
+}
+
+// Entry (a, b) of the block-diagonal matrix made of equal blocks H_n.
+double blockdiag_entry(int n, double inv, int a, int b) {
+  if (a / n != b / n) return 0.0;
+  return hadamard_entry(inv, a % n, b % n);
+}
+
+double inv_sqrt(int n) { return 1.0 / std::sqrt((double)n); }
+
+bool shape_ok(int d, int n) { return d > 0 && is_pow2(n) && d % n == 0; }
+
+// Textbook in-place Walsh-Hadamard butterflies on one block of length n,
+// stages h = 1, 2, 4, ..., n/2: (x[j], x[j+h]) <- (x[j] + x[j+h], x[j] - x[j+h]).
+void butterflies(double *x, int n) {
+  for (int h = 1; h < n; h <<= 1)
+    for (int j = 0; j < n; ++j)
+      if ((j & h) == 0) {
+        double a = x[j], b = x[j + h];
+        x[j] = a + b;
+        x[j + h] = a - b;
+      }
+}
+
+// Pairwise sum in index order over the length rounded up to a power of two
+// (missing terms are zero): sum(v[0:m]) = sum(v[0:m/2]) + sum(v[m/2:m]).
+double pairwise_sum(const double *v, int64_t len) {
+  int64_t m = 1;
+  while (m < len) m <<= 1;
+  std::vector<double> buf(m, 0.0);
+  for (int64_t i = 0; i < len; ++i) buf[i] = v[i];
+  for (int64_t w = m; w > 1; w >>= 1)
+    for (int64_t i = 0; i < w / 2; ++i) buf[i] = buf[2 * i] + buf[2 * i + 1];
+  return buf[0];
+}
+
+// Dense dW = F H, F given in CSR by output row. [P1 设计1; P2 2.1: dW = F H^-1]
+void delta_w(int d_out, int d_in, int n, const int32_t *row_ptr, const int32_t *col_idx,
+             const double *coef, double *dW) {
+  const double inv = inv_sqrt(n);
+  parallel_for(d_out, [&](int64_t r) {
+    double *row = dW + r * (int64_t)d_in;
+    for (int k = 0; k < d_in; ++k) row[k] = 0.0;
+    for (int32_t j = row_ptr[r]; j < row_ptr[r + 1]; ++j)
+      for (int k = 0; k < d_in; ++k) row[k] += coef[j] * blockdiag_entry(n, inv, col_idx[j], k);
+  });
+}
+
+}  // namespace
+
+extern "C" {
+
+// Thread count override for timing (0 = automatic). Returns the count in use.
+int oracle_set_threads(int n) {
+  g_threads = n;
+  return thread_count();
+}
+
+// Dense orthonormal Sylvester Hadamard matrix H_n, n a power of two. [P2 2.1:
+// H is fixed in advance and never trained; P1 设计1: its entries are +-1 up to
+// the scale]
+int oracle_hadamard(int32_t n, double *H) {
+  if (!is_pow2(n)) return 1;
+  const double inv = inv_sqrt(n);
+  for (int a = 0; a < n; ++a)
+    for (int b = 0; b < n; ++b) H[(int64_t)a * n + b] = hadamard_entry(inv, a, b);
+  return 0;
+}
+
+// Z = X H by the definition of a matrix product with the dense (block-diagonal)
+// H. X is [rows, d] row-major.
+int oracle_transform_dense(const double *X, int64_t rows, int32_t d, int32_t n, double *Z) {
+  if (!shape_ok(d, n)) return 1;
+  const double inv = inv_sqrt(n);
+  parallel_for(rows, [&](int64_t t) {
+    const double *x = X + t * d;
+    double *z = Z + t * d;
+    for (int k = 0; k < d; ++k) {
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i) acc += x[i] * blockdiag_entry(n, inv, i, k);
+      z[k] = acc;
+    }
+  });
+  return 0;
+}
+
+// The fast transform [P1 设计1 and P2 2.1: because every entry of H is +-1, the
+// transform is a recursion of sums and differences with no multiplications],
+// per block of n, textbook stage order; then, if `normalize`, each output times
+// 1/sqrt(n).
+int oracle_fwht(const double *X, int64_t rows, int32_t d, int32_t n, int32_t normalize, double *Z) {
+  if (!shape_ok(d, n)) return 1;
+  const double inv = inv_sqrt(n);
+  parallel_for(rows, [&](int64_t t) {
+    std::vector<double> b(n);
+    for (int blk = 0; blk < d / n; ++blk) {
+      const double *x = X + t * d + (int64_t)blk * n;
+      double *z = Z + t * d + (int64_t)blk * n;
+      for (int i = 0; i < n; ++i) b[i] = x[i];
+      butterflies(b.data(), n);
+      for (int i = 0; i < n; ++i) z[i] = normalize ? b[i] * inv : b[i];
+    }
+  });
+  return 0;
+}
+
+// W_Q[i,k] = s[i,g] * (q[i,k] - z[i,g]) in single precision, g = k / group;
+// q[i,k] is bits [bits*k, bits*k + bits) of row i's little-endian bit stream
+// (row stride d_in*bits/8 bytes). Returned widened to double.
+int oracle_dequant(int32_t bits, int32_t group, int32_t d_out, int32_t d_in, const uint8_t *qweight,
+                   const float *scales, const uint8_t *zeros, double *Wq) {
+  if (bits < 1 || bits > 8 || group <= 0 || d_in % group || (d_in * bits) % 8) return 1;
+  const int64_t stride = (int64_t)d_in * bits / 8;
+  const int ng = d_in / group;
+  parallel_for(d_out, [&](int64_t i) {
+    const uint8_t *row = qweight + i * stride;
+    for (int k = 0; k < d_in; ++k) {
+      int q = 0;
+      for (int b = 0; b < bits; ++b) {
+        int64_t bit = (int64_t)bits * k + b;
+        q |= ((row[bit >> 3] >> (bit & 7)) & 1) << b;
+      }
+      float s = scales[i * ng + k / group];
+      float diff = (float)q - (float)zeros[i * ng + k / group];
+      float w = s * diff;
+      Wq[i * d_in + k] = (double)w;
+    }
+  });
+  return 0;
+}
+
+// Dense dW = F H for inspection by the tests.
+int oracle_delta_w(int32_t d_out, int32_t d_in, int32_t n, const int32_t *row_ptr,
+                   const int32_t *col_idx, const double *coef, double *dW) {
+  if (!shape_ok(d_in, n) || d_out <= 0) return 1;
+  delta_w(d_out, d_in, n, row_ptr, col_idx, coef, dW);
+  return 0;
+}
+
+// Forward of the adapted layer by its definition [P1 整体框架, P2 2.1]:
+//   Z = X H,   Y = X W_Q^T + alpha * X (F H)^T.
+// Wq may be null (adapter only). X [T, d_in]; Z [T, d_in] (nullable); Y [T, d_out].
+int oracle_adapter_fwd(int32_t d_out, int32_t d_in, int32_t n, const int32_t *row_ptr,
+                       const int32_t *col_idx, const double *coef, const double *Wq, const double *X,
+                       int64_t T, double alpha, double *Z, double *Y) {
+  if (!shape_ok(d_in, n) || d_out <= 0 || T < 0) return 1;
+  std::vector<double> dW((size_t)d_out * d_in);
+  delta_w(d_out, d_in, n, row_ptr, col_idx, coef, dW.data());
+  if (Z) oracle_transform_dense(X, T, d_in, n, Z);
+  parallel_for(T, [&](int64_t t) {
+    const double *x = X + t * d_in;
+    for (int r = 0; r < d_out; ++r) {
+      const double *a = dW.data() + (int64_t)r * d_in;
+      double base = 0.0, ad = 0.0;
+      if (Wq) {
+        const double *w = Wq + (int64_t)r * d_in;
+        for (int k = 0; k < d_in; ++k) base += x[k] * w[k];
+      }
+      for (int k = 0; k < d_in; ++k) ad += x[k] * a[k];
+      Y[t * d_out + r] = base + alpha * ad;
+    }
+  });
+  return 0;
+}
+
+// The same adapter output by the sparse route [P1 整体框架: F = Scatter(c, E)]:
+//   Y_ad[t, r] = alpha * sum over nonzeros j of row r of c_j * (X H)[t, k_j],
+// with X H from the fast transform. Used to cross-check the dense route.
+int oracle_adapter_fwd_sparse(int32_t d_out, int32_t d_in, int32_t n, const int32_t *row_ptr,
+                              const int32_t *col_idx, const double *coef, const double *X, int64_t T,
+                              double alpha, double *Y) {
+  if (!shape_ok(d_in, n) || d_out <= 0 || T < 0) return 1;
+  std::vector<double> Z((size_t)T * d_in);
+  oracle_fwht(X, T, d_in, n, 1, Z.data());
+  parallel_for(T, [&](int64_t t) {
+    const double *z = Z.data() + t * d_in;
+    for (int r = 0; r < d_out; ++r) {
+      double acc = 0.0;
+      for (int32_t j = row_ptr[r]; j < row_ptr[r + 1]; ++j) acc += coef[j] * z[col_idx[j]];
+      Y[t * d_out + r] = alpha * acc;
+    }
+  });
+  return 0;
+}
+
+// Backward, input gradient, for L = <Y, dY>:
+//   dX = dY W_Q + alpha * dY (F H).
+// Wq nullable. dY [T, d_out]; dX [T, d_in].
+int oracle_adapter_bwd_dx(int32_t d_out, int32_t d_in, int32_t n, const int32_t *row_ptr,
+                          const int32_t *col_idx, const double *coef, const double *Wq,
+                          const double *dY, int64_t T, double alpha, double *dX) {
+  if (!shape_ok(d_in, n) || d_out <= 0 || T < 0) return 1;
+  std::vector<double> dW((size_t)d_out * d_in);
+  delta_w(d_out, d_in, n, row_ptr, col_idx, coef, dW.data());
+  parallel_for(T, [&](int64_t t) {
+    const double *g = dY + t * d_out;
+    double *o = dX + t * d_in;
+    for (int k = 0; k < d_in; ++k) {
+      double base = 0.0, ad = 0.0;
+      for (int r = 0; r < d_out; ++r) {
+        if (Wq) base += g[r] * Wq[(int64_t)r * d_in + k];
+        ad += g[r] * dW[(int64_t)r * d_in + k];
+      }
+      o[k] = base + alpha * ad;
+    }
+  });
+  return 0;
+}
+
+// Backward, coefficient gradient at m given positions (r_j, k_j):
+//   dc_j = alpha * sum_t dY[t, r_j] * (X H)[t, k_j],
+// with (X H)[t, k] = sum_i X[t, i] H[i, k] by the definition of the product.
+// X [T, d_in]; dY [T, d_out]; dc [m].
+int oracle_adapter_bwd_dc(int32_t d_out, int32_t d_in, int32_t n, const double *X, const double *dY,
+                          int64_t T, double alpha, int64_t m, const int32_t *rows,
+                          const int32_t *cols, double *dc) {
+  if (!shape_ok(d_in, n) || d_out <= 0 || T < 0) return 1;
+  const double inv = inv_sqrt(n);
+  parallel_for(m, [&](int64_t j) {
+    const int r = rows[j], k = cols[j];
+    double acc = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+      const double *x = X + t * d_in;
+      double z = 0.0;
+      for (int i = 0; i < d_in; ++i) z += x[i] * blockdiag_entry(n, inv, i, k);
+      acc += dY[t * d_out + r] * z;
+    }
+    dc[j] = alpha * acc;
+  });
+  return 0;
+}
+
+// AdaAlloc initialisation [P1 设计2 and 设计3 (dense solution x0); P2 2.2].
+//   e_i    = ||dW_Q[i,:]||_2 (squares in double, pairwise tree)       -> err_norm
+//   budget = min_per_row + floor(pool * e_i / sum_active e), pool = p - min_per_row*d_out,
+//            capped at d_in (capped rows leave; the rest re-share what is left);
+//            remainder p - sum(budget) given one each, in order, to
+//            mode 0: the least-allocated rows (budget asc, index asc)  [P1 设计2]
+//            mode 1: the largest-error rows (e_i desc, index asc)
+//   V      = dW_Q[i,:] H, unnormalised butterflies in textbook order, double
+//   E row i = the budget_i indices of largest |V| (ties: lower index), ascending
+//   c      = float(V * (1/sqrt(n)))
+// Outputs: budgets [d_out], row_ptr [d_out+1], col_idx [p], coef [p],
+// err_norm [d_out] (nullable).
+int oracle_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, int64_t p,
+                      int32_t min_per_row, int32_t mode, int32_t *budgets, int32_t *row_ptr,
+                      int32_t *col_idx, float *coef, double *err_norm) {
+  if (!shape_ok(d_in, n) || d_out <= 0 || min_per_row < 0 || min_per_row > d_in) return 1;
+  if (p < (int64_t)min_per_row * d_out || p > (int64_t)d_in * d_out || p > 2147483647LL) return 1;
+  if (mode != 0 && mode != 1) return 1;
+
+  // Per-channel error norms.
+  std::vector<double> e(d_out);
+  parallel_for(d_out, [&](int64_t i) {
+    std::vector<double> sq(d_in);
+    for (int k = 0; k < d_in; ++k) {
+      double w = (double)dWq[i * d_in + k];
+      sq[k] = w * w;
+    }
+    e[i] = std::sqrt(pairwise_sum(sq.data(), d_in));
+  });
+  if (err_norm)
+    for (int i = 0; i < d_out; ++i) err_norm[i] = e[i];
+
+  // Budgets: floor share of the pool, capped at d_in, surplus re-shared.
+  std::vector<int64_t> b(d_out, min_per_row);
+  std::vector<char> capped(d_out, 0);
+  double pool = (double)(p - (int64_t)min_per_row * d_out);
+  for (;;) {
+    std::vector<double> ea(d_out);
+    int64_t n_active = 0;
+    for (int i = 0; i < d_out; ++i) {
+      ea[i] = capped[i] ? 0.0 : e[i];
+      n_active += !capped[i];
+    }
+    if (n_active == 0) break;
+    const double S = pairwise_sum(ea.data(), d_out);
+    bool any_new = false;
+    for (int i = 0; i < d_out; ++i) {
+      if (capped[i]) continue;
+      double share = S > 0.0 ? std::floor((pool * e[i]) / S) : std::floor(pool / (double)n_active);
+      b[i] = min_per_row + (int64_t)share;
+      if (b[i] > d_in) any_new = true;
+    }
+    if (!any_new) break;
+    for (int i = 0; i < d_out; ++i)
+      if (!capped[i] && b[i] > d_in) {
+        b[i] = d_in;
+        capped[i] = 1;
+        pool -= (double)(d_in - min_per_row);
+      }
+  }
+  int64_t R = p - std::accumulate(b.begin(), b.end(), (int64_t)0);
+  std::vector<int> order(d_out);
+  std::iota(order.begin(), order.end(), 0);
+  if (mode == 0)
+    std::stable_sort(order.begin(), order.end(), [&](int a, int c) { return b[a] < b[c]; });
+  else
+    std::stable_sort(order.begin(), order.end(), [&](int a, int c) { return e[a] > e[c]; });
+  while (R > 0)
+    for (int i : order)
+      if (R > 0 && b[i] < d_in) {
+        ++b[i];
+        --R;
+      }
+  row_ptr[0] = 0;
+  for (int i = 0; i < d_out; ++i) {
+    budgets[i] = (int32_t)b[i];
+    row_ptr[i + 1] = row_ptr[i] + (int32_t)b[i];
+  }
+
+  // In-channel selection of the largest transform magnitudes.
+  const double inv = inv_sqrt(n);
+  parallel_for(d_out, [&](int64_t i) {
+    std::vector<double> v(d_in);
+    for (int k = 0; k < d_in; ++k) v[k] = (double)dWq[i * d_in + k];
+    for (int blk = 0; blk < d_in / n; ++blk) butterflies(v.data() + (int64_t)blk * n, n);
+    std::vector<int> idx(d_in);
+    std::iota(idx.begin(), idx.end(), 0);
+    std::sort(idx.begin(), idx.end(), [&](int a, int c) {
+      double fa = std::fabs(v[a]), fc = std::fabs(v[c]);
+      return fa > fc || (fa == fc && a < c);
+    });
+    std::vector<int> pick(idx.begin(), idx.begin() + budgets[i]);
+    std::sort(pick.begin(), pick.end());
+    for (int q = 0; q < budgets[i]; ++q) {
+      col_idx[row_ptr[i] + q] = pick[q];
+      coef[row_ptr[i] + q] = (float)(v[pick[q]] * inv);
+    }
+  });
+  return 0;
+}
+
+// Column view of the CSR pattern: for every column k the nonzeros j with
+// col_idx[j] == k, in increasing j: col_ptr [d_in+1], row_idx [p] (their rows),
+// perm [p] (their CSR positions).
+int oracle_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr,
+                      const int32_t *col_idx, int32_t *col_ptr, int32_t *row_idx, int32_t *perm) {
+  if (d_out <= 0 || d_in <= 0 || p < 0 || row_ptr[d_out] != p) return 1;
+  for (int k = 0; k <= d_in; ++k) col_ptr[k] = 0;
+  for (int64_t j = 0; j < p; ++j) {
+    if (col_idx[j] < 0 || col_idx[j] >= d_in) return 1;
+    col_ptr[col_idx[j] + 1]++;
+  }
+  for (int k = 0; k < d_in; ++k) col_ptr[k + 1] += col_ptr[k];
+  std::vector<int32_t> next(col_ptr, col_ptr + d_in);
+  for (int r = 0; r < d_out; ++r)
+    for (int32_t j = row_ptr[r]; j < row_ptr[r + 1]; ++j) {
+      int32_t pos = next[col_idx[j]]++;
+      row_idx[pos] = r;
+      perm[pos] = j;
+    }
+  return 0;
+}
+
+}  // extern "C"
