@@ -1,0 +1,201 @@
+/*
+ * qwha.h -- C ABI of the B200 (sm_100a) implementation of the Walsh-Hadamard
+ * adapter (WHA) layer on a group-quantized linear layer.
+ *
+ * The layer, after "QWHA: Quantization-Aware Walsh-Hadamard Adaptation for
+ * Parameter-Efficient Fine-Tuning on Large Language Models" (papernotes.org,
+ * section 整体框架 and 关键设计 1; gist.science, section 2.1 Adapter Design):
+ *
+ *     Y = X W_Q^T + alpha * X (F H^-1)^T
+ *
+ * W_Q is the frozen quantized base weight [d_out, d_in]; H is the frozen
+ * Walsh-Hadamard matrix over d_in; F = Scatter(c, E) is a sparse [d_out, d_in]
+ * matrix with p nonzeros whose values c are the only trained parameters.
+ * This library takes H to be the Sylvester-ordered matrix normalised to be
+ * orthonormal, H_n[i][j] = (-1)^popcount(i & j) / sqrt(n), so H^-1 = H = H^T;
+ * when d_in is not a power of two, H is block-diagonal with d_in / had_block
+ * equal blocks H_had_block. Then
+ *
+ *     Z    = X H                               (fast transform, no multiply)
+ *     Y    = X W_Q^T + alpha * Z F^T           (forward)
+ *     dc_j = alpha * sum_t dY[t, r_j] Z[t, k_j]  (backward, E = {(r_j, k_j)})
+ *     dX   = dY W_Q + alpha * (dY F) H
+ *
+ * Conventions for every call:
+ *   - Matrices are dense, row-major, with no padding between rows.
+ *   - Pointers named d_* or documented as "device" are CUDA device pointers;
+ *     the library reads them on `stream` and never frees or keeps them.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call
+ *     only enqueues work on it and returns without synchronising, except
+ *     qwha_validate_plan and qwha_check_stream_status, which synchronise it.
+ *   - Device buffers must be 16-byte aligned (QWHA_ERR_MISALIGNED otherwise).
+ *   - The caller owns all memory. Calls that need scratch take `ws` (device,
+ *     256-byte aligned) and `ws_bytes`; qwha_workspace_size gives the need.
+ *   - Errors are returned as qwha_status; nothing is thrown across the ABI.
+ *     qwha_last_error() gives a message for the last failing call of the
+ *     calling thread. Arguments are checked on the host before any launch; a
+ *     failed check launches nothing.
+ */
+#ifndef QWHA_H
+#define QWHA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QWHA_OK = 0,
+  QWHA_ERR_INVALID_ARG = 1, /* a shape, size, pointer or enum value is out of range */
+  QWHA_ERR_MISALIGNED = 2,  /* a device buffer is not 16-byte aligned */
+  QWHA_ERR_UNSUPPORTED = 3, /* a valid combination this build does not implement */
+  QWHA_ERR_WORKSPACE = 4,   /* ws is NULL or ws_bytes is below qwha_workspace_size */
+  QWHA_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  QWHA_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (see qwha_check_stream_status) */
+} qwha_status;
+
+typedef enum { QWHA_F32 = 0, QWHA_BF16 = 1 } qwha_dtype;
+
+/* Where the rounding remainder of the AdaAlloc budget goes: one extra
+ * coefficient each to the least-allocated channels (the rule the pages state,
+ * papernotes.org 关键设计 2) or to the channels of largest error. */
+typedef enum { QWHA_REM_FEWEST_ALLOC = 0, QWHA_REM_LARGEST_ERROR = 1 } qwha_remainder;
+
+/* Edge of the square blocks of F into which the coefficient-gradient kernel
+ * tiles the nonzeros (the tile view built by qwha_plan_build). */
+#define QWHA_TILE 512
+
+/* The sparse coefficient matrix F = Scatter(c, E) and its index views. All
+ * arrays are device memory owned by the caller.
+ *   row_ptr [d_out+1], col_idx [p], coef [p]: CSR by output channel; within a
+ *       row col_idx is strictly increasing (qwha_init_alloc writes this form).
+ *   col_ptr [d_in+1], row_idx [p], perm [p]: CSC view; for column k the
+ *       nonzeros in increasing CSR position; perm[q] is the CSR position of CSC
+ *       entry q and row_idx[q] its row.
+ *   tile_ptr [n_tiles+1], tile_pos [p], tile_rk [p]: the nonzeros grouped by
+ *       QWHA_TILE x QWHA_TILE block of F (block (rb, kb) has id
+ *       kb * ceil(d_out/QWHA_TILE) + rb), in CSC order inside a block;
+ *       tile_pos is the CSR position, tile_rk packs (r mod QWHA_TILE) << 16 |
+ *       (k mod QWHA_TILE).
+ * The views are written by qwha_plan_build and depend on E only; the forward
+ * needs the CSR arrays only, the backward needs all three views. */
+typedef struct {
+  int32_t d_in, d_out, had_block;
+  int64_t p;
+  const int32_t *row_ptr, *col_idx;
+  const float *coef;
+  const int32_t *col_ptr, *row_idx, *perm;
+  const int32_t *tile_ptr, *tile_pos, *tile_rk;
+} qwha_adapter;
+
+/* The frozen quantized base weight W_Q [d_out, d_in], device memory.
+ * Code q[i][k] (0 <= q < 2^bits) is bits [bits*k, bits*k + bits) of row i's
+ * little-endian bit stream, qweight holds d_out rows of d_in*bits/8 bytes;
+ * W_Q[i][k] = scales[i][k/group] * (q[i][k] - zeros[i][k/group]) in fp32;
+ * scales fp32 and zeros u8 are [d_out, d_in/group]. bits in {2, 3, 4}; group a
+ * multiple of 8 that divides d_in. The tensor cores consume W_Q rounded to
+ * bf16. (The pages start from an already quantized model, papernotes.org
+ * 整体框架; this format is the library's own.) */
+typedef struct {
+  int32_t bits, group;
+  const uint8_t *qweight;
+  const float *scales;
+  const uint8_t *zeros;
+} qwha_qweight;
+
+/* Operations for qwha_workspace_size. */
+typedef enum {
+  QWHA_OP_FWD = 0,
+  QWHA_OP_BWD = 1,
+  QWHA_OP_INIT = 2,
+  QWHA_OP_PLAN = 3
+} qwha_op;
+
+/* Z = X H row by row: x and z are [rows, n] of dtype dt (device), each row
+ * transformed by the block-diagonal orthonormal Hadamard matrix with blocks
+ * of had_block. had_block is a power of two in [2, 32768] dividing n; x and z
+ * must not overlap. Arithmetic in fp32.
+ * (papernotes.org 关键设计 1 and gist.science 2.1: the +-1 kernel turns the
+ * transform into a recursion of sums and differences.) */
+qwha_status qwha_fwht(qwha_dtype dt, const void *x, void *z, int64_t rows, int32_t n,
+                      int32_t had_block, void *stream);
+
+/* Forward of the adapted layer (gist.science 2.1; papernotes.org 整体框架):
+ *   Z_out = X H                 [T, d_in], dtype dt (kept for the backward)
+ *   Y     = X W_Q^T + alpha Z F^T  [T, d_out], dtype dt
+ * wq == NULL computes the adapter alone (Y = alpha Z F^T). With wq, dt must be
+ * QWHA_BF16. X, Z_out, Y are device buffers; a->row_ptr/col_idx/coef are
+ * required, the other views are not read. T >= 0 (T = 0 does nothing). */
+qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt,
+                             const void *X, int64_t T, float alpha, void *Z_out, void *Y,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* Backward with only c trained (papernotes.org 整体框架 and 训练策略):
+ *   dc[j] = alpha * sum_t dY[t, r_j] Z[t, k_j]   fp32 [p], CSR order
+ *   dX    = dY W_Q + alpha (dY F) H              [T, d_in], dtype dt
+ * Z is the Z_out of the matching forward. dc is overwritten (not accumulated).
+ * Needs all views of `a` (qwha_plan_build). dX may be NULL to skip it. The
+ * dc reduction runs in a fixed order: results are bitwise reproducible. */
+qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt,
+                             const void *dY, const void *Z, int64_t T, float alpha, float *dc,
+                             void *dX, void *ws, size_t ws_bytes, void *stream);
+
+/* AdaAlloc initialisation from the quantization error dW_Q = W0 - W_Q
+ * (papernotes.org 关键设计 2 and 3; gist.science 2.2). dWq fp32 [d_out, d_in]
+ * device. Per channel i:
+ *   e_i = ||dWq[i,:]||_2 (fp64 squares, pairwise sum in index order);
+ *   budget_i = min_per_row + floor(pool * e_i / sum e), pool = p -
+ *       min_per_row * d_out; a channel above d_in is capped and the others
+ *       re-share the rest; the remainder p - sum(budget) goes one each in the
+ *       order given by `mode`;
+ *   V = dWq[i,:] H_unnormalised (fp64 butterflies, stages h = 1, 2, 4, ...);
+ *   E row i = the budget_i largest |V| (ties to the lower index), ascending;
+ *   c = float(V * 1/sqrt(had_block)) (the dense solution values).
+ * Outputs (device): budgets [d_out], row_ptr [d_out+1], col_idx [p], coef [p].
+ * Requires min_per_row*d_out <= p <= d_in*d_out, p < 2^31, d_in <= 32768.
+ * Budgets and E are bitwise deterministic. */
+qwha_status qwha_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block,
+                            int64_t p, int32_t min_per_row, qwha_remainder mode,
+                            int32_t *budgets, int32_t *row_ptr, int32_t *col_idx, float *coef,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* Index views of E for the backward (E stays fixed while c trains,
+ * papernotes.org 整体框架): from the CSR row_ptr/col_idx (device) write the
+ * CSC view (col_ptr [d_in+1], row_idx [p], perm [p]) and the tile view
+ * (tile_ptr [qwha_plan_tiles(d_out, d_in) + 1], tile_pos [p], tile_rk [p]).
+ * col_idx must be within [0, d_in); duplicates inside a row are not checked
+ * here (qwha_validate_plan does). */
+qwha_status qwha_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr,
+                            const int32_t *col_idx, int32_t *col_ptr, int32_t *row_idx,
+                            int32_t *perm, int32_t *tile_ptr, int32_t *tile_pos,
+                            int32_t *tile_rk, void *ws, size_t ws_bytes, void *stream);
+
+/* Number of QWHA_TILE x QWHA_TILE blocks of F. */
+int64_t qwha_plan_tiles(int32_t d_out, int32_t d_in);
+
+/* Scratch bytes a call needs (0 if none). T is the token count for FWD/BWD,
+ * with_base is 1 when a qwha_qweight is passed. */
+size_t qwha_workspace_size(qwha_op op, int32_t d_out, int32_t d_in, int64_t p, int64_t T,
+                           int32_t with_base);
+
+/* Check E and its views on the device: row_ptr non-decreasing from 0 to p,
+ * col_idx in range and strictly increasing per row, and, if present, the CSC
+ * and tile views consistent with it. Synchronises the stream.
+ * QWHA_ERR_INVALID_ARG names the first failure in qwha_last_error(). */
+qwha_status qwha_validate_plan(const qwha_adapter *a, void *stream);
+
+/* Synchronise `stream` and report a device-side error word set by a bounded
+ * wait (QWHA_ERR_TIMEOUT) or a CUDA error (QWHA_ERR_CUDA); clears the word. */
+qwha_status qwha_check_stream_status(void *stream);
+
+const char *qwha_status_string(qwha_status s);
+const char *qwha_last_error(void);
+const char *qwha_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QWHA_H */

@@ -1,0 +1,285 @@
+"""Forward, backward, plan and AdaAlloc through the C ABI, against the oracle."""
+
+import numpy as np
+import pytest
+
+import oracle
+from _util import TOL_BF16, TOL_F32, bf16_dev, host, rel_fro, to_dev
+from workloads import (
+    CONFIGS,
+    bf16_bits_to_f32,
+    f32_to_bf16_bits,
+    layer_inputs,
+    pack_codes,
+    quantize_rtn,
+    random_pattern,
+    rng_for,
+)
+
+pytestmark = pytest.mark.gpu
+
+
+def _W():
+    import walsh_hadamard_sparse_b200 as W
+
+    return W
+
+
+def device_adapter(d_in, d_out, n, rp, ci, cf, plan=True):
+    import torch
+
+    W = _W()
+    a = W.Adapter(d_in, d_out, n, int(ci.size), to_dev(rp), to_dev(ci) if ci.size else torch.zeros(1, dtype=torch.int32, device="cuda"),
+                  to_dev(cf) if cf.size else torch.zeros(1, device="cuda"))
+    if plan:
+        W.plan_build(a)
+    return a
+
+
+def synth_layer(seed, d_in, d_out, n, T, p, dtype, bits=4, group=64, pattern="init"):
+    """Seeded layer: activations, gradients, a quantized weight, and E/c from the oracle's AdaAlloc
+    (or a random pattern for edge cases)."""
+    g = rng_for(seed, "adapter-test", d_in, d_out, n, T, p)
+    group = group if d_in % group == 0 else 32
+    w0 = (g.standard_normal((d_out, d_in)).astype(np.float32) * np.float32(0.02))
+    w0[g.random((d_out, d_in)) < 0.002] *= np.float32(15.0)
+    q, s, z, wq, dwq = quantize_rtn(w0, bits, group)
+    X = g.standard_normal((T, d_in)).astype(np.float32)
+    X[:, g.choice(d_in, max(1, d_in // 100), replace=False)] *= np.float32(20.0)
+    dY = g.standard_normal((T, d_out)).astype(np.float32)
+    if dtype == "bf16":
+        X = bf16_bits_to_f32(f32_to_bf16_bits(X))
+        dY = bf16_bits_to_f32(f32_to_bf16_bits(dY))
+    if pattern == "init":
+        e = oracle.init_alloc(dwq, p, n, 2, "fewest")
+        rp, ci, cf = e["row_ptr"], e["col_idx"], e["coef"]
+    else:
+        rp, ci, cf = random_pattern(d_out, d_in, p=p, rng=g)
+    return dict(X=X, dY=dY, rp=rp, ci=ci, cf=cf, qweight=pack_codes(q, bits), scales=s, zeros=z, Wq=wq,
+                dWq=dwq, bits=bits, group=group)
+
+
+def dev_act(a, dtype):
+    if dtype == "bf16":
+        return bf16_dev(f32_to_bf16_bits(a))
+    return to_dev(a)
+
+
+def dev_qweight(L):
+    W = _W()
+    return W.QWeight(L["bits"], L["group"], to_dev(L["qweight"]), to_dev(L["scales"]), to_dev(L["zeros"]))
+
+
+# --------------------------------------------------------------------------- plan
+
+
+def expected_tiles(rp, ci, d_out, d_in):
+    cp, ri, pm = oracle.plan_build(rp, ci, d_in)
+    n_rb = -(-d_out // 512)
+    n_kb = -(-d_in // 512)
+    cols = np.repeat(np.arange(d_in), np.diff(cp))
+    tile = (cols // 512) * n_rb + ri // 512
+    order = np.argsort(tile, kind="stable")
+    tile_ptr = np.zeros(n_rb * n_kb + 1, dtype=np.int64)
+    tile_ptr[1:] = np.cumsum(np.bincount(tile, minlength=n_rb * n_kb))
+    rk = ((ri % 512) << 16) | (cols % 512)
+    return cp, ri, pm, tile_ptr, pm[order], rk[order]
+
+
+@pytest.mark.parametrize(
+    "d_out,d_in,counts",
+    [
+        (64, 256, "random"),
+        (1200, 1104, "random"),  # several row and column blocks, ragged edges
+        (40, 96, "edge"),  # empty rows, full rows
+        (8, 8, "full"),
+        (16, 32, "empty"),
+    ],
+)
+def test_plan_build_matches_oracle(d_out, d_in, counts):
+    import torch
+
+    W = _W()
+    g = rng_for(30, "plan", d_out, d_in)
+    if counts == "random":
+        rp, ci, cf = random_pattern(d_out, d_in, p=min(d_out * d_in, 40 * d_out), rng=g)
+    elif counts == "edge":
+        c = g.integers(0, 12, d_out)
+        c[::7] = 0
+        c[3] = d_in
+        rp, ci, cf = random_pattern(d_out, d_in, counts=c, rng=g)
+    elif counts == "full":
+        rp, ci, cf = random_pattern(d_out, d_in, counts=np.full(d_out, d_in), rng=g)
+    else:
+        rp, ci, cf = random_pattern(d_out, d_in, counts=np.zeros(d_out, dtype=np.int64), rng=g)
+    a = device_adapter(d_in, d_out, 8, rp, ci, cf)
+    torch.cuda.synchronize()
+    cp, ri, pm, tp, tpos, trk = expected_tiles(rp, ci, d_out, d_in)
+    p = ci.size
+    assert np.array_equal(a.col_ptr.cpu().numpy(), cp)
+    assert np.array_equal(a.row_idx.cpu().numpy()[:p], ri)
+    assert np.array_equal(a.perm.cpu().numpy()[:p], pm)
+    assert np.array_equal(a.tile_ptr.cpu().numpy(), tp)
+    assert np.array_equal(a.tile_pos.cpu().numpy()[:p], tpos)
+    assert np.array_equal(a.tile_rk.cpu().numpy()[:p], trk)
+    W.validate_plan(a)
+
+
+def test_validate_plan_rejects_bad_patterns():
+    import torch
+
+    W = _W()
+    rp, ci, cf = random_pattern(32, 64, p=200, rng=rng_for(31, "bad"))
+    a = device_adapter(64, 32, 64, rp, ci, cf)
+    W.validate_plan(a)
+    bad = ci.copy()
+    r = 5
+    bad[rp[r]], bad[rp[r] + 1] = bad[rp[r] + 1], bad[rp[r]]  # unsorted inside row 5
+    a.col_idx = to_dev(bad)
+    with pytest.raises(W.QwhaError, match="increasing"):
+        W.validate_plan(a)
+    bad2 = ci.copy()
+    bad2[7] = 64  # out of range
+    a.col_idx = to_dev(bad2)
+    with pytest.raises(W.QwhaError, match="out of"):
+        W.validate_plan(a)
+    a.col_idx = to_dev(ci)
+    a.perm = torch.flip(a.perm[: ci.size], [0]).contiguous()
+    with pytest.raises(W.QwhaError):
+        W.validate_plan(a)
+
+
+# --------------------------------------------------------------------------- init
+
+
+@pytest.mark.parametrize("mode", ["fewest", "largest"])
+def test_init_tiny_workload_bitexact(mode):
+    W = _W()
+    spec = CONFIGS["tiny"][0]
+    d = layer_inputs(spec, 0, "tiny", parts=("W",))
+    got = W.init_alloc(to_dev(d["dWq"]), spec.p, spec.had_block, 2, mode)
+    ref = oracle.init_alloc(d["dWq"], spec.p, spec.had_block, 2, mode)
+    for k in ("budgets", "row_ptr", "col_idx"):
+        assert np.array_equal(got[k].cpu().numpy(), ref[k]), k
+    assert np.array_equal(got["coef"].cpu().numpy().view(np.uint32), ref["coef"].view(np.uint32))
+
+
+@pytest.mark.parametrize(
+    "d_out,d_in,n,p,mode,kind",
+    [
+        (96, 128, 128, 96 * 9 + 5, "fewest", "normal"),
+        (80, 3 * 64, 64, 80 * 5 + 33, "largest", "normal"),  # block-diagonal transform
+        (1000, 1024, 1024, 1000 * 40 + 123, "fewest", "normal"),  # several budget threads per row
+        (64, 64, 64, 64 * 6, "fewest", "cap"),  # a few rows hit the cap d_in
+        (64, 64, 64, 64 * 6, "largest", "cap"),
+        (48, 32, 32, 48 * 3 + 7, "fewest", "ties"),  # zero rows and integer data: many equal |V|
+        (16, 16, 16, 16 * 16, "fewest", "normal"),  # p = d_in * d_out
+        (24, 2048, 2048, 24 * 3, "largest", "normal"),  # p = 3 per row, long rows
+    ],
+)
+def test_init_bitexact(d_out, d_in, n, p, mode, kind):
+    W = _W()
+    g = rng_for(32, "init", d_out, d_in, n, p, kind)
+    w = g.standard_normal((d_out, d_in)).astype(np.float32) * np.float32(0.01)
+    if kind == "cap":
+        w[:3] *= np.float32(1000.0)
+    if kind == "ties":
+        w = g.integers(-2, 3, size=(d_out, d_in)).astype(np.float32)
+        w[::5] = 0.0
+    got = W.init_alloc(to_dev(w), p, n, 2, mode)
+    ref = oracle.init_alloc(w, p, n, 2, mode)
+    if kind == "cap":
+        assert ref["budgets"].max() == d_in
+    for k in ("budgets", "row_ptr", "col_idx"):
+        assert np.array_equal(got[k].cpu().numpy(), ref[k]), k
+    assert np.array_equal(got["coef"].cpu().numpy().view(np.uint32), ref["coef"].view(np.uint32))
+
+
+# --------------------------------------------------------------------------- forward / backward
+
+
+CASES = [
+    # d_in, d_out, n, T, p, dtype, pattern
+    (256, 256, 256, 64, 1024, "f32", "init"),
+    (512, 384, 128, 77, 384 * 20, "f32", "init"),
+    (1024, 768, 1024, 300, 768 * 24, "bf16", "init"),
+    (768, 512, 256, 33, 512 * 30, "bf16", "random"),  # block-diagonal transform
+    (96, 40, 32, 5, 300, "bf16", "random"),
+]
+
+
+@pytest.mark.parametrize("d_in,d_out,n,T,p,dtype,pattern", CASES)
+def test_adapter_forward_backward(d_in, d_out, n, T, p, dtype, pattern):
+    import torch
+
+    W = _W()
+    L = synth_layer(33, d_in, d_out, n, T, p, dtype, pattern=pattern)
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"])
+    alpha = 0.8
+    Xd, dYd = dev_act(L["X"], dtype), dev_act(L["dY"], dtype)
+    Z, Y = W.adapter_fwd(a, Xd, alpha)
+    dc, dX = W.adapter_bwd(a, dYd, Z, alpha)
+    torch.cuda.synchronize()
+    Zr, Yr = oracle.adapter_fwd(L["rp"], L["ci"], L["cf"], L["X"], d_out, n, alpha)
+    dXr = oracle.adapter_bwd_dx(L["rp"], L["ci"], L["cf"], L["dY"], d_in, n, alpha)
+    rows = oracle.csr_rows(L["rp"])
+    sel = np.arange(L["ci"].size)
+    if sel.size > 3000:
+        sel = np.sort(rng_for(34, "dcsel").choice(sel.size, 3000, replace=False))
+    dcr = oracle.adapter_bwd_dc(L["X"], L["dY"], rows[sel], L["ci"][sel], n, alpha)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    errs = dict(Z=rel_fro(host(Z), Zr), Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr),
+                dc=rel_fro(dc.cpu().numpy()[sel], dcr))
+    assert all(v <= tol for v in errs.values()), errs
+    # fixed-order reduction: a second backward is bitwise identical
+    dc2, _ = W.adapter_bwd(a, dYd, Z, alpha)
+    assert torch.equal(dc, dc2)
+
+
+@pytest.mark.parametrize(
+    "d_in,d_out,n,T,bits,group",
+    [
+        (512, 256, 512, 200, 4, 64),  # ragged token tile (200 = 128 + 72)
+        (1024, 768, 1024, 300, 3, 128),  # int3 bit stream
+        (640, 1280, 128, 129, 2, 64),  # int2, ragged token tile, K of 10 ring blocks
+        (256, 264, 256, 7, 4, 64),  # N = 264: partial 32-column epilogue chunk
+    ],
+)
+def test_base_gemm_forward_backward(d_in, d_out, n, T, bits, group):
+    import torch
+
+    W = _W()
+    p = d_out * 8
+    L = synth_layer(35, d_in, d_out, n, T, p, "bf16", bits=bits, group=group)
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"])
+    wq = dev_qweight(L)
+    alpha = 1.0
+    Xd, dYd = dev_act(L["X"], "bf16"), dev_act(L["dY"], "bf16")
+    Z, Y = W.adapter_fwd(a, Xd, alpha, wq=wq)
+    dc, dX = W.adapter_bwd(a, dYd, Z, alpha, wq=wq)
+    torch.cuda.synchronize()
+    Wq = oracle.dequant(L["qweight"], L["scales"], L["zeros"], bits, group, d_out, d_in)
+    _, Yr = oracle.adapter_fwd(L["rp"], L["ci"], L["cf"], L["X"], d_out, n, alpha, Wq, want_z=False)
+    dXr = oracle.adapter_bwd_dx(L["rp"], L["ci"], L["cf"], L["dY"], d_in, n, alpha, Wq)
+    errs = dict(Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr))
+    assert all(v <= TOL_BF16 for v in errs.values()), errs
+    # the base term alone (empty adapter) against the oracle's X W_Q^T
+    e = device_adapter(d_in, d_out, n, np.zeros(d_out + 1, np.int32), np.zeros(0, np.int32), np.zeros(0, np.float32))
+    _, Yb = W.adapter_fwd(e, Xd, alpha, wq=wq)
+    torch.cuda.synchronize()
+    assert rel_fro(host(Yb), L["X"].astype(np.float64) @ Wq.T) <= TOL_BF16
+
+
+def test_workspace_and_dtype_errors():
+    import torch
+
+    W = _W()
+    L = synth_layer(36, 256, 256, 256, 16, 512, "bf16", pattern="random")
+    a = device_adapter(256, 256, 256, L["rp"], L["ci"], L["cf"])
+    Xd = dev_act(L["X"], "bf16")
+    with pytest.raises(W.QwhaError) as ei:
+        W.adapter_fwd(a, Xd, 1.0, wq=dev_qweight(L), ws=torch.empty(256, dtype=torch.uint8, device="cuda"))
+    assert ei.value.status == 4
+    with pytest.raises(W.QwhaError) as ei:
+        W.adapter_fwd(a, to_dev(L["X"]), 1.0, wq=dev_qweight(L))  # base GEMM needs bf16
+    assert ei.value.status == 3

@@ -1,0 +1,22 @@
+"""B200 (sm_100a) Walsh-Hadamard adapter layer: Python binding of libqwha.
+
+The arithmetic runs in the CUDA kernels of libqwha.so; this package only
+marshals torch tensors (device memory and the current stream) into the C ABI
+of include/qwha.h. Import fails if the library is not built.
+"""
+
+from ._lib import QwhaError, lib  # noqa: F401
+from .api import (  # noqa: F401
+    Adapter,
+    QWeight,
+    adapter_bwd,
+    adapter_fwd,
+    fwht,
+    init_alloc,
+    plan_build,
+    plan_tiles,
+    validate_plan,
+    workspace_size,
+)
+
+lib()  # fail loudly at import when libqwha.so is missing

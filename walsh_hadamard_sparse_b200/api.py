@@ -1,0 +1,190 @@
+"""torch-facing wrappers of the C ABI (argument marshalling only).
+
+Tensors must be CUDA tensors, contiguous, of the documented dtypes; work is
+enqueued on torch's current stream. Scratch space comes from torch's
+allocator and is passed to the library as the `ws` argument.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, fields
+
+import torch
+
+from ._lib import QwhaAdapter, QwhaQweight, check, lib
+
+F32, BF16 = 0, 1
+OP_FWD, OP_BWD, OP_INIT, OP_PLAN = 0, 1, 2, 3
+REMAINDER = {"fewest": 0, "largest": 1}
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t) -> ctypes.c_void_p | None:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ws(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+@dataclass
+class Adapter:
+    """F = Scatter(c, E) on the device: CSR arrays plus the views from plan_build."""
+
+    d_in: int
+    d_out: int
+    had_block: int
+    p: int
+    row_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    coef: torch.Tensor
+    col_ptr: torch.Tensor | None = None
+    row_idx: torch.Tensor | None = None
+    perm: torch.Tensor | None = None
+    tile_ptr: torch.Tensor | None = None
+    tile_pos: torch.Tensor | None = None
+    tile_rk: torch.Tensor | None = None
+
+    def c_struct(self) -> QwhaAdapter:
+        s = QwhaAdapter()
+        s.d_in, s.d_out, s.had_block, s.p = self.d_in, self.d_out, self.had_block, self.p
+        for f in fields(self):
+            if f.name in ("d_in", "d_out", "had_block", "p"):
+                continue
+            v = getattr(self, f.name)
+            setattr(s, f.name, None if v is None else v.data_ptr())
+        return s
+
+
+@dataclass
+class QWeight:
+    """Packed b-bit codes [d_out, d_in*bits/8] u8, scales f32 and zeros u8 [d_out, d_in/group]."""
+
+    bits: int
+    group: int
+    qweight: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+
+    def c_struct(self) -> QwhaQweight:
+        s = QwhaQweight()
+        s.bits, s.group = self.bits, self.group
+        s.qweight, s.scales, s.zeros = self.qweight.data_ptr(), self.scales.data_ptr(), self.zeros.data_ptr()
+        return s
+
+
+def workspace_size(op: int, d_out: int, d_in: int, p: int, T: int, with_base: bool) -> int:
+    return int(lib().qwha_workspace_size(op, d_out, d_in, p, T, int(bool(with_base))))
+
+
+def plan_tiles(d_out: int, d_in: int) -> int:
+    return int(lib().qwha_plan_tiles(d_out, d_in))
+
+
+def fwht(x: torch.Tensor, had_block: int | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Z = X H over the last dimension (block-diagonal with blocks of had_block)."""
+    n = x.shape[-1]
+    had_block = had_block or n
+    out = torch.empty_like(x) if out is None else out
+    rows = x.numel() // n if n else 0
+    check(lib().qwha_fwht(_dt(x), _ptr(x), _ptr(out), rows, n, had_block, _stream()), "qwha_fwht")
+    return out
+
+
+def adapter_fwd(a: Adapter, X: torch.Tensor, alpha: float = 1.0, wq: QWeight | None = None,
+                Z_out: torch.Tensor | None = None, Y: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """(Z, Y) with Z = X H and Y = X W_Q^T + alpha Z F^T (W_Q term only with wq)."""
+    T = X.shape[0]
+    Z_out = torch.empty_like(X) if Z_out is None else Z_out
+    Y = torch.empty((T, a.d_out), dtype=X.dtype, device=X.device) if Y is None else Y
+    need = workspace_size(OP_FWD, a.d_out, a.d_in, a.p, T, wq is not None)
+    ws = _ws(need, X.device) if ws is None else ws
+    cs = a.c_struct()
+    cw = wq.c_struct() if wq is not None else None
+    rc = lib().qwha_adapter_fwd(ctypes.byref(cs), ctypes.byref(cw) if cw is not None else None, _dt(X), _ptr(X), T,
+                                float(alpha), _ptr(Z_out), _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(), _stream())
+    check(rc, "qwha_adapter_fwd")
+    return Z_out, Y
+
+
+def adapter_bwd(a: Adapter, dY: torch.Tensor, Z: torch.Tensor, alpha: float = 1.0, wq: QWeight | None = None,
+                dc: torch.Tensor | None = None, dX: torch.Tensor | None = None, want_dx: bool = True,
+                ws: torch.Tensor | None = None):
+    """(dc, dX): dc_j = alpha sum_t dY[t,r_j] Z[t,k_j]; dX = dY W_Q + alpha (dY F) H."""
+    T = dY.shape[0]
+    dc = torch.empty(a.p, dtype=torch.float32, device=dY.device) if dc is None else dc
+    if want_dx and dX is None:
+        dX = torch.empty((T, a.d_in), dtype=dY.dtype, device=dY.device)
+    need = workspace_size(OP_BWD, a.d_out, a.d_in, a.p, T, wq is not None)
+    ws = _ws(need, dY.device) if ws is None else ws
+    cs = a.c_struct()
+    cw = wq.c_struct() if wq is not None else None
+    rc = lib().qwha_adapter_bwd(ctypes.byref(cs), ctypes.byref(cw) if cw is not None else None, _dt(dY), _ptr(dY),
+                                _ptr(Z), T, float(alpha), _ptr(dc), _ptr(dX) if want_dx else None, _ptr(ws),
+                                0 if ws is None else ws.numel(), _stream())
+    check(rc, "qwha_adapter_bwd")
+    return dc, dX
+
+
+def init_alloc(dWq: torch.Tensor, p: int, had_block: int, min_per_row: int = 2, mode: str = "fewest",
+               ws: torch.Tensor | None = None) -> dict:
+    """AdaAlloc on the device: dict(budgets, row_ptr, col_idx, coef)."""
+    d_out, d_in = dWq.shape
+    dev = dWq.device
+    out = dict(
+        budgets=torch.empty(d_out, dtype=torch.int32, device=dev),
+        row_ptr=torch.empty(d_out + 1, dtype=torch.int32, device=dev),
+        col_idx=torch.empty(max(p, 1), dtype=torch.int32, device=dev),
+        coef=torch.empty(max(p, 1), dtype=torch.float32, device=dev),
+    )
+    need = workspace_size(OP_INIT, d_out, d_in, p, 0, False)
+    ws = _ws(need, dev) if ws is None else ws
+    rc = lib().qwha_init_alloc(_ptr(dWq), d_out, d_in, had_block, p, min_per_row, REMAINDER[mode],
+                               _ptr(out["budgets"]), _ptr(out["row_ptr"]), _ptr(out["col_idx"]), _ptr(out["coef"]),
+                               _ptr(ws), 0 if ws is None else ws.numel(), _stream())
+    check(rc, "qwha_init_alloc")
+    out["col_idx"], out["coef"] = out["col_idx"][:p], out["coef"][:p]
+    return out
+
+
+def plan_build(a: Adapter, ws: torch.Tensor | None = None) -> Adapter:
+    """Fill the CSC and tile views of `a` (new tensors) and return it."""
+    dev = a.row_ptr.device
+    n_tiles = plan_tiles(a.d_out, a.d_in)
+    pp = max(a.p, 1)
+    a.col_ptr = torch.empty(a.d_in + 1, dtype=torch.int32, device=dev)
+    a.row_idx = torch.empty(pp, dtype=torch.int32, device=dev)
+    a.perm = torch.empty(pp, dtype=torch.int32, device=dev)
+    a.tile_ptr = torch.empty(n_tiles + 1, dtype=torch.int32, device=dev)
+    a.tile_pos = torch.empty(pp, dtype=torch.int32, device=dev)
+    a.tile_rk = torch.empty(pp, dtype=torch.int32, device=dev)
+    need = workspace_size(OP_PLAN, a.d_out, a.d_in, a.p, 0, False)
+    ws = _ws(need, dev) if ws is None else ws
+    rc = lib().qwha_plan_build(a.d_out, a.d_in, a.p, _ptr(a.row_ptr), _ptr(a.col_idx), _ptr(a.col_ptr),
+                               _ptr(a.row_idx), _ptr(a.perm), _ptr(a.tile_ptr), _ptr(a.tile_pos), _ptr(a.tile_rk),
+                               _ptr(ws), 0 if ws is None else ws.numel(), _stream())
+    check(rc, "qwha_plan_build")
+    return a
+
+
+def validate_plan(a: Adapter) -> None:
+    cs = a.c_struct()
+    check(lib().qwha_validate_plan(ctypes.byref(cs), _stream()), "qwha_validate_plan")

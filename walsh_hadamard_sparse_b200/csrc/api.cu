@@ -1,0 +1,358 @@
+// C ABI of libqwha: argument checks, workspace carving and launch sequencing.
+// Every entry point validates on the host and launches nothing on failure.
+
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qwha {
+
+namespace {
+thread_local char g_msg[512] = "";
+}
+
+qwha_status fail(qwha_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+qwha_status cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return QWHA_OK;
+  return fail(QWHA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+}  // namespace qwha
+
+using namespace qwha;
+
+namespace {
+
+const char *dtype_name(qwha_dtype d) { return d == QWHA_F32 ? "f32" : d == QWHA_BF16 ? "bf16" : "?"; }
+
+bool valid_dtype(qwha_dtype d) { return d == QWHA_F32 || d == QWHA_BF16; }
+
+qwha_status check_hadamard(int32_t n, int32_t had_block) {
+  if (n <= 0) return fail(QWHA_ERR_INVALID_ARG, "row length %d must be positive", n);
+  if (had_block < 2 || had_block > 32768 || !is_pow2(had_block))
+    return fail(QWHA_ERR_INVALID_ARG, "had_block %d must be a power of two in [2, 32768]", had_block);
+  if (n % had_block)
+    return fail(QWHA_ERR_INVALID_ARG, "had_block %d does not divide the row length %d", had_block, n);
+  return QWHA_OK;
+}
+
+#define QWHA_CHECK_PTR(p, name)                                                        \
+  do {                                                                                 \
+    if (!(p)) return fail(QWHA_ERR_INVALID_ARG, "%s is NULL", name);                   \
+    if (!aligned16(p)) return fail(QWHA_ERR_MISALIGNED, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *qwha_status_string(qwha_status s) {
+  switch (s) {
+    case QWHA_OK: return "ok";
+    case QWHA_ERR_INVALID_ARG: return "invalid argument";
+    case QWHA_ERR_MISALIGNED: return "misaligned buffer";
+    case QWHA_ERR_UNSUPPORTED: return "unsupported";
+    case QWHA_ERR_WORKSPACE: return "workspace too small";
+    case QWHA_ERR_CUDA: return "CUDA error";
+    case QWHA_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char *qwha_last_error(void) { return g_msg; }
+
+const char *qwha_version(void) { return "qwha-b200 0.1 (sm_100a)"; }
+
+qwha_status qwha_fwht(qwha_dtype dt, const void *x, void *z, int64_t rows, int32_t n,
+                      int32_t had_block, void *stream) {
+  if (!valid_dtype(dt)) return fail(QWHA_ERR_INVALID_ARG, "dtype %d", (int)dt);
+  qwha_status st = check_hadamard(n, had_block);
+  if (st != QWHA_OK) return st;
+  if (rows < 0) return fail(QWHA_ERR_INVALID_ARG, "rows %lld < 0", (long long)rows);
+  if (rows == 0) return QWHA_OK;
+  QWHA_CHECK_PTR(x, "x");
+  QWHA_CHECK_PTR(z, "z");
+  const size_t esz = dt == QWHA_F32 ? 4 : 2;
+  const char *xb = static_cast<const char *>(x), *zb = static_cast<const char *>(z);
+  const size_t bytes = (size_t)rows * n * esz;
+  if (xb < zb + bytes && zb < xb + bytes) return fail(QWHA_ERR_INVALID_ARG, "x and z overlap");
+  const int logn = ilog2(had_block);
+  const float scale = (float)(1.0 / sqrt((double)had_block));
+  (void)dtype_name;
+  return cuda_status(launch_fwht(dt, dt, x, z, rows * (n / had_block), logn, scale, (cudaStream_t)stream),
+                     "fwht launch");
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- adapter
+
+namespace {
+
+struct Carver {  // hands out 256-byte aligned slices of the caller's workspace
+  char *base;
+  size_t off = 0;
+  explicit Carver(void *b) : base(static_cast<char *>(b)) {}
+  void *take(size_t bytes) {
+    void *p = base ? base + off : nullptr;
+    off += align_up(bytes, 256);
+    return p;
+  }
+};
+
+size_t esize(qwha_dtype d) { return d == QWHA_F32 ? 4 : 2; }
+
+qwha_status check_adapter_shape(const qwha_adapter *a) {
+  if (!a) return fail(QWHA_ERR_INVALID_ARG, "adapter is NULL");
+  if (a->d_in <= 0 || a->d_out <= 0 || a->d_in % 8 || a->d_out % 8)
+    return fail(QWHA_ERR_INVALID_ARG, "d_in %d and d_out %d must be positive multiples of 8", a->d_in, a->d_out);
+  qwha_status st = check_hadamard(a->d_in, a->had_block);
+  if (st != QWHA_OK) return st;
+  if (a->p < 0 || a->p > (int64_t)a->d_in * a->d_out || a->p > 2147483647LL)
+    return fail(QWHA_ERR_INVALID_ARG, "p = %lld out of range", (long long)a->p);
+  QWHA_CHECK_PTR(a->row_ptr, "row_ptr");
+  if (a->p > 0) {
+    QWHA_CHECK_PTR(a->col_idx, "col_idx");
+    QWHA_CHECK_PTR(a->coef, "coef");
+  }
+  return QWHA_OK;
+}
+
+qwha_status check_views(const qwha_adapter *a) {
+  QWHA_CHECK_PTR(a->col_ptr, "col_ptr");
+  QWHA_CHECK_PTR(a->tile_ptr, "tile_ptr");
+  if (a->p > 0) {
+    QWHA_CHECK_PTR(a->row_idx, "row_idx");
+    QWHA_CHECK_PTR(a->perm, "perm");
+    QWHA_CHECK_PTR(a->tile_pos, "tile_pos");
+    QWHA_CHECK_PTR(a->tile_rk, "tile_rk");
+  }
+  if (cdiv(a->d_out, QWHA_TILE) > plan_max_row_blocks())
+    return fail(QWHA_ERR_UNSUPPORTED, "d_out %d above %d", a->d_out, plan_max_row_blocks() * QWHA_TILE);
+  return QWHA_OK;
+}
+
+qwha_status check_qweight(const qwha_qweight *wq, int32_t d_out, int32_t d_in, qwha_dtype dt) {
+  if (!wq) return QWHA_OK;
+  if (dt != QWHA_BF16) return fail(QWHA_ERR_UNSUPPORTED, "the base GEMM needs dtype bf16");
+  if (wq->bits < 2 || wq->bits > 4) return fail(QWHA_ERR_INVALID_ARG, "bits %d not in {2,3,4}", wq->bits);
+  if (wq->group <= 0 || wq->group % 8 || d_in % wq->group)
+    return fail(QWHA_ERR_INVALID_ARG, "group %d must be a multiple of 8 dividing d_in %d", wq->group, d_in);
+  QWHA_CHECK_PTR(wq->qweight, "qweight");
+  QWHA_CHECK_PTR(wq->scales, "scales");
+  QWHA_CHECK_PTR(wq->zeros, "zeros");
+  (void)d_out;
+  return QWHA_OK;
+}
+
+qwha_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return QWHA_OK;
+  if (!ws || ws_bytes < need)
+    return fail(QWHA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws ? ws_bytes : (size_t)0, need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(QWHA_ERR_MISALIGNED, "workspace not 256-byte aligned");
+  return QWHA_OK;
+}
+
+size_t fwd_ws(int32_t d_out, int32_t d_in, int64_t T, bool base) {
+  if (!base) return 0;
+  return align_up((size_t)T * d_out * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
+}
+
+size_t bwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
+  size_t n = align_up((size_t)kSddmmMaxChunks * (size_t)(p > 0 ? p : 1) * 4, 256);
+  n += align_up((size_t)T * d_in * 4, 256);  // dZ
+  if (base) n += align_up((size_t)T * d_in * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t qwha_plan_tiles(int32_t d_out, int32_t d_in) {
+  if (d_out <= 0 || d_in <= 0) return 0;
+  return cdiv(d_out, QWHA_TILE) * cdiv(d_in, QWHA_TILE);
+}
+
+size_t qwha_workspace_size(qwha_op op, int32_t d_out, int32_t d_in, int64_t p, int64_t T, int32_t with_base) {
+  if (d_out <= 0 || d_in <= 0 || T < 0 || p < 0) return 0;
+  switch (op) {
+    case QWHA_OP_FWD: return fwd_ws(d_out, d_in, T, with_base != 0);
+    case QWHA_OP_BWD: return bwd_ws(d_out, d_in, p, T, with_base != 0);
+    case QWHA_OP_INIT: return init_workspace(d_out, d_in);
+    case QWHA_OP_PLAN: return plan_workspace(d_out, d_in);
+  }
+  return 0;
+}
+
+qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt, const void *X,
+                             int64_t T, float alpha, void *Z_out, void *Y, void *ws, size_t ws_bytes,
+                             void *stream) {
+  qwha_status st = check_adapter_shape(a);
+  if (st != QWHA_OK) return st;
+  if (!valid_dtype(dt)) return fail(QWHA_ERR_INVALID_ARG, "dtype %d", (int)dt);
+  if ((st = check_qweight(wq, a->d_out, a->d_in, dt)) != QWHA_OK) return st;
+  if (T < 0) return fail(QWHA_ERR_INVALID_ARG, "T %lld < 0", (long long)T);
+  if (T == 0) return QWHA_OK;
+  QWHA_CHECK_PTR(X, "X");
+  QWHA_CHECK_PTR(Z_out, "Z_out");
+  QWHA_CHECK_PTR(Y, "Y");
+  if ((st = check_ws(ws, ws_bytes, fwd_ws(a->d_out, a->d_in, T, wq != nullptr))) != QWHA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int logn = ilog2(a->had_block);
+  const float inv = (float)(1.0 / sqrt((double)a->had_block));
+  cudaError_t e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
+  if (e != cudaSuccess) return cuda_status(e, "fwht");
+  if (!wq) {
+    e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
+                        alpha, Y, s);
+    return cuda_status(e, "spmm");
+  }
+  Carver cv(ws);
+  float *y_ad = static_cast<float *>(cv.take((size_t)T * a->d_out * 4));
+  void *wdeq = cv.take(wdeq_bytes(a->d_out, a->d_in));
+  e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
+                      alpha, y_ad, s);
+  if (e != cudaSuccess) return cuda_status(e, "spmm");
+  e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, false, s);
+  if (e != cudaSuccess) return cuda_status(e, "dequant");
+  return cuda_status(launch_gemm_fwd(X, wdeq, y_ad, Y, T, a->d_out, a->d_in, s), "base GEMM");
+}
+
+qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt, const void *dY,
+                             const void *Z, int64_t T, float alpha, float *dc, void *dX, void *ws,
+                             size_t ws_bytes, void *stream) {
+  qwha_status st = check_adapter_shape(a);
+  if (st != QWHA_OK) return st;
+  if ((st = check_views(a)) != QWHA_OK) return st;
+  if (!valid_dtype(dt)) return fail(QWHA_ERR_INVALID_ARG, "dtype %d", (int)dt);
+  if ((st = check_qweight(wq, a->d_out, a->d_in, dt)) != QWHA_OK) return st;
+  if (T < 0) return fail(QWHA_ERR_INVALID_ARG, "T %lld < 0", (long long)T);
+  if (a->p > 0) QWHA_CHECK_PTR(dc, "dc");
+  if (T > 0) {
+    QWHA_CHECK_PTR(dY, "dY");
+    QWHA_CHECK_PTR(Z, "Z");
+    if (dX) QWHA_CHECK_PTR(dX, "dX");
+  }
+  if ((st = check_ws(ws, ws_bytes, bwd_ws(a->d_out, a->d_in, a->p, T, wq != nullptr))) != QWHA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  Carver cv(ws);
+  float *partial = static_cast<float *>(cv.take((size_t)kSddmmMaxChunks * (size_t)(a->p > 0 ? a->p : 1) * 4));
+  float *dz = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
+  cudaError_t e = launch_sddmm(dt, dY, Z, T, a->d_out, a->d_in, a->tile_ptr, a->tile_pos, a->tile_rk, a->p, alpha,
+                               partial, dc, s);
+  if (e != cudaSuccess) return cuda_status(e, "sddmm");
+  if (!dX || T == 0) return QWHA_OK;
+  e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, a->coef, a->perm, a->p, a->d_in, alpha,
+                      dz, s);
+  if (e != cudaSuccess) return cuda_status(e, "gather");
+  const int logn = ilog2(a->had_block);
+  const float inv = (float)(1.0 / sqrt((double)a->had_block));
+  const int64_t blocks = T * (a->d_in / a->had_block);
+  if (!wq) return cuda_status(launch_fwht(QWHA_F32, dt, dz, dX, blocks, logn, inv, s), "fwht");
+  float *dx_ad = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
+  void *wdeq = cv.take(wdeq_bytes(a->d_out, a->d_in));
+  e = launch_fwht(QWHA_F32, QWHA_F32, dz, dx_ad, blocks, logn, inv, s);
+  if (e != cudaSuccess) return cuda_status(e, "fwht");
+  e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, true, s);
+  if (e != cudaSuccess) return cuda_status(e, "dequant");
+  return cuda_status(launch_gemm_bwd(dY, wdeq, dx_ad, dX, T, a->d_out, a->d_in, s), "base GEMM (dX)");
+}
+
+qwha_status qwha_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr, const int32_t *col_idx,
+                            int32_t *col_ptr, int32_t *row_idx, int32_t *perm, int32_t *tile_ptr,
+                            int32_t *tile_pos, int32_t *tile_rk, void *ws, size_t ws_bytes, void *stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(QWHA_ERR_INVALID_ARG, "d_out %d, d_in %d", d_out, d_in);
+  if (cdiv(d_out, QWHA_TILE) > plan_max_row_blocks())
+    return fail(QWHA_ERR_UNSUPPORTED, "d_out %d above %d", d_out, plan_max_row_blocks() * QWHA_TILE);
+  if (p < 0 || p > (int64_t)d_in * d_out || p > 2147483647LL)
+    return fail(QWHA_ERR_INVALID_ARG, "p = %lld out of range", (long long)p);
+  QWHA_CHECK_PTR(row_ptr, "row_ptr");
+  QWHA_CHECK_PTR(col_ptr, "col_ptr");
+  QWHA_CHECK_PTR(tile_ptr, "tile_ptr");
+  if (p > 0) {
+    QWHA_CHECK_PTR(col_idx, "col_idx");
+    QWHA_CHECK_PTR(row_idx, "row_idx");
+    QWHA_CHECK_PTR(perm, "perm");
+    QWHA_CHECK_PTR(tile_pos, "tile_pos");
+    QWHA_CHECK_PTR(tile_rk, "tile_rk");
+  }
+  qwha_status st = check_ws(ws, ws_bytes, plan_workspace(d_out, d_in));
+  if (st != QWHA_OK) return st;
+  return cuda_status(launch_plan_build(d_out, d_in, p, row_ptr, col_idx, col_ptr, row_idx, perm, tile_ptr, tile_pos,
+                                       tile_rk, ws, (cudaStream_t)stream),
+                     "plan_build");
+}
+
+qwha_status qwha_validate_plan(const qwha_adapter *a, void *stream) {
+  qwha_status st = check_adapter_shape(a);
+  if (st != QWHA_OK) return st;
+  uint32_t code = 0;
+  int64_t where = 0;
+  cudaError_t e = launch_validate(a, (cudaStream_t)stream, &code, &where);
+  if (e != cudaSuccess) return cuda_status(e, "validate");
+  if (code) return fail(QWHA_ERR_INVALID_ARG, "%s (at %lld)", validate_message(code), (long long)where);
+  return QWHA_OK;
+}
+
+qwha_status qwha_check_stream_status(void *stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "stream");
+  unsigned int word = 0;
+  e = read_and_clear_error_word(&word, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "error word");
+  if (word) return fail(QWHA_ERR_TIMEOUT, "device wait gave up (code 0x%x)", word);
+  return QWHA_OK;
+}
+
+qwha_status qwha_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p,
+                            int32_t min_per_row, qwha_remainder mode, int32_t *budgets, int32_t *row_ptr,
+                            int32_t *col_idx, float *coef, void *ws, size_t ws_bytes, void *stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(QWHA_ERR_INVALID_ARG, "d_out %d, d_in %d", d_out, d_in);
+  qwha_status st = check_hadamard(d_in, had_block);
+  if (st != QWHA_OK) return st;
+  if (d_in > init_max_din()) return fail(QWHA_ERR_UNSUPPORTED, "d_in %d above %d", d_in, init_max_din());
+  if (min_per_row < 0 || min_per_row > d_in) return fail(QWHA_ERR_INVALID_ARG, "min_per_row %d", min_per_row);
+  if (p < (int64_t)min_per_row * d_out || p > (int64_t)d_in * d_out || p > 2147483647LL)
+    return fail(QWHA_ERR_INVALID_ARG, "p = %lld outside [%lld, %lld]", (long long)p,
+                (long long)min_per_row * d_out, (long long)d_in * d_out);
+  if (mode != QWHA_REM_FEWEST_ALLOC && mode != QWHA_REM_LARGEST_ERROR)
+    return fail(QWHA_ERR_INVALID_ARG, "remainder mode %d", (int)mode);
+  QWHA_CHECK_PTR(dWq, "dWq");
+  QWHA_CHECK_PTR(budgets, "budgets");
+  QWHA_CHECK_PTR(row_ptr, "row_ptr");
+  if (p > 0) {
+    QWHA_CHECK_PTR(col_idx, "col_idx");
+    QWHA_CHECK_PTR(coef, "coef");
+  }
+  if ((st = check_ws(ws, ws_bytes, init_workspace(d_out, d_in))) != QWHA_OK) return st;
+  return cuda_status(launch_init_alloc(dWq, d_out, d_in, had_block, p, min_per_row, (int)mode, budgets, row_ptr,
+                                       col_idx, coef, ws, (cudaStream_t)stream),
+                     "init_alloc");
+}
+
+}  // extern "C"

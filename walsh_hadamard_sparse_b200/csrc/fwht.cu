@@ -1,0 +1,283 @@
+// Row-wise fast Walsh-Hadamard transform (Sylvester order, orthonormal).
+//
+// The adapter's transform is the +-1 Walsh-Hadamard matrix, computed as a
+// recursion of sums and differences with no multiplications ("QWHA",
+// papernotes.org 关键设计 1; gist.science 2.1). Each block of n = 2^m
+// consecutive elements of a row is replaced by its transform times `scale`
+// (1/sqrt(n) for the orthonormal H, times alpha where the adapter folds it).
+//
+// Layout of the main kernel (128 <= n <= 4096). The m index bits of an element
+// are split into three fields: low (LV bits, one 16-byte vector of the narrow
+// I/O type), middle (PB bits) and high (HB bits).
+//   phase A: a thread holds the low and high fields in registers (R = 2^RB
+//            values) and the middle field is its index inside the row's
+//            P = 2^PB threads. Global loads and stores are coalesced 16-byte
+//            vectors. All RB register bits get their butterflies.
+//   phase B: after a transpose through shared memory, a thread holds the middle
+//            field (plus, for odd m, one high bit as a batch bit) and does the
+//            remaining butterflies.
+// The transpose buffer is fp32 and XOR-swizzled (the middle field's low bits
+// are flipped by the high field's low bits) so that phase-B scalar accesses hit
+// 32 distinct banks and phase-A 16-byte accesses stay contiguous. The result
+// goes back through the same buffer (in the output type) to phase-A layout for
+// coalesced stores. Arithmetic is fp32 whatever the I/O type.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qwha {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <int LOGN, int V>
+struct Geo {
+  static constexpr int N = 1 << LOGN;
+  static constexpr int LV = V == 8 ? 3 : 2;
+  static constexpr int RB = (LOGN + 1) / 2;
+  static constexpr int R = 1 << RB;
+  static constexpr int PB = LOGN - RB;
+  static constexpr int P = 1 << PB;
+  static constexpr int NB = 2 * RB - LOGN;  // batch bits in phase B (0 or 1)
+  static constexpr int HB = RB - LV;        // high bits in phase-A registers
+  static constexpr int S0 = 5 - LV;
+  static constexpr int S1 = PB < S0 ? PB : S0;
+  static constexpr int S = (HB - NB) < S1 ? (HB - NB) : S1;  // swizzle bits
+  static constexpr int SMASK = (1 << S) - 1;
+  static_assert(HB >= NB && HB >= 0 && PB >= LV, "row too short for this layout");
+  static_assert(P <= kThreads, "row too long for this layout");
+
+  // element index of register q of thread t, phase A
+  __device__ __forceinline__ static int eA(int t, int q) {
+    return (q & (V - 1)) | (t << LV) | ((q >> LV) << (LV + PB));
+  }
+  // element index of register q of thread t, phase B
+  __device__ __forceinline__ static int eB(int t, int q) {
+    return (t & (V - 1)) | ((q & (P - 1)) << LV) | ((t >> LV) << (LV + PB)) |
+           ((q >> PB) << (LV + PB + HB - NB));
+  }
+  // swizzled position in the transpose buffer
+  __device__ __forceinline__ static int phys(int e) {
+    return e ^ (((e >> (LV + PB)) & SMASK) << LV);
+  }
+};
+
+template <typename T, int V>
+__device__ __forceinline__ void load_group(const T *p, float *o) {
+  constexpr int NU = V * (int)sizeof(T) / 16;
+#pragma unroll
+  for (int u = 0; u < NU; ++u) io<T>::unpack(ld_stream(p + u * io<T>::kVec), o + u * io<T>::kVec);
+}
+
+template <typename T, int V>
+__device__ __forceinline__ void store_group(T *p, const float *i) {
+  constexpr int NU = V * (int)sizeof(T) / 16;
+#pragma unroll
+  for (int u = 0; u < NU; ++u) st_stream(p + u * io<T>::kVec, io<T>::pack(i + u * io<T>::kVec));
+}
+
+// Butterflies on register-index bits [B0, B0 + NBITS) of v[0..R).
+template <int R, int B0, int NBITS>
+__device__ __forceinline__ void butterflies(float *v) {
+#pragma unroll
+  for (int b = B0; b < B0 + NBITS; ++b) {
+    const int h = 1 << b;
+#pragma unroll
+    for (int q = 0; q < R; ++q)
+      if (!(q & h)) {
+        const float a = v[q], c = v[q + h];
+        v[q] = a + c;
+        v[q + h] = a - c;
+      }
+  }
+}
+
+template <int LOGN, int V, typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads) fwht_rows_kernel(const Tin *__restrict__ x,
+                                                             Tout *__restrict__ z, int64_t rows,
+                                                             float scale) {
+  using G = Geo<LOGN, V>;
+  constexpr int RPC = kThreads / G::P;  // rows per CTA iteration
+  extern __shared__ __align__(16) float smem[];
+  const int rl = threadIdx.x / G::P;
+  const int t = threadIdx.x % G::P;
+  float *buf = smem + rl * G::N;
+
+  for (int64_t base = (int64_t)blockIdx.x * RPC; base < rows; base += (int64_t)gridDim.x * RPC) {
+    const int64_t row = base + rl;
+    const bool active = row < rows;
+    float v[G::R];
+    if (active) {
+      const Tin *xr = x + row * G::N;
+#pragma unroll
+      for (int h = 0; h < (1 << G::HB); ++h) load_group<Tin, V>(xr + G::eA(t, h << G::LV), v + h * V);
+    } else {
+#pragma unroll
+      for (int q = 0; q < G::R; ++q) v[q] = 0.f;
+    }
+    butterflies<G::R, 0, G::RB>(v);
+
+    __syncthreads();  // the previous iteration's readers are done with buf
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+      float *dst = buf + G::phys(G::eA(t, h << G::LV));
+#pragma unroll
+      for (int u = 0; u < V; u += 4)
+        *reinterpret_cast<float4 *>(dst + u) =
+            make_float4(v[h * V + u], v[h * V + u + 1], v[h * V + u + 2], v[h * V + u + 3]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
+    butterflies<G::R, 0, G::PB>(v);
+    __syncthreads();  // all phase-B reads done before the buffer is reused
+
+    Tout *st = reinterpret_cast<Tout *>(buf);
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) io<Tout>::store1(st + G::phys(G::eB(t, q)), v[q] * scale);
+    __syncthreads();
+    if (active) {
+      Tout *zr = z + row * G::N;
+#pragma unroll
+      for (int h = 0; h < (1 << G::HB); ++h) {
+        const int e = G::eA(t, h << G::LV);
+        const Tout *src = st + G::phys(e);
+        float o[V];
+#pragma unroll
+        for (int u = 0; u < V; u += io<Tout>::kVec)
+          io<Tout>::unpack(*reinterpret_cast<const uint4 *>(src + u), o + u);
+        store_group<Tout, V>(zr + e, o);
+      }
+    }
+  }
+}
+
+// n <= 64: one thread per block, all in registers.
+template <int LOGN, typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads) fwht_small_kernel(const Tin *__restrict__ x,
+                                                              Tout *__restrict__ z, int64_t rows,
+                                                              float scale) {
+  constexpr int N = 1 << LOGN;
+  for (int64_t row = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; row < rows;
+       row += (int64_t)gridDim.x * blockDim.x) {
+    float v[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = io<Tin>::load1(x + row * N + i);
+    butterflies<N, 0, LOGN>(v);
+#pragma unroll
+    for (int i = 0; i < N; ++i) io<Tout>::store1(z + row * N + i, v[i] * scale);
+  }
+}
+
+// 8192 <= n <= 32768: one CTA per block, the block in shared memory, three
+// stages per pass over groups of 8 elements.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(512) fwht_large_kernel(const Tin *__restrict__ x,
+                                                         Tout *__restrict__ z, int64_t rows,
+                                                         int logn, float scale) {
+  extern __shared__ __align__(16) float smem[];
+  const int N = 1 << logn;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) smem[i] = io<Tin>::load1(x + row * N + i);
+    __syncthreads();
+    for (int s = 0; s < logn; s += 3) {
+      const int nb = (logn - s) < 3 ? (logn - s) : 3;
+      const int gsz = 1 << nb;
+      for (int g = threadIdx.x; g < (N >> nb); g += blockDim.x) {
+        const int lo = g & ((1 << s) - 1);
+        const int base = ((g >> s) << (s + nb)) | lo;
+        float v[8];
+        for (int i = 0; i < gsz; ++i) v[i] = smem[base + (i << s)];
+        for (int b = 0; b < nb; ++b)
+          for (int i = 0; i < gsz; ++i)
+            if (!(i & (1 << b))) {
+              const float a = v[i], c = v[i + (1 << b)];
+              v[i] = a + c;
+              v[i + (1 << b)] = a - c;
+            }
+        for (int i = 0; i < gsz; ++i) smem[base + (i << s)] = v[i];
+      }
+      __syncthreads();
+    }
+    for (int i = threadIdx.x; i < N; i += blockDim.x) io<Tout>::store1(z + row * N + i, smem[i] * scale);
+  }
+}
+
+template <int LOGN, typename Tin, typename Tout>
+cudaError_t run_rows(const Tin *x, Tout *z, int64_t rows, float scale, cudaStream_t s) {
+  constexpr int V = (sizeof(Tin) == 2 || sizeof(Tout) == 2) ? 8 : 4;
+  using G = Geo<LOGN, V>;
+  constexpr int RPC = kThreads / G::P;
+  const size_t smem = (size_t)RPC * G::N * sizeof(float);
+  auto k = fwht_rows_kernel<LOGN, V, Tin, Tout>;
+  static bool attr_done = false;  // per instantiation
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  int occ = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  const int64_t need = cdiv(rows, RPC);
+  const int64_t cap = (int64_t)sm_count() * occ;
+  const int grid = (int)(need < cap ? need : cap);
+  k<<<grid, kThreads, smem, s>>>(x, z, rows, scale);
+  return cudaGetLastError();
+}
+
+template <int LOGN, typename Tin, typename Tout>
+cudaError_t run_small(const Tin *x, Tout *z, int64_t rows, float scale, cudaStream_t s) {
+  const int64_t need = cdiv(rows, kThreads);
+  const int64_t cap = (int64_t)sm_count() * 8;
+  fwht_small_kernel<LOGN, Tin, Tout><<<(int)(need < cap ? need : cap), kThreads, 0, s>>>(x, z, rows, scale);
+  return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout>
+cudaError_t run_large(const Tin *x, Tout *z, int64_t rows, int logn, float scale, cudaStream_t s) {
+  const size_t smem = sizeof(float) << logn;
+  auto k = fwht_large_kernel<Tin, Tout>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t cap = (int64_t)sm_count() * 2;
+  k<<<(int)(rows < cap ? rows : cap), 512, smem, s>>>(x, z, rows, logn, scale);
+  return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout>
+cudaError_t dispatch(const void *xv, void *zv, int64_t rows, int logn, float scale, cudaStream_t s) {
+  const Tin *x = static_cast<const Tin *>(xv);
+  Tout *z = static_cast<Tout *>(zv);
+  switch (logn) {
+    case 1: return run_small<1>(x, z, rows, scale, s);
+    case 2: return run_small<2>(x, z, rows, scale, s);
+    case 3: return run_small<3>(x, z, rows, scale, s);
+    case 4: return run_small<4>(x, z, rows, scale, s);
+    case 5: return run_small<5>(x, z, rows, scale, s);
+    case 6: return run_small<6>(x, z, rows, scale, s);
+    case 7: return run_rows<7>(x, z, rows, scale, s);
+    case 8: return run_rows<8>(x, z, rows, scale, s);
+    case 9: return run_rows<9>(x, z, rows, scale, s);
+    case 10: return run_rows<10>(x, z, rows, scale, s);
+    case 11: return run_rows<11>(x, z, rows, scale, s);
+    case 12: return run_rows<12>(x, z, rows, scale, s);
+    default: return run_large(x, z, rows, logn, scale, s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fwht(qwha_dtype din, qwha_dtype dout, const void *x, void *z, int64_t blocks,
+                        int logn, float scale, cudaStream_t s) {
+  if (blocks <= 0) return cudaSuccess;
+  using bf = __nv_bfloat16;
+  if (din == QWHA_F32 && dout == QWHA_F32) return dispatch<float, float>(x, z, blocks, logn, scale, s);
+  if (din == QWHA_BF16 && dout == QWHA_BF16) return dispatch<bf, bf>(x, z, blocks, logn, scale, s);
+  if (din == QWHA_F32 && dout == QWHA_BF16) return dispatch<float, bf>(x, z, blocks, logn, scale, s);
+  return dispatch<bf, float>(x, z, blocks, logn, scale, s);
+}
+
+}  // namespace qwha

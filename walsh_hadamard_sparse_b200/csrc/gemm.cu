@@ -1,0 +1,374 @@
+// Base GEMM of the adapted layer on the 5th-generation tensor cores:
+//   out[M, N] = bf16( A[M, K] . B[N, K]^T + addend[M, N] )
+// with A, B bf16 K-major (row-major with K contiguous) and addend fp32.
+//   forward:  Y  = X W_Q^T + Y_adapter   (A = X, B = W_Q, K = d_in)
+//   backward: dX = dY W_Q + dX_adapter   (A = dY, B = W_Q^T, K = d_out)
+// The adapter term rides in the epilogue, so it costs one fp32 read.
+//
+// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0, one thread : TMA producer. 2-D tensor copies (128B swizzle, no
+//                        multicast) of A and B k-blocks of 64 into a 4-stage
+//                        shared-memory ring, completion counted in bytes on
+//                        the stage's "full" mbarrier.
+//   warp 1, one thread : MMA issuer. tcgen05.mma kind::f16 (bf16 x bf16 ->
+//                        fp32) M=128 N=256 K=16, accumulator in TMEM;
+//                        tcgen05.commit frees the stage ("empty") and, after
+//                        the tile's last k-block, publishes the accumulator.
+//                        Warp 1 also owns the TMEM allocation (512 columns:
+//                        two accumulators, so the epilogue of tile i overlaps
+//                        the main loop of tile i+1).
+//   warps 2..5         : epilogue. tcgen05.ld 32 lanes x 32 columns at a
+//                        time (warp w reads TMEM lanes 32*(w%4)..+31), add
+//                        the fp32 addend, round to bf16, store.
+// Every mbarrier wait is bounded by time: on expiry the thread records a code
+// in the library's device error word, the CTA stops issuing work, drains what
+// it issued, frees TMEM and exits.
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qwha {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t A_BYTES = BM * BK * 2;
+constexpr uint32_t B_BYTES = BN * BK * 2;
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr size_t kGemmSmem = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
+// B bf16 (10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
+// M >> 4 at bit 24.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after kWaitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (now_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  // start >> 4 | LBO 16 B (unused for swizzled K-major) | SBO 1024 B (8 rows of
+  // 128 B) | descriptor version 1 | layout SWIZZLE_128B (2)
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const float *__restrict__ addend, __nv_bfloat16 *__restrict__ out, int M, int N, int K,
+                             unsigned int *err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint32_t base = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+  uint8_t *smem = smem_raw + pad;
+  base += pad;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto tempty = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull(b), 1);
+      mbar_init(tempty(b), 4);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_tiles = (M + BM - 1) / BM, n_tiles = (N + BN - 1) / BN;
+  const int k_blocks = (K + BK - 1) / BK;
+  const int num_tiles = m_tiles * n_tiles;
+
+  auto give_up = [&](unsigned code) {
+    atomicOr(err, code);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int last_parity[STAGES];
+    for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(empty(stage), phase ^ 1)) {
+          give_up(0x1u);
+          break;
+        }
+        if (*abort_flag) break;
+        mbar_expect_tx(full(stage), STAGE_BYTES);
+        tma_load_2d(base + stage * STAGE_BYTES, &tmA, full(stage), kb * BK, m_blk * BM);
+        tma_load_2d(base + stage * STAGE_BYTES + A_BYTES, &tmB, full(stage), kb * BK, n_blk * BN);
+        last_parity[stage] = (int)phase;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    // drain: every copy this thread issued has landed before the CTA exits
+    for (int s = 0; s < STAGES; ++s)
+      if (last_parity[s] >= 0 && !mbar_wait(full(s), (uint32_t)last_parity[s])) give_up(0x2u);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      if (!mbar_wait(tempty(buf), (use & 1) ^ 1)) {
+        give_up(0x4u);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+      bool ok = true;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(full(stage), phase)) {
+          give_up(0x8u);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t da = sw128_desc(base + stage * STAGE_BYTES);
+        const uint64_t db = sw128_desc(base + stage * STAGE_BYTES + A_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_bf16(d_tmem, da + 2ull * k, db + 2ull * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+        umma_commit(empty(stage));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      umma_commit(tfull(buf));
+    }
+    // drain: all issued MMAs complete before TMEM is released
+    umma_commit(done_bar);
+    if (!mbar_wait(done_bar, 0)) give_up(0x10u);
+  } else if (warp >= 2) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      if (*abort_flag) break;
+      if (!mbar_wait(tfull(buf), use & 1)) {
+        give_up(0x20u);
+        break;
+      }
+      tc_fence_after();
+      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      const int row = m_blk * BM + q * 32 + lane;
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
+        const int col0 = n_blk * BN + c * 32;
+        if (row < M && col0 < N) {
+          const float *ad = addend + (int64_t)row * N + col0;
+          __nv_bfloat16 *o = out + (int64_t)row * N + col0;
+          if (col0 + 32 <= N) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 a0 = *reinterpret_cast<const float4 *>(ad + 8 * v);
+              const float4 a1 = *reinterpret_cast<const float4 *>(ad + 8 * v + 4);
+              float f[8] = {__uint_as_float(r[8 * v + 0]) + a0.x, __uint_as_float(r[8 * v + 1]) + a0.y,
+                            __uint_as_float(r[8 * v + 2]) + a0.z, __uint_as_float(r[8 * v + 3]) + a0.w,
+                            __uint_as_float(r[8 * v + 4]) + a1.x, __uint_as_float(r[8 * v + 5]) + a1.y,
+                            __uint_as_float(r[8 * v + 6]) + a1.z, __uint_as_float(r[8 * v + 7]) + a1.w};
+              *reinterpret_cast<uint4 *>(o + 8 * v) = io<__nv_bfloat16>::pack(f);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < N) o[j] = __float2bfloat16_rn(__uint_as_float(r[j]) + ad[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(buf));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// rows x cols bf16 row-major, box = box_rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
+                        int64_t K, cudaStream_t s) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kGemmSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int64_t tiles = cdiv(M, BM) * cdiv(N, BN);
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  gemm_bf16_tcgen05_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, addend, static_cast<__nv_bfloat16 *>(out),
+                                                                (int)M, (int)N, (int)K, device_error_word());
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_fwd(const void *X, const void *wdeq, const float *y_ad, void *Y, int64_t T, int32_t d_out,
+                            int32_t d_in, cudaStream_t s) {
+  return launch_gemm(X, wdeq, y_ad, Y, T, d_out, d_in, s);
+}
+
+cudaError_t launch_gemm_bwd(const void *dY, const void *wdeq_t, const float *dx_ad, void *dX, int64_t T,
+                            int32_t d_out, int32_t d_in, cudaStream_t s) {
+  return launch_gemm(dY, wdeq_t, dx_ad, dX, T, d_in, d_out, s);
+}
+
+}  // namespace qwha

@@ -1,0 +1,370 @@
+// AdaAlloc initialisation of the adapter ("QWHA", papernotes.org 关键设计 2 and
+// 3; gist.science 2.2): a per-channel budget proportional to the channel's
+// quantization error, then inside each channel the largest coefficients of
+// the transformed error dW_Q H, valued by the dense solution.
+//
+// Every rounding that decides an integer is fixed so that budgets and E are
+// reproducible bit for bit by an independent implementation:
+//   * e_i = sqrt(sum_k dW[i,k]^2): squares in fp64 (exact for fp32 inputs),
+//     summed by the pairwise tree in index order over the zero-padded
+//     power-of-two length (any larger padding gives the same value: the extra
+//     leaves are exact zeros). A thread sums an aligned run with a stack of
+//     partial sums (a binary counter), threads combine level by level.
+//   * budget_i = min + floor(fl(pool * e_i) / S) with IEEE fp64 multiply and
+//     divide, capped at d_in with the pool re-shared among the rest.
+//   * the rank key is |V| of the unnormalised transform, fp64 butterflies in
+//     the textbook stage order h = 1, 2, 4, ... (pure adds: no contraction).
+//   * top-b by a most-significant-digit radix select on the fp64 bit patterns,
+//     equal keys taken in increasing index.
+//   * c = float(V * (1/sqrt(n))), one fp64 multiply then one rounding.
+//
+// Kernels: row_norm (one CTA per row), budget (one CTA), select (one CTA per
+// row: butterflies in shared memory, radix select, ordered compaction).
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qwha {
+namespace {
+
+constexpr int kNormThreads = 256;
+constexpr int kBudgetThreads = 1024;
+constexpr int kSelThreads = 256;
+constexpr int kMaxInitDin = 16384;
+
+__device__ __forceinline__ int next_pow2(int v) {
+  int m = 1;
+  while (m < v) m <<= 1;
+  return m;
+}
+
+// Pairwise sum of v[0..L) (L a power of two) in the canonical tree, by a
+// stack of partial sums keyed by level.
+template <typename F>
+__device__ double run_pairwise(int L, F value) {
+  double st[17];
+  int lv[17];
+  int top = 0;
+  for (int i = 0; i < L; ++i) {
+    double s = value(i);
+    int l = 0;
+    while (top > 0 && lv[top - 1] == l) {
+      s = __dadd_rn(st[top - 1], s);
+      --top;
+      ++l;
+    }
+    st[top] = s;
+    lv[top] = l;
+    ++top;
+  }
+  return st[0];
+}
+
+// Canonical tree over the per-thread sums held in sh[0..blockDim) (a power of two).
+__device__ double block_pairwise(double mine, double *sh) {
+  const int t = threadIdx.x;
+  sh[t] = mine;
+  __syncthreads();
+  for (int w = blockDim.x; w > 1; w >>= 1) {
+    double v = 0;
+    if (t < w / 2) v = __dadd_rn(sh[2 * t], sh[2 * t + 1]);
+    __syncthreads();
+    if (t < w / 2) sh[t] = v;
+    __syncthreads();
+  }
+  const double r = sh[0];
+  __syncthreads();
+  return r;
+}
+
+template <typename T>
+__device__ T block_sum(T v, T *sh) {
+  const int t = threadIdx.x;
+  sh[t] = v;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (t < w) sh[t] += sh[t + w];
+    __syncthreads();
+  }
+  const T r = sh[0];
+  __syncthreads();
+  return r;
+}
+
+// Exclusive prefix over threads of v (blockDim a power of two); returns the total in *tot.
+__device__ int64_t block_excl_scan(int64_t v, int64_t *sh, int64_t *tot) {
+  const int t = threadIdx.x;
+  sh[t] = v;
+  __syncthreads();
+  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+    const int64_t a = t >= off ? sh[t - off] : 0;
+    __syncthreads();
+    sh[t] += a;
+    __syncthreads();
+  }
+  const int64_t incl = sh[t];
+  *tot = sh[blockDim.x - 1];
+  __syncthreads();
+  return incl - v;
+}
+
+__global__ void __launch_bounds__(kNormThreads) row_norm_kernel(const float *__restrict__ dW, int d_in,
+                                                                double *__restrict__ e) {
+  __shared__ double sh[kNormThreads];
+  const int64_t row = blockIdx.x;
+  const float *w = dW + row * d_in;
+  int m = next_pow2(d_in);
+  const int L = m > kNormThreads ? m / kNormThreads : 1;
+  const int base = threadIdx.x * L;
+  const double mine = run_pairwise(L, [&](int i) {
+    const int k = base + i;
+    if (k >= d_in) return 0.0;
+    const double x = (double)w[k];
+    return __dmul_rn(x, x);
+  });
+  const double s = block_pairwise(mine, sh);
+  if (threadIdx.x == 0) e[row] = __dsqrt_rn(s);
+}
+
+// Radix select over `n` keys produced by key(i) (eligible when ok(i)): the
+// `want`-th smallest key K and how many keys equal to K are to be taken.
+template <typename KeyF, typename OkF>
+__device__ void radix_select_smallest(int n, int64_t want, KeyF key, OkF ok, uint32_t *hist, uint64_t *K_out,
+                                      int64_t *need_out) {
+  uint64_t prefix = 0;
+  int64_t need = want;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const uint64_t hi_mask = shift == 56 ? 0 : (~0ull << (shift + 8));
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      if (!ok(i)) continue;
+      const uint64_t k = key(i);
+      if ((k & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(k >> shift) & 255], 1u);
+    }
+    __syncthreads();
+    __shared__ int sel_digit;
+    __shared__ int64_t sel_need;
+    if (threadIdx.x == 0) {
+      int64_t cum = 0;
+      int d = 255;
+      for (int b = 0; b < 256; ++b) {
+        if (cum + hist[b] >= need) {
+          d = b;
+          break;
+        }
+        cum += hist[b];
+      }
+      sel_digit = d;
+      sel_need = need - cum;
+    }
+    __syncthreads();
+    prefix |= (uint64_t)sel_digit << shift;
+    need = sel_need;
+    __syncthreads();
+  }
+  *K_out = prefix;
+  *need_out = need;
+}
+
+// Mark, in increasing index order, every eligible key < K and the first `need`
+// keys == K; calls take(i) for each, in an order-preserving compaction whose
+// output slot is passed too.
+template <typename KeyF, typename OkF, typename TakeF>
+__device__ void ordered_take(int n, uint64_t K, int64_t need, KeyF key, OkF ok, TakeF take, int64_t *sh64) {
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int a = threadIdx.x * per, b = min(n, a + per);
+  int64_t eq = 0;
+  for (int i = a; i < b; ++i)
+    if (ok(i) && key(i) == K) ++eq;
+  int64_t tot;
+  const int64_t eq_before = block_excl_scan(eq, sh64, &tot);
+  int64_t cnt = 0;
+  {
+    int64_t e_seen = eq_before;
+    for (int i = a; i < b; ++i) {
+      if (!ok(i)) continue;
+      const uint64_t k = key(i);
+      if (k < K || (k == K && e_seen++ < need)) ++cnt;
+    }
+  }
+  const int64_t slot0 = block_excl_scan(cnt, sh64, &tot);
+  int64_t slot = slot0, e_seen = eq_before;
+  for (int i = a; i < b; ++i) {
+    if (!ok(i)) continue;
+    const uint64_t k = key(i);
+    if (k < K || (k == K && e_seen++ < need)) take(i, slot++);
+  }
+}
+
+__global__ void __launch_bounds__(kBudgetThreads)
+    budget_kernel(const double *__restrict__ e, int d_out, int d_in, int64_t p, int min_per_row, int mode,
+                  int32_t *__restrict__ budgets, int32_t *__restrict__ row_ptr, unsigned char *__restrict__ capped) {
+  __shared__ double shd[kBudgetThreads];
+  __shared__ int64_t sh64[kBudgetThreads];
+  __shared__ uint32_t hist[256];
+  __shared__ int any_new;
+  const int t = threadIdx.x;
+  for (int i = t; i < d_out; i += blockDim.x) capped[i] = 0;
+  __syncthreads();
+  double pool = (double)(p - (int64_t)min_per_row * d_out);
+  const int m = next_pow2(d_out);
+  const int L = m > kBudgetThreads ? m / kBudgetThreads : 1;
+  for (;;) {
+    const double mine = run_pairwise(L, [&](int i) {
+      const int r = t * L + i;
+      return (r < d_out && !capped[r]) ? e[r] : 0.0;
+    });
+    const double S = block_pairwise(mine, shd);
+    int64_t na = 0;
+    for (int i = t; i < d_out; i += blockDim.x) na += !capped[i];
+    const int64_t n_active = block_sum<int64_t>(na, sh64);
+    if (n_active == 0) break;
+    if (t == 0) any_new = 0;
+    __syncthreads();
+    for (int i = t; i < d_out; i += blockDim.x) {
+      if (capped[i]) continue;
+      const double share = S > 0.0 ? floor(__ddiv_rn(__dmul_rn(pool, e[i]), S)) : floor(__ddiv_rn(pool, (double)n_active));
+      const int64_t b = (int64_t)min_per_row + (int64_t)share;
+      budgets[i] = (int32_t)(b > d_in ? d_in + 1 : b);  // d_in + 1 marks "over"
+      if (b > d_in) any_new = 1;
+    }
+    __syncthreads();
+    if (!any_new) break;
+    int64_t nc = 0;
+    for (int i = t; i < d_out; i += blockDim.x)
+      if (!capped[i] && budgets[i] > d_in) {
+        budgets[i] = d_in;
+        capped[i] = 1;
+        ++nc;
+      }
+    const int64_t newly = block_sum<int64_t>(nc, sh64);
+    pool -= (double)newly * (double)(d_in - min_per_row);
+    __syncthreads();
+  }
+  int64_t mysum = 0;
+  for (int i = t; i < d_out; i += blockDim.x) mysum += budgets[i];
+  int64_t R = p - block_sum<int64_t>(mysum, sh64);
+  // remainder: one each, in the mode's order, to rows below d_in
+  while (R > 0) {
+    int64_t el = 0;
+    for (int i = t; i < d_out; i += blockDim.x) el += budgets[i] < d_in;
+    const int64_t n_el = block_sum<int64_t>(el, sh64);
+    if (n_el == 0) break;  // cannot happen for p <= d_in * d_out
+    if (R >= n_el) {
+      for (int i = t; i < d_out; i += blockDim.x)
+        if (budgets[i] < d_in) budgets[i] += 1;
+      R -= n_el;
+      __syncthreads();
+      continue;
+    }
+    auto ok = [&](int i) { return budgets[i] < d_in; };
+    auto key = [&](int i) -> uint64_t {
+      return mode == 0 ? (uint64_t)budgets[i] : ~(uint64_t)__double_as_longlong(e[i]);
+    };
+    uint64_t K;
+    int64_t need;
+    radix_select_smallest(d_out, R, key, ok, hist, &K, &need);
+    __syncthreads();
+    // mark first, then add: the keys must not change while being read
+    ordered_take(d_out, K, need, key, ok, [&](int i, int64_t) { capped[i] = 2; }, sh64);
+    __syncthreads();
+    for (int i = t; i < d_out; i += blockDim.x)
+      if (capped[i] == 2) {
+        budgets[i] += 1;
+        capped[i] = 1;
+      }
+    R = 0;
+    __syncthreads();
+  }
+  __syncthreads();
+  // row_ptr = exclusive scan of budgets, in chunks of blockDim
+  int64_t carry = 0;
+  if (t == 0) row_ptr[0] = 0;
+  for (int base = 0; base < d_out; base += blockDim.x) {
+    const int i = base + t;
+    const int64_t v = i < d_out ? budgets[i] : 0;
+    int64_t tot;
+    const int64_t ex = block_excl_scan(v, sh64, &tot);
+    if (i < d_out) row_ptr[i + 1] = (int32_t)(carry + ex + v);
+    carry += tot;
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+    select_kernel(const float *__restrict__ dW, int d_in, int n, const int32_t *__restrict__ budgets,
+                  const int32_t *__restrict__ row_ptr, int64_t p, int32_t *__restrict__ col_idx,
+                  float *__restrict__ coef) {
+  extern __shared__ __align__(16) double v[];  // d_in values of the row
+  __shared__ uint32_t hist[256];
+  __shared__ int64_t sh64[kSelThreads];
+  const int64_t row = blockIdx.x;
+  const float *w = dW + row * d_in;
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[k] = (double)w[k];
+  __syncthreads();
+  // textbook stage order, three stages per pass over aligned groups of 8
+  const int logn = 31 - __clz(n);
+  for (int s = 0; s < logn; s += 3) {
+    const int nb = min(3, logn - s);
+    const int gsz = 1 << nb;
+    for (int g = threadIdx.x; g < (d_in >> nb); g += blockDim.x) {
+      const int lo = g & ((1 << s) - 1);
+      const int base = ((g >> s) << (s + nb)) | lo;
+      double x[8];
+      for (int i = 0; i < gsz; ++i) x[i] = v[base + (i << s)];
+      for (int b = 0; b < nb; ++b)
+        for (int i = 0; i < gsz; ++i)
+          if (!(i & (1 << b))) {
+            const double a = x[i], c = x[i + (1 << b)];
+            x[i] = __dadd_rn(a, c);
+            x[i + (1 << b)] = __dsub_rn(a, c);
+          }
+      for (int i = 0; i < gsz; ++i) v[base + (i << s)] = x[i];
+    }
+    __syncthreads();
+  }
+  const int b = budgets[row];
+  int64_t start = row_ptr[row];
+  if (b <= 0 || start < 0 || start + b > p) return;
+  const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)n));
+  // largest |V| = smallest complemented magnitude bits
+  auto key = [&](int k) -> uint64_t { return ~((uint64_t)__double_as_longlong(v[k]) & 0x7fffffffffffffffull); };
+  auto ok = [&](int) { return true; };
+  uint64_t K;
+  int64_t need;
+  radix_select_smallest(d_in, b, key, ok, hist, &K, &need);
+  __syncthreads();
+  ordered_take(d_in, K, need, key, ok,
+               [&](int k, int64_t slot) {
+                 if (slot < b) {
+                   col_idx[start + slot] = k;
+                   coef[start + slot] = __double2float_rn(__dmul_rn(v[k], inv));
+                 }
+               },
+               sh64);
+}
+
+}  // namespace
+
+size_t init_workspace(int32_t d_out, int32_t d_in) {
+  (void)d_in;
+  return align_up((size_t)d_out * 8, 256) + align_up((size_t)d_out, 256);
+}
+
+int init_max_din() { return kMaxInitDin; }
+
+cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p,
+                              int32_t min_per_row, int mode, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx,
+                              float *coef, void *ws, cudaStream_t s) {
+  double *e = static_cast<double *>(ws);
+  unsigned char *capped = static_cast<unsigned char *>(ws) + align_up((size_t)d_out * 8, 256);
+  row_norm_kernel<<<d_out, kNormThreads, 0, s>>>(dW, d_in, e);
+  budget_kernel<<<1, kBudgetThreads, 0, s>>>(e, d_out, d_in, p, min_per_row, mode, budgets, row_ptr, capped);
+  const size_t smem = (size_t)d_in * sizeof(double);
+  cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  if (p > 0) select_kernel<<<d_out, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
+  return cudaGetLastError();
+}
+
+}  // namespace qwha

@@ -1,0 +1,71 @@
+// Internal launchers of libqwha (not part of the C ABI). Each enqueues its
+// kernels on `s` and returns the launch status; argument checks live in api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qwha.h"
+
+namespace qwha {
+
+// Transform `blocks` consecutive blocks of 2^logn elements; out = H_unnorm(in) * scale.
+cudaError_t launch_fwht(qwha_dtype din, qwha_dtype dout, const void *x, void *z, int64_t blocks,
+                        int logn, float scale, cudaStream_t s);
+
+}  // namespace qwha
+
+namespace qwha {
+
+// Upper bound on the token chunks of the coefficient-gradient kernel (its
+// partial sums take kSddmmMaxChunks * p floats of workspace at most).
+constexpr int kSddmmMaxChunks = 16;
+
+// out[t, i] = alpha * sum_{j in [seg_ptr[i], seg_ptr[i+1])} val[val_perm ? val_perm[j] : j] * in[t, idx[j]]
+cudaError_t launch_seg_spmm(qwha_dtype din, qwha_dtype dout, const void *in, int64_t T, int W_in,
+                            const int32_t *seg_ptr, const int32_t *idx, const float *val, const int32_t *val_perm,
+                            int64_t nnz, int n_seg, float alpha, void *out, cudaStream_t s);
+
+int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in);
+
+// dc[j] = alpha * sum_t dY[t, r_j] Z[t, k_j] through the tile view; partial is
+// workspace of sddmm_chunks(...) * p floats.
+cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T, int32_t d_out, int32_t d_in,
+                         const int32_t *tile_ptr, const int32_t *tile_pos, const int32_t *tile_rk, int64_t p,
+                         float alpha, float *partial, float *dc, cudaStream_t s);
+
+size_t plan_workspace(int32_t d_out, int32_t d_in);
+int plan_max_row_blocks();
+cudaError_t launch_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr,
+                              const int32_t *col_idx, int32_t *col_ptr, int32_t *row_idx, int32_t *perm,
+                              int32_t *tile_ptr, int32_t *tile_pos, int32_t *tile_rk, void *ws,
+                              cudaStream_t s);
+
+}  // namespace qwha
+
+namespace qwha {
+
+// AdaAlloc (init.cu)
+size_t init_workspace(int32_t d_out, int32_t d_in);
+int init_max_din();
+cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p,
+                              int32_t min_per_row, int mode, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx,
+                              float *coef, void *ws, cudaStream_t s);
+
+// Base weight (dequant.cu): bf16 W_Q [d_out, d_in] or its transpose [d_in, d_out].
+size_t wdeq_bytes(int32_t d_out, int32_t d_in);
+cudaError_t launch_dequant(int bits, int group, int32_t d_out, int32_t d_in, const uint8_t *qw, const float *scales,
+                           const uint8_t *zeros, void *out, bool transposed, cudaStream_t s);
+
+// Base GEMM with fp32 addend in the epilogue (gemm.cu).
+cudaError_t launch_gemm_fwd(const void *X, const void *wdeq, const float *y_ad, void *Y, int64_t T, int32_t d_out,
+                            int32_t d_in, cudaStream_t s);
+cudaError_t launch_gemm_bwd(const void *dY, const void *wdeq_t, const float *dx_ad, void *dX, int64_t T,
+                            int32_t d_out, int32_t d_in, cudaStream_t s);
+
+// Device error word and plan validation (misc.cu).
+cudaError_t read_and_clear_error_word(unsigned int *word, cudaStream_t s);
+const char *validate_message(unsigned int code);
+cudaError_t launch_validate(const qwha_adapter *a, cudaStream_t s, uint32_t *code, int64_t *where);
+
+}  // namespace qwha
