@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Throughput of one Walsh-Hadamard-adapted linear layer (forward + backward) on B200.
+
+A step is one pass of the whole hot path over one batch of seeded synthetic
+tokens: forward transform Z = X H, sparse product, dequantized base GEMM with
+the adapter term in its epilogue; backward coefficient gradient (SDDMM), CSC
+gather + transform, base GEMM for dX; and, with N > 1 GPUs, the data-parallel
+sum of the coefficient gradients (NCCL all-reduce). The workload is the
+LLaMA-7B q_proj shape: d_in = d_out = 4096, 8192 tokens per GPU (16 x 512),
+4-bit group-128 round-to-nearest base weight, p = 524288 coefficients chosen
+by AdaAlloc. AdaAlloc itself (a one-off per layer) is timed separately.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs its own tokens; rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, layer_inputs, rank_rows  # noqa: E402
+
+METRIC = "WHA adapter fwd+bwd tokens/s per layer; achieved HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+WORKLOAD = "q_proj"
+FLUSH_BYTES = 512 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+ALU_LANES_PER_SM = 128  # fp32 FMA lanes per SM (4 partitions x 32)
+
+KERNEL_SOURCES = {
+    "fwht_fwd": ["fwht.cu"], "fwht_bwd": ["fwht.cu"], "spmm_fwd": ["sparse.cu"], "gather_bwd": ["sparse.cu"],
+    "sddmm_dc": ["sparse.cu"], "dequant": ["dequant.cu"], "dequant_t": ["dequant.cu"], "gemm_fwd": ["gemm.cu"],
+    "gemm_bwd": ["gemm.cu"], "init_alloc": ["init.cu"], "plan_build": ["plan.cu"],
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def source_sha(files):
+    h = hashlib.sha256()
+    for f in files + ["common.cuh"]:
+        h.update(open(os.path.join(ROOT, "walsh_hadamard_sparse_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(stage):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(stage)
+    if not d or d.get("source_sha") != source_sha(KERNEL_SOURCES.get(stage, [])):
+        return None
+    return d.get("dram_bytes_per_launch_full_size")
+
+
+# --------------------------------------------------------------------------- work per stage
+
+
+def stage_work(stage, spec, T, bits):
+    """(kind, amount per launch, unit) of algorithmic work; kind in {hbm, tensor, alu}."""
+    di, do, p = spec.d_in, spec.d_out, spec.p
+    qbytes = do * di * bits // 8 + (do * di // spec.group) * 5
+    table = {
+        "fwht_fwd": ("hbm", 4.0 * T * di),  # read X bf16, write Z bf16
+        "fwht_bwd": ("hbm", 8.0 * T * di),  # read dZ fp32, write dX_adapter fp32
+        "dequant": ("hbm", qbytes + 2.0 * do * di),
+        "dequant_t": ("hbm", qbytes + 2.0 * do * di),
+        "spmm_fwd": ("alu", 2.0 * p * T),
+        "gather_bwd": ("alu", 2.0 * p * T),
+        "sddmm_dc": ("alu", 2.0 * p * T),
+        "gemm_fwd": ("tensor", 2.0 * T * di * do),
+        "gemm_bwd": ("tensor", 2.0 * T * di * do),
+    }
+    return table.get(stage)
+
+
+def stage_bytes(stage, spec, T, bits):
+    """Algorithmic HBM bytes per launch (every stage), for the GB/s column."""
+    di, do, p = spec.d_in, spec.d_out, spec.p
+    qbytes = do * di * bits // 8 + (do * di // spec.group) * 5
+    return {
+        "fwht_fwd": 4.0 * T * di,
+        "fwht_bwd": 8.0 * T * di,
+        "dequant": qbytes + 2.0 * do * di,
+        "dequant_t": qbytes + 2.0 * do * di,
+        "spmm_fwd": 2.0 * T * di + 4.0 * T * do + 8.0 * p + 4.0 * do,
+        "gather_bwd": 2.0 * T * do + 4.0 * T * di + 12.0 * p + 4.0 * di,
+        "sddmm_dc": 2.0 * T * (di + do) + 8.0 * p,
+        "gemm_fwd": 2.0 * T * di + 2.0 * do * di + 4.0 * T * do + 2.0 * T * do,
+        "gemm_bwd": 2.0 * T * do + 2.0 * do * di + 4.0 * T * di + 2.0 * T * di,
+    }.get(stage, 0.0)
+
+
+def peak_for(kind, peaks):
+    if kind == "hbm":
+        return peaks["hbm_gbs"], "GB/s", "HBM copy bandwidth, " + peaks["_source"]
+    if kind == "tensor":
+        return peaks["bf16_tflops_sustained"], "TFLOP/s", "cuBLAS bf16 sustained, " + peaks["_source"]
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    return 148 * ALU_LANES_PER_SM * 2 * mhz * 1e6 / 1e12, "TFLOP/s", "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock"
+
+
+# --------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (read-only queries)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            v = [x.strip() for x in line.split(",")]
+            if len(v) < 10:
+                continue
+            try:
+                rows.append(dict(sm=float(v[1]), mx=float(v[2]), util=float(v[4]), hw=v[6], hwt=v[7], swt=v[8],
+                                 pcap=v[9]))
+            except ValueError:
+                continue
+        load = [r for r in rows if r["util"] >= 50] or rows
+        if not load:
+            return None
+        reasons = set()
+        for r in load:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                            ("pcap", "sw_power_cap")):
+                if r[k].lower() in ("active", "1", "yes"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["mx"] for r in load),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+
+_ORACLE_INIT = {}
+
+
+def oracle_tokens_per_s(spec, d, X, dY, tokens, threads=0):
+    """The oracle's forward + backward over `tokens` token rows (dc over all p entries); returns (tokens/s, s, cores).
+    E and c come from the oracle's own AdaAlloc on the same dW_Q (computed once, untimed)."""
+    import oracle
+
+    cores = oracle.set_threads(threads)
+    if spec.name not in _ORACLE_INIT:
+        _ORACLE_INIT[spec.name] = oracle.init_alloc(d["dWq"], spec.p, spec.had_block, spec.min_per_row, spec.remainder)
+    init = _ORACLE_INIT[spec.name]
+    rp, ci, cf = init["row_ptr"], init["col_idx"], init["coef"]
+    rows = oracle.csr_rows(rp)
+    t0 = time.perf_counter()
+    Wq = oracle.dequant(d["qweight"], d["scales"], d["zeros"], spec.bits, spec.group, spec.d_out, spec.d_in)
+    oracle.adapter_fwd(rp, ci, cf, X[:tokens], spec.d_out, spec.had_block, 1.0, Wq)
+    oracle.adapter_bwd_dx(rp, ci, cf, dY[:tokens], spec.d_in, spec.had_block, 1.0, Wq)
+    oracle.adapter_bwd_dc(X[:tokens], dY[:tokens], rows, ci, spec.had_block, 1.0)
+    dt = time.perf_counter() - t0
+    return tokens / dt, dt, cores
+
+
+def run_reference(args, spec):
+    """The oracle as the reference arm: every step is one sampled token's full fwd+bwd."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    d = layer_inputs(spec, args.seed, WORKLOAD, parts=("W", "X", "dY"), rows=np.arange(64))
+    probe, t_probe, cores = oracle_tokens_per_s(spec, d, d["X"], d["dY"], 1)
+    budget_s = 150.0
+    steps = int(max(1, min(args.steps, budget_s // max(t_probe, 1e-3) - min(args.warmup, 1))))
+    for w in range(min(args.warmup, 1)):
+        oracle_tokens_per_s(spec, d, d["X"][w + 1 :], d["dY"][w + 1 :], 1)
+    total = 0.0
+    for i in range(steps):
+        r = (i + 2) % 64
+        _, dt, _ = oracle_tokens_per_s(spec, d, d["X"][r:], d["dY"][r:], 1)
+        total += dt
+    value = steps / total
+    sample = (f"1 token per step (Y and dX for that token, dc over all {spec.p} coefficients); {steps} of "
+              f"{args.steps} requested steps timed, bounded to ~{int(budget_s)} s of host time")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
+        "warmup": min(args.warmup, 1), "ms_per_step": 1e3 * total / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(spec, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(spec, n):
+    return {
+        "workload": (f"{WORKLOAD}: d_in={spec.d_in} d_out={spec.d_out} T={spec.T} tokens per GPU (16 x 512), "
+                     f"{spec.bits}-bit g{spec.group} RTN base weight, p={spec.p} (LoRA r=64 count), AdaAlloc E"),
+        "global_batch": spec.T * n, "seq_len": 512, "parallelism": f"dp{n}",
+        "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write)",
+    }
+
+
+# --------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    spec = CONFIGS[WORKLOAD][0]
+    if args.impl == "reference":
+        return run_reference(args, spec)
+
+    import torch
+    import torch.distributed as dist
+
+    import walsh_hadamard_sparse_b200 as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    T = spec.T
+    d = layer_inputs(spec, args.seed, WORKLOAD, parts=("W",))
+    act = layer_inputs(spec, args.seed, WORKLOAD, parts=("X", "dY"), rows=rank_rows(rank, T))
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    X, dY = bf16(act["X_bits"]), bf16(act["dY_bits"])
+    dWq = torch.from_numpy(d["dWq"]).to(dev)
+    wq = W.QWeight(spec.bits, spec.group, torch.from_numpy(d["qweight"]).to(dev),
+                   torch.from_numpy(d["scales"]).to(dev), torch.from_numpy(d["zeros"]).to(dev))
+    peaks = load_peaks()
+
+    # ---- AdaAlloc (one-off per layer), timed on its own
+    for _ in range(2):
+        e = W.init_alloc(dWq, spec.p, spec.had_block, spec.min_per_row, spec.remainder)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    init_ms = []
+    for _ in range(5):
+        ev[0].record()
+        e = W.init_alloc(dWq, spec.p, spec.had_block, spec.min_per_row, spec.remainder)
+        ev[1].record()
+        torch.cuda.synchronize()
+        init_ms.append(ev[0].elapsed_time(ev[1]))
+    a = W.Adapter(spec.d_in, spec.d_out, spec.had_block, spec.p, e["row_ptr"], e["col_idx"], e["coef"])
+    W.plan_build(a)
+
+    alpha = 1.0
+    Z = torch.empty_like(X)
+    Y = torch.empty((T, spec.d_out), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty_like(X)
+    dc = torch.empty(spec.p, dtype=torch.float32, device=dev)
+    ws_f = torch.empty(W.workspace_size(0, spec.d_out, spec.d_in, spec.p, T, True), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(W.workspace_size(1, spec.d_out, spec.d_in, spec.p, T, True), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        W.adapter_fwd(a, X, alpha, wq, Z_out=Z, Y=Y, ws=ws_f)
+        W.adapter_bwd(a, dY, Z, alpha, wq, dc=dc, dX=dX, ws=ws_b)
+        if world > 1:
+            dist.all_reduce(dc)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if not (torch.isfinite(Y.float()).all() and torch.isfinite(dc).all() and torch.isfinite(dX.float()).all()):
+        raise RuntimeError("non-finite output")
+
+    # ---- timed region
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    W.stage_report()
+    W.stage_timing(True)
+    clocks = ClockSampler() if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    W.stage_timing(False)
+    rep = W.stage_report()
+    t_ms = sum(s.elapsed_time(e_) for s, e_ in zip(starts, ends))
+    if world > 1:
+        tt = torch.tensor([t_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms = float(tt.item())
+    value = world * T * K / (t_ms / 1e3)
+
+    # ---- per-stage roofline (this rank's stage events, same timed region)
+    kernels = {}
+    for name, (calls, launches, ms) in rep.items():
+        if calls == 0:
+            continue
+        w = stage_work(name, spec, T, spec.bits)
+        per = ms / calls
+        k = {"launches": launches, "ms_per_launch": per, "share": None,
+             "alg_bytes": stage_bytes(name, spec, T, spec.bits)}
+        k["alg_GBps"] = k["alg_bytes"] / (per / 1e3) / 1e9
+        if w:
+            kind, amount = w
+            peak, unit, _ = peak_for(kind, peaks)
+            ach = amount / (per / 1e3) / (1e9 if unit == "GB/s" else 1e12)
+            k.update(bound=kind, achieved=ach, peak=peak, unit=unit, frac=ach / peak)
+        kernels[name] = k
+    total_stage_ms = sum(v["ms_per_launch"] * rep[n][0] for n, v in kernels.items())
+    for n, v in kernels.items():
+        v["share"] = v["ms_per_launch"] * rep[n][0] / total_stage_ms
+    dom = max((n for n in kernels if "bound" in kernels[n]), key=lambda n: kernels[n]["share"])
+    kd = kernels[dom]
+    _, _, peak_note = peak_for(kd["bound"], peaks)
+    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
+                "unit": kd["unit"], "frac": kd["frac"], "traffic": ncu_traffic(dom), "peak_source": peak_note}
+    launches = sum(v[1] for v in rep.values())
+
+    # ---- end to end through host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        Xh = torch.empty_like(X, device="cpu").pin_memory()
+        dYh = torch.empty_like(dY, device="cpu").pin_memory()
+        Xh.copy_(X)
+        dYh.copy_(dY)
+        dch = torch.empty_like(dc, device="cpu").pin_memory()
+        Ke = args.e2e_steps
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            X.copy_(Xh, non_blocking=True)
+            dY.copy_(dYh, non_blocking=True)
+            step()
+            dch.copy_(dc, non_blocking=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0.record()
+        for _ in range(Ke):
+            X.copy_(Xh, non_blocking=True)
+            dY.copy_(dYh, non_blocking=True)
+            step()
+            dch.copy_(dc, non_blocking=True)
+        s1.record()
+        torch.cuda.synchronize()
+        te = s0.elapsed_time(s1)
+        if world > 1:
+            tt = torch.tensor([te], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            te = float(tt.item())
+        e2e = {"value": world * T * Ke / (te / 1e3), "unit": UNIT, "steps": Ke,
+               "h2d_bytes_per_step": X.numel() * 2 + dY.numel() * 2, "d2h_bytes_per_step": dc.numel() * 4,
+               "note": "pinned host X and dY copied in and dc read back every step; Y, Z and dX stay on the GPU"}
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host_act = {"X": act["X"][:64].astype(np.float64), "dY": act["dY"][:64].astype(np.float64)}
+        _, t1, cores = oracle_tokens_per_s(spec, d, host_act["X"], host_act["dY"], 1)
+        toks = int(max(1, min(64, 15.0 / max(t1, 1e-3))))
+        rate, dt, cores = oracle_tokens_per_s(spec, d, host_act["X"], host_act["dY"], toks)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{toks} tokens of the same layer (Y, dX for them; dc over all {spec.p} coefficients), "
+                         f"{dt:.1f} s of host time"}
+
+    init_bytes = 2 * 4.0 * spec.d_in * spec.d_out + 8.0 * spec.p
+    init_med = statistics.median(init_ms)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": t_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; stands in for LLaMA-7B q_proj weights and activations)",
+        "config": config_block(spec, world),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "kernels": kernels,
+        "init": {"ms": init_med, "alg_GBps": init_bytes / (init_med / 1e3) / 1e9,
+                 "frac_hbm": init_bytes / (init_med / 1e3) / 1e9 / peaks["hbm_gbs"],
+                 "what": "AdaAlloc on dW_Q (4096 x 4096 fp32): norms, budgets, fp64 transform, top-k; one-off per layer"},
+        "hbm_GBps_step": sum(stage_bytes(n, spec, T, spec.bits) * rep[n][0] for n in kernels) / (t_ms / 1e3) / 1e9,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -190,6 +190,20 @@ qwha_status qwha_validate_plan(const qwha_adapter *a, void *stream);
  * wait (QWHA_ERR_TIMEOUT) or a CUDA error (QWHA_ERR_CUDA); clears the word. */
 qwha_status qwha_check_stream_status(void *stream);
 
+/* Tracing aid: per-stage device time of the library's own kernels. While
+ * enabled (off by default), every stage a call runs (the kernels of one step
+ * of the path, e.g. the forward transform or the base GEMM) is bracketed by a
+ * pair of CUDA events recorded on the call's stream. qwha_stage_report waits
+ * for those events and fills, for each stage i < qwha_stage_count(), the
+ * number of stage executions calls[i], the kernels they launched launches[i]
+ * and their total device time ms[i] since the previous report; then it
+ * resets the counters. Arrays are host memory of qwha_stage_count() entries.
+ * Not for use inside CUDA graph capture. */
+void qwha_stage_timing(int32_t enable);
+int32_t qwha_stage_count(void);
+const char *qwha_stage_name(int32_t i);
+qwha_status qwha_stage_report(int64_t *calls, int64_t *launches, double *ms);
+
 const char *qwha_status_string(qwha_status s);
 const char *qwha_last_error(void);
 const char *qwha_version(void);

@@ -15,6 +15,8 @@ from .api import (  # noqa: F401
     init_alloc,
     plan_build,
     plan_tiles,
+    stage_report,
+    stage_timing,
     validate_plan,
     workspace_size,
 )

@@ -54,6 +54,10 @@ _SIGNATURES = {
     "qwha_workspace_size": (sz, [ctypes.c_int, i32, i32, i64, i64, i32]),
     "qwha_validate_plan": (ctypes.c_int, [ctypes.POINTER(QwhaAdapter), P]),
     "qwha_check_stream_status": (ctypes.c_int, [P]),
+    "qwha_stage_timing": (None, [i32]),
+    "qwha_stage_count": (i32, []),
+    "qwha_stage_name": (ctypes.c_char_p, [i32]),
+    "qwha_stage_report": (ctypes.c_int, [P, P, P]),
     "qwha_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qwha_last_error": (ctypes.c_char_p, []),
     "qwha_version": (ctypes.c_char_p, []),

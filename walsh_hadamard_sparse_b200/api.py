@@ -188,3 +188,22 @@ def plan_build(a: Adapter, ws: torch.Tensor | None = None) -> Adapter:
 def validate_plan(a: Adapter) -> None:
     cs = a.c_struct()
     check(lib().qwha_validate_plan(ctypes.byref(cs), _stream()), "qwha_validate_plan")
+
+
+def stage_timing(enable: bool) -> None:
+    """Turn the library's per-stage event timing on or off."""
+    lib().qwha_stage_timing(int(bool(enable)))
+
+
+def stage_report() -> dict:
+    """{stage: (calls, kernel launches, total ms)} since the previous report (synchronises)."""
+    import numpy as np
+
+    h = lib()
+    n = h.qwha_stage_count()
+    calls = np.zeros(n, dtype=np.int64)
+    launches = np.zeros(n, dtype=np.int64)
+    ms = np.zeros(n, dtype=np.float64)
+    check(h.qwha_stage_report(calls.ctypes.data_as(ctypes.c_void_p), launches.ctypes.data_as(ctypes.c_void_p),
+                              ms.ctypes.data_as(ctypes.c_void_p)), "qwha_stage_report")
+    return {h.qwha_stage_name(i).decode(): (int(calls[i]), int(launches[i]), float(ms[i])) for i in range(n)}

@@ -6,6 +6,7 @@
 #include <stdio.h>
 
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -68,6 +69,112 @@ qwha_status check_hadamard(int32_t n, int32_t had_block) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- stage timing
+
+namespace {
+
+enum Stage {
+  ST_FWHT_FWD,
+  ST_SPMM_FWD,
+  ST_DEQUANT,
+  ST_GEMM_FWD,
+  ST_SDDMM,
+  ST_GATHER_BWD,
+  ST_FWHT_BWD,
+  ST_DEQUANT_T,
+  ST_GEMM_BWD,
+  ST_INIT,
+  ST_PLAN,
+  ST_FWHT,
+  ST_COUNT
+};
+const char *kStageNames[ST_COUNT] = {"fwht_fwd",  "spmm_fwd",  "dequant",  "gemm_fwd",   "sddmm_dc",   "gather_bwd",
+                                     "fwht_bwd",  "dequant_t", "gemm_bwd", "init_alloc", "plan_build", "fwht"};
+
+struct StageRec {
+  int stage, kernels;
+  cudaEvent_t a, b;
+};
+
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<StageRec> g_pending;
+std::vector<cudaEvent_t> g_pool;
+int64_t g_calls[ST_COUNT], g_launches[ST_COUNT];
+double g_ms[ST_COUNT];
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one stage with events when timing is on; counts launches always-on cheaply.
+struct StageScope {
+  int stage, kernels;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  StageScope(int st, int k, cudaStream_t str) : stage(st), kernels(k), s(str) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    if (!g_prof_on) return;
+    a = take_event();
+    if (a) cudaEventRecord(a, s);
+  }
+  ~StageScope() {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    if (!g_prof_on || !a) return;
+    cudaEvent_t b = take_event();
+    if (!b) return;
+    cudaEventRecord(b, s);
+    g_pending.push_back({stage, kernels, a, b});
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+void qwha_stage_timing(int32_t enable) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = enable != 0;
+}
+
+int32_t qwha_stage_count(void) { return ST_COUNT; }
+
+const char *qwha_stage_name(int32_t i) { return (i >= 0 && i < ST_COUNT) ? kStageNames[i] : ""; }
+
+qwha_status qwha_stage_report(int64_t *calls, int64_t *launches, double *ms) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  qwha_status st = QWHA_OK;
+  for (const StageRec &r : g_pending) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess && st == QWHA_OK) st = cuda_status(e, "stage events");
+    g_calls[r.stage] += 1;
+    g_launches[r.stage] += r.kernels;
+    g_ms[r.stage] += t;
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_pending.clear();
+  for (int i = 0; i < ST_COUNT; ++i) {
+    if (calls) calls[i] = g_calls[i];
+    if (launches) launches[i] = g_launches[i];
+    if (ms) ms[i] = g_ms[i];
+    g_calls[i] = g_launches[i] = 0;
+    g_ms[i] = 0.0;
+  }
+  return st;
+}
+
+}  // extern "C"
+
 extern "C" {
 
 const char *qwha_status_string(qwha_status s) {
@@ -103,6 +210,7 @@ qwha_status qwha_fwht(qwha_dtype dt, const void *x, void *z, int64_t rows, int32
   const int logn = ilog2(had_block);
   const float scale = (float)(1.0 / sqrt((double)had_block));
   (void)dtype_name;
+  StageScope sc(ST_FWHT, 1, (cudaStream_t)stream);
   return cuda_status(launch_fwht(dt, dt, x, z, rows * (n / had_block), logn, scale, (cudaStream_t)stream),
                      "fwht launch");
 }
@@ -225,9 +333,14 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   cudaStream_t s = (cudaStream_t)stream;
   const int logn = ilog2(a->had_block);
   const float inv = (float)(1.0 / sqrt((double)a->had_block));
-  cudaError_t e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
+  cudaError_t e;
+  {
+    StageScope sc(ST_FWHT_FWD, 1, s);
+    e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "fwht");
   if (!wq) {
+    StageScope sc(ST_SPMM_FWD, 1, s);
     e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
                         alpha, Y, s);
     return cuda_status(e, "spmm");
@@ -235,11 +348,18 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   Carver cv(ws);
   float *y_ad = static_cast<float *>(cv.take((size_t)T * a->d_out * 4));
   void *wdeq = cv.take(wdeq_bytes(a->d_out, a->d_in));
-  e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
-                      alpha, y_ad, s);
+  {
+    StageScope sc(ST_SPMM_FWD, 1, s);
+    e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
+                        alpha, y_ad, s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "spmm");
-  e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, false, s);
+  {
+    StageScope sc(ST_DEQUANT, 1, s);
+    e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, false, s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "dequant");
+  StageScope sc(ST_GEMM_FWD, 1, s);
   return cuda_status(launch_gemm_fwd(X, wdeq, y_ad, Y, T, a->d_out, a->d_in, s), "base GEMM");
 }
 
@@ -263,23 +383,40 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   Carver cv(ws);
   float *partial = static_cast<float *>(cv.take((size_t)kSddmmMaxChunks * (size_t)(a->p > 0 ? a->p : 1) * 4));
   float *dz = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
-  cudaError_t e = launch_sddmm(dt, dY, Z, T, a->d_out, a->d_in, a->tile_ptr, a->tile_pos, a->tile_rk, a->p, alpha,
-                               partial, dc, s);
+  cudaError_t e;
+  {
+    StageScope sc(ST_SDDMM, 2, s);
+    e = launch_sddmm(dt, dY, Z, T, a->d_out, a->d_in, a->tile_ptr, a->tile_pos, a->tile_rk, a->p, alpha, partial, dc,
+                     s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "sddmm");
   if (!dX || T == 0) return QWHA_OK;
-  e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, a->coef, a->perm, a->p, a->d_in, alpha,
-                      dz, s);
+  {
+    StageScope sc(ST_GATHER_BWD, 1, s);
+    e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, a->coef, a->perm, a->p, a->d_in,
+                        alpha, dz, s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "gather");
   const int logn = ilog2(a->had_block);
   const float inv = (float)(1.0 / sqrt((double)a->had_block));
   const int64_t blocks = T * (a->d_in / a->had_block);
-  if (!wq) return cuda_status(launch_fwht(QWHA_F32, dt, dz, dX, blocks, logn, inv, s), "fwht");
+  if (!wq) {
+    StageScope sc(ST_FWHT_BWD, 1, s);
+    return cuda_status(launch_fwht(QWHA_F32, dt, dz, dX, blocks, logn, inv, s), "fwht");
+  }
   float *dx_ad = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
   void *wdeq = cv.take(wdeq_bytes(a->d_out, a->d_in));
-  e = launch_fwht(QWHA_F32, QWHA_F32, dz, dx_ad, blocks, logn, inv, s);
+  {
+    StageScope sc(ST_FWHT_BWD, 1, s);
+    e = launch_fwht(QWHA_F32, QWHA_F32, dz, dx_ad, blocks, logn, inv, s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "fwht");
-  e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, true, s);
+  {
+    StageScope sc(ST_DEQUANT_T, 1, s);
+    e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, true, s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "dequant");
+  StageScope sc(ST_GEMM_BWD, 1, s);
   return cuda_status(launch_gemm_bwd(dY, wdeq, dx_ad, dX, T, a->d_out, a->d_in, s), "base GEMM (dX)");
 }
 
@@ -303,6 +440,7 @@ qwha_status qwha_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_
   }
   qwha_status st = check_ws(ws, ws_bytes, plan_workspace(d_out, d_in));
   if (st != QWHA_OK) return st;
+  StageScope sc(ST_PLAN, 5, (cudaStream_t)stream);
   return cuda_status(launch_plan_build(d_out, d_in, p, row_ptr, col_idx, col_ptr, row_idx, perm, tile_ptr, tile_pos,
                                        tile_rk, ws, (cudaStream_t)stream),
                      "plan_build");
@@ -350,6 +488,7 @@ qwha_status qwha_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32
     QWHA_CHECK_PTR(coef, "coef");
   }
   if ((st = check_ws(ws, ws_bytes, init_workspace(d_out, d_in))) != QWHA_OK) return st;
+  StageScope sc(ST_INIT, 3, (cudaStream_t)stream);
   return cuda_status(launch_init_alloc(dWq, d_out, d_in, had_block, p, min_per_row, (int)mode, budgets, row_ptr,
                                        col_idx, coef, ws, (cudaStream_t)stream),
                      "init_alloc");

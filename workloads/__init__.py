@@ -19,5 +19,6 @@ from .synth import (  # noqa: F401
     pack_codes,
     quantize_rtn,
     random_pattern,
+    rank_rows,
     rng_for,
 )

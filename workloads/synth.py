@@ -315,3 +315,8 @@ __all__ = [
     "random_pattern",
     "rng_for",
 ]
+
+
+def rank_rows(rank: int, tokens_per_rank: int) -> np.ndarray:
+    """Token rows of the seeded stream that data-parallel rank `rank` processes."""
+    return np.arange(rank * tokens_per_rank, (rank + 1) * tokens_per_rank)
