@@ -172,6 +172,30 @@ qwha_status qwha_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_
                             int32_t *perm, int32_t *tile_ptr, int32_t *tile_pos,
                             int32_t *tile_rk, void *ws, size_t ws_bytes, void *stream);
 
+/* Size of the library's own static device scratch used by
+ * qwha_coef_grad_noalloc (16 MiB, held on every GPU that loads the library
+ * until the process exits). */
+#define QWHA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* The coefficient gradient dc of qwha_adapter_bwd, for callers that cannot
+ * allocate device memory and cannot pass a workspace: for example a custom-op
+ * slot of a host framework that hands the op only its inputs and outputs, or
+ * a step that must not call cudaMalloc (it may synchronise the device and can
+ * fail under a fixed memory budget). There is no counterpart on the pages; it
+ * is an engineering variant of the backward's first stage.
+ *   dc[j] = alpha * sum_t dY[t, r_j] Z[t, k_j]   fp32 [p], CSR order
+ * Same arguments and result as the dc of qwha_adapter_bwd (tile view of `a`
+ * required; dX is not computed). The partial sums live in one static array of
+ * QWHA_NOALLOC_SCRATCH_BYTES inside the library; a call needing more returns
+ * QWHA_ERR_WORKSPACE and launches nothing (the q_proj layer, p = 524288 at
+ * 8192 tokens, needs about 10.5 MB). Nothing is allocated. All calls on a
+ * device share that array: calls whose work overlaps on the GPU race and must
+ * be serialised by the caller; each call clears the partial sums it uses. The
+ * first call on a device looks up the array's device address (once, with
+ * that device current), so it must come before any stream capture. */
+qwha_status qwha_coef_grad_noalloc(const qwha_adapter *a, qwha_dtype dt, const void *dY, const void *Z,
+                                   int64_t T, float alpha, float *dc, void *stream);
+
 /* Number of QWHA_TILE x QWHA_TILE blocks of F. */
 int64_t qwha_plan_tiles(int32_t d_out, int32_t d_in);
 

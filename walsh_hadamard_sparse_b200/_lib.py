@@ -48,6 +48,7 @@ _SIGNATURES = {
         ctypes.c_int,
         [ctypes.POINTER(QwhaAdapter), ctypes.POINTER(QwhaQweight), ctypes.c_int, P, P, i64, f32, P, P, P, sz, P],
     ),
+    "qwha_coef_grad_noalloc": (ctypes.c_int, [ctypes.POINTER(QwhaAdapter), ctypes.c_int, P, P, i64, f32, P, P]),
     "qwha_init_alloc": (ctypes.c_int, [P, i32, i32, i32, i64, i32, ctypes.c_int, P, P, P, P, P, sz, P]),
     "qwha_plan_build": (ctypes.c_int, [i32, i32, i64, P, P, P, P, P, P, P, P, P, sz, P]),
     "qwha_plan_tiles": (i64, [i32, i32]),
