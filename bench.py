@@ -79,38 +79,31 @@ def ncu_traffic(stage):
 
 
 def stage_work(stage, spec, T, bits):
-    """(kind, amount per launch, unit) of algorithmic work; kind in {hbm, tensor, alu}."""
+    """(bound, algorithmic work per stage call, HBM bytes per stage call) for the layer of `spec` at T tokens.
+    bound is hbm (work = bytes), tensor or alu (work = FLOP); None for stages without a model."""
     di, do, p = spec.d_in, spec.d_out, spec.p
-    qbytes = do * di * bits // 8 + (do * di // spec.group) * 5
-    table = {
-        "fwht_fwd": ("hbm", 4.0 * T * di),  # read X bf16, write Z bf16
-        "fwht_bwd": ("hbm", 8.0 * T * di),  # read dZ fp32, write dX_adapter fp32
-        "dequant": ("hbm", qbytes + 2.0 * do * di),
-        "dequant_t": ("hbm", qbytes + 2.0 * do * di),
-        "spmm_fwd": ("alu", 2.0 * p * T),
-        "gather_bwd": ("alu", 2.0 * p * T),
-        "sddmm_dc": ("alu", 2.0 * p * T),
-        "gemm_fwd": ("tensor", 2.0 * T * di * do),
-        "gemm_bwd": ("tensor", 2.0 * T * di * do),
+    qbytes = do * di * bits / 8 + (do * di / spec.group) * 5
+    w = {
+        # forward transform: read X, write Z (bf16)
+        "fwht_fwd": ("hbm", 4.0 * T * di, 4.0 * T * di),
+        # backward transform: read dZ (fp32), write dX_adapter (fp32)
+        "fwht_bwd": ("hbm", 8.0 * T * di, 8.0 * T * di),
+        "dequant": ("hbm", qbytes + 2.0 * do * di, qbytes + 2.0 * do * di),
+        "dequant_t": ("hbm", qbytes + 2.0 * do * di, qbytes + 2.0 * do * di),
+        # sparse products: 2 p T FLOP; bytes = activations in and out + the index arrays
+        "spmm_fwd": ("alu", 2.0 * p * T, 2.0 * T * di + 4.0 * T * do + 8.0 * p),
+        "gather_bwd": ("alu", 2.0 * p * T, 2.0 * T * do + 4.0 * T * di + 12.0 * p),
+        "sddmm_dc": ("alu", 2.0 * p * T, 2.0 * T * (di + do) + 8.0 * p),
+        "gemm_fwd": ("tensor", 2.0 * T * di * do, 2.0 * T * di + 2.0 * do * di + 2.0 * T * do),
+        "gemm_bwd": ("tensor", 2.0 * T * di * do, 2.0 * T * do + 2.0 * do * di + 2.0 * T * di),
+        "gemm_dc": ("tensor", 2.0 * T * di * do, 2.0 * T * (di + do) + 4.0 * do * di),
+        # W_eff = W_Q + alpha F H: codes + CSR in, bf16 out
+        "weff": ("hbm", qbytes + 8.0 * p + 2.0 * do * di, qbytes + 8.0 * p + 2.0 * do * di),
+        "transpose_w": ("hbm", 4.0 * do * di, 4.0 * do * di),
+        "transpose_act": ("hbm", 4.0 * T * (di + do), 4.0 * T * (di + do)),
+        "gather_dc": ("hbm", 12.0 * p, 12.0 * p),
     }
-    return table.get(stage)
-
-
-def stage_bytes(stage, spec, T, bits):
-    """Algorithmic HBM bytes per launch (every stage), for the GB/s column."""
-    di, do, p = spec.d_in, spec.d_out, spec.p
-    qbytes = do * di * bits // 8 + (do * di // spec.group) * 5
-    return {
-        "fwht_fwd": 4.0 * T * di,
-        "fwht_bwd": 8.0 * T * di,
-        "dequant": qbytes + 2.0 * do * di,
-        "dequant_t": qbytes + 2.0 * do * di,
-        "spmm_fwd": 2.0 * T * di + 4.0 * T * do + 8.0 * p + 4.0 * do,
-        "gather_bwd": 2.0 * T * do + 4.0 * T * di + 12.0 * p + 4.0 * di,
-        "sddmm_dc": 2.0 * T * (di + do) + 8.0 * p,
-        "gemm_fwd": 2.0 * T * di + 2.0 * do * di + 4.0 * T * do + 2.0 * T * do,
-        "gemm_bwd": 2.0 * T * do + 2.0 * do * di + 4.0 * T * di + 2.0 * T * di,
-    }.get(stage, 0.0)
+    return w.get(stage)
 
 
 def peak_for(kind, peaks):
@@ -253,6 +246,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--sparse-steps", type=int, default=40)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -301,85 +295,110 @@ def main():
         torch.cuda.synchronize()
         init_ms.append(ev[0].elapsed_time(ev[1]))
     a = W.Adapter(spec.d_in, spec.d_out, spec.had_block, spec.p, e["row_ptr"], e["col_idx"], e["coef"])
-    W.plan_build(a)
+    W.plan_build(a)  # the views the sparse backward needs
 
     alpha = 1.0
     Z = torch.empty_like(X)
     Y = torch.empty((T, spec.d_out), dtype=torch.bfloat16, device=dev)
     dX = torch.empty_like(X)
     dc = torch.empty(spec.p, dtype=torch.float32, device=dev)
-    ws_f = torch.empty(W.workspace_size(0, spec.d_out, spec.d_in, spec.p, T, True), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(W.workspace_size(1, spec.d_out, spec.d_in, spec.p, T, True), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    adapters = {
+        algo: W.Adapter(spec.d_in, spec.d_out, spec.had_block, spec.p, a.row_ptr, a.col_idx, a.coef, a.col_ptr,
+                        a.row_idx, a.perm, a.tile_ptr, a.tile_pos, a.tile_rk, algo=algo)
+        for algo in ("dense", "sparse")
+    }
+    ws = {}
+    for algo, ops in (("dense", (4, 5)), ("sparse", (0, 1))):
+        ws[algo] = [torch.empty(max(1, W.workspace_size(op, spec.d_out, spec.d_in, spec.p, T, True)),
+                                dtype=torch.uint8, device=dev) for op in ops]
 
-    def step():
-        W.adapter_fwd(a, X, alpha, wq, Z_out=Z, Y=Y, ws=ws_f)
-        W.adapter_bwd(a, dY, Z, alpha, wq, dc=dc, dX=dX, ws=ws_b)
+    def make_step(algo):
+        ad, (wf, wb) = adapters[algo], ws[algo]
+
+        def step():
+            W.adapter_fwd(ad, X, alpha, wq, Z_out=Z, Y=Y, ws=wf)
+            W.adapter_bwd(ad, dY, Z, alpha, wq, dc=dc, dX=dX, ws=wb)
+            if world > 1:
+                dist.all_reduce(dc)
+
+        return step
+
+    def timed(step, K, sample_clocks):
+        """K steps, each bracketed by events on the current stream after an L2 flush; (ms, stage report, clocks)."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        W.stage_report()
+        W.stage_timing(True)
+        clocks = ClockSampler() if (rank == 0 and sample_clocks) else None
         if world > 1:
-            dist.all_reduce(dc)
+            dist.barrier()
+        torch.cuda.synchronize()
+        if clocks:
+            clocks.start()
+            time.sleep(0.3)
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        clk = clocks.stop() if clocks else None
+        W.stage_timing(False)
+        rep = W.stage_report()
+        t_ms = sum(s_.elapsed_time(e_) for s_, e_ in zip(starts, ends))
+        if world > 1:
+            tt = torch.tensor([t_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t_ms = float(tt.item())
+        return t_ms, rep, clk
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if not (torch.isfinite(Y.float()).all() and torch.isfinite(dc).all() and torch.isfinite(dX.float()).all()):
-        raise RuntimeError("non-finite output")
+    def kernel_table(rep, K):
+        kernels = {}
+        for name, (calls, launches, ms) in rep.items():
+            if calls == 0:
+                continue
+            per = ms / calls
+            k = {"calls": calls, "launches": launches, "ms_per_call": per}
+            wk = stage_work(name, spec, T, spec.bits)
+            if wk:
+                kind, amount, nbytes = wk
+                peak, unit, _ = peak_for(kind, peaks)
+                ach = amount / (per / 1e3) / (1e9 if unit == "GB/s" else 1e12)
+                k.update(bound=kind, achieved=ach, peak=peak, unit=unit, frac=ach / peak,
+                         alg_GBps=nbytes / (per / 1e3) / 1e9)
+            kernels[name] = k
+        tot = sum(v["ms_per_call"] * v["calls"] for v in kernels.values())
+        for v in kernels.values():
+            v["share"] = v["ms_per_call"] * v["calls"] / tot
+        return kernels
 
-    # ---- timed region
-    K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    W.stage_report()
-    W.stage_timing(True)
-    clocks = ClockSampler() if rank == 0 else None
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    for i in range(K):
-        flush.fill_(i & 0xFF)
-        starts[i].record()
-        step()
-        ends[i].record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop() if clocks else None
-    W.stage_timing(False)
-    rep = W.stage_report()
-    t_ms = sum(s.elapsed_time(e_) for s, e_ in zip(starts, ends))
-    if world > 1:
-        tt = torch.tensor([t_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_ms = float(tt.item())
-    value = world * T * K / (t_ms / 1e3)
+    def roofline_of(kernels):
+        dom = max((n for n in kernels if "bound" in kernels[n]), key=lambda n: kernels[n]["share"])
+        kd = kernels[dom]
+        _, _, note = peak_for(kd["bound"], peaks)
+        return {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
+                "unit": kd["unit"], "frac": kd["frac"], "traffic": ncu_traffic(dom), "peak_source": note}
 
-    # ---- per-stage roofline (this rank's stage events, same timed region)
-    kernels = {}
-    for name, (calls, launches, ms) in rep.items():
-        if calls == 0:
-            continue
-        w = stage_work(name, spec, T, spec.bits)
-        per = ms / calls
-        k = {"launches": launches, "ms_per_launch": per, "share": None,
-             "alg_bytes": stage_bytes(name, spec, T, spec.bits)}
-        k["alg_GBps"] = k["alg_bytes"] / (per / 1e3) / 1e9
-        if w:
-            kind, amount = w
-            peak, unit, _ = peak_for(kind, peaks)
-            ach = amount / (per / 1e3) / (1e9 if unit == "GB/s" else 1e12)
-            k.update(bound=kind, achieved=ach, peak=peak, unit=unit, frac=ach / peak)
-        kernels[name] = k
-    total_stage_ms = sum(v["ms_per_launch"] * rep[n][0] for n, v in kernels.items())
-    for n, v in kernels.items():
-        v["share"] = v["ms_per_launch"] * rep[n][0] / total_stage_ms
-    dom = max((n for n in kernels if "bound" in kernels[n]), key=lambda n: kernels[n]["share"])
-    kd = kernels[dom]
-    _, _, peak_note = peak_for(kd["bound"], peaks)
-    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
-                "unit": kd["unit"], "frac": kd["frac"], "traffic": ncu_traffic(dom), "peak_source": peak_note}
-    launches = sum(v[1] for v in rep.values())
+    results = {}
+    for algo in ("dense", "sparse"):
+        step = make_step(algo)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        if not (torch.isfinite(Y.float()).all() and torch.isfinite(dc).all() and torch.isfinite(dX.float()).all()):
+            raise RuntimeError(f"non-finite output ({algo})")
+        K = args.steps if algo == "dense" else max(3, min(args.steps, args.sparse_steps))
+        t_ms, rep, clk = timed(step, K, algo == "dense")
+        kernels = kernel_table(rep, K)
+        results[algo] = dict(K=K, t_ms=t_ms, value=world * T * K / (t_ms / 1e3), kernels=kernels,
+                             roofline=roofline_of(kernels), launches=sum(v[1] for v in rep.values()), clocks=clk)
+    head = results["dense"]
+    K, t_ms, value, kernels, clk = head["K"], head["t_ms"], head["value"], head["kernels"], head["clocks"]
+    roofline, launches = head["roofline"], head["launches"]
+    step = make_step("dense")
 
     # ---- end to end through host buffers
     e2e = None
@@ -429,21 +448,27 @@ def main():
 
     init_bytes = 2 * 4.0 * spec.d_in * spec.d_out + 8.0 * spec.p
     init_med = statistics.median(init_ms)
+    sp = results["sparse"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": t_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; stands in for LLaMA-7B q_proj weights and activations)",
         "config": config_block(spec, world),
+        "algorithm": "dense: adapter folded into the tcgen05 GEMMs (W_eff = W_Q + alpha F H), dc from G = dY^T Z",
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
         "kernels": kernels,
+        "paths": {
+            "sparse": {"value": sp["value"], "unit": UNIT, "steps": sp["K"], "ms_per_step": sp["t_ms"] / sp["K"],
+                       "roofline": sp["roofline"], "gpu_launches": sp["launches"], "kernels": sp["kernels"],
+                       "what": "segment SpMM over CSR, tiled SDDMM, CSC gather on the FMA units; base GEMMs on tcgen05"},
+        },
         "init": {"ms": init_med, "alg_GBps": init_bytes / (init_med / 1e3) / 1e9,
                  "frac_hbm": init_bytes / (init_med / 1e3) / 1e9 / peaks["hbm_gbs"],
                  "what": "AdaAlloc on dW_Q (4096 x 4096 fp32): norms, budgets, fp64 transform, top-k; one-off per layer"},
-        "hbm_GBps_step": sum(stage_bytes(n, spec, T, spec.bits) * rep[n][0] for n in kernels) / (t_ms / 1e3) / 1e9,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

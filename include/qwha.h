@@ -63,6 +63,18 @@ typedef enum { QWHA_F32 = 0, QWHA_BF16 = 1 } qwha_dtype;
  * papernotes.org 关键设计 2) or to the channels of largest error. */
 typedef enum { QWHA_REM_FEWEST_ALLOC = 0, QWHA_REM_LARGEST_ERROR = 1 } qwha_remainder;
 
+/* How qwha_adapter_fwd/bwd compute the adapter terms. Both give the same
+ * results up to rounding order.
+ *   QWHA_ALGO_SPARSE: the sparse kernels on the FMA units -- the product
+ *     Z F^T over the CSR rows, the coefficient gradient over the tile view,
+ *     the transposed gather over the CSC view -- with the adapter terms added
+ *     in fp32 in the base GEMM's epilogue. Any dtype.
+ *   QWHA_ALGO_DENSE: the adapter folded into the tensor-core GEMMs.
+ *     W_eff = W_Q + alpha F H is built in bf16 (one transform of F's rows),
+ *     Y = X W_eff^T and dX = dY W_eff are single GEMMs, and dc is gathered at
+ *     E from the dense G = dY^T Z (fp32). bf16 only. */
+typedef enum { QWHA_ALGO_SPARSE = 0, QWHA_ALGO_DENSE = 1 } qwha_algo;
+
 /* Edge of the square blocks of F into which the coefficient-gradient kernel
  * tiles the nonzeros (the tile view built by qwha_plan_build). */
 #define QWHA_TILE 512
@@ -80,9 +92,11 @@ typedef enum { QWHA_REM_FEWEST_ALLOC = 0, QWHA_REM_LARGEST_ERROR = 1 } qwha_rema
  *       tile_pos is the CSR position, tile_rk packs (r mod QWHA_TILE) << 16 |
  *       (k mod QWHA_TILE).
  * The views are written by qwha_plan_build and depend on E only; the forward
- * needs the CSR arrays only, the backward needs all three views. */
+ * needs the CSR arrays only; the sparse backward needs all three views, the
+ * dense backward the CSR arrays only. */
 typedef struct {
   int32_t d_in, d_out, had_block;
+  int32_t algo; /* qwha_algo; 0 (sparse) for a zero-initialised struct */
   int64_t p;
   const int32_t *row_ptr, *col_idx;
   const float *coef;
@@ -107,10 +121,12 @@ typedef struct {
 
 /* Operations for qwha_workspace_size. */
 typedef enum {
-  QWHA_OP_FWD = 0,
-  QWHA_OP_BWD = 1,
-  QWHA_OP_INIT = 2,
-  QWHA_OP_PLAN = 3
+  QWHA_OP_FWD = 0,       /* qwha_adapter_fwd, algo sparse */
+  QWHA_OP_BWD = 1,       /* qwha_adapter_bwd, algo sparse */
+  QWHA_OP_INIT = 2,      /* qwha_init_alloc */
+  QWHA_OP_PLAN = 3,      /* qwha_plan_build */
+  QWHA_OP_FWD_DENSE = 4, /* qwha_adapter_fwd, algo dense */
+  QWHA_OP_BWD_DENSE = 5  /* qwha_adapter_bwd, algo dense */
 } qwha_op;
 
 /* Z = X H row by row: x and z are [rows, n] of dtype dt (device), each row
@@ -125,9 +141,10 @@ qwha_status qwha_fwht(qwha_dtype dt, const void *x, void *z, int64_t rows, int32
 /* Forward of the adapted layer (gist.science 2.1; papernotes.org 整体框架):
  *   Z_out = X H                 [T, d_in], dtype dt (kept for the backward)
  *   Y     = X W_Q^T + alpha Z F^T  [T, d_out], dtype dt
- * wq == NULL computes the adapter alone (Y = alpha Z F^T). With wq, dt must be
- * QWHA_BF16. X, Z_out, Y are device buffers; a->row_ptr/col_idx/coef are
- * required, the other views are not read. T >= 0 (T = 0 does nothing). */
+ * wq == NULL computes the adapter alone (Y = alpha Z F^T). With wq, or with
+ * a->algo == QWHA_ALGO_DENSE, dt must be QWHA_BF16. X, Z_out, Y are device
+ * buffers; a->row_ptr/col_idx/coef are required, the other views are not
+ * read. T >= 0 (T = 0 does nothing). */
 qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt,
                              const void *X, int64_t T, float alpha, void *Z_out, void *Y,
                              void *ws, size_t ws_bytes, void *stream);
@@ -136,8 +153,9 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
  *   dc[j] = alpha * sum_t dY[t, r_j] Z[t, k_j]   fp32 [p], CSR order
  *   dX    = dY W_Q + alpha (dY F) H              [T, d_in], dtype dt
  * Z is the Z_out of the matching forward. dc is overwritten (not accumulated).
- * Needs all views of `a` (qwha_plan_build). dX may be NULL to skip it. The
- * dc reduction runs in a fixed order: results are bitwise reproducible. */
+ * The sparse algorithm needs all views of `a` (qwha_plan_build). dX may be
+ * NULL to skip it. Every reduction runs in a fixed order: results are bitwise
+ * reproducible. */
 qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt,
                              const void *dY, const void *Z, int64_t T, float alpha, float *dc,
                              void *dX, void *ws, size_t ws_bytes, void *stream);

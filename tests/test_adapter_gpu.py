@@ -25,12 +25,12 @@ def _W():
     return W
 
 
-def device_adapter(d_in, d_out, n, rp, ci, cf, plan=True):
+def device_adapter(d_in, d_out, n, rp, ci, cf, plan=True, algo="sparse"):
     import torch
 
     W = _W()
     a = W.Adapter(d_in, d_out, n, int(ci.size), to_dev(rp), to_dev(ci) if ci.size else torch.zeros(1, dtype=torch.int32, device="cuda"),
-                  to_dev(cf) if cf.size else torch.zeros(1, device="cuda"))
+                  to_dev(cf) if cf.size else torch.zeros(1, device="cuda"), algo=algo)
     if plan:
         W.plan_build(a)
     return a
@@ -208,13 +208,16 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("d_in,d_out,n,T,p,dtype,pattern", CASES)
-def test_adapter_forward_backward(d_in, d_out, n, T, p, dtype, pattern):
+ALGO_CASES = [c + ("sparse",) for c in CASES] + [c + ("dense",) for c in CASES if c[5] == "bf16"]
+
+
+@pytest.mark.parametrize("d_in,d_out,n,T,p,dtype,pattern,algo", ALGO_CASES)
+def test_adapter_forward_backward(d_in, d_out, n, T, p, dtype, pattern, algo):
     import torch
 
     W = _W()
     L = synth_layer(33, d_in, d_out, n, T, p, dtype, pattern=pattern)
-    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"])
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"], algo=algo)
     alpha = 0.8
     Xd, dYd = dev_act(L["X"], dtype), dev_act(L["dY"], dtype)
     Z, Y = W.adapter_fwd(a, Xd, alpha)
@@ -236,22 +239,23 @@ def test_adapter_forward_backward(d_in, d_out, n, T, p, dtype, pattern):
     assert torch.equal(dc, dc2)
 
 
-@pytest.mark.parametrize(
-    "d_in,d_out,n,T,bits,group",
-    [
-        (512, 256, 512, 200, 4, 64),  # ragged token tile (200 = 128 + 72)
-        (1024, 768, 1024, 300, 3, 128),  # int3 bit stream
-        (640, 1280, 128, 129, 2, 64),  # int2, ragged token tile, K of 10 ring blocks
-        (256, 264, 256, 7, 4, 64),  # N = 264: partial 32-column epilogue chunk
-    ],
-)
-def test_base_gemm_forward_backward(d_in, d_out, n, T, bits, group):
+GEMM_CASES = [
+    (512, 256, 512, 200, 4, 64),  # ragged token tile (200 = 128 + 72)
+    (1024, 768, 1024, 300, 3, 128),  # int3 bit stream
+    (640, 1280, 128, 129, 2, 64),  # int2, ragged token tile, K of 10 ring blocks
+    (256, 264, 256, 7, 4, 64),  # N = 264: partial 32-column epilogue chunk
+]
+
+
+@pytest.mark.parametrize("algo", ["sparse", "dense"])
+@pytest.mark.parametrize("d_in,d_out,n,T,bits,group", GEMM_CASES)
+def test_base_gemm_forward_backward(d_in, d_out, n, T, bits, group, algo):
     import torch
 
     W = _W()
     p = d_out * 8
     L = synth_layer(35, d_in, d_out, n, T, p, "bf16", bits=bits, group=group)
-    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"])
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"], algo=algo)
     wq = dev_qweight(L)
     alpha = 1.0
     Xd, dYd = dev_act(L["X"], "bf16"), dev_act(L["dY"], "bf16")
@@ -261,10 +265,13 @@ def test_base_gemm_forward_backward(d_in, d_out, n, T, bits, group):
     Wq = oracle.dequant(L["qweight"], L["scales"], L["zeros"], bits, group, d_out, d_in)
     _, Yr = oracle.adapter_fwd(L["rp"], L["ci"], L["cf"], L["X"], d_out, n, alpha, Wq, want_z=False)
     dXr = oracle.adapter_bwd_dx(L["rp"], L["ci"], L["cf"], L["dY"], d_in, n, alpha, Wq)
-    errs = dict(Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr))
+    sel = np.sort(rng_for(37, "dcsel", d_out).choice(L["ci"].size, min(1500, L["ci"].size), replace=False))
+    dcr = oracle.adapter_bwd_dc(L["X"], L["dY"], oracle.csr_rows(L["rp"])[sel], L["ci"][sel], n, alpha)
+    errs = dict(Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr), dc=rel_fro(dc.cpu().numpy()[sel], dcr))
     assert all(v <= TOL_BF16 for v in errs.values()), errs
     # the base term alone (empty adapter) against the oracle's X W_Q^T
-    e = device_adapter(d_in, d_out, n, np.zeros(d_out + 1, np.int32), np.zeros(0, np.int32), np.zeros(0, np.float32))
+    e = device_adapter(d_in, d_out, n, np.zeros(d_out + 1, np.int32), np.zeros(0, np.int32), np.zeros(0, np.float32),
+                       algo=algo)
     _, Yb = W.adapter_fwd(e, Xd, alpha, wq=wq)
     torch.cuda.synchronize()
     assert rel_fro(host(Yb), L["X"].astype(np.float64) @ Wq.T) <= TOL_BF16
@@ -282,4 +289,13 @@ def test_workspace_and_dtype_errors():
     assert ei.value.status == 4
     with pytest.raises(W.QwhaError) as ei:
         W.adapter_fwd(a, to_dev(L["X"]), 1.0, wq=dev_qweight(L))  # base GEMM needs bf16
+    assert ei.value.status == 3
+
+
+def test_dense_rejects_fp32():
+    W = _W()
+    L = synth_layer(38, 256, 256, 256, 16, 512, "f32", pattern="random")
+    a = device_adapter(256, 256, 256, L["rp"], L["ci"], L["cf"], algo="dense")
+    with pytest.raises(W.QwhaError) as ei:
+        W.adapter_fwd(a, to_dev(L["X"]), 1.0)
     assert ei.value.status == 3

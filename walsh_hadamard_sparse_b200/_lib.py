@@ -21,6 +21,7 @@ class QwhaAdapter(ctypes.Structure):
         ("d_in", i32),
         ("d_out", i32),
         ("had_block", i32),
+        ("algo", i32),
         ("p", i64),
         ("row_ptr", P),
         ("col_idx", P),

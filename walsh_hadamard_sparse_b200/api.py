@@ -15,7 +15,8 @@ import torch
 from ._lib import QwhaAdapter, QwhaQweight, check, lib
 
 F32, BF16 = 0, 1
-OP_FWD, OP_BWD, OP_INIT, OP_PLAN = 0, 1, 2, 3
+OP_FWD, OP_BWD, OP_INIT, OP_PLAN, OP_FWD_DENSE, OP_BWD_DENSE = 0, 1, 2, 3, 4, 5
+ALGO = {"sparse": 0, "dense": 1}
 REMAINDER = {"fewest": 0, "largest": 1}
 
 
@@ -62,12 +63,14 @@ class Adapter:
     tile_ptr: torch.Tensor | None = None
     tile_pos: torch.Tensor | None = None
     tile_rk: torch.Tensor | None = None
+    algo: str = "sparse"
 
     def c_struct(self) -> QwhaAdapter:
         s = QwhaAdapter()
         s.d_in, s.d_out, s.had_block, s.p = self.d_in, self.d_out, self.had_block, self.p
+        s.algo = ALGO[self.algo]
         for f in fields(self):
-            if f.name in ("d_in", "d_out", "had_block", "p"):
+            if f.name in ("d_in", "d_out", "had_block", "p", "algo"):
                 continue
             v = getattr(self, f.name)
             setattr(s, f.name, None if v is None else v.data_ptr())
@@ -115,7 +118,7 @@ def adapter_fwd(a: Adapter, X: torch.Tensor, alpha: float = 1.0, wq: QWeight | N
     T = X.shape[0]
     Z_out = torch.empty_like(X) if Z_out is None else Z_out
     Y = torch.empty((T, a.d_out), dtype=X.dtype, device=X.device) if Y is None else Y
-    need = workspace_size(OP_FWD, a.d_out, a.d_in, a.p, T, wq is not None)
+    need = workspace_size(OP_FWD_DENSE if a.algo == "dense" else OP_FWD, a.d_out, a.d_in, a.p, T, wq is not None)
     ws = _ws(need, X.device) if ws is None else ws
     cs = a.c_struct()
     cw = wq.c_struct() if wq is not None else None
@@ -133,7 +136,7 @@ def adapter_bwd(a: Adapter, dY: torch.Tensor, Z: torch.Tensor, alpha: float = 1.
     dc = torch.empty(a.p, dtype=torch.float32, device=dY.device) if dc is None else dc
     if want_dx and dX is None:
         dX = torch.empty((T, a.d_in), dtype=dY.dtype, device=dY.device)
-    need = workspace_size(OP_BWD, a.d_out, a.d_in, a.p, T, wq is not None)
+    need = workspace_size(OP_BWD_DENSE if a.algo == "dense" else OP_BWD, a.d_out, a.d_in, a.p, T, wq is not None)
     ws = _ws(need, dY.device) if ws is None else ws
     cs = a.c_struct()
     cw = wq.c_struct() if wq is not None else None

@@ -86,10 +86,17 @@ enum Stage {
   ST_INIT,
   ST_PLAN,
   ST_FWHT,
+  ST_WEFF,
+  ST_TRANSPOSE_W,
+  ST_TRANSPOSE_ACT,
+  ST_GEMM_DC,
+  ST_GATHER_DC,
   ST_COUNT
 };
-const char *kStageNames[ST_COUNT] = {"fwht_fwd",  "spmm_fwd",  "dequant",  "gemm_fwd",   "sddmm_dc",   "gather_bwd",
-                                     "fwht_bwd",  "dequant_t", "gemm_bwd", "init_alloc", "plan_build", "fwht"};
+const char *kStageNames[ST_COUNT] = {"fwht_fwd",   "spmm_fwd",   "dequant",  "gemm_fwd",  "sddmm_dc",
+                                     "gather_bwd", "fwht_bwd",   "dequant_t", "gemm_bwd", "init_alloc",
+                                     "plan_build", "fwht",       "weff",      "transpose_w", "transpose_act",
+                                     "gemm_dc",    "gather_dc"};
 
 struct StageRec {
   int stage, kernels;
@@ -242,6 +249,10 @@ qwha_status check_adapter_shape(const qwha_adapter *a) {
   if (st != QWHA_OK) return st;
   if (a->p < 0 || a->p > (int64_t)a->d_in * a->d_out || a->p > 2147483647LL)
     return fail(QWHA_ERR_INVALID_ARG, "p = %lld out of range", (long long)a->p);
+  if (a->algo != QWHA_ALGO_SPARSE && a->algo != QWHA_ALGO_DENSE)
+    return fail(QWHA_ERR_INVALID_ARG, "algo %d", (int)a->algo);
+  if (a->algo == QWHA_ALGO_DENSE && weff_smem(a->d_in) > 200 * 1024)
+    return fail(QWHA_ERR_UNSUPPORTED, "dense algorithm: d_in %d above 51200", a->d_in);
   QWHA_CHECK_PTR(a->row_ptr, "row_ptr");
   if (a->p > 0) {
     QWHA_CHECK_PTR(a->col_idx, "col_idx");
@@ -290,11 +301,69 @@ size_t fwd_ws(int32_t d_out, int32_t d_in, int64_t T, bool base) {
   return align_up((size_t)T * d_out * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
 }
 
+size_t fwd_dense_ws(int32_t d_out, int32_t d_in) { return align_up((size_t)d_out * d_in * 2, 256); }
+
+int64_t pad8(int64_t v) { return (v + 7) / 8 * 8; }
+
+size_t bwd_dense_ws(int32_t d_out, int32_t d_in, int64_t T) {
+  const int64_t Tp = pad8(T);
+  return 2 * align_up((size_t)d_out * d_in * 2, 256)        // W_eff and its transpose
+         + align_up((size_t)d_out * Tp * 2, 256)            // dY^T
+         + align_up((size_t)d_in * Tp * 2, 256)             // Z^T
+         + align_up((size_t)d_out * d_in * 4, 256);         // G = dY^T Z
+}
+
 size_t bwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
   size_t n = align_up((size_t)kSddmmMaxChunks * (size_t)(p > 0 ? p : 1) * 4, 256);
   n += align_up((size_t)T * d_in * 4, 256);  // dZ
+  n += align_up((size_t)(p > 0 ? p : 1) * 4, 256);  // coefficients in CSC order
   if (base) n += align_up((size_t)T * d_in * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
   return n;
+}
+
+// Dense backward: W_eff and W_eff^T, dX = dY W_eff, G = dY^T Z, dc = alpha G at E.
+qwha_status dense_bwd(const qwha_adapter *a, const qwha_qweight *wq, const void *dY, const void *Z, int64_t T,
+                      float alpha, float *dc, void *dX, void *ws, cudaStream_t s) {
+  const int64_t Tp = pad8(T);
+  Carver cv(ws);
+  void *weff = cv.take((size_t)a->d_out * a->d_in * 2);
+  void *weff_t = cv.take((size_t)a->d_out * a->d_in * 2);
+  void *dyt = cv.take((size_t)a->d_out * Tp * 2);
+  void *zt = cv.take((size_t)a->d_in * Tp * 2);
+  float *G = static_cast<float *>(cv.take((size_t)a->d_out * a->d_in * 4));
+  cudaError_t e = cudaSuccess;
+  if (dX && T > 0) {
+    {
+      StageScope sc(ST_WEFF, 1, s);
+      e = launch_weff(a, wq, 1.0f * alpha, weff, s);
+    }
+    if (e != cudaSuccess) return cuda_status(e, "W_eff");
+    {
+      StageScope sc(ST_TRANSPOSE_W, 1, s);
+      e = launch_transpose_bf16(weff, a->d_out, a->d_in, weff_t, a->d_out, s);
+    }
+    if (e != cudaSuccess) return cuda_status(e, "transpose W_eff");
+    {
+      StageScope sc(ST_GEMM_BWD, 1, s);
+      e = launch_gemm_nt(dY, weff_t, nullptr, dX, false, T, a->d_in, a->d_out, s);
+    }
+    if (e != cudaSuccess) return cuda_status(e, "GEMM dX");
+  }
+  if (a->p == 0) return QWHA_OK;
+  if (T == 0) return cuda_status(cudaMemsetAsync(dc, 0, (size_t)a->p * 4, s), "dc = 0");
+  {
+    StageScope sc(ST_TRANSPOSE_ACT, 2, s);
+    e = launch_transpose_bf16(dY, T, a->d_out, dyt, Tp, s);
+    if (e == cudaSuccess) e = launch_transpose_bf16(Z, T, a->d_in, zt, Tp, s);
+  }
+  if (e != cudaSuccess) return cuda_status(e, "transpose dY, Z");
+  {
+    StageScope sc(ST_GEMM_DC, 1, s);
+    e = launch_gemm_nt(dyt, zt, nullptr, G, true, a->d_out, a->d_in, Tp, s);
+  }
+  if (e != cudaSuccess) return cuda_status(e, "GEMM dY^T Z");
+  StageScope sc(ST_GATHER_DC, 1, s);
+  return cuda_status(launch_gather_dc(G, a->row_ptr, a->col_idx, a->d_out, a->d_in, a->p, alpha, dc, s), "gather dc");
 }
 
 }  // namespace
@@ -313,6 +382,8 @@ size_t qwha_workspace_size(qwha_op op, int32_t d_out, int32_t d_in, int64_t p, i
     case QWHA_OP_BWD: return bwd_ws(d_out, d_in, p, T, with_base != 0);
     case QWHA_OP_INIT: return init_workspace(d_out, d_in);
     case QWHA_OP_PLAN: return plan_workspace(d_out, d_in);
+    case QWHA_OP_FWD_DENSE: return fwd_dense_ws(d_out, d_in);
+    case QWHA_OP_BWD_DENSE: return bwd_dense_ws(d_out, d_in, T);
   }
   return 0;
 }
@@ -329,7 +400,10 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   QWHA_CHECK_PTR(X, "X");
   QWHA_CHECK_PTR(Z_out, "Z_out");
   QWHA_CHECK_PTR(Y, "Y");
-  if ((st = check_ws(ws, ws_bytes, fwd_ws(a->d_out, a->d_in, T, wq != nullptr))) != QWHA_OK) return st;
+  const bool dense = a->algo == QWHA_ALGO_DENSE;
+  if (dense && dt != QWHA_BF16) return fail(QWHA_ERR_UNSUPPORTED, "the dense algorithm needs dtype bf16");
+  const size_t need = dense ? fwd_dense_ws(a->d_out, a->d_in) : fwd_ws(a->d_out, a->d_in, T, wq != nullptr);
+  if ((st = check_ws(ws, ws_bytes, need)) != QWHA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int logn = ilog2(a->had_block);
   const float inv = (float)(1.0 / sqrt((double)a->had_block));
@@ -339,10 +413,19 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
     e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
   }
   if (e != cudaSuccess) return cuda_status(e, "fwht");
+  if (dense) {
+    void *weff = ws;
+    {
+      StageScope sc(ST_WEFF, 1, s);
+      e = launch_weff(a, wq, alpha, weff, s);
+    }
+    if (e != cudaSuccess) return cuda_status(e, "W_eff");
+    StageScope sc(ST_GEMM_FWD, 1, s);
+    return cuda_status(launch_gemm_nt(X, weff, nullptr, Y, false, T, a->d_out, a->d_in, s), "GEMM with W_eff");
+  }
   if (!wq) {
     StageScope sc(ST_SPMM_FWD, 1, s);
-    e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
-                        alpha, Y, s);
+    e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, a->p, a->d_out, alpha, Y, s);
     return cuda_status(e, "spmm");
   }
   Carver cv(ws);
@@ -350,8 +433,8 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   void *wdeq = cv.take(wdeq_bytes(a->d_out, a->d_in));
   {
     StageScope sc(ST_SPMM_FWD, 1, s);
-    e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
-                        alpha, y_ad, s);
+    e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, a->p, a->d_out, alpha,
+                        y_ad, s);
   }
   if (e != cudaSuccess) return cuda_status(e, "spmm");
   {
@@ -368,8 +451,10 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
                              size_t ws_bytes, void *stream) {
   qwha_status st = check_adapter_shape(a);
   if (st != QWHA_OK) return st;
-  if ((st = check_views(a)) != QWHA_OK) return st;
+  const bool dense = a->algo == QWHA_ALGO_DENSE;
+  if (!dense && (st = check_views(a)) != QWHA_OK) return st;
   if (!valid_dtype(dt)) return fail(QWHA_ERR_INVALID_ARG, "dtype %d", (int)dt);
+  if (dense && dt != QWHA_BF16) return fail(QWHA_ERR_UNSUPPORTED, "the dense algorithm needs dtype bf16");
   if ((st = check_qweight(wq, a->d_out, a->d_in, dt)) != QWHA_OK) return st;
   if (T < 0) return fail(QWHA_ERR_INVALID_ARG, "T %lld < 0", (long long)T);
   if (a->p > 0) QWHA_CHECK_PTR(dc, "dc");
@@ -378,11 +463,14 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
     QWHA_CHECK_PTR(Z, "Z");
     if (dX) QWHA_CHECK_PTR(dX, "dX");
   }
-  if ((st = check_ws(ws, ws_bytes, bwd_ws(a->d_out, a->d_in, a->p, T, wq != nullptr))) != QWHA_OK) return st;
+  const size_t need = dense ? bwd_dense_ws(a->d_out, a->d_in, T) : bwd_ws(a->d_out, a->d_in, a->p, T, wq != nullptr);
+  if ((st = check_ws(ws, ws_bytes, need)) != QWHA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
+  if (dense) return dense_bwd(a, wq, dY, Z, T, alpha, dc, dX, ws, s);
   Carver cv(ws);
   float *partial = static_cast<float *>(cv.take((size_t)kSddmmMaxChunks * (size_t)(a->p > 0 ? a->p : 1) * 4));
   float *dz = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
+  float *coef_csc = static_cast<float *>(cv.take((size_t)(a->p > 0 ? a->p : 1) * 4));
   cudaError_t e;
   {
     StageScope sc(ST_SDDMM, 2, s);
@@ -392,9 +480,11 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   if (e != cudaSuccess) return cuda_status(e, "sddmm");
   if (!dX || T == 0) return QWHA_OK;
   {
-    StageScope sc(ST_GATHER_BWD, 1, s);
-    e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, a->coef, a->perm, a->p, a->d_in,
-                        alpha, dz, s);
+    StageScope sc(ST_GATHER_BWD, 2, s);
+    e = launch_permute(a->coef, a->perm, a->p, coef_csc, s);
+    if (e == cudaSuccess)
+      e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, coef_csc, a->p, a->d_in, alpha, dz,
+                          s);
   }
   if (e != cudaSuccess) return cuda_status(e, "gather");
   const int logn = ilog2(a->had_block);

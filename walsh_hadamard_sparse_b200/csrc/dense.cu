@@ -1,0 +1,171 @@
+// Dense tensor-core formulation of the adapter (the same results as the
+// sparse kernels, computed as dense contractions on tcgen05).
+//
+// Because H is fixed, the adapter's weight update dW = F H is a dense matrix
+// that costs one transform of F's rows to build ("QWHA", papernotes.org
+// 关键设计 1: the update is F times the inverse transform). Folding it into the
+// base weight,
+//     W_eff = W_Q + alpha * F H,
+// makes the forward Y = X W_eff^T and the input gradient dX = dY W_eff plain
+// GEMMs: the adapter costs nothing in either. The coefficient gradient is the
+// sampled product dc_j = alpha * (dY^T Z)[r_j, k_j]: one dense GEMM
+// G = dY^T Z (contraction over tokens) and a gather at E.
+//
+// Kernels here: weff_kernel (one CTA per row of W_eff: scatter the row of F
+// into shared memory, fp32 butterflies per Hadamard block, add the dequantized
+// base row, one bf16 rounding; used for Hadamard blocks outside 128..4096,
+// the main path is weff_rows_kernel in fwht.cu on the transform's register
+// layout), transpose_bf16_kernel (64 x 64 tiles, zero pad of the output's
+// leading dimension), gather_dc_kernel.
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qwha {
+namespace {
+
+constexpr int kWeffThreads = 512;
+
+__global__ void __launch_bounds__(kWeffThreads)
+    weff_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
+                const float *__restrict__ coef, int64_t p, int d_in, int logn, float scale, int bits, int group,
+                const uint8_t *__restrict__ qw, const float *__restrict__ scales, const uint8_t *__restrict__ zeros,
+                __nv_bfloat16 *__restrict__ out) {
+  extern __shared__ __align__(16) float row[];
+  const int64_t r = blockIdx.x;
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) row[k] = 0.f;
+  __syncthreads();
+  int64_t b = row_ptr[r], e = row_ptr[r + 1];
+  if (b < 0) b = 0;
+  if (e > p) e = p;
+  for (int64_t j = b + threadIdx.x; j < e; j += blockDim.x) {
+    const int k = col_idx[j];
+    if ((unsigned)k < (unsigned)d_in) row[k] = coef[j];
+  }
+  __syncthreads();
+  // butterflies on index bits [0, logn): per block of 2^logn, three stages per pass
+  for (int s = 0; s < logn; s += 3) {
+    const int nb = min(3, logn - s);
+    const int gsz = 1 << nb;
+    for (int g = threadIdx.x; g < (d_in >> nb); g += blockDim.x) {
+      const int lo = g & ((1 << s) - 1);
+      const int base = ((g >> s) << (s + nb)) | lo;
+      float v[8];
+      for (int i = 0; i < gsz; ++i) v[i] = row[base + (i << s)];
+      for (int bb = 0; bb < nb; ++bb)
+        for (int i = 0; i < gsz; ++i)
+          if (!(i & (1 << bb))) {
+            const float a = v[i], c = v[i + (1 << bb)];
+            v[i] = a + c;
+            v[i + (1 << bb)] = a - c;
+          }
+      for (int i = 0; i < gsz; ++i) row[base + (i << s)] = v[i];
+    }
+    __syncthreads();
+  }
+  // + dequantized base row, one rounding to bf16, 8 values per thread
+  const int64_t row_bytes = (int64_t)d_in * bits / 8;
+  const int ng = qw ? d_in / group : 0;
+  for (int k0 = threadIdx.x * 8; k0 < d_in; k0 += blockDim.x * 8) {
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = scale * row[k0 + i];
+    if (qw) {
+      const uint8_t *src = qw + r * row_bytes + (int64_t)k0 * bits / 8;
+      uint32_t w = 0;
+      for (int bb = 0; bb < bits; ++bb) w |= (uint32_t)src[bb] << (8 * bb);
+      const uint32_t mask = (1u << bits) - 1u;
+      const float sc = scales[r * ng + k0 / group], z = (float)zeros[r * ng + k0 / group];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] += sc * ((float)((w >> (bits * i)) & mask) - z);
+    }
+    *reinterpret_cast<uint4 *>(out + r * d_in + k0) = io<__nv_bfloat16>::pack(f);
+  }
+}
+
+// out[c][r] = in[r][c] for r < R, c < C; out rows have leading dimension ldo >= R,
+// columns R..ldo-1 are written as zeros. 64 x 64 tiles, 256 threads.
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ in, int64_t R,
+                                                             int64_t C, __nv_bfloat16 *__restrict__ out, int64_t ldo) {
+  __shared__ uint16_t tile[64][64 + 2];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const uint16_t *src = reinterpret_cast<const uint16_t *>(in);
+  for (int it = threadIdx.x; it < 64 * 8; it += 256) {
+    const int rr = it / 8, cc = (it % 8) * 8;
+    const int64_t r = r0 + rr, c = c0 + cc;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < R && c < C) v = *reinterpret_cast<const uint4 *>(src + r * C + c);
+    const uint16_t *h = reinterpret_cast<const uint16_t *>(&v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tile[rr][cc + i] = h[i];
+  }
+  __syncthreads();
+  uint16_t *dst = reinterpret_cast<uint16_t *>(out);
+  for (int it = threadIdx.x; it < 64 * 8; it += 256) {
+    const int cc = it / 8, rr = (it % 8) * 8;
+    const int64_t c = c0 + cc, r = r0 + rr;
+    if (c >= C || r >= ldo) continue;
+    uint16_t h[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = (r + i < R) ? tile[rr + i][cc] : 0;
+    *reinterpret_cast<uint4 *>(dst + c * ldo + r) = *reinterpret_cast<const uint4 *>(h);
+  }
+}
+
+// dc[j] = alpha * G[r_j, col_idx[j]]: one warp per row of F.
+__global__ void gather_dc_kernel(const float *__restrict__ G, const int32_t *__restrict__ row_ptr,
+                                 const int32_t *__restrict__ col_idx, int d_out, int d_in, int64_t p, float alpha,
+                                 float *__restrict__ dc) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; r < d_out;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    int64_t b = row_ptr[r], e = row_ptr[r + 1];
+    if (b < 0) b = 0;
+    if (e > p) e = p;
+    for (int64_t j = b + lane; j < e; j += 32) {
+      const int k = col_idx[j];
+      dc[j] = (unsigned)k < (unsigned)d_in ? alpha * G[r * d_in + k] : 0.f;
+    }
+  }
+}
+
+}  // namespace
+
+size_t weff_smem(int32_t d_in) { return (size_t)d_in * sizeof(float); }
+
+cudaError_t launch_weff(const qwha_adapter *a, const qwha_qweight *wq, float alpha, void *out, cudaStream_t s) {
+  const int logn = ilog2(a->had_block);
+  const float scale = (float)(alpha / sqrt((double)a->had_block));
+  if (weff_rows_supported(logn))
+    return launch_weff_rows(a->row_ptr, a->col_idx, a->coef, a->p, a->d_in, a->d_out, logn, scale,
+                            wq ? wq->bits : 0, wq ? wq->group : 1, wq ? wq->qweight : nullptr,
+                            wq ? wq->scales : nullptr, wq ? wq->zeros : nullptr, out, s);
+  const size_t smem = weff_smem(a->d_in);
+  cudaError_t e = cudaFuncSetAttribute(weff_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  weff_kernel<<<a->d_out, kWeffThreads, smem, s>>>(a->row_ptr, a->col_idx, a->coef, a->p, a->d_in, logn, scale,
+                                                   wq ? wq->bits : 0, wq ? wq->group : 1, wq ? wq->qweight : nullptr,
+                                                   wq ? wq->scales : nullptr, wq ? wq->zeros : nullptr,
+                                                   static_cast<__nv_bfloat16 *>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_bf16(const void *in, int64_t R, int64_t C, void *out, int64_t ldo, cudaStream_t s) {
+  if (R <= 0 || C <= 0) return cudaSuccess;
+  dim3 grid((unsigned)cdiv(C, 64), (unsigned)cdiv(ldo, 64));
+  transpose_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(in), R, C,
+                                             static_cast<__nv_bfloat16 *>(out), ldo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_dc(const float *G, const int32_t *row_ptr, const int32_t *col_idx, int32_t d_out,
+                             int32_t d_in, int64_t p, float alpha, float *dc, cudaStream_t s) {
+  if (p <= 0) return cudaSuccess;
+  const int64_t grid = std::min<int64_t>(cdiv((int64_t)d_out * 32, 256), (int64_t)sm_count() * 8);
+  gather_dc_kernel<<<(unsigned)grid, 256, 0, s>>>(G, row_ptr, col_idx, d_out, d_in, p, alpha, dc);
+  return cudaGetLastError();
+}
+
+}  // namespace qwha

@@ -204,6 +204,121 @@ __global__ void __launch_bounds__(512) fwht_large_kernel(const Tin *__restrict__
   }
 }
 
+// W_eff block rows: for block b of row r (n = 2^LOGN columns starting at
+// blk * n), scatter that row's coefficients into the swizzled buffer, run the
+// two butterfly phases, then in phase-A layout (8 consecutive columns per
+// vector) add the dequantized base weight in fp32 and store one bf16 rounding:
+//   out[r, k] = bf16( W_Q[r, k] + scale * (sum_j c_j H_unnorm[k_j, k]) ).
+template <int LOGN>
+__global__ void __launch_bounds__(kThreads)
+    weff_rows_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
+                     const float *__restrict__ coef, int64_t p, int d_in, int64_t n_rows, float scale, int bits,
+                     int group, const uint8_t *__restrict__ qw, const float *__restrict__ scales,
+                     const uint8_t *__restrict__ zeros, __nv_bfloat16 *__restrict__ out) {
+  using G = Geo<LOGN, 8>;
+  constexpr int RPC = kThreads / G::P;
+  extern __shared__ __align__(16) float smem[];
+  const int rl = threadIdx.x / G::P;
+  const int t = threadIdx.x % G::P;
+  float *buf = smem + rl * G::N;
+  const int nb = d_in >> LOGN;
+  const int64_t blocks = n_rows * nb;
+  const int64_t row_bytes = (int64_t)d_in * bits / 8;
+  const int ng = qw ? d_in / group : 0;
+
+  for (int64_t base = (int64_t)blockIdx.x * RPC; base < blocks; base += (int64_t)gridDim.x * RPC) {
+    const int64_t bi = base + rl;
+    const bool active = bi < blocks;
+    const int64_t r = active ? bi / nb : 0;
+    const int k0 = active ? (int)(bi % nb) << LOGN : 0;
+    __syncthreads();  // the previous iteration's readers are done with buf
+    for (int i = t; i < G::N; i += G::P) buf[i] = 0.f;
+    __syncthreads();
+    if (active) {
+      int64_t b = row_ptr[r], e = row_ptr[r + 1];
+      if (b < 0) b = 0;
+      if (e > p) e = p;
+      for (int64_t j = b + t; j < e; j += G::P) {
+        const int k = col_idx[j] - k0;
+        if ((unsigned)k < (unsigned)G::N) buf[G::phys(k)] = coef[j];
+      }
+    }
+    __syncthreads();
+    float v[G::R];
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+      const float *src = buf + G::phys(G::eA(t, h << G::LV));
+#pragma unroll
+      for (int u = 0; u < 8; u += 4) {
+        const float4 f = *reinterpret_cast<const float4 *>(src + u);
+        v[h * 8 + u] = f.x, v[h * 8 + u + 1] = f.y, v[h * 8 + u + 2] = f.z, v[h * 8 + u + 3] = f.w;
+      }
+    }
+    butterflies<G::R, 0, G::RB>(v);
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+      float *dst = buf + G::phys(G::eA(t, h << G::LV));
+#pragma unroll
+      for (int u = 0; u < 8; u += 4)
+        *reinterpret_cast<float4 *>(dst + u) = make_float4(v[h * 8 + u], v[h * 8 + u + 1], v[h * 8 + u + 2], v[h * 8 + u + 3]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
+    butterflies<G::R, 0, G::PB>(v);
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) buf[G::phys(G::eB(t, q))] = v[q] * scale;
+    __syncthreads();
+    if (active) {
+#pragma unroll
+      for (int h = 0; h < (1 << G::HB); ++h) {
+        const int e = G::eA(t, h << G::LV);
+        const float *src = buf + G::phys(e);
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; u += 4) {
+          const float4 a = *reinterpret_cast<const float4 *>(src + u);
+          f[u] = a.x, f[u + 1] = a.y, f[u + 2] = a.z, f[u + 3] = a.w;
+        }
+        const int k = k0 + e;
+        if (qw) {
+          const uint8_t *cp = qw + r * row_bytes + (int64_t)k * bits / 8;
+          uint32_t w = 0;
+          for (int bb = 0; bb < bits; ++bb) w |= (uint32_t)cp[bb] << (8 * bb);
+          const uint32_t mask = (1u << bits) - 1u;
+          const float sc = scales[r * ng + k / group], z = (float)zeros[r * ng + k / group];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] += sc * ((float)((w >> (bits * i)) & mask) - z);
+        }
+        st_stream(out + r * d_in + k, io<__nv_bfloat16>::pack(f));
+      }
+    }
+  }
+}
+
+template <int LOGN>
+cudaError_t run_weff(const int32_t *row_ptr, const int32_t *col_idx, const float *coef, int64_t p, int d_in,
+                     int64_t n_rows, float scale, int bits, int group, const uint8_t *qw, const float *scales,
+                     const uint8_t *zeros, __nv_bfloat16 *out, cudaStream_t s) {
+  using G = Geo<LOGN, 8>;
+  constexpr int RPC = kThreads / G::P;
+  const size_t smem = (size_t)RPC * G::N * sizeof(float);
+  auto k = weff_rows_kernel<LOGN>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  const int64_t need = cdiv(n_rows * (d_in >> LOGN), RPC);
+  const int64_t cap = (int64_t)sm_count() * occ;
+  k<<<(unsigned)(need < cap ? need : cap), kThreads, smem, s>>>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits,
+                                                               group, qw, scales, zeros, out);
+  return cudaGetLastError();
+}
+
 template <int LOGN, typename Tin, typename Tout>
 cudaError_t run_rows(const Tin *x, Tout *z, int64_t rows, float scale, cudaStream_t s) {
   constexpr int V = (sizeof(Tin) == 2 || sizeof(Tout) == 2) ? 8 : 4;
@@ -278,6 +393,27 @@ cudaError_t launch_fwht(qwha_dtype din, qwha_dtype dout, const void *x, void *z,
   if (din == QWHA_BF16 && dout == QWHA_BF16) return dispatch<bf, bf>(x, z, blocks, logn, scale, s);
   if (din == QWHA_F32 && dout == QWHA_BF16) return dispatch<float, bf>(x, z, blocks, logn, scale, s);
   return dispatch<bf, float>(x, z, blocks, logn, scale, s);
+}
+
+}  // namespace qwha
+
+namespace qwha {
+
+bool weff_rows_supported(int logn) { return logn >= 7 && logn <= 12; }
+
+cudaError_t launch_weff_rows(const int32_t *row_ptr, const int32_t *col_idx, const float *coef, int64_t p, int d_in,
+                             int64_t n_rows, int logn, float scale, int bits, int group, const uint8_t *qw,
+                             const float *scales, const uint8_t *zeros, void *out, cudaStream_t s) {
+  __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+  switch (logn) {
+    case 7: return run_weff<7>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group, qw, scales, zeros, o, s);
+    case 8: return run_weff<8>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group, qw, scales, zeros, o, s);
+    case 9: return run_weff<9>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group, qw, scales, zeros, o, s);
+    case 10: return run_weff<10>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group, qw, scales, zeros, o, s);
+    case 11: return run_weff<11>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group, qw, scales, zeros, o, s);
+    case 12: return run_weff<12>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group, qw, scales, zeros, o, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace qwha

@@ -1,5 +1,5 @@
-// Base GEMM of the adapted layer on the 5th-generation tensor cores:
-//   out[M, N] = bf16( A[M, K] . B[N, K]^T + addend[M, N] )
+// Dense contractions of the adapted layer on the 5th-generation tensor cores:
+//   out[M, N] = A[M, K] . B[N, K]^T (+ addend[M, N]), out bf16 or fp32
 // with A, B bf16 K-major (row-major with K contiguous) and addend fp32.
 //   forward:  Y  = X W_Q^T + Y_adapter   (A = X, B = W_Q, K = d_in)
 //   backward: dX = dY W_Q + dX_adapter   (A = dY, B = W_Q^T, K = d_out)
@@ -19,7 +19,7 @@
 //                        the main loop of tile i+1).
 //   warps 2..5         : epilogue. tcgen05.ld 32 lanes x 32 columns at a
 //                        time (warp w reads TMEM lanes 32*(w%4)..+31), add
-//                        the fp32 addend, round to bf16, store.
+//                        the fp32 addend (if any), store bf16 or fp32.
 // Every mbarrier wait is bounded by time: on expiry the thread records a code
 // in the library's device error word, the CTA stops issuing work, drains what
 // it issued, frees TMEM and exits.
@@ -137,9 +137,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// kF32Out: write fp32 D (no rounding); otherwise bf16. addend may be NULL.
+template <bool kF32Out>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const float *__restrict__ addend, __nv_bfloat16 *__restrict__ out, int M, int N, int K,
+                             const float *__restrict__ addend, void *__restrict__ out_v, int M, int N, int K,
                              unsigned int *err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t base = smem_u32(smem_raw);
@@ -277,23 +279,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
         const int col0 = n_blk * BN + c * 32;
         if (row < M && col0 < N) {
-          const float *ad = addend + (int64_t)row * N + col0;
-          __nv_bfloat16 *o = out + (int64_t)row * N + col0;
-          if (col0 + 32 <= N) {
+          const int64_t off = (int64_t)row * N + col0;
+          float f[32];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const float4 a0 = *reinterpret_cast<const float4 *>(ad + 8 * v);
-              const float4 a1 = *reinterpret_cast<const float4 *>(ad + 8 * v + 4);
-              float f[8] = {__uint_as_float(r[8 * v + 0]) + a0.x, __uint_as_float(r[8 * v + 1]) + a0.y,
-                            __uint_as_float(r[8 * v + 2]) + a0.z, __uint_as_float(r[8 * v + 3]) + a0.w,
-                            __uint_as_float(r[8 * v + 4]) + a1.x, __uint_as_float(r[8 * v + 5]) + a1.y,
-                            __uint_as_float(r[8 * v + 6]) + a1.z, __uint_as_float(r[8 * v + 7]) + a1.w};
-              *reinterpret_cast<uint4 *>(o + 8 * v) = io<__nv_bfloat16>::pack(f);
+          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
+          if (addend) {
+            const float *ad = addend + off;
+            if (col0 + 32 <= N) {
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(ad + 4 * v);
+                f[4 * v] += a4.x, f[4 * v + 1] += a4.y, f[4 * v + 2] += a4.z, f[4 * v + 3] += a4.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < N) f[j] += ad[j];
+            }
+          }
+          if (kF32Out) {
+            float *o = static_cast<float *>(out_v) + off;
+            if (col0 + 32 <= N) {
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                *reinterpret_cast<float4 *>(o + 4 * v) = make_float4(f[4 * v], f[4 * v + 1], f[4 * v + 2], f[4 * v + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < N) o[j] = f[j];
             }
           } else {
+            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out_v) + off;
+            if (col0 + 32 <= N) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < N) o[j] = __float2bfloat16_rn(__uint_as_float(r[j]) + ad[j]);
+              for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4 *>(o + 8 * v) = io<__nv_bfloat16>::pack(f + 8 * v);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < N) o[j] = __float2bfloat16_rn(f[j]);
+            }
           }
         }
       }
@@ -340,23 +364,29 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, uint3
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
-                        int64_t K, cudaStream_t s) {
+template <bool kF32Out>
+cudaError_t launch_gemm_t(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
+                          int64_t K, cudaStream_t s) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kGemmSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05_kernel<kF32Out>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int64_t tiles = cdiv(M, BM) * cdiv(N, BN);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  gemm_bf16_tcgen05_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, addend, static_cast<__nv_bfloat16 *>(out),
-                                                                (int)M, (int)N, (int)K, device_error_word());
+  gemm_bf16_tcgen05_kernel<kF32Out><<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, addend, out, (int)M, (int)N,
+                                                                          (int)K, device_error_word());
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
+                        int64_t K, cudaStream_t s) {
+  return launch_gemm_t<false>(A, B, addend, out, M, N, K, s);
 }
 
 }  // namespace
@@ -369,6 +399,12 @@ cudaError_t launch_gemm_fwd(const void *X, const void *wdeq, const float *y_ad, 
 cudaError_t launch_gemm_bwd(const void *dY, const void *wdeq_t, const float *dx_ad, void *dX, int64_t T,
                             int32_t d_out, int32_t d_in, cudaStream_t s) {
   return launch_gemm(dY, wdeq_t, dx_ad, dX, T, d_in, d_out, s);
+}
+
+cudaError_t launch_gemm_nt(const void *A, const void *B, const float *addend, void *out, bool f32_out, int64_t M,
+                           int64_t N, int64_t K, cudaStream_t s) {
+  return f32_out ? launch_gemm_t<true>(A, B, addend, out, M, N, K, s)
+                 : launch_gemm_t<false>(A, B, addend, out, M, N, K, s);
 }
 
 }  // namespace qwha

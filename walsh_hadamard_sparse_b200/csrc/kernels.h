@@ -9,6 +9,12 @@
 
 namespace qwha {
 
+// W_eff rows for Hadamard blocks of 2^logn, 7 <= logn <= 12 (fwht.cu).
+bool weff_rows_supported(int logn);
+cudaError_t launch_weff_rows(const int32_t *row_ptr, const int32_t *col_idx, const float *coef, int64_t p, int d_in,
+                             int64_t n_rows, int logn, float scale, int bits, int group, const uint8_t *qw,
+                             const float *scales, const uint8_t *zeros, void *out, cudaStream_t s);
+
 // Transform `blocks` consecutive blocks of 2^logn elements; out = H_unnorm(in) * scale.
 cudaError_t launch_fwht(qwha_dtype din, qwha_dtype dout, const void *x, void *z, int64_t blocks,
                         int logn, float scale, cudaStream_t s);
@@ -21,10 +27,13 @@ namespace qwha {
 // partial sums take kSddmmMaxChunks * p floats of workspace at most).
 constexpr int kSddmmMaxChunks = 16;
 
-// out[t, i] = alpha * sum_{j in [seg_ptr[i], seg_ptr[i+1])} val[val_perm ? val_perm[j] : j] * in[t, idx[j]]
+// out[t, i] = alpha * sum_{j in [seg_ptr[i], seg_ptr[i+1])} val[j] * in[t, idx[j]]
 cudaError_t launch_seg_spmm(qwha_dtype din, qwha_dtype dout, const void *in, int64_t T, int W_in,
-                            const int32_t *seg_ptr, const int32_t *idx, const float *val, const int32_t *val_perm,
-                            int64_t nnz, int n_seg, float alpha, void *out, cudaStream_t s);
+                            const int32_t *seg_ptr, const int32_t *idx, const float *val, int64_t nnz, int n_seg,
+                            float alpha, void *out, cudaStream_t s);
+
+// dst[q] = src[perm[q]]
+cudaError_t launch_permute(const float *src, const int32_t *perm, int64_t p, float *dst, cudaStream_t s);
 
 int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in);
 
@@ -62,10 +71,27 @@ cudaError_t launch_gemm_fwd(const void *X, const void *wdeq, const float *y_ad, 
                             int32_t d_in, cudaStream_t s);
 cudaError_t launch_gemm_bwd(const void *dY, const void *wdeq_t, const float *dx_ad, void *dX, int64_t T,
                             int32_t d_out, int32_t d_in, cudaStream_t s);
+// out[M, N] = A[M, K] B[N, K]^T (+ addend), A and B bf16 K-major, out fp32 or bf16.
+cudaError_t launch_gemm_nt(const void *A, const void *B, const float *addend, void *out, bool f32_out, int64_t M,
+                           int64_t N, int64_t K, cudaStream_t s);
 
 // Device error word and plan validation (misc.cu).
 cudaError_t read_and_clear_error_word(unsigned int *word, cudaStream_t s);
 const char *validate_message(unsigned int code);
 cudaError_t launch_validate(const qwha_adapter *a, cudaStream_t s, uint32_t *code, int64_t *where);
+
+}  // namespace qwha
+
+namespace qwha {
+
+// Dense formulation (dense.cu).
+size_t weff_smem(int32_t d_in);
+// out = bf16(dequant(W_Q) + alpha * (F H)) [d_out, d_in]; wq may be NULL (adapter alone).
+cudaError_t launch_weff(const qwha_adapter *a, const qwha_qweight *wq, float alpha, void *out, cudaStream_t s);
+// out[c][r] = in[r][c], out leading dimension ldo >= R (padding columns zeroed).
+cudaError_t launch_transpose_bf16(const void *in, int64_t R, int64_t C, void *out, int64_t ldo, cudaStream_t s);
+// dc[j] = alpha * G[r_j, col_idx[j]]
+cudaError_t launch_gather_dc(const float *G, const int32_t *row_ptr, const int32_t *col_idx, int32_t d_out,
+                             int32_t d_in, int64_t p, float alpha, float *dc, cudaStream_t s);
 
 }  // namespace qwha
