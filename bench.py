@@ -41,8 +41,9 @@ ALU_LANES_PER_SM = 128  # fp32 FMA lanes per SM (4 partitions x 32)
 
 KERNEL_SOURCES = {
     "fwht_fwd": ["fwht.cu"], "fwht_bwd": ["fwht.cu"], "spmm_fwd": ["sparse.cu"], "gather_bwd": ["sparse.cu"],
-    "sddmm_dc": ["sparse.cu"], "dequant": ["dequant.cu"], "dequant_t": ["dequant.cu"], "gemm_fwd": ["gemm.cu"],
-    "gemm_bwd": ["gemm.cu"], "init_alloc": ["init.cu"], "plan_build": ["plan.cu"],
+    "sddmm_dc": ["sparse.cu"], "dequant": ["dequant.cu"], "gemm_fwd": ["gemm.cu"], "gemm_bwd": ["gemm.cu"],
+    "gemm_dc": ["gemm.cu"], "weff": ["fwht.cu", "dense.cu"], "init_alloc": ["init.cu"],
+    "plan_build": ["plan.cu"],
 }
 
 
@@ -89,19 +90,15 @@ def stage_work(stage, spec, T, bits):
         # backward transform: read dZ (fp32), write dX_adapter (fp32)
         "fwht_bwd": ("hbm", 8.0 * T * di, 8.0 * T * di),
         "dequant": ("hbm", qbytes + 2.0 * do * di, qbytes + 2.0 * do * di),
-        "dequant_t": ("hbm", qbytes + 2.0 * do * di, qbytes + 2.0 * do * di),
         # sparse products: 2 p T FLOP; bytes = activations in and out + the index arrays
         "spmm_fwd": ("alu", 2.0 * p * T, 2.0 * T * di + 4.0 * T * do + 8.0 * p),
         "gather_bwd": ("alu", 2.0 * p * T, 2.0 * T * do + 4.0 * T * di + 12.0 * p),
         "sddmm_dc": ("alu", 2.0 * p * T, 2.0 * T * (di + do) + 8.0 * p),
         "gemm_fwd": ("tensor", 2.0 * T * di * do, 2.0 * T * di + 2.0 * do * di + 2.0 * T * do),
         "gemm_bwd": ("tensor", 2.0 * T * di * do, 2.0 * T * do + 2.0 * do * di + 2.0 * T * di),
-        "gemm_dc": ("tensor", 2.0 * T * di * do, 2.0 * T * (di + do) + 4.0 * do * di),
+        "gemm_dc": ("tensor", 2.0 * T * di * do, 2.0 * T * (di + do) + 12.0 * p),
         # W_eff = W_Q + alpha F H: codes + CSR in, bf16 out
         "weff": ("hbm", qbytes + 8.0 * p + 2.0 * do * di, qbytes + 8.0 * p + 2.0 * do * di),
-        "transpose_w": ("hbm", 4.0 * do * di, 4.0 * do * di),
-        "transpose_act": ("hbm", 4.0 * T * (di + do), 4.0 * T * (di + do)),
-        "gather_dc": ("hbm", 12.0 * p, 12.0 * p),
     }
     return w.get(stage)
 
@@ -308,6 +305,8 @@ def main():
                         a.row_idx, a.perm, a.tile_ptr, a.tile_pos, a.tile_rk, algo=algo)
         for algo in ("dense", "sparse")
     }
+    # the dense forward keeps W_eff = W_Q + alpha F H for its backward (like Z)
+    adapters["dense"].weff = torch.empty((spec.d_out, spec.d_in), dtype=torch.bfloat16, device=dev)
     ws = {}
     for algo, ops in (("dense", (4, 5)), ("sparse", (0, 1))):
         ws[algo] = [torch.empty(max(1, W.workspace_size(op, spec.d_out, spec.d_in, spec.p, T, True)),
@@ -454,7 +453,8 @@ def main():
         "ms_per_step": t_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; stands in for LLaMA-7B q_proj weights and activations)",
         "config": config_block(spec, world),
-        "algorithm": "dense: adapter folded into the tcgen05 GEMMs (W_eff = W_Q + alpha F H), dc from G = dY^T Z",
+        "algorithm": ("dense: adapter folded into the tcgen05 GEMMs (W_eff = W_Q + alpha F H, kept from the forward "
+                      "for the backward); dc from dY^T Z sampled at E in the GEMM epilogue"),
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -102,6 +102,13 @@ typedef struct {
   const float *coef;
   const int32_t *col_ptr, *row_idx, *perm;
   const int32_t *tile_ptr, *tile_pos, *tile_rk;
+  /* Optional (dense algorithm): bf16 [d_out, d_in] device buffer for
+   * W_eff = W_Q + alpha F H. When set, qwha_adapter_fwd writes W_eff there and
+   * qwha_adapter_bwd reads it as it stands instead of rebuilding it, like a
+   * tensor saved for the backward: the caller must run the forward after every
+   * change of coef, the base weight or alpha. NULL: each call builds its own
+   * copy in the workspace. */
+  void *weff;
 } qwha_adapter;
 
 /* The frozen quantized base weight W_Q [d_out, d_in], device memory.

@@ -205,6 +205,7 @@ CASES = [
     (1024, 768, 1024, 300, 768 * 24, "bf16", "init"),
     (768, 512, 256, 33, 512 * 30, "bf16", "random"),  # block-diagonal transform
     (96, 40, 32, 5, 300, "bf16", "random"),
+    (1024, 1024, 1024, 600, 1024 * 20, "bf16", "init"),  # dense: dc GEMM split in two along tokens
 ]
 
 
@@ -237,6 +238,12 @@ def test_adapter_forward_backward(d_in, d_out, n, T, p, dtype, pattern, algo):
     # fixed-order reduction: a second backward is bitwise identical
     dc2, _ = W.adapter_bwd(a, dYd, Z, alpha)
     assert torch.equal(dc, dc2)
+    if algo == "dense":
+        # W_eff saved by the forward and reused by the backward gives the same bits
+        a.weff = torch.empty((d_out, d_in), dtype=torch.bfloat16, device="cuda")
+        Z3, Y3 = W.adapter_fwd(a, Xd, alpha)
+        dc3, dX3 = W.adapter_bwd(a, dYd, Z3, alpha)
+        assert torch.equal(Y3, Y) and torch.equal(dc3, dc) and torch.equal(dX3, dX)
 
 
 GEMM_CASES = [

@@ -32,6 +32,7 @@ class QwhaAdapter(ctypes.Structure):
         ("tile_ptr", P),
         ("tile_pos", P),
         ("tile_rk", P),
+        ("weff", P),
     ]
 
 

@@ -64,6 +64,7 @@ class Adapter:
     tile_pos: torch.Tensor | None = None
     tile_rk: torch.Tensor | None = None
     algo: str = "sparse"
+    weff: torch.Tensor | None = None  # dense: W_eff kept from the forward for the backward
 
     def c_struct(self) -> QwhaAdapter:
         s = QwhaAdapter()

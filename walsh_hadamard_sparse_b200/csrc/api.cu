@@ -81,22 +81,17 @@ enum Stage {
   ST_SDDMM,
   ST_GATHER_BWD,
   ST_FWHT_BWD,
-  ST_DEQUANT_T,
   ST_GEMM_BWD,
   ST_INIT,
   ST_PLAN,
   ST_FWHT,
   ST_WEFF,
-  ST_TRANSPOSE_W,
-  ST_TRANSPOSE_ACT,
   ST_GEMM_DC,
-  ST_GATHER_DC,
   ST_COUNT
 };
 const char *kStageNames[ST_COUNT] = {"fwht_fwd",   "spmm_fwd",   "dequant",  "gemm_fwd",  "sddmm_dc",
-                                     "gather_bwd", "fwht_bwd",   "dequant_t", "gemm_bwd", "init_alloc",
-                                     "plan_build", "fwht",       "weff",      "transpose_w", "transpose_act",
-                                     "gemm_dc",    "gather_dc"};
+                                     "gather_bwd", "fwht_bwd",   "gemm_bwd", "init_alloc",
+                                     "plan_build", "fwht",       "weff",      "gemm_dc"};
 
 struct StageRec {
   int stage, kernels;
@@ -253,6 +248,7 @@ qwha_status check_adapter_shape(const qwha_adapter *a) {
     return fail(QWHA_ERR_INVALID_ARG, "algo %d", (int)a->algo);
   if (a->algo == QWHA_ALGO_DENSE && weff_smem(a->d_in) > 200 * 1024)
     return fail(QWHA_ERR_UNSUPPORTED, "dense algorithm: d_in %d above 51200", a->d_in);
+  if (a->weff && !aligned16(a->weff)) return fail(QWHA_ERR_MISALIGNED, "weff is not 16-byte aligned");
   QWHA_CHECK_PTR(a->row_ptr, "row_ptr");
   if (a->p > 0) {
     QWHA_CHECK_PTR(a->col_idx, "col_idx");
@@ -306,11 +302,8 @@ size_t fwd_dense_ws(int32_t d_out, int32_t d_in) { return align_up((size_t)d_out
 int64_t pad8(int64_t v) { return (v + 7) / 8 * 8; }
 
 size_t bwd_dense_ws(int32_t d_out, int32_t d_in, int64_t T) {
-  const int64_t Tp = pad8(T);
-  return 2 * align_up((size_t)d_out * d_in * 2, 256)        // W_eff and its transpose
-         + align_up((size_t)d_out * Tp * 2, 256)            // dY^T
-         + align_up((size_t)d_in * Tp * 2, 256)             // Z^T
-         + align_up((size_t)d_out * d_in * 4, 256);         // G = dY^T Z
+  (void)T;
+  return align_up((size_t)d_out * d_in * 2, 256);  // W_eff (unless the adapter carries one)
 }
 
 size_t bwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
@@ -321,49 +314,34 @@ size_t bwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
   return n;
 }
 
-// Dense backward: W_eff and W_eff^T, dX = dY W_eff, G = dY^T Z, dc = alpha G at E.
+// Dense backward: W_eff, dX = dY W_eff (W_eff read MN-major), and dc = alpha *
+// (dY^T Z) sampled at E by the GEMM epilogue (both operands read MN-major as
+// stored).
 qwha_status dense_bwd(const qwha_adapter *a, const qwha_qweight *wq, const void *dY, const void *Z, int64_t T,
                       float alpha, float *dc, void *dX, void *ws, cudaStream_t s) {
-  const int64_t Tp = pad8(T);
   Carver cv(ws);
-  void *weff = cv.take((size_t)a->d_out * a->d_in * 2);
-  void *weff_t = cv.take((size_t)a->d_out * a->d_in * 2);
-  void *dyt = cv.take((size_t)a->d_out * Tp * 2);
-  void *zt = cv.take((size_t)a->d_in * Tp * 2);
-  float *G = static_cast<float *>(cv.take((size_t)a->d_out * a->d_in * 4));
+  void *weff = a->weff ? a->weff : cv.take((size_t)a->d_out * a->d_in * 2);
   cudaError_t e = cudaSuccess;
   if (dX && T > 0) {
-    {
+    if (!a->weff) {  // otherwise the forward's W_eff is used as it stands
       StageScope sc(ST_WEFF, 1, s);
-      e = launch_weff(a, wq, 1.0f * alpha, weff, s);
+      e = launch_weff(a, wq, alpha, weff, s);
     }
     if (e != cudaSuccess) return cuda_status(e, "W_eff");
     {
-      StageScope sc(ST_TRANSPOSE_W, 1, s);
-      e = launch_transpose_bf16(weff, a->d_out, a->d_in, weff_t, a->d_out, s);
-    }
-    if (e != cudaSuccess) return cuda_status(e, "transpose W_eff");
-    {
       StageScope sc(ST_GEMM_BWD, 1, s);
-      e = launch_gemm_nt(dY, weff_t, nullptr, dX, false, T, a->d_in, a->d_out, s);
+      e = launch_gemm_any(dY, false, weff, true, nullptr, dX, false, T, a->d_in, a->d_out, s);
     }
     if (e != cudaSuccess) return cuda_status(e, "GEMM dX");
   }
   if (a->p == 0) return QWHA_OK;
   if (T == 0) return cuda_status(cudaMemsetAsync(dc, 0, (size_t)a->p * 4, s), "dc = 0");
-  {
-    StageScope sc(ST_TRANSPOSE_ACT, 2, s);
-    e = launch_transpose_bf16(dY, T, a->d_out, dyt, Tp, s);
-    if (e == cudaSuccess) e = launch_transpose_bf16(Z, T, a->d_in, zt, Tp, s);
-  }
-  if (e != cudaSuccess) return cuda_status(e, "transpose dY, Z");
-  {
-    StageScope sc(ST_GEMM_DC, 1, s);
-    e = launch_gemm_nt(dyt, zt, nullptr, G, true, a->d_out, a->d_in, Tp, s);
-  }
-  if (e != cudaSuccess) return cuda_status(e, "GEMM dY^T Z");
-  StageScope sc(ST_GATHER_DC, 1, s);
-  return cuda_status(launch_gather_dc(G, a->row_ptr, a->col_idx, a->d_out, a->d_in, a->p, alpha, dc, s), "gather dc");
+  // the coefficient gradient as a sampled dense product: the tcgen05 GEMM's
+  // epilogue writes alpha * (dY^T Z)[r_j, k_j] for the entries of E only
+  StageScope sc(ST_GEMM_DC, 1, s);
+  return cuda_status(launch_gemm_sampled(dY, true, Z, true, a->d_out, a->d_in, T, a->row_ptr, a->col_idx, a->p, alpha,
+                                         dc, s),
+                     "sampled GEMM dY^T Z");
 }
 
 }  // namespace
@@ -414,7 +392,7 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   }
   if (e != cudaSuccess) return cuda_status(e, "fwht");
   if (dense) {
-    void *weff = ws;
+    void *weff = a->weff ? a->weff : ws;
     {
       StageScope sc(ST_WEFF, 1, s);
       e = launch_weff(a, wq, alpha, weff, s);
@@ -439,7 +417,7 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   if (e != cudaSuccess) return cuda_status(e, "spmm");
   {
     StageScope sc(ST_DEQUANT, 1, s);
-    e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, false, s);
+    e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, s);
   }
   if (e != cudaSuccess) return cuda_status(e, "dequant");
   StageScope sc(ST_GEMM_FWD, 1, s);
@@ -502,12 +480,14 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   }
   if (e != cudaSuccess) return cuda_status(e, "fwht");
   {
-    StageScope sc(ST_DEQUANT_T, 1, s);
-    e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, true, s);
+    StageScope sc(ST_DEQUANT, 1, s);
+    e = launch_dequant(wq->bits, wq->group, a->d_out, a->d_in, wq->qweight, wq->scales, wq->zeros, wdeq, s);
   }
   if (e != cudaSuccess) return cuda_status(e, "dequant");
   StageScope sc(ST_GEMM_BWD, 1, s);
-  return cuda_status(launch_gemm_bwd(dY, wdeq, dx_ad, dX, T, a->d_out, a->d_in, s), "base GEMM (dX)");
+  // dX = dY W_Q + dX_adapter: W_Q [d_out, d_in] is the MN-major B operand as stored
+  return cuda_status(launch_gemm_any(dY, false, wdeq, true, dx_ad, dX, false, T, a->d_in, a->d_out, s),
+                     "base GEMM (dX)");
 }
 
 qwha_status qwha_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr, const int32_t *col_idx,

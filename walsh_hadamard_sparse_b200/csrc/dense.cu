@@ -8,15 +8,16 @@
 //     W_eff = W_Q + alpha * F H,
 // makes the forward Y = X W_eff^T and the input gradient dX = dY W_eff plain
 // GEMMs: the adapter costs nothing in either. The coefficient gradient is the
-// sampled product dc_j = alpha * (dY^T Z)[r_j, k_j]: one dense GEMM
-// G = dY^T Z (contraction over tokens) and a gather at E.
+// sampled product dc_j = alpha * (dY^T Z)[r_j, k_j]: one dense GEMM over
+// tokens whose epilogue keeps only the entries of E.
 //
 // Kernels here: weff_kernel (one CTA per row of W_eff: scatter the row of F
 // into shared memory, fp32 butterflies per Hadamard block, add the dequantized
 // base row, one bf16 rounding; used for Hadamard blocks outside 128..4096,
 // the main path is weff_rows_kernel in fwht.cu on the transform's register
-// layout), transpose_bf16_kernel (64 x 64 tiles, zero pad of the output's
-// leading dimension), gather_dc_kernel.
+// layout). The GEMMs read dY, Z and W_eff as stored (MN-major operands), so
+// nothing is transposed, and the coefficient gradient is written by the
+// sampled epilogue of the dY^T Z GEMM (gemm.cu), so G never reaches memory.
 
 #include <algorithm>
 
@@ -85,52 +86,6 @@ __global__ void __launch_bounds__(kWeffThreads)
   }
 }
 
-// out[c][r] = in[r][c] for r < R, c < C; out rows have leading dimension ldo >= R,
-// columns R..ldo-1 are written as zeros. 64 x 64 tiles, 256 threads.
-__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ in, int64_t R,
-                                                             int64_t C, __nv_bfloat16 *__restrict__ out, int64_t ldo) {
-  __shared__ uint16_t tile[64][64 + 2];
-  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
-  const uint16_t *src = reinterpret_cast<const uint16_t *>(in);
-  for (int it = threadIdx.x; it < 64 * 8; it += 256) {
-    const int rr = it / 8, cc = (it % 8) * 8;
-    const int64_t r = r0 + rr, c = c0 + cc;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < R && c < C) v = *reinterpret_cast<const uint4 *>(src + r * C + c);
-    const uint16_t *h = reinterpret_cast<const uint16_t *>(&v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) tile[rr][cc + i] = h[i];
-  }
-  __syncthreads();
-  uint16_t *dst = reinterpret_cast<uint16_t *>(out);
-  for (int it = threadIdx.x; it < 64 * 8; it += 256) {
-    const int cc = it / 8, rr = (it % 8) * 8;
-    const int64_t c = c0 + cc, r = r0 + rr;
-    if (c >= C || r >= ldo) continue;
-    uint16_t h[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) h[i] = (r + i < R) ? tile[rr + i][cc] : 0;
-    *reinterpret_cast<uint4 *>(dst + c * ldo + r) = *reinterpret_cast<const uint4 *>(h);
-  }
-}
-
-// dc[j] = alpha * G[r_j, col_idx[j]]: one warp per row of F.
-__global__ void gather_dc_kernel(const float *__restrict__ G, const int32_t *__restrict__ row_ptr,
-                                 const int32_t *__restrict__ col_idx, int d_out, int d_in, int64_t p, float alpha,
-                                 float *__restrict__ dc) {
-  const int lane = threadIdx.x & 31;
-  for (int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; r < d_out;
-       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    int64_t b = row_ptr[r], e = row_ptr[r + 1];
-    if (b < 0) b = 0;
-    if (e > p) e = p;
-    for (int64_t j = b + lane; j < e; j += 32) {
-      const int k = col_idx[j];
-      dc[j] = (unsigned)k < (unsigned)d_in ? alpha * G[r * d_in + k] : 0.f;
-    }
-  }
-}
-
 }  // namespace
 
 size_t weff_smem(int32_t d_in) { return (size_t)d_in * sizeof(float); }
@@ -149,22 +104,6 @@ cudaError_t launch_weff(const qwha_adapter *a, const qwha_qweight *wq, float alp
                                                    wq ? wq->bits : 0, wq ? wq->group : 1, wq ? wq->qweight : nullptr,
                                                    wq ? wq->scales : nullptr, wq ? wq->zeros : nullptr,
                                                    static_cast<__nv_bfloat16 *>(out));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_transpose_bf16(const void *in, int64_t R, int64_t C, void *out, int64_t ldo, cudaStream_t s) {
-  if (R <= 0 || C <= 0) return cudaSuccess;
-  dim3 grid((unsigned)cdiv(C, 64), (unsigned)cdiv(ldo, 64));
-  transpose_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(in), R, C,
-                                             static_cast<__nv_bfloat16 *>(out), ldo);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_dc(const float *G, const int32_t *row_ptr, const int32_t *col_idx, int32_t d_out,
-                             int32_t d_in, int64_t p, float alpha, float *dc, cudaStream_t s) {
-  if (p <= 0) return cudaSuccess;
-  const int64_t grid = std::min<int64_t>(cdiv((int64_t)d_out * 32, 256), (int64_t)sm_count() * 8);
-  gather_dc_kernel<<<(unsigned)grid, 256, 0, s>>>(G, row_ptr, col_idx, d_out, d_in, p, alpha, dc);
   return cudaGetLastError();
 }
 

@@ -3,9 +3,8 @@
 // rounded once to bf16. q[i][k] is bits [b*k, b*k+b) of row i's little-endian
 // bit stream. Eight consecutive codes share a group (group % 8 == 0) and span
 // exactly b bytes, so a thread dequantizes one 8-code run from b byte loads.
-//   natural:    out[i][k]  ([d_out, d_in], K-major B operand of Y = X W_Q^T)
-//   transposed: out[k][i]  ([d_in, d_out], K-major B operand of dX = dY W_Q),
-//               through a 64 x 64 shared-memory tile.
+// out[i][k] is [d_out, d_in]: the K-major B operand of Y = X W_Q^T and, read
+// MN-major, the B operand of dX = dY W_Q.
 
 #include <algorithm>
 
@@ -42,53 +41,16 @@ __global__ void dequant_kernel(const uint8_t *__restrict__ qw, const float *__re
   }
 }
 
-// 64 x 64 tiles: a thread dequantizes one 8-code run of a W row, the tile is
-// written transposed with 16-byte stores along i.
-__global__ void __launch_bounds__(512) dequant_t_kernel(const uint8_t *__restrict__ qw, const float *__restrict__ scales,
-                                                        const uint8_t *__restrict__ zeros, int bits, int group,
-                                                        int d_out, int d_in, __nv_bfloat16 *__restrict__ out) {
-  __shared__ float tile[64][65];
-  const int i0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
-  const int64_t row_bytes = (int64_t)d_in * bits / 8;
-  const int ng = d_in / group;
-  {
-    const int ii = threadIdx.x / 8, run = threadIdx.x % 8;  // 64 rows x 8 runs
-    const int i = i0 + ii, k = k0 + run * 8;
-    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (i < d_out && k < d_in) dequant8(qw + (int64_t)i * row_bytes, bits, k, scales[(int64_t)i * ng + k / group],
-                                        (float)zeros[(int64_t)i * ng + k / group], v);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) tile[ii][run * 8 + u] = v[u];
-  }
-  __syncthreads();
-  {
-    const int kk = threadIdx.x / 8, run = threadIdx.x % 8;  // 64 k-rows x 8 runs of i
-    const int k = k0 + kk, i = i0 + run * 8;
-    if (k < d_in && i < d_out) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = tile[run * 8 + u][kk];
-      *reinterpret_cast<uint4 *>(out + (int64_t)k * d_out + i) = io<__nv_bfloat16>::pack(v);
-    }
-  }
-}
-
 }  // namespace
 
 size_t wdeq_bytes(int32_t d_out, int32_t d_in) { return (size_t)d_out * d_in * 2; }
 
 cudaError_t launch_dequant(int bits, int group, int32_t d_out, int32_t d_in, const uint8_t *qw, const float *scales,
-                           const uint8_t *zeros, void *out, bool transposed, cudaStream_t s) {
-  if (!transposed) {
-    const int64_t total = (int64_t)d_out * (d_in / 8);
-    const int64_t grid = std::min<int64_t>(cdiv(total, 256), (int64_t)sm_count() * 16);
-    dequant_kernel<<<(unsigned)grid, 256, 0, s>>>(qw, scales, zeros, bits, group, d_out, d_in,
-                                                  static_cast<__nv_bfloat16 *>(out));
-  } else {
-    dim3 grid((unsigned)cdiv(d_in, 64), (unsigned)cdiv(d_out, 64));
-    dequant_t_kernel<<<grid, 512, 0, s>>>(qw, scales, zeros, bits, group, d_out, d_in,
-                                          static_cast<__nv_bfloat16 *>(out));
-  }
+                           const uint8_t *zeros, void *out, cudaStream_t s) {
+  const int64_t total = (int64_t)d_out * (d_in / 8);
+  const int64_t grid = std::min<int64_t>(cdiv(total, 256), (int64_t)sm_count() * 16);
+  dequant_kernel<<<(unsigned)grid, 256, 0, s>>>(qw, scales, zeros, bits, group, d_out, d_in,
+                                                static_cast<__nv_bfloat16 *>(out));
   return cudaGetLastError();
 }
 

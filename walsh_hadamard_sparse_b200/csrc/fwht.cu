@@ -20,7 +20,8 @@
 // are flipped by the high field's low bits) so that phase-B scalar accesses hit
 // 32 distinct banks and phase-A 16-byte accesses stay contiguous. The result
 // goes back through the same buffer (in the output type) to phase-A layout for
-// coalesced stores. Arithmetic is fp32 whatever the I/O type.
+// coalesced stores. Arithmetic is fp32 whatever the I/O type. The next rows'
+// inputs are prefetched with cp.async into shared memory during the arithmetic.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -63,13 +64,6 @@ struct Geo {
 };
 
 template <typename T, int V>
-__device__ __forceinline__ void load_group(const T *p, float *o) {
-  constexpr int NU = V * (int)sizeof(T) / 16;
-#pragma unroll
-  for (int u = 0; u < NU; ++u) io<T>::unpack(ld_stream(p + u * io<T>::kVec), o + u * io<T>::kVec);
-}
-
-template <typename T, int V>
 __device__ __forceinline__ void store_group(T *p, const float *i) {
   constexpr int NU = V * (int)sizeof(T) / 16;
 #pragma unroll
@@ -92,32 +86,99 @@ __device__ __forceinline__ void butterflies(float *v) {
   }
 }
 
+// Two butterflies at once with the packed fp32x2 add/sub of sm_100:
+// (a0, a1), (b0, b1) <- (a0 + b0, a1 + b1), (a0 - b0, a1 - b1).
+__device__ __forceinline__ void bfly2(float &a0, float &a1, float &b0, float &b1) {
+  unsigned long long a, b, sum, dif;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(sum) : "l"(a), "l"(b));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(dif) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(sum));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(dif));
+}
+
+// Same result as butterflies<R, B0, NBITS>, registers paired along index bit PB:
+// stages on other bits run two butterflies per packed add and sub; a stage on
+// PB itself (if in range) runs scalar.
+template <int R, int B0, int NBITS, int PB>
+__device__ __forceinline__ void butterflies_x2(float *v) {
+  constexpr int P = 1 << PB;
+#pragma unroll
+  for (int b = B0; b < B0 + NBITS; ++b) {
+    const int h = 1 << b;
+    if (b == PB) {
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+        if (!(q & h)) {
+          const float a = v[q], c = v[q + h];
+          v[q] = a + c;
+          v[q + h] = a - c;
+        }
+    } else {
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+        if (!(q & h) && !(q & P)) bfly2(v[q], v[q + P], v[q + h], v[q + h + P]);
+    }
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// The input rows of the next iteration are copied into a shared-memory staging
+// buffer with cp.async while the current rows are transformed; phase A then
+// reads its 16-byte vectors from shared memory.
 template <int LOGN, int V, typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads) fwht_rows_kernel(const Tin *__restrict__ x,
-                                                             Tout *__restrict__ z, int64_t rows,
-                                                             float scale) {
+__global__ void __launch_bounds__(kThreads) fwht_rows_kernel(const Tin *__restrict__ x, Tout *__restrict__ z,
+                                                             int64_t rows, float scale) {
   using G = Geo<LOGN, V>;
   constexpr int RPC = kThreads / G::P;  // rows per CTA iteration
+  constexpr int ROW_CHUNKS = G::N * (int)sizeof(Tin) / 16;
   extern __shared__ __align__(16) float smem[];
   const int rl = threadIdx.x / G::P;
   const int t = threadIdx.x % G::P;
   float *buf = smem + rl * G::N;
+  Tin *stage = reinterpret_cast<Tin *>(smem + RPC * G::N);
 
-  for (int64_t base = (int64_t)blockIdx.x * RPC; base < rows; base += (int64_t)gridDim.x * RPC) {
+  auto prefetch = [&](int64_t first) {
+    const int64_t left = rows - first;
+    const int nrow = left < RPC ? (int)left : RPC;
+    const char *src = reinterpret_cast<const char *>(x + first * G::N);
+    char *dst = reinterpret_cast<char *>(stage);
+    for (int c = threadIdx.x; c < nrow * ROW_CHUNKS; c += kThreads) cp_async16(dst + 16 * c, src + 16 * (int64_t)c);
+    cp_async_commit();
+  };
+
+  int64_t base = (int64_t)blockIdx.x * RPC;
+  if (base < rows) prefetch(base);
+  for (; base < rows; base += (int64_t)gridDim.x * RPC) {
     const int64_t row = base + rl;
     const bool active = row < rows;
+    cp_async_wait_all();
+    __syncthreads();  // this iteration's rows are staged; last iteration's readers of buf are done
     float v[G::R];
     if (active) {
-      const Tin *xr = x + row * G::N;
+      const Tin *xr = stage + rl * G::N;
 #pragma unroll
-      for (int h = 0; h < (1 << G::HB); ++h) load_group<Tin, V>(xr + G::eA(t, h << G::LV), v + h * V);
+      for (int h = 0; h < (1 << G::HB); ++h) {
+        const Tin *src = xr + G::eA(t, h << G::LV);
+#pragma unroll
+        for (int u = 0; u < V; u += io<Tin>::kVec)
+          io<Tin>::unpack(*reinterpret_cast<const uint4 *>(src + u), v + h * V + u);
+      }
     } else {
 #pragma unroll
       for (int q = 0; q < G::R; ++q) v[q] = 0.f;
     }
-    butterflies<G::R, 0, G::RB>(v);
+    __syncthreads();  // the staging buffer is free: fetch the next rows during the arithmetic
+    if (base + (int64_t)gridDim.x * RPC < rows) prefetch(base + (int64_t)gridDim.x * RPC);
+    butterflies_x2<G::R, 0, G::RB, 0>(v);
 
-    __syncthreads();  // the previous iteration's readers are done with buf
 #pragma unroll
     for (int h = 0; h < (1 << G::HB); ++h) {
       float *dst = buf + G::phys(G::eA(t, h << G::LV));
@@ -129,7 +190,7 @@ __global__ void __launch_bounds__(kThreads) fwht_rows_kernel(const Tin *__restri
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
-    butterflies<G::R, 0, G::PB>(v);
+    butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
     __syncthreads();  // all phase-B reads done before the buffer is reused
 
     Tout *st = reinterpret_cast<Tout *>(buf);
@@ -254,7 +315,7 @@ __global__ void __launch_bounds__(kThreads)
         v[h * 8 + u] = f.x, v[h * 8 + u + 1] = f.y, v[h * 8 + u + 2] = f.z, v[h * 8 + u + 3] = f.w;
       }
     }
-    butterflies<G::R, 0, G::RB>(v);
+    butterflies_x2<G::R, 0, G::RB, 0>(v);
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < (1 << G::HB); ++h) {
@@ -266,7 +327,7 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
-    butterflies<G::R, 0, G::PB>(v);
+    butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < G::R; ++q) buf[G::phys(G::eB(t, q))] = v[q] * scale;
@@ -324,7 +385,7 @@ cudaError_t run_rows(const Tin *x, Tout *z, int64_t rows, float scale, cudaStrea
   constexpr int V = (sizeof(Tin) == 2 || sizeof(Tout) == 2) ? 8 : 4;
   using G = Geo<LOGN, V>;
   constexpr int RPC = kThreads / G::P;
-  const size_t smem = (size_t)RPC * G::N * sizeof(float);
+  const size_t smem = (size_t)RPC * G::N * (sizeof(float) + sizeof(Tin));
   auto k = fwht_rows_kernel<LOGN, V, Tin, Tout>;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {

@@ -2,14 +2,17 @@
 //   out[M, N] = A[M, K] . B[N, K]^T (+ addend[M, N]), out bf16 or fp32
 // with A, B bf16 K-major (row-major with K contiguous) and addend fp32.
 //   forward:  Y  = X W_Q^T + Y_adapter   (A = X, B = W_Q, K = d_in)
-//   backward: dX = dY W_Q + dX_adapter   (A = dY, B = W_Q^T, K = d_out)
+//   backward: dX = dY W_Q + dX_adapter   (A = dY, B = W_Q read MN-major, K = d_out)
 // The adapter term rides in the epilogue, so it costs one fp32 read.
 //
 // Structure (one CTA per SM, persistent over 128 x 256 output tiles):
 //   warp 0, one thread : TMA producer. 2-D tensor copies (128B swizzle, no
 //                        multicast) of A and B k-blocks of 64 into a 4-stage
 //                        shared-memory ring, completion counted in bytes on
-//                        the stage's "full" mbarrier.
+//                        the stage's "full" mbarrier. An operand may be K-major
+//                        (one box of rows x 64 K) or MN-major (64 x 64 boxes
+//                        along MN); the UMMA descriptors and the instruction
+//                        descriptor's major bits follow.
 //   warp 1, one thread : MMA issuer. tcgen05.mma kind::f16 (bf16 x bf16 ->
 //                        fp32) M=128 N=256 K=16, accumulator in TMEM;
 //                        tcgen05.commit frees the stage ("empty") and, after
@@ -26,6 +29,8 @@
 
 #include <cuda.h>
 
+#include <cmath>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,7 +43,20 @@ constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr uint32_t B_BYTES = BN * BK * 2;
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr size_t kGemmSmem = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int kEpiStride = 33;  // per-warp staging row (floats) of the sampled epilogue
+constexpr size_t kEpiSmem = 4 * 32 * kEpiStride * sizeof(float);
+constexpr size_t kGemmSmem = (size_t)STAGES * STAGE_BYTES + 1024 + 256 + kEpiSmem;
+
+enum { kOutBf16 = 0, kOutF32 = 1, kOutSampled = 2 };
+
+// Sampled output: dc[j] (+)= alpha * D[r_j, k_j] for the CSR entries of E.
+struct SampleArgs {
+  const int32_t *row_ptr;
+  const int32_t *col_idx;
+  float *dc;
+  float alpha;
+  int64_t p;
+};
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
@@ -102,9 +120,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 }
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  // start >> 4 | LBO 16 B (unused for swizzled K-major) | SBO 1024 B (8 rows of
-  // 128 B) | descriptor version 1 | layout SWIZZLE_128B (2)
+  // K-major: start >> 4 | LBO 16 B (unused for swizzled K-major) | SBO 1024 B
+  // (8 rows of 128 B) | descriptor version 1 | layout SWIZZLE_128B (2)
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
+  // MN-major: the stage holds 64(MN) x 64(K) boxes of 8 KB each, rows of 128 B
+  // along MN, one box after the other along MN. LBO = 8 KB (next 64 MN
+  // elements), SBO = 1024 B (next 8 K rows), version 1, SWIZZLE_128B.
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(8192 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
@@ -138,11 +164,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
 }
 
 // kF32Out: write fp32 D (no rounding); otherwise bf16. addend may be NULL.
-template <bool kF32Out>
+// a_mn / b_mn: the operand is MN-major in global memory ([K rows][M or N
+// contiguous]); its stage is then filled by BM/64 or BN/64 boxes of 64 x 64.
+// k_splits > 1 (sampled output only): each tile's K range is cut into that
+// many parts, each part a separate work unit adding its share into dc.
+template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const float *__restrict__ addend, void *__restrict__ out_v, int M, int N, int K,
-                             unsigned int *err) {
+                             int a_mn, int b_mn, int group_m, int k_splits, SampleArgs sa_args, unsigned int *err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t base = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
@@ -157,6 +187,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *epi_stage = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -186,7 +217,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int m_tiles = (M + BM - 1) / BM, n_tiles = (N + BN - 1) / BN;
   const int k_blocks = (K + BK - 1) / BK;
+  const int kb_per_split = (k_blocks + k_splits - 1) / k_splits;
   const int num_tiles = m_tiles * n_tiles;
+  const int num_units = num_tiles * k_splits;
+  // Tile order: groups of group_m row blocks; inside a group, the row block
+  // changes fastest and the column block slowest, so the tiles in flight share
+  // a few row blocks of A and a run of column blocks of B in L2.
+  auto tile_coords = [&](int tile, int &m_blk, int &n_blk) {
+    const int gsize = group_m * n_tiles;
+    const int g = tile / gsize, rem = tile % gsize;
+    const int gm = min(group_m, m_tiles - g * group_m);
+    m_blk = g * group_m + rem % gm;
+    n_blk = rem / gm;
+  };
 
   auto give_up = [&](unsigned code) {
     atomicOr(err, code);
@@ -199,17 +242,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     int last_parity[STAGES];
     for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
-    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
-      for (int kb = 0; kb < k_blocks; ++kb) {
+    for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
+      const int tile = unit / k_splits, split = unit % k_splits;
+      int m_blk, n_blk;
+      tile_coords(tile, m_blk, n_blk);
+      const int kb0 = split * kb_per_split, kb1 = min(k_blocks, kb0 + kb_per_split);
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(empty(stage), phase ^ 1)) {
           give_up(0x1u);
           break;
         }
         if (*abort_flag) break;
         mbar_expect_tx(full(stage), STAGE_BYTES);
-        tma_load_2d(base + stage * STAGE_BYTES, &tmA, full(stage), kb * BK, m_blk * BM);
-        tma_load_2d(base + stage * STAGE_BYTES + A_BYTES, &tmB, full(stage), kb * BK, n_blk * BN);
+        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+        if (a_mn) {
+#pragma unroll
+          for (int h = 0; h < BM / 64; ++h) tma_load_2d(sa + h * 8192, &tmA, full(stage), m_blk * BM + 64 * h, kb * BK);
+        } else {
+          tma_load_2d(sa, &tmA, full(stage), kb * BK, m_blk * BM);
+        }
+        if (b_mn) {
+#pragma unroll
+          for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmB, full(stage), n_blk * BN + 64 * h, kb * BK);
+        } else {
+          tma_load_2d(sb, &tmB, full(stage), kb * BK, n_blk * BN);
+        }
         last_parity[stage] = (int)phase;
         if (++stage == STAGES) {
           stage = 0;
@@ -225,7 +282,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, ++it) {
+    for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x, ++it) {
+      const int split = unit % k_splits;
+      const int kb0 = split * kb_per_split, kb1 = min(k_blocks, kb0 + kb_per_split);
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (!mbar_wait(tempty(buf), (use & 1) ^ 1)) {
@@ -235,18 +294,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
       bool ok = true;
-      for (int kb = 0; kb < k_blocks; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(full(stage), phase)) {
           give_up(0x8u);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t da = sw128_desc(base + stage * STAGE_BYTES);
-        const uint64_t db = sw128_desc(base + stage * STAGE_BYTES + A_BYTES);
+        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+        const uint64_t da = a_mn ? sw128_desc_mn(sa) : sw128_desc(sa);
+        const uint64_t db = b_mn ? sw128_desc_mn(sb) : sw128_desc(sb);
+        // next 16 of K: +32 B inside the 128 B rows (K-major), +2 KB = 16 rows (MN-major)
+        const uint64_t sta = a_mn ? 128ull : 2ull, stb = b_mn ? 128ull : 2ull;
+        const uint32_t idesc = kIdesc | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
-          umma_bf16(d_tmem, da + 2ull * k, db + 2ull * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          umma_bf16(d_tmem, da + sta * k, db + stb * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
         umma_commit(empty(stage));
         if (++stage == STAGES) {
           stage = 0;
@@ -263,7 +326,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    float *my_stage = epi_stage + (warp - 2) * 32 * kEpiStride;
+    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++it) {
+      const int tile = unit / k_splits;
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (*abort_flag) break;
@@ -272,12 +337,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m_blk = tile % m_tiles, n_blk = tile / m_tiles;
+      int m_blk, n_blk;
+      tile_coords(tile, m_blk, n_blk);
       const int row = m_blk * BM + q * 32 + lane;
+      // sampled output: this row's CSR entries with column in [n0, n0 + BN)
+      int64_t j = 0, j_end = 0;
+      if (kMode == kOutSampled && row < M) {
+        j = sa_args.row_ptr[row];
+        j_end = sa_args.row_ptr[row + 1];
+        if (j < 0) j = 0;
+        if (j_end > sa_args.p) j_end = sa_args.p;
+        int64_t hi = j_end;  // first entry with column >= n0 (columns ascend within a row)
+        while (j < hi) {
+          const int64_t mid = (j + hi) >> 1;
+          if (sa_args.col_idx[mid] < n_blk * BN) j = mid + 1;
+          else hi = mid;
+        }
+      }
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
         const int col0 = n_blk * BN + c * 32;
+        if (kMode == kOutSampled) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) my_stage[lane * kEpiStride + i] = __uint_as_float(r[i]);
+          __syncwarp();
+          for (; j < j_end; ++j) {
+            const int k = sa_args.col_idx[j] - col0;
+            if (k >= 32) break;
+            if (k >= 0) {
+              const float v = sa_args.alpha * my_stage[lane * kEpiStride + k];
+              if (k_splits > 1) atomicAdd(sa_args.dc + j, v);
+              else sa_args.dc[j] = v;
+            }
+          }
+          __syncwarp();
+          continue;
+        }
         if (row < M && col0 < N) {
           const int64_t off = (int64_t)row * N + col0;
           float f[32];
@@ -297,7 +393,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (col0 + j < N) f[j] += ad[j];
             }
           }
-          if (kF32Out) {
+          if (kMode == kOutF32) {
             float *o = static_cast<float *>(out_v) + off;
             if (col0 + 32 <= N) {
 #pragma unroll
@@ -357,36 +453,65 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, uint3
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t box[2] = {64u, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kF32Out>
+// A is [M, K] (K-major) or, with a_mn, [K, M]; B is [N, K] or, with b_mn, [K, N].
+template <int kMode>
 cudaError_t launch_gemm_t(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
-                          int64_t K, cudaStream_t s) {
+                          int64_t K, bool a_mn, bool b_mn, const SampleArgs &sa, cudaStream_t s) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, B, N, K, BN)) return cudaErrorInvalidValue;
+  const bool ok_a = a_mn ? make_map(&ta, A, K, M, 64) : make_map(&ta, A, M, K, BM);
+  const bool ok_b = b_mn ? make_map(&tb, B, K, N, 64) : make_map(&tb, B, N, K, BN);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05_kernel<kF32Out>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05_kernel<kMode>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int64_t tiles = cdiv(M, BM) * cdiv(N, BN);
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  gemm_bf16_tcgen05_kernel<kF32Out><<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, addend, out, (int)M, (int)N,
-                                                                          (int)K, device_error_word());
+  const int64_t m_tiles = cdiv(M, BM), n_tiles = cdiv(N, BN);
+  const int64_t tiles = m_tiles * n_tiles;
+  // Rows of A per group: all column blocks of B for one row block at a time
+  // when B fits comfortably in L2 (it is then read from DRAM once); otherwise
+  // enough row blocks that the tiles in flight span a bounded slice of B.
+  const int64_t b_bytes = N * K * 2;
+  int64_t group_m = 1;
+  if (b_bytes > (48ll << 20)) {
+    group_m = 8;
+    if (group_m > m_tiles) group_m = m_tiles;
+  }
+  // Sampled output: split K in two when the tiles alone would leave the last
+  // wave of SMs mostly idle (each dc then receives exactly two additions onto
+  // zero, whose result does not depend on their order).
+  int k_splits = 1;
+  const int sms = sm_count();
+  if (kMode == kOutSampled && cdiv(K, BK) >= 8) {
+    const double waves1 = (double)tiles / sms, waves2 = 2.0 * tiles / sms;
+    const double eff1 = waves1 / std::ceil(waves1), eff2 = waves2 / std::ceil(waves2);
+    if (eff2 > eff1 + 0.02) k_splits = 2;
+  }
+  if (kMode == kOutSampled) {
+    cudaError_t e = k_splits > 1 ? cudaMemsetAsync(sa.dc, 0, (size_t)sa.p * sizeof(float), s) : cudaSuccess;
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t units = tiles * k_splits;
+  const int grid = (int)(units < sms ? units : sms);
+  gemm_bf16_tcgen05_kernel<kMode><<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, addend, out, (int)M, (int)N, (int)K,
+                                                                       a_mn ? 1 : 0, b_mn ? 1 : 0, (int)group_m,
+                                                                       k_splits, sa, device_error_word());
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
                         int64_t K, cudaStream_t s) {
-  return launch_gemm_t<false>(A, B, addend, out, M, N, K, s);
+  return launch_gemm_t<kOutBf16>(A, B, addend, out, M, N, K, false, false, SampleArgs{}, s);
 }
 
 }  // namespace
@@ -396,15 +521,23 @@ cudaError_t launch_gemm_fwd(const void *X, const void *wdeq, const float *y_ad, 
   return launch_gemm(X, wdeq, y_ad, Y, T, d_out, d_in, s);
 }
 
-cudaError_t launch_gemm_bwd(const void *dY, const void *wdeq_t, const float *dx_ad, void *dX, int64_t T,
-                            int32_t d_out, int32_t d_in, cudaStream_t s) {
-  return launch_gemm(dY, wdeq_t, dx_ad, dX, T, d_in, d_out, s);
-}
-
 cudaError_t launch_gemm_nt(const void *A, const void *B, const float *addend, void *out, bool f32_out, int64_t M,
                            int64_t N, int64_t K, cudaStream_t s) {
-  return f32_out ? launch_gemm_t<true>(A, B, addend, out, M, N, K, s)
-                 : launch_gemm_t<false>(A, B, addend, out, M, N, K, s);
+  return f32_out ? launch_gemm_t<kOutF32>(A, B, addend, out, M, N, K, false, false, SampleArgs{}, s)
+                 : launch_gemm_t<kOutBf16>(A, B, addend, out, M, N, K, false, false, SampleArgs{}, s);
+}
+
+cudaError_t launch_gemm_any(const void *A, bool a_mn, const void *B, bool b_mn, const float *addend, void *out,
+                            bool f32_out, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
+  return f32_out ? launch_gemm_t<kOutF32>(A, B, addend, out, M, N, K, a_mn, b_mn, SampleArgs{}, s)
+                 : launch_gemm_t<kOutBf16>(A, B, addend, out, M, N, K, a_mn, b_mn, SampleArgs{}, s);
+}
+
+cudaError_t launch_gemm_sampled(const void *A, bool a_mn, const void *B, bool b_mn, int64_t M, int64_t N, int64_t K,
+                                const int32_t *row_ptr, const int32_t *col_idx, int64_t p, float alpha, float *dc,
+                                cudaStream_t s) {
+  SampleArgs sa{row_ptr, col_idx, dc, alpha, p};
+  return launch_gemm_t<kOutSampled>(A, B, nullptr, nullptr, M, N, K, a_mn, b_mn, sa, s);
 }
 
 }  // namespace qwha

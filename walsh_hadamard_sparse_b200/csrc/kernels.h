@@ -61,19 +61,25 @@ cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int3
                               int32_t min_per_row, int mode, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx,
                               float *coef, void *ws, cudaStream_t s);
 
-// Base weight (dequant.cu): bf16 W_Q [d_out, d_in] or its transpose [d_in, d_out].
+// Base weight (dequant.cu): bf16 W_Q [d_out, d_in].
 size_t wdeq_bytes(int32_t d_out, int32_t d_in);
 cudaError_t launch_dequant(int bits, int group, int32_t d_out, int32_t d_in, const uint8_t *qw, const float *scales,
-                           const uint8_t *zeros, void *out, bool transposed, cudaStream_t s);
+                           const uint8_t *zeros, void *out, cudaStream_t s);
 
 // Base GEMM with fp32 addend in the epilogue (gemm.cu).
 cudaError_t launch_gemm_fwd(const void *X, const void *wdeq, const float *y_ad, void *Y, int64_t T, int32_t d_out,
                             int32_t d_in, cudaStream_t s);
-cudaError_t launch_gemm_bwd(const void *dY, const void *wdeq_t, const float *dx_ad, void *dX, int64_t T,
-                            int32_t d_out, int32_t d_in, cudaStream_t s);
 // out[M, N] = A[M, K] B[N, K]^T (+ addend), A and B bf16 K-major, out fp32 or bf16.
 cudaError_t launch_gemm_nt(const void *A, const void *B, const float *addend, void *out, bool f32_out, int64_t M,
                            int64_t N, int64_t K, cudaStream_t s);
+// dc[j] = alpha * (A B^T)[r_j, col_idx[j]] for the CSR entries of E, written
+// by the GEMM epilogue (no dense output).
+cudaError_t launch_gemm_sampled(const void *A, bool a_mn, const void *B, bool b_mn, int64_t M, int64_t N, int64_t K,
+                                const int32_t *row_ptr, const int32_t *col_idx, int64_t p, float alpha, float *dc,
+                                cudaStream_t s);
+// Same with either operand MN-major: A [K, M] when a_mn, B [K, N] when b_mn.
+cudaError_t launch_gemm_any(const void *A, bool a_mn, const void *B, bool b_mn, const float *addend, void *out,
+                            bool f32_out, int64_t M, int64_t N, int64_t K, cudaStream_t s);
 
 // Device error word and plan validation (misc.cu).
 cudaError_t read_and_clear_error_word(unsigned int *word, cudaStream_t s);
@@ -88,10 +94,5 @@ namespace qwha {
 size_t weff_smem(int32_t d_in);
 // out = bf16(dequant(W_Q) + alpha * (F H)) [d_out, d_in]; wq may be NULL (adapter alone).
 cudaError_t launch_weff(const qwha_adapter *a, const qwha_qweight *wq, float alpha, void *out, cudaStream_t s);
-// out[c][r] = in[r][c], out leading dimension ldo >= R (padding columns zeroed).
-cudaError_t launch_transpose_bf16(const void *in, int64_t R, int64_t C, void *out, int64_t ldo, cudaStream_t s);
-// dc[j] = alpha * G[r_j, col_idx[j]]
-cudaError_t launch_gather_dc(const float *G, const int32_t *row_ptr, const int32_t *col_idx, int32_t d_out,
-                             int32_t d_in, int64_t p, float alpha, float *dc, cudaStream_t s);
 
 }  // namespace qwha
