@@ -52,6 +52,34 @@ const char *dtype_name(qwha_dtype d) { return d == QWHA_F32 ? "f32" : d == QWHA_
 
 bool valid_dtype(qwha_dtype d) { return d == QWHA_F32 || d == QWHA_BF16; }
 
+// A second stream per device on which the dense forward computes Z = X H while
+// the caller's stream builds W_eff and runs the GEMM (they do not depend on each
+// other). Fork and join go through events, so the work stays ordered with the
+// caller's stream and is captured with it in a CUDA graph.
+struct Fork {
+  cudaStream_t aux = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+std::mutex g_fork_mu;
+Fork g_fork[64];
+
+cudaError_t get_fork(Fork **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  Fork &f = g_fork[dev];
+  if (!f.aux) {
+    e = cudaStreamCreateWithFlags(&f.aux, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&f.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&f.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  *out = &f;
+  return cudaSuccess;
+}
+
 qwha_status check_hadamard(int32_t n, int32_t had_block) {
   if (n <= 0) return fail(QWHA_ERR_INVALID_ARG, "row length %d must be positive", n);
   if (had_block < 2 || had_block > 32768 || !is_pow2(had_block))
@@ -386,21 +414,39 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   const int logn = ilog2(a->had_block);
   const float inv = (float)(1.0 / sqrt((double)a->had_block));
   cudaError_t e;
-  {
-    StageScope sc(ST_FWHT_FWD, 1, s);
-    e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
-  }
-  if (e != cudaSuccess) return cuda_status(e, "fwht");
   if (dense) {
+    // Z = X H (kept for the backward) on the auxiliary stream, concurrently
+    // with W_eff and Y = X W_eff^T on the caller's stream.
+    std::lock_guard<std::mutex> g(g_fork_mu);
+    Fork *f = nullptr;
+    e = get_fork(&f);
+    if (e == cudaSuccess) e = cudaEventRecord(f->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(f->aux, f->fork, 0);
+    if (e != cudaSuccess) return cuda_status(e, "fork");
+    {
+      StageScope sc(ST_FWHT_FWD, 1, f->aux);
+      e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, f->aux);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(f->join, f->aux);
+    if (e != cudaSuccess) return cuda_status(e, "fwht");
     void *weff = a->weff ? a->weff : ws;
     {
       StageScope sc(ST_WEFF, 1, s);
       e = launch_weff(a, wq, alpha, weff, s);
     }
-    if (e != cudaSuccess) return cuda_status(e, "W_eff");
-    StageScope sc(ST_GEMM_FWD, 1, s);
-    return cuda_status(launch_gemm_nt(X, weff, nullptr, Y, false, T, a->d_out, a->d_in, s), "GEMM with W_eff");
+    if (e == cudaSuccess) {
+      StageScope sc(ST_GEMM_FWD, 1, s);
+      e = launch_gemm_nt(X, weff, nullptr, Y, false, T, a->d_out, a->d_in, s);
+    }
+    const cudaError_t ej = cudaStreamWaitEvent(s, f->join, 0);  // join even after a failed launch
+    if (e != cudaSuccess) return cuda_status(e, "W_eff / GEMM");
+    return cuda_status(ej, "join");
   }
+  {
+    StageScope sc(ST_FWHT_FWD, 1, s);
+    e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
+  }
+  if (e != cudaSuccess) return cuda_status(e, "fwht");
   if (!wq) {
     StageScope sc(ST_SPMM_FWD, 1, s);
     e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, a->p, a->d_out, alpha, Y, s);

@@ -49,6 +49,7 @@ class LayerSpec:
     remainder: str = "fewest"  # "fewest" (pages) or "largest"
     x_stream: str = ""  # layers with the same x_stream read the same X
     min_per_row: int = 2
+    w_stream: str = ""  # layers with the same w_stream share W0 (the init sweep over r)
 
 
 def _llama8b_block(T: int, bits: int, group: int, r: int, dtype: str) -> list[LayerSpec]:
@@ -74,7 +75,7 @@ def _init_sweep() -> list[LayerSpec]:
             out.append(
                 LayerSpec(
                     f"{s.name}_r{r}", s.d_in, s.d_out, s.had_block, 0, 2, 64, s.p, "f32",
-                    remainder="largest",
+                    remainder="largest", w_stream=s.name,
                 )
             )
     return out
@@ -137,10 +138,11 @@ def bf16_bits_to_f32(b) -> np.ndarray:
 
 def _weights(spec: LayerSpec, seed: int, workload: str) -> np.ndarray:
     """W0 [d_out, d_in] as float32 values (bf16-representable for bf16 layers)."""
-    g = rng_for(seed, workload, spec.name, "W0")
+    key = spec.w_stream or spec.name
+    g = rng_for(seed, workload, key, "W0")
     w = g.standard_normal((spec.d_out, spec.d_in), dtype=np.float32) * np.float32(spec.w_std)
     if spec.w_outlier_frac > 0:
-        m = rng_for(seed, workload, spec.name, "W0_outliers").random((spec.d_out, spec.d_in)) < spec.w_outlier_frac
+        m = rng_for(seed, workload, key, "W0_outliers").random((spec.d_out, spec.d_in)) < spec.w_outlier_frac
         w[m] *= np.float32(spec.w_outlier_scale)
     if spec.dtype == "bf16":
         w = bf16_bits_to_f32(f32_to_bf16_bits(w))
