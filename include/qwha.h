@@ -77,7 +77,7 @@ typedef enum { QWHA_ALGO_SPARSE = 0, QWHA_ALGO_DENSE = 1 } qwha_algo;
 
 /* Edge of the square blocks of F into which the coefficient-gradient kernel
  * tiles the nonzeros (the tile view built by qwha_plan_build). */
-#define QWHA_TILE 512
+#define QWHA_TILE 256
 
 /* The sparse coefficient matrix F = Scatter(c, E) and its index views. All
  * arrays are device memory owned by the caller.

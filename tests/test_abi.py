@@ -5,7 +5,7 @@ import os
 import subprocess
 import sys
 
-from _util import ROOT, header_functions
+from _util import HEADER, ROOT, header_functions
 
 LIB = os.path.join(ROOT, "walsh_hadamard_sparse_b200", "libqwha.so")
 
@@ -46,4 +46,5 @@ def test_status_strings_and_host_checks():
     assert h.qwha_fwht(0, ctypes.c_void_p(8), ctypes.c_void_p(4096), 4, 256, 256, None) == 2  # misaligned
     assert h.qwha_fwht(7, None, None, 4, 256, 256, None) == 1  # bad dtype
     assert h.qwha_fwht(0, None, None, 0, 256, 256, None) == 0  # nothing to do
-    assert h.qwha_plan_tiles(4096, 14336) == 8 * 28
+    tile = int(next(l.split()[2] for l in open(HEADER) if l.startswith("#define QWHA_TILE")))
+    assert h.qwha_plan_tiles(4096, 14336) == -(-4096 // tile) * -(-14336 // tile)

@@ -18,6 +18,9 @@ from workloads import (
 
 pytestmark = pytest.mark.gpu
 
+# edge of the tile view's blocks (QWHA_TILE in include/qwha.h)
+TILE = int(next(l.split()[2] for l in open(__import__("_util").HEADER) if l.startswith("#define QWHA_TILE")))
+
 
 def _W():
     import walsh_hadamard_sparse_b200 as W
@@ -75,14 +78,15 @@ def dev_qweight(L):
 
 def expected_tiles(rp, ci, d_out, d_in):
     cp, ri, pm = oracle.plan_build(rp, ci, d_in)
-    n_rb = -(-d_out // 512)
-    n_kb = -(-d_in // 512)
+    E = TILE
+    n_rb = -(-d_out // E)
+    n_kb = -(-d_in // E)
     cols = np.repeat(np.arange(d_in), np.diff(cp))
-    tile = (cols // 512) * n_rb + ri // 512
+    tile = (cols // E) * n_rb + ri // E
     order = np.argsort(tile, kind="stable")
     tile_ptr = np.zeros(n_rb * n_kb + 1, dtype=np.int64)
     tile_ptr[1:] = np.cumsum(np.bincount(tile, minlength=n_rb * n_kb))
-    rk = ((ri % 512) << 16) | (cols % 512)
+    rk = ((ri % E) << 16) | (cols % E)
     return cp, ri, pm, tile_ptr, pm[order], rk[order]
 
 

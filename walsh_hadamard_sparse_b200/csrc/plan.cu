@@ -20,8 +20,8 @@ namespace qwha {
 namespace {
 
 constexpr int kChunkRows = 32;
-constexpr int kTileThreads = 128;
-constexpr int kMaxRowBlocks = 64;  // d_out <= 64 * QWHA_TILE
+constexpr int kTileThreads = 64;
+constexpr int kMaxRowBlocks = 128;  // d_out <= 128 * QWHA_TILE
 
 __global__ void chunk_hist_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
                                   int d_out, int d_in, int64_t p, int32_t *__restrict__ hist) {

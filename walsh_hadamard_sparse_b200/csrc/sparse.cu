@@ -14,13 +14,13 @@
 //   tile view of E (QWHA_TILE x QWHA_TILE blocks of F). Grid = tiles x token
 //   chunks; a CTA stages dY[:, row block] and Z[:, column block] for TT tokens
 //   at a time, transposed, with the next sub-tile's global loads issued into
-//   registers before the current one is consumed; each thread accumulates a
-//   run of consecutive tile entries (same column mostly: the Z vector is
-//   reloaded only when the column changes).
+//   registers before the current one is consumed (see sddmm_kernel for the
+//   lane layout).
 // sddmm_reduce: dc[j] = alpha * sum_c partial[c, j] in increasing c (fixed
 //   order: the result is bitwise reproducible).
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -29,7 +29,7 @@ namespace qwha {
 namespace {
 
 constexpr int kSpmmThreads = 512;
-constexpr size_t kSpmmSmemCap = 160 * 1024;
+constexpr size_t kSpmmSmemCap = 220 * 1024;
 
 template <typename T>
 __device__ __forceinline__ void load_vals(const T *p, float *o, int n);
@@ -67,6 +67,26 @@ __device__ __forceinline__ void load_vals<float>(const float *p, float *o, int n
   }
 }
 
+// d = a * b + c with a, b bf16 (the low or high half of a 32-bit word) and
+// c, d fp32: the product of two bf16 values is exact in fp32, so this is an
+// fp32 FMA on the widened operands without the widening instructions.
+__device__ __forceinline__ float fma_bf16_lo(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}"
+      : "=f"(d)
+      : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fma_bf16_hi(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}"
+      : "=f"(d)
+      : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+
 // Stage rows [t0, t0+TT) of in[T, W] into s[k * TT + t] (zeros past T).
 template <typename T, int TT>
 __device__ __forceinline__ void stage_transposed(const T *__restrict__ in, int64_t T_, int W, int64_t t0,
@@ -92,62 +112,164 @@ __device__ __forceinline__ void stage_transposed(const T *__restrict__ in, int64
   (void)W;
 }
 
-// One warp per segment at a time. A lane holds 4 consecutive tokens of the
-// tile (Q = TT/4 lanes cover the tile) for one of NSLOT = 32/Q nonzero slots:
-// lane = q + Q * slot. The slots walk the segment's nonzeros 8 or 16 at a time
-// (coalesced index/value loads, each nonzero's 4-token vector is one 8- or
-// 16-byte shared load); a shuffle tree over the slots ends the segment and the
-// Q lanes of slot 0 write its TT outputs.
+// One warp per segment at a time. A lane holds G = min(TT, 8) consecutive
+// tokens of the tile (Q = TT/G lanes cover it) for one of NSLOT = 32/Q nonzero
+// slots: lane = q + Q * slot. A segment is cut into blocks of NSLOT * kUnroll
+// nonzeros; slot s takes nonzeros base + s + NSLOT * u. Entries past the
+// segment end, or with a column outside the tile, get index 0 and value 0.
+// The next block's (index, value) loads go into the other register set while
+// the current block is multiplied (the two sets alternate roles: no copies).
+// bf16 tiles multiply with fma.rn.f32.bf16 (coefficient rounded to bf16, exact
+// product, fp32 accumulation). At a segment's end a reduce-scatter over the
+// slots leaves each token's sum in one lane, which writes it.
+constexpr int kUnroll = 8;
+
+// acc[i] += v * row[i] for the G tokens (4 or 8) a lane holds.
+template <int G>
+__device__ __forceinline__ void mac_tokens(const __nv_bfloat16 *row, float v, float *acc) {
+  const __nv_bfloat162 vb2 = __floats2bfloat162_rn(v, v);
+  const uint32_t vv = *reinterpret_cast<const uint32_t *>(&vb2);
+  uint32_t w[G / 2];
+  if constexpr (G == 8) {
+    const uint4 t = *reinterpret_cast<const uint4 *>(row);
+    w[0] = t.x, w[1] = t.y, w[2] = t.z, w[3] = t.w;
+  } else {
+    const uint2 t = *reinterpret_cast<const uint2 *>(row);
+    w[0] = t.x, w[1] = t.y;
+  }
+#pragma unroll
+  for (int i = 0; i < G / 2; ++i) {
+    acc[2 * i] = fma_bf16_lo(w[i], vv, acc[2 * i]);
+    acc[2 * i + 1] = fma_bf16_hi(w[i], vv, acc[2 * i + 1]);
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void mac_tokens(const float *row, float v, float *acc) {
+#pragma unroll
+  for (int h = 0; h < G / 4; ++h) {
+    const float4 a = *reinterpret_cast<const float4 *>(row + 4 * h);
+    acc[4 * h + 0] = fmaf(v, a.x, acc[4 * h + 0]);
+    acc[4 * h + 1] = fmaf(v, a.y, acc[4 * h + 1]);
+    acc[4 * h + 2] = fmaf(v, a.z, acc[4 * h + 2]);
+    acc[4 * h + 3] = fmaf(v, a.w, acc[4 * h + 3]);
+  }
+}
+
 template <typename Tin, typename Tout, int TT>
 __global__ void __launch_bounds__(kSpmmThreads)
     seg_spmm_kernel(const Tin *__restrict__ in, int64_t T, int W_in, const int32_t *__restrict__ seg_ptr,
-                    const int32_t *__restrict__ idx, const float *__restrict__ val, int64_t nnz, int n_seg,
+                    const int32_t *__restrict__ idx, const float *__restrict__ val, int64_t nnz64, int n_seg,
                     float alpha, Tout *__restrict__ out) {
-  constexpr int Q = TT / 4;        // lanes per nonzero (4 tokens each)
-  constexpr int NSLOT = 32 / Q;    // nonzeros in flight per warp
+  static_assert(TT == 4 || TT == 8 || TT == 16, "token tile");
+  constexpr int G = TT < 8 ? TT : 8;  // tokens per lane
+  constexpr int LV = G == 8 ? 3 : 2;  // reduce-scatter levels (log2 G)
+  constexpr int Q = TT / G;           // lanes per nonzero
+  constexpr int NSLOT = 32 / Q;    // slots per warp
+  constexpr int BLOCK = NSLOT * kUnroll;
+  constexpr int kWarps = kSpmmThreads / 32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Tin *s_in = reinterpret_cast<Tin *>(smem_raw);
+  int32_t *s_ptr = reinterpret_cast<int32_t *>(smem_raw + (size_t)W_in * TT * sizeof(Tin));
+  const int nnz = (int)nnz64;
   const int64_t t0 = (int64_t)blockIdx.x * TT;
+  for (int i = threadIdx.x; i <= n_seg; i += kSpmmThreads) {
+    const int v = seg_ptr[i];
+    s_ptr[i] = v < 0 ? 0 : (v > nnz ? nnz : v);
+  }
   stage_transposed<Tin, TT>(in, T, W_in, t0, 0, W_in, W_in, s_in);
   __syncthreads();
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int q = lane % Q, slot = lane / Q;
-  constexpr int kWarps = kSpmmThreads / 32;
-  for (int seg = warp; seg < n_seg; seg += kWarps) {
-    int64_t b = seg_ptr[seg], e = seg_ptr[seg + 1];
-    if (b < 0) b = 0;
-    if (e > nnz) e = nnz;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int64_t j = b + slot; j < e; j += NSLOT) {
-      const int k = __ldg(idx + j);
-      const float v = __ldg(val + j);
-      if ((unsigned)k < (unsigned)W_in) {
-        float x[4];
-        load_vals<Tin>(s_in + (int64_t)k * TT + 4 * q, x, 4);
+  const Tin *s_q = s_in + G * q;
+
+  int seg = warp, pos = 0, end = 0;
+  if (seg < n_seg) {
+    pos = s_ptr[seg];
+    end = s_ptr[seg + 1];
+  }
+  auto load_block = [&](int p0, int e, int *kk, float *vv) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] = fmaf(v, x[i], acc[i]);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int j = p0 + slot + NSLOT * u;
+      kk[u] = W_in;  // marks "no entry"
+      vv[u] = 0.f;
+      if (j < e) {
+        kk[u] = __ldg(idx + j);
+        vv[u] = __ldg(val + j);
       }
     }
+  };
+  int ka[kUnroll], kb[kUnroll];
+  float va[kUnroll], vb[kUnroll];
+  float acc[G];
 #pragma unroll
-    for (int off = Q; off < 32; off <<= 1)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-    if (slot == 0) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t t = t0 + 4 * q + i;
-        if (t < T) io<Tout>::store1(out + t * n_seg + seg, alpha * acc[i]);
+  for (int i = 0; i < G; ++i) acc[i] = 0.f;
+
+  auto step = [&](const int *kc, const float *vc, int *kn, float *vn) {
+    int nseg = seg, npos = pos + BLOCK, nend = end;
+    const bool last_of_seg = npos >= end;
+    if (last_of_seg) {
+      nseg = seg + kWarps;
+      if (nseg < n_seg) {
+        npos = s_ptr[nseg];
+        nend = s_ptr[nseg + 1];
       }
     }
+    if (nseg < n_seg) load_block(npos, nend, kn, vn);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const bool ok = (unsigned)kc[u] < (unsigned)W_in;
+      mac_tokens<G>(s_q + (ok ? kc[u] : 0) * TT, ok ? vc[u] : 0.f, acc);
+    }
+    if (last_of_seg) {
+      // reduce-scatter over the top LV slot bits of the lane (16, 8[, 4]):
+      // each level keeps half of the values and adds the partner's other half
+      float r[G];
+#pragma unroll
+      for (int i = 0; i < G; ++i) r[i] = acc[i];
+      int ti = 0;  // token (within the lane's G) that r[0] ends up holding
+#pragma unroll
+      for (int lvl = 0; lvl < LV; ++lvl) {
+        const int off = 16 >> lvl;
+        const int n = G >> (lvl + 1);
+        const bool upper = (lane & off) != 0;
+        if (upper) ti += n;
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+          const float keep = upper ? r[i + n] : r[i];
+          const float send = upper ? r[i] : r[i + n];
+          r[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      // the slot bits below those: a plain butterfly sum
+      constexpr int kLow = 32 >> LV;
+#pragma unroll
+      for (int off = Q; off < kLow; off <<= 1) r[0] += __shfl_xor_sync(0xffffffffu, r[0], off);
+      if ((lane & (kLow - 1) & ~(Q - 1)) == 0) {
+        const int64_t t = t0 + G * q + ti;
+        if (t < T) io<Tout>::store1(out + t * n_seg + seg, alpha * r[0]);
+      }
+#pragma unroll
+      for (int i = 0; i < G; ++i) acc[i] = 0.f;
+    }
+    seg = nseg;
+    pos = npos;
+    end = nend;
+  };
+  if (seg < n_seg) load_block(pos, end, ka, va);
+  while (seg < n_seg) {
+    step(ka, va, kb, vb);
+    if (seg >= n_seg) break;
+    step(kb, vb, ka, va);
   }
 }
 
 template <typename Tin, typename Tout, int TT>
 cudaError_t run_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
                      const float *val, int64_t nnz, int n_seg, float alpha, void *out, cudaStream_t s) {
-  const size_t smem = (size_t)W_in * TT * sizeof(Tin);
+  const size_t smem = (size_t)W_in * TT * sizeof(Tin) + ((size_t)n_seg + 1) * sizeof(int32_t);
   auto k = seg_spmm_kernel<Tin, Tout, TT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -161,11 +283,15 @@ template <typename Tin, typename Tout>
 cudaError_t pick_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
                       const float *val, int64_t nnz, int n_seg, float alpha, void *out, cudaStream_t s) {
   const size_t row = (size_t)W_in * sizeof(Tin);
-  if (row * 16 <= kSpmmSmemCap)
+  const size_t ptrs = ((size_t)n_seg + 1) * sizeof(int32_t);
+  const size_t cap = kSpmmSmemCap > ptrs ? kSpmmSmemCap - ptrs : 0;
+  if (row * 16 <= cap)
     return run_spmm<Tin, Tout, 16>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
-  if (row * 8 <= kSpmmSmemCap)
+  if (row * 8 <= cap)
     return run_spmm<Tin, Tout, 8>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
-  return run_spmm<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
+  if (row * 4 <= cap)
+    return run_spmm<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
+  return cudaErrorInvalidValue;  // rows too long for one staged token tile
 }
 
 __global__ void permute_kernel(const float *__restrict__ src, const int32_t *__restrict__ perm, int64_t p,
@@ -179,9 +305,10 @@ __global__ void permute_kernel(const float *__restrict__ src, const int32_t *__r
 // ---------------------------------------------------------------- SDDMM
 
 constexpr int kSddmmThreads = 512;
-constexpr int kSddmmEPT = 16;  // tile entries per thread per pass
+constexpr int kSddmmSlotEntries = 16;                                     // consecutive entries per slot
+constexpr int kSddmmPass = (kSddmmThreads / 32) * 8 * kSddmmSlotEntries;  // entries per CTA pass
 
-// tokens per staged sub-tile: 2 x QWHA_TILE x TT values = 64 KB
+// tokens per staged sub-tile (2 x QWHA_TILE x TT values = 32 KB); a lane covers TT/4 of them
 template <typename T>
 __host__ __device__ constexpr int sddmm_tt() {
   return sizeof(T) == 2 ? 32 : 16;
@@ -192,19 +319,18 @@ __host__ __device__ constexpr int sddmm_tt() {
 // the current sub-tile's arithmetic.
 template <typename T, int TT>
 struct SubTile {
-  static constexpr int V = 16 / (int)sizeof(T);                       // values per vector
-  static constexpr int ITEMS = 2 * (QWHA_TILE / V) * TT / kSddmmThreads;  // vectors per thread
+  static constexpr int V = 16 / (int)sizeof(T);                           // values per vector
+  static constexpr int HALF = (QWHA_TILE / V) * TT;                        // vectors per operand
+  static constexpr int ITEMS = 2 * HALF / kSddmmThreads;                   // vectors per thread
   uint4 v[ITEMS];
 
-  // item it -> (operand, token, vector c along the row/column block)
   __device__ __forceinline__ void load(const T *dY, const T *Z, int64_t tb, int d_out, int d_in, int64_t t0, int r0,
                                        int r_len, int k0, int k_len) {
 #pragma unroll
     for (int u = 0; u < ITEMS; ++u) {
       const int it = threadIdx.x + u * kSddmmThreads;
-      const int half = (QWHA_TILE / V) * TT;
-      const int which = it >= half;
-      const int w = it - which * half;
+      const int which = it >= HALF;
+      const int w = it - which * HALF;
       const int t = w % TT, c = w / TT;
       const int64_t tg = t0 + t;
       const int len = which ? k_len : r_len;
@@ -219,9 +345,8 @@ struct SubTile {
 #pragma unroll
     for (int u = 0; u < ITEMS; ++u) {
       const int it = threadIdx.x + u * kSddmmThreads;
-      const int half = (QWHA_TILE / V) * TT;
-      const int which = it >= half;
-      const int w = it - which * half;
+      const int which = it >= HALF;
+      const int w = it - which * HALF;
       const int t = w % TT, c = w / TT;
       float f[V];
       io<T>::unpack(v[u], f);
@@ -232,6 +357,13 @@ struct SubTile {
   }
 };
 
+// One CTA per (QWHA_TILE x QWHA_TILE tile of F, token chunk). Lanes are
+// (slot, q): q picks TT/4 tokens of a staged row, slot one of 8 entries in
+// flight; slot s of warp w owns 16 consecutive tile entries (CSC order inside
+// the tile: mostly one column, whose Z vector is reloaded only when it
+// changes). Per entry and sub-tile a lane does one 16-byte shared load of dY
+// and TT/4 FMAs; at the end of the chunk the 4 q lanes of an entry are summed
+// by shuffles and written to the chunk's partial sums.
 template <typename T>
 __global__ void __launch_bounds__(kSddmmThreads)
     sddmm_kernel(const T *__restrict__ dY, const T *__restrict__ Z, int64_t T_, int d_out, int d_in,
@@ -239,9 +371,9 @@ __global__ void __launch_bounds__(kSddmmThreads)
                  const int32_t *__restrict__ tile_rk, int n_rb, int64_t chunk_tokens, int64_t p,
                  float *__restrict__ partial) {
   constexpr int TT = sddmm_tt<T>();
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  T *s_dy = reinterpret_cast<T *>(smem_raw);
-  T *s_z = s_dy + QWHA_TILE * TT;
+  constexpr int G = TT / 4;  // tokens per lane
+  __shared__ __align__(16) T s_dy[QWHA_TILE * TT];
+  __shared__ __align__(16) T s_z[QWHA_TILE * TT];
   const int tile = blockIdx.x;
   const int rb = tile % n_rb, kb = tile / n_rb;
   const int r0 = rb * QWHA_TILE, k0 = kb * QWHA_TILE;
@@ -252,19 +384,20 @@ __global__ void __launch_bounds__(kSddmmThreads)
   const int64_t c = blockIdx.y;
   const int64_t ta = c * chunk_tokens, tb = (ta + chunk_tokens < T_) ? ta + chunk_tokens : T_;
   float *part = partial + c * p;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = lane & 3, slot = lane >> 2;
 
-  for (int64_t eb = e_begin; eb < e_end; eb += (int64_t)kSddmmThreads * kSddmmEPT) {
-    const int64_t my0 = eb + (int64_t)threadIdx.x * kSddmmEPT;
-    const int64_t left = e_end - my0;
-    const int n_mine = left <= 0 ? 0 : (left < kSddmmEPT ? (int)left : kSddmmEPT);
-    int rk[kSddmmEPT];  // (row << 16 | column) inside the tile, -1 when unused
-    float acc[kSddmmEPT];
+  for (int64_t eb = e_begin; eb < e_end; eb += kSddmmPass) {
+    const int64_t my0 = eb + (int64_t)(warp * 8 + slot) * kSddmmSlotEntries;
+    int rk[kSddmmSlotEntries];  // (row << 16 | column) inside the tile, -1 when unused
+    float acc[kSddmmSlotEntries];
 #pragma unroll
-    for (int q = 0; q < kSddmmEPT; ++q) {
-      const int v = q < n_mine ? tile_rk[my0 + q] : -1;
+    for (int i = 0; i < kSddmmSlotEntries; ++i) {
+      const int64_t e = my0 + i;
+      const int v = e < e_end ? tile_rk[e] : -1;
       const int r_ = (v >> 16) & 0xffff, k_ = v & 0xffff;
-      rk[q] = (q < n_mine && r_ < r_len && k_ < k_len) ? v : -1;
-      acc[q] = 0.f;
+      rk[i] = (e < e_end && r_ < r_len && k_ < k_len) ? v : -1;
+      acc[i] = 0.f;
     }
     SubTile<T, TT> nxt;
     if (ta < tb) nxt.load(dY, Z, tb, d_out, d_in, ta, r0, r_len, k0, k_len);
@@ -273,34 +406,65 @@ __global__ void __launch_bounds__(kSddmmThreads)
       nxt.store(s_dy, s_z);
       __syncthreads();
       if (t0 + TT < tb) nxt.load(dY, Z, tb, d_out, d_in, t0 + TT, r0, r_len, k0, k_len);
-      int cur_k = -2;
-      float zv[TT];
+      int cur_k = -1;
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        static_assert(G == 8, "one 16-byte row slice per lane");
+        uint4 zr = make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int q = 0; q < kSddmmEPT; ++q) {
-        if (rk[q] < 0) continue;
-        const int kq = rk[q] & 0xffff, rq = rk[q] >> 16;
-        if (kq != cur_k) {
-#pragma unroll
-          for (int u = 0; u < TT; u += 8) load_vals<T>(s_z + kq * TT + u, zv + u, 8);
-          cur_k = kq;
+        for (int i = 0; i < kSddmmSlotEntries; ++i) {
+          if (rk[i] < 0) continue;
+          const int kq = rk[i] & 0xffff, rq = rk[i] >> 16;
+          if (kq != cur_k) {
+            zr = *reinterpret_cast<const uint4 *>(s_z + kq * TT + G * q);
+            cur_k = kq;
+          }
+          const uint4 yr = *reinterpret_cast<const uint4 *>(s_dy + rq * TT + G * q);
+          // bf16 x bf16 products are exact in fp32: no widening needed
+          float a0 = fma_bf16_lo(yr.x, zr.x, 0.f);
+          float a1 = fma_bf16_hi(yr.x, zr.x, 0.f);
+          a0 = fma_bf16_lo(yr.y, zr.y, a0);
+          a1 = fma_bf16_hi(yr.y, zr.y, a1);
+          a0 = fma_bf16_lo(yr.z, zr.z, a0);
+          a1 = fma_bf16_hi(yr.z, zr.z, a1);
+          a0 = fma_bf16_lo(yr.w, zr.w, a0);
+          a1 = fma_bf16_hi(yr.w, zr.w, a1);
+          acc[i] += a0 + a1;
         }
-        float a = acc[q];
+      } else {
+        float zv[G];
 #pragma unroll
-        for (int u = 0; u < TT; u += 8) {
-          float yv[8];
-          load_vals<T>(s_dy + rq * TT + u, yv, 8);
+        for (int i = 0; i < kSddmmSlotEntries; ++i) {
+          if (rk[i] < 0) continue;
+          const int kq = rk[i] & 0xffff, rq = rk[i] >> 16;
+          if (kq != cur_k) {
+            load_vals<T>(s_z + kq * TT + G * q, zv, G);
+            cur_k = kq;
+          }
+          float yv[G];
+          load_vals<T>(s_dy + rq * TT + G * q, yv, G);
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) a = fmaf(yv[i], zv[u + i], a);
+          for (int u = 0; u < G; u += 2) {
+            a0 = fmaf(yv[u], zv[u], a0);
+            a1 = fmaf(yv[u + 1], zv[u + 1], a1);
+          }
+          acc[i] += a0 + a1;
         }
-        acc[q] = a;
       }
     }
 #pragma unroll
-    for (int q = 0; q < kSddmmEPT; ++q)
-      if (q < n_mine) {
-        const int j = tile_pos[my0 + q];
-        if ((uint64_t)j < (uint64_t)p) part[j] = acc[q];
-      }
+    for (int i = 0; i < kSddmmSlotEntries; ++i) {
+      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 1);
+      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
+    }
+    if (q == 0) {
+#pragma unroll
+      for (int i = 0; i < kSddmmSlotEntries; ++i)
+        if (rk[i] >= 0) {
+          const int j = tile_pos[my0 + i];
+          if ((uint64_t)j < (uint64_t)p) part[j] = acc[i];
+        }
+    }
     __syncthreads();
   }
 }
@@ -358,21 +522,14 @@ cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T
   if (e != cudaSuccess) return e;
   if (T > 0) {
     dim3 grid((unsigned)tiles, (unsigned)n_chunks);
-    const size_t smem = 64 * 1024;
-    if (dt == QWHA_BF16) {
-      auto k = sddmm_kernel<__nv_bfloat16>;
-      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      k<<<grid, kSddmmThreads, smem, s>>>(static_cast<const __nv_bfloat16 *>(dY),
-                                          static_cast<const __nv_bfloat16 *>(Z), T, d_out, d_in, tile_ptr, tile_pos,
-                                          tile_rk, n_rb, chunk_tokens, p, partial);
-    } else {
-      auto k = sddmm_kernel<float>;
-      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      k<<<grid, kSddmmThreads, smem, s>>>(static_cast<const float *>(dY), static_cast<const float *>(Z), T, d_out,
-                                          d_in, tile_ptr, tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
-    }
+    if (dt == QWHA_BF16)
+      sddmm_kernel<__nv_bfloat16><<<grid, kSddmmThreads, 0, s>>>(
+          static_cast<const __nv_bfloat16 *>(dY), static_cast<const __nv_bfloat16 *>(Z), T, d_out, d_in, tile_ptr,
+          tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
+    else
+      sddmm_kernel<float><<<grid, kSddmmThreads, 0, s>>>(static_cast<const float *>(dY),
+                                                         static_cast<const float *>(Z), T, d_out, d_in, tile_ptr,
+                                                         tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
