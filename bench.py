@@ -65,24 +65,27 @@ def source_sha(files):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(stage):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's source is unchanged since."""
+def ncu_traffic(path_name, stage):
+    """DRAM bytes (read + write) per launch of `stage` on the `path_name` path ("dense" or "sparse"), from the
+    committed ncu summary, if the kernel's sources are unchanged since it was taken; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
-    d = json.load(open(path)).get(stage)
+    d = json.load(open(path)).get(path_name, {}).get(stage)
     if not d or d.get("source_sha") != source_sha(KERNEL_SOURCES.get(stage, [])):
         return None
-    return d.get("dram_bytes_per_launch_full_size")
+    return d.get("dram_bytes_per_launch")
 
 
 # --------------------------------------------------------------------------- work per stage
 
 
-def stage_work(stage, spec, T, bits):
-    """(bound, algorithmic work per stage call, HBM bytes per stage call) for the layer of `spec` at T tokens.
-    bound is hbm (work = bytes), tensor or alu (work = FLOP); None for stages without a model."""
+def stage_work(stage, spec, T, bits, algo="dense"):
+    """(bound, algorithmic work per stage call, HBM bytes per stage call) for the layer of `spec` at T tokens on
+    the `algo` path. bound is hbm (work = bytes), tensor or alu (work = FLOP); None for stages without a model."""
     di, do, p = spec.d_in, spec.d_out, spec.p
+    # the sparse path's GEMMs also read the fp32 adapter term in their epilogue
+    addend = (4.0 * T * do if stage == "gemm_fwd" else 4.0 * T * di) if algo == "sparse" else 0.0
     qbytes = do * di * bits / 8 + (do * di / spec.group) * 5
     w = {
         # forward transform: read X, write Z (bf16)
@@ -94,8 +97,8 @@ def stage_work(stage, spec, T, bits):
         "spmm_fwd": ("alu", 2.0 * p * T, 2.0 * T * di + 4.0 * T * do + 8.0 * p),
         "gather_bwd": ("alu", 2.0 * p * T, 2.0 * T * do + 4.0 * T * di + 12.0 * p),
         "sddmm_dc": ("alu", 2.0 * p * T, 2.0 * T * (di + do) + 8.0 * p),
-        "gemm_fwd": ("tensor", 2.0 * T * di * do, 2.0 * T * di + 2.0 * do * di + 2.0 * T * do),
-        "gemm_bwd": ("tensor", 2.0 * T * di * do, 2.0 * T * do + 2.0 * do * di + 2.0 * T * di),
+        "gemm_fwd": ("tensor", 2.0 * T * di * do, 2.0 * T * di + 2.0 * do * di + 2.0 * T * do + addend),
+        "gemm_bwd": ("tensor", 2.0 * T * di * do, 2.0 * T * do + 2.0 * do * di + 2.0 * T * di + addend),
         "gemm_dc": ("tensor", 2.0 * T * di * do, 2.0 * T * (di + do) + 12.0 * p),
         # W_eff = W_Q + alpha F H: codes + CSR in, bf16 out
         "weff": ("hbm", qbytes + 8.0 * p + 2.0 * do * di, qbytes + 8.0 * p + 2.0 * do * di),
@@ -354,32 +357,32 @@ def main():
             t_ms = float(tt.item())
         return t_ms, rep, clk
 
-    def kernel_table(rep, K):
+    def kernel_table(rep, K, algo):
         kernels = {}
         for name, (calls, launches, ms) in rep.items():
             if calls == 0:
                 continue
             per = ms / calls
             k = {"calls": calls, "launches": launches, "ms_per_call": per}
-            wk = stage_work(name, spec, T, spec.bits)
+            wk = stage_work(name, spec, T, spec.bits, algo)
             if wk:
                 kind, amount, nbytes = wk
                 peak, unit, _ = peak_for(kind, peaks)
                 ach = amount / (per / 1e3) / (1e9 if unit == "GB/s" else 1e12)
                 k.update(bound=kind, achieved=ach, peak=peak, unit=unit, frac=ach / peak,
-                         alg_GBps=nbytes / (per / 1e3) / 1e9)
+                         alg_GBps=nbytes / (per / 1e3) / 1e9, alg_bytes=nbytes, traffic=ncu_traffic(algo, name))
             kernels[name] = k
         tot = sum(v["ms_per_call"] * v["calls"] for v in kernels.values())
         for v in kernels.values():
             v["share"] = v["ms_per_call"] * v["calls"] / tot
         return kernels
 
-    def roofline_of(kernels):
+    def roofline_of(kernels, algo):
         dom = max((n for n in kernels if "bound" in kernels[n]), key=lambda n: kernels[n]["share"])
         kd = kernels[dom]
         _, _, note = peak_for(kd["bound"], peaks)
         return {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
-                "unit": kd["unit"], "frac": kd["frac"], "traffic": ncu_traffic(dom), "peak_source": note}
+                "unit": kd["unit"], "frac": kd["frac"], "traffic": ncu_traffic(algo, dom), "peak_source": note}
 
     results = {}
     for algo in ("dense", "sparse"):
@@ -391,9 +394,9 @@ def main():
             raise RuntimeError(f"non-finite output ({algo})")
         K = args.steps if algo == "dense" else max(3, min(args.steps, args.sparse_steps))
         t_ms, rep, clk = timed(step, K, algo == "dense")
-        kernels = kernel_table(rep, K)
+        kernels = kernel_table(rep, K, algo)
         results[algo] = dict(K=K, t_ms=t_ms, value=world * T * K / (t_ms / 1e3), kernels=kernels,
-                             roofline=roofline_of(kernels), launches=sum(v[1] for v in rep.values()), clocks=clk)
+                             roofline=roofline_of(kernels, algo), launches=sum(v[1] for v in rep.values()), clocks=clk)
     head = results["dense"]
     K, t_ms, value, kernels, clk = head["K"], head["t_ms"], head["value"], head["kernels"], head["clocks"]
     roofline, launches = head["roofline"], head["launches"]
