@@ -5,16 +5,16 @@
 //   backward: dX = dY W_Q + dX_adapter   (A = dY, B = W_Q read MN-major, K = d_out)
 // The adapter term rides in the epilogue, so it costs one fp32 read.
 //
-// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
+// Structure (persistent; one CTA per SM, or one CTA pair per two SMs):
 //   warp 0, one thread : TMA producer. 2-D tensor copies (128B swizzle, no
-//                        multicast) of A and B k-blocks of 64 into a 4-stage
-//                        shared-memory ring, completion counted in bytes on
-//                        the stage's "full" mbarrier. An operand may be K-major
+//                        multicast) of A and B k-blocks of 64 into a shared-
+//                        memory ring, completion counted in bytes on the
+//                        stage's "full" mbarrier. An operand may be K-major
 //                        (one box of rows x 64 K) or MN-major (64 x 64 boxes
 //                        along MN); the UMMA descriptors and the instruction
 //                        descriptor's major bits follow.
 //   warp 1, one thread : MMA issuer. tcgen05.mma kind::f16 (bf16 x bf16 ->
-//                        fp32) M=128 N=256 K=16, accumulator in TMEM;
+//                        fp32), K=16 per instruction, accumulator in TMEM;
 //                        tcgen05.commit frees the stage ("empty") and, after
 //                        the tile's last k-block, publishes the accumulator.
 //                        Warp 1 also owns the TMEM allocation (512 columns:
@@ -23,6 +23,18 @@
 //   warps 2..5         : epilogue. tcgen05.ld 32 lanes x 32 columns at a
 //                        time (warp w reads TMEM lanes 32*(w%4)..+31), add
 //                        the fp32 addend (if any), store bf16 or fp32.
+// Two variants of the same kernel:
+//   CG = 1: one CTA computes a 128 x 256 tile (M = 128 MMA), 48 KB per stage,
+//           4 stages.
+//   CG = 2: a cluster of two CTAs on two SMs computes a 256 x 256 tile with
+//           cta_group::2 MMAs (M = 256) issued by the even CTA. Each CTA loads
+//           its own 128 rows of A and its own 128 rows (half) of B, 32 KB per
+//           stage, 6 stages; both CTAs' copies complete on the even CTA's
+//           "full" barrier, the MMA commits arrive on the barriers of both
+//           CTAs (stage free, accumulator ready), and the odd CTA's epilogue
+//           reports a drained accumulator on the even CTA's barrier. Every SM
+//           then streams 2/3 of the operand bytes of the CG = 1 tile for the
+//           same MMA work.
 // Every mbarrier wait is bounded by time: on expiry the thread records a code
 // in the library's device error word, the CTA stops issuing work, drains what
 // it issued, frees TMEM and exits.
@@ -37,15 +49,26 @@
 namespace qwha {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;  // accumulator rows per CTA, tile columns, k-block
 constexpr int kGemmThreads = 192;
-constexpr uint32_t A_BYTES = BM * BK * 2;
-constexpr uint32_t B_BYTES = BN * BK * 2;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int kEpiStride = 33;  // per-warp staging row (floats) of the sampled epilogue
 constexpr size_t kEpiSmem = 4 * 32 * kEpiStride * sizeof(float);
-constexpr size_t kGemmSmem = (size_t)STAGES * STAGE_BYTES + 1024 + 256 + kEpiSmem;
+
+template <int CG>
+struct Cfg {
+  static constexpr int kStages = CG == 1 ? 4 : 6;
+  static constexpr uint32_t kABytes = BM * BK * 2;
+  static constexpr int kBRows = BN / CG;  // rows of B this CTA loads
+  static constexpr uint32_t kBBytes = kBRows * BK * 2;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256 + kEpiSmem;
+  // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
+  // B bf16 (10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
+  // M >> 4 at bit 24 (M = 128 per CTA of the group).
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                     ((uint32_t)((BM * CG) >> 4) << 24);
+};
 
 enum { kOutBf16 = 0, kOutF32 = 1, kOutSampled = 2 };
 
@@ -58,12 +81,6 @@ struct SampleArgs {
   int64_t p;
 };
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
-
-// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
-// B bf16 (10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
-// M >> 4 at bit 24.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -111,12 +128,47 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// 2-D tensor copy into this CTA's shared memory. With CG = 2 the completion
+// may be counted on the mbarrier of the other CTA of the pair (bar is then a
+// shared::cluster address). No multicast.
+template <int CG>
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
+  if constexpr (CG == 1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// All threads of both CTAs of the cluster (the non-.aligned form: lanes of a
+// warp may arrive at different times).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -134,18 +186,71 @@ __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+template <int CG>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
+  if constexpr (CG == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+  }
 }
 
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+// Arrive on `bar` (same offset) in every CTA of the group once the MMAs issued
+// so far have completed.
+template <int CG>
+__device__ __forceinline__ void umma_commit_all(uint32_t bar) {
+  if constexpr (CG == 1) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+  } else {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                     "r"(bar),
+                 "h"((unsigned short)3)
+                 : "memory");
+  }
+}
+
+// Arrive on this CTA's `bar` once the MMAs issued so far have completed.
+template <int CG>
+__device__ __forceinline__ void umma_commit_local(uint32_t bar) {
+  if constexpr (CG == 1) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+  } else {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+  }
+}
+
+template <int CG>
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols) {
+  if constexpr (CG == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+}
+
+template <int CG>
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  if constexpr (CG == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -168,17 +273,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
 // contiguous]); its stage is then filled by BM/64 or BN/64 boxes of 64 x 64.
 // k_splits > 1 (sampled output only): each tile's K range is cut into that
 // many parts, each part a separate work unit adding its share into dc.
-template <int kMode>
+template <int kMode, int CG>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const float *__restrict__ addend, void *__restrict__ out_v, int M, int N, int K,
                              int a_mn, int b_mn, int group_m, int k_splits, SampleArgs sa_args, unsigned int *err) {
+  using C = Cfg<CG>;
+  constexpr int STAGES = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t base = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
   uint8_t *smem = smem_raw + pad;
   base += pad;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -187,9 +294,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  float *epi_stage = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256);
+  float *epi_stage = reinterpret_cast<float *>(smem + STAGES * C::kStageBytes + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;  // position in the CTA pair
+  const bool leader = rank == 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full(s), 1);
@@ -197,29 +306,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull(b), 1);
-      mbar_init(tempty(b), 4);
+      mbar_init(tempty(b), 4 * CG);  // the epilogue warps of every CTA of the group
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 1) tmem_alloc<CG>(smem_u32(tmem_slot), TMEM_COLS);
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync();  // the peer's barriers and TMEM exist before any copy or MMA
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int m_tiles = (M + BM - 1) / BM, n_tiles = (N + BN - 1) / BN;
+  constexpr int TM = BM * CG;  // tile rows
+  const int m_tiles = (M + TM - 1) / TM, n_tiles = (N + BN - 1) / BN;
   const int k_blocks = (K + BK - 1) / BK;
   const int kb_per_split = (k_blocks + k_splits - 1) / k_splits;
   const int num_tiles = m_tiles * n_tiles;
   const int num_units = num_tiles * k_splits;
+  const int group_id = blockIdx.x / CG, n_groups = gridDim.x / CG;
   // Tile order: groups of group_m row blocks; inside a group, the row block
   // changes fastest and the column block slowest, so the tiles in flight share
   // a few row blocks of A and a run of column blocks of B in L2.
@@ -237,15 +345,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   };
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA producer (every CTA)
     int stage = 0;
     uint32_t phase = 0;
     int last_parity[STAGES];
     for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
-    for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x) {
+    for (int unit = group_id; unit < num_units && !*abort_flag; unit += n_groups) {
       const int tile = unit / k_splits, split = unit % k_splits;
       int m_blk, n_blk;
       tile_coords(tile, m_blk, n_blk);
+      const int a_row = m_blk * TM + (int)rank * BM;
+      const int b_row = n_blk * BN + (int)rank * C::kBRows;
       const int kb0 = split * kb_per_split, kb1 = min(k_blocks, kb0 + kb_per_split);
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(empty(stage), phase ^ 1)) {
@@ -253,19 +363,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         if (*abort_flag) break;
-        mbar_expect_tx(full(stage), STAGE_BYTES);
-        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+        // both CTAs' bytes complete on the leader's barrier; only the leader arrives
+        if (leader) mbar_expect_tx(full(stage), C::kStageBytes * CG);
+        const uint32_t fb = CG == 2 ? peer_addr(full(stage), 0) : full(stage);
+        const uint32_t sa = base + stage * C::kStageBytes, sb = sa + C::kABytes;
         if (a_mn) {
 #pragma unroll
-          for (int h = 0; h < BM / 64; ++h) tma_load_2d(sa + h * 8192, &tmA, full(stage), m_blk * BM + 64 * h, kb * BK);
+          for (int h = 0; h < BM / 64; ++h) tma_load_2d<CG>(sa + h * 8192, &tmA, fb, a_row + 64 * h, kb * BK);
         } else {
-          tma_load_2d(sa, &tmA, full(stage), kb * BK, m_blk * BM);
+          tma_load_2d<CG>(sa, &tmA, fb, kb * BK, a_row);
         }
         if (b_mn) {
 #pragma unroll
-          for (int h = 0; h < BN / 64; ++h) tma_load_2d(sb + h * 8192, &tmB, full(stage), n_blk * BN + 64 * h, kb * BK);
+          for (int h = 0; h < C::kBRows / 64; ++h) tma_load_2d<CG>(sb + h * 8192, &tmB, fb, b_row + 64 * h, kb * BK);
         } else {
-          tma_load_2d(sb, &tmB, full(stage), kb * BK, n_blk * BN);
+          tma_load_2d<CG>(sb, &tmB, fb, kb * BK, b_row);
         }
         last_parity[stage] = (int)phase;
         if (++stage == STAGES) {
@@ -274,15 +386,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     }
-    // drain: every copy this thread issued has landed before the CTA exits
-    for (int s = 0; s < STAGES; ++s)
-      if (last_parity[s] >= 0 && !mbar_wait(full(s), (uint32_t)last_parity[s])) give_up(0x2u);
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------ MMA issuer
+    // drain: every copy of the group has landed before the CTAs exit (the
+    // leader's barriers count the copies of both CTAs of a pair)
+    if (leader)
+      for (int s = 0; s < STAGES; ++s)
+        if (last_parity[s] >= 0 && !mbar_wait(full(s), (uint32_t)last_parity[s])) give_up(0x2u);
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ------------------------------------------------ MMA issuer (leader CTA)
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
-    for (int unit = blockIdx.x; unit < num_units && !*abort_flag; unit += gridDim.x, ++it) {
+    for (int unit = group_id; unit < num_units && !*abort_flag; unit += n_groups, ++it) {
       const int split = unit % k_splits;
       const int kb0 = split * kb_per_split, kb1 = min(k_blocks, kb0 + kb_per_split);
       const int buf = it & 1;
@@ -301,33 +415,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+        const uint32_t sa = base + stage * C::kStageBytes, sb = sa + C::kABytes;
         const uint64_t da = a_mn ? sw128_desc_mn(sa) : sw128_desc(sa);
         const uint64_t db = b_mn ? sw128_desc_mn(sb) : sw128_desc(sb);
         // next 16 of K: +32 B inside the 128 B rows (K-major), +2 KB = 16 rows (MN-major)
         const uint64_t sta = a_mn ? 128ull : 2ull, stb = b_mn ? 128ull : 2ull;
-        const uint32_t idesc = kIdesc | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
+        const uint32_t idesc = C::kIdesc | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
-          umma_bf16(d_tmem, da + sta * k, db + stb * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-        umma_commit(empty(stage));
+          umma_bf16<CG>(d_tmem, da + sta * k, db + stb * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+        umma_commit_all<CG>(empty(stage));
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (!ok) break;
-      umma_commit(tfull(buf));
+      umma_commit_all<CG>(tfull(buf));
     }
     // drain: all issued MMAs complete before TMEM is released
-    umma_commit(done_bar);
+    umma_commit_local<CG>(done_bar);
     if (!mbar_wait(done_bar, 0)) give_up(0x10u);
   } else if (warp >= 2) {
-    // ------------------------------------------------ epilogue
+    // ------------------------------------------------ epilogue (every CTA)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int it = 0;
     float *my_stage = epi_stage + (warp - 2) * 32 * kEpiStride;
-    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++it) {
+    for (int unit = group_id; unit < num_units; unit += n_groups, ++it) {
       const int tile = unit / k_splits;
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
@@ -339,7 +453,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       int m_blk, n_blk;
       tile_coords(tile, m_blk, n_blk);
-      const int row = m_blk * BM + q * 32 + lane;
+      const int row = m_blk * TM + (int)rank * BM + q * 32 + lane;
       // sampled output: this row's CSR entries with column in [n0, n0 + BN)
       int64_t j = 0, j_end = 0;
       if (kMode == kOutSampled && row < M) {
@@ -419,15 +533,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty(buf));
+      if (lane == 0) {
+        // the accumulator half in this CTA's TMEM is drained: tell the MMA issuer
+        if constexpr (CG == 2) mbar_arrive_remote(peer_addr(tempty(buf), 0));
+        else mbar_arrive(tempty(buf));
+      }
     }
   }
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  // no CTA of a pair leaves (or frees TMEM) while the other may still signal
+  // its barriers or the leader's MMAs may still use its memory
+  if constexpr (CG == 2) cluster_sync();
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
-                 : "memory");
+    tmem_dealloc<CG>(tmem_base, TMEM_COLS);
   }
 }
 
@@ -460,23 +581,51 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, uint3
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Co-resident CTA groups of the CG variant (one CTA per SM; pairs need two SMs
+// of one cluster slot).
+template <int kMode, int CG>
+int resident_groups() {
+  static int n = 0;
+  if (n) return n;
+  const int sms = sm_count();
+  if (CG == 1) return n = sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(sms - sms % CG));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = Cfg<CG>::kSmem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CG;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_bf16_tcgen05_kernel<kMode, CG>, &cfg) != cudaSuccess ||
+      clusters < 1) {
+    (void)cudaGetLastError();
+    clusters = sms / CG;
+  }
+  return n = clusters;
+}
+
 // A is [M, K] (K-major) or, with a_mn, [K, M]; B is [N, K] or, with b_mn, [K, N].
-template <int kMode>
-cudaError_t launch_gemm_t(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
-                          int64_t K, bool a_mn, bool b_mn, const SampleArgs &sa, cudaStream_t s) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
+template <int kMode, int CG>
+cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
+                           int64_t K, bool a_mn, bool b_mn, const SampleArgs &sa, cudaStream_t s) {
+  using C = Cfg<CG>;
   CUtensorMap ta, tb;
   const bool ok_a = a_mn ? make_map(&ta, A, K, M, 64) : make_map(&ta, A, M, K, BM);
-  const bool ok_b = b_mn ? make_map(&tb, B, K, N, 64) : make_map(&tb, B, N, K, BN);
+  const bool ok_b = b_mn ? make_map(&tb, B, K, N, 64) : make_map(&tb, B, N, K, C::kBRows);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+  auto kern = gemm_bf16_tcgen05_kernel<kMode, CG>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05_kernel<kMode>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int64_t m_tiles = cdiv(M, BM), n_tiles = cdiv(N, BN);
+  const int64_t m_tiles = cdiv(M, (int64_t)BM * CG), n_tiles = cdiv(N, BN);
   const int64_t tiles = m_tiles * n_tiles;
   // Rows of A per group: all column blocks of B for one row block at a time
   // when B fits comfortably in L2 (it is then read from DRAM once); otherwise
@@ -484,16 +633,16 @@ cudaError_t launch_gemm_t(const void *A, const void *B, const float *addend, voi
   const int64_t b_bytes = N * K * 2;
   int64_t group_m = 1;
   if (b_bytes > (48ll << 20)) {
-    group_m = 8;
+    group_m = 8 / CG;
     if (group_m > m_tiles) group_m = m_tiles;
   }
+  const int groups = resident_groups<kMode, CG>();
   // Sampled output: split K in two when the tiles alone would leave the last
-  // wave of SMs mostly idle (each dc then receives exactly two additions onto
-  // zero, whose result does not depend on their order).
+  // wave of groups mostly idle (each dc then receives exactly two additions
+  // onto zero, whose result does not depend on their order).
   int k_splits = 1;
-  const int sms = sm_count();
   if (kMode == kOutSampled && cdiv(K, BK) >= 8) {
-    const double waves1 = (double)tiles / sms, waves2 = 2.0 * tiles / sms;
+    const double waves1 = (double)tiles / groups, waves2 = 2.0 * tiles / groups;
     const double eff1 = waves1 / std::ceil(waves1), eff2 = waves2 / std::ceil(waves2);
     if (eff2 > eff1 + 0.02) k_splits = 2;
   }
@@ -502,11 +651,30 @@ cudaError_t launch_gemm_t(const void *A, const void *B, const float *addend, voi
     if (e != cudaSuccess) return e;
   }
   const int64_t units = tiles * k_splits;
-  const int grid = (int)(units < sms ? units : sms);
-  gemm_bf16_tcgen05_kernel<kMode><<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, addend, out, (int)M, (int)N, (int)K,
-                                                                       a_mn ? 1 : 0, b_mn ? 1 : 0, (int)group_m,
-                                                                       k_splits, sa, device_error_word());
-  return cudaGetLastError();
+  const int64_t n_launch = units < groups ? units : groups;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(n_launch * CG));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CG;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = CG > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, addend, out, (int)M, (int)N, (int)K, a_mn ? 1 : 0, b_mn ? 1 : 0,
+                            (int)group_m, k_splits, sa, device_error_word());
+}
+
+// The pair variant once there are at least two 128-row blocks of output.
+template <int kMode>
+cudaError_t launch_gemm_t(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
+                          int64_t K, bool a_mn, bool b_mn, const SampleArgs &sa, cudaStream_t s) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  if (M > BM) return launch_gemm_cg<kMode, 2>(A, B, addend, out, M, N, K, a_mn, b_mn, sa, s);
+  return launch_gemm_cg<kMode, 1>(A, B, addend, out, M, N, K, a_mn, b_mn, sa, s);
 }
 
 cudaError_t launch_gemm(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
