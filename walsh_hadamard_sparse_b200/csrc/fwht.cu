@@ -127,6 +127,10 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
 }
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gmem_src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
@@ -359,12 +363,216 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Same result as weff_rows_kernel, software-pipelined: while the butterflies of
+// the current row blocks run, cp.async copies the next row blocks' inputs into
+// shared memory: their CSR slice (column, coefficient; up to kWeffCsrCap
+// entries per row, the rest is read directly) and their block of base-weight
+// codes, scales and zero points (double-buffered, as the current block's are
+// still needed by the final add). The row_ptr pair of the block after that is
+// loaded into registers one iteration ahead. So no global-memory latency sits
+// between the arithmetic phases. Requires 16-byte aligned code blocks and
+// scales, 4-byte aligned zero points (checked by the launcher).
+template <int LOGN>
+constexpr int weff_csr_cap() {
+  return (1 << LOGN) < 512 ? (1 << LOGN) : 512;
+}
+
+__host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
+
+template <int LOGN>
+__global__ void __launch_bounds__(kThreads, 2)
+    weff_pipe_kernel(const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
+                     const float *__restrict__ coef, int64_t p, int d_in, int64_t n_rows, float scale, int bits,
+                     int group, const uint8_t *__restrict__ qw, const float *__restrict__ scales,
+                     const uint8_t *__restrict__ zeros, __nv_bfloat16 *__restrict__ out, int dq_stride) {
+  using G = Geo<LOGN, 8>;
+  constexpr int RPC = kThreads / G::P;
+  constexpr int CAP = weff_csr_cap<LOGN>();
+  extern __shared__ __align__(16) float smem[];
+  const int rl = threadIdx.x / G::P;
+  const int t = threadIdx.x % G::P;
+  float *buf = smem + rl * G::N;
+  int32_t *my_k = reinterpret_cast<int32_t *>(smem + RPC * G::N) + rl * CAP;
+  float *my_v = reinterpret_cast<float *>(smem + RPC * G::N + RPC * CAP) + rl * CAP;
+  uint8_t *dq = reinterpret_cast<uint8_t *>(smem + RPC * G::N + 2 * RPC * CAP);
+  const int nb = d_in >> LOGN;
+  const int64_t blocks = n_rows * nb;
+  const int64_t row_bytes = (int64_t)d_in * bits / 8;
+  const int ng = qw ? d_in / group : 0;
+  const int gpb = qw ? G::N / group : 0;  // quantization groups per block
+  const int qb = G::N * bits / 8;         // code bytes per block
+  const int64_t stride = (int64_t)gridDim.x * RPC;
+
+  auto row_range = [&](int64_t bi, int64_t &b, int64_t &e) {
+    b = 0;
+    e = 0;
+    if (bi < blocks) {
+      const int64_t r = bi / nb;
+      b = row_ptr[r];
+      e = row_ptr[r + 1];
+      if (b < 0) b = 0;
+      if (e > p) e = p;
+      if (e < b) e = b;
+    }
+  };
+  // this thread's share of the copies of block bi's inputs into row slot rl
+  auto prefetch = [&](int64_t bi, int64_t b, int64_t e, int d) {
+    if (bi < blocks) {
+      const int n = (int)(e - b < CAP ? e - b : CAP);
+      for (int j = t; j < n; j += G::P) {
+        cp_async4(my_k + j, col_idx + b + j);
+        cp_async4(my_v + j, coef + b + j);
+      }
+      if (qw) {
+        const int64_t r = bi / nb;
+        const int blk = (int)(bi % nb);
+        uint8_t *dst = dq + ((size_t)d * RPC + rl) * dq_stride;
+        const uint8_t *qsrc = qw + r * row_bytes + (int64_t)blk * qb;
+        for (int c = t; c < qb / 16; c += G::P) cp_async16(dst + 16 * c, qsrc + 16 * c);
+        const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales + r * ng + (int64_t)blk * gpb);
+        uint8_t *sdst = dst + round16(qb);
+        for (int c = t; c < gpb / 4; c += G::P) cp_async16(sdst + 16 * c, ssrc + 16 * c);
+        const uint8_t *zsrc = zeros + r * ng + (int64_t)blk * gpb;
+        uint8_t *zdst = sdst + round16(gpb * 4);
+        for (int c = t; c < gpb / 4; c += G::P) cp_async4(zdst + 4 * c, zsrc + 4 * c);
+      }
+    }
+    cp_async_commit();
+  };
+
+  int64_t bi = (int64_t)blockIdx.x * RPC + rl;
+  int64_t b, e, b_next, e_next;
+  row_range(bi, b, e);
+  prefetch(bi, b, e, 0);
+  row_range(bi + stride, b_next, e_next);
+  int d = 0;
+  for (int64_t base = (int64_t)blockIdx.x * RPC; base < blocks; base += stride, d ^= 1) {
+    const bool active = bi < blocks;
+    const int64_t r = active ? bi / nb : 0;
+    const int k0 = active ? (int)(bi % nb) << LOGN : 0;
+    cp_async_wait_all();
+    __syncthreads();  // this block's inputs are staged; the previous iteration is done with buf
+    for (int i = 4 * t; i < G::N; i += 4 * G::P) *reinterpret_cast<float4 *>(buf + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    if (active) {
+      const int n = (int)(e - b < CAP ? e - b : CAP);
+      for (int j = t; j < n; j += G::P) {
+        const int k = my_k[j] - k0;
+        if ((unsigned)k < (unsigned)G::N) buf[G::phys(k)] = my_v[j];
+      }
+      for (int64_t j = b + CAP + t; j < e; j += G::P) {  // entries beyond the staged ones
+        const int k = col_idx[j] - k0;
+        if ((unsigned)k < (unsigned)G::N) buf[G::phys(k)] = coef[j];
+      }
+    }
+    __syncthreads();  // the staged CSR slice is consumed: copy the next block's inputs
+    const int64_t bi_next = bi + stride;
+    prefetch(bi_next, b_next, e_next, d ^ 1);
+    bi = bi_next;
+    b = b_next;
+    e = e_next;
+    row_range(bi + stride, b_next, e_next);  // used one iteration from now
+
+    float v[G::R];
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+      const float *src = buf + G::phys(G::eA(t, h << G::LV));
+#pragma unroll
+      for (int u = 0; u < 8; u += 4) {
+        const float4 f = *reinterpret_cast<const float4 *>(src + u);
+        v[h * 8 + u] = f.x, v[h * 8 + u + 1] = f.y, v[h * 8 + u + 2] = f.z, v[h * 8 + u + 3] = f.w;
+      }
+    }
+    butterflies_x2<G::R, 0, G::RB, 0>(v);
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+      float *dst = buf + G::phys(G::eA(t, h << G::LV));
+#pragma unroll
+      for (int u = 0; u < 8; u += 4)
+        *reinterpret_cast<float4 *>(dst + u) = make_float4(v[h * 8 + u], v[h * 8 + u + 1], v[h * 8 + u + 2], v[h * 8 + u + 3]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
+    butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) buf[G::phys(G::eB(t, q))] = v[q] * scale;
+    __syncthreads();
+    if (active) {
+      const uint8_t *dqc = dq + ((size_t)d * RPC + rl) * dq_stride;
+      const float *s_sc = reinterpret_cast<const float *>(dqc + round16(qb));
+      const uint8_t *s_z = dqc + round16(qb) + round16(gpb * 4);
+#pragma unroll
+      for (int h = 0; h < (1 << G::HB); ++h) {
+        const int el = G::eA(t, h << G::LV);
+        const float *src = buf + G::phys(el);
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; u += 4) {
+          const float4 a = *reinterpret_cast<const float4 *>(src + u);
+          f[u] = a.x, f[u + 1] = a.y, f[u + 2] = a.z, f[u + 3] = a.w;
+        }
+        if (qw) {
+          const uint8_t *cp = dqc + el * bits / 8;
+          uint32_t w;
+          if (bits == 4) {
+            w = *reinterpret_cast<const uint32_t *>(cp);
+          } else if (bits == 2) {
+            w = *reinterpret_cast<const uint16_t *>(cp);
+          } else {
+            w = 0;
+            for (int bb = 0; bb < bits; ++bb) w |= (uint32_t)cp[bb] << (8 * bb);
+          }
+          const uint32_t mask = (1u << bits) - 1u;
+          const int g = el / group;
+          const float sc = s_sc[g], z = (float)s_z[g];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] += sc * ((float)((w >> (bits * i)) & mask) - z);
+        }
+        st_stream(out + r * d_in + k0 + el, io<__nv_bfloat16>::pack(f));
+      }
+    }
+  }
+  cp_async_wait_all();  // no copy is left in flight when the CTA exits
+}
+
 template <int LOGN>
 cudaError_t run_weff(const int32_t *row_ptr, const int32_t *col_idx, const float *coef, int64_t p, int d_in,
                      int64_t n_rows, float scale, int bits, int group, const uint8_t *qw, const float *scales,
                      const uint8_t *zeros, __nv_bfloat16 *out, cudaStream_t s) {
   using G = Geo<LOGN, 8>;
   constexpr int RPC = kThreads / G::P;
+  const int64_t blocks = n_rows * (d_in >> LOGN);
+  // the pipelined kernel copies code blocks and scales in 16-byte pieces and
+  // zero points in 4-byte pieces
+  bool pipe = true;
+  int dq_stride = 0;
+  if (qw) {
+    const int64_t qb = (int64_t)G::N * bits / 8, row_bytes = (int64_t)d_in * bits / 8;
+    const int gpb = G::N / group, ng = d_in / group;
+    pipe = qb % 16 == 0 && row_bytes % 16 == 0 && gpb % 4 == 0 && ng % 4 == 0 &&
+           reinterpret_cast<uintptr_t>(qw) % 16 == 0 && reinterpret_cast<uintptr_t>(scales) % 16 == 0 &&
+           reinterpret_cast<uintptr_t>(zeros) % 4 == 0;
+    dq_stride = round16((int)qb) + round16(gpb * 4) + round16(gpb);
+  }
+  if (pipe) {
+    const size_t smem = (size_t)RPC * G::N * sizeof(float) + 2ull * RPC * weff_csr_cap<LOGN>() * 4 +
+                        2ull * RPC * dq_stride;
+    auto k = weff_pipe_kernel<LOGN>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    const int64_t need = cdiv(blocks, RPC);
+    const int64_t cap = (int64_t)sm_count() * occ;
+    k<<<(unsigned)(need < cap ? need : cap), kThreads, smem, s>>>(row_ptr, col_idx, coef, p, d_in, n_rows, scale,
+                                                                 bits, group, qw, scales, zeros, out, dq_stride);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)RPC * G::N * sizeof(float);
   auto k = weff_rows_kernel<LOGN>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -373,7 +581,7 @@ cudaError_t run_weff(const int32_t *row_ptr, const int32_t *col_idx, const float
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, smem);
   if (e != cudaSuccess) return e;
   if (occ < 1) occ = 1;
-  const int64_t need = cdiv(n_rows * (d_in >> LOGN), RPC);
+  const int64_t need = cdiv(blocks, RPC);
   const int64_t cap = (int64_t)sm_count() * occ;
   k<<<(unsigned)(need < cap ? need : cap), kThreads, smem, s>>>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits,
                                                                group, qw, scales, zeros, out);
