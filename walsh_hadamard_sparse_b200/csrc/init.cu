@@ -108,6 +108,28 @@ __device__ int64_t block_excl_scan(int64_t v, int64_t *sh, int64_t *tot) {
   return incl - v;
 }
 
+// Pairwise sum of the squares of w[base .. base + L) (zero past d_in), the
+// canonical tree of an aligned run of L (a power of two), in registers.
+template <int L>
+__device__ __forceinline__ double tree_sq(const float *__restrict__ w, int base, int d_in) {
+  double x[L];
+#pragma unroll
+  for (int i = 0; i < L; ++i) {
+    const int k = base + i;
+    const double v = k < d_in ? (double)w[k] : 0.0;
+    x[i] = __dmul_rn(v, v);
+  }
+#pragma unroll
+  for (int h = 1; h < L; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < L; i += 2 * h) x[i] = __dadd_rn(x[i], x[i + h]);
+  return x[0];
+}
+
+// e[row] = sqrt of the canonical pairwise sum of squares over the zero-padded
+// power-of-two length m: thread t sums the aligned run [t*L, t*L + L) with
+// L = m / blockDim (runs of 16 in registers, longer runs as a tree of those),
+// then the threads' sums meet in the block-level tree.
 __global__ void __launch_bounds__(kNormThreads) row_norm_kernel(const float *__restrict__ dW, int d_in,
                                                                 double *__restrict__ e) {
   __shared__ double sh[kNormThreads];
@@ -116,47 +138,83 @@ __global__ void __launch_bounds__(kNormThreads) row_norm_kernel(const float *__r
   int m = next_pow2(d_in);
   const int L = m > kNormThreads ? m / kNormThreads : 1;
   const int base = threadIdx.x * L;
-  const double mine = run_pairwise(L, [&](int i) {
-    const int k = base + i;
-    if (k >= d_in) return 0.0;
-    const double x = (double)w[k];
-    return __dmul_rn(x, x);
-  });
+  double mine;
+  switch (L) {
+    case 1: mine = tree_sq<1>(w, base, d_in); break;
+    case 2: mine = tree_sq<2>(w, base, d_in); break;
+    case 4: mine = tree_sq<4>(w, base, d_in); break;
+    case 8: mine = tree_sq<8>(w, base, d_in); break;
+    case 16: mine = tree_sq<16>(w, base, d_in); break;
+    default: mine = run_pairwise(L / 16, [&](int c) { return tree_sq<16>(w, base + 16 * c, d_in); }); break;
+  }
   const double s = block_pairwise(mine, sh);
   if (threadIdx.x == 0) e[row] = __dsqrt_rn(s);
 }
 
 // Radix select over `n` keys produced by key(i) (eligible when ok(i)): the
 // `want`-th smallest key K and how many keys equal to K are to be taken.
+// Eight passes of 8 bits, most significant first. The histogram adds one
+// count per distinct digit per warp (the leading bytes of fp64 patterns are
+// shared by nearly all keys, so per-key atomics would serialise), and warp 0
+// finds the digit holding the `need`-th key with a shuffle scan over the 256
+// bins (8 per lane).
 template <typename KeyF, typename OkF>
 __device__ void radix_select_smallest(int n, int64_t want, KeyF key, OkF ok, uint32_t *hist, uint64_t *K_out,
                                       int64_t *need_out) {
+  __shared__ int sel_digit;
+  __shared__ int64_t sel_need;
   uint64_t prefix = 0;
   int64_t need = want;
+  const int lane = threadIdx.x & 31;
+  const int n_round = (n + blockDim.x - 1) / blockDim.x * blockDim.x;  // whole warps iterate together
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     const uint64_t hi_mask = shift == 56 ? 0 : (~0ull << (shift + 8));
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      if (!ok(i)) continue;
-      const uint64_t k = key(i);
-      if ((k & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(k >> shift) & 255], 1u);
+    for (int i = threadIdx.x; i < n_round; i += blockDim.x) {
+      int bin = 256;  // no count
+      if (i < n && ok(i)) {
+        const uint64_t k = key(i);
+        if ((k & hi_mask) == (prefix & hi_mask)) bin = (int)((k >> shift) & 255);
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    __shared__ int sel_digit;
-    __shared__ int64_t sel_need;
-    if (threadIdx.x == 0) {
-      int64_t cum = 0;
-      int d = 255;
-      for (int b = 0; b < 256; ++b) {
-        if (cum + hist[b] >= need) {
-          d = b;
-          break;
-        }
-        cum += hist[b];
+    if (threadIdx.x < 32) {
+      uint32_t c[8];
+      uint32_t mine = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[8 * lane + j];
+        mine += c[j];
       }
-      sel_digit = d;
-      sel_need = need - cum;
+      uint32_t incl = mine;  // inclusive scan over lanes
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const int64_t excl = (int64_t)(incl - mine);
+      const bool hit = (excl < need && (int64_t)incl >= need) || (lane == 0 && need <= 0);
+      const unsigned who = __ballot_sync(0xffffffffu, hit);
+      if (hit) {
+        int64_t cum = excl;
+        int d = 8 * lane + 7;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (cum + c[j] >= need) {
+            d = 8 * lane + j;
+            break;
+          }
+          cum += c[j];
+        }
+        sel_digit = d;
+        sel_need = need - cum;
+      } else if (who == 0 && lane == 31) {  // fewer eligible keys than wanted: past the last digit
+        sel_digit = 255;
+        sel_need = need - (int64_t)incl;
+      }
     }
     __syncthreads();
     prefix |= (uint64_t)sel_digit << shift;
