@@ -109,6 +109,12 @@ typedef struct {
    * change of coef, the base weight or alpha. NULL: each call builds its own
    * copy in the workspace. */
   void *weff;
+  /* Nonzero: Z_out of this forward call already holds X H for the same X and
+   * had_block (written by the forward of another layer that reads the same
+   * input, e.g. q, k and v of an attention block, or gate and up of an MLP);
+   * the forward reads it instead of computing it. The backward is unaffected.
+   * 0 (default): the forward computes Z_out. */
+  int32_t z_given;
 } qwha_adapter;
 
 /* The frozen quantized base weight W_Q [d_out, d_in], device memory.

@@ -33,6 +33,7 @@ class QwhaAdapter(ctypes.Structure):
         ("tile_pos", P),
         ("tile_rk", P),
         ("weff", P),
+        ("z_given", i32),
     ]
 
 

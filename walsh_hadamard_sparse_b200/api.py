@@ -114,14 +114,20 @@ def fwht(x: torch.Tensor, had_block: int | None = None, out: torch.Tensor | None
 
 
 def adapter_fwd(a: Adapter, X: torch.Tensor, alpha: float = 1.0, wq: QWeight | None = None,
-                Z_out: torch.Tensor | None = None, Y: torch.Tensor | None = None, ws: torch.Tensor | None = None):
-    """(Z, Y) with Z = X H and Y = X W_Q^T + alpha Z F^T (W_Q term only with wq)."""
+                Z_out: torch.Tensor | None = None, Y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                z_given: bool = False):
+    """(Z, Y) with Z = X H and Y = X W_Q^T + alpha Z F^T (W_Q term only with wq).
+    z_given: Z_out already holds X H (from the forward of another layer reading the same X with the same
+    had_block) and is read instead of computed."""
     T = X.shape[0]
+    if z_given and Z_out is None:
+        raise ValueError("z_given needs Z_out")
     Z_out = torch.empty_like(X) if Z_out is None else Z_out
     Y = torch.empty((T, a.d_out), dtype=X.dtype, device=X.device) if Y is None else Y
     need = workspace_size(OP_FWD_DENSE if a.algo == "dense" else OP_FWD, a.d_out, a.d_in, a.p, T, wq is not None)
     ws = _ws(need, X.device) if ws is None else ws
     cs = a.c_struct()
+    cs.z_given = 1 if z_given else 0
     cw = wq.c_struct() if wq is not None else None
     rc = lib().qwha_adapter_fwd(ctypes.byref(cs), ctypes.byref(cw) if cw is not None else None, _dt(X), _ptr(X), T,
                                 float(alpha), _ptr(Z_out), _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(), _stream())

@@ -27,7 +27,7 @@ qwha_status fail(qwha_status s, const char *fmt, ...) {
 
 qwha_status cuda_status(cudaError_t e, const char *what) {
   if (e == cudaSuccess) return QWHA_OK;
-  return fail(QWHA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return fail(QWHA_ERR_CUDA, "%s: %s (cudaError %d)", what, cudaGetErrorString(e), (int)e);
 }
 
 int sm_count() {
@@ -413,7 +413,17 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   cudaStream_t s = (cudaStream_t)stream;
   const int logn = ilog2(a->had_block);
   const float inv = (float)(1.0 / sqrt((double)a->had_block));
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
+  if (dense && a->z_given) {  // Z_out is an input: W_eff and the GEMM only
+    void *weff = a->weff ? a->weff : ws;
+    {
+      StageScope sc(ST_WEFF, 1, s);
+      e = launch_weff(a, wq, alpha, weff, s);
+    }
+    if (e != cudaSuccess) return cuda_status(e, "W_eff");
+    StageScope sc(ST_GEMM_FWD, 1, s);
+    return cuda_status(launch_gemm_nt(X, weff, nullptr, Y, false, T, a->d_out, a->d_in, s), "GEMM");
+  }
   if (dense) {
     // Z = X H (kept for the backward) on the auxiliary stream, concurrently
     // with W_eff and Y = X W_eff^T on the caller's stream.
@@ -442,7 +452,7 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
     if (e != cudaSuccess) return cuda_status(e, "W_eff / GEMM");
     return cuda_status(ej, "join");
   }
-  {
+  if (!a->z_given) {
     StageScope sc(ST_FWHT_FWD, 1, s);
     e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
   }
@@ -495,7 +505,7 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   float *partial = static_cast<float *>(cv.take((size_t)kSddmmMaxChunks * (size_t)(a->p > 0 ? a->p : 1) * 4));
   float *dz = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
   float *coef_csc = static_cast<float *>(cv.take((size_t)(a->p > 0 ? a->p : 1) * 4));
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   {
     StageScope sc(ST_SDDMM, 2, s);
     e = launch_sddmm(dt, dY, Z, T, a->d_out, a->d_in, a->tile_ptr, a->tile_pos, a->tile_rk, a->p, alpha, partial, dc,
