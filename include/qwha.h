@@ -185,12 +185,38 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
  *   E row i = the budget_i largest |V| (ties to the lower index), ascending;
  *   c = float(V * 1/sqrt(had_block)) (the dense solution values).
  * Outputs (device): budgets [d_out], row_ptr [d_out+1], col_idx [p], coef [p].
- * Requires min_per_row*d_out <= p <= d_in*d_out, p < 2^31, d_in <= 32768.
+ * Requires min_per_row*d_out <= p <= d_in*d_out, p < 2^31, d_in <= 16384.
  * Budgets and E are bitwise deterministic. */
 qwha_status qwha_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block,
                             int64_t p, int32_t min_per_row, qwha_remainder mode,
                             int32_t *budgets, int32_t *row_ptr, int32_t *col_idx, float *coef,
                             void *ws, size_t ws_bytes, void *stream);
+
+/* The three steps of qwha_init_alloc as separate calls, for AdaAlloc sharded
+ * by output rows over data-parallel ranks: each rank computes the norms of its
+ * rows (qwha_init_norms), the ranks exchange them so that every rank holds all
+ * d_out norms, every rank computes the same budgets from them
+ * (qwha_init_budgets; bitwise identical, as the norms are), each rank selects
+ * E and c for its rows (qwha_init_select), and the ranks exchange their CSR
+ * slices. Run over all rows in one process, the three calls give bit for bit
+ * the outputs of qwha_init_alloc. Same requirements as qwha_init_alloc; all
+ * pointers are device memory. */
+/* e[i] = ||dWq[i,:]||_2 for the `rows` rows of dWq [rows, d_in] fp32 (fp64
+ * squares, pairwise sum in index order); e fp64 [rows]. */
+qwha_status qwha_init_norms(const float *dWq, int32_t rows, int32_t d_in, double *e, void *stream);
+/* budgets [d_out] and row_ptr [d_out+1] from all d_out norms e (fp64) by the
+ * rule of qwha_init_alloc. ws: qwha_workspace_size(QWHA_OP_INIT, ...) bytes. */
+qwha_status qwha_init_budgets(const double *e, int32_t d_out, int32_t d_in, int64_t p,
+                              int32_t min_per_row, qwha_remainder mode, int32_t *budgets,
+                              int32_t *row_ptr, void *ws, size_t ws_bytes, void *stream);
+/* E and c of `rows` consecutive rows: dWq [rows, d_in] fp32 holds those rows,
+ * budgets [rows] and row_ptr [rows+1] are the matching slices of the global
+ * budgets and row_ptr (row_ptr need not start at 0). Row i's entries go to
+ * col_idx / coef [row_ptr[i] - row_ptr[0], + budgets[i]); p_local =
+ * row_ptr[rows] - row_ptr[0] is the capacity of col_idx and coef. */
+qwha_status qwha_init_select(const float *dWq, int32_t rows, int32_t d_in, int32_t had_block,
+                             const int32_t *budgets, const int32_t *row_ptr, int64_t p_local,
+                             int32_t *col_idx, float *coef, void *stream);
 
 /* Index views of E for the backward (E stays fixed while c trains,
  * papernotes.org 整体框架): from the CSR row_ptr/col_idx (device) write the

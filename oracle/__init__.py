@@ -59,6 +59,9 @@ def _load():
                 "oracle_adapter_bwd_dx": [i32, i32, i32, P, P, P, P, P, i64, f64, P],
                 "oracle_adapter_bwd_dc": [i32, i32, i32, P, P, i64, f64, i64, P, P, P],
                 "oracle_init_alloc": [P, i32, i32, i32, i64, i32, i32, P, P, P, P, P],
+                "oracle_init_norms": [P, i32, i32, P],
+                "oracle_init_budgets": [P, i32, i32, i64, i32, i32, P, P],
+                "oracle_init_select": [P, i32, i32, i32, P, P, P, P],
                 "oracle_plan_build": [i32, i32, i64, P, P, P, P, P],
             }
             for name, args in sig.items():
@@ -197,6 +200,38 @@ def init_alloc(dWq, p: int, n: int, min_per_row: int = 2, mode: str = "fewest"):
     rc = _load().oracle_init_alloc(_p(w), d_out, d_in, n, int(p), int(min_per_row), m, _p(b), _p(rp), _p(ci), _p(c), _p(e))
     _check(rc, "init_alloc")
     return dict(budgets=b, row_ptr=rp, col_idx=ci, coef=c, err_norm=e)
+
+
+def init_norms(dWq_rows):
+    """AdaAlloc step 1 for a block of rows: e_i = ||dW_Q[i,:]||_2 (fp64)."""
+    w = np.ascontiguousarray(dWq_rows, dtype=np.float32)
+    rows, d_in = w.shape
+    e = np.empty(rows, dtype=np.float64)
+    _check(_load().oracle_init_norms(_p(w), rows, d_in, _p(e)), "init_norms")
+    return e
+
+
+def init_budgets(e, d_in: int, p: int, min_per_row: int = 2, mode: str = "fewest"):
+    """AdaAlloc step 2 from all d_out norms: (budgets [d_out], row_ptr [d_out+1])."""
+    e = _f64(e)
+    d_out = e.size
+    b = np.empty(d_out, dtype=np.int32)
+    rp = np.empty(d_out + 1, dtype=np.int32)
+    m = {"fewest": 0, "largest": 1}[mode]
+    _check(_load().oracle_init_budgets(_p(e), d_out, d_in, int(p), int(min_per_row), m, _p(b), _p(rp)), "init_budgets")
+    return b, rp
+
+
+def init_select(dWq_rows, n: int, budgets, row_ptr):
+    """AdaAlloc step 3 for a block of rows given its slices of budgets and row_ptr: (col_idx, coef)."""
+    w = np.ascontiguousarray(dWq_rows, dtype=np.float32)
+    rows, d_in = w.shape
+    b, rp = _i32(budgets), _i32(row_ptr)
+    cnt = int(rp[-1] - rp[0]) if rows else 0
+    ci = np.empty(cnt, dtype=np.int32)
+    c = np.empty(cnt, dtype=np.float32)
+    _check(_load().oracle_init_select(_p(w), rows, d_in, n, _p(b), _p(rp), _p(ci), _p(c)), "init_select")
+    return ci, c
 
 
 def plan_build(row_ptr, col_idx, d_in: int):

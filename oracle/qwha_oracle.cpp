@@ -332,16 +332,10 @@ int oracle_adapter_bwd_dc(int32_t d_out, int32_t d_in, int32_t n, const double *
 //   c      = float(V * (1/sqrt(n)))
 // Outputs: budgets [d_out], row_ptr [d_out+1], col_idx [p], coef [p],
 // err_norm [d_out] (nullable).
-int oracle_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, int64_t p,
-                      int32_t min_per_row, int32_t mode, int32_t *budgets, int32_t *row_ptr,
-                      int32_t *col_idx, float *coef, double *err_norm) {
-  if (!shape_ok(d_in, n) || d_out <= 0 || min_per_row < 0 || min_per_row > d_in) return 1;
-  if (p < (int64_t)min_per_row * d_out || p > (int64_t)d_in * d_out || p > 2147483647LL) return 1;
-  if (mode != 0 && mode != 1) return 1;
-
-  // Per-channel error norms.
-  std::vector<double> e(d_out);
-  parallel_for(d_out, [&](int64_t i) {
+// Step 1: e_i = ||dW_Q[i,:]||_2 for `rows` rows (fp64 squares, pairwise sum).
+int oracle_init_norms(const float *dWq, int32_t rows, int32_t d_in, double *e) {
+  if (rows < 0 || d_in <= 0) return 1;
+  parallel_for(rows, [&](int64_t i) {
     std::vector<double> sq(d_in);
     for (int k = 0; k < d_in; ++k) {
       double w = (double)dWq[i * d_in + k];
@@ -349,10 +343,16 @@ int oracle_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, 
     }
     e[i] = std::sqrt(pairwise_sum(sq.data(), d_in));
   });
-  if (err_norm)
-    for (int i = 0; i < d_out; ++i) err_norm[i] = e[i];
+  return 0;
+}
 
-  // Budgets: floor share of the pool, capped at d_in, surplus re-shared.
+// Step 2: budgets from all d_out norms. Floor share of the pool, capped at
+// d_in, surplus re-shared; the remainder one each in the order of `mode`.
+int oracle_init_budgets(const double *e, int32_t d_out, int32_t d_in, int64_t p, int32_t min_per_row,
+                        int32_t mode, int32_t *budgets, int32_t *row_ptr) {
+  if (d_out <= 0 || d_in <= 0 || min_per_row < 0 || min_per_row > d_in) return 1;
+  if (p < (int64_t)min_per_row * d_out || p > (int64_t)d_in * d_out || p > 2147483647LL) return 1;
+  if (mode != 0 && mode != 1) return 1;
   std::vector<int64_t> b(d_out, min_per_row);
   std::vector<char> capped(d_out, 0);
   double pool = (double)(p - (int64_t)min_per_row * d_out);
@@ -398,10 +398,19 @@ int oracle_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, 
     budgets[i] = (int32_t)b[i];
     row_ptr[i + 1] = row_ptr[i] + (int32_t)b[i];
   }
+  return 0;
+}
 
-  // In-channel selection of the largest transform magnitudes.
+// Step 3: in-channel selection of the largest transform magnitudes for `rows`
+// rows; row i's entries go to [row_ptr[i] - row_ptr[0], + budgets[i]).
+int oracle_init_select(const float *dWq, int32_t rows, int32_t d_in, int32_t n, const int32_t *budgets,
+                       const int32_t *row_ptr, int32_t *col_idx, float *coef) {
+  if (rows < 0 || !shape_ok(d_in, n)) return 1;
+  for (int i = 0; i < rows; ++i)
+    if (budgets[i] < 0 || budgets[i] > d_in || row_ptr[i + 1] - row_ptr[i] != budgets[i]) return 1;
   const double inv = inv_sqrt(n);
-  parallel_for(d_out, [&](int64_t i) {
+  const int32_t base = rows > 0 ? row_ptr[0] : 0;
+  parallel_for(rows, [&](int64_t i) {
     std::vector<double> v(d_in);
     for (int k = 0; k < d_in; ++k) v[k] = (double)dWq[i * d_in + k];
     for (int blk = 0; blk < d_in / n; ++blk) butterflies(v.data() + (int64_t)blk * n, n);
@@ -414,11 +423,23 @@ int oracle_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, 
     std::vector<int> pick(idx.begin(), idx.begin() + budgets[i]);
     std::sort(pick.begin(), pick.end());
     for (int q = 0; q < budgets[i]; ++q) {
-      col_idx[row_ptr[i] + q] = pick[q];
-      coef[row_ptr[i] + q] = (float)(v[pick[q]] * inv);
+      col_idx[row_ptr[i] - base + q] = pick[q];
+      coef[row_ptr[i] - base + q] = (float)(v[pick[q]] * inv);
     }
   });
   return 0;
+}
+
+int oracle_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, int64_t p,
+                      int32_t min_per_row, int32_t mode, int32_t *budgets, int32_t *row_ptr,
+                      int32_t *col_idx, float *coef, double *err_norm) {
+  if (!shape_ok(d_in, n) || d_out <= 0) return 1;
+  std::vector<double> e(d_out);
+  if (oracle_init_norms(dWq, d_out, d_in, e.data())) return 1;
+  if (err_norm)
+    for (int i = 0; i < d_out; ++i) err_norm[i] = e[i];
+  if (oracle_init_budgets(e.data(), d_out, d_in, p, min_per_row, mode, budgets, row_ptr)) return 1;
+  return oracle_init_select(dWq, d_out, d_in, n, budgets, row_ptr, col_idx, coef);
 }
 
 // Column view of the CSR pattern: for every column k the nonzeros j with

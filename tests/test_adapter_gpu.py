@@ -199,6 +199,37 @@ def test_init_bitexact(d_out, d_in, n, p, mode, kind):
     assert np.array_equal(got["coef"].cpu().numpy().view(np.uint32), ref["coef"].view(np.uint32))
 
 
+@pytest.mark.parametrize("shards,mode", [(1, "fewest"), (3, "largest")])
+def test_init_split_steps_bitexact(shards, mode):
+    """qwha_init_norms / _budgets / _select over row shards (as the ranks of a sharded AdaAlloc run them)
+    reproduce qwha_init_alloc and the oracle bit for bit; the shards' row_ptr slices do not start at 0."""
+    import torch
+
+    from walsh_hadamard_sparse_b200.api import shard_rows
+
+    W = _W()
+    d_out, d_in, n = 301, 1024, 512
+    p = d_out * 17 + 9
+    g = rng_for(34, "init-split", shards, mode)
+    w = g.standard_normal((d_out, d_in)).astype(np.float32) * np.float32(0.01)
+    w[7] *= np.float32(500.0)  # capped row
+    dw = to_dev(w)
+    whole = W.init_alloc(dw, p, n, 2, mode)
+    bounds = [shard_rows(d_out, r, shards) for r in range(shards)]
+    e = torch.cat([W.init_norms(dw[r0:r1]) for r0, r1 in bounds])
+    b, rp = W.init_budgets(e, d_in, p, 2, mode)
+    sel = [W.init_select(dw[r0:r1], n, b[r0:r1], rp[r0:r1 + 1]) for r0, r1 in bounds]
+    ci = torch.cat([s[0] for s in sel]).cpu().numpy()
+    cf = torch.cat([s[1] for s in sel]).cpu().numpy()
+    ref = oracle.init_alloc(w, p, n, 2, mode)
+    assert ref["budgets"].max() == d_in
+    for got in ({"budgets": b.cpu().numpy(), "row_ptr": rp.cpu().numpy(), "col_idx": ci, "coef": cf},
+                {k: v.cpu().numpy() for k, v in whole.items()}):
+        for k in ("budgets", "row_ptr", "col_idx"):
+            assert np.array_equal(got[k], ref[k]), k
+        assert np.array_equal(got["coef"].view(np.uint32), ref["coef"].view(np.uint32))
+
+
 # --------------------------------------------------------------------------- forward / backward
 
 

@@ -13,8 +13,13 @@ from .api import (  # noqa: F401
     adapter_fwd,
     fwht,
     init_alloc,
+    init_alloc_sharded,
+    init_budgets,
+    init_norms,
+    init_select,
     plan_build,
     plan_tiles,
+    shard_rows,
     stage_report,
     stage_timing,
     validate_plan,

@@ -175,6 +175,91 @@ def init_alloc(dWq: torch.Tensor, p: int, had_block: int, min_per_row: int = 2, 
     return out
 
 
+def init_norms(dWq_rows: torch.Tensor) -> torch.Tensor:
+    """e[i] = ||dWq_rows[i, :]||_2 in fp64 (the first step of AdaAlloc) for a block of rows."""
+    rows, d_in = dWq_rows.shape
+    e = torch.empty(rows, dtype=torch.float64, device=dWq_rows.device)
+    check(lib().qwha_init_norms(_ptr(dWq_rows), rows, d_in, _ptr(e), _stream()), "qwha_init_norms")
+    return e
+
+
+def init_budgets(e: torch.Tensor, d_in: int, p: int, min_per_row: int = 2, mode: str = "fewest",
+                 ws: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """(budgets [d_out], row_ptr [d_out+1]) from all d_out row norms (fp64)."""
+    d_out = e.shape[0]
+    dev = e.device
+    budgets = torch.empty(d_out, dtype=torch.int32, device=dev)
+    row_ptr = torch.empty(d_out + 1, dtype=torch.int32, device=dev)
+    need = workspace_size(OP_INIT, d_out, d_in, p, 0, False)
+    ws = _ws(need, dev) if ws is None else ws
+    rc = lib().qwha_init_budgets(_ptr(e), d_out, d_in, p, min_per_row, REMAINDER[mode], _ptr(budgets), _ptr(row_ptr),
+                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream())
+    check(rc, "qwha_init_budgets")
+    return budgets, row_ptr
+
+
+def init_select(dWq_rows: torch.Tensor, had_block: int, budgets: torch.Tensor,
+                row_ptr: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """(col_idx, coef) of a block of rows: budgets [rows] and row_ptr [rows+1] are the block's slices of the global
+    budgets and row_ptr (row_ptr need not start at 0)."""
+    rows, d_in = dWq_rows.shape
+    p_local = int(row_ptr[-1].item() - row_ptr[0].item()) if rows else 0
+    dev = dWq_rows.device
+    col_idx = torch.empty(max(p_local, 1), dtype=torch.int32, device=dev)
+    coef = torch.empty(max(p_local, 1), dtype=torch.float32, device=dev)
+    rc = lib().qwha_init_select(_ptr(dWq_rows), rows, d_in, had_block, _ptr(budgets), _ptr(row_ptr), p_local,
+                                _ptr(col_idx), _ptr(coef), _stream())
+    check(rc, "qwha_init_select")
+    return col_idx[:p_local], coef[:p_local]
+
+
+def shard_rows(d_out: int, rank: int, world: int) -> tuple[int, int]:
+    """Rows [r0, r1) of output channels held by `rank` of `world` in sharded AdaAlloc."""
+    return rank * d_out // world, (rank + 1) * d_out // world
+
+
+def init_alloc_sharded(dWq_rows: torch.Tensor, d_out: int, p: int, had_block: int, min_per_row: int = 2,
+                       mode: str = "fewest", group=None, steps=None) -> dict:
+    """AdaAlloc with the rows of dW_Q sharded over the ranks of `group` (rank r holds rows shard_rows(d_out, r,
+    world)): the ranks exchange their row norms (fp64), compute the same budgets from all of them, select E and c
+    for their own rows and exchange the CSR slices. Every rank returns the full result of init_alloc on the whole
+    dW_Q: dict(budgets, row_ptr, col_idx, coef).
+
+    `steps` = (norms, budgets, select) replaces the three device steps (defaults: init_norms, init_budgets,
+    init_select); the collectives run on whatever device the tensors live on."""
+    import torch.distributed as dist
+
+    norms_fn, budgets_fn, select_fn = steps or (init_norms, init_budgets, init_select)
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    r0, r1 = shard_rows(d_out, rank, world)
+    d_in = dWq_rows.shape[1]
+    if dWq_rows.shape[0] != r1 - r0:
+        raise ValueError(f"rank {rank} holds {dWq_rows.shape[0]} rows, expected {r1 - r0}")
+    e_local = norms_fn(dWq_rows)
+    bounds = [shard_rows(d_out, r, world) for r in range(world)]
+    most = max(b1 - b0 for b0, b1 in bounds)
+    pad = torch.zeros(most, dtype=torch.float64, device=e_local.device)
+    pad[: r1 - r0] = e_local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    e_all = torch.cat([parts[r][: b1 - b0] for r, (b0, b1) in enumerate(bounds)])
+    budgets, row_ptr = budgets_fn(e_all, d_in, p, min_per_row, mode)
+    col_local, coef_local = select_fn(dWq_rows, had_block, budgets[r0:r1], row_ptr[r0:r1 + 1])
+    rp_host = row_ptr.cpu()
+    sizes = [int(rp_host[b1] - rp_host[b0]) for b0, b1 in bounds]
+    cap = max(max(sizes), 1)
+    out = {}
+    for name, t in (("col_idx", col_local), ("coef", coef_local)):
+        buf = torch.zeros(cap, dtype=t.dtype, device=t.device)
+        buf[: t.numel()] = t
+        gathered = [torch.empty_like(buf) for _ in range(world)]
+        dist.all_gather(gathered, buf, group=group)
+        out[name] = torch.cat([gathered[r][: sizes[r]] for r in range(world)])
+    out["budgets"], out["row_ptr"] = budgets, row_ptr
+    return out
+
+
 def plan_build(a: Adapter, ws: torch.Tensor | None = None) -> Adapter:
     """Fill the CSC and tile views of `a` (new tensors) and return it."""
     dev = a.row_ptr.device

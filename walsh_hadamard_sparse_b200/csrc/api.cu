@@ -620,4 +620,53 @@ qwha_status qwha_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32
                      "init_alloc");
 }
 
+qwha_status qwha_init_norms(const float *dWq, int32_t rows, int32_t d_in, double *e, void *stream) {
+  if (rows < 0 || d_in <= 0) return fail(QWHA_ERR_INVALID_ARG, "rows %d, d_in %d", rows, d_in);
+  if (rows == 0) return QWHA_OK;
+  QWHA_CHECK_PTR(dWq, "dWq");
+  QWHA_CHECK_PTR(e, "e");
+  StageScope sc(ST_INIT, 1, (cudaStream_t)stream);
+  return cuda_status(launch_init_norms(dWq, rows, d_in, e, (cudaStream_t)stream), "init_norms");
+}
+
+qwha_status qwha_init_budgets(const double *e, int32_t d_out, int32_t d_in, int64_t p, int32_t min_per_row,
+                              qwha_remainder mode, int32_t *budgets, int32_t *row_ptr, void *ws, size_t ws_bytes,
+                              void *stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(QWHA_ERR_INVALID_ARG, "d_out %d, d_in %d", d_out, d_in);
+  if (min_per_row < 0 || min_per_row > d_in) return fail(QWHA_ERR_INVALID_ARG, "min_per_row %d", min_per_row);
+  if (p < (int64_t)min_per_row * d_out || p > (int64_t)d_in * d_out || p > 2147483647LL)
+    return fail(QWHA_ERR_INVALID_ARG, "p = %lld outside [%lld, %lld]", (long long)p,
+                (long long)min_per_row * d_out, (long long)d_in * d_out);
+  if (mode != QWHA_REM_FEWEST_ALLOC && mode != QWHA_REM_LARGEST_ERROR)
+    return fail(QWHA_ERR_INVALID_ARG, "remainder mode %d", (int)mode);
+  QWHA_CHECK_PTR(e, "e");
+  QWHA_CHECK_PTR(budgets, "budgets");
+  QWHA_CHECK_PTR(row_ptr, "row_ptr");
+  qwha_status st = check_ws(ws, ws_bytes, init_workspace(d_out, d_in));
+  if (st != QWHA_OK) return st;
+  StageScope sc(ST_INIT, 1, (cudaStream_t)stream);
+  return cuda_status(launch_init_budgets(e, d_out, d_in, p, min_per_row, (int)mode, budgets, row_ptr, ws,
+                                         (cudaStream_t)stream),
+                     "init_budgets");
+}
+
+qwha_status qwha_init_select(const float *dWq, int32_t rows, int32_t d_in, int32_t had_block, const int32_t *budgets,
+                             const int32_t *row_ptr, int64_t p_local, int32_t *col_idx, float *coef, void *stream) {
+  if (rows < 0) return fail(QWHA_ERR_INVALID_ARG, "rows %d", rows);
+  qwha_status st = check_hadamard(d_in, had_block);
+  if (st != QWHA_OK) return st;
+  if (d_in > init_max_din()) return fail(QWHA_ERR_UNSUPPORTED, "d_in %d above %d", d_in, init_max_din());
+  if (p_local < 0 || p_local > 2147483647LL) return fail(QWHA_ERR_INVALID_ARG, "p_local %lld", (long long)p_local);
+  if (rows == 0 || p_local == 0) return QWHA_OK;
+  QWHA_CHECK_PTR(dWq, "dWq");
+  QWHA_CHECK_PTR(budgets, "budgets");
+  QWHA_CHECK_PTR(row_ptr, "row_ptr");
+  QWHA_CHECK_PTR(col_idx, "col_idx");
+  QWHA_CHECK_PTR(coef, "coef");
+  StageScope sc(ST_INIT, 1, (cudaStream_t)stream);
+  return cuda_status(launch_init_select(dWq, rows, d_in, had_block, budgets, row_ptr, p_local, col_idx, coef,
+                                        (cudaStream_t)stream),
+                     "init_select");
+}
+
 }  // extern "C"

@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kSelThreads)
     __syncthreads();
   }
   const int b = budgets[row];
-  int64_t start = row_ptr[row];
+  int64_t start = (int64_t)row_ptr[row] - row_ptr[0];  // row_ptr may be a slice of a longer one
   if (b <= 0 || start < 0 || start + b > p) return;
   const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)n));
   // largest |V| = smallest complemented magnitude bits
@@ -422,6 +422,29 @@ cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int3
   cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (p > 0) select_kernel<<<d_out, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_init_norms(const float *dW, int32_t rows, int32_t d_in, double *e, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  row_norm_kernel<<<rows, kNormThreads, 0, s>>>(dW, d_in, e);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_init_budgets(const double *e, int32_t d_out, int32_t d_in, int64_t p, int32_t min_per_row, int mode,
+                                int32_t *budgets, int32_t *row_ptr, void *ws, cudaStream_t s) {
+  unsigned char *capped = static_cast<unsigned char *>(ws) + align_up((size_t)d_out * 8, 256);
+  budget_kernel<<<1, kBudgetThreads, 0, s>>>(e, d_out, d_in, p, min_per_row, mode, budgets, row_ptr, capped);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_init_select(const float *dW, int32_t rows, int32_t d_in, int32_t had_block, const int32_t *budgets,
+                               const int32_t *row_ptr, int64_t p, int32_t *col_idx, float *coef, cudaStream_t s) {
+  if (rows <= 0 || p <= 0) return cudaSuccess;
+  const size_t smem = (size_t)d_in * sizeof(double);
+  cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  select_kernel<<<rows, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
   return cudaGetLastError();
 }
 
