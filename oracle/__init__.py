@@ -62,6 +62,7 @@ def _load():
                 "oracle_init_norms": [P, i32, i32, P],
                 "oracle_init_budgets": [P, i32, i32, i64, i32, i32, P, P],
                 "oracle_init_select": [P, i32, i32, i32, P, P, P, P],
+                "oracle_init_select_global": [P, i32, i32, i32, i64, i32, ctypes.c_uint64, P, P, P, P],
                 "oracle_plan_build": [i32, i32, i64, P, P, P, P, P],
             }
             for name, args in sig.items():
@@ -232,6 +233,22 @@ def init_select(dWq_rows, n: int, budgets, row_ptr):
     c = np.empty(cnt, dtype=np.float32)
     _check(_load().oracle_init_select(_p(w), rows, d_in, n, _p(b), _p(rp), _p(ci), _p(c)), "init_select")
     return ci, c
+
+
+def init_select_global(dWq, p: int, n: int, sel: str = "magnitude", seed: int = 0):
+    """E over the whole matrix (the pages' alternatives to AdaAlloc): "magnitude" = the p largest |V| (ties to the
+    lower flat index), "random" = the p smallest SplitMix64 keys; dict(budgets, row_ptr, col_idx, coef)."""
+    w = np.ascontiguousarray(dWq, dtype=np.float32)
+    d_out, d_in = w.shape
+    b = np.empty(d_out, dtype=np.int32)
+    rp = np.empty(d_out + 1, dtype=np.int32)
+    ci = np.empty(p, dtype=np.int32)
+    c = np.empty(p, dtype=np.float32)
+    s = {"magnitude": 0, "random": 1}[sel]
+    rc = _load().oracle_init_select_global(_p(w), d_out, d_in, n, int(p), s, ctypes.c_uint64(seed & (2**64 - 1)),
+                                           _p(b), _p(rp), _p(ci), _p(c))
+    _check(rc, "init_select_global")
+    return dict(budgets=b, row_ptr=rp, col_idx=ci, coef=c)
 
 
 def plan_build(row_ptr, col_idx, d_in: int):

@@ -442,6 +442,64 @@ int oracle_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, 
   return oracle_init_select(dWq, d_out, d_in, n, budgets, row_ptr, col_idx, coef);
 }
 
+// SplitMix64 (Steele, Lea and Flood, "Fast splittable pseudorandom number
+// generators", 2014): output n >= 1 of the generator seeded with `seed` is the
+// finaliser applied to seed + n * 0x9E3779B97F4A7C15 (mod 2^64).
+uint64_t splitmix64_output(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + n * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Selection over the whole matrix, the alternatives to AdaAlloc that the
+// pages compare it with (papernotes.org 消融实验, table 4: random and
+// magnitude selection; gist.science 2.2: they may cluster the parameters in
+// a few channels). V = dW_Q H (unnormalised, textbook stage order, double);
+// flat index j = i * d_in + k.
+//   sel 0 (magnitude): the p entries of largest |V|, ties to the lower j;
+//   sel 1 (random):    the p entries of smallest u_j = SplitMix64 output
+//                      j + 1 for `seed`, ties to the lower j;
+// c = float(V * (1/sqrt(n))) at E (the dense solution, as in AdaAlloc).
+// Outputs: budgets [d_out] (entries per row), row_ptr [d_out+1], col_idx [p]
+// ascending within a row, coef [p].
+int oracle_init_select_global(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, int64_t p, int32_t sel,
+                              uint64_t seed, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx, float *coef) {
+  if (!shape_ok(d_in, n) || d_out <= 0 || (sel != 0 && sel != 1)) return 1;
+  const int64_t N = (int64_t)d_out * d_in;
+  if (p < 0 || p > N || p > 2147483647LL) return 1;
+  std::vector<double> V((size_t)N);
+  parallel_for(d_out, [&](int64_t i) {
+    double *v = V.data() + i * d_in;
+    for (int k = 0; k < d_in; ++k) v[k] = (double)dWq[i * d_in + k];
+    for (int blk = 0; blk < d_in / n; ++blk) butterflies(v + (int64_t)blk * n, n);
+  });
+  std::vector<int64_t> order((size_t)N);
+  std::iota(order.begin(), order.end(), (int64_t)0);
+  if (sel == 0) {
+    std::sort(order.begin(), order.end(), [&](int64_t a, int64_t b) {
+      const double fa = std::fabs(V[a]), fb = std::fabs(V[b]);
+      return fa > fb || (fa == fb && a < b);
+    });
+  } else {
+    std::vector<uint64_t> u((size_t)N);
+    for (int64_t j = 0; j < N; ++j) u[j] = splitmix64_output(seed, (uint64_t)j + 1);
+    std::sort(order.begin(), order.end(), [&](int64_t a, int64_t b) { return u[a] < u[b] || (u[a] == u[b] && a < b); });
+  }
+  std::vector<int64_t> pick(order.begin(), order.begin() + p);
+  std::sort(pick.begin(), pick.end());  // row-major order = CSR order with ascending columns
+  for (int i = 0; i < d_out; ++i) budgets[i] = 0;
+  for (int64_t j : pick) ++budgets[j / d_in];
+  row_ptr[0] = 0;
+  for (int i = 0; i < d_out; ++i) row_ptr[i + 1] = row_ptr[i] + budgets[i];
+  const double inv = inv_sqrt(n);
+  for (int64_t q = 0; q < p; ++q) {
+    col_idx[q] = (int32_t)(pick[q] % d_in);
+    coef[q] = (float)(V[pick[q]] * inv);
+  }
+  return 0;
+}
+
 // Column view of the CSR pattern: for every column k the nonzeros j with
 // col_idx[j] == k, in increasing j: col_ptr [d_in+1], row_idx [p] (their rows),
 // perm [p] (their CSR positions).

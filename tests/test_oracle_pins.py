@@ -318,3 +318,68 @@ def test_plan_build_matches_scipy_csc():
     M.sort_indices()
     assert np.array_equal(cp, M.indptr) and np.array_equal(ri, M.indices)
     assert np.array_equal(pm, M.data.astype(np.int64) - 1)
+
+
+# --------------------------------------------------------------------------- selection over the whole matrix
+
+MASK64 = (1 << 64) - 1
+
+
+def splitmix64(seed, n):
+    """Output n (n >= 1) of SplitMix64 seeded with `seed`, from the generator's published definition."""
+    z = (seed + n * 0x9E3779B97F4A7C15) & MASK64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & MASK64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & MASK64
+    return z ^ (z >> 31)
+
+
+def test_splitmix64_published_outputs():
+    # the first outputs of the reference generator for seed 0, and the first for seed 1234567
+    assert [splitmix64(0, n) for n in (1, 2, 3)] == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+    assert splitmix64(1234567, 1) == 6457827717110365317
+
+
+def _expected_global(w, n, p, keys_lex):
+    """CSR of the p flat positions first in np.lexsort order of keys_lex (last key primary)."""
+    d_out, d_in = w.shape
+    order = np.lexsort(keys_lex)
+    pick = np.sort(order[:p])
+    rows, cols = pick // d_in, pick % d_in
+    budgets = np.bincount(rows, minlength=d_out).astype(np.int32)
+    rp = np.concatenate([[0], np.cumsum(budgets)]).astype(np.int32)
+    V = w.astype(np.float64) @ scipy.linalg.block_diag(*[scipy.linalg.hadamard(n)] * (d_in // n)).astype(np.float64)
+    coef = (V.reshape(-1)[pick] * (1.0 / np.sqrt(n))).astype(np.float32)  # c = float(V * (1/sqrt(n)))
+    return budgets, rp, cols.astype(np.int32), coef
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties"])
+def test_select_global_magnitude_matches_sort(kind):
+    g = rng_for(70, "global-mag", kind)
+    d_out, d_in, n, p = 24, 64, 32, 150
+    if kind == "ties":  # small integers: many equal |V|, the tie rule decides
+        w = g.integers(-1, 2, size=(d_out, d_in)).astype(np.float32)
+    else:
+        w = g.standard_normal((d_out, d_in)).astype(np.float32)
+    V = w.astype(np.float64) @ scipy.linalg.block_diag(*[scipy.linalg.hadamard(n)] * (d_in // n))
+    flat = np.arange(d_out * d_in)
+    b, rp, ci, cf = _expected_global(w, n, p, (flat, -np.abs(V.reshape(-1))))
+    got = oracle.init_select_global(w, p, n, "magnitude")
+    assert np.array_equal(got["budgets"], b) and np.array_equal(got["row_ptr"], rp)
+    assert np.array_equal(got["col_idx"], ci)
+    assert np.array_equal(got["coef"].view(np.uint32), cf.view(np.uint32))
+
+
+def test_select_global_random_matches_generator():
+    g = rng_for(71, "global-rand")
+    d_out, d_in, n, p, seed = 20, 32, 32, 97, 0xDEADBEEF12345
+    w = g.standard_normal((d_out, d_in)).astype(np.float32)
+    flat = np.arange(d_out * d_in)
+    u = np.array([splitmix64(seed, int(j) + 1) for j in flat], dtype=np.uint64)
+    b, rp, ci, cf = _expected_global(w, n, p, (flat, u))
+    got = oracle.init_select_global(w, p, n, "random", seed)
+    assert np.array_equal(got["budgets"], b) and np.array_equal(got["row_ptr"], rp)
+    assert np.array_equal(got["col_idx"], ci)
+    assert np.array_equal(got["coef"].view(np.uint32), cf.view(np.uint32))
+    # a uniform p-subset: another seed gives another one, with the same count
+    other = oracle.init_select_global(w, p, n, "random", seed + 1)
+    assert other["row_ptr"][-1] == p and not np.array_equal(other["col_idx"], got["col_idx"])
