@@ -294,6 +294,21 @@ def main():
         ev[1].record()
         torch.cuda.synchronize()
         init_ms.append(ev[0].elapsed_time(ev[1]))
+    # the pages' alternatives to AdaAlloc (whole-matrix magnitude top-p, seeded random E), timed the same way
+    sel_ms = {}
+    for sel in ("magnitude", "random"):
+        sws = torch.empty(W.workspace_size(6, spec.d_out, spec.d_in, spec.p, 0, False), dtype=torch.uint8, device=dev)
+        W.init_select_global(dWq, spec.p, spec.had_block, sel, 1, ws=sws)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(3):
+            ev[0].record()
+            W.init_select_global(dWq, spec.p, spec.had_block, sel, 1, ws=sws)
+            ev[1].record()
+            torch.cuda.synchronize()
+            ts.append(ev[0].elapsed_time(ev[1]))
+        sel_ms[sel] = statistics.median(ts)
+        del sws
     a = W.Adapter(spec.d_in, spec.d_out, spec.had_block, spec.p, e["row_ptr"], e["col_idx"], e["coef"])
     W.plan_build(a)  # the views the sparse backward needs
 
@@ -492,7 +507,10 @@ def main():
         },
         "init": {"ms": init_med, "alg_GBps": init_bytes / (init_med / 1e3) / 1e9,
                  "frac_hbm": init_bytes / (init_med / 1e3) / 1e9 / peaks["hbm_gbs"],
-                 "what": "AdaAlloc on dW_Q (4096 x 4096 fp32): norms, budgets, fp64 transform, top-k; one-off per layer"},
+                 "what": "AdaAlloc on dW_Q (4096 x 4096 fp32): norms, budgets, fp64 transform, top-k; one-off per layer",
+                 "select_global_ms": sel_ms,
+                 "select_global_what": ("whole-matrix selection (magnitude top-p; seeded random E): fp64 transform of "
+                                        "all rows kept in HBM, 8 radix passes over 16.8 M keys, per-row compaction")},
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -139,7 +139,8 @@ typedef enum {
   QWHA_OP_INIT = 2,      /* qwha_init_alloc */
   QWHA_OP_PLAN = 3,      /* qwha_plan_build */
   QWHA_OP_FWD_DENSE = 4, /* qwha_adapter_fwd, algo dense */
-  QWHA_OP_BWD_DENSE = 5  /* qwha_adapter_bwd, algo dense */
+  QWHA_OP_BWD_DENSE = 5, /* qwha_adapter_bwd, algo dense */
+  QWHA_OP_SELECT_GLOBAL = 6 /* qwha_init_select_global */
 } qwha_op;
 
 /* Z = X H row by row: x and z are [rows, n] of dtype dt (device), each row
@@ -217,6 +218,28 @@ qwha_status qwha_init_budgets(const double *e, int32_t d_out, int32_t d_in, int6
 qwha_status qwha_init_select(const float *dWq, int32_t rows, int32_t d_in, int32_t had_block,
                              const int32_t *budgets, const int32_t *row_ptr, int64_t p_local,
                              int32_t *col_idx, float *coef, void *stream);
+
+/* Selection rules the pages compare AdaAlloc with (papernotes.org 消融实验,
+ * table 4; gist.science 2.2 notes that they may crowd the parameters into a few
+ * channels): E is chosen over the whole d_out x d_in matrix, not per channel. */
+typedef enum {
+  QWHA_SEL_MAGNITUDE = 0, /* the p largest |V|, V = dWq H_unnormalised as in qwha_init_alloc */
+  QWHA_SEL_RANDOM = 1     /* p positions uniformly at random (seeded) */
+} qwha_selection;
+
+/* E and c by a whole-matrix rule. Flat index j = i * d_in + k; key_j is the
+ * magnitude (largest |V| first) or, for QWHA_SEL_RANDOM, output j + 1 of the
+ * SplitMix64 generator seeded with `seed` (smallest first); E = the p first
+ * keys, equal keys in increasing j; c = float(V * 1/sqrt(had_block)) at E
+ * (the dense solution). Outputs (device) as qwha_init_alloc: budgets [d_out]
+ * (E's count per row, no minimum), row_ptr [d_out+1], col_idx [p] ascending
+ * within a row, coef [p]. Requires 0 <= p <= d_in*d_out, p < 2^31,
+ * d_in <= 16384; ws: qwha_workspace_size(QWHA_OP_SELECT_GLOBAL, ...) bytes
+ * (V in fp64 for every entry, plus a few arrays of d_out). Deterministic. */
+qwha_status qwha_init_select_global(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block,
+                                    int64_t p, qwha_selection sel, uint64_t seed, int32_t *budgets,
+                                    int32_t *row_ptr, int32_t *col_idx, float *coef, void *ws,
+                                    size_t ws_bytes, void *stream);
 
 /* Index views of E for the backward (E stays fixed while c trains,
  * papernotes.org 整体框架): from the CSR row_ptr/col_idx (device) write the

@@ -230,6 +230,34 @@ def test_init_split_steps_bitexact(shards, mode):
         assert np.array_equal(got["coef"].view(np.uint32), ref["coef"].view(np.uint32))
 
 
+@pytest.mark.parametrize(
+    "d_out,d_in,n,p,sel,kind",
+    [
+        (96, 128, 128, 96 * 9 + 5, "magnitude", "normal"),
+        (80, 3 * 64, 64, 700, "magnitude", "normal"),  # block-diagonal transform
+        (48, 32, 32, 300, "magnitude", "ties"),  # integer data: many equal |V|, decided by the flat index
+        (300, 512, 512, 300 * 20, "random", "normal"),
+        (64, 64, 64, 64 * 64, "random", "normal"),  # p = all entries
+        (64, 64, 64, 1, "magnitude", "normal"),
+        (64, 64, 64, 0, "random", "normal"),
+    ],
+)
+def test_select_global_bitexact(d_out, d_in, n, p, sel, kind):
+    """Whole-matrix selection (magnitude top-p, seeded random E) bit for bit against the oracle."""
+    W = _W()
+    g = rng_for(36, "select-global", d_out, d_in, p, sel, kind)
+    if kind == "ties":
+        w = g.integers(-1, 2, size=(d_out, d_in)).astype(np.float32)
+    else:
+        w = g.standard_normal((d_out, d_in)).astype(np.float32) * np.float32(0.01)
+    seed = 0x5EED0000 + p
+    got = W.init_select_global(to_dev(w), p, n, sel, seed)
+    ref = oracle.init_select_global(w, p, n, sel, seed)
+    for k in ("budgets", "row_ptr", "col_idx"):
+        assert np.array_equal(got[k].cpu().numpy(), ref[k]), k
+    assert np.array_equal(got["coef"].cpu().numpy().view(np.uint32), ref["coef"].view(np.uint32))
+
+
 # --------------------------------------------------------------------------- forward / backward
 
 

@@ -88,3 +88,19 @@ def test_init_sweep_full_size_bitexact():
         for k in ("budgets", "row_ptr", "col_idx"):
             assert np.array_equal(got[k].cpu().numpy(), ref[k]), (spec.name, k)
         assert np.array_equal(got["coef"].cpu().numpy().view(np.uint32), ref["coef"].view(np.uint32)), spec.name
+
+
+@pytest.mark.parametrize("sel", ["magnitude", "random"])
+def test_select_global_full_size_bitexact(sel):
+    """The pages' alternatives to AdaAlloc on the q_proj layer (4096 x 4096, p = 524288): whole-matrix magnitude
+    top-p and seeded random E, budgets, E and c bit for bit against the oracle."""
+    import torch
+    import walsh_hadamard_sparse_b200 as W
+
+    spec = CONFIGS["q_proj"][0]
+    w = layer_inputs(spec, 0, "q_proj", parts=("W",))["dWq"]
+    got = W.init_select_global(torch.from_numpy(w).cuda(), spec.p, spec.had_block, sel, 2024)
+    ref = oracle.init_select_global(w, spec.p, spec.had_block, sel, 2024)
+    for k in ("budgets", "row_ptr", "col_idx"):
+        assert np.array_equal(got[k].cpu().numpy(), ref[k]), (sel, k)
+    assert np.array_equal(got["coef"].cpu().numpy().view(np.uint32), ref["coef"].view(np.uint32)), sel

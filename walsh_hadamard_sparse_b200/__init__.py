@@ -17,6 +17,7 @@ from .api import (  # noqa: F401
     init_budgets,
     init_norms,
     init_select,
+    init_select_global,
     plan_build,
     plan_tiles,
     shard_rows,

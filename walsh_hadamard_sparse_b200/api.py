@@ -15,7 +15,8 @@ import torch
 from ._lib import QwhaAdapter, QwhaQweight, check, lib
 
 F32, BF16 = 0, 1
-OP_FWD, OP_BWD, OP_INIT, OP_PLAN, OP_FWD_DENSE, OP_BWD_DENSE = 0, 1, 2, 3, 4, 5
+OP_FWD, OP_BWD, OP_INIT, OP_PLAN, OP_FWD_DENSE, OP_BWD_DENSE, OP_SELECT_GLOBAL = 0, 1, 2, 3, 4, 5, 6
+SELECTION = {"magnitude": 0, "random": 1}
 ALGO = {"sparse": 0, "dense": 1}
 REMAINDER = {"fewest": 0, "largest": 1}
 
@@ -171,6 +172,28 @@ def init_alloc(dWq: torch.Tensor, p: int, had_block: int, min_per_row: int = 2, 
                                _ptr(out["budgets"]), _ptr(out["row_ptr"]), _ptr(out["col_idx"]), _ptr(out["coef"]),
                                _ptr(ws), 0 if ws is None else ws.numel(), _stream())
     check(rc, "qwha_init_alloc")
+    out["col_idx"], out["coef"] = out["col_idx"][:p], out["coef"][:p]
+    return out
+
+
+def init_select_global(dWq: torch.Tensor, p: int, had_block: int, sel: str = "magnitude", seed: int = 0,
+                       ws: torch.Tensor | None = None) -> dict:
+    """E and c by a whole-matrix rule ("magnitude": the p largest |V|; "random": p seeded uniform positions):
+    dict(budgets, row_ptr, col_idx, coef)."""
+    d_out, d_in = dWq.shape
+    dev = dWq.device
+    out = dict(
+        budgets=torch.empty(d_out, dtype=torch.int32, device=dev),
+        row_ptr=torch.empty(d_out + 1, dtype=torch.int32, device=dev),
+        col_idx=torch.empty(max(p, 1), dtype=torch.int32, device=dev),
+        coef=torch.empty(max(p, 1), dtype=torch.float32, device=dev),
+    )
+    need = workspace_size(OP_SELECT_GLOBAL, d_out, d_in, p, 0, False)
+    ws = _ws(need, dev) if ws is None else ws
+    rc = lib().qwha_init_select_global(_ptr(dWq), d_out, d_in, had_block, p, SELECTION[sel], seed & (2**64 - 1),
+                                       _ptr(out["budgets"]), _ptr(out["row_ptr"]), _ptr(out["col_idx"]),
+                                       _ptr(out["coef"]), _ptr(ws), 0 if ws is None else ws.numel(), _stream())
+    check(rc, "qwha_init_select_global")
     out["col_idx"], out["coef"] = out["col_idx"][:p], out["coef"][:p]
     return out
 

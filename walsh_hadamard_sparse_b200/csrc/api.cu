@@ -390,6 +390,7 @@ size_t qwha_workspace_size(qwha_op op, int32_t d_out, int32_t d_in, int64_t p, i
     case QWHA_OP_PLAN: return plan_workspace(d_out, d_in);
     case QWHA_OP_FWD_DENSE: return fwd_dense_ws(d_out, d_in);
     case QWHA_OP_BWD_DENSE: return bwd_dense_ws(d_out, d_in, T);
+    case QWHA_OP_SELECT_GLOBAL: return select_global_workspace(d_out, d_in);
   }
   return 0;
 }
@@ -618,6 +619,30 @@ qwha_status qwha_init_alloc(const float *dWq, int32_t d_out, int32_t d_in, int32
   return cuda_status(launch_init_alloc(dWq, d_out, d_in, had_block, p, min_per_row, (int)mode, budgets, row_ptr,
                                        col_idx, coef, ws, (cudaStream_t)stream),
                      "init_alloc");
+}
+
+qwha_status qwha_init_select_global(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p,
+                                    qwha_selection sel, uint64_t seed, int32_t *budgets, int32_t *row_ptr,
+                                    int32_t *col_idx, float *coef, void *ws, size_t ws_bytes, void *stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(QWHA_ERR_INVALID_ARG, "d_out %d, d_in %d", d_out, d_in);
+  qwha_status st = check_hadamard(d_in, had_block);
+  if (st != QWHA_OK) return st;
+  if (d_in > init_max_din()) return fail(QWHA_ERR_UNSUPPORTED, "d_in %d above %d", d_in, init_max_din());
+  if (p < 0 || p > (int64_t)d_in * d_out || p > 2147483647LL)
+    return fail(QWHA_ERR_INVALID_ARG, "p = %lld outside [0, %lld]", (long long)p, (long long)d_in * d_out);
+  if (sel != QWHA_SEL_MAGNITUDE && sel != QWHA_SEL_RANDOM) return fail(QWHA_ERR_INVALID_ARG, "selection %d", (int)sel);
+  QWHA_CHECK_PTR(dWq, "dWq");
+  QWHA_CHECK_PTR(budgets, "budgets");
+  QWHA_CHECK_PTR(row_ptr, "row_ptr");
+  if (p > 0) {
+    QWHA_CHECK_PTR(col_idx, "col_idx");
+    QWHA_CHECK_PTR(coef, "coef");
+  }
+  if ((st = check_ws(ws, ws_bytes, select_global_workspace(d_out, d_in))) != QWHA_OK) return st;
+  StageScope sc(ST_INIT, 21, (cudaStream_t)stream);
+  return cuda_status(launch_select_global(dWq, d_out, d_in, had_block, p, (int)sel, seed, budgets, row_ptr, col_idx,
+                                          coef, ws, (cudaStream_t)stream),
+                     "init_select_global");
 }
 
 qwha_status qwha_init_norms(const float *dWq, int32_t rows, int32_t d_in, double *e, void *stream) {

@@ -21,6 +21,8 @@
 // Kernels: row_norm (one CTA per row), budget (one CTA), select (one CTA per
 // row: butterflies in shared memory, radix select, ordered compaction).
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -349,18 +351,12 @@ __global__ void __launch_bounds__(kBudgetThreads)
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads)
-    select_kernel(const float *__restrict__ dW, int d_in, int n, const int32_t *__restrict__ budgets,
-                  const int32_t *__restrict__ row_ptr, int64_t p, int32_t *__restrict__ col_idx,
-                  float *__restrict__ coef) {
-  extern __shared__ __align__(16) double v[];  // d_in values of the row
-  __shared__ uint32_t hist[256];
-  __shared__ int64_t sh64[kSelThreads];
-  const int64_t row = blockIdx.x;
-  const float *w = dW + row * d_in;
+// v[0..d_in) = w[0..d_in) H_unnormalised per block of n, fp64 butterflies in
+// the textbook stage order (three stages per pass over aligned groups of 8);
+// v is shared memory, every thread of the block takes part.
+__device__ void row_transform_fp64(const float *__restrict__ w, int d_in, int n, double *v) {
   for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[k] = (double)w[k];
   __syncthreads();
-  // textbook stage order, three stages per pass over aligned groups of 8
   const int logn = 31 - __clz(n);
   for (int s = 0; s < logn; s += 3) {
     const int nb = min(3, logn - s);
@@ -381,6 +377,17 @@ __global__ void __launch_bounds__(kSelThreads)
     }
     __syncthreads();
   }
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+    select_kernel(const float *__restrict__ dW, int d_in, int n, const int32_t *__restrict__ budgets,
+                  const int32_t *__restrict__ row_ptr, int64_t p, int32_t *__restrict__ col_idx,
+                  float *__restrict__ coef) {
+  extern __shared__ __align__(16) double v[];  // d_in values of the row
+  __shared__ uint32_t hist[256];
+  __shared__ int64_t sh64[kSelThreads];
+  const int64_t row = blockIdx.x;
+  row_transform_fp64(dW + row * d_in, d_in, n, v);
   const int b = budgets[row];
   int64_t start = (int64_t)row_ptr[row] - row_ptr[0];  // row_ptr may be a slice of a longer one
   if (b <= 0 || start < 0 || start + b > p) return;
@@ -395,6 +402,197 @@ __global__ void __launch_bounds__(kSelThreads)
   ordered_take(d_in, K, need, key, ok,
                [&](int k, int64_t slot) {
                  if (slot < b) {
+                   col_idx[start + slot] = k;
+                   coef[start + slot] = __double2float_rn(__dmul_rn(v[k], inv));
+                 }
+               },
+               sh64);
+}
+
+// ------------------------------------------------------------ selection over the whole matrix
+//
+// E = the p smallest keys over all d_out x d_in entries, equal keys taken in
+// increasing flat index j = i * d_in + k: magnitude selection (key = the
+// complemented magnitude bits of V, so the largest |V| come first) or random
+// selection (key = SplitMix64 output j + 1 for the seed: Steele, Lea and
+// Flood, 2014). V (fp64, unnormalised transform) is kept in the workspace: the
+// magnitude keys read it in every pass and c = float(V / sqrt(n)) at E.
+
+constexpr int kGselThreads = 256;
+
+struct GselState {
+  unsigned long long prefix;  // digits of K fixed so far
+  long long need;             // how many keys equal to the prefix are still to be taken
+  uint32_t hist[256];
+};
+
+__device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + n * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ uint64_t gsel_key(const double *__restrict__ V, int64_t j, int sel, uint64_t seed) {
+  if (sel == 0) return ~((uint64_t)__double_as_longlong(V[j]) & 0x7fffffffffffffffull);
+  return splitmix64_at(seed, (uint64_t)j + 1);
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+    gsel_transform_kernel(const float *__restrict__ dW, int d_in, int n, double *__restrict__ V) {
+  extern __shared__ __align__(16) double v[];
+  const int64_t row = blockIdx.x;
+  row_transform_fp64(dW + row * d_in, d_in, n, v);
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) V[row * d_in + k] = v[k];
+}
+
+__global__ void gsel_init_kernel(GselState *st, int64_t p) {
+  if (threadIdx.x == 0) {
+    st->prefix = 0;
+    st->need = p;
+  }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) st->hist[i] = 0;
+}
+
+// Histogram of digit `shift` over the keys that match the prefix so far.
+__global__ void __launch_bounds__(kGselThreads)
+    gsel_hist_kernel(const double *__restrict__ V, int64_t N, int sel, uint64_t seed, int shift, GselState *st) {
+  __shared__ uint32_t hist[256];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const uint64_t prefix = st->prefix;
+  const uint64_t hi_mask = shift == 56 ? 0 : (~0ull << (shift + 8));
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t n_round = (N + stride - 1) / stride * stride;  // whole warps iterate together
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n_round; j += stride) {
+    int bin = 256;
+    if (j < N) {
+      const uint64_t k = gsel_key(V, j, sel, seed);
+      if ((k & hi_mask) == (prefix & hi_mask)) bin = (int)((k >> shift) & 255);
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+    if (hist[i]) atomicAdd(&st->hist[i], hist[i]);
+}
+
+// One warp: the digit that holds the need-th key, then clear the histogram.
+__global__ void gsel_pick_kernel(GselState *st, int shift) {
+  const int lane = threadIdx.x;
+  const long long need = st->need;
+  uint32_t c[8];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = st->hist[8 * lane + j];
+    mine += c[j];
+  }
+  uint32_t incl = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const long long excl = (long long)(incl - mine);
+  const bool hit = (excl < need && (long long)incl >= need) || (lane == 0 && need <= 0);
+  const unsigned who = __ballot_sync(0xffffffffu, hit);
+  if (hit) {
+    long long cum = excl;
+    int d = 8 * lane + 7;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (cum + c[j] >= need) {
+        d = 8 * lane + j;
+        break;
+      }
+      cum += c[j];
+    }
+    st->prefix |= (unsigned long long)d << shift;
+    st->need = need - cum;
+  } else if (who == 0 && lane == 31) {
+    st->prefix |= 255ull << shift;
+    st->need = need - (long long)incl;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 8; ++j) st->hist[8 * lane + j] = 0;
+}
+
+// Per row: keys below K and keys equal to K.
+__global__ void __launch_bounds__(kGselThreads)
+    gsel_count_kernel(const double *__restrict__ V, int d_in, int sel, uint64_t seed, const GselState *st,
+                      int32_t *__restrict__ lt, int32_t *__restrict__ eq) {
+  __shared__ int32_t sh[kGselThreads];
+  const uint64_t K = st->prefix;
+  const int64_t row = blockIdx.x;
+  int a = 0, b = 0;
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) {
+    const uint64_t key = gsel_key(V, row * d_in + k, sel, seed);
+    a += key < K;
+    b += key == K;
+  }
+  const int la = block_sum(a, sh), lb = block_sum(b, sh);
+  if (threadIdx.x == 0) {
+    lt[row] = la;
+    eq[row] = lb;
+  }
+}
+
+// One CTA: rows take all their keys below K and, in row order, the first
+// `need` keys equal to K; budgets and row_ptr follow.
+__global__ void __launch_bounds__(kBudgetThreads)
+    gsel_budget_kernel(const int32_t *__restrict__ lt, const int32_t *__restrict__ eq, int d_out, const GselState *st,
+                       int32_t *__restrict__ take_eq, int32_t *__restrict__ budgets, int32_t *__restrict__ row_ptr) {
+  __shared__ int64_t sh64[kBudgetThreads];
+  const int t = threadIdx.x;
+  const int64_t need = st->need;
+  int64_t eq_carry = 0, b_carry = 0;
+  if (t == 0) row_ptr[0] = 0;
+  for (int base = 0; base < d_out; base += blockDim.x) {
+    const int i = base + t;
+    const int64_t e = i < d_out ? eq[i] : 0;
+    int64_t tot;
+    const int64_t before = eq_carry + block_excl_scan(e, sh64, &tot);
+    eq_carry += tot;
+    int64_t take = need - before;
+    take = take < 0 ? 0 : (take > e ? e : take);
+    const int64_t bud = i < d_out ? lt[i] + take : 0;
+    const int64_t ex = block_excl_scan(bud, sh64, &tot);
+    if (i < d_out) {
+      take_eq[i] = (int32_t)take;
+      budgets[i] = (int32_t)bud;
+      row_ptr[i + 1] = (int32_t)(b_carry + ex + bud);
+    }
+    b_carry += tot;
+  }
+}
+
+// Per row: the selected columns in increasing order, with c = float(V / sqrt(n)).
+__global__ void __launch_bounds__(kSelThreads)
+    gsel_take_kernel(const double *__restrict__ V, int d_in, int n, int sel, uint64_t seed, const GselState *st,
+                     const int32_t *__restrict__ take_eq, const int32_t *__restrict__ row_ptr, int64_t p,
+                     int32_t *__restrict__ col_idx, float *__restrict__ coef) {
+  extern __shared__ __align__(16) double v[];
+  __shared__ int64_t sh64[kSelThreads];
+  const int64_t row = blockIdx.x;
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[k] = V[row * d_in + k];
+  __syncthreads();
+  const int64_t start = row_ptr[row];
+  const int64_t cnt = (int64_t)row_ptr[row + 1] - start;
+  if (cnt <= 0 || start < 0 || start + cnt > p) return;
+  const uint64_t K = st->prefix;
+  const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)n));
+  auto key = [&](int k) -> uint64_t {
+    if (sel == 0) return ~((uint64_t)__double_as_longlong(v[k]) & 0x7fffffffffffffffull);
+    return splitmix64_at(seed, (uint64_t)(row * d_in + k) + 1);
+  };
+  auto ok = [&](int) { return true; };
+  ordered_take(d_in, K, take_eq[row], key, ok,
+               [&](int k, int64_t slot) {
+                 if (slot < cnt) {
                    col_idx[start + slot] = k;
                    coef[start + slot] = __double2float_rn(__dmul_rn(v[k], inv));
                  }
@@ -422,6 +620,44 @@ cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int3
   cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (p > 0) select_kernel<<<d_out, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
+  return cudaGetLastError();
+}
+
+size_t select_global_workspace(int32_t d_out, int32_t d_in) {
+  return align_up((size_t)d_out * d_in * 8, 256) + align_up(sizeof(GselState), 256) + 3 * align_up((size_t)d_out * 4, 256);
+}
+
+cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p, int sel,
+                                 uint64_t seed, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx, float *coef,
+                                 void *ws, cudaStream_t s) {
+  char *w = static_cast<char *>(ws);
+  double *V = reinterpret_cast<double *>(w);
+  w += align_up((size_t)d_out * d_in * 8, 256);
+  GselState *st = reinterpret_cast<GselState *>(w);
+  w += align_up(sizeof(GselState), 256);
+  int32_t *lt = reinterpret_cast<int32_t *>(w);
+  w += align_up((size_t)d_out * 4, 256);
+  int32_t *eq = reinterpret_cast<int32_t *>(w);
+  w += align_up((size_t)d_out * 4, 256);
+  int32_t *take = reinterpret_cast<int32_t *>(w);
+  const size_t smem = (size_t)d_in * sizeof(double);
+  cudaError_t e = cudaFuncSetAttribute(gsel_transform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gsel_take_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t N = (int64_t)d_out * d_in;
+  gsel_transform_kernel<<<d_out, kSelThreads, smem, s>>>(dW, d_in, had_block, V);
+  gsel_init_kernel<<<1, 256, 0, s>>>(st, p);
+  const int64_t grid = std::min<int64_t>(cdiv(N, (int64_t)kGselThreads), (int64_t)sm_count() * 8);
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    gsel_hist_kernel<<<(unsigned)grid, kGselThreads, 0, s>>>(V, N, sel, seed, shift, st);
+    gsel_pick_kernel<<<1, 32, 0, s>>>(st, shift);
+  }
+  gsel_count_kernel<<<d_out, kGselThreads, 0, s>>>(V, d_in, sel, seed, st, lt, eq);
+  gsel_budget_kernel<<<1, kBudgetThreads, 0, s>>>(lt, eq, d_out, st, take, budgets, row_ptr);
+  if (p > 0)
+    gsel_take_kernel<<<d_out, kSelThreads, smem, s>>>(V, d_in, had_block, sel, seed, st, take, row_ptr, p, col_idx,
+                                                      coef);
   return cudaGetLastError();
 }
 

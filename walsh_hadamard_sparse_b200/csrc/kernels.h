@@ -57,6 +57,10 @@ namespace qwha {
 // AdaAlloc (init.cu)
 size_t init_workspace(int32_t d_out, int32_t d_in);
 int init_max_din();
+size_t select_global_workspace(int32_t d_out, int32_t d_in);
+cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p, int sel,
+                                 uint64_t seed, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx, float *coef,
+                                 void *ws, cudaStream_t s);
 cudaError_t launch_init_norms(const float *dW, int32_t rows, int32_t d_in, double *e, cudaStream_t s);
 cudaError_t launch_init_budgets(const double *e, int32_t d_out, int32_t d_in, int64_t p, int32_t min_per_row, int mode,
                                 int32_t *budgets, int32_t *row_ptr, void *ws, cudaStream_t s);
