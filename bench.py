@@ -476,9 +476,12 @@ def main():
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host_act = {"X": act["X"][:64].astype(np.float64), "dY": act["dY"][:64].astype(np.float64)}
+        host_act = {"X": act["X"][:512].astype(np.float64), "dY": act["dY"][:512].astype(np.float64)}
+        # size the sample for ~15 s of host work: a call costs a fixed part (dequantizing W_Q) plus a part per token
         _, t1, cores = oracle_tokens_per_s(spec, d, host_act["X"], host_act["dY"], 1)
-        toks = int(max(1, min(64, 15.0 / max(t1, 1e-3))))
+        _, t2, cores = oracle_tokens_per_s(spec, d, host_act["X"], host_act["dY"], 2)
+        per_tok = max(t2 - t1, 1e-3)
+        toks = int(max(1, min(512, (15.0 - max(t1 - per_tok, 0.0)) / per_tok)))
         rate, dt, cores = oracle_tokens_per_s(spec, d, host_act["X"], host_act["dY"], toks)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{toks} tokens of the same layer (Y, dX for them; dc over all {spec.p} coefficients), "
