@@ -2,13 +2,17 @@
 """Throughput of one Walsh-Hadamard-adapted linear layer (forward + backward) on B200.
 
 A step is one pass of the whole hot path over one batch of seeded synthetic
-tokens: forward transform Z = X H, sparse product, dequantized base GEMM with
-the adapter term in its epilogue; backward coefficient gradient (SDDMM), CSC
-gather + transform, base GEMM for dX; and, with N > 1 GPUs, the data-parallel
-sum of the coefficient gradients (NCCL all-reduce). The workload is the
-LLaMA-7B q_proj shape: d_in = d_out = 4096, 8192 tokens per GPU (16 x 512),
-4-bit group-128 round-to-nearest base weight, p = 524288 coefficients chosen
-by AdaAlloc. AdaAlloc itself (a one-off per layer) is timed separately.
+tokens: the forward (Z = X H and Y = X W_Q^T + alpha Z F^T) and the backward
+(dc at E and dX = dY W_Q + alpha dY F H) of one adapted layer with its base
+GEMMs, and, with N > 1 GPUs, the data-parallel sum of the coefficient
+gradients (NCCL all-reduce). The headline runs the dense algorithm (the
+adapter folded into W_eff = W_Q + alpha F H and three tcgen05 GEMMs, dc from
+the sampled epilogue of dY^T Z); the same run times the sparse algorithm
+(segment SpMM, tiled SDDMM, CSC gather on the FMA units) under paths.sparse.
+The workload is the LLaMA-7B q_proj shape: d_in = d_out = 4096, 8192 tokens
+per GPU (16 x 512), 4-bit group-128 round-to-nearest base weight, p = 524288
+coefficients chosen by AdaAlloc. AdaAlloc and the whole-matrix selection
+rules (one-off per layer) are timed separately.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun every rank runs its own tokens; rank 0 prints one JSON line.
