@@ -347,6 +347,29 @@ def test_base_gemm_forward_backward(d_in, d_out, n, T, bits, group, algo):
     assert rel_fro(host(Yb), L["X"].astype(np.float64) @ Wq.T) <= TOL_BF16
 
 
+@pytest.mark.parametrize("d_in,d_out,n,T", [(4096, 512, 4096, 300), (3 * 2048, 384, 2048, 129), (4096, 256, 4096, 8)])
+def test_dense_forward_fused_transform(d_in, d_out, n, T):
+    """The dense forward with Hadamard blocks of 2048 / 4096 writes Z from extra warps of the GEMM launch: Z bit for
+    bit what the standalone transform gives, Y and dX against the oracle (ragged token counts, several blocks)."""
+    import torch
+
+    W = _W()
+    L = synth_layer(41, d_in, d_out, n, T, d_out * 24, "bf16", bits=4, group=128, pattern="random")
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"], algo="dense")
+    wq = dev_qweight(L)
+    Xd, dYd = dev_act(L["X"], "bf16"), dev_act(L["dY"], "bf16")
+    Z, Y = W.adapter_fwd(a, Xd, 0.9, wq=wq)
+    dc, dX = W.adapter_bwd(a, dYd, Z, 0.9, wq=wq)
+    Zs = W.fwht(Xd, n)
+    torch.cuda.synchronize()
+    assert torch.equal(Z, Zs)
+    Wq = oracle.dequant(L["qweight"], L["scales"], L["zeros"], 4, 128, d_out, d_in)
+    _, Yr = oracle.adapter_fwd(L["rp"], L["ci"], L["cf"], L["X"], d_out, n, 0.9, Wq, want_z=False)
+    dXr = oracle.adapter_bwd_dx(L["rp"], L["ci"], L["cf"], L["dY"], d_in, n, 0.9, Wq)
+    errs = dict(Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr))
+    assert all(v <= TOL_BF16 for v in errs.values()), errs
+
+
 def test_dense_long_rows_with_base():
     """W_eff for rows with more nonzeros than the transform stages per row block
     (700 per row; the rest is read straight from the CSR arrays), 4-bit g128."""

@@ -425,6 +425,19 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
     StageScope sc(ST_GEMM_FWD, 1, s);
     return cuda_status(launch_gemm_nt(X, weff, nullptr, Y, false, T, a->d_out, a->d_in, s), "GEMM");
   }
+  if (dense && gemm_fused_fwht_supported(T, logn)) {
+    // W_eff, then one launch for Y = X W_eff^T whose extra warps write Z = X H
+    // (kept for the backward) while the tensor cores run the GEMM.
+    void *weff = a->weff ? a->weff : ws;
+    {
+      StageScope sc(ST_WEFF, 1, s);
+      e = launch_weff(a, wq, alpha, weff, s);
+    }
+    if (e != cudaSuccess) return cuda_status(e, "W_eff");
+    StageScope sc(ST_GEMM_FWD, 1, s);
+    return cuda_status(launch_gemm_fwd_fused(X, weff, Y, T, a->d_out, a->d_in, Z_out, logn, inv, s),
+                       "GEMM + transform");
+  }
   if (dense) {
     // Z = X H (kept for the backward) on the auxiliary stream, concurrently
     // with W_eff and Y = X W_eff^T on the caller's stream.

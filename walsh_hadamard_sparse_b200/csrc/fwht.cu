@@ -24,6 +24,7 @@
 // inputs are prefetched with cp.async into shared memory during the arithmetic.
 
 #include "common.cuh"
+#include "fwht_body.cuh"
 #include "kernels.h"
 
 namespace qwha {
@@ -31,190 +32,12 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <int LOGN, int V>
-struct Geo {
-  static constexpr int N = 1 << LOGN;
-  static constexpr int LV = V == 8 ? 3 : 2;
-  static constexpr int RB = (LOGN + 1) / 2;
-  static constexpr int R = 1 << RB;
-  static constexpr int PB = LOGN - RB;
-  static constexpr int P = 1 << PB;
-  static constexpr int NB = 2 * RB - LOGN;  // batch bits in phase B (0 or 1)
-  static constexpr int HB = RB - LV;        // high bits in phase-A registers
-  static constexpr int S0 = 5 - LV;
-  static constexpr int S1 = PB < S0 ? PB : S0;
-  static constexpr int S = (HB - NB) < S1 ? (HB - NB) : S1;  // swizzle bits
-  static constexpr int SMASK = (1 << S) - 1;
-  static_assert(HB >= NB && HB >= 0 && PB >= LV, "row too short for this layout");
-  static_assert(P <= kThreads, "row too long for this layout");
-
-  // element index of register q of thread t, phase A
-  __device__ __forceinline__ static int eA(int t, int q) {
-    return (q & (V - 1)) | (t << LV) | ((q >> LV) << (LV + PB));
-  }
-  // element index of register q of thread t, phase B
-  __device__ __forceinline__ static int eB(int t, int q) {
-    return (t & (V - 1)) | ((q & (P - 1)) << LV) | ((t >> LV) << (LV + PB)) |
-           ((q >> PB) << (LV + PB + HB - NB));
-  }
-  // swizzled position in the transpose buffer
-  __device__ __forceinline__ static int phys(int e) {
-    return e ^ (((e >> (LV + PB)) & SMASK) << LV);
-  }
-};
-
-template <typename T, int V>
-__device__ __forceinline__ void store_group(T *p, const float *i) {
-  constexpr int NU = V * (int)sizeof(T) / 16;
-#pragma unroll
-  for (int u = 0; u < NU; ++u) st_stream(p + u * io<T>::kVec, io<T>::pack(i + u * io<T>::kVec));
-}
-
-// Butterflies on register-index bits [B0, B0 + NBITS) of v[0..R).
-template <int R, int B0, int NBITS>
-__device__ __forceinline__ void butterflies(float *v) {
-#pragma unroll
-  for (int b = B0; b < B0 + NBITS; ++b) {
-    const int h = 1 << b;
-#pragma unroll
-    for (int q = 0; q < R; ++q)
-      if (!(q & h)) {
-        const float a = v[q], c = v[q + h];
-        v[q] = a + c;
-        v[q + h] = a - c;
-      }
-  }
-}
-
-// Two butterflies at once with the packed fp32x2 add/sub of sm_100:
-// (a0, a1), (b0, b1) <- (a0 + b0, a1 + b1), (a0 - b0, a1 - b1).
-__device__ __forceinline__ void bfly2(float &a0, float &a1, float &b0, float &b1) {
-  unsigned long long a, b, sum, dif;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(sum) : "l"(a), "l"(b));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(dif) : "l"(a), "l"(b));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(sum));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(dif));
-}
-
-// Same result as butterflies<R, B0, NBITS>, registers paired along index bit PB:
-// stages on other bits run two butterflies per packed add and sub; a stage on
-// PB itself (if in range) runs scalar.
-template <int R, int B0, int NBITS, int PB>
-__device__ __forceinline__ void butterflies_x2(float *v) {
-  constexpr int P = 1 << PB;
-#pragma unroll
-  for (int b = B0; b < B0 + NBITS; ++b) {
-    const int h = 1 << b;
-    if (b == PB) {
-#pragma unroll
-      for (int q = 0; q < R; ++q)
-        if (!(q & h)) {
-          const float a = v[q], c = v[q + h];
-          v[q] = a + c;
-          v[q + h] = a - c;
-        }
-    } else {
-#pragma unroll
-      for (int q = 0; q < R; ++q)
-        if (!(q & h) && !(q & P)) bfly2(v[q], v[q + P], v[q + h], v[q + h + P]);
-    }
-  }
-}
-
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// The input rows of the next iteration are copied into a shared-memory staging
-// buffer with cp.async while the current rows are transformed; phase A then
-// reads its 16-byte vectors from shared memory.
 template <int LOGN, int V, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads) fwht_rows_kernel(const Tin *__restrict__ x, Tout *__restrict__ z,
                                                              int64_t rows, float scale) {
-  using G = Geo<LOGN, V>;
-  constexpr int RPC = kThreads / G::P;  // rows per CTA iteration
-  constexpr int ROW_CHUNKS = G::N * (int)sizeof(Tin) / 16;
   extern __shared__ __align__(16) float smem[];
-  const int rl = threadIdx.x / G::P;
-  const int t = threadIdx.x % G::P;
-  float *buf = smem + rl * G::N;
-  Tin *stage = reinterpret_cast<Tin *>(smem + RPC * G::N);
-
-  auto prefetch = [&](int64_t first) {
-    const int64_t left = rows - first;
-    const int nrow = left < RPC ? (int)left : RPC;
-    const char *src = reinterpret_cast<const char *>(x + first * G::N);
-    char *dst = reinterpret_cast<char *>(stage);
-    for (int c = threadIdx.x; c < nrow * ROW_CHUNKS; c += kThreads) cp_async16(dst + 16 * c, src + 16 * (int64_t)c);
-    cp_async_commit();
-  };
-
-  int64_t base = (int64_t)blockIdx.x * RPC;
-  if (base < rows) prefetch(base);
-  for (; base < rows; base += (int64_t)gridDim.x * RPC) {
-    const int64_t row = base + rl;
-    const bool active = row < rows;
-    cp_async_wait_all();
-    __syncthreads();  // this iteration's rows are staged; last iteration's readers of buf are done
-    float v[G::R];
-    if (active) {
-      const Tin *xr = stage + rl * G::N;
-#pragma unroll
-      for (int h = 0; h < (1 << G::HB); ++h) {
-        const Tin *src = xr + G::eA(t, h << G::LV);
-#pragma unroll
-        for (int u = 0; u < V; u += io<Tin>::kVec)
-          io<Tin>::unpack(*reinterpret_cast<const uint4 *>(src + u), v + h * V + u);
-      }
-    } else {
-#pragma unroll
-      for (int q = 0; q < G::R; ++q) v[q] = 0.f;
-    }
-    __syncthreads();  // the staging buffer is free: fetch the next rows during the arithmetic
-    if (base + (int64_t)gridDim.x * RPC < rows) prefetch(base + (int64_t)gridDim.x * RPC);
-    butterflies_x2<G::R, 0, G::RB, 0>(v);
-
-#pragma unroll
-    for (int h = 0; h < (1 << G::HB); ++h) {
-      float *dst = buf + G::phys(G::eA(t, h << G::LV));
-#pragma unroll
-      for (int u = 0; u < V; u += 4)
-        *reinterpret_cast<float4 *>(dst + u) =
-            make_float4(v[h * V + u], v[h * V + u + 1], v[h * V + u + 2], v[h * V + u + 3]);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
-    butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
-    __syncthreads();  // all phase-B reads done before the buffer is reused
-
-    Tout *st = reinterpret_cast<Tout *>(buf);
-#pragma unroll
-    for (int q = 0; q < G::R; ++q) io<Tout>::store1(st + G::phys(G::eB(t, q)), v[q] * scale);
-    __syncthreads();
-    if (active) {
-      Tout *zr = z + row * G::N;
-#pragma unroll
-      for (int h = 0; h < (1 << G::HB); ++h) {
-        const int e = G::eA(t, h << G::LV);
-        const Tout *src = st + G::phys(e);
-        float o[V];
-#pragma unroll
-        for (int u = 0; u < V; u += io<Tout>::kVec)
-          io<Tout>::unpack(*reinterpret_cast<const uint4 *>(src + u), o + u);
-        store_group<Tout, V>(zr + e, o);
-      }
-    }
-  }
+  fwht_rows_body<LOGN, V, Tin, Tout, kThreads>(x, z, rows, scale, smem, threadIdx.x, blockIdx.x, gridDim.x,
+                                               [] { __syncthreads(); });
 }
 
 // n <= 64: one thread per block, all in registers.

@@ -44,6 +44,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "fwht_body.cuh"
 #include "kernels.h"
 
 namespace qwha {
@@ -55,14 +56,28 @@ constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int kEpiStride = 33;  // per-warp staging row (floats) of the sampled epilogue
 constexpr size_t kEpiSmem = 4 * 32 * kEpiStride * sizeof(float);
 
-template <int CG>
+enum { kOutBf16 = 0, kOutF32 = 1, kOutSampled = 2 };
+
+// Extra warps of the fused forward: they transform rows of X (Z = X H, bf16,
+// blocks of 2^kZ) while the other warps run the GEMM.
+constexpr int kZThreads = 128;
+template <int kZ>
+constexpr size_t z_smem() {
+  if constexpr (kZ == 0) return 0;
+  else return (size_t)(kZThreads / Geo<kZ, 8>::P) * (1u << kZ) * (sizeof(float) + sizeof(__nv_bfloat16));
+}
+
+template <int CG, int kMode = kOutBf16, int kZ = 0>
 struct Cfg {
-  static constexpr int kStages = CG == 1 ? 4 : 6;
+  static constexpr int kStages = CG == 1 ? 4 : (kZ ? 5 : 6);
   static constexpr uint32_t kABytes = BM * BK * 2;
   static constexpr int kBRows = BN / CG;  // rows of B this CTA loads
   static constexpr uint32_t kBBytes = kBRows * BK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256 + kEpiSmem;
+  static constexpr size_t kEpiBytes = kMode == kOutSampled ? kEpiSmem : 0;
+  static constexpr size_t kZOffset = (size_t)kStages * kStageBytes + 256 + kEpiBytes;  // from the aligned base
+  static constexpr size_t kSmem = kZOffset + 1024 + z_smem<kZ>();
+  static constexpr int kThreads = kGemmThreads + (kZ ? kZThreads : 0);
   // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
   // B bf16 (10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
   // M >> 4 at bit 24 (M = 128 per CTA of the group).
@@ -70,7 +85,13 @@ struct Cfg {
                                      ((uint32_t)((BM * CG) >> 4) << 24);
 };
 
-enum { kOutBf16 = 0, kOutF32 = 1, kOutSampled = 2 };
+// The transform the fused forward runs beside the GEMM.
+struct ZArgs {
+  const __nv_bfloat16 *x;
+  __nv_bfloat16 *z;
+  int64_t rows;  // rows of 2^kZ values
+  float scale;
+};
 
 // Sampled output: dc[j] (+)= alpha * D[r_j, k_j] for the CSR entries of E.
 struct SampleArgs {
@@ -273,12 +294,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
 // contiguous]); its stage is then filled by BM/64 or BN/64 boxes of 64 x 64.
 // k_splits > 1 (sampled output only): each tile's K range is cut into that
 // many parts, each part a separate work unit adding its share into dc.
-template <int kMode, int CG>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int kMode, int CG, int kZ>
+__global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const float *__restrict__ addend, void *__restrict__ out_v, int M, int N, int K,
-                             int a_mn, int b_mn, int group_m, int k_splits, SampleArgs sa_args, unsigned int *err) {
-  using C = Cfg<CG>;
+                             int a_mn, int b_mn, int group_m, int k_splits, SampleArgs sa_args, ZArgs za,
+                             unsigned int *err) {
+  using C = Cfg<CG, kMode, kZ>;
   constexpr int STAGES = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t base = smem_u32(smem_raw);
@@ -436,6 +458,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // drain: all issued MMAs complete before TMEM is released
     umma_commit_local<CG>(done_bar);
     if (!mbar_wait(done_bar, 0)) give_up(0x10u);
+  } else if (kZ && warp >= 6) {
+    // ------------------------------------------------ fused transform Z = X H (every CTA)
+    if constexpr (kZ != 0) {
+      float *zs = reinterpret_cast<float *>(smem + C::kZOffset);
+      fwht_rows_body<kZ, 8, __nv_bfloat16, __nv_bfloat16, kZThreads>(
+          za.x, za.z, za.rows, za.scale, zs, (int)threadIdx.x - kGemmThreads, blockIdx.x, gridDim.x,
+          [] { asm volatile("bar.sync 1, %0;" ::"n"(kZThreads) : "memory"); });
+    }
   } else if (warp >= 2) {
     // ------------------------------------------------ epilogue (every CTA)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -583,16 +613,17 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, uint3
 
 // Co-resident CTA groups of the CG variant (one CTA per SM; pairs need two SMs
 // of one cluster slot).
-template <int kMode, int CG>
+template <int kMode, int CG, int kZ>
 int resident_groups() {
   static int n = 0;
   if (n) return n;
+  using C = Cfg<CG, kMode, kZ>;
   const int sms = sm_count();
   if (CG == 1) return n = sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(sms - sms % CG));
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = Cfg<CG>::kSmem;
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = CG;
@@ -601,7 +632,7 @@ int resident_groups() {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_bf16_tcgen05_kernel<kMode, CG>, &cfg) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_bf16_tcgen05_kernel<kMode, CG, kZ>, &cfg) != cudaSuccess ||
       clusters < 1) {
     (void)cudaGetLastError();
     clusters = sms / CG;
@@ -610,15 +641,17 @@ int resident_groups() {
 }
 
 // A is [M, K] (K-major) or, with a_mn, [K, M]; B is [N, K] or, with b_mn, [K, N].
-template <int kMode, int CG>
+// With kZ, the launch also transforms za.rows rows of za.x into za.z.
+template <int kMode, int CG, int kZ = 0>
 cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, void *out, int64_t M, int64_t N,
-                           int64_t K, bool a_mn, bool b_mn, const SampleArgs &sa, cudaStream_t s) {
-  using C = Cfg<CG>;
+                           int64_t K, bool a_mn, bool b_mn, const SampleArgs &sa, cudaStream_t s,
+                           const ZArgs &za = ZArgs{}) {
+  using C = Cfg<CG, kMode, kZ>;
   CUtensorMap ta, tb;
   const bool ok_a = a_mn ? make_map(&ta, A, K, M, 64) : make_map(&ta, A, M, K, BM);
   const bool ok_b = b_mn ? make_map(&tb, B, K, N, 64) : make_map(&tb, B, N, K, C::kBRows);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
-  auto kern = gemm_bf16_tcgen05_kernel<kMode, CG>;
+  auto kern = gemm_bf16_tcgen05_kernel<kMode, CG, kZ>;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
@@ -636,7 +669,7 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
     group_m = 8 / CG;
     if (group_m > m_tiles) group_m = m_tiles;
   }
-  const int groups = resident_groups<kMode, CG>();
+  const int groups = resident_groups<kMode, CG, kZ>();
   // Sampled output: split K in two when the tiles alone would leave the last
   // wave of groups mostly idle (each dc then receives exactly two additions
   // onto zero, whose result does not depend on their order).
@@ -651,10 +684,11 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
     if (e != cudaSuccess) return e;
   }
   const int64_t units = tiles * k_splits;
-  const int64_t n_launch = units < groups ? units : groups;
+  // the fused transform runs in every CTA: launch all resident groups even when there are fewer tiles
+  const int64_t n_launch = kZ ? groups : (units < groups ? units : groups);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(n_launch * CG));
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute at[1];
@@ -665,7 +699,7 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
   cfg.attrs = at;
   cfg.numAttrs = CG > 1 ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, addend, out, (int)M, (int)N, (int)K, a_mn ? 1 : 0, b_mn ? 1 : 0,
-                            (int)group_m, k_splits, sa, device_error_word());
+                            (int)group_m, k_splits, sa, za, device_error_word());
 }
 
 // The pair variant once there are at least two 128-row blocks of output.
@@ -699,6 +733,18 @@ cudaError_t launch_gemm_any(const void *A, bool a_mn, const void *B, bool b_mn, 
                             bool f32_out, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
   return f32_out ? launch_gemm_t<kOutF32>(A, B, addend, out, M, N, K, a_mn, b_mn, SampleArgs{}, s)
                  : launch_gemm_t<kOutBf16>(A, B, addend, out, M, N, K, a_mn, b_mn, SampleArgs{}, s);
+}
+
+bool gemm_fused_fwht_supported(int64_t M, int logn) { return M > BM && (logn == 11 || logn == 12); }
+
+cudaError_t launch_gemm_fwd_fused(const void *X, const void *W, void *Y, int64_t T, int32_t d_out, int32_t d_in,
+                                  void *Z, int logn, float scale, cudaStream_t s) {
+  if (T <= 0 || d_out <= 0) return cudaSuccess;
+  if (!gemm_fused_fwht_supported(T, logn)) return cudaErrorNotSupported;
+  ZArgs za{static_cast<const __nv_bfloat16 *>(X), static_cast<__nv_bfloat16 *>(Z), T * (d_in >> logn), scale};
+  if (logn == 12)
+    return launch_gemm_cg<kOutBf16, 2, 12>(X, W, nullptr, Y, T, d_out, d_in, false, false, SampleArgs{}, s, za);
+  return launch_gemm_cg<kOutBf16, 2, 11>(X, W, nullptr, Y, T, d_out, d_in, false, false, SampleArgs{}, s, za);
 }
 
 cudaError_t launch_gemm_sampled(const void *A, bool a_mn, const void *B, bool b_mn, int64_t M, int64_t N, int64_t K,

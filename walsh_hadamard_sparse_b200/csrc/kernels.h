@@ -83,6 +83,11 @@ cudaError_t launch_gemm_nt(const void *A, const void *B, const float *addend, vo
                            int64_t N, int64_t K, cudaStream_t s);
 // dc[j] = alpha * (A B^T)[r_j, col_idx[j]] for the CSR entries of E, written
 // by the GEMM epilogue (no dense output).
+// Forward GEMM Y = X W^T (bf16, K-major) whose launch also writes Z = X H
+// (bf16, Hadamard blocks of 2^logn, times scale) from extra warps.
+bool gemm_fused_fwht_supported(int64_t M, int logn);
+cudaError_t launch_gemm_fwd_fused(const void *X, const void *W, void *Y, int64_t T, int32_t d_out, int32_t d_in,
+                                  void *Z, int logn, float scale, cudaStream_t s);
 cudaError_t launch_gemm_sampled(const void *A, bool a_mn, const void *B, bool b_mn, int64_t M, int64_t N, int64_t K,
                                 const int32_t *row_ptr, const int32_t *col_idx, int64_t p, float alpha, float *dc,
                                 cudaStream_t s);
