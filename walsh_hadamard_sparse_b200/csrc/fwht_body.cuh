@@ -160,8 +160,6 @@ __device__ __forceinline__ void fwht_rows_body(const Tin *__restrict__ x, Tout *
 #pragma unroll
       for (int q = 0; q < G::R; ++q) v[q] = 0.f;
     }
-    bar();  // the staging buffer is free: fetch the next rows during the arithmetic
-    if (base + (int64_t)n_cta * RPC < rows) prefetch(base + (int64_t)n_cta * RPC);
     butterflies_x2<G::R, 0, G::RB, 0>(v);
 
 #pragma unroll
@@ -172,26 +170,30 @@ __device__ __forceinline__ void fwht_rows_body(const Tin *__restrict__ x, Tout *
         *reinterpret_cast<float4 *>(dst + u) =
             make_float4(v[h * V + u], v[h * V + u + 1], v[h * V + u + 2], v[h * V + u + 3]);
     }
-    bar();
+    bar();  // phase A is in buf, and every thread has read its staged input: fetch the next rows
+    if (base + (int64_t)n_cta * RPC < rows) prefetch(base + (int64_t)n_cta * RPC);
 #pragma unroll
     for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
     butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
     bar();  // all phase-B reads done before the buffer is reused
 
-    Tout *st = reinterpret_cast<Tout *>(buf);
+    // scaled fp32 back through the buffer (the phase-B pattern is conflict-free),
+    // then phase-A vectors are packed once into the output type
 #pragma unroll
-    for (int q = 0; q < G::R; ++q) io<Tout>::store1(st + G::phys(G::eB(t, q)), v[q] * scale);
+    for (int q = 0; q < G::R; ++q) buf[G::phys(G::eB(t, q))] = v[q] * scale;
     bar();
     if (active) {
       Tout *zr = z + row * G::N;
 #pragma unroll
       for (int h = 0; h < (1 << G::HB); ++h) {
         const int e = G::eA(t, h << G::LV);
-        const Tout *src = st + G::phys(e);
+        const float *src = buf + G::phys(e);
         float o[V];
 #pragma unroll
-        for (int u = 0; u < V; u += io<Tout>::kVec)
-          io<Tout>::unpack(*reinterpret_cast<const uint4 *>(src + u), o + u);
+        for (int u = 0; u < V; u += 4) {
+          const float4 f = *reinterpret_cast<const float4 *>(src + u);
+          o[u] = f.x, o[u + 1] = f.y, o[u + 2] = f.z, o[u + 3] = f.w;
+        }
         store_group<Tout, V>(zr + e, o);
       }
     }
