@@ -63,6 +63,7 @@ def _load():
                 "oracle_init_budgets": [P, i32, i32, i64, i32, i32, P, P],
                 "oracle_init_select": [P, i32, i32, i32, P, P, P, P],
                 "oracle_init_select_global": [P, i32, i32, i32, i64, i32, ctypes.c_uint64, P, P, P, P],
+                "oracle_refine_values": [P, i32, i32, i32, P, f64, P, P, i32, P, P],
                 "oracle_plan_build": [i32, i32, i64, P, P, P, P, P],
             }
             for name, args in sig.items():
@@ -249,6 +250,25 @@ def init_select_global(dWq, p: int, n: int, sel: str = "magnitude", seed: int = 
                                            _p(b), _p(rp), _p(ci), _p(c))
     _check(rc, "init_select_global")
     return dict(budgets=b, row_ptr=rp, col_idx=ci, coef=c)
+
+
+def refine_values(dWq, S, row_ptr, col_idx, n: int, damp: float = 0.0, rows=None):
+    """Value Refinement: least-squares values at E for the calibration Hessian S = X^T X [d_in, d_in] (fp64),
+    S damped by damp * mean(diag S). Returns coef [p] (float32); only the entries of `rows` (all when None) are
+    computed, the others are NaN."""
+    w = np.ascontiguousarray(dWq, dtype=np.float32)
+    d_out, d_in = w.shape
+    S = _f64(S)
+    assert S.shape == (d_in, d_in)
+    rp, ci = _i32(row_ptr), _i32(col_idx)
+    c = np.full(ci.size, np.nan, dtype=np.float32)
+    sel = None if rows is None else _i32(rows)
+    rc = _load().oracle_refine_values(_p(w), d_out, d_in, n, _p(S), float(damp), _p(rp), _p(ci),
+                                      0 if sel is None else sel.size, _p(sel), _p(c))
+    if rc == 2:
+        raise ValueError("refine_values: a system is not positive definite")
+    _check(rc, "refine_values")
+    return c
 
 
 def plan_build(row_ptr, col_idx, d_in: int):

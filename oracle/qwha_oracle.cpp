@@ -45,6 +45,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <mutex>
 #include <numeric>
 #include <thread>
 #include <vector>
@@ -498,6 +499,112 @@ int oracle_init_select_global(const float *dWq, int32_t d_out, int32_t d_in, int
     coef[q] = (float)(V[pick[q]] * inv);
   }
   return 0;
+}
+
+// Value Refinement [P1 设计3]: the values at E that minimise the layer-output
+// error for calibration inputs, instead of the dense solution x0. For channel
+// i the page states min_x ||v - x B||^2 with v = dW_Q[i,:] R, B = H^-1 R,
+// R R^T = X X^T (the calibration Hessian, called S here), x non-zero only at
+// E_i; the closed form itself is lost from the page. Its plain reading, the
+// least-squares solution over the selected rows B' of B, is
+//   x* = v B'^T (B' B'^T)^-1 = u_i[E_i] (G[E_i, E_i])^-1,
+//   G = H S H,  u_i = dW_Q[i,:] S H   (H orthonormal, symmetric, H^-1 = H),
+// which equals x0 = (dW_Q H)[i, E_i] when S = I. `damp` adds damp * mean(diag S)
+// to the diagonal of S first (0: none). S is [d_in, d_in] (the caller forms
+// X^T X from calibration rows X [T, d_in]). Rows `rows` (all when NULL) get
+// their coef entries written as float(x*); returns 2 if a system is not
+// positive definite.
+// Steps in double: A = S H (rows), G^T = (A^T) H (rows of the transpose), and
+// per row y = w S, u = y H, then a plain Cholesky factorisation and the two
+// triangular solves.
+int oracle_refine_values(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, const double *S, double damp,
+                         const int32_t *row_ptr, const int32_t *col_idx, int32_t n_rows, const int32_t *rows,
+                         float *coef) {
+  if (!shape_ok(d_in, n) || d_out <= 0 || damp < 0) return 1;
+  const double inv = inv_sqrt(n);
+  const size_t D = (size_t)d_in;
+  std::vector<double> Sd(S, S + D * D);
+  double tr = 0;
+  for (size_t k = 0; k < D; ++k) tr += Sd[k * D + k];
+  const double lam = damp * tr / (double)d_in;
+  for (size_t k = 0; k < D; ++k) Sd[k * D + k] += lam;
+  auto transform_rows = [&](std::vector<double> &M) {
+    parallel_for(d_in, [&](int64_t r) {
+      for (int blk = 0; blk < d_in / n; ++blk) {
+        double *x = M.data() + (size_t)r * D + (size_t)blk * n;
+        butterflies(x, n);
+        for (int k = 0; k < n; ++k) x[k] *= inv;
+      }
+    });
+  };
+  auto transpose = [&](const std::vector<double> &M) {
+    std::vector<double> T(D * D);
+    for (size_t a = 0; a < D; ++a)
+      for (size_t b = 0; b < D; ++b) T[b * D + a] = M[a * D + b];
+    return T;
+  };
+  std::vector<double> A = Sd;
+  transform_rows(A);                // A = S H
+  std::vector<double> Gt = transpose(A);
+  transform_rows(Gt);               // Gt = A^T H = (H A)^T = G^T
+  std::vector<int32_t> all;
+  if (!rows) {
+    all.resize(d_out);
+    std::iota(all.begin(), all.end(), 0);
+    rows = all.data();
+    n_rows = d_out;
+  }
+  int status = 0;
+  std::mutex mu;
+  parallel_for(n_rows, [&](int64_t q) {
+    const int i = rows[q];
+    if (i < 0 || i >= d_out) return;
+    std::vector<double> y(D, 0.0);
+    for (size_t a = 0; a < D; ++a) {
+      const double w = (double)dWq[(size_t)i * D + a];
+      const double *srow = Sd.data() + a * D;
+      for (size_t b = 0; b < D; ++b) y[b] += w * srow[b];
+    }
+    for (int blk = 0; blk < d_in / n; ++blk) {
+      double *x = y.data() + (size_t)blk * n;
+      butterflies(x, n);
+      for (int k = 0; k < n; ++k) x[k] *= inv;
+    }
+    const int b0 = row_ptr[i], m = row_ptr[i + 1] - row_ptr[i];
+    if (m <= 0) return;
+    std::vector<double> L((size_t)m * m), z(m);
+    for (int r = 0; r < m; ++r)
+      for (int c = 0; c <= r; ++c)  // G[E_r][E_c] = Gt[E_c][E_r]
+        L[(size_t)r * m + c] = Gt[(size_t)col_idx[b0 + c] * D + col_idx[b0 + r]];
+    for (int j = 0; j < m; ++j) {  // Cholesky, lower triangle in place
+      double d = L[(size_t)j * m + j];
+      for (int k = 0; k < j; ++k) d -= L[(size_t)j * m + k] * L[(size_t)j * m + k];
+      if (!(d > 0)) {
+        std::lock_guard<std::mutex> g(mu);
+        status = 2;
+        return;
+      }
+      d = std::sqrt(d);
+      L[(size_t)j * m + j] = d;
+      for (int r = j + 1; r < m; ++r) {
+        double v = L[(size_t)r * m + j];
+        for (int k = 0; k < j; ++k) v -= L[(size_t)r * m + k] * L[(size_t)j * m + k];
+        L[(size_t)r * m + j] = v / d;
+      }
+    }
+    for (int r = 0; r < m; ++r) {  // L z = u[E]
+      double v = y[col_idx[b0 + r]];
+      for (int k = 0; k < r; ++k) v -= L[(size_t)r * m + k] * z[k];
+      z[r] = v / L[(size_t)r * m + r];
+    }
+    for (int r = m - 1; r >= 0; --r) {  // L^T x = z
+      double v = z[r];
+      for (int k = r + 1; k < m; ++k) v -= L[(size_t)k * m + r] * z[k];
+      z[r] = v / L[(size_t)r * m + r];
+    }
+    for (int r = 0; r < m; ++r) coef[b0 + r] = (float)z[r];
+  });
+  return status;
 }
 
 // Column view of the CSR pattern: for every column k the nonzeros j with

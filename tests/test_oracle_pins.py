@@ -383,3 +383,59 @@ def test_select_global_random_matches_generator():
     # a uniform p-subset: another seed gives another one, with the same count
     other = oracle.init_select_global(w, p, n, "random", seed + 1)
     assert other["row_ptr"][-1] == p and not np.array_equal(other["col_idx"], got["col_idx"])
+
+
+# --------------------------------------------------------------------------- value refinement
+
+
+def _refine_case(seed, d_out=20, d_in=64, n=32, per=7, T=300):
+    g = rng_for(seed, "refine")
+    w = (g.standard_normal((d_out, d_in)) * 0.01).astype(np.float32)
+    e = oracle.init_alloc(w, d_out * per, n, 2, "fewest")
+    X = g.standard_normal((T, d_in))
+    X[:, g.choice(d_in, 3, replace=False)] *= 20.0  # outlier input channels, as in the workloads
+    return w, e, X.T @ X
+
+
+def test_refine_identity_hessian_is_dense_solution():
+    # the page: with R proportional to I the refinement changes nothing (x* = x0), for any scale of S
+    w, e, _ = _refine_case(80)
+    d_in = w.shape[1]
+    for scale in (1.0, 7.5):
+        c = oracle.refine_values(w, scale * np.eye(d_in), e["row_ptr"], e["col_idx"], 32)
+        assert np.array_equal(c.view(np.uint32), e["coef"].view(np.uint32))
+
+
+def test_refine_matches_least_squares_on_the_page_formulation():
+    """x* from an independent route: R = U Sigma^(1/2) from an eigendecomposition of the (damped) Hessian,
+    v = dW_Q[i,:] R, B = H^-1 R with H from scipy, and numpy's least squares over the selected rows of B."""
+    w, e, S = _refine_case(81)
+    d_out, d_in = w.shape
+    damp = 0.01
+    Sd = S + damp * np.trace(S) / d_in * np.eye(d_in)
+    lam, U = np.linalg.eigh(Sd)
+    R = U * np.sqrt(lam)
+    Hinv = H_block(d_in, 32)  # orthonormal, its own inverse
+    B = Hinv @ R
+    got = oracle.refine_values(w, S, e["row_ptr"], e["col_idx"], 32, damp)
+    rp, ci = e["row_ptr"], e["col_idx"]
+    for i in range(d_out):
+        sel = ci[rp[i]:rp[i + 1]]
+        v = w[i].astype(np.float64) @ R
+        x, *_ = np.linalg.lstsq(B[sel].T, v, rcond=None)
+        assert np.allclose(got[rp[i]:rp[i + 1]], x, rtol=1e-5, atol=1e-9), i
+
+
+def test_refine_never_worse_than_dense_solution():
+    # the refined values minimise the per-channel output error, so they never do worse than x0 on it
+    w, e, S = _refine_case(82)
+    d_out, d_in = w.shape
+    H = H_block(d_in, 32)
+    got = oracle.refine_values(w, S, e["row_ptr"], e["col_idx"], 32)
+    rp, ci = e["row_ptr"], e["col_idx"]
+    for i in range(d_out):
+        sel = ci[rp[i]:rp[i + 1]]
+        def err(x):
+            r = w[i].astype(np.float64) - x @ H[sel]  # dW_Q[i,:] - (F H^-1)[i,:]
+            return r @ S @ r  # || r X^T ||^2
+        assert err(got[rp[i]:rp[i + 1]].astype(np.float64)) <= err(e["coef"][rp[i]:rp[i + 1]].astype(np.float64)) + 1e-12
