@@ -313,6 +313,20 @@ def main():
             ts.append(ev[0].elapsed_time(ev[1]))
         sel_ms[sel] = statistics.median(ts)
         del sws
+    # Value Refinement of the AdaAlloc values with this GPU's tokens as calibration rows
+    rws = torch.empty(W.workspace_size(7, spec.d_out, spec.d_in, spec.p, 0, False), dtype=torch.uint8, device=dev)
+    S_cal = torch.empty((spec.d_in, spec.d_in), dtype=torch.float32, device=dev)
+    c_ref = torch.empty(spec.p, dtype=torch.float32, device=dev)
+    refine_ms = []
+    for it in range(4):
+        ev[0].record()
+        W.calib_hessian(X, S_cal)
+        W.refine_values(dWq, S_cal, e["row_ptr"], e["col_idx"], spec.had_block, 0.01, coef=c_ref, ws=rws)
+        ev[1].record()
+        torch.cuda.synchronize()
+        if it:
+            refine_ms.append(ev[0].elapsed_time(ev[1]))
+    del rws, S_cal, c_ref
     a = W.Adapter(spec.d_in, spec.d_out, spec.had_block, spec.p, e["row_ptr"], e["col_idx"], e["coef"])
     W.plan_build(a)  # the views the sparse backward needs
 
@@ -516,6 +530,9 @@ def main():
                  "frac_hbm": init_bytes / (init_med / 1e3) / 1e9 / peaks["hbm_gbs"],
                  "what": "AdaAlloc on dW_Q (4096 x 4096 fp32): norms, budgets, fp64 transform, top-k; one-off per layer",
                  "select_global_ms": sel_ms,
+                 "refine_ms": statistics.median(refine_ms),
+                 "refine_what": ("Value Refinement at E: calibration Hessian X^T X over the 8192 tokens, G = H S H, "
+                                 "dW_Q S H, per-channel fp64 Cholesky solves"),
                  "select_global_what": ("whole-matrix selection (magnitude top-p; seeded random E): fp64 transform of "
                                         "all rows kept in HBM, 8 radix passes over 16.8 M keys, per-row compaction")},
     }

@@ -140,7 +140,8 @@ typedef enum {
   QWHA_OP_PLAN = 3,      /* qwha_plan_build */
   QWHA_OP_FWD_DENSE = 4, /* qwha_adapter_fwd, algo dense */
   QWHA_OP_BWD_DENSE = 5, /* qwha_adapter_bwd, algo dense */
-  QWHA_OP_SELECT_GLOBAL = 6 /* qwha_init_select_global */
+  QWHA_OP_SELECT_GLOBAL = 6, /* qwha_init_select_global */
+  QWHA_OP_REFINE = 7         /* qwha_refine_values */
 } qwha_op;
 
 /* Z = X H row by row: x and z are [rows, n] of dtype dt (device), each row
@@ -240,6 +241,29 @@ qwha_status qwha_init_select_global(const float *dWq, int32_t d_out, int32_t d_i
                                     int64_t p, qwha_selection sel, uint64_t seed, int32_t *budgets,
                                     int32_t *row_ptr, int32_t *col_idx, float *coef, void *ws,
                                     size_t ws_bytes, void *stream);
+
+/* Calibration Hessian for Value Refinement: S = X^T X, fp32 [d_in, d_in]
+ * (device), from calibration rows X bf16 [T, d_in] (device, T >= 1, d_in a
+ * multiple of 8), on the tensor cores with fp32 accumulation. */
+qwha_status qwha_calib_hessian(const void *X, int64_t T, int32_t d_in, float *S, void *stream);
+
+/* Value Refinement (papernotes.org 关键设计 3): for a fixed E (CSR row_ptr,
+ * col_idx, p entries; e.g. from qwha_init_alloc) the values that minimise each
+ * channel's layer-output error for the calibration Hessian S fp32
+ * [d_in, d_in] (symmetric, from qwha_calib_hessian). The page keeps the
+ * per-channel problem min ||v - x B'|| (v = dWq[i,:] R, B = H^-1 R,
+ * R R^T = S) and loses its closed form; this is its least-squares solution
+ *   c[E_i] = u_i[E_i] (G[E_i, E_i])^-1,  G = H S H,  u_i = dWq[i,:] S H,
+ * with S first damped by damp * mean(diag S) (damp >= 0; G[E_i, E_i] must be
+ * positive definite). With S = I it returns the dense solution of
+ * qwha_init_alloc. dWq fp32 [d_out, d_in]; coef fp32 [p] written (device).
+ * Channels with more than min(d_in, 1024) entries are not solved: their
+ * coef become NaN and qwha_check_stream_status reports it.
+ * ws: qwha_workspace_size(QWHA_OP_REFINE, ...) bytes. */
+qwha_status qwha_refine_values(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block,
+                               const float *S, float damp, const int32_t *row_ptr,
+                               const int32_t *col_idx, int64_t p, float *coef, void *ws,
+                               size_t ws_bytes, void *stream);
 
 /* Index views of E for the backward (E stays fixed while c trains,
  * papernotes.org 整体框架): from the CSR row_ptr/col_idx (device) write the

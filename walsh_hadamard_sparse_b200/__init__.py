@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     QWeight,
     adapter_bwd,
     adapter_fwd,
+    calib_hessian,
     fwht,
     init_alloc,
     init_alloc_sharded,
@@ -20,6 +21,7 @@ from .api import (  # noqa: F401
     init_select_global,
     plan_build,
     plan_tiles,
+    refine_values,
     shard_rows,
     stage_report,
     stage_timing,

@@ -54,6 +54,8 @@ _SIGNATURES = {
     "qwha_coef_grad_noalloc": (ctypes.c_int, [ctypes.POINTER(QwhaAdapter), ctypes.c_int, P, P, i64, f32, P, P]),
     "qwha_init_alloc": (ctypes.c_int, [P, i32, i32, i32, i64, i32, ctypes.c_int, P, P, P, P, P, sz, P]),
     "qwha_init_norms": (ctypes.c_int, [P, i32, i32, P, P]),
+    "qwha_calib_hessian": (ctypes.c_int, [P, i64, i32, P, P]),
+    "qwha_refine_values": (ctypes.c_int, [P, i32, i32, i32, P, f32, P, P, i64, P, P, sz, P]),
     "qwha_init_select_global": (ctypes.c_int, [P, i32, i32, i32, i64, ctypes.c_int, ctypes.c_uint64, P, P, P, P, P, sz,
                                                P]),
     "qwha_init_budgets": (ctypes.c_int, [P, i32, i32, i64, i32, ctypes.c_int, P, P, P, sz, P]),

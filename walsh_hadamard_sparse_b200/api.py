@@ -15,7 +15,7 @@ import torch
 from ._lib import QwhaAdapter, QwhaQweight, check, lib
 
 F32, BF16 = 0, 1
-OP_FWD, OP_BWD, OP_INIT, OP_PLAN, OP_FWD_DENSE, OP_BWD_DENSE, OP_SELECT_GLOBAL = 0, 1, 2, 3, 4, 5, 6
+OP_FWD, OP_BWD, OP_INIT, OP_PLAN, OP_FWD_DENSE, OP_BWD_DENSE, OP_SELECT_GLOBAL, OP_REFINE = 0, 1, 2, 3, 4, 5, 6, 7
 SELECTION = {"magnitude": 0, "random": 1}
 ALGO = {"sparse": 0, "dense": 1}
 REMAINDER = {"fewest": 0, "largest": 1}
@@ -196,6 +196,29 @@ def init_select_global(dWq: torch.Tensor, p: int, had_block: int, sel: str = "ma
     check(rc, "qwha_init_select_global")
     out["col_idx"], out["coef"] = out["col_idx"][:p], out["coef"][:p]
     return out
+
+
+def calib_hessian(X: torch.Tensor, S: torch.Tensor | None = None) -> torch.Tensor:
+    """S = X^T X (fp32 [d_in, d_in]) from bf16 calibration rows X [T, d_in]."""
+    T, d_in = X.shape
+    S = torch.empty((d_in, d_in), dtype=torch.float32, device=X.device) if S is None else S
+    check(lib().qwha_calib_hessian(_ptr(X), T, d_in, _ptr(S), _stream()), "qwha_calib_hessian")
+    return S
+
+
+def refine_values(dWq: torch.Tensor, S: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor, had_block: int,
+                  damp: float = 0.01, coef: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Value Refinement: least-squares coefficients at E (row_ptr, col_idx) for the calibration Hessian S."""
+    d_out, d_in = dWq.shape
+    p = col_idx.numel()
+    coef = torch.empty(max(p, 1), dtype=torch.float32, device=dWq.device) if coef is None else coef
+    need = workspace_size(OP_REFINE, d_out, d_in, p, 0, False)
+    ws = _ws(need, dWq.device) if ws is None else ws
+    rc = lib().qwha_refine_values(_ptr(dWq), d_out, d_in, had_block, _ptr(S), float(damp), _ptr(row_ptr),
+                                  _ptr(col_idx) if p else None, p, _ptr(coef), _ptr(ws), 0 if ws is None else ws.numel(),
+                                  _stream())
+    check(rc, "qwha_refine_values")
+    return coef[:p]
 
 
 def init_norms(dWq_rows: torch.Tensor) -> torch.Tensor:

@@ -391,6 +391,7 @@ size_t qwha_workspace_size(qwha_op op, int32_t d_out, int32_t d_in, int64_t p, i
     case QWHA_OP_FWD_DENSE: return fwd_dense_ws(d_out, d_in);
     case QWHA_OP_BWD_DENSE: return bwd_dense_ws(d_out, d_in, T);
     case QWHA_OP_SELECT_GLOBAL: return select_global_workspace(d_out, d_in);
+    case QWHA_OP_REFINE: return refine_workspace(d_out, d_in);
   }
   return 0;
 }
@@ -656,6 +657,37 @@ qwha_status qwha_init_select_global(const float *dWq, int32_t d_out, int32_t d_i
   return cuda_status(launch_select_global(dWq, d_out, d_in, had_block, p, (int)sel, seed, budgets, row_ptr, col_idx,
                                           coef, ws, (cudaStream_t)stream),
                      "init_select_global");
+}
+
+qwha_status qwha_calib_hessian(const void *X, int64_t T, int32_t d_in, float *S, void *stream) {
+  if (T < 1 || d_in <= 0 || d_in % 8) return fail(QWHA_ERR_INVALID_ARG, "T %lld, d_in %d (a multiple of 8)", (long long)T, d_in);
+  QWHA_CHECK_PTR(X, "X");
+  QWHA_CHECK_PTR(S, "S");
+  if ((uintptr_t)X % 16 || (uintptr_t)S % 16) return fail(QWHA_ERR_MISALIGNED, "X and S must be 16-byte aligned");
+  StageScope sc(ST_INIT, 1, (cudaStream_t)stream);
+  return cuda_status(launch_calib_hessian(X, T, d_in, S, (cudaStream_t)stream), "calib_hessian");
+}
+
+qwha_status qwha_refine_values(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block, const float *S,
+                               float damp, const int32_t *row_ptr, const int32_t *col_idx, int64_t p, float *coef,
+                               void *ws, size_t ws_bytes, void *stream) {
+  if (d_out <= 0 || d_in <= 0 || d_in % 8) return fail(QWHA_ERR_INVALID_ARG, "d_out %d, d_in %d (a multiple of 8)", d_out, d_in);
+  qwha_status st = check_hadamard(d_in, had_block);
+  if (st != QWHA_OK) return st;
+  if (!(damp >= 0.0f)) return fail(QWHA_ERR_INVALID_ARG, "damp %g", (double)damp);
+  if (p < 0 || p > (int64_t)d_in * d_out || p > 2147483647LL) return fail(QWHA_ERR_INVALID_ARG, "p %lld", (long long)p);
+  if (p == 0) return QWHA_OK;
+  QWHA_CHECK_PTR(dWq, "dWq");
+  QWHA_CHECK_PTR(S, "S");
+  QWHA_CHECK_PTR(row_ptr, "row_ptr");
+  QWHA_CHECK_PTR(col_idx, "col_idx");
+  QWHA_CHECK_PTR(coef, "coef");
+  if ((uintptr_t)dWq % 16 || (uintptr_t)S % 16) return fail(QWHA_ERR_MISALIGNED, "dWq and S must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, refine_workspace(d_out, d_in))) != QWHA_OK) return st;
+  StageScope sc(ST_INIT, 14, (cudaStream_t)stream);
+  return cuda_status(launch_refine(dWq, d_out, d_in, had_block, S, damp, row_ptr, col_idx, p, coef, ws,
+                                   (cudaStream_t)stream),
+                     "refine_values");
 }
 
 qwha_status qwha_init_norms(const float *dWq, int32_t rows, int32_t d_in, double *e, void *stream) {

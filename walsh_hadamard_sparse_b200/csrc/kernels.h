@@ -57,6 +57,13 @@ namespace qwha {
 // AdaAlloc (init.cu)
 size_t init_workspace(int32_t d_out, int32_t d_in);
 int init_max_din();
+// Value Refinement (refine.cu)
+int refine_cap(int32_t d_in);
+size_t refine_workspace(int32_t d_out, int32_t d_in);
+cudaError_t launch_calib_hessian(const void *X, int64_t T, int32_t d_in, float *S, cudaStream_t s);
+cudaError_t launch_refine(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block, const float *S,
+                          float damp, const int32_t *row_ptr, const int32_t *col_idx, int64_t p, float *coef,
+                          void *ws, cudaStream_t s);
 size_t select_global_workspace(int32_t d_out, int32_t d_in);
 cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p, int sel,
                                  uint64_t seed, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx, float *coef,
