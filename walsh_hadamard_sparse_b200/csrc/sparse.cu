@@ -305,75 +305,103 @@ __global__ void permute_kernel(const float *__restrict__ src, const int32_t *__r
 // ---------------------------------------------------------------- SDDMM
 
 constexpr int kSddmmThreads = 512;
-constexpr int kSddmmSlotEntries = 16;                                     // consecutive entries per slot
-constexpr int kSddmmPass = (kSddmmThreads / 32) * 8 * kSddmmSlotEntries;  // entries per CTA pass
-
-// tokens per staged sub-tile (2 x QWHA_TILE x TT values = 32 KB); a lane covers TT/4 of them
+constexpr int kSddmmTT = 32;                    // tokens per staged sub-tile
+constexpr int kSddmmSlots = kSddmmThreads / 4;  // 4 lanes per slot, each two 16-byte chunks (8 tokens)
+// shared memory: the fp32 dY and Z sub-tiles plus two raw staging buffers
 template <typename T>
-__host__ __device__ constexpr int sddmm_tt() {
-  return sizeof(T) == 2 ? 32 : 16;
+constexpr size_t sddmm_smem() {
+  return 2ull * QWHA_TILE * kSddmmTT * sizeof(float) + 2 * (2ull * QWHA_TILE * kSddmmTT * sizeof(T));
 }
 
-// Per thread: the 16-byte global vectors of one sub-tile it stages (dY slice
-// and Z slice), held in registers so that the next sub-tile's loads overlap
-// the current sub-tile's arithmetic.
-template <typename T, int TT>
-struct SubTile {
-  static constexpr int V = 16 / (int)sizeof(T);                           // values per vector
-  static constexpr int HALF = (QWHA_TILE / V) * TT;                        // vectors per operand
-  static constexpr int ITEMS = 2 * HALF / kSddmmThreads;                   // vectors per thread
-  uint4 v[ITEMS];
+// entries per slot and pass (the per-entry accumulators and offsets live in registers)
+template <typename T>
+__host__ __device__ constexpr int sddmm_entries() {
+  return sizeof(T) == 2 ? 18 : 12;
+}
 
-  __device__ __forceinline__ void load(const T *dY, const T *Z, int64_t tb, int d_out, int d_in, int64_t t0, int r0,
-                                       int r_len, int k0, int k_len) {
+// Staged sub-tiles are fp32 s[row][token], 32 tokens (128 B) per row; the
+// 16-byte chunk c (tokens 4c .. 4c+3) of row r sits at chunk c ^ ((r & 3) << 1)
+// (a permutation that keeps the chunk's parity). A staging write (a warp
+// covers the 32 tokens of one row) is free of bank conflicts; so is a read:
+// the 8 lanes of a quarter warp are two slots of 4 lanes, the even slot
+// reads even chunks and the odd slot odd ones, so they meet 8 distinct chunk
+// positions whatever their rows.
+__device__ __forceinline__ int sdd_phys(int r, int t) {
+  return r * kSddmmTT + ((((t >> 2) ^ ((r & 3) << 1)) << 2) | (t & 3));
+}
+
+// A sub-tile of dY and Z (32 tokens x QWHA_TILE rows each, as stored) is
+// copied raw into a double-buffered staging area with cp.async (16-byte
+// pieces; rows or tokens past the edge are zero-filled), then widened to fp32
+// into the swizzled layout. A thread moves vectors of V consecutive rows at
+// one token; the lanes of a warp take 32 consecutive tokens.
+template <typename T>
+struct SddStage {
+  static constexpr int V = 16 / (int)sizeof(T);
+  static constexpr int HALF = (QWHA_TILE / V) * kSddmmTT;  // vectors per operand
+  static constexpr int ITEMS = 2 * HALF / kSddmmThreads;    // vectors per thread
+  static constexpr size_t kRawBytes = 2ull * QWHA_TILE * kSddmmTT * sizeof(T);  // one buffer, both operands
+
+  static __device__ __forceinline__ void copy(T *raw, const T *dY, const T *Z, int64_t tb, int d_out, int d_in,
+                                              int64_t t0, int r0, int r_len, int k0, int k_len) {
 #pragma unroll
     for (int u = 0; u < ITEMS; ++u) {
       const int it = threadIdx.x + u * kSddmmThreads;
       const int which = it >= HALF;
       const int w = it - which * HALF;
-      const int t = w % TT, c = w / TT;
+      const int t = w % kSddmmTT, c = w / kSddmmTT;
       const int64_t tg = t0 + t;
       const int len = which ? k_len : r_len;
-      v[u] = make_uint4(0, 0, 0, 0);
-      if (tg < tb && c * V < len) {
-        const T *src = which ? Z + tg * d_in + k0 + c * V : dY + tg * d_out + r0 + c * V;
-        v[u] = *reinterpret_cast<const uint4 *>(src);
-      }
+      const bool in = tg < tb && c * V < len;
+      const T *src = in ? (which ? Z + tg * d_in + k0 + c * V : dY + tg * d_out + r0 + c * V) : dY;
+      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(raw + (size_t)it * V));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(in ? 16 : 0)
+                   : "memory");
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
-  __device__ __forceinline__ void store(T *s_dy, T *s_z) const {
+  static __device__ __forceinline__ void widen(const T *raw, float *s_dy, float *s_z) {
 #pragma unroll
     for (int u = 0; u < ITEMS; ++u) {
       const int it = threadIdx.x + u * kSddmmThreads;
       const int which = it >= HALF;
       const int w = it - which * HALF;
-      const int t = w % TT, c = w / TT;
+      const int t = w % kSddmmTT, c = w / kSddmmTT;
       float f[V];
-      io<T>::unpack(v[u], f);
-      T *dst = which ? s_z : s_dy;
+      io<T>::unpack(*reinterpret_cast<const uint4 *>(raw + (size_t)it * V), f);
+      float *dst = which ? s_z : s_dy;
 #pragma unroll
-      for (int i = 0; i < V; ++i) io<T>::store1(dst + (c * V + i) * TT + t, f[i]);
+      for (int i = 0; i < V; ++i) dst[sdd_phys(c * V + i, t)] = f[i];
     }
   }
 };
 
-// One CTA per (QWHA_TILE x QWHA_TILE tile of F, token chunk). Lanes are
-// (slot, q): q picks TT/4 tokens of a staged row, slot one of 8 entries in
-// flight; slot s of warp w owns 16 consecutive tile entries (CSC order inside
-// the tile: mostly one column, whose Z vector is reloaded only when it
-// changes). Per entry and sub-tile a lane does one 16-byte shared load of dY
-// and TT/4 FMAs; at the end of the chunk the 4 q lanes of an entry are summed
-// by shuffles and written to the chunk's partial sums.
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// One CTA per (QWHA_TILE x QWHA_TILE tile of F, token chunk). A warp is 8
+// slots of 4 lanes; lane q of a slot holds tokens 8q .. 8q+7 of the staged
+// sub-tile (chunks 2q and 2q+1, whose swizzled offsets differ in bit 2).
+// Slot s of the CTA owns E consecutive tile entries (CSC order inside the
+// tile: mostly one column, whose Z chunks are reloaded only when it changes).
+// Per entry and sub-tile a lane does two 16-byte shared loads of dY and four
+// packed fp32x2 FMAs; at the end of the chunk the 4 lanes of a slot are summed
+// by shuffles and the sum is written to the chunk's partial sums.
 template <typename T>
-__global__ void __launch_bounds__(kSddmmThreads)
+__global__ void __launch_bounds__(kSddmmThreads, 1)
     sddmm_kernel(const T *__restrict__ dY, const T *__restrict__ Z, int64_t T_, int d_out, int d_in,
                  const int32_t *__restrict__ tile_ptr, const int32_t *__restrict__ tile_pos,
                  const int32_t *__restrict__ tile_rk, int n_rb, int64_t chunk_tokens, int64_t p,
                  float *__restrict__ partial) {
-  constexpr int TT = sddmm_tt<T>();
-  constexpr int G = TT / 4;  // tokens per lane
-  __shared__ __align__(16) T s_dy[QWHA_TILE * TT];
-  __shared__ __align__(16) T s_z[QWHA_TILE * TT];
+  constexpr int E = sddmm_entries<T>();
+  constexpr int kPass = kSddmmSlots * E;
+  extern __shared__ __align__(16) float sdd_smem[];
+  float *s_dy = sdd_smem;
+  float *s_z = sdd_smem + QWHA_TILE * kSddmmTT;
+  T *raw = reinterpret_cast<T *>(sdd_smem + 2 * QWHA_TILE * kSddmmTT);  // two staging buffers
   const int tile = blockIdx.x;
   const int rb = tile % n_rb, kb = tile / n_rb;
   const int r0 = rb * QWHA_TILE, k0 = kb * QWHA_TILE;
@@ -385,85 +413,69 @@ __global__ void __launch_bounds__(kSddmmThreads)
   const int64_t ta = c * chunk_tokens, tb = (ta + chunk_tokens < T_) ? ta + chunk_tokens : T_;
   float *part = partial + c * p;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int q = lane & 3, slot = lane >> 2;
+  const int q = lane & 3, slot = warp * 8 + (lane >> 2);
 
-  for (int64_t eb = e_begin; eb < e_end; eb += kSddmmPass) {
-    const int64_t my0 = eb + (int64_t)(warp * 8 + slot) * kSddmmSlotEntries;
-    int rk[kSddmmSlotEntries];  // (row << 16 | column) inside the tile, -1 when unused
-    float acc[kSddmmSlotEntries];
+  for (int64_t eb = e_begin; eb < e_end; eb += kPass) {
+    const int64_t my0 = eb + (int64_t)slot * E;
+    // per entry, fixed over the token range: the shared offsets of this lane's
+    // dY and Z chunks (dY high half, Z low half; an unused entry reads row 0
+    // and is not stored), whether its column differs from the previous one's,
+    // and whether it is in use
+    uint32_t off[E];
+    uint32_t newcol = 0, valid = 0;
+    float acc[E];
 #pragma unroll
-    for (int i = 0; i < kSddmmSlotEntries; ++i) {
+    for (int i = 0; i < E; ++i) {
       const int64_t e = my0 + i;
       const int v = e < e_end ? tile_rk[e] : -1;
       const int r_ = (v >> 16) & 0xffff, k_ = v & 0xffff;
-      rk[i] = (e < e_end && r_ < r_len && k_ < k_len) ? v : -1;
+      const bool ok = e < e_end && v >= 0 && r_ < r_len && k_ < k_len;
+      const int rr = ok ? r_ : 0, kk = ok ? k_ : 0;
+      // this lane's tokens 8q .. 8q+7 are chunks 2q and 2q+1; it starts with the one of its slot's parity
+      const int t_first = 8 * q + 4 * (slot & 1);
+      off[i] = ((uint32_t)sdd_phys(rr, t_first) << 16) | (uint32_t)sdd_phys(kk, t_first);
+      if (i == 0 || (off[i] & 0xffffu) != (off[i - 1] & 0xffffu)) newcol |= 1u << i;
+      if (ok) valid |= 1u << i;
       acc[i] = 0.f;
     }
-    SubTile<T, TT> nxt;
-    if (ta < tb) nxt.load(dY, Z, tb, d_out, d_in, ta, r0, r_len, k0, k_len);
-    for (int64_t t0 = ta; t0 < tb; t0 += TT) {
-      __syncthreads();  // the previous sub-tile is consumed
-      nxt.store(s_dy, s_z);
+    using St = SddStage<T>;
+    if (ta < tb) St::copy(raw, dY, Z, tb, d_out, d_in, ta, r0, r_len, k0, k_len);
+    int buf = 0;
+    for (int64_t t0 = ta; t0 < tb; t0 += kSddmmTT, buf ^= 1) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();  // this sub-tile is staged; the previous one is consumed
+      St::widen(raw + buf * (St::kRawBytes / sizeof(T)), s_dy, s_z);
       __syncthreads();
-      if (t0 + TT < tb) nxt.load(dY, Z, tb, d_out, d_in, t0 + TT, r0, r_len, k0, k_len);
-      int cur_k = -1;
-      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        static_assert(G == 8, "one 16-byte row slice per lane");
-        uint4 zr = make_uint4(0, 0, 0, 0);
+      if (t0 + kSddmmTT < tb)  // the other buffer was widened one iteration ago
+        St::copy(raw + (buf ^ 1) * (St::kRawBytes / sizeof(T)), dY, Z, tb, d_out, d_in, t0 + kSddmmTT, r0, r_len,
+                 k0, k_len);
+      ulonglong2 z0 = make_ulonglong2(0ull, 0ull), z1 = z0;
 #pragma unroll
-        for (int i = 0; i < kSddmmSlotEntries; ++i) {
-          if (rk[i] < 0) continue;
-          const int kq = rk[i] & 0xffff, rq = rk[i] >> 16;
-          if (kq != cur_k) {
-            zr = *reinterpret_cast<const uint4 *>(s_z + kq * TT + G * q);
-            cur_k = kq;
-          }
-          const uint4 yr = *reinterpret_cast<const uint4 *>(s_dy + rq * TT + G * q);
-          // bf16 x bf16 products are exact in fp32: no widening needed
-          float a0 = fma_bf16_lo(yr.x, zr.x, 0.f);
-          float a1 = fma_bf16_hi(yr.x, zr.x, 0.f);
-          a0 = fma_bf16_lo(yr.y, zr.y, a0);
-          a1 = fma_bf16_hi(yr.y, zr.y, a1);
-          a0 = fma_bf16_lo(yr.z, zr.z, a0);
-          a1 = fma_bf16_hi(yr.z, zr.z, a1);
-          a0 = fma_bf16_lo(yr.w, zr.w, a0);
-          a1 = fma_bf16_hi(yr.w, zr.w, a1);
-          acc[i] += a0 + a1;
+      for (int i = 0; i < E; ++i) {
+        if (newcol & (1u << i)) {
+          const uint32_t oz = off[i] & 0xffffu;
+          z0 = *reinterpret_cast<const ulonglong2 *>(s_z + oz);
+          z1 = *reinterpret_cast<const ulonglong2 *>(s_z + (oz ^ 4u));
         }
-      } else {
-        float zv[G];
-#pragma unroll
-        for (int i = 0; i < kSddmmSlotEntries; ++i) {
-          if (rk[i] < 0) continue;
-          const int kq = rk[i] & 0xffff, rq = rk[i] >> 16;
-          if (kq != cur_k) {
-            load_vals<T>(s_z + kq * TT + G * q, zv, G);
-            cur_k = kq;
-          }
-          float yv[G];
-          load_vals<T>(s_dy + rq * TT + G * q, yv, G);
-          float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-          for (int u = 0; u < G; u += 2) {
-            a0 = fmaf(yv[u], zv[u], a0);
-            a1 = fmaf(yv[u + 1], zv[u + 1], a1);
-          }
-          acc[i] += a0 + a1;
-        }
+        const uint32_t oy = off[i] >> 16;
+        const ulonglong2 y0 = *reinterpret_cast<const ulonglong2 *>(s_dy + oy);
+        const ulonglong2 y1 = *reinterpret_cast<const ulonglong2 *>(s_dy + (oy ^ 4u));
+        unsigned long long t2 = ffma2(y0.x, z0.x, 0ull);
+        t2 = ffma2(y0.y, z0.y, t2);
+        t2 = ffma2(y1.x, z1.x, t2);
+        t2 = ffma2(y1.y, z1.y, t2);
+        acc[i] += __uint_as_float((uint32_t)t2) + __uint_as_float((uint32_t)(t2 >> 32));
       }
     }
 #pragma unroll
-    for (int i = 0; i < kSddmmSlotEntries; ++i) {
-      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 1);
-      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
-    }
-    if (q == 0) {
-#pragma unroll
-      for (int i = 0; i < kSddmmSlotEntries; ++i)
-        if (rk[i] >= 0) {
-          const int j = tile_pos[my0 + i];
-          if ((uint64_t)j < (uint64_t)p) part[j] = acc[i];
-        }
+    for (int i = 0; i < E; ++i) {
+      float s = acc[i];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (q == 0 && (valid & (1u << i))) {
+        const int j = tile_pos[my0 + i];
+        if ((uint64_t)j < (uint64_t)p) part[j] = s;
+      }
     }
     __syncthreads();
   }
@@ -522,12 +534,16 @@ cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T
   if (e != cudaSuccess) return e;
   if (T > 0) {
     dim3 grid((unsigned)tiles, (unsigned)n_chunks);
+    const size_t smem = dt == QWHA_BF16 ? sddmm_smem<__nv_bfloat16>() : sddmm_smem<float>();
+    e = cudaFuncSetAttribute(dt == QWHA_BF16 ? (const void *)sddmm_kernel<__nv_bfloat16> : (const void *)sddmm_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     if (dt == QWHA_BF16)
-      sddmm_kernel<__nv_bfloat16><<<grid, kSddmmThreads, 0, s>>>(
+      sddmm_kernel<__nv_bfloat16><<<grid, kSddmmThreads, smem, s>>>(
           static_cast<const __nv_bfloat16 *>(dY), static_cast<const __nv_bfloat16 *>(Z), T, d_out, d_in, tile_ptr,
           tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
     else
-      sddmm_kernel<float><<<grid, kSddmmThreads, 0, s>>>(static_cast<const float *>(dY),
+      sddmm_kernel<float><<<grid, kSddmmThreads, smem, s>>>(static_cast<const float *>(dY),
                                                          static_cast<const float *>(Z), T, d_out, d_in, tile_ptr,
                                                          tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
     e = cudaGetLastError();
