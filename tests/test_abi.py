@@ -48,3 +48,34 @@ def test_status_strings_and_host_checks():
     assert h.qwha_fwht(0, None, None, 0, 256, 256, None) == 0  # nothing to do
     tile = int(next(l.split()[2] for l in open(HEADER) if l.startswith("#define QWHA_TILE")))
     assert h.qwha_plan_tiles(4096, 14336) == -(-4096 // tile) * -(-14336 // tile)
+
+
+def test_host_checks_of_init_variants_and_refinement():
+    """The selection, refinement and split-AdaAlloc entry points reject bad arguments on the host, before any CUDA
+    call (no GPU needed), and name the problem."""
+    _ensure_built()
+    import walsh_hadamard_sparse_b200._lib as L
+
+    h = L.lib()
+    P = ctypes.c_void_p
+    dummy = P(4096)
+    # p above d_out * d_in
+    assert h.qwha_init_select_global(dummy, 4, 8, 8, 33, 0, 7, dummy, dummy, dummy, dummy, dummy, 1 << 20, None) == 1
+    # unknown selection rule
+    assert h.qwha_init_select_global(dummy, 4, 8, 8, 8, 5, 7, dummy, dummy, dummy, dummy, dummy, 1 << 20, None) == 1
+    # d_in not a multiple of 8 (row strides of the tensor-core operands)
+    assert h.qwha_calib_hessian(dummy, 16, 12, dummy, None) == 1
+    assert h.qwha_calib_hessian(dummy, 0, 64, dummy, None) == 1  # no calibration rows
+    assert h.qwha_refine_values(dummy, 4, 12, 4, dummy, ctypes.c_float(0.0), dummy, dummy, 8, dummy, dummy, 1 << 20,
+                                None) == 1
+    assert h.qwha_refine_values(dummy, 4, 64, 64, dummy, ctypes.c_float(-1.0), dummy, dummy, 8, dummy, dummy, 1 << 20,
+                                None) == 1  # negative damping
+    assert b"damp" in h.qwha_last_error()
+    # workspace below the need
+    assert h.qwha_refine_values(dummy, 4, 64, 64, dummy, ctypes.c_float(0.0), dummy, dummy, 8, dummy, dummy, 16,
+                                None) == 4
+    # split AdaAlloc: bad remainder mode, p out of range
+    assert h.qwha_init_budgets(dummy, 4, 8, 16, 2, 9, dummy, dummy, dummy, 1 << 20, None) == 1
+    assert h.qwha_init_budgets(dummy, 4, 8, 4, 2, 0, dummy, dummy, dummy, 1 << 20, None) == 1  # p < 2 * d_out
+    assert h.qwha_init_select(dummy, 4, 96, 64, dummy, dummy, 8, dummy, dummy, None) == 1  # 64 does not divide 96
+    assert h.qwha_workspace_size(7, 64, 64, 100, 0, 0) > 0 and h.qwha_workspace_size(6, 64, 64, 100, 0, 0) > 0

@@ -42,6 +42,12 @@ int sm_count() {
   return counts[dev];
 }
 
+int device_slot() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  return dev;
+}
+
 }  // namespace qwha
 
 using namespace qwha;

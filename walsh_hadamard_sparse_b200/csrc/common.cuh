@@ -26,6 +26,7 @@ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 int sm_count();  // multiprocessors of the current device
+int device_slot();  // index of the current device in [0, 64) (0 if unreadable), for per-device caches
 
 // Device error word for bounded waits (set by kernels, read by
 // qwha_check_stream_status). One per device, in __device__ memory.

@@ -418,11 +418,12 @@ cudaError_t run_rows(const Tin *x, Tout *z, int64_t rows, float scale, cudaStrea
   constexpr int RPC = kThreads / G::P;
   const size_t smem = (size_t)RPC * G::N * (sizeof(float) + sizeof(Tin));
   auto k = fwht_rows_kernel<LOGN, V, Tin, Tout>;
-  static bool attr_done = false;  // per instantiation
-  if (!attr_done) {
+  static bool attr_done[64] = {};  // per instantiation and device
+  const int slot = device_slot();
+  if (!attr_done[slot]) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    attr_done[slot] = true;
   }
   int occ = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, smem);

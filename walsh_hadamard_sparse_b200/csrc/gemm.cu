@@ -615,7 +615,8 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, uint3
 // of one cluster slot).
 template <int kMode, int CG, int kZ>
 int resident_groups() {
-  static int n = 0;
+  static int cached[64] = {};  // per device
+  int &n = cached[device_slot()];
   if (n) return n;
   using C = Cfg<CG, kMode, kZ>;
   const int sms = sm_count();
@@ -652,11 +653,12 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
   const bool ok_b = b_mn ? make_map(&tb, B, K, N, 64) : make_map(&tb, B, N, K, C::kBRows);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   auto kern = gemm_bf16_tcgen05_kernel<kMode, CG, kZ>;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[64] = {};  // per device
+  bool &attr_done = attr[device_slot()];
+  if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr_done = true;
   }
   const int64_t m_tiles = cdiv(M, (int64_t)BM * CG), n_tiles = cdiv(N, BN);
   const int64_t tiles = m_tiles * n_tiles;
