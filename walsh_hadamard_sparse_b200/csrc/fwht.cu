@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kThreads)
   extern __shared__ __align__(16) float smem[];
   const int rl = threadIdx.x / G::P;
   const int t = threadIdx.x % G::P;
-  float *buf = smem + rl * G::N;
+  float *buf = smem + rl * G::NP;
   const int nb = d_in >> LOGN;
   const int64_t blocks = n_rows * nb;
   const int64_t row_bytes = (int64_t)d_in * bits / 8;
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t r = active ? bi / nb : 0;
     const int k0 = active ? (int)(bi % nb) << LOGN : 0;
     __syncthreads();  // the previous iteration's readers are done with buf
-    for (int i = t; i < G::N; i += G::P) buf[i] = 0.f;
+    for (int i = t; i < G::NP; i += G::P) buf[i] = 0.f;
     __syncthreads();
     if (active) {
       int64_t b = row_ptr[r], e = row_ptr[r + 1];
@@ -214,10 +214,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ __align__(16) float smem[];
   const int rl = threadIdx.x / G::P;
   const int t = threadIdx.x % G::P;
-  float *buf = smem + rl * G::N;
-  int32_t *my_k = reinterpret_cast<int32_t *>(smem + RPC * G::N) + rl * CAP;
-  float *my_v = reinterpret_cast<float *>(smem + RPC * G::N + RPC * CAP) + rl * CAP;
-  uint8_t *dq = reinterpret_cast<uint8_t *>(smem + RPC * G::N + 2 * RPC * CAP);
+  float *buf = smem + rl * G::NP;
+  int32_t *my_k = reinterpret_cast<int32_t *>(smem + RPC * G::NP) + rl * CAP;
+  float *my_v = reinterpret_cast<float *>(smem + RPC * G::NP + RPC * CAP) + rl * CAP;
+  uint8_t *dq = reinterpret_cast<uint8_t *>(smem + RPC * G::NP + 2 * RPC * CAP);
   const int nb = d_in >> LOGN;
   const int64_t blocks = n_rows * nb;
   const int64_t row_bytes = (int64_t)d_in * bits / 8;
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int k0 = active ? (int)(bi % nb) << LOGN : 0;
     cp_async_wait_all();
     __syncthreads();  // this block's inputs are staged; the previous iteration is done with buf
-    for (int i = 4 * t; i < G::N; i += 4 * G::P) *reinterpret_cast<float4 *>(buf + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 4 * t; i < G::NP; i += 4 * G::P) *reinterpret_cast<float4 *>(buf + i) = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
     if (active) {
       const int n = (int)(e - b < CAP ? e - b : CAP);
@@ -381,7 +381,7 @@ cudaError_t run_weff(const int32_t *row_ptr, const int32_t *col_idx, const float
     dq_stride = round16((int)qb) + round16(gpb * 4) + round16(gpb);
   }
   if (pipe) {
-    const size_t smem = (size_t)RPC * G::N * sizeof(float) + 2ull * RPC * weff_csr_cap<LOGN>() * 4 +
+    const size_t smem = (size_t)RPC * G::NP * sizeof(float) + 2ull * RPC * weff_csr_cap<LOGN>() * 4 +
                         2ull * RPC * dq_stride;
     auto k = weff_pipe_kernel<LOGN>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -396,7 +396,7 @@ cudaError_t run_weff(const int32_t *row_ptr, const int32_t *col_idx, const float
                                                                  bits, group, qw, scales, zeros, out, dq_stride);
     return cudaGetLastError();
   }
-  const size_t smem = (size_t)RPC * G::N * sizeof(float);
+  const size_t smem = (size_t)RPC * G::NP * sizeof(float);
   auto k = weff_rows_kernel<LOGN>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -416,7 +416,7 @@ cudaError_t run_rows(const Tin *x, Tout *z, int64_t rows, float scale, cudaStrea
   constexpr int V = (sizeof(Tin) == 2 || sizeof(Tout) == 2) ? 8 : 4;
   using G = Geo<LOGN, V>;
   constexpr int RPC = kThreads / G::P;
-  const size_t smem = (size_t)RPC * G::N * (sizeof(float) + sizeof(Tin));
+  const size_t smem = (size_t)RPC * ((size_t)G::NP * sizeof(float) + (size_t)G::N * sizeof(Tin));
   auto k = fwht_rows_kernel<LOGN, V, Tin, Tout>;
   static bool attr_done[64] = {};  // per instantiation and device
   const int slot = device_slot();

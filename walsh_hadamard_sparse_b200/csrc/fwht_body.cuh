@@ -18,10 +18,9 @@ struct Geo {
   static constexpr int P = 1 << PB;
   static constexpr int NB = 2 * RB - LOGN;  // batch bits in phase B (0 or 1)
   static constexpr int HB = RB - LV;        // high bits in phase-A registers
-  static constexpr int S0 = 5 - LV;
-  static constexpr int S1 = PB < S0 ? PB : S0;
-  static constexpr int S = (HB - NB) < S1 ? (HB - NB) : S1;  // swizzle bits
-  static constexpr int SMASK = (1 << S) - 1;
+  // the transpose buffer holds a row with V padding floats after every block
+  // of 2^(LV+PB) elements (one value of the high field), NP floats in all
+  static constexpr int NP = N + (N >> (LV + PB)) * V;
   static_assert(HB >= NB && HB >= 0 && PB >= LV, "row too short for this layout");
 
   // element index of register q of thread t, phase A
@@ -33,10 +32,11 @@ struct Geo {
     return (t & (V - 1)) | ((q & (P - 1)) << LV) | ((t >> LV) << (LV + PB)) |
            ((q >> PB) << (LV + PB + HB - NB));
   }
-  // swizzled position in the transpose buffer
-  __device__ __forceinline__ static int phys(int e) {
-    return e ^ (((e >> (LV + PB)) & SMASK) << LV);
-  }
+  // position in the transpose buffer. The padding shifts each block of the
+  // high field by V banks, so the phase-B lanes (low field t % V, high field
+  // t / V) meet 32 distinct banks, and every position is a per-thread base
+  // plus a constant of the register index (no per-access arithmetic).
+  __device__ __forceinline__ static int phys(int e) { return e + (e >> (LV + PB)) * V; }
 };
 
 template <typename T, int V>
@@ -116,7 +116,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // takes rows cta*RPC, (cta + n_cta)*RPC, ... The input rows of the next
 // iteration are copied into a shared-memory staging buffer with cp.async while
 // the current rows are transformed; phase A then reads its 16-byte vectors
-// from shared memory. smem: NT/P rows x (n floats + n input values).
+// from shared memory. smem: NT/P rows x (Geo::NP floats + n input values).
 template <int LOGN, int V, typename Tin, typename Tout, int NT, typename Bar>
 __device__ __forceinline__ void fwht_rows_body(const Tin *__restrict__ x, Tout *__restrict__ z, int64_t rows,
                                                float scale, float *smem, int tid, int cta, int n_cta,
@@ -127,8 +127,8 @@ __device__ __forceinline__ void fwht_rows_body(const Tin *__restrict__ x, Tout *
   constexpr int ROW_CHUNKS = G::N * (int)sizeof(Tin) / 16;
   const int rl = tid / G::P;
   const int t = tid % G::P;
-  float *buf = smem + rl * G::N;
-  Tin *stage = reinterpret_cast<Tin *>(smem + RPC * G::N);
+  float *buf = smem + rl * G::NP;
+  Tin *stage = reinterpret_cast<Tin *>(smem + RPC * G::NP);
 
   auto prefetch = [&](int64_t first) {
     const int64_t left = rows - first;

@@ -64,7 +64,9 @@ constexpr int kZThreads = 128;
 template <int kZ>
 constexpr size_t z_smem() {
   if constexpr (kZ == 0) return 0;
-  else return (size_t)(kZThreads / Geo<kZ, 8>::P) * (1u << kZ) * (sizeof(float) + sizeof(__nv_bfloat16));
+  else
+    return (size_t)(kZThreads / Geo<kZ, 8>::P) *
+           ((size_t)Geo<kZ, 8>::NP * sizeof(float) + (size_t)(1u << kZ) * sizeof(__nv_bfloat16));
 }
 
 template <int CG, int kMode = kOutBf16, int kZ = 0>
