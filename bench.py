@@ -245,6 +245,85 @@ def config_block(spec, n):
 # --------------------------------------------------------------------------- main
 
 
+def run_block(args):
+    """The decoder-block workload (seven LLaMA-3-8B-shaped linears, 32768 tokens, 4-bit g128, r = 64): forward of
+    every layer then backward in reverse order, dense algorithm, with the transform Z = X H shared by the layers
+    that read the same input (q, k, v; gate, up) and, for comparison, computed by every layer. Weights and
+    AdaAlloc as in the tests (host-generated seeded weights, AdaAlloc on the GPU); the activations are drawn on
+    the GPU from a seeded generator with the workload's distribution (N(0, 1), 1% of input channels x20)."""
+    import torch
+
+    import walsh_hadamard_sparse_b200 as W
+    from workloads.synth import _x_channels
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    specs = CONFIGS["block"]
+    T = specs[0].T
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed)
+    layers, X, Zb, dY, Y, dX, dc = [], {}, {}, {}, {}, {}, {}
+    for spec in specs:
+        d = layer_inputs(spec, args.seed, "block", parts=("W",))
+        dWq = torch.from_numpy(d["dWq"]).to(dev)
+        e = W.init_alloc(dWq, spec.p, spec.had_block, spec.min_per_row, spec.remainder)
+        del dWq
+        wq = W.QWeight(spec.bits, spec.group, torch.from_numpy(d["qweight"]).to(dev),
+                       torch.from_numpy(d["scales"]).to(dev), torch.from_numpy(d["zeros"]).to(dev))
+        a = W.Adapter(spec.d_in, spec.d_out, spec.had_block, spec.p, e["row_ptr"], e["col_idx"], e["coef"],
+                      algo="dense")
+        a.weff = torch.empty((spec.d_out, spec.d_in), dtype=torch.bfloat16, device=dev)
+        layers.append((spec, a, wq))
+        if spec.x_stream not in X:
+            x = torch.randn((T, spec.d_in), generator=gen, device=dev)
+            ch = torch.from_numpy(_x_channels(spec, args.seed, "block")).to(dev)
+            x[:, ch] *= spec.x_outlier_scale
+            X[spec.x_stream] = x.to(torch.bfloat16)
+            Zb[spec.x_stream] = torch.empty_like(X[spec.x_stream])
+            del x
+        dY[spec.name] = torch.randn((T, spec.d_out), generator=gen, device=dev).to(torch.bfloat16)
+        Y[spec.name] = torch.empty((T, spec.d_out), dtype=torch.bfloat16, device=dev)
+        dX[spec.name] = torch.empty((T, spec.d_in), dtype=torch.bfloat16, device=dev)
+        dc[spec.name] = torch.empty(spec.p, dtype=torch.float32, device=dev)
+
+    def step(shared):
+        seen = set()
+        for spec, a, wq in layers:
+            given = shared and spec.x_stream in seen
+            W.adapter_fwd(a, X[spec.x_stream], 1.0, wq, Z_out=Zb[spec.x_stream], Y=Y[spec.name], z_given=given)
+            seen.add(spec.x_stream)
+        for spec, a, wq in reversed(layers):
+            W.adapter_bwd(a, dY[spec.name], Zb[spec.x_stream], 1.0, wq, dc=dc[spec.name], dX=dX[spec.name])
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    res = {}
+    K = max(3, min(args.steps, 10))
+    for shared in (True, False):
+        for _ in range(max(args.warmup, 3)):
+            step(shared)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record()
+            step(shared)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        res[shared] = sum(s_.elapsed_time(e_) for s_, e_ in ev) / K
+    flops = sum(3 * 2.0 * T * sp.d_in * sp.d_out for sp in specs)
+    line = {
+        "metric": "decoder block (7 adapted linears) fwd+bwd tokens/s", "value": T / (res[True] / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": K, "ms_per_step": res[True], "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic (seeded; weights host-generated, activations drawn on the GPU)",
+        "config": {"workload": "block: LLaMA-3-8B q/k/v/o/gate/up/down, T=32768 (8 x 4096), 4-bit g128, r=64",
+                   "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write)"},
+        "algorithm": "dense; Z = X H shared by q/k/v and by gate/up (z_given)",
+        "gemm_tflops": flops / (res[True] / 1e3) / 1e12,
+        "without_sharing": {"ms_per_step": res[False], "value": T / (res[False] / 1e3)},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -255,11 +334,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--sparse-steps", type=int, default=40)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["q_proj", "block"], default="q_proj",
+                    help="block: time the decoder-block workload (seven linears) instead of the q_proj step")
     ap.add_argument("--no-init-extras", action="store_true",
                     help="skip timing the selection variants and Value Refinement (one-off setup, not the step)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     spec = CONFIGS[WORKLOAD][0]
+    if args.workload == "block" and args.impl == "ours":
+        return run_block(args)
     if args.impl == "reference":
         return run_reference(args, spec)
 
