@@ -98,4 +98,42 @@ __device__ __forceinline__ void st_stream(void *p, const uint4 &v) {
                : "memory");
 }
 
+// One pass of NB butterfly stages (h = 2^s .. 2^(s+NB-1)) over v[0..d) of
+// fp32 values in shared memory: each thread takes aligned groups of 2^NB
+// elements into registers (compile-time indices, no local memory).
+template <int NB>
+__device__ __forceinline__ void butterfly_pass_f32(float *v, int d, int s) {
+  constexpr int GS = 1 << NB;
+  for (int g = threadIdx.x; g < (d >> NB); g += blockDim.x) {
+    const int lo = g & ((1 << s) - 1);
+    const int base = ((g >> s) << (s + NB)) | lo;
+    float x[GS];
+#pragma unroll
+    for (int i = 0; i < GS; ++i) x[i] = v[base + (i << s)];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int i = 0; i < GS; ++i)
+        if (!(i & (1 << b))) {
+          const float a = x[i], c = x[i + (1 << b)];
+          x[i] = a + c;
+          x[i + (1 << b)] = a - c;
+        }
+#pragma unroll
+    for (int i = 0; i < GS; ++i) v[base + (i << s)] = x[i];
+  }
+}
+
+// All logn stages, three per pass (the last pass one or two), with a block
+// barrier after each pass.
+__device__ __forceinline__ void butterflies_smem_f32(float *v, int d, int logn) {
+  for (int s = 0; s < logn; s += 3) {
+    const int nb = (logn - s) < 3 ? (logn - s) : 3;
+    if (nb == 3) butterfly_pass_f32<3>(v, d, s);
+    else if (nb == 2) butterfly_pass_f32<2>(v, d, s);
+    else butterfly_pass_f32<1>(v, d, s);
+    __syncthreads();
+  }
+}
+
 }  // namespace qwha

@@ -47,25 +47,7 @@ __global__ void __launch_bounds__(kWeffThreads)
   }
   __syncthreads();
   // butterflies on index bits [0, logn): per block of 2^logn, three stages per pass
-  for (int s = 0; s < logn; s += 3) {
-    const int nb = min(3, logn - s);
-    const int gsz = 1 << nb;
-    for (int g = threadIdx.x; g < (d_in >> nb); g += blockDim.x) {
-      const int lo = g & ((1 << s) - 1);
-      const int base = ((g >> s) << (s + nb)) | lo;
-      float v[8];
-      for (int i = 0; i < gsz; ++i) v[i] = row[base + (i << s)];
-      for (int bb = 0; bb < nb; ++bb)
-        for (int i = 0; i < gsz; ++i)
-          if (!(i & (1 << bb))) {
-            const float a = v[i], c = v[i + (1 << bb)];
-            v[i] = a + c;
-            v[i + (1 << bb)] = a - c;
-          }
-      for (int i = 0; i < gsz; ++i) row[base + (i << s)] = v[i];
-    }
-    __syncthreads();
-  }
+  butterflies_smem_f32(row, d_in, logn);
   // + dequantized base row, one rounding to bf16, 8 values per thread
   const int64_t row_bytes = (int64_t)d_in * bits / 8;
   const int ng = qw ? d_in / group : 0;

@@ -69,25 +69,7 @@ __global__ void __launch_bounds__(512) fwht_large_kernel(const Tin *__restrict__
     __syncthreads();
     for (int i = threadIdx.x; i < N; i += blockDim.x) smem[i] = io<Tin>::load1(x + row * N + i);
     __syncthreads();
-    for (int s = 0; s < logn; s += 3) {
-      const int nb = (logn - s) < 3 ? (logn - s) : 3;
-      const int gsz = 1 << nb;
-      for (int g = threadIdx.x; g < (N >> nb); g += blockDim.x) {
-        const int lo = g & ((1 << s) - 1);
-        const int base = ((g >> s) << (s + nb)) | lo;
-        float v[8];
-        for (int i = 0; i < gsz; ++i) v[i] = smem[base + (i << s)];
-        for (int b = 0; b < nb; ++b)
-          for (int i = 0; i < gsz; ++i)
-            if (!(i & (1 << b))) {
-              const float a = v[i], c = v[i + (1 << b)];
-              v[i] = a + c;
-              v[i + (1 << b)] = a - c;
-            }
-        for (int i = 0; i < gsz; ++i) smem[base + (i << s)] = v[i];
-      }
-      __syncthreads();
-    }
+    butterflies_smem_f32(smem, N, logn);
     for (int i = threadIdx.x; i < N; i += blockDim.x) io<Tout>::store1(z + row * N + i, smem[i] * scale);
   }
 }

@@ -160,29 +160,52 @@ __global__ void __launch_bounds__(kNormThreads) row_norm_kernel(const float *__r
 // shared by nearly all keys, so per-key atomics would serialise), and warp 0
 // finds the digit holding the `need`-th key with a shuffle scan over the 256
 // bins (8 per lane).
+constexpr int kCandCap = 1024;  // candidate list of the radix select (indices)
+
 template <typename KeyF, typename OkF>
 __device__ void radix_select_smallest(int n, int64_t want, KeyF key, OkF ok, uint32_t *hist, uint64_t *K_out,
                                       int64_t *need_out) {
   __shared__ int sel_digit;
   __shared__ int64_t sel_need;
+  // Once the keys that still match the prefix are at most kCandCap, the next
+  // pass also lists their indices, and the passes after it scan that list
+  // instead of all n keys (the digits found are the same).
+  __shared__ int cand[kCandCap];
+  __shared__ int cand_n;
+  __shared__ uint32_t match_count;  // keys matching the prefix after the last pass
   uint64_t prefix = 0;
   int64_t need = want;
   const int lane = threadIdx.x & 31;
-  const int n_round = (n + blockDim.x - 1) / blockDim.x * blockDim.x;  // whole warps iterate together
+  bool listing = false, listed = false;
+  if (threadIdx.x == 0) {
+    cand_n = 0;
+    match_count = 0xffffffffu;
+  }
+  __syncthreads();
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    listing = !listed && match_count <= (uint32_t)kCandCap;
     __syncthreads();
     const uint64_t hi_mask = shift == 56 ? 0 : (~0ull << (shift + 8));
-    for (int i = threadIdx.x; i < n_round; i += blockDim.x) {
+    const int m = listed ? cand_n : n;
+    const int m_round = (m + blockDim.x - 1) / blockDim.x * blockDim.x;  // whole warps iterate together
+    for (int it = threadIdx.x; it < m_round; it += blockDim.x) {
       int bin = 256;  // no count
-      if (i < n && ok(i)) {
-        const uint64_t k = key(i);
-        if ((k & hi_mask) == (prefix & hi_mask)) bin = (int)((k >> shift) & 255);
+      if (it < m) {
+        const int i = listed ? cand[it] : it;
+        if (listed || ok(i)) {
+          const uint64_t k = key(i);
+          if ((k & hi_mask) == (prefix & hi_mask)) {
+            bin = (int)((k >> shift) & 255);
+            if (listing) cand[atomicAdd(&cand_n, 1)] = i;
+          }
+        }
       }
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
       if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
+    if (listing) listed = true;
     if (threadIdx.x < 32) {
       uint32_t c[8];
       uint32_t mine = 0;
@@ -203,19 +226,23 @@ __device__ void radix_select_smallest(int n, int64_t want, KeyF key, OkF ok, uin
       if (hit) {
         int64_t cum = excl;
         int d = 8 * lane + 7;
+        uint32_t cnt = c[7];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (cum + c[j] >= need) {
             d = 8 * lane + j;
+            cnt = c[j];
             break;
           }
           cum += c[j];
         }
         sel_digit = d;
         sel_need = need - cum;
+        match_count = cnt;
       } else if (who == 0 && lane == 31) {  // fewer eligible keys than wanted: past the last digit
         sel_digit = 255;
         sel_need = need - (int64_t)incl;
+        match_count = c[7];
       }
     }
     __syncthreads();
@@ -351,30 +378,45 @@ __global__ void __launch_bounds__(kBudgetThreads)
   }
 }
 
+// One pass of NB butterfly stages (h = 2^s .. 2^(s+NB-1)) over v[0..d) in
+// shared memory: each thread takes aligned groups of 2^NB elements into
+// registers (compile-time indices), textbook order inside the group.
+template <int NB>
+__device__ __forceinline__ void butterfly_pass_fp64(double *v, int d, int s) {
+  constexpr int GS = 1 << NB;
+  for (int g = threadIdx.x; g < (d >> NB); g += blockDim.x) {
+    const int lo = g & ((1 << s) - 1);
+    const int base = ((g >> s) << (s + NB)) | lo;
+    double x[GS];
+#pragma unroll
+    for (int i = 0; i < GS; ++i) x[i] = v[base + (i << s)];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int i = 0; i < GS; ++i)
+        if (!(i & (1 << b))) {
+          const double a = x[i], c = x[i + (1 << b)];
+          x[i] = __dadd_rn(a, c);
+          x[i + (1 << b)] = __dsub_rn(a, c);
+        }
+#pragma unroll
+    for (int i = 0; i < GS; ++i) v[base + (i << s)] = x[i];
+  }
+}
+
 // v[0..d_in) = w[0..d_in) H_unnormalised per block of n, fp64 butterflies in
-// the textbook stage order (three stages per pass over aligned groups of 8);
-// v is shared memory, every thread of the block takes part.
+// the textbook stage order (three stages per pass over aligned groups of 8,
+// the last pass one or two when log2 n is not a multiple of 3); v is shared
+// memory, every thread of the block takes part.
 __device__ void row_transform_fp64(const float *__restrict__ w, int d_in, int n, double *v) {
   for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[k] = (double)w[k];
   __syncthreads();
   const int logn = 31 - __clz(n);
   for (int s = 0; s < logn; s += 3) {
     const int nb = min(3, logn - s);
-    const int gsz = 1 << nb;
-    for (int g = threadIdx.x; g < (d_in >> nb); g += blockDim.x) {
-      const int lo = g & ((1 << s) - 1);
-      const int base = ((g >> s) << (s + nb)) | lo;
-      double x[8];
-      for (int i = 0; i < gsz; ++i) x[i] = v[base + (i << s)];
-      for (int b = 0; b < nb; ++b)
-        for (int i = 0; i < gsz; ++i)
-          if (!(i & (1 << b))) {
-            const double a = x[i], c = x[i + (1 << b)];
-            x[i] = __dadd_rn(a, c);
-            x[i + (1 << b)] = __dsub_rn(a, c);
-          }
-      for (int i = 0; i < gsz; ++i) v[base + (i << s)] = x[i];
-    }
+    if (nb == 3) butterfly_pass_fp64<3>(v, d_in, s);
+    else if (nb == 2) butterfly_pass_fp64<2>(v, d_in, s);
+    else butterfly_pass_fp64<1>(v, d_in, s);
     __syncthreads();
   }
 }
