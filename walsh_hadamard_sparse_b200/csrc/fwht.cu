@@ -11,33 +11,207 @@
 // I/O type), middle (PB bits) and high (HB bits).
 //   phase A: a thread holds the low and high fields in registers (R = 2^RB
 //            values) and the middle field is its index inside the row's
-//            P = 2^PB threads. Global loads and stores are coalesced 16-byte
-//            vectors. All RB register bits get their butterflies.
-//   phase B: after a transpose through shared memory, a thread holds the middle
-//            field (plus, for odd m, one high bit as a batch bit) and does the
-//            remaining butterflies.
-// The transpose buffer is fp32 and XOR-swizzled (the middle field's low bits
-// are flipped by the high field's low bits) so that phase-B scalar accesses hit
-// 32 distinct banks and phase-A 16-byte accesses stay contiguous. The result
-// goes back through the same buffer (in the output type) to phase-A layout for
-// coalesced stores. Arithmetic is fp32 whatever the I/O type. The next rows'
-// inputs are prefetched with cp.async into shared memory during the arithmetic.
+//            P = 2^PB threads; its input vectors come from a shared-memory
+//            ring that bulk copies fill. All RB register bits get their
+//            butterflies.
+//   phase B: after a transpose through an fp32 shared-memory buffer, a thread
+//            holds the middle field (plus, for odd m, one high bit as a batch
+//            bit) and does the remaining butterflies; it writes the scaled
+//            results, in the output type, into per-segment staging that bulk
+//            copies send to global memory.
+// The transpose buffer is XOR-swizzled (RingGeo::phys) so that both phases'
+// accesses are free of bank conflicts. Arithmetic is fp32 whatever the I/O
+// type. fwht_body.cuh holds the same arithmetic for the fused forward GEMM and
+// the W_eff kernels below.
 
 #include "common.cuh"
 #include "fwht_body.cuh"
+#include "bulk.cuh"
 #include "kernels.h"
 
 namespace qwha {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kRingSlots = 2;  // ring depth of the transform kernel (measured best of 2, 3, 4)
 
-template <int LOGN, int V, typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads) fwht_rows_kernel(const Tin *__restrict__ x, Tout *__restrict__ z,
-                                                             int64_t rows, float scale) {
-  extern __shared__ __align__(16) float smem[];
-  fwht_rows_body<LOGN, V, Tin, Tout, kThreads>(x, z, rows, scale, smem, threadIdx.x, blockIdx.x, gridDim.x,
-                                               [] { __syncthreads(); });
+// Row transform for contiguous rows of 128 <= n <= 4096: a CTA is one worker
+// of RW = max(P, 64) threads (RW / P rows per iteration) that streams its rows
+// through an S-slot shared-memory ring filled by bulk copies (the TMA engine,
+// one copy per iteration, issued S iterations ahead), so loads are always in
+// flight without costing the threads issue slots or registers, and the CTA's
+// barriers span only its own warps. Results leave through bulk stores of
+// staged segments. Requires x and z 16-byte aligned.
+template <int LOGN, int V>
+struct RingGeo {
+  using G = Geo<LOGN, V>;
+  static constexpr int RW = G::P < 64 ? 64 : G::P;  // threads of the worker
+  static constexpr int RPW = RW / G::P;             // rows per iteration
+  // Exchange-buffer position of element e of local row rl, XOR-swizzled
+  // instead of padded. The low field splits into i (the 4 floats of a 16-byte
+  // access) and u (which 16-byte half of a narrow vector); u moves above the
+  // middle field m, and m's low 3 bits are flipped by s(u, high, rl). Phase-A
+  // 16-byte accesses (fixed h, u; lanes = consecutive m) then cover 128
+  // contiguous bytes per quarter warp, and phase-B scalar accesses (fixed m;
+  // lanes = i, u, high bits, rows) meet 32 distinct banks. Rows are N floats
+  // apart (no padding).
+  __device__ __forceinline__ static int swz(int u, int hh, int rl) {
+    return ((u | (hh << (G::LV - 2))) ^ (rl << (G::PB - 2))) & 7;
+  }
+  __device__ __forceinline__ static int phys(int e, int rl) {
+    const int i = e & 3, u = (e & (V - 1)) >> 2, m = (e >> G::LV) & (G::P - 1), hh = e >> (G::LV + G::PB);
+    return rl * G::N + (i | ((m ^ swz(u, hh, rl)) << 2) | (u << (2 + G::PB)) | (hh << (G::LV + G::PB)));
+  }
+  // output staging: a segment per (row, high field) value holds the SEGE
+  // contiguous output elements of that value, segp() elements apart: one
+  // vector (V elements) of padding moves each segment by as many banks as a
+  // vector spans, so the phase-B lanes of one store meet distinct banks
+  // (two-way for fp32 output at n = 128 and 512)
+  static constexpr int SEGE = 1 << (G::LV + G::PB);
+  template <typename T>
+  __host__ __device__ static constexpr int segp() { return SEGE + V; }
+  // the exchange buffer (RPW rows of N floats) and the output staging, which
+  // reuses it: the larger of the two, rounded to 128 bytes
+  template <typename T>
+  __host__ __device__ static constexpr int buf_bytes() {
+    const int a = RPW * G::N * 4, b = RPW * (1 << G::HB) * segp<T>() * (int)sizeof(T);
+    return ((a > b ? a : b) + 127) & ~127;
+  }
+  // phase A, half u of the vector of high index h: the swizzle's compile-time
+  // part and the offset beyond the thread's base pointer
+  __host__ __device__ static constexpr int sA(int u, int h) { return (u | (h << (G::LV - 2))) & 7; }
+  __host__ __device__ static constexpr int offA(int u, int h) { return (u << (2 + G::PB)) | (h << (G::LV + G::PB)); }
+  // phase B, register q: middle field q % P, batch bit q / P (the top high bit)
+  __host__ __device__ static constexpr int sB(int q) {
+    return ((q & 7) ^ (((q >> G::PB) << (G::HB - G::NB + G::LV - 2)) & 7)) & 7;
+  }
+  __host__ __device__ static constexpr int offB(int q) {
+    return (((q & (G::P - 1)) & ~7) << 2) | ((q >> G::PB) << (G::LV + G::PB + G::HB - G::NB));
+  }
+};
+
+template <int LOGN, int V, typename Tin, typename Tout, int S>
+__global__ void __launch_bounds__(RingGeo<LOGN, V>::RW) fwht_ring_kernel(const Tin *__restrict__ x,
+                                                                         Tout *__restrict__ z, int64_t rows,
+                                                                         float scale, unsigned int *err) {
+  using G = Geo<LOGN, V>;
+  using RG = RingGeo<LOGN, V>;
+  constexpr int RPW = RG::RPW;
+  constexpr int SLOT = RPW * G::N * (int)sizeof(Tin);  // bytes, a multiple of 16
+  constexpr int BUF = RG::template buf_bytes<Tout>();
+  static_assert(G::PB >= 3, "the swizzle needs 3 middle bits");
+
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  float *buf = reinterpret_cast<float *>(smem_raw);
+  unsigned char *ring = smem_raw + BUF;
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + S * SLOT);
+  const int tid = threadIdx.x;
+  const int rl = tid / G::P, t = tid % G::P;
+  const int64_t stride = (int64_t)gridDim.x * RPW;
+  const int64_t first = (int64_t)blockIdx.x * RPW;
+  const int64_t iters = first < rows ? (rows - first + stride - 1) / stride : 0;
+  // RG::phys unrolled: eight base pointers per phase (one per value of the
+  // swizzled low middle bits); everything else is a compile-time offset
+  const int rsw = (rl << (G::PB - 2)) & 7;
+  float *pa[8], *pb[8];
+  {
+    float *rb = buf + rl * G::N;
+    const int l = t & (V - 1), hB = t >> G::LV;
+    const int s0 = ((l >> 2) | (hB << (G::LV - 2))) ^ rsw;
+    float *bb = rb + (l & 3) + ((l >> 2) << (2 + G::PB)) + (hB << (G::LV + G::PB));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      pa[j] = rb + ((((t ^ j ^ rsw) & 7) | (t & ~7)) << 2);
+      pb[j] = bb + (((j ^ s0) & 7) << 2);
+    }
+  }
+
+  auto issue = [&](int64_t it) {  // thread 0: copy iteration it's rows into its slot
+    const int64_t r0 = first + it * stride;
+    const int64_t left = rows - r0;
+    const uint32_t bytes = (uint32_t)((left < RPW ? left : RPW) * G::N * (int64_t)sizeof(Tin));
+    const int s = (int)(it % S);
+    bulk::fence_proxy();
+    bulk::load(bulk::saddr(ring + s * SLOT), x + r0 * G::N, bytes, bulk::saddr(full + s));
+  };
+
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) bulk::init(bulk::saddr(full + s), 1);
+    bulk::fence_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int64_t it = 0; it < S && it < iters; ++it) issue(it);
+
+  for (int64_t it = 0; it < iters; ++it) {
+    const int s = (int)(it % S);
+    const int64_t row = first + it * stride + rl;
+    const bool active = row < rows;
+    const bool ok = bulk::wait(bulk::saddr(full + s), (uint32_t)((it / S) & 1));
+    if (tid == 0) bulk::wait_stores_read();  // the last iteration's output copies have read buf
+    // every thread has left the previous iteration's output reads of buf
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) {
+        atomicOr(err, 0x200u);
+        // let the copies already issued land (bounded) before the CTA exits
+        for (int64_t j = it; j < iters && j < it + S; ++j)
+          (void)bulk::wait(bulk::saddr(full + (int)(j % S)), (uint32_t)((j / S) & 1));
+      }
+      return;
+    }
+    float v[G::R];
+    if (active) {
+      const Tin *xr = reinterpret_cast<const Tin *>(ring + s * SLOT) + rl * G::N;
+#pragma unroll
+      for (int h = 0; h < (1 << G::HB); ++h) {
+        const Tin *src = xr + G::eA(t, h << G::LV);
+#pragma unroll
+        for (int u = 0; u < V; u += io<Tin>::kVec)
+          io<Tin>::unpack(*reinterpret_cast<const uint4 *>(src + u), v + h * V + u);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < G::R; ++q) v[q] = 0.f;
+    }
+    butterflies_x2<G::R, 0, G::RB, 0>(v);
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+#pragma unroll
+      for (int u = 0; u < V; u += 4)
+        *reinterpret_cast<float4 *>(pa[RG::sA(u >> 2, h)] + RG::offA(u >> 2, h)) =
+            make_float4(v[h * V + u], v[h * V + u + 1], v[h * V + u + 2], v[h * V + u + 3]);
+    }
+    __syncthreads();  // phase A is in buf and slot s is consumed: refill it
+    if (tid == 0 && it + S < iters) issue(it + S);
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) v[q] = pb[RG::sB(q)][RG::offB(q)];
+    butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
+    __syncthreads();  // all phase-B reads done before the buffer is reused
+    // results straight from phase B into the buffer in the output type, one
+    // padded segment per (row, high field) value, written to global memory by
+    // bulk copies from one thread, so no thread re-reads them
+    Tout *ob = reinterpret_cast<Tout *>(smem_raw) + (rl * (1 << G::HB) + (t >> G::LV)) * RG::template segp<Tout>() +
+               (t & (V - 1));
+#pragma unroll
+    for (int q = 0; q < G::R; ++q)
+      io<Tout>::store1(ob + (q >> G::PB) * (1 << (G::HB - G::NB)) * RG::template segp<Tout>() +
+                           ((q & (G::P - 1)) << G::LV),
+                       v[q] * scale);
+    bulk::fence_proxy();  // these writes before the copy engine's reads
+    __syncthreads();
+    if (tid == 0) {
+      const int64_t r0 = first + it * stride;
+      const int nrow = rows - r0 < RPW ? (int)(rows - r0) : RPW;
+      for (int r = 0; r < nrow; ++r)
+        for (int hh = 0; hh < (1 << G::HB); ++hh)
+          bulk::store(z + (r0 + r) * G::N + hh * RG::SEGE,
+                      bulk::saddr(reinterpret_cast<Tout *>(smem_raw) + (r * (1 << G::HB) + hh) * RG::template segp<Tout>()),
+                      RG::SEGE * (int)sizeof(Tout));
+      bulk::commit();
+    }
+  }
+  if (tid == 0) bulk::wait_stores();  // the buffer stays valid until the last copy has read it
 }
 
 // n <= 64: one thread per block, all in registers.
@@ -393,13 +567,13 @@ cudaError_t run_weff(const int32_t *row_ptr, const int32_t *col_idx, const float
   return cudaGetLastError();
 }
 
-template <int LOGN, typename Tin, typename Tout>
-cudaError_t run_rows(const Tin *x, Tout *z, int64_t rows, float scale, cudaStream_t s) {
+template <int LOGN, typename Tin, typename Tout, int S>
+cudaError_t run_ring(const Tin *x, Tout *z, int64_t rows, float scale, cudaStream_t s) {
   constexpr int V = (sizeof(Tin) == 2 || sizeof(Tout) == 2) ? 8 : 4;
   using G = Geo<LOGN, V>;
-  constexpr int RPC = kThreads / G::P;
-  const size_t smem = (size_t)RPC * ((size_t)G::NP * sizeof(float) + (size_t)G::N * sizeof(Tin));
-  auto k = fwht_rows_kernel<LOGN, V, Tin, Tout>;
+  using RG = RingGeo<LOGN, V>;
+  const size_t smem = (size_t)RG::template buf_bytes<Tout>() + (size_t)S * RG::RPW * G::N * sizeof(Tin) + (size_t)S * 8;
+  auto k = fwht_ring_kernel<LOGN, V, Tin, Tout, S>;
   static bool attr_done[64] = {};  // per instantiation and device
   const int slot = device_slot();
   if (!attr_done[slot]) {
@@ -408,13 +582,13 @@ cudaError_t run_rows(const Tin *x, Tout *z, int64_t rows, float scale, cudaStrea
     attr_done[slot] = true;
   }
   int occ = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kThreads, smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, RG::RW, smem);
   if (e != cudaSuccess) return e;
   if (occ < 1) occ = 1;
-  const int64_t need = cdiv(rows, RPC);
+  const int64_t need = cdiv(rows, RG::RPW);
   const int64_t cap = (int64_t)sm_count() * occ;
   const int grid = (int)(need < cap ? need : cap);
-  k<<<grid, kThreads, smem, s>>>(x, z, rows, scale);
+  k<<<grid, RG::RW, smem, s>>>(x, z, rows, scale, device_error_word());
   return cudaGetLastError();
 }
 
@@ -448,12 +622,12 @@ cudaError_t dispatch(const void *xv, void *zv, int64_t rows, int logn, float sca
     case 4: return run_small<4>(x, z, rows, scale, s);
     case 5: return run_small<5>(x, z, rows, scale, s);
     case 6: return run_small<6>(x, z, rows, scale, s);
-    case 7: return run_rows<7>(x, z, rows, scale, s);
-    case 8: return run_rows<8>(x, z, rows, scale, s);
-    case 9: return run_rows<9>(x, z, rows, scale, s);
-    case 10: return run_rows<10>(x, z, rows, scale, s);
-    case 11: return run_rows<11>(x, z, rows, scale, s);
-    case 12: return run_rows<12>(x, z, rows, scale, s);
+    case 7: return run_ring<7, Tin, Tout, kRingSlots>(x, z, rows, scale, s);
+    case 8: return run_ring<8, Tin, Tout, kRingSlots>(x, z, rows, scale, s);
+    case 9: return run_ring<9, Tin, Tout, kRingSlots>(x, z, rows, scale, s);
+    case 10: return run_ring<10, Tin, Tout, kRingSlots>(x, z, rows, scale, s);
+    case 11: return run_ring<11, Tin, Tout, kRingSlots>(x, z, rows, scale, s);
+    case 12: return run_ring<12, Tin, Tout, kRingSlots>(x, z, rows, scale, s);
     default: return run_large(x, z, rows, logn, scale, s);
   }
 }
