@@ -34,6 +34,12 @@ constexpr int kBudgetThreads = 1024;
 constexpr int kSelThreads = 256;
 constexpr int kMaxInitDin = 16384;
 
+// Position of entry k of a row's fp64 values in shared memory: one padding
+// double after every 16, so the butterfly passes (aligned groups of 8 at any
+// stride) and the coalesced sweeps meet distinct banks.
+__host__ __device__ __forceinline__ int vpos(int k) { return k + (k >> 4); }
+__host__ __device__ __forceinline__ size_t vbytes(int d_in) { return (size_t)vpos(d_in) * sizeof(double); }
+
 __device__ __forceinline__ int next_pow2(int v) {
   int m = 1;
   while (m < v) m <<= 1;
@@ -154,65 +160,177 @@ __global__ void __launch_bounds__(kNormThreads) row_norm_kernel(const float *__r
 }
 
 // Radix select over `n` keys produced by key(i) (eligible when ok(i)): the
-// `want`-th smallest key K and how many keys equal to K are to be taken.
-// Eight passes of 8 bits, most significant first. The histogram adds one
-// count per distinct digit per warp (the leading bytes of fp64 patterns are
-// shared by nearly all keys, so per-key atomics would serialise), and warp 0
-// finds the digit holding the `need`-th key with a shuffle scan over the 256
-// bins (8 per lane).
+// `want`-th smallest key K and how many keys equal to K are to be taken
+// (want minus the number of keys below K).
+//  * A first sweep finds the bits that all eligible keys share (AND and OR
+//    of the keys): the digits start right below them, so no pass is spent on
+//    the leading bytes that fp64 magnitudes of similar size have in common.
+//  * Pass 1 takes a kHistBins-wide (10-bit) digit, later passes 8 bits. The
+//    histogram adds one count per distinct digit per warp (__match_any_sync),
+//    and warp 0 finds the digit holding the need-th key by a shuffle scan.
+//  * Once the keys left are at most kCandCap, one sweep lists their indices
+//    and later passes read only the list; once they are at most 32, warp 0
+//    ranks them against each other and K follows directly.
+// hist holds kHistBins entries.
 constexpr int kCandCap = 1024;  // candidate list of the radix select (indices)
+constexpr int kHistBins = 1024;
 
-template <typename KeyF, typename OkF>
+// Warp 0 of a block: among the candidates cand[0..cand_n) whose keys match
+// `pm` under `hi_mask` (at most 32 of them), the need-th smallest key and how
+// many keys equal to it are to be taken; one lane stores them to *K and
+// *need_out and sets *done. The matching keys are staged in fk[0..32) (shared)
+// and every lane ranks its own against all of them.
+template <typename KeyF>
+__device__ __forceinline__ void warp_rank_finish(KeyF key, const int *cand, int cand_n, uint64_t hi_mask, uint64_t pm,
+                                                 int64_t need, unsigned long long *fk, unsigned long long *K,
+                                                 long long *need_out, int *done) {
+  const int lane = threadIdx.x & 31;
+  const unsigned below = (1u << lane) - 1u;
+  int have = 0;
+  for (int c0 = 0; c0 < cand_n; c0 += 32) {
+    const int c = c0 + lane;
+    uint64_t k = 0;
+    bool m = false;
+    if (c < cand_n) {
+      k = key(cand[c]);
+      m = (k & hi_mask) == pm;
+    }
+    const unsigned mm = __ballot_sync(0xffffffffu, m);
+    if (m && have + __popc(mm & below) < 32) fk[have + __popc(mm & below)] = k;
+    have += __popc(mm);
+  }
+  __syncwarp();
+  if (have > 32) have = 32;  // cannot happen: the caller checked the count
+  const uint64_t mine = lane < have ? fk[lane] : ~0ull;
+  int less = 0, eq = 0;
+  for (int src = 0; src < have; ++src) {
+    const uint64_t ks = fk[src];
+    less += ks < mine;
+    eq += ks == mine;
+  }
+  const bool hit = lane < have && less < need && need <= less + eq;
+  const unsigned who = __ballot_sync(0xffffffffu, hit);
+  if (who && lane == __ffs(who) - 1) {
+    *K = mine;
+    *need_out = need - less;
+    *done = 1;
+  }
+}
+
+template <bool AGG, typename KeyF, typename OkF>
 __device__ void radix_select_smallest(int n, int64_t want, KeyF key, OkF ok, uint32_t *hist, uint64_t *K_out,
                                       int64_t *need_out) {
   __shared__ int sel_digit;
   __shared__ int64_t sel_need;
-  // Once the keys that still match the prefix are at most kCandCap, the next
-  // pass also lists their indices, and the passes after it scan that list
-  // instead of all n keys (the digits found are the same).
   __shared__ int cand[kCandCap];
   __shared__ int cand_n;
   __shared__ uint32_t match_count;  // keys matching the prefix after the last pass
-  uint64_t prefix = 0;
-  int64_t need = want;
+  __shared__ unsigned long long s_and, s_or, s_K, fk[32];
+  __shared__ long long sel_need_ll;
+  __shared__ int s_cnt, s_done;
   const int lane = threadIdx.x & 31;
-  bool listing = false, listed = false;
   if (threadIdx.x == 0) {
     cand_n = 0;
-    match_count = 0xffffffffu;
+    s_and = ~0ull;
+    s_or = 0ull;
+    s_cnt = 0;
+    s_done = 0;
   }
   __syncthreads();
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    listing = !listed && match_count <= (uint32_t)kCandCap;
+  {
+    uint64_t ka = ~0ull, ko = 0ull;
+    int c = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+      if (ok(i)) {
+        const uint64_t k = key(i);
+        ka &= k;
+        ko |= k;
+        ++c;
+      }
+    const uint32_t alo = __reduce_and_sync(0xffffffffu, (uint32_t)ka);
+    const uint32_t ahi = __reduce_and_sync(0xffffffffu, (uint32_t)(ka >> 32));
+    const uint32_t olo = __reduce_or_sync(0xffffffffu, (uint32_t)ko);
+    const uint32_t ohi = __reduce_or_sync(0xffffffffu, (uint32_t)(ko >> 32));
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) {
+      atomicAnd(&s_and, ((unsigned long long)ahi << 32) | alo);
+      atomicOr(&s_or, ((unsigned long long)ohi << 32) | olo);
+      atomicAdd(&s_cnt, c);
+    }
+  }
+  __syncthreads();
+  const uint64_t kand = s_and, kor = s_or;
+  const int cnt = s_cnt;
+  if (want <= 0 || want > cnt || kand == kor) {
+    // nothing to take; everything; or all eligible keys equal: K needs no pass
+    *K_out = want <= 0 ? 0ull : (want > cnt ? ~0ull : kand);
+    *need_out = want;
+    return;
+  }
+  const int hb = 63 - __clzll((long long)(kand ^ kor));  // highest bit where eligible keys differ
+  uint64_t prefix = hb == 63 ? 0ull : (kand & ~((2ull << hb) - 1ull));
+  int64_t need = want;
+  int bits = hb + 1 < 10 ? hb + 1 : 10;
+  int shift = hb + 1 - bits;
+  bool listed = false;
+  if (threadIdx.x == 0) match_count = (uint32_t)cnt;
+  __syncthreads();
+  for (;;) {
+    const uint64_t hi_mask = shift + bits >= 64 ? 0ull : ~((1ull << (shift + bits)) - 1ull);
+    const int bins = 1 << bits;
+    if (!listed && match_count <= (uint32_t)kCandCap) {
+      // list the keys that match the prefix (no histogram in this sweep)
+      const int n_round = (n + blockDim.x - 1) / blockDim.x * blockDim.x;
+      for (int i = threadIdx.x; i < n_round; i += blockDim.x) {
+        bool m = false;
+        if (i < n && ok(i)) m = (key(i) & hi_mask) == (prefix & hi_mask);
+        const unsigned mm = __ballot_sync(0xffffffffu, m);
+        int base = 0;
+        if (lane == 0 && mm) base = atomicAdd(&cand_n, __popc(mm));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (m) cand[base + __popc(mm & ((1u << lane) - 1u))] = i;
+      }
+      listed = true;
+      __syncthreads();
+    }
+    if (listed && match_count <= 32u) {
+      // warp 0 ranks the (at most 32) keys that match the prefix
+      if (threadIdx.x < 32)
+        warp_rank_finish(key, cand, cand_n, hi_mask, prefix & hi_mask, need, fk, &s_K, &sel_need_ll, &s_done);
+      __syncthreads();
+      if (s_done) {
+        *K_out = s_K;
+        *need_out = sel_need_ll;
+        return;
+      }
+    }
+    for (int i = threadIdx.x; i < bins; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    const uint64_t hi_mask = shift == 56 ? 0 : (~0ull << (shift + 8));
     const int m = listed ? cand_n : n;
     const int m_round = (m + blockDim.x - 1) / blockDim.x * blockDim.x;  // whole warps iterate together
     for (int it = threadIdx.x; it < m_round; it += blockDim.x) {
-      int bin = 256;  // no count
+      int bin = kHistBins;  // no count
       if (it < m) {
         const int i = listed ? cand[it] : it;
         if (listed || ok(i)) {
           const uint64_t k = key(i);
-          if ((k & hi_mask) == (prefix & hi_mask)) {
-            bin = (int)((k >> shift) & 255);
-            if (listing) cand[atomicAdd(&cand_n, 1)] = i;
-          }
+          if ((k & hi_mask) == (prefix & hi_mask)) bin = (int)((k >> shift) & (uint64_t)(bins - 1));
         }
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      if (AGG) {  // one count per distinct digit per warp: for keys with many duplicates
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin < kHistBins && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      } else if (bin < kHistBins) {
+        atomicAdd(&hist[bin], 1u);
+      }
     }
     __syncthreads();
-    if (listing) listed = true;
     if (threadIdx.x < 32) {
-      uint32_t c[8];
+      const int per = (bins + 31) / 32;  // bins per lane
       uint32_t mine = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c[j] = hist[8 * lane + j];
-        mine += c[j];
+      for (int j = 0; j < per; ++j) {
+        const int bb = lane * per + j;
+        mine += bb < bins ? hist[bb] : 0u;
       }
       uint32_t incl = mine;  // inclusive scan over lanes
 #pragma unroll
@@ -221,67 +339,87 @@ __device__ void radix_select_smallest(int n, int64_t want, KeyF key, OkF ok, uin
         if (lane >= off) incl += o;
       }
       const int64_t excl = (int64_t)(incl - mine);
-      const bool hit = (excl < need && (int64_t)incl >= need) || (lane == 0 && need <= 0);
-      const unsigned who = __ballot_sync(0xffffffffu, hit);
+      const bool hit = excl < need && (int64_t)incl >= need;
       if (hit) {
         int64_t cum = excl;
-        int d = 8 * lane + 7;
-        uint32_t cnt = c[7];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (cum + c[j] >= need) {
-            d = 8 * lane + j;
-            cnt = c[j];
+        for (int j = 0; j < per; ++j) {
+          const int bb = lane * per + j;
+          const uint32_t c = bb < bins ? hist[bb] : 0u;
+          if (cum + c >= need) {
+            sel_digit = bb;
+            sel_need = need - cum;
+            match_count = c;
             break;
           }
-          cum += c[j];
+          cum += c;
         }
-        sel_digit = d;
-        sel_need = need - cum;
-        match_count = cnt;
-      } else if (who == 0 && lane == 31) {  // fewer eligible keys than wanted: past the last digit
-        sel_digit = 255;
-        sel_need = need - (int64_t)incl;
-        match_count = c[7];
       }
     }
     __syncthreads();
     prefix |= (uint64_t)sel_digit << shift;
     need = sel_need;
     __syncthreads();
+    if (shift == 0) break;
+    bits = shift < 8 ? shift : 8;
+    shift -= bits;
   }
   *K_out = prefix;
   *need_out = need;
 }
 
 // Mark, in increasing index order, every eligible key < K and the first `need`
-// keys == K; calls take(i) for each, in an order-preserving compaction whose
-// output slot is passed too.
+// keys == K; calls take(i, slot) for each, slot being its place in the
+// order-preserving compaction. Each warp takes a contiguous range of indices in
+// rounds of 32 consecutive ones (coalesced key reads): a first sweep counts the
+// keys < K and == K per warp, a scan over the warps places the ranges, and in
+// the second sweep ballots rank the marked keys inside a round. sh64 holds at
+// least 2 * (blockDim / 32) entries.
 template <typename KeyF, typename OkF, typename TakeF>
 __device__ void ordered_take(int n, uint64_t K, int64_t need, KeyF key, OkF ok, TakeF take, int64_t *sh64) {
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int a = threadIdx.x * per, b = min(n, a + per);
-  int64_t eq = 0;
-  for (int i = a; i < b; ++i)
-    if (ok(i) && key(i) == K) ++eq;
-  int64_t tot;
-  const int64_t eq_before = block_excl_scan(eq, sh64, &tot);
-  int64_t cnt = 0;
-  {
-    int64_t e_seen = eq_before;
-    for (int i = a; i < b; ++i) {
-      if (!ok(i)) continue;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int per = (((n + nw - 1) / nw) + 31) & ~31;
+  const int a = warp * per, b = min(n, a + per);
+  int lt = 0, eq = 0;
+  for (int i = a + lane; i < b; i += 32)
+    if (ok(i)) {
       const uint64_t k = key(i);
-      if (k < K || (k == K && e_seen++ < need)) ++cnt;
+      lt += k < K;
+      eq += k == K;
     }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    lt += __shfl_xor_sync(0xffffffffu, lt, off);
+    eq += __shfl_xor_sync(0xffffffffu, eq, off);
   }
-  const int64_t slot0 = block_excl_scan(cnt, sh64, &tot);
-  int64_t slot = slot0, e_seen = eq_before;
-  for (int i = a; i < b; ++i) {
-    if (!ok(i)) continue;
-    const uint64_t k = key(i);
-    if (k < K || (k == K && e_seen++ < need)) take(i, slot++);
+  int64_t *s_eq = sh64, *s_take = sh64 + nw;
+  if (lane == 0) s_eq[warp] = eq;
+  __syncthreads();
+  int64_t eq_before = 0;
+  for (int w = 0; w < warp; ++w) eq_before += s_eq[w];
+  int64_t eq_take = need - eq_before;
+  eq_take = eq_take < 0 ? 0 : (eq_take > eq ? eq : eq_take);
+  if (lane == 0) s_take[warp] = lt + eq_take;
+  __syncthreads();
+  int64_t slot = 0;
+  for (int w = 0; w < warp; ++w) slot += s_take[w];
+  int64_t e_seen = eq_before;
+  const unsigned below = (1u << lane) - 1u;
+  for (int i0 = a; i0 < b; i0 += 32) {  // warp-uniform rounds
+    const int i = i0 + lane;
+    bool is_lt = false, is_eq = false;
+    if (i < b && ok(i)) {
+      const uint64_t k = key(i);
+      is_lt = k < K;
+      is_eq = k == K;
+    }
+    const unsigned m_eq = __ballot_sync(0xffffffffu, is_eq);
+    const bool t = is_lt || (is_eq && e_seen + __popc(m_eq & below) < need);
+    const unsigned m_t = __ballot_sync(0xffffffffu, t);
+    if (t) take(i, slot + __popc(m_t & below));
+    slot += __popc(m_t);
+    e_seen += __popc(m_eq);
   }
+  __syncthreads();  // the caller reuses sh64
 }
 
 __global__ void __launch_bounds__(kBudgetThreads)
@@ -289,7 +427,7 @@ __global__ void __launch_bounds__(kBudgetThreads)
                   int32_t *__restrict__ budgets, int32_t *__restrict__ row_ptr, unsigned char *__restrict__ capped) {
   __shared__ double shd[kBudgetThreads];
   __shared__ int64_t sh64[kBudgetThreads];
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[kHistBins];
   __shared__ int any_new;
   const int t = threadIdx.x;
   for (int i = t; i < d_out; i += blockDim.x) capped[i] = 0;
@@ -351,7 +489,7 @@ __global__ void __launch_bounds__(kBudgetThreads)
     };
     uint64_t K;
     int64_t need;
-    radix_select_smallest(d_out, R, key, ok, hist, &K, &need);
+    radix_select_smallest<true>(d_out, R, key, ok, hist, &K, &need);
     __syncthreads();
     // mark first, then add: the keys must not change while being read
     ordered_take(d_out, K, need, key, ok, [&](int i, int64_t) { capped[i] = 2; }, sh64);
@@ -389,7 +527,7 @@ __device__ __forceinline__ void butterfly_pass_fp64(double *v, int d, int s) {
     const int base = ((g >> s) << (s + NB)) | lo;
     double x[GS];
 #pragma unroll
-    for (int i = 0; i < GS; ++i) x[i] = v[base + (i << s)];
+    for (int i = 0; i < GS; ++i) x[i] = v[vpos(base + (i << s))];
 #pragma unroll
     for (int b = 0; b < NB; ++b)
 #pragma unroll
@@ -400,16 +538,16 @@ __device__ __forceinline__ void butterfly_pass_fp64(double *v, int d, int s) {
           x[i + (1 << b)] = __dsub_rn(a, c);
         }
 #pragma unroll
-    for (int i = 0; i < GS; ++i) v[base + (i << s)] = x[i];
+    for (int i = 0; i < GS; ++i) v[vpos(base + (i << s))] = x[i];
   }
 }
 
 // v[0..d_in) = w[0..d_in) H_unnormalised per block of n, fp64 butterflies in
 // the textbook stage order (three stages per pass over aligned groups of 8,
 // the last pass one or two when log2 n is not a multiple of 3); v is shared
-// memory, every thread of the block takes part.
+// memory at the padded positions vpos(k), every thread of the block takes part.
 __device__ void row_transform_fp64(const float *__restrict__ w, int d_in, int n, double *v) {
-  for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[k] = (double)w[k];
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[vpos(k)] = (double)w[k];
   __syncthreads();
   const int logn = 31 - __clz(n);
   for (int s = 0; s < logn; s += 3) {
@@ -426,7 +564,7 @@ __global__ void __launch_bounds__(kSelThreads)
                   const int32_t *__restrict__ row_ptr, int64_t p, int32_t *__restrict__ col_idx,
                   float *__restrict__ coef) {
   extern __shared__ __align__(16) double v[];  // d_in values of the row
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[kHistBins];
   __shared__ int64_t sh64[kSelThreads];
   const int64_t row = blockIdx.x;
   row_transform_fp64(dW + row * d_in, d_in, n, v);
@@ -435,20 +573,292 @@ __global__ void __launch_bounds__(kSelThreads)
   if (b <= 0 || start < 0 || start + b > p) return;
   const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)n));
   // largest |V| = smallest complemented magnitude bits
-  auto key = [&](int k) -> uint64_t { return ~((uint64_t)__double_as_longlong(v[k]) & 0x7fffffffffffffffull); };
+  auto key = [&](int k) -> uint64_t { return ~((uint64_t)__double_as_longlong(v[vpos(k)]) & 0x7fffffffffffffffull); };
   auto ok = [&](int) { return true; };
   uint64_t K;
   int64_t need;
-  radix_select_smallest(d_in, b, key, ok, hist, &K, &need);
+  radix_select_smallest<false>(d_in, b, key, ok, hist, &K, &need);
   __syncthreads();
   ordered_take(d_in, K, need, key, ok,
                [&](int k, int64_t slot) {
                  if (slot < b) {
                    col_idx[start + slot] = k;
-                   coef[start + slot] = __double2float_rn(__dmul_rn(v[k], inv));
+                   coef[start + slot] = __double2float_rn(__dmul_rn(v[vpos(k)], inv));
                  }
                },
                sh64);
+}
+
+// Rows of exactly 4096 entries (every workload shape but down_proj): the same
+// selection with the row in registers. 256 threads x 16 values; the 12
+// butterfly stages run in three register phases of 4 stages (textbook order,
+// so the fp64 results are those of row_transform_fp64 bit for bit):
+//   phase 1: thread t holds entries 16t + j       (stages h = 1 .. 8)
+//   phase 2: entries (t % 16) + 16 j + 256 (t / 16) (h = 16 .. 128)
+//   phase 3: entries t + 256 j                      (h = 256 .. 2048)
+// with two exchanges through the padded shared buffer (conflict-free for all
+// four access patterns). Stages at or above the Hadamard block are skipped.
+// The values then stay in registers (and, for the candidate lists, in the
+// buffer): the common-prefix sweep, one 10-bit histogram pass, a listing sweep
+// and the warp-level finish of radix_select_smallest, then the ordered
+// compaction in index order (index 256 j + t: rounds j, warps in order inside
+// a round).
+constexpr int kRow4k = 4096;
+
+__device__ __forceinline__ void bfly16(double *x, int b0, int logn) {
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    if (b0 + b >= logn) break;
+    const int h = 1 << b;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (!(j & h)) {
+        const double a = x[j], c = x[j + h];
+        x[j] = __dadd_rn(a, c);
+        x[j + h] = __dsub_rn(a, c);
+      }
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads, 3)
+    select4k_kernel(const float *__restrict__ dW, int n, const int32_t *__restrict__ budgets,
+                    const int32_t *__restrict__ row_ptr, int64_t p, int32_t *__restrict__ col_idx,
+                    float *__restrict__ coef) {
+  extern __shared__ __align__(16) double v[];  // vpos(4096) doubles
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ int cand[kCandCap];
+  __shared__ int cand_n;
+  __shared__ unsigned long long s_and, s_or, s_K, fk[32];
+  __shared__ int s_digit, s_done;
+  __shared__ long long s_need;
+  __shared__ uint32_t s_match;
+  __shared__ int s_cnt[2][16][8];  // per (round j, warp): keys < K, keys == K
+  __shared__ int s_base[16][8];    // output slot of each (round, warp)
+  __shared__ int s_eqb[16][8];     // keys == K before each (round, warp)
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int64_t row = blockIdx.x;
+  const int logn = 31 - __clz(n);
+  const int b = budgets[row];
+  const int64_t start = (int64_t)row_ptr[row] - row_ptr[0];  // row_ptr may be a slice of a longer one
+  if (b <= 0 || start < 0 || start + b > p) return;
+
+  double x[16];
+  {
+    const float4 *src = reinterpret_cast<const float4 *>(dW + row * kRow4k + 16 * t);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = src[q];
+      x[4 * q] = (double)f.x, x[4 * q + 1] = (double)f.y, x[4 * q + 2] = (double)f.z, x[4 * q + 3] = (double)f.w;
+    }
+  }
+  bfly16(x, 0, logn);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[vpos(16 * t + j)] = x[j];
+  __syncthreads();
+  const int e2 = (t & 15) + 256 * (t >> 4);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) x[j] = v[vpos(e2 + 16 * j)];
+  bfly16(x, 4, logn);
+  // each thread rewrites only the positions it has just read: no barrier
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[vpos(e2 + 16 * j)] = x[j];
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) x[j] = v[vpos(t + 256 * j)];
+  bfly16(x, 8, logn);
+  // the final values back in place (own positions again), for the candidate lists
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[vpos(t + 256 * j)] = x[j];
+
+  // keys: largest |V| = smallest complemented magnitude bits
+  auto kx = [](double d) -> uint64_t { return ~((uint64_t)__double_as_longlong(d) & 0x7fffffffffffffffull); };
+  if (t == 0) {
+    s_and = ~0ull;
+    s_or = 0ull;
+    cand_n = 0;
+    s_done = 0;
+  }
+  __syncthreads();
+  {
+    uint64_t ka = ~0ull, ko = 0ull;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      ka &= kx(x[j]);
+      ko |= kx(x[j]);
+    }
+    const uint32_t alo = __reduce_and_sync(0xffffffffu, (uint32_t)ka);
+    const uint32_t ahi = __reduce_and_sync(0xffffffffu, (uint32_t)(ka >> 32));
+    const uint32_t olo = __reduce_or_sync(0xffffffffu, (uint32_t)ko);
+    const uint32_t ohi = __reduce_or_sync(0xffffffffu, (uint32_t)(ko >> 32));
+    if (lane == 0) {
+      atomicAnd(&s_and, ((unsigned long long)ahi << 32) | alo);
+      atomicOr(&s_or, ((unsigned long long)ohi << 32) | olo);
+    }
+  }
+  __syncthreads();
+  const uint64_t kand = s_and, kor = s_or;
+  uint64_t K;
+  int64_t need = b;
+  if (b >= kRow4k || kand == kor) {
+    K = b >= kRow4k ? ~0ull : kand;  // everything, or all keys equal
+  } else {
+    const int hb = 63 - __clzll((long long)(kand ^ kor));
+    uint64_t prefix = hb == 63 ? 0ull : (kand & ~((2ull << hb) - 1ull));
+    int bits = hb + 1 < 10 ? hb + 1 : 10;
+    int shift = hb + 1 - bits;
+    uint32_t match = kRow4k;
+    bool listed = false;
+    for (;;) {
+      const uint64_t hi_mask = shift + bits >= 64 ? 0ull : ~((1ull << (shift + bits)) - 1ull);
+      const uint64_t pm = prefix & hi_mask;
+      const int bins = 1 << bits;
+      if (!listed && match <= (uint32_t)kCandCap) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const bool m = (kx(x[j]) & hi_mask) == pm;
+          const unsigned mm = __ballot_sync(0xffffffffu, m);
+          int base = 0;
+          if (lane == 0 && mm) base = atomicAdd(&cand_n, __popc(mm));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (m) cand[base + __popc(mm & ((1u << lane) - 1u))] = t + 256 * j;
+        }
+        listed = true;
+        __syncthreads();
+      }
+      if (listed && match <= 32u) {
+        if (warp == 0)
+          warp_rank_finish([&](int e) { return kx(v[vpos(e)]); }, cand, cand_n, hi_mask, pm, need, fk, &s_K, &s_need,
+                           &s_done);
+        __syncthreads();
+        if (s_done) {
+          prefix = s_K;
+          need = s_need;
+          break;
+        }
+      }
+      for (int i = t; i < bins; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      if (listed) {
+        const int m_round = (cand_n + kSelThreads - 1) / kSelThreads * kSelThreads;
+        for (int it = t; it < m_round; it += kSelThreads) {
+          int bin = kHistBins;
+          if (it < cand_n) {
+            const uint64_t kc = kx(v[vpos(cand[it])]);
+            if ((kc & hi_mask) == pm) bin = (int)((kc >> shift) & (uint64_t)(bins - 1));
+          }
+          if (bin < kHistBins) atomicAdd(&hist[bin], 1u);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const uint64_t kj = kx(x[j]);
+          const int bin = (kj & hi_mask) == pm ? (int)((kj >> shift) & (uint64_t)(bins - 1)) : kHistBins;
+          if (bin < kHistBins) atomicAdd(&hist[bin], 1u);
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int per = (bins + 31) / 32;
+        uint32_t mine = 0;
+        for (int j = 0; j < per; ++j) {
+          const int bb = lane * per + j;
+          mine += bb < bins ? hist[bb] : 0u;
+        }
+        uint32_t incl = mine;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        const int64_t excl = (int64_t)(incl - mine);
+        if (excl < need && (int64_t)incl >= need) {
+          int64_t cum = excl;
+          for (int j = 0; j < per; ++j) {
+            const int bb = lane * per + j;
+            const uint32_t c = bb < bins ? hist[bb] : 0u;
+            if (cum + c >= need) {
+              s_digit = bb;
+              s_need = need - cum;
+              s_match = c;
+              break;
+            }
+            cum += c;
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= (uint64_t)s_digit << shift;
+      need = s_need;
+      match = s_match;
+      __syncthreads();
+      if (shift == 0) break;
+      bits = shift < 8 ? shift : 8;
+      shift -= bits;
+    }
+    K = prefix;
+  }
+
+  // ordered compaction: index 256 j + t, rounds j, warps in order inside a round
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const unsigned m_lt = __ballot_sync(0xffffffffu, kx(x[j]) < K);
+    const unsigned m_eq = __ballot_sync(0xffffffffu, kx(x[j]) == K);
+    if (lane == 0) {
+      s_cnt[0][j][warp] = __popc(m_lt);
+      s_cnt[1][j][warp] = __popc(m_eq);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // 128 chunks in index order (chunk c = 8 j + w), four per lane
+    int lt4[4], eq4[4];
+    int lt_s = 0, eq_s = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = 4 * lane + q;
+      lt4[q] = s_cnt[0][c >> 3][c & 7];
+      eq4[q] = s_cnt[1][c >> 3][c & 7];
+      lt_s += lt4[q];
+      eq_s += eq4[q];
+    }
+    int lt_x = lt_s, eq_x = eq_s;  // inclusive scans over lanes
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, lt_x, off), e = __shfl_up_sync(0xffffffffu, eq_x, off);
+      if (lane >= off) {
+        lt_x += a;
+        eq_x += e;
+      }
+    }
+    int lt_before = lt_x - lt_s, eq_before = eq_x - eq_s;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = 4 * lane + q;
+      // keys < K before the chunk, plus the keys == K taken before it
+      s_base[c >> 3][c & 7] = lt_before + (int)(need < eq_before ? need : eq_before);
+      s_eqb[c >> 3][c & 7] = eq_before;
+      lt_before += lt4[q];
+      eq_before += eq4[q];
+    }
+  }
+  __syncthreads();
+  const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)n));
+  const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint64_t kj = kx(x[j]);
+    const bool is_lt = kj < K, is_eq = kj == K;
+    const unsigned m_eq = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = is_lt || (is_eq && s_eqb[j][warp] + __popc(m_eq & below) < need);
+    const unsigned m_t = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int slot = s_base[j][warp] + __popc(m_t & below);
+      if (slot < b) {
+        col_idx[start + slot] = t + 256 * j;
+        coef[start + slot] = __double2float_rn(__dmul_rn(x[j], inv));
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------ selection over the whole matrix
@@ -485,7 +895,7 @@ __global__ void __launch_bounds__(kSelThreads)
   extern __shared__ __align__(16) double v[];
   const int64_t row = blockIdx.x;
   row_transform_fp64(dW + row * d_in, d_in, n, v);
-  for (int k = threadIdx.x; k < d_in; k += blockDim.x) V[row * d_in + k] = v[k];
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) V[row * d_in + k] = v[vpos(k)];
 }
 
 __global__ void gsel_init_kernel(GselState *st, int64_t p) {
@@ -620,7 +1030,7 @@ __global__ void __launch_bounds__(kSelThreads)
   extern __shared__ __align__(16) double v[];
   __shared__ int64_t sh64[kSelThreads];
   const int64_t row = blockIdx.x;
-  for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[k] = V[row * d_in + k];
+  for (int k = threadIdx.x; k < d_in; k += blockDim.x) v[vpos(k)] = V[row * d_in + k];
   __syncthreads();
   const int64_t start = row_ptr[row];
   const int64_t cnt = (int64_t)row_ptr[row + 1] - start;
@@ -628,7 +1038,7 @@ __global__ void __launch_bounds__(kSelThreads)
   const uint64_t K = st->prefix;
   const double inv = __ddiv_rn(1.0, __dsqrt_rn((double)n));
   auto key = [&](int k) -> uint64_t {
-    if (sel == 0) return ~((uint64_t)__double_as_longlong(v[k]) & 0x7fffffffffffffffull);
+    if (sel == 0) return ~((uint64_t)__double_as_longlong(v[vpos(k)]) & 0x7fffffffffffffffull);
     return splitmix64_at(seed, (uint64_t)(row * d_in + k) + 1);
   };
   auto ok = [&](int) { return true; };
@@ -636,7 +1046,7 @@ __global__ void __launch_bounds__(kSelThreads)
                [&](int k, int64_t slot) {
                  if (slot < cnt) {
                    col_idx[start + slot] = k;
-                   coef[start + slot] = __double2float_rn(__dmul_rn(v[k], inv));
+                   coef[start + slot] = __double2float_rn(__dmul_rn(v[vpos(k)], inv));
                  }
                },
                sh64);
@@ -651,6 +1061,24 @@ size_t init_workspace(int32_t d_out, int32_t d_in) {
 
 int init_max_din() { return kMaxInitDin; }
 
+// The per-row selection: rows of 4096 entries in registers, others through
+// the generic shared-memory kernel.
+cudaError_t launch_select_rows(const float *dW, int32_t rows, int32_t d_in, int32_t had_block, const int32_t *budgets,
+                               const int32_t *row_ptr, int64_t p, int32_t *col_idx, float *coef, cudaStream_t s) {
+  const size_t smem = vbytes(d_in);
+  if (d_in == kRow4k && aligned16(dW)) {
+    auto k = select4k_kernel;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    k<<<rows, kSelThreads, smem, s>>>(dW, had_block, budgets, row_ptr, p, col_idx, coef);
+    return cudaGetLastError();
+  }
+  cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  select_kernel<<<rows, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p,
                               int32_t min_per_row, int mode, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx,
                               float *coef, void *ws, cudaStream_t s) {
@@ -658,10 +1086,7 @@ cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int3
   unsigned char *capped = static_cast<unsigned char *>(ws) + align_up((size_t)d_out * 8, 256);
   row_norm_kernel<<<d_out, kNormThreads, 0, s>>>(dW, d_in, e);
   budget_kernel<<<1, kBudgetThreads, 0, s>>>(e, d_out, d_in, p, min_per_row, mode, budgets, row_ptr, capped);
-  const size_t smem = (size_t)d_in * sizeof(double);
-  cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  if (p > 0) select_kernel<<<d_out, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
+  if (p > 0) return launch_select_rows(dW, d_out, d_in, had_block, budgets, row_ptr, p, col_idx, coef, s);
   return cudaGetLastError();
 }
 
@@ -682,7 +1107,7 @@ cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, i
   int32_t *eq = reinterpret_cast<int32_t *>(w);
   w += align_up((size_t)d_out * 4, 256);
   int32_t *take = reinterpret_cast<int32_t *>(w);
-  const size_t smem = (size_t)d_in * sizeof(double);
+  const size_t smem = vbytes(d_in);
   cudaError_t e = cudaFuncSetAttribute(gsel_transform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gsel_take_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -719,11 +1144,7 @@ cudaError_t launch_init_budgets(const double *e, int32_t d_out, int32_t d_in, in
 cudaError_t launch_init_select(const float *dW, int32_t rows, int32_t d_in, int32_t had_block, const int32_t *budgets,
                                const int32_t *row_ptr, int64_t p, int32_t *col_idx, float *coef, cudaStream_t s) {
   if (rows <= 0 || p <= 0) return cudaSuccess;
-  const size_t smem = (size_t)d_in * sizeof(double);
-  cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  select_kernel<<<rows, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
-  return cudaGetLastError();
+  return launch_select_rows(dW, rows, d_in, had_block, budgets, row_ptr, p, col_idx, coef, s);
 }
 
 }  // namespace qwha
