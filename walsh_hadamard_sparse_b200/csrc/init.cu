@@ -68,52 +68,85 @@ __device__ double run_pairwise(int L, F value) {
   return st[0];
 }
 
-// Canonical tree over the per-thread sums held in sh[0..blockDim) (a power of two).
+// Canonical tree over the per-thread values `mine` (blockDim a power of two,
+// at most 1024): levels inside a warp by shuffles (the left operand is always
+// the lower-index subtree), then the warps' sums through sh[0..32) by warp 0.
 __device__ double block_pairwise(double mine, double *sh) {
-  const int t = threadIdx.x;
-  sh[t] = mine;
-  __syncthreads();
-  for (int w = blockDim.x; w > 1; w >>= 1) {
-    double v = 0;
-    if (t < w / 2) v = __dadd_rn(sh[2 * t], sh[2 * t + 1]);
-    __syncthreads();
-    if (t < w / 2) sh[t] = v;
-    __syncthreads();
+  const int t = threadIdx.x, lane = t & 31;
+  const int width = blockDim.x < 32 ? (int)blockDim.x : 32;
+  for (int h = 1; h < width; h <<= 1) {
+    const double o = __shfl_down_sync(0xffffffffu, mine, h);
+    if ((lane & (2 * h - 1)) == 0) mine = __dadd_rn(mine, o);
   }
-  const double r = sh[0];
+  const int nw = (int)blockDim.x / 32;
+  if (nw > 1) {
+    if (lane == 0) sh[t >> 5] = mine;
+    __syncthreads();
+    if (t < 32) {
+      double x = t < nw ? sh[t] : 0.0;
+      for (int h = 1; h < nw; h <<= 1) {
+        const double o = __shfl_down_sync(0xffffffffu, x, h);
+        if ((lane & (2 * h - 1)) == 0) x = __dadd_rn(x, o);
+      }
+      if (t == 0) sh[32] = x;
+    }
+  } else if (t == 0) {
+    sh[32] = mine;
+  }
+  __syncthreads();
+  const double r = sh[32];
   __syncthreads();
   return r;
 }
 
+// Sum over the block (integers: any order); sh holds 33 entries.
 template <typename T>
 __device__ T block_sum(T v, T *sh) {
-  const int t = threadIdx.x;
-  sh[t] = v;
+  const int t = threadIdx.x, lane = t & 31;
+#pragma unroll
+  for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  if (lane == 0) sh[t >> 5] = v;
   __syncthreads();
-  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-    if (t < w) sh[t] += sh[t + w];
-    __syncthreads();
+  if (t < 32) {
+    T x = t < (int)(blockDim.x >> 5) ? sh[t] : T(0);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if (t == 0) sh[32] = x;
   }
-  const T r = sh[0];
+  __syncthreads();
+  const T r = sh[32];
   __syncthreads();
   return r;
 }
 
-// Exclusive prefix over threads of v (blockDim a power of two); returns the total in *tot.
+// Exclusive prefix over threads of v (blockDim a multiple of 32); returns the
+// total in *tot. Warp scans by shuffles, the warps' totals scanned by warp 0.
 __device__ int64_t block_excl_scan(int64_t v, int64_t *sh, int64_t *tot) {
-  const int t = threadIdx.x;
-  sh[t] = v;
-  __syncthreads();
-  for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-    const int64_t a = t >= off ? sh[t - off] : 0;
-    __syncthreads();
-    sh[t] += a;
-    __syncthreads();
+  const int t = threadIdx.x, lane = t & 31, nw = (int)blockDim.x >> 5;
+  int64_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int64_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
   }
-  const int64_t incl = sh[t];
-  *tot = sh[blockDim.x - 1];
+  if (lane == 31) sh[t >> 5] = incl;
   __syncthreads();
-  return incl - v;
+  if (t < 32) {
+    const int64_t w = t < nw ? sh[t] : 0;
+    int64_t x = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int64_t o = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += o;
+    }
+    sh[32 + t] = x - w;  // exclusive over warps
+    if (t == 31) sh[64] = x;
+  }
+  __syncthreads();
+  const int64_t r = sh[32 + (t >> 5)] + incl - v;
+  *tot = sh[64];
+  __syncthreads();
+  return r;
 }
 
 // Pairwise sum of the squares of w[base .. base + L) (zero past d_in), the
@@ -121,11 +154,22 @@ __device__ int64_t block_excl_scan(int64_t v, int64_t *sh, int64_t *tot) {
 template <int L>
 __device__ __forceinline__ double tree_sq(const float *__restrict__ w, int base, int d_in) {
   double x[L];
+  if (L % 4 == 0 && base + L <= d_in && (reinterpret_cast<uintptr_t>(w + base) & 15u) == 0) {
 #pragma unroll
-  for (int i = 0; i < L; ++i) {
-    const int k = base + i;
-    const double v = k < d_in ? (double)w[k] : 0.0;
-    x[i] = __dmul_rn(v, v);
+    for (int i = 0; i < L; i += 4) {  // 16-byte loads where the run is inside the row and aligned
+      const float4 f = *reinterpret_cast<const float4 *>(w + base + i);
+      x[i] = __dmul_rn((double)f.x, (double)f.x);
+      x[i + 1] = __dmul_rn((double)f.y, (double)f.y);
+      x[i + 2] = __dmul_rn((double)f.z, (double)f.z);
+      x[i + 3] = __dmul_rn((double)f.w, (double)f.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < L; ++i) {
+      const int k = base + i;
+      const double v = k < d_in ? (double)w[k] : 0.0;
+      x[i] = __dmul_rn(v, v);
+    }
   }
 #pragma unroll
   for (int h = 1; h < L; h <<= 1)
