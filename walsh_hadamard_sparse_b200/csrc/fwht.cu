@@ -19,8 +19,8 @@
 //            bit) and does the remaining butterflies; it writes the scaled
 //            results, in the output type, into per-segment staging that bulk
 //            copies send to global memory.
-// The transpose buffer is XOR-swizzled (RingGeo::phys) so that both phases'
-// accesses are free of bank conflicts. Arithmetic is fp32 whatever the I/O
+// The transpose buffer is padded (Geo::phys, fwht_body.cuh) so that both
+// phases' accesses are free of bank conflicts. Arithmetic is fp32 whatever the I/O
 // type. fwht_body.cuh holds the same arithmetic for the fused forward GEMM and
 // the W_eff kernels below.
 
@@ -47,21 +47,6 @@ struct RingGeo {
   using G = Geo<LOGN, V>;
   static constexpr int RW = G::P < 64 ? 64 : G::P;  // threads of the worker
   static constexpr int RPW = RW / G::P;             // rows per iteration
-  // Exchange-buffer position of element e of local row rl, XOR-swizzled
-  // instead of padded. The low field splits into i (the 4 floats of a 16-byte
-  // access) and u (which 16-byte half of a narrow vector); u moves above the
-  // middle field m, and m's low 3 bits are flipped by s(u, high, rl). Phase-A
-  // 16-byte accesses (fixed h, u; lanes = consecutive m) then cover 128
-  // contiguous bytes per quarter warp, and phase-B scalar accesses (fixed m;
-  // lanes = i, u, high bits, rows) meet 32 distinct banks. Rows are N floats
-  // apart (no padding).
-  __device__ __forceinline__ static int swz(int u, int hh, int rl) {
-    return ((u | (hh << (G::LV - 2))) ^ (rl << (G::PB - 2))) & 7;
-  }
-  __device__ __forceinline__ static int phys(int e, int rl) {
-    const int i = e & 3, u = (e & (V - 1)) >> 2, m = (e >> G::LV) & (G::P - 1), hh = e >> (G::LV + G::PB);
-    return rl * G::N + (i | ((m ^ swz(u, hh, rl)) << 2) | (u << (2 + G::PB)) | (hh << (G::LV + G::PB)));
-  }
   // output staging: a segment per (row, high field) value holds the SEGE
   // contiguous output elements of that value, segp() elements apart: one
   // vector (V elements) of padding moves each segment by as many banks as a
@@ -70,23 +55,12 @@ struct RingGeo {
   static constexpr int SEGE = 1 << (G::LV + G::PB);
   template <typename T>
   __host__ __device__ static constexpr int segp() { return SEGE + V; }
-  // the exchange buffer (RPW rows of N floats) and the output staging, which
+  // the exchange buffer (RPW rows of Geo::NP floats) and the output staging, which
   // reuses it: the larger of the two, rounded to 128 bytes
   template <typename T>
   __host__ __device__ static constexpr int buf_bytes() {
-    const int a = RPW * G::N * 4, b = RPW * (1 << G::HB) * segp<T>() * (int)sizeof(T);
+    const int a = RPW * G::NP * 4, b = RPW * (1 << G::HB) * segp<T>() * (int)sizeof(T);
     return ((a > b ? a : b) + 127) & ~127;
-  }
-  // phase A, half u of the vector of high index h: the swizzle's compile-time
-  // part and the offset beyond the thread's base pointer
-  __host__ __device__ static constexpr int sA(int u, int h) { return (u | (h << (G::LV - 2))) & 7; }
-  __host__ __device__ static constexpr int offA(int u, int h) { return (u << (2 + G::PB)) | (h << (G::LV + G::PB)); }
-  // phase B, register q: middle field q % P, batch bit q / P (the top high bit)
-  __host__ __device__ static constexpr int sB(int q) {
-    return ((q & 7) ^ (((q >> G::PB) << (G::HB - G::NB + G::LV - 2)) & 7)) & 7;
-  }
-  __host__ __device__ static constexpr int offB(int q) {
-    return (((q & (G::P - 1)) & ~7) << 2) | ((q >> G::PB) << (G::LV + G::PB + G::HB - G::NB));
   }
 };
 
@@ -99,7 +73,6 @@ __global__ void __launch_bounds__(RingGeo<LOGN, V>::RW) fwht_ring_kernel(const T
   constexpr int RPW = RG::RPW;
   constexpr int SLOT = RPW * G::N * (int)sizeof(Tin);  // bytes, a multiple of 16
   constexpr int BUF = RG::template buf_bytes<Tout>();
-  static_assert(G::PB >= 3, "the swizzle needs 3 middle bits");
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
   float *buf = reinterpret_cast<float *>(smem_raw);
@@ -110,21 +83,7 @@ __global__ void __launch_bounds__(RingGeo<LOGN, V>::RW) fwht_ring_kernel(const T
   const int64_t stride = (int64_t)gridDim.x * RPW;
   const int64_t first = (int64_t)blockIdx.x * RPW;
   const int64_t iters = first < rows ? (rows - first + stride - 1) / stride : 0;
-  // RG::phys unrolled: eight base pointers per phase (one per value of the
-  // swizzled low middle bits); everything else is a compile-time offset
-  const int rsw = (rl << (G::PB - 2)) & 7;
-  float *pa[8], *pb[8];
-  {
-    float *rb = buf + rl * G::N;
-    const int l = t & (V - 1), hB = t >> G::LV;
-    const int s0 = ((l >> 2) | (hB << (G::LV - 2))) ^ rsw;
-    float *bb = rb + (l & 3) + ((l >> 2) << (2 + G::PB)) + (hB << (G::LV + G::PB));
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      pa[j] = rb + ((((t ^ j ^ rsw) & 7) | (t & ~7)) << 2);
-      pb[j] = bb + (((j ^ s0) & 7) << 2);
-    }
-  }
+  float *rb = buf + rl * G::NP;  // this row's part of the transpose buffer
 
   auto issue = [&](int64_t it) {  // thread 0: copy iteration it's rows into its slot
     const int64_t r0 = first + it * stride;
@@ -179,13 +138,13 @@ __global__ void __launch_bounds__(RingGeo<LOGN, V>::RW) fwht_ring_kernel(const T
     for (int h = 0; h < (1 << G::HB); ++h) {
 #pragma unroll
       for (int u = 0; u < V; u += 4)
-        *reinterpret_cast<float4 *>(pa[RG::sA(u >> 2, h)] + RG::offA(u >> 2, h)) =
+        *reinterpret_cast<float4 *>(rb + G::phys(G::eA(t, h << G::LV) + u)) =
             make_float4(v[h * V + u], v[h * V + u + 1], v[h * V + u + 2], v[h * V + u + 3]);
     }
     __syncthreads();  // phase A is in buf and slot s is consumed: refill it
     if (tid == 0 && it + S < iters) issue(it + S);
 #pragma unroll
-    for (int q = 0; q < G::R; ++q) v[q] = pb[RG::sB(q)][RG::offB(q)];
+    for (int q = 0; q < G::R; ++q) v[q] = rb[G::phys(G::eB(t, q))];
     butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
     __syncthreads();  // all phase-B reads done before the buffer is reused
     // results straight from phase B into the buffer in the output type, one
@@ -249,7 +208,7 @@ __global__ void __launch_bounds__(512) fwht_large_kernel(const Tin *__restrict__
 }
 
 // W_eff block rows: for block b of row r (n = 2^LOGN columns starting at
-// blk * n), scatter that row's coefficients into the swizzled buffer, run the
+// blk * n), scatter that row's coefficients into the padded buffer, run the
 // two butterfly phases, then in phase-A layout (8 consecutive columns per
 // vector) add the dequantized base weight in fp32 and store one bf16 rounding:
 //   out[r, k] = bf16( W_Q[r, k] + scale * (sum_j c_j H_unnorm[k_j, k]) ).
@@ -291,10 +250,9 @@ __global__ void __launch_bounds__(kThreads)
     float v[G::R];
 #pragma unroll
     for (int h = 0; h < (1 << G::HB); ++h) {
-      const float *src = buf + G::phys(G::eA(t, h << G::LV));
 #pragma unroll
       for (int u = 0; u < 8; u += 4) {
-        const float4 f = *reinterpret_cast<const float4 *>(src + u);
+        const float4 f = *reinterpret_cast<const float4 *>(buf + G::phys(G::eA(t, h << G::LV) + u));
         v[h * 8 + u] = f.x, v[h * 8 + u + 1] = f.y, v[h * 8 + u + 2] = f.z, v[h * 8 + u + 3] = f.w;
       }
     }
@@ -302,10 +260,9 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < (1 << G::HB); ++h) {
-      float *dst = buf + G::phys(G::eA(t, h << G::LV));
 #pragma unroll
       for (int u = 0; u < 8; u += 4)
-        *reinterpret_cast<float4 *>(dst + u) = make_float4(v[h * 8 + u], v[h * 8 + u + 1], v[h * 8 + u + 2], v[h * 8 + u + 3]);
+        *reinterpret_cast<float4 *>(buf + G::phys(G::eA(t, h << G::LV) + u)) = make_float4(v[h * 8 + u], v[h * 8 + u + 1], v[h * 8 + u + 2], v[h * 8 + u + 3]);
     }
     __syncthreads();
 #pragma unroll
@@ -319,11 +276,10 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
       for (int h = 0; h < (1 << G::HB); ++h) {
         const int e = G::eA(t, h << G::LV);
-        const float *src = buf + G::phys(e);
         float f[8];
 #pragma unroll
         for (int u = 0; u < 8; u += 4) {
-          const float4 a = *reinterpret_cast<const float4 *>(src + u);
+          const float4 a = *reinterpret_cast<const float4 *>(buf + G::phys(e + u));
           f[u] = a.x, f[u + 1] = a.y, f[u + 2] = a.z, f[u + 3] = a.w;
         }
         const int k = k0 + e;
@@ -455,10 +411,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     float v[G::R];
 #pragma unroll
     for (int h = 0; h < (1 << G::HB); ++h) {
-      const float *src = buf + G::phys(G::eA(t, h << G::LV));
 #pragma unroll
       for (int u = 0; u < 8; u += 4) {
-        const float4 f = *reinterpret_cast<const float4 *>(src + u);
+        const float4 f = *reinterpret_cast<const float4 *>(buf + G::phys(G::eA(t, h << G::LV) + u));
         v[h * 8 + u] = f.x, v[h * 8 + u + 1] = f.y, v[h * 8 + u + 2] = f.z, v[h * 8 + u + 3] = f.w;
       }
     }
@@ -466,10 +421,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
 #pragma unroll
     for (int h = 0; h < (1 << G::HB); ++h) {
-      float *dst = buf + G::phys(G::eA(t, h << G::LV));
 #pragma unroll
       for (int u = 0; u < 8; u += 4)
-        *reinterpret_cast<float4 *>(dst + u) = make_float4(v[h * 8 + u], v[h * 8 + u + 1], v[h * 8 + u + 2], v[h * 8 + u + 3]);
+        *reinterpret_cast<float4 *>(buf + G::phys(G::eA(t, h << G::LV) + u)) = make_float4(v[h * 8 + u], v[h * 8 + u + 1], v[h * 8 + u + 2], v[h * 8 + u + 3]);
     }
     __syncthreads();
 #pragma unroll
@@ -486,11 +440,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int h = 0; h < (1 << G::HB); ++h) {
         const int el = G::eA(t, h << G::LV);
-        const float *src = buf + G::phys(el);
         float f[8];
 #pragma unroll
         for (int u = 0; u < 8; u += 4) {
-          const float4 a = *reinterpret_cast<const float4 *>(src + u);
+          const float4 a = *reinterpret_cast<const float4 *>(buf + G::phys(el + u));
           f[u] = a.x, f[u + 1] = a.y, f[u + 2] = a.z, f[u + 3] = a.w;
         }
         if (qw) {

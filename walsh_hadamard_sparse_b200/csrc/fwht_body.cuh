@@ -1,7 +1,7 @@
 // Register/shared-memory row Walsh-Hadamard transform shared by the
 // standalone transform kernels (fwht.cu) and the forward GEMM, whose extra
 // warps transform X while the tensor cores run (gemm.cu). See fwht.cu for the
-// layout (phase A / phase B index maps, swizzled transpose buffer).
+// layout (phase A / phase B index maps, padded transpose buffer).
 #pragma once
 
 #include "common.cuh"
@@ -18,10 +18,13 @@ struct Geo {
   static constexpr int P = 1 << PB;
   static constexpr int NB = 2 * RB - LOGN;  // batch bits in phase B (0 or 1)
   static constexpr int HB = RB - LV;        // high bits in phase-A registers
-  // the transpose buffer holds a row with V padding floats after every block
-  // of 2^(LV+PB) elements (one value of the high field), NP floats in all
-  static constexpr int NP = N + (N >> (LV + PB)) * V;
-  static_assert(HB >= NB && HB >= 0 && PB >= LV, "row too short for this layout");
+  // Transpose-buffer row: blocks of 4P floats, one per (high field, 16-byte
+  // half u of a narrow vector), each followed by 4 padding floats; rows that
+  // share a warp (P < 32) are further padded so that they start P banks apart.
+  static constexpr int BLK = 4 * P + 4;
+  static constexpr int RP = P < 32 ? ((P - V * (1 << HB)) & 31) : 0;
+  static constexpr int NP = N + V * (1 << HB) + RP;  // floats per row
+  static_assert(HB >= NB && HB >= 0 && PB >= LV && P >= 8, "row too short for this layout");
 
   // element index of register q of thread t, phase A
   __device__ __forceinline__ static int eA(int t, int q) {
@@ -32,11 +35,18 @@ struct Geo {
     return (t & (V - 1)) | ((q & (P - 1)) << LV) | ((t >> LV) << (LV + PB)) |
            ((q >> PB) << (LV + PB + HB - NB));
   }
-  // position in the transpose buffer. The padding shifts each block of the
-  // high field by V banks, so the phase-B lanes (low field t % V, high field
-  // t / V) meet 32 distinct banks, and every position is a per-thread base
-  // plus a constant of the register index (no per-access arithmetic).
-  __device__ __forceinline__ static int phys(int e) { return e + (e >> (LV + PB)) * V; }
+  // Position of element e in its row of the transpose buffer. The low field
+  // splits into i (the 4 floats of a 16-byte access) and u (which 16-byte half
+  // of a narrow vector); u and the high field select the block, the middle
+  // field m the 16-byte slot in it. Phase-A 16-byte accesses (fixed h, u;
+  // lanes = consecutive m) cover 128 contiguous bytes per quarter warp;
+  // phase-B scalar accesses (fixed m; lanes = i, u, high bits, rows) meet 32
+  // distinct banks thanks to the padding. Every position is a per-thread base
+  // plus a compile-time offset in both phases.
+  __device__ __forceinline__ static int phys(int e) {
+    const int i = e & 3, m = (e >> LV) & (P - 1), ub = ((e & (V - 1)) >> 2) | ((e >> (LV + PB)) << (LV - 2));
+    return i + 4 * m + BLK * ub;
+  }
 };
 
 template <typename T, int V>
@@ -164,10 +174,9 @@ __device__ __forceinline__ void fwht_rows_body(const Tin *__restrict__ x, Tout *
 
 #pragma unroll
     for (int h = 0; h < (1 << G::HB); ++h) {
-      float *dst = buf + G::phys(G::eA(t, h << G::LV));
 #pragma unroll
       for (int u = 0; u < V; u += 4)
-        *reinterpret_cast<float4 *>(dst + u) =
+        *reinterpret_cast<float4 *>(buf + G::phys(G::eA(t, h << G::LV) + u)) =
             make_float4(v[h * V + u], v[h * V + u + 1], v[h * V + u + 2], v[h * V + u + 3]);
     }
     bar();  // phase A is in buf, and every thread has read its staged input: fetch the next rows
@@ -187,11 +196,10 @@ __device__ __forceinline__ void fwht_rows_body(const Tin *__restrict__ x, Tout *
 #pragma unroll
       for (int h = 0; h < (1 << G::HB); ++h) {
         const int e = G::eA(t, h << G::LV);
-        const float *src = buf + G::phys(e);
         float o[V];
 #pragma unroll
         for (int u = 0; u < V; u += 4) {
-          const float4 f = *reinterpret_cast<const float4 *>(src + u);
+          const float4 f = *reinterpret_cast<const float4 *>(buf + G::phys(e + u));
           o[u] = f.x, o[u + 1] = f.y, o[u + 2] = f.z, o[u + 3] = f.w;
         }
         store_group<Tout, V>(zr + e, o);
