@@ -44,11 +44,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 ALU_LANES_PER_SM = 128  # fp32 FMA lanes per SM (4 partitions x 32)
 
 KERNEL_SOURCES = {
-    "fwht_fwd": ["fwht.cu", "fwht_body.cuh"], "fwht_bwd": ["fwht.cu", "fwht_body.cuh"], "spmm_fwd": ["sparse.cu"],
-    "gather_bwd": ["sparse.cu"], "sddmm_dc": ["sparse.cu"], "dequant": ["dequant.cu"],
+    "fwht_fwd": ["fwht.cu", "fwht_body.cuh", "bulk.cuh"], "fwht_bwd": ["fwht.cu", "fwht_body.cuh", "bulk.cuh"],
+    "spmm_fwd": ["sparse.cu"], "gather_bwd": ["sparse.cu"], "sddmm_dc": ["sparse.cu"], "dequant": ["dequant.cu"],
     "gemm_fwd": ["gemm.cu", "fwht_body.cuh"], "gemm_bwd": ["gemm.cu", "fwht_body.cuh"],
-    "gemm_dc": ["gemm.cu", "fwht_body.cuh"], "weff": ["fwht.cu", "dense.cu", "fwht_body.cuh"], "init_alloc": ["init.cu"],
-    "plan_build": ["plan.cu"],
+    "gemm_dc": ["gemm.cu", "fwht_body.cuh"], "weff": ["fwht.cu", "dense.cu", "fwht_body.cuh", "bulk.cuh"],
+    "init_alloc": ["init.cu"], "plan_build": ["plan.cu"],
 }
 
 
