@@ -179,6 +179,13 @@ def test_init_tiny_workload_bitexact(mode):
         (48, 32, 32, 48 * 3 + 7, "fewest", "ties"),  # zero rows and integer data: many equal |V|
         (16, 16, 16, 16 * 16, "fewest", "normal"),  # p = d_in * d_out
         (24, 2048, 2048, 24 * 3, "largest", "normal"),  # p = 3 per row, long rows
+        # rows of 4096 entries take the register-resident selection kernel
+        (40, 4096, 4096, 40 * 50 + 7, "fewest", "normal"),
+        (33, 4096, 1024, 33 * 20 + 5, "largest", "normal"),  # block-diagonal: stages above 1024 skipped
+        (17, 4096, 64, 17 * 9 + 3, "fewest", "normal"),  # 64-point blocks: two of three register phases
+        (20, 4096, 4096, 20 * 700, "fewest", "cap"),  # capped rows take all 4096 entries
+        (24, 4096, 4096, 24 * 30 + 11, "largest", "ties"),  # zero rows (all keys equal), many ties
+        (12, 4096, 4096, 12 * 2, "fewest", "normal"),  # the minimum: 2 entries per row
     ],
 )
 def test_init_bitexact(d_out, d_in, n, p, mode, kind):
@@ -199,8 +206,8 @@ def test_init_bitexact(d_out, d_in, n, p, mode, kind):
     assert np.array_equal(got["coef"].cpu().numpy().view(np.uint32), ref["coef"].view(np.uint32))
 
 
-@pytest.mark.parametrize("shards,mode", [(1, "fewest"), (3, "largest")])
-def test_init_split_steps_bitexact(shards, mode):
+@pytest.mark.parametrize("shards,mode,d_in", [(1, "fewest", 1024), (3, "largest", 1024), (2, "fewest", 4096)])
+def test_init_split_steps_bitexact(shards, mode, d_in):
     """qwha_init_norms / _budgets / _select over row shards (as the ranks of a sharded AdaAlloc run them)
     reproduce qwha_init_alloc and the oracle bit for bit; the shards' row_ptr slices do not start at 0."""
     import torch
@@ -208,17 +215,17 @@ def test_init_split_steps_bitexact(shards, mode):
     from walsh_hadamard_sparse_b200.api import shard_rows
 
     W = _W()
-    d_out, d_in, n = 301, 1024, 512
+    d_out, n = 301, 512
     p = d_out * 17 + 9
-    g = rng_for(34, "init-split", shards, mode)
+    g = rng_for(34, "init-split", shards, mode) if d_in == 1024 else rng_for(34, "init-split", shards, mode, d_in)
     w = g.standard_normal((d_out, d_in)).astype(np.float32) * np.float32(0.01)
-    w[7] *= np.float32(500.0)  # capped row
+    w[7] *= np.float32(500.0 if d_in == 1024 else 5000.0)  # capped row
     dw = to_dev(w)
     whole = W.init_alloc(dw, p, n, 2, mode)
     bounds = [shard_rows(d_out, r, shards) for r in range(shards)]
     e = torch.cat([W.init_norms(dw[r0:r1]) for r0, r1 in bounds])
     b, rp = W.init_budgets(e, d_in, p, 2, mode)
-    sel = [W.init_select(dw[r0:r1], n, b[r0:r1], rp[r0:r1 + 1]) for r0, r1 in bounds]
+    sel = [W.init_select(dw[r0:r1], n, b[r0:r1], rp[r0:r1 + 1]) for r0, r1 in bounds]  # slices at any offset
     ci = torch.cat([s[0] for s in sel]).cpu().numpy()
     cf = torch.cat([s[1] for s in sel]).cpu().numpy()
     ref = oracle.init_alloc(w, p, n, 2, mode)

@@ -251,6 +251,8 @@ def init_select(dWq_rows: torch.Tensor, had_block: int, budgets: torch.Tensor,
     rows, d_in = dWq_rows.shape
     p_local = int(row_ptr[-1].item() - row_ptr[0].item()) if rows else 0
     dev = dWq_rows.device
+    # the ABI takes 16-byte aligned pointers: a slice that starts elsewhere is copied
+    dWq_rows, budgets, row_ptr = (t if t.data_ptr() % 16 == 0 else t.clone() for t in (dWq_rows, budgets, row_ptr))
     col_idx = torch.empty(max(p_local, 1), dtype=torch.int32, device=dev)
     coef = torch.empty(max(p_local, 1), dtype=torch.float32, device=dev)
     rc = lib().qwha_init_select(_ptr(dWq_rows), rows, d_in, had_block, _ptr(budgets), _ptr(row_ptr), p_local,

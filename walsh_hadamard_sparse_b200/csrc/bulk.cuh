@@ -72,10 +72,9 @@ __device__ __forceinline__ void store(void *dst, uint32_t src, uint32_t bytes) {
                : "memory");
 }
 __device__ __forceinline__ void commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// This thread's committed stores have read their shared-memory sources.
+// This thread's committed stores have read their shared-memory sources (the
+// writes themselves complete before the grid does).
 __device__ __forceinline__ void wait_stores_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// This thread's committed stores are complete.
-__device__ __forceinline__ void wait_stores() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 }  // namespace bulk
 }  // namespace qwha

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(RingGeo<LOGN, V>::RW) fwht_ring_kernel(const T
       bulk::commit();
     }
   }
-  if (tid == 0) bulk::wait_stores();  // the buffer stays valid until the last copy has read it
+  if (tid == 0) bulk::wait_stores_read();  // the buffer stays valid until the last copy has read it
 }
 
 // n <= 64: one thread per block, all in registers.
