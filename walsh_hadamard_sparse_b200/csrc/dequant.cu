@@ -25,26 +25,50 @@ __device__ __forceinline__ uint32_t code_word(const uint8_t *__restrict__ row, i
   return w;
 }
 
-// One CTA per row at a time (grid-stride over rows), a thread per run of 8
-// codes: no 64-bit index arithmetic, coalesced loads and 16-byte stores.
-__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict__ qw, const float *__restrict__ scales,
-                                                      const uint8_t *__restrict__ zeros, int bits, int group,
-                                                      int d_out, int d_in, __nv_bfloat16 *__restrict__ out) {
-  const int runs = d_in / 8;
+// Grid-stride over blocks of kRuns x 256 runs of 8 codes (a run never crosses
+// a row: d_in is a multiple of 8). A thread issues the loads of its kRuns runs
+// (code word, scale, zero point) before using any of them, so each thread keeps
+// several independent DRAM requests in flight; stores are 16 bytes.
+constexpr int kDeqThreads = 256;
+constexpr int kRuns = 4;
+
+__global__ void __launch_bounds__(kDeqThreads) dequant_kernel(const uint8_t *__restrict__ qw,
+                                                              const float *__restrict__ scales,
+                                                              const uint8_t *__restrict__ zeros, int bits, int group,
+                                                              int d_out, int d_in, __nv_bfloat16 *__restrict__ out) {
+  const int runs_per_row = d_in / 8;
+  const int64_t total = (int64_t)d_out * runs_per_row;
   const int64_t row_bytes = (int64_t)d_in * bits / 8;
   const int ng = d_in / group;
   const uint32_t mask = (1u << bits) - 1u;
-  for (int i = blockIdx.x; i < d_out; i += gridDim.x) {
-    const uint8_t *row = qw + i * row_bytes;
-    for (int r = threadIdx.x; r < runs; r += blockDim.x) {
-      const int k0 = r * 8;
-      const int g = k0 / group;
-      const float sc = scales[(int64_t)i * ng + g], z = (float)zeros[(int64_t)i * ng + g];
-      const uint32_t w = code_word(row, bits, k0);
+  for (int64_t base = (int64_t)blockIdx.x * kDeqThreads * kRuns; base < total;
+       base += (int64_t)gridDim.x * kDeqThreads * kRuns) {
+    uint32_t w[kRuns];
+    float sc[kRuns], z[kRuns];
+    int64_t off[kRuns];
+#pragma unroll
+    for (int u = 0; u < kRuns; ++u) {
+      const int64_t r = base + u * kDeqThreads + threadIdx.x;
+      off[u] = -1;
+      w[u] = 0;
+      sc[u] = 0.f;
+      z[u] = 0.f;
+      if (r < total) {
+        const int i = (int)r / runs_per_row, k0 = ((int)r - i * runs_per_row) * 8;  // total < 2^31
+        const int g = k0 / group;
+        w[u] = code_word(qw + i * row_bytes, bits, k0);
+        sc[u] = scales[(int64_t)i * ng + g];
+        z[u] = (float)zeros[(int64_t)i * ng + g];
+        off[u] = (int64_t)i * d_in + k0;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRuns; ++u) {
+      if (off[u] < 0) continue;
       float v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = sc * ((float)((w >> (bits * q)) & mask) - z);
-      *reinterpret_cast<uint4 *>(out + (int64_t)i * d_in + k0) = io<__nv_bfloat16>::pack(v);
+      for (int q = 0; q < 8; ++q) v[q] = sc[u] * ((float)((w[u] >> (bits * q)) & mask) - z[u]);
+      *reinterpret_cast<uint4 *>(out + off[u]) = io<__nv_bfloat16>::pack(v);
     }
   }
 }
@@ -55,8 +79,10 @@ size_t wdeq_bytes(int32_t d_out, int32_t d_in) { return (size_t)d_out * d_in * 2
 
 cudaError_t launch_dequant(int bits, int group, int32_t d_out, int32_t d_in, const uint8_t *qw, const float *scales,
                            const uint8_t *zeros, void *out, cudaStream_t s) {
-  const int64_t grid = std::min<int64_t>(d_out, (int64_t)sm_count() * 8);
-  dequant_kernel<<<(unsigned)grid, 256, 0, s>>>(qw, scales, zeros, bits, group, d_out, d_in,
+  const int64_t total = (int64_t)d_out * (d_in / 8);
+  if (total > 0x7fffffff) return cudaErrorInvalidValue;  // run indices are 32-bit
+  const int64_t grid = std::min<int64_t>(cdiv(total, (int64_t)kDeqThreads * kRuns), (int64_t)sm_count() * 8);
+  dequant_kernel<<<(unsigned)grid, kDeqThreads, 0, s>>>(qw, scales, zeros, bits, group, d_out, d_in,
                                                 static_cast<__nv_bfloat16 *>(out));
   return cudaGetLastError();
 }

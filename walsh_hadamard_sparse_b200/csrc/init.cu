@@ -603,13 +603,16 @@ __device__ void row_transform_fp64(const float *__restrict__ w, int d_in, int n,
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads)
+// NT threads per row: 256, or 1024 for long rows, whose buffer leaves room for
+// one CTA per SM only.
+template <int NT>
+__global__ void __launch_bounds__(NT)
     select_kernel(const float *__restrict__ dW, int d_in, int n, const int32_t *__restrict__ budgets,
                   const int32_t *__restrict__ row_ptr, int64_t p, int32_t *__restrict__ col_idx,
                   float *__restrict__ coef) {
   extern __shared__ __align__(16) double v[];  // d_in values of the row
   __shared__ uint32_t hist[kHistBins];
-  __shared__ int64_t sh64[kSelThreads];
+  __shared__ int64_t sh64[128];
   const int64_t row = blockIdx.x;
   row_transform_fp64(dW + row * d_in, d_in, n, v);
   const int b = budgets[row];
@@ -1117,9 +1120,11 @@ cudaError_t launch_select_rows(const float *dW, int32_t rows, int32_t d_in, int3
     k<<<rows, kSelThreads, smem, s>>>(dW, had_block, budgets, row_ptr, p, col_idx, coef);
     return cudaGetLastError();
   }
-  cudaError_t err = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool wide = smem > 64 * 1024;
+  auto k = wide ? select_kernel<1024> : select_kernel<kSelThreads>;
+  cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  select_kernel<<<rows, kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
+  k<<<rows, wide ? 1024 : kSelThreads, smem, s>>>(dW, d_in, had_block, budgets, row_ptr, p, col_idx, coef);
   return cudaGetLastError();
 }
 
