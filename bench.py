@@ -442,9 +442,14 @@ def main():
 
         def step():
             W.adapter_fwd(ad, X, alpha, wq, Z_out=Z, Y=Y, ws=wf)
-            W.adapter_bwd(ad, dY, Z, alpha, wq, dc=dc, dX=dX, ws=wb)
             if world > 1:
-                dist.all_reduce(dc)
+                # dc first; its all-reduce (the path's one exchange) overlaps the dX computation
+                W.adapter_bwd(ad, dY, Z, alpha, wq, dc=dc, want_dx=False, ws=wb)
+                work = dist.all_reduce(dc, async_op=True)
+                W.adapter_bwd(ad, dY, Z, alpha, wq, dX=dX, want_dc=False, ws=wb)
+                work.wait()
+            else:
+                W.adapter_bwd(ad, dY, Z, alpha, wq, dc=dc, dX=dX, ws=wb)
 
         return step
 
@@ -554,9 +559,13 @@ def main():
                     ready[b].record(cs)
                 comp.wait_event(ready[b])
                 W.adapter_fwd(ad, Xb, alpha, wq, Z_out=Z, Y=Y, ws=wf)
-                W.adapter_bwd(ad, dYb, Z, alpha, wq, dc=dc, dX=dX, ws=wb)
                 if world > 1:
-                    dist.all_reduce(dc)
+                    W.adapter_bwd(ad, dYb, Z, alpha, wq, dc=dc, want_dx=False, ws=wb)
+                    work = dist.all_reduce(dc, async_op=True)
+                    W.adapter_bwd(ad, dYb, Z, alpha, wq, dX=dX, want_dc=False, ws=wb)
+                    work.wait()
+                else:
+                    W.adapter_bwd(ad, dYb, Z, alpha, wq, dc=dc, dX=dX, ws=wb)
                 free[b].record(comp)
                 dch.copy_(dc, non_blocking=True)
 

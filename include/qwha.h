@@ -169,8 +169,10 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
  *   dX    = dY W_Q + alpha (dY F) H              [T, d_in], dtype dt
  * Z is the Z_out of the matching forward. dc is overwritten (not accumulated).
  * The sparse algorithm needs all views of `a` (qwha_plan_build). dX may be
- * NULL to skip it. Every reduction runs in a fixed order: results are bitwise
- * reproducible. */
+ * NULL to skip it, and dc may be NULL to skip the coefficient gradient (a
+ * data-parallel caller computes dc first, starts its all-reduce, then dX; the
+ * results are the same as from one call). Every reduction runs in a fixed
+ * order: results are bitwise reproducible. */
 qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt,
                              const void *dY, const void *Z, int64_t T, float alpha, float *dc,
                              void *dX, void *ws, size_t ws_bytes, void *stream);

@@ -354,6 +354,30 @@ def test_base_gemm_forward_backward(d_in, d_out, n, T, bits, group, algo):
     assert rel_fro(host(Yb), L["X"].astype(np.float64) @ Wq.T) <= TOL_BF16
 
 
+@pytest.mark.parametrize("algo", ["sparse", "dense"])
+def test_backward_in_two_calls_bitwise(algo):
+    """dc alone (dX NULL), then dX alone (dc NULL), as a data-parallel step issues them around the all-reduce of dc:
+    bit for bit the outputs of one call."""
+    import torch
+
+    W = _W()
+    d_in, d_out, n, T = 1024, 768, 1024, 300
+    L = synth_layer(38, d_in, d_out, n, T, d_out * 8, "bf16", bits=4, group=128)
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"], algo=algo)
+    if algo == "dense":
+        a.weff = torch.empty((d_out, d_in), dtype=torch.bfloat16, device="cuda")
+    wq = dev_qweight(L)
+    Z, _ = W.adapter_fwd(a, dev_act(L["X"], "bf16"), 0.8, wq=wq)
+    dYd = dev_act(L["dY"], "bf16")
+    dc1, dX1 = W.adapter_bwd(a, dYd, Z, 0.8, wq=wq)
+    dc2, none_dx = W.adapter_bwd(a, dYd, Z, 0.8, wq=wq, want_dx=False)
+    none_dc, dX2 = W.adapter_bwd(a, dYd, Z, 0.8, wq=wq, want_dc=False)
+    torch.cuda.synchronize()
+    assert none_dx is None and none_dc is None
+    assert torch.equal(dc1.view(torch.int32), dc2.view(torch.int32))
+    assert torch.equal(dX1.view(torch.int16), dX2.view(torch.int16))
+
+
 @pytest.mark.parametrize("d_in,d_out,n,T", [(4096, 512, 4096, 300), (3 * 2048, 384, 2048, 129), (4096, 256, 4096, 8)])
 def test_dense_forward_fused_transform(d_in, d_out, n, T):
     """The dense forward with Hadamard blocks of 2048 / 4096 writes Z from extra warps of the GEMM launch: Z bit for

@@ -138,10 +138,13 @@ def adapter_fwd(a: Adapter, X: torch.Tensor, alpha: float = 1.0, wq: QWeight | N
 
 def adapter_bwd(a: Adapter, dY: torch.Tensor, Z: torch.Tensor, alpha: float = 1.0, wq: QWeight | None = None,
                 dc: torch.Tensor | None = None, dX: torch.Tensor | None = None, want_dx: bool = True,
-                ws: torch.Tensor | None = None):
-    """(dc, dX): dc_j = alpha sum_t dY[t,r_j] Z[t,k_j]; dX = dY W_Q + alpha (dY F) H."""
+                ws: torch.Tensor | None = None, want_dc: bool = True):
+    """(dc, dX): dc_j = alpha sum_t dY[t,r_j] Z[t,k_j]; dX = dY W_Q + alpha (dY F) H.
+    want_dc / want_dx False skip that output (returned as None): a data-parallel step computes dc, starts its
+    all-reduce, then computes dX while the all-reduce runs."""
     T = dY.shape[0]
-    dc = torch.empty(a.p, dtype=torch.float32, device=dY.device) if dc is None else dc
+    if want_dc and dc is None:
+        dc = torch.empty(a.p, dtype=torch.float32, device=dY.device)
     if want_dx and dX is None:
         dX = torch.empty((T, a.d_in), dtype=dY.dtype, device=dY.device)
     need = workspace_size(OP_BWD_DENSE if a.algo == "dense" else OP_BWD, a.d_out, a.d_in, a.p, T, wq is not None)
@@ -149,10 +152,10 @@ def adapter_bwd(a: Adapter, dY: torch.Tensor, Z: torch.Tensor, alpha: float = 1.
     cs = a.c_struct()
     cw = wq.c_struct() if wq is not None else None
     rc = lib().qwha_adapter_bwd(ctypes.byref(cs), ctypes.byref(cw) if cw is not None else None, _dt(dY), _ptr(dY),
-                                _ptr(Z), T, float(alpha), _ptr(dc), _ptr(dX) if want_dx else None, _ptr(ws),
-                                0 if ws is None else ws.numel(), _stream())
+                                _ptr(Z), T, float(alpha), _ptr(dc) if want_dc else None,
+                                _ptr(dX) if want_dx else None, _ptr(ws), 0 if ws is None else ws.numel(), _stream())
     check(rc, "qwha_adapter_bwd")
-    return dc, dX
+    return (dc if want_dc else None), (dX if want_dx else None)
 
 
 def init_alloc(dWq: torch.Tensor, p: int, had_block: int, min_per_row: int = 2, mode: str = "fewest",

@@ -368,7 +368,7 @@ qwha_status dense_bwd(const qwha_adapter *a, const qwha_qweight *wq, const void 
     }
     if (e != cudaSuccess) return cuda_status(e, "GEMM dX");
   }
-  if (a->p == 0) return QWHA_OK;
+  if (a->p == 0 || !dc) return QWHA_OK;
   if (T == 0) return cuda_status(cudaMemsetAsync(dc, 0, (size_t)a->p * 4, s), "dc = 0");
   // the coefficient gradient as a sampled dense product: the tcgen05 GEMM's
   // epilogue writes alpha * (dY^T Z)[r_j, k_j] for the entries of E only
@@ -512,7 +512,7 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   if (dense && dt != QWHA_BF16) return fail(QWHA_ERR_UNSUPPORTED, "the dense algorithm needs dtype bf16");
   if ((st = check_qweight(wq, a->d_out, a->d_in, dt)) != QWHA_OK) return st;
   if (T < 0) return fail(QWHA_ERR_INVALID_ARG, "T %lld < 0", (long long)T);
-  if (a->p > 0) QWHA_CHECK_PTR(dc, "dc");
+  if (a->p > 0 && dc) QWHA_CHECK_PTR(dc, "dc");
   if (T > 0) {
     QWHA_CHECK_PTR(dY, "dY");
     QWHA_CHECK_PTR(Z, "Z");
@@ -527,7 +527,7 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   float *dz = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
   float *coef_csc = static_cast<float *>(cv.take((size_t)(a->p > 0 ? a->p : 1) * 4));
   cudaError_t e = cudaSuccess;
-  {
+  if (dc) {
     StageScope sc(ST_SDDMM, 2, s);
     e = launch_sddmm(dt, dY, Z, T, a->d_out, a->d_in, a->tile_ptr, a->tile_pos, a->tile_rk, a->p, alpha, partial, dc,
                      s);
