@@ -43,6 +43,10 @@ FLUSH_BYTES = 512 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 ALU_LANES_PER_SM = 128  # fp32 FMA lanes per SM (4 partitions x 32)
 
+# the stages of a step that exist only because of the adapter (the rest is the frozen layer's own GEMMs)
+ADAPTER_STAGES = {"dense": ["weff", "gemm_dc"],
+                  "sparse": ["fwht_fwd", "spmm_fwd", "sddmm_dc", "gather_bwd", "fwht_bwd"]}
+
 KERNEL_SOURCES = {
     "fwht_fwd": ["fwht.cu", "fwht_body.cuh", "bulk.cuh"], "fwht_bwd": ["fwht.cu", "fwht_body.cuh", "bulk.cuh"],
     "spmm_fwd": ["sparse.cu"], "gather_bwd": ["sparse.cu"], "sddmm_dc": ["sparse.cu"], "dequant": ["dequant.cu"],
@@ -606,6 +610,15 @@ def main():
     init_bytes = 2 * 4.0 * spec.d_in * spec.d_out + 8.0 * spec.p
     init_med = statistics.median(init_ms)
     sp = results["sparse"]
+
+    def adapter_only(res, algo):
+        """The adapter's share of a step (tokens/s over its stages alone): the sparse path's transforms, SpMM, SDDMM
+        and gather; the dense path's W_eff and coefficient-gradient GEMM (its forward and dX ride in the GEMMs the
+        frozen layer runs anyway; the transform inside the forward GEMM's launch is counted there, not here)."""
+        names = ADAPTER_STAGES[algo]
+        ms = sum(res["kernels"][n]["ms_per_call"] * res["kernels"][n]["calls"] for n in names if n in res["kernels"])
+        ms /= res["K"]
+        return {"ms_per_step": ms, "value": world * T / (ms / 1e3), "unit": UNIT, "stages": names}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": t_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -619,8 +632,10 @@ def main():
         "gpu_launches": launches,
         "clocks": clk,
         "kernels": kernels,
+        "adapter_only": adapter_only(head, "dense"),
         "paths": {
             "sparse": {"value": sp["value"], "unit": UNIT, "steps": sp["K"], "ms_per_step": sp["t_ms"] / sp["K"],
+                       "adapter_only": adapter_only(sp, "sparse"),
                        "roofline": sp["roofline"], "gpu_launches": sp["launches"], "kernels": sp["kernels"],
                        "what": "segment SpMM over CSR, tiled SDDMM, CSC gather on the FMA units; base GEMMs on tcgen05"},
         },

@@ -54,6 +54,16 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Copy `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
+// memory into this CTA's shared memory, completing on `bar` (whose expected
+// transaction count the caller has raised). No multicast.
+__device__ __forceinline__ void copy(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // Arrive on `bar` announcing `bytes` of copies that will complete on it, then
 // copy `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
 // memory into this CTA's shared memory. No multicast.

@@ -470,11 +470,266 @@ __global__ void __launch_bounds__(kThreads, 2)
   cp_async_wait_all();  // no copy is left in flight when the CTA exits
 }
 
+// W_eff blocks of 2048 or 4096 columns, ring-fed like fwht_ring_kernel: a CTA
+// of 64 threads takes 64/P blocks per iteration; one thread copies each
+// block's code block, scales, zero points and a 16-byte aligned window of its
+// row's CSR slice (column, coefficient) into an S-slot shared-memory ring with
+// bulk copies, S - 1 iterations ahead (a slot is refilled once its codes have
+// been used by the final add). The row_ptr pair of the block to copy next is
+// loaded one iteration before it is needed. Entries past the window (rows of
+// more than kWeffWin - 8 entries, or the last entries of the arrays) are read
+// directly. Arithmetic as weff_pipe_kernel: scatter into the padded buffer,
+// two butterfly phases, base weight added in fp32 in phase-A layout, one bf16
+// rounding. Needs the 16-byte alignments checked by run_weff.
+constexpr int kWeffWin = 520;  // CSR window entries per block (a multiple of 4)
+
+struct WeffRingLayout {
+  int qb, gpb;         // code bytes and quantization groups per block
+  int o_sc, o_z, o_k;  // byte offsets of scales, zero points and the CSR window in a block's part of a slot
+  int blk;             // bytes of a block's part of a slot
+  __host__ __device__ WeffRingLayout(int n, int bits, int group) {
+    qb = n * bits / 8;
+    gpb = n / group;
+    o_sc = round16(qb);
+    o_z = o_sc + round16(gpb * 4);
+    o_k = o_z + round16(gpb);
+    blk = o_k + 2 * kWeffWin * 4;
+  }
+};
+
+template <int LOGN, int S>
+__global__ void __launch_bounds__(64) weff_ring_kernel(const int32_t *__restrict__ row_ptr,
+                                                       const int32_t *__restrict__ col_idx,
+                                                       const float *__restrict__ coef, int64_t p, int d_in,
+                                                       int64_t n_rows, float scale, int bits, int group,
+                                                       const uint8_t *__restrict__ qw, const float *__restrict__ scales,
+                                                       const uint8_t *__restrict__ zeros,
+                                                       __nv_bfloat16 *__restrict__ out, unsigned int *err) {
+  using G = Geo<LOGN, 8>;
+  static_assert(G::P >= 32, "one warp or more per block");
+  constexpr int RW = 64, RPW = RW / G::P;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  float *buf_all = reinterpret_cast<float *>(smem_raw);
+  const WeffRingLayout L(G::N, bits, group);
+  const int slot_bytes = RPW * L.blk;
+  unsigned char *ring = smem_raw + ((RPW * G::NP * 4 + 127) & ~127);
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + S * slot_bytes);
+  int *meta = reinterpret_cast<int *>(full + S);  // per slot and block: b, e, a0, a1
+  const int tid = threadIdx.x, rl = tid / G::P, t = tid % G::P;
+  float *buf = buf_all + rl * G::NP;
+  const int nb = d_in >> LOGN;
+  const int64_t blocks = n_rows * nb;
+  const int64_t row_bytes = (int64_t)d_in * bits / 8;
+  const int ng = d_in / group;
+  const int64_t stride = (int64_t)gridDim.x * RPW;
+  const int64_t first = (int64_t)blockIdx.x * RPW;
+  const int64_t iters = first < blocks ? (blocks - first + stride - 1) / stride : 0;
+  const int64_t p4 = p & ~(int64_t)3;
+
+  // thread 0: copy the inputs of iteration it (row_ptr pairs in rp) into its slot
+  auto issue = [&](int64_t it, const int *rp) {
+    const int s = (int)(it % S);
+    unsigned char *sl = ring + s * slot_bytes;
+    uint32_t bytes = 0;
+    int a[RPW][2];
+    for (int q = 0; q < RPW; ++q) {
+      const int64_t bi = first + it * stride + q;
+      int b = 0, e = 0, a0 = 0, a1 = 0;
+      if (bi < blocks) {
+        b = rp[2 * q];
+        e = rp[2 * q + 1];
+        if (b < 0) b = 0;
+        if (e > p) e = (int)p;
+        if (e < b) e = b;
+        a0 = b & ~3;
+        int64_t hi = ((int64_t)e + 3) & ~(int64_t)3;
+        if (hi > p4) hi = p4;
+        if (hi > a0 + kWeffWin) hi = a0 + kWeffWin;
+        a1 = hi > a0 ? (int)hi : a0;
+        bytes += L.qb + L.gpb * 4 + L.gpb + 8 * (a1 - a0);
+      }
+      int *m = meta + 4 * (s * RPW + q);
+      m[0] = b, m[1] = e, m[2] = a0, m[3] = a1;
+      a[q][0] = a0, a[q][1] = a1;
+    }
+    bulk::fence_proxy();
+    const uint32_t bar = bulk::saddr(full + s);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    for (int q = 0; q < RPW; ++q) {
+      const int64_t bi = first + it * stride + q;
+      if (bi >= blocks) continue;
+      const int64_t r = bi / nb;
+      const int kb = (int)(bi % nb);
+      unsigned char *d = sl + q * L.blk;
+      bulk::copy(bulk::saddr(d), qw + r * row_bytes + (int64_t)kb * L.qb, L.qb, bar);
+      bulk::copy(bulk::saddr(d + L.o_sc), scales + r * ng + (int64_t)kb * L.gpb, L.gpb * 4, bar);
+      bulk::copy(bulk::saddr(d + L.o_z), zeros + r * ng + (int64_t)kb * L.gpb, L.gpb, bar);
+      const int a0 = a[q][0], a1 = a[q][1];
+      if (a1 > a0) {
+        bulk::copy(bulk::saddr(d + L.o_k), col_idx + a0, 4 * (a1 - a0), bar);
+        bulk::copy(bulk::saddr(d + L.o_k + 4 * kWeffWin), coef + a0, 4 * (a1 - a0), bar);
+      }
+    }
+  };
+  auto load_rp = [&](int64_t it, int *rp) {  // row_ptr pairs of iteration it's blocks
+    for (int q = 0; q < RPW; ++q) {
+      const int64_t bi = first + it * stride + q;
+      rp[2 * q] = rp[2 * q + 1] = 0;
+      if (it < iters && bi < blocks) {
+        const int64_t r = bi / nb;
+        rp[2 * q] = row_ptr[r];
+        rp[2 * q + 1] = row_ptr[r + 1];
+      }
+    }
+  };
+
+  int rp_next[2 * RPW];
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) bulk::init(bulk::saddr(full + s), 1);
+    bulk::fence_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int64_t it = 0; it < S && it < iters; ++it) {
+      load_rp(it, rp_next);
+      issue(it, rp_next);
+    }
+  }
+
+  for (int64_t it = 0; it < iters; ++it) {
+    const int s = (int)(it % S);
+    if (tid == 0) load_rp(it + S, rp_next);  // consumed at the end of this iteration
+    const bool ok = bulk::wait(bulk::saddr(full + s), (uint32_t)((it / S) & 1));
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) {
+        atomicOr(err, 0x400u);
+        for (int64_t j = it; j < iters && j < it + S; ++j)
+          (void)bulk::wait(bulk::saddr(full + (int)(j % S)), (uint32_t)((j / S) & 1));
+      }
+      return;
+    }
+    const unsigned char *sl = ring + s * slot_bytes + rl * L.blk;
+    const int64_t bi = first + it * stride + rl;
+    const bool active = bi < blocks;
+    const int64_t r = active ? bi / nb : 0;
+    const int k0 = active ? (int)(bi % nb) << LOGN : 0;
+    for (int i = 4 * tid; i < RPW * G::NP; i += 4 * RW)
+      *reinterpret_cast<float4 *>(buf_all + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    if (active) {
+      const int *m = meta + 4 * (s * RPW + rl);
+      const int b = m[0], e = m[1], a0 = m[2], a1 = m[3];
+      const int32_t *wk = reinterpret_cast<const int32_t *>(sl + L.o_k);
+      const float *wv = reinterpret_cast<const float *>(sl + L.o_k + 4 * kWeffWin);
+      for (int j = b + t; j < e; j += G::P) {
+        const bool in_win = j < a1;
+        const int k = (in_win ? wk[j - a0] : col_idx[j]) - k0;
+        if ((unsigned)k < (unsigned)G::N) buf[G::phys(k)] = in_win ? wv[j - a0] : coef[j];
+      }
+    }
+    __syncthreads();
+    float v[G::R];
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+#pragma unroll
+      for (int u = 0; u < 8; u += 4) {
+        const float4 f = *reinterpret_cast<const float4 *>(buf + G::phys(G::eA(t, h << G::LV) + u));
+        v[h * 8 + u] = f.x, v[h * 8 + u + 1] = f.y, v[h * 8 + u + 2] = f.z, v[h * 8 + u + 3] = f.w;
+      }
+    }
+    butterflies_x2<G::R, 0, G::RB, 0>(v);
+#pragma unroll
+    for (int h = 0; h < (1 << G::HB); ++h) {
+#pragma unroll
+      for (int u = 0; u < 8; u += 4)
+        *reinterpret_cast<float4 *>(buf + G::phys(G::eA(t, h << G::LV) + u)) =
+            make_float4(v[h * 8 + u], v[h * 8 + u + 1], v[h * 8 + u + 2], v[h * 8 + u + 3]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) v[q] = buf[G::phys(G::eB(t, q))];
+    butterflies_x2<G::R, 0, G::PB, (G::NB ? G::PB : 0)>(v);
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < G::R; ++q) buf[G::phys(G::eB(t, q))] = v[q] * scale;
+    __syncthreads();
+    if (active) {
+      const uint8_t *cq = sl;
+      const float *s_sc = reinterpret_cast<const float *>(sl + L.o_sc);
+      const uint8_t *s_z = sl + L.o_z;
+      const uint32_t mask = (1u << bits) - 1u;
+#pragma unroll
+      for (int h = 0; h < (1 << G::HB); ++h) {
+        const int el = G::eA(t, h << G::LV);
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; u += 4) {
+          const float4 a = *reinterpret_cast<const float4 *>(buf + G::phys(el + u));
+          f[u] = a.x, f[u + 1] = a.y, f[u + 2] = a.z, f[u + 3] = a.w;
+        }
+        const uint8_t *cp = cq + el * bits / 8;
+        uint32_t w;
+        if (bits == 4) {
+          w = *reinterpret_cast<const uint32_t *>(cp);
+        } else if (bits == 2) {
+          w = *reinterpret_cast<const uint16_t *>(cp);
+        } else {
+          w = 0;
+          for (int bb = 0; bb < bits; ++bb) w |= (uint32_t)cp[bb] << (8 * bb);
+        }
+        const int g = el / group;
+        const float sc = s_sc[g], z = (float)s_z[g];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] += sc * ((float)((w >> (bits * i)) & mask) - z);
+        st_stream(out + r * d_in + k0 + el, io<__nv_bfloat16>::pack(f));
+      }
+    }
+    __syncthreads();  // slot s and the buffer are free
+    if (tid == 0 && it + S < iters) issue(it + S, rp_next);
+  }
+}
+
+constexpr int kWeffRingSlots = 3;
+
+template <int LOGN>
+cudaError_t run_weff_ring(const int32_t *row_ptr, const int32_t *col_idx, const float *coef, int64_t p, int d_in,
+                          int64_t n_rows, float scale, int bits, int group, const uint8_t *qw, const float *scales,
+                          const uint8_t *zeros, __nv_bfloat16 *out, cudaStream_t s) {
+  using G = Geo<LOGN, 8>;
+  constexpr int S = kWeffRingSlots, RPW = 64 / G::P;
+  const WeffRingLayout L(G::N, bits, group);
+  const size_t smem = (((size_t)RPW * G::NP * 4 + 127) & ~(size_t)127) + (size_t)S * RPW * L.blk + (size_t)S * 8 +
+                      (size_t)S * RPW * 16;
+  auto k = weff_ring_kernel<LOGN, S>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, 64, smem);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  const int64_t blocks = n_rows * (d_in >> LOGN);
+  const int64_t need = cdiv(blocks, RPW), cap = (int64_t)sm_count() * occ;
+  k<<<(unsigned)(need < cap ? need : cap), 64, smem, s>>>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group,
+                                                         qw, scales, zeros, out, device_error_word());
+  return cudaGetLastError();
+}
+
 template <int LOGN>
 cudaError_t run_weff(const int32_t *row_ptr, const int32_t *col_idx, const float *coef, int64_t p, int d_in,
                      int64_t n_rows, float scale, int bits, int group, const uint8_t *qw, const float *scales,
                      const uint8_t *zeros, __nv_bfloat16 *out, cudaStream_t s) {
   using G = Geo<LOGN, 8>;
+  if constexpr (LOGN >= 11) {
+    // the ring-fed kernel copies every per-block input with 16-byte aligned bulk copies
+    const int gpb = G::N / group, ng = d_in / group;
+    const bool ring = qw && (int64_t)G::N * bits % 128 == 0 && (int64_t)d_in * bits % 128 == 0 && gpb % 16 == 0 &&
+                      ng % 16 == 0 && aligned16(qw) && aligned16(scales) && aligned16(zeros) && aligned16(col_idx) &&
+                      aligned16(coef);
+    if (ring)
+      return run_weff_ring<LOGN>(row_ptr, col_idx, coef, p, d_in, n_rows, scale, bits, group, qw, scales, zeros, out,
+                                 s);
+  }
   constexpr int RPC = kThreads / G::P;
   const int64_t blocks = n_rows * (d_in >> LOGN);
   // the pipelined kernel copies code blocks and scales in 16-byte pieces and
