@@ -13,11 +13,13 @@
 //
 // Kernels here: weff_kernel (one CTA per row of W_eff: scatter the row of F
 // into shared memory, fp32 butterflies per Hadamard block, add the dequantized
-// base row, one bf16 rounding; used for Hadamard blocks outside 128..4096,
-// the main path is weff_rows_kernel in fwht.cu on the transform's register
-// layout). The GEMMs read dY, Z and W_eff as stored (MN-major operands), so
-// nothing is transposed, and the coefficient gradient is written by the
-// sampled epilogue of the dY^T Z GEMM (gemm.cu), so G never reaches memory.
+// base row, one bf16 rounding; used for Hadamard blocks outside 128..4096).
+// Blocks of 128..4096 take the kernels in fwht.cu that share the transform's
+// register layout (weff_ring_kernel for blocks of 2048 and 4096 with a base
+// weight, weff_pipe_kernel and weff_rows_kernel otherwise). The GEMMs read
+// dY, Z and W_eff as stored (MN-major operands), so nothing is transposed,
+// and the coefficient gradient is written by the sampled epilogue of the
+// dY^T Z GEMM (gemm.cu), so G never reaches memory.
 
 #include <algorithm>
 
