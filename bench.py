@@ -647,7 +647,9 @@ def main():
                  "refine_what": ("Value Refinement at E: calibration Hessian X^T X over the 8192 tokens, G = H S H, "
                                  "dW_Q S H, per-channel fp64 Cholesky solves"),
                  "select_global_what": ("whole-matrix selection (magnitude top-p; seeded random E): fp64 transform of "
-                                        "all rows kept in HBM, 8 radix passes over 16.8 M keys, per-row compaction")},
+                                        "all rows kept in HBM, 8-bit radix passes over the 16.8 M keys until the "
+                                        "candidates fit a 64 K list, one CTA finishes on the list, per-row "
+                                        "compaction")},
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -920,10 +920,19 @@ __global__ void __launch_bounds__(kSelThreads, 3)
 constexpr int kGselThreads = 256;
 
 struct GselState {
-  unsigned long long prefix;  // digits of K fixed so far
+  unsigned long long prefix;  // digits of K fixed so far (all of K once `listed`)
   long long need;             // how many keys equal to the prefix are still to be taken
   uint32_t hist[256];
+  unsigned long long cand_n;  // keys in the candidate list
+  uint32_t match;             // keys that match the prefix after the last pass
+  int want_list;              // the keys matching the prefix fit the list: list them
+  int listed;                 // K and need are final; later passes do nothing
 };
+
+// Once the keys that match the prefix number at most kGselCap, one pass copies
+// them into a list in the workspace and a single CTA finishes the selection on
+// the list (the remaining passes over all keys are skipped).
+constexpr int kGselCap = 1 << 16;
 
 __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t n) {
   uint64_t z = seed + n * 0x9E3779B97F4A7C15ull;
@@ -949,6 +958,10 @@ __global__ void gsel_init_kernel(GselState *st, int64_t p) {
   if (threadIdx.x == 0) {
     st->prefix = 0;
     st->need = p;
+    st->cand_n = 0;
+    st->match = 0xffffffffu;
+    st->want_list = 0;
+    st->listed = 0;
   }
   for (int i = threadIdx.x; i < 256; i += blockDim.x) st->hist[i] = 0;
 }
@@ -956,6 +969,7 @@ __global__ void gsel_init_kernel(GselState *st, int64_t p) {
 // Histogram of digit `shift` over the keys that match the prefix so far.
 __global__ void __launch_bounds__(kGselThreads)
     gsel_hist_kernel(const double *__restrict__ V, int64_t N, int sel, uint64_t seed, int shift, GselState *st) {
+  if (st->listed) return;
   __shared__ uint32_t hist[256];
   for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
   __syncthreads();
@@ -980,6 +994,7 @@ __global__ void __launch_bounds__(kGselThreads)
 
 // One warp: the digit that holds the need-th key, then clear the histogram.
 __global__ void gsel_pick_kernel(GselState *st, int shift) {
+  if (st->listed) return;
   const int lane = threadIdx.x;
   const long long need = st->need;
   uint32_t c[8];
@@ -1001,16 +1016,20 @@ __global__ void gsel_pick_kernel(GselState *st, int shift) {
   if (hit) {
     long long cum = excl;
     int d = 8 * lane + 7;
+    uint32_t cnt = c[7];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (cum + c[j] >= need) {
         d = 8 * lane + j;
+        cnt = c[j];
         break;
       }
       cum += c[j];
     }
     st->prefix |= (unsigned long long)d << shift;
     st->need = need - cum;
+    st->match = cnt;
+    st->want_list = need - cum > 0 && cnt <= (uint32_t)kGselCap;
   } else if (who == 0 && lane == 31) {
     st->prefix |= 255ull << shift;
     st->need = need - (long long)incl;
@@ -1018,6 +1037,51 @@ __global__ void gsel_pick_kernel(GselState *st, int shift) {
   __syncwarp();
 #pragma unroll
   for (int j = 0; j < 8; ++j) st->hist[8 * lane + j] = 0;
+}
+
+// The keys that match the prefix after pass `shift` (at most kGselCap) into cand.
+__global__ void __launch_bounds__(kGselThreads)
+    gsel_list_kernel(const double *__restrict__ V, int64_t N, int sel, uint64_t seed, int shift, GselState *st,
+                     unsigned long long *__restrict__ cand) {
+  if (st->listed || !st->want_list) return;
+  const uint64_t prefix = st->prefix;
+  const uint64_t mask = ~0ull << shift;
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t n_round = (N + stride - 1) / stride * stride;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n_round; j += stride) {
+    uint64_t k = 0;
+    bool m = false;
+    if (j < N) {
+      k = gsel_key(V, j, sel, seed);
+      m = (k & mask) == (prefix & mask);
+    }
+    const unsigned mm = __ballot_sync(0xffffffffu, m);
+    unsigned long long base = 0;
+    if (lane == 0 && mm) base = atomicAdd(&st->cand_n, (unsigned long long)__popc(mm));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const unsigned long long at = base + __popc(mm & ((1u << lane) - 1u));
+    if (m && at < (unsigned long long)kGselCap) cand[at] = k;
+  }
+}
+
+// One CTA: K and its need from the candidate list (the radix select of the
+// per-row selection, over the list); the remaining passes then do nothing.
+__global__ void __launch_bounds__(1024) gsel_finish_kernel(GselState *st, const unsigned long long *__restrict__ cand) {
+  if (st->listed || !st->want_list) return;
+  __shared__ uint32_t hist[kHistBins];
+  const unsigned long long n64 = st->cand_n;
+  const int n = (int)(n64 < (unsigned long long)kGselCap ? n64 : (unsigned long long)kGselCap);
+  uint64_t K;
+  int64_t need;
+  radix_select_smallest<false>(n, st->need, [&](int i) -> uint64_t { return cand[i]; }, [](int) { return true; },
+                               hist, &K, &need);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    st->prefix = K;
+    st->need = need;
+    st->listed = 1;
+  }
 }
 
 // Per row: keys below K and keys equal to K.
@@ -1140,7 +1204,8 @@ cudaError_t launch_init_alloc(const float *dW, int32_t d_out, int32_t d_in, int3
 }
 
 size_t select_global_workspace(int32_t d_out, int32_t d_in) {
-  return align_up((size_t)d_out * d_in * 8, 256) + align_up(sizeof(GselState), 256) + 3 * align_up((size_t)d_out * 4, 256);
+  return align_up((size_t)d_out * d_in * 8, 256) + align_up(sizeof(GselState), 256) + 3 * align_up((size_t)d_out * 4, 256) +
+         (size_t)kGselCap * 8;
 }
 
 cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p, int sel,
@@ -1156,6 +1221,8 @@ cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, i
   int32_t *eq = reinterpret_cast<int32_t *>(w);
   w += align_up((size_t)d_out * 4, 256);
   int32_t *take = reinterpret_cast<int32_t *>(w);
+  w += align_up((size_t)d_out * 4, 256);
+  unsigned long long *cand = reinterpret_cast<unsigned long long *>(w);
   const size_t smem = vbytes(d_in);
   cudaError_t e = cudaFuncSetAttribute(gsel_transform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess)
@@ -1168,6 +1235,10 @@ cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, i
   for (int shift = 56; shift >= 0; shift -= 8) {
     gsel_hist_kernel<<<(unsigned)grid, kGselThreads, 0, s>>>(V, N, sel, seed, shift, st);
     gsel_pick_kernel<<<1, 32, 0, s>>>(st, shift);
+    if (shift > 0) {  // after the last pass the prefix is K itself
+      gsel_list_kernel<<<(unsigned)grid, kGselThreads, 0, s>>>(V, N, sel, seed, shift, st, cand);
+      gsel_finish_kernel<<<1, 1024, 0, s>>>(st, cand);
+    }
   }
   gsel_count_kernel<<<d_out, kGselThreads, 0, s>>>(V, d_in, sel, seed, st, lt, eq);
   gsel_budget_kernel<<<1, kBudgetThreads, 0, s>>>(lt, eq, d_out, st, take, budgets, row_ptr);
