@@ -29,6 +29,25 @@ namespace qwha {
 namespace {
 
 constexpr int kSpmmThreads = 512;
+
+// For a kernel that runs one CTA per SM over `units` independent CTAs: the
+// smallest factor s <= max_split by which to subdivide each unit so that the
+// last wave is at least 95% full (else the factor with the fullest last wave).
+int wave_split(int64_t units, int max_split) {
+  const int64_t slots = sm_count();
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= max_split; ++s) {
+    const int64_t n = units * s;
+    const double eff = (double)n / (double)(cdiv(n, slots) * slots);
+    if (eff >= 0.95) return s;
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
 constexpr size_t kSpmmSmemCap = 220 * 1024;
 
 template <typename T>
@@ -173,6 +192,9 @@ __global__ void __launch_bounds__(kSpmmThreads)
   int32_t *s_ptr = reinterpret_cast<int32_t *>(smem_raw + (size_t)W_in * TT * sizeof(Tin));
   const int nnz = (int)nnz64;
   const int64_t t0 = (int64_t)blockIdx.x * TT;
+  // this CTA's share of the segments (blockIdx.y of gridDim.y equal parts)
+  const int s_begin = (int)((int64_t)blockIdx.y * n_seg / gridDim.y);
+  const int s_end = (int)((int64_t)(blockIdx.y + 1) * n_seg / gridDim.y);
   for (int i = threadIdx.x; i <= n_seg; i += kSpmmThreads) {
     const int v = seg_ptr[i];
     s_ptr[i] = v < 0 ? 0 : (v > nnz ? nnz : v);
@@ -184,8 +206,8 @@ __global__ void __launch_bounds__(kSpmmThreads)
   const int q = lane % Q, slot = lane / Q;
   const Tin *s_q = s_in + G * q;
 
-  int seg = warp, pos = 0, end = 0;
-  if (seg < n_seg) {
+  int seg = s_begin + warp, pos = 0, end = 0;
+  if (seg < s_end) {
     pos = s_ptr[seg];
     end = s_ptr[seg + 1];
   }
@@ -212,12 +234,12 @@ __global__ void __launch_bounds__(kSpmmThreads)
     const bool last_of_seg = npos >= end;
     if (last_of_seg) {
       nseg = seg + kWarps;
-      if (nseg < n_seg) {
+      if (nseg < s_end) {
         npos = s_ptr[nseg];
         nend = s_ptr[nseg + 1];
       }
     }
-    if (nseg < n_seg) load_block(npos, nend, kn, vn);
+    if (nseg < s_end) load_block(npos, nend, kn, vn);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const bool ok = (unsigned)kc[u] < (unsigned)W_in;
@@ -258,10 +280,10 @@ __global__ void __launch_bounds__(kSpmmThreads)
     pos = npos;
     end = nend;
   };
-  if (seg < n_seg) load_block(pos, end, ka, va);
-  while (seg < n_seg) {
+  if (seg < s_end) load_block(pos, end, ka, va);
+  while (seg < s_end) {
     step(ka, va, kb, vb);
-    if (seg >= n_seg) break;
+    if (seg >= s_end) break;
     step(kb, vb, ka, va);
   }
 }
@@ -273,8 +295,10 @@ cudaError_t run_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr
   auto k = seg_spmm_kernel<Tin, Tout, TT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = cdiv(T, TT);
-  k<<<(unsigned)grid, kSpmmThreads, smem, s>>>(static_cast<const Tin *>(in), T, W_in, seg_ptr, idx, val, nnz, n_seg,
+  const int64_t tiles = cdiv(T, TT);
+  // one CTA per SM: split the segments so that the token tiles fill whole waves
+  const dim3 grid((unsigned)tiles, (unsigned)wave_split(tiles, n_seg >= 4 * kSpmmThreads / 32 ? 4 : 1));
+  k<<<grid, kSpmmThreads, smem, s>>>(static_cast<const Tin *>(in), T, W_in, seg_ptr, idx, val, nnz, n_seg,
                                               alpha, static_cast<Tout *>(out));
   return cudaGetLastError();
 }
@@ -513,12 +537,28 @@ cudaError_t launch_permute(const float *src, const int32_t *perm, int64_t p, flo
 }
 
 int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in) {
+  // at least two waves of CTAs (one per SM), the last one nearly full
   const int64_t tiles = cdiv(d_out, QWHA_TILE) * cdiv(d_in, QWHA_TILE);
-  int64_t want = cdiv(2 * (int64_t)sm_count(), tiles);
   const int64_t max_by_tokens = cdiv(T, 32);
-  if (want > max_by_tokens) want = max_by_tokens;
-  if (want > kSddmmMaxChunks) want = kSddmmMaxChunks;
-  if (want < 1) want = 1;
+  int64_t cap = kSddmmMaxChunks < max_by_tokens ? kSddmmMaxChunks : max_by_tokens;
+  if (cap < 1) cap = 1;
+  int64_t lo = cdiv(2 * (int64_t)sm_count(), tiles);
+  if (lo > cap) lo = cap;
+  if (lo < 1) lo = 1;
+  int64_t want = lo;
+  double best = -1.0;
+  for (int64_t c = lo; c <= cap; ++c) {
+    const int64_t n = tiles * c, slots = sm_count();
+    const double eff = (double)n / (double)(cdiv(n, slots) * slots);
+    if (eff >= 0.95) {
+      want = c;
+      break;
+    }
+    if (eff > best + 1e-9) {
+      best = eff;
+      want = c;
+    }
+  }
   return (int)want;
 }
 
