@@ -55,6 +55,8 @@ constexpr int kGemmThreads = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int kEpiStride = 33;  // per-warp staging row (floats) of the sampled epilogue
 constexpr size_t kEpiSmem = 4 * 32 * kEpiStride * sizeof(float);
+// bf16 output: each epilogue warp stages its 32 x 32 block (2 KB) before the coalesced stores
+constexpr size_t kEpiBf16Smem = 4 * 2048;
 
 enum { kOutBf16 = 0, kOutF32 = 1, kOutSampled = 2 };
 
@@ -76,7 +78,7 @@ struct Cfg {
   static constexpr int kBRows = BN / CG;  // rows of B this CTA loads
   static constexpr uint32_t kBBytes = kBRows * BK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr size_t kEpiBytes = kMode == kOutSampled ? kEpiSmem : 0;
+  static constexpr size_t kEpiBytes = kMode == kOutSampled ? kEpiSmem : (kMode == kOutBf16 ? kEpiBf16Smem : 0);
   static constexpr size_t kZOffset = (size_t)kStages * kStageBytes + 256 + kEpiBytes;  // from the aligned base
   static constexpr size_t kSmem = kZOffset + 1024 + z_smem<kZ>();
   static constexpr int kThreads = kGemmThreads + (kZ ? kZThreads : 0);
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     // ------------------------------------------------ epilogue (every CTA)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int it = 0;
-    float *my_stage = epi_stage + (warp - 2) * 32 * kEpiStride;
+    float *my_stage = epi_stage + (warp - 2) * (kMode == kOutSampled ? 32 * kEpiStride : 512);
     for (int unit = group_id; unit < num_units; unit += n_groups, ++it) {
       const int tile = unit / k_splits;
       const int buf = it & 1;
@@ -518,6 +520,31 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
             }
           }
           __syncwarp();
+          continue;
+        }
+        if (kMode == kOutBf16 && !addend && col0 + 32 <= N) {
+          // Through shared memory, so that a store instruction writes 8 rows x 64 B
+          // (whole sectors) rather than 32 rows x 16 B. Rows are 64 B apart and the
+          // 16-byte segment s of row r sits at s ^ ((r >> 1) & 3): both the
+          // row-per-lane writes and the transposed reads are free of bank conflicts.
+          unsigned char *st = reinterpret_cast<unsigned char *>(my_stage);
+          float f[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4 *>(st + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4)) =
+                io<__nv_bfloat16>::pack(f + 8 * v);
+          __syncwarp();
+          const int row0 = row - lane;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int rr = 8 * v + (lane >> 2), sg = lane & 3;
+            const uint4 w = *reinterpret_cast<const uint4 *>(st + rr * 64 + ((sg ^ ((rr >> 1) & 3)) << 4));
+            if (row0 + rr < M)
+              *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out_v) + (int64_t)(row0 + rr) * N + col0 + 8 * sg) = w;
+          }
+          __syncwarp();  // the next chunk reuses the staging
           continue;
         }
         if (row < M && col0 < N) {
