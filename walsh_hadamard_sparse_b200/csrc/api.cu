@@ -326,9 +326,13 @@ qwha_status check_ws(void *ws, size_t ws_bytes, size_t need) {
   return QWHA_OK;
 }
 
-size_t fwd_ws(int32_t d_out, int32_t d_in, int64_t T, bool base) {
-  if (!base) return 0;
-  return align_up((size_t)T * d_out * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
+// packed (index, value) entries of the SpMM in gather order
+size_t ent_bytes(int64_t p) { return align_up((size_t)(p > 0 ? p : 1) * 8, 256); }
+
+size_t fwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
+  const size_t n = ent_bytes(p);
+  if (!base) return n;
+  return n + align_up((size_t)T * d_out * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
 }
 
 size_t fwd_dense_ws(int32_t d_out, int32_t d_in) { return align_up((size_t)d_out * d_in * 2, 256); }
@@ -343,7 +347,7 @@ size_t bwd_dense_ws(int32_t d_out, int32_t d_in, int64_t T) {
 size_t bwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
   size_t n = align_up((size_t)kSddmmMaxChunks * (size_t)(p > 0 ? p : 1) * 4, 256);
   n += align_up((size_t)T * d_in * 4, 256);  // dZ
-  n += align_up((size_t)(p > 0 ? p : 1) * 4, 256);  // coefficients in CSC order
+  n += ent_bytes(p);  // CSC entries in gather order
   if (base) n += align_up((size_t)T * d_in * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
   return n;
 }
@@ -390,7 +394,7 @@ int64_t qwha_plan_tiles(int32_t d_out, int32_t d_in) {
 size_t qwha_workspace_size(qwha_op op, int32_t d_out, int32_t d_in, int64_t p, int64_t T, int32_t with_base) {
   if (d_out <= 0 || d_in <= 0 || T < 0 || p < 0) return 0;
   switch (op) {
-    case QWHA_OP_FWD: return fwd_ws(d_out, d_in, T, with_base != 0);
+    case QWHA_OP_FWD: return fwd_ws(d_out, d_in, p, T, with_base != 0);
     case QWHA_OP_BWD: return bwd_ws(d_out, d_in, p, T, with_base != 0);
     case QWHA_OP_INIT: return init_workspace(d_out, d_in);
     case QWHA_OP_PLAN: return plan_workspace(d_out, d_in);
@@ -416,7 +420,7 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   QWHA_CHECK_PTR(Y, "Y");
   const bool dense = a->algo == QWHA_ALGO_DENSE;
   if (dense && dt != QWHA_BF16) return fail(QWHA_ERR_UNSUPPORTED, "the dense algorithm needs dtype bf16");
-  const size_t need = dense ? fwd_dense_ws(a->d_out, a->d_in) : fwd_ws(a->d_out, a->d_in, T, wq != nullptr);
+  const size_t need = dense ? fwd_dense_ws(a->d_out, a->d_in) : fwd_ws(a->d_out, a->d_in, a->p, T, wq != nullptr);
   if ((st = check_ws(ws, ws_bytes, need)) != QWHA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int logn = ilog2(a->had_block);
@@ -478,18 +482,20 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
     e = launch_fwht(dt, dt, X, Z_out, T * (a->d_in / a->had_block), logn, inv, s);
   }
   if (e != cudaSuccess) return cuda_status(e, "fwht");
+  Carver cv(ws);
+  int2 *ent = static_cast<int2 *>(cv.take(ent_bytes(a->p)));
   if (!wq) {
-    StageScope sc(ST_SPMM_FWD, 1, s);
-    e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, a->p, a->d_out, alpha, Y, s);
+    StageScope sc(ST_SPMM_FWD, 2, s);
+    e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out, alpha,
+                        ent, Y, s);
     return cuda_status(e, "spmm");
   }
-  Carver cv(ws);
   float *y_ad = static_cast<float *>(cv.take((size_t)T * a->d_out * 4));
   void *wdeq = cv.take(wdeq_bytes(a->d_out, a->d_in));
   {
-    StageScope sc(ST_SPMM_FWD, 1, s);
-    e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, a->p, a->d_out, alpha,
-                        y_ad, s);
+    StageScope sc(ST_SPMM_FWD, 2, s);
+    e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
+                        alpha, ent, y_ad, s);
   }
   if (e != cudaSuccess) return cuda_status(e, "spmm");
   {
@@ -525,7 +531,7 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   Carver cv(ws);
   float *partial = static_cast<float *>(cv.take((size_t)kSddmmMaxChunks * (size_t)(a->p > 0 ? a->p : 1) * 4));
   float *dz = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
-  float *coef_csc = static_cast<float *>(cv.take((size_t)(a->p > 0 ? a->p : 1) * 4));
+  int2 *ent = static_cast<int2 *>(cv.take(ent_bytes(a->p)));
   cudaError_t e = cudaSuccess;
   if (dc) {
     StageScope sc(ST_SDDMM, 2, s);
@@ -536,10 +542,8 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   if (!dX || T == 0) return QWHA_OK;
   {
     StageScope sc(ST_GATHER_BWD, 2, s);
-    e = launch_permute(a->coef, a->perm, a->p, coef_csc, s);
-    if (e == cudaSuccess)
-      e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, coef_csc, a->p, a->d_in, alpha, dz,
-                          s);
+    e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, a->coef, a->perm, a->p, a->d_in, alpha,
+                        ent, dz, s);
   }
   if (e != cudaSuccess) return cuda_status(e, "gather");
   const int logn = ilog2(a->had_block);

@@ -27,13 +27,12 @@ namespace qwha {
 // partial sums take kSddmmMaxChunks * p floats of workspace at most).
 constexpr int kSddmmMaxChunks = 16;
 
-// out[t, i] = alpha * sum_{j in [seg_ptr[i], seg_ptr[i+1])} val[j] * in[t, idx[j]]
+// out[t, i] = alpha * sum_{j in [seg_ptr[i], seg_ptr[i+1])} v_j * in[t, idx[j]], with
+// v_j = val[perm[j]] when perm is given (the CSC view), else val[j]. ent is
+// scratch for max(nnz, 1) packed (index, value) entries (8-byte aligned).
 cudaError_t launch_seg_spmm(qwha_dtype din, qwha_dtype dout, const void *in, int64_t T, int W_in,
-                            const int32_t *seg_ptr, const int32_t *idx, const float *val, int64_t nnz, int n_seg,
-                            float alpha, void *out, cudaStream_t s);
-
-// dst[q] = src[perm[q]]
-cudaError_t launch_permute(const float *src, const int32_t *perm, int64_t p, float *dst, cudaStream_t s);
+                            const int32_t *seg_ptr, const int32_t *idx, const float *val, const int32_t *perm,
+                            int64_t nnz, int n_seg, float alpha, int2 *ent, void *out, cudaStream_t s);
 
 int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in);
 

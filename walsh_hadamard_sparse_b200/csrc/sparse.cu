@@ -7,8 +7,11 @@
 //   One CTA owns TT tokens: their input rows are staged transposed in shared
 //   memory as s_in[k][TT] (a column of the tile is TT contiguous values), then
 //   each warp runs one segment at a time (see seg_spmm_kernel). The segment
-//   arrays stream from L2 once per token tile. The backward passes the
-//   coefficients already permuted to CSC order (permute_kernel).
+//   entries stream from L2 once per token tile, as packed (index, value)
+//   words that arrange_kernel writes first: it orders each segment so that
+//   the rows one shared-memory wavefront gathers sit on distinct banks as far
+//   as the indices allow, and for the backward applies the CSC permutation
+//   to the coefficients.
 //
 // sddmm: partial[c, j] = sum_{t in chunk c} dY[t, r_j] * Z[t, k_j] over the
 //   tile view of E (QWHA_TILE x QWHA_TILE blocks of F). Grid = tiles x token
@@ -28,7 +31,7 @@
 namespace qwha {
 namespace {
 
-constexpr int kSpmmThreads = 512;
+constexpr int kSpmmThreads = 1024;
 
 // For a kernel that runs one CTA per SM over `units` independent CTAs: the
 // smallest factor s <= max_split by which to subdivide each unit so that the
@@ -131,6 +134,83 @@ __device__ __forceinline__ void stage_transposed(const T *__restrict__ in, int64
   (void)W;
 }
 
+// Gather order. The SpMM stages the token tile transposed, one row of
+// R = TT * sizeof(Tin) bytes per input column (32 bytes for 16 bf16 tokens),
+// so a 128-byte bank line holds M = 128 / R rows and column k lands at line
+// position k mod M. One shared-memory wavefront of the gather serves the
+// lanes of M consecutive entries of a segment (counted from the segment
+// start): two of them with equal k mod M and different k are a bank
+// conflict. arrange_kernel (one warp per segment) orders the entries by
+// (rank within their residue class, residue), round robin over the classes:
+// an aligned group of M entries then holds M distinct residues until the
+// smaller classes run out. The entry of residue m and rank q goes to
+//   start + sum_m' min(cnt[m'], q) + #{m' < m : cnt[m'] > q},
+// a bijection onto the segment. It writes (index, value bits) pairs, the
+// value taken through perm when there is one. The order only changes the
+// fp32 summation order, and it depends on E and R alone (not on T), so the
+// results are repeatable.
+template <int M>
+__global__ void __launch_bounds__(256)
+    arrange_kernel(const int32_t *__restrict__ seg_ptr, int n_seg, const int32_t *__restrict__ idx,
+                   const float *__restrict__ val, const int32_t *__restrict__ perm, int64_t nnz64,
+                   int2 *__restrict__ ent) {
+  static_assert(M >= 1 && M <= 32 && (M & (M - 1)) == 0, "residue classes");
+  const int lane = threadIdx.x & 31;
+  const int nnz = (int)nnz64;
+  const unsigned below = (1u << lane) - 1u;
+  const int warps = (int)gridDim.x * (int)(blockDim.x >> 5);
+  for (int seg = (int)blockIdx.x * (int)(blockDim.x >> 5) + (int)(threadIdx.x >> 5); seg < n_seg;
+       seg += warps) {
+    // the segment as the SpMM reads it: both ends clamped to [0, nnz]
+    int s = seg_ptr[seg], e = seg_ptr[seg + 1];
+    s = s < 0 ? 0 : (s > nnz ? nnz : s);
+    e = e < s ? s : (e > nnz ? nnz : e);
+    int cnt[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) cnt[m] = 0;
+    for (int j = s + lane; j < e; j += 32) {
+      const int r = __ldg(idx + j) & (M - 1);
+#pragma unroll
+      for (int m = 0; m < M; ++m) cnt[m] += r == m ? 1 : 0;
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) cnt[m] += __shfl_xor_sync(0xffffffffu, cnt[m], off);
+    int run[M];  // entries of each class in earlier 32-entry chunks
+#pragma unroll
+    for (int m = 0; m < M; ++m) run[m] = 0;
+    for (int b = s; b < e; b += 32) {
+      const int j = b + lane;
+      int k = 0, r = -1;
+      float v = 0.f;
+      if (j < e) {
+        k = __ldg(idx + j);
+        r = k & (M - 1);
+        if (perm) {
+          const int32_t src = __ldg(perm + j);
+          v = (unsigned)src < (unsigned)nnz ? __ldg(val + src) : 0.f;
+        } else {
+          v = __ldg(val + j);
+        }
+      }
+      int q = 0;
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const unsigned bal = __ballot_sync(0xffffffffu, r == m);
+        if (r == m) q = run[m] + __popc(bal & below);
+        run[m] += __popc(bal);
+      }
+      if (j < e) {
+        int pos = s;
+#pragma unroll
+        for (int m = 0; m < M; ++m) pos += (cnt[m] < q ? cnt[m] : q) + (m < r && cnt[m] > q ? 1 : 0);
+        ent[pos] = make_int2(k, __float_as_int(v));
+      }
+    }
+  }
+}
+
 // One warp per segment at a time. A lane holds G = min(TT, 8) consecutive
 // tokens of the tile (Q = TT/G lanes cover it) for one of NSLOT = 32/Q nonzero
 // slots: lane = q + Q * slot. A segment is cut into blocks of NSLOT * kUnroll
@@ -140,7 +220,9 @@ __device__ __forceinline__ void stage_transposed(const T *__restrict__ in, int64
 // the current block is multiplied (the two sets alternate roles: no copies).
 // bf16 tiles multiply with fma.rn.f32.bf16 (coefficient rounded to bf16, exact
 // product, fp32 accumulation). At a segment's end a reduce-scatter over the
-// slots leaves each token's sum in one lane, which writes it.
+// slots leaves each token's sum in one lane, which writes it. The shared
+// loads and products of a step u whose slots all lie past the segment end
+// are skipped (a warp-uniform test).
 constexpr int kUnroll = 8;
 
 // acc[i] += v * row[i] for the G tokens (4 or 8) a lane holds.
@@ -178,8 +260,8 @@ __device__ __forceinline__ void mac_tokens(const float *row, float v, float *acc
 template <typename Tin, typename Tout, int TT>
 __global__ void __launch_bounds__(kSpmmThreads)
     seg_spmm_kernel(const Tin *__restrict__ in, int64_t T, int W_in, const int32_t *__restrict__ seg_ptr,
-                    const int32_t *__restrict__ idx, const float *__restrict__ val, int64_t nnz64, int n_seg,
-                    float alpha, Tout *__restrict__ out) {
+                    const int2 *__restrict__ ent, int64_t nnz64, int n_seg, float alpha,
+                    Tout *__restrict__ out) {
   static_assert(TT == 4 || TT == 8 || TT == 16, "token tile");
   constexpr int G = TT < 8 ? TT : 8;  // tokens per lane
   constexpr int LV = G == 8 ? 3 : 2;  // reduce-scatter levels (log2 G)
@@ -218,8 +300,9 @@ __global__ void __launch_bounds__(kSpmmThreads)
       kk[u] = W_in;  // marks "no entry"
       vv[u] = 0.f;
       if (j < e) {
-        kk[u] = __ldg(idx + j);
-        vv[u] = __ldg(val + j);
+        const int2 w = __ldg(ent + j);
+        kk[u] = w.x;
+        vv[u] = __int_as_float(w.y);
       }
     }
   };
@@ -242,6 +325,7 @@ __global__ void __launch_bounds__(kSpmmThreads)
     if (nseg < s_end) load_block(npos, nend, kn, vn);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
+      if (pos + NSLOT * u >= end) break;  // no slot of this or later u holds an entry (warp-uniform)
       const bool ok = (unsigned)kc[u] < (unsigned)W_in;
       mac_tokens<G>(s_q + (ok ? kc[u] : 0) * TT, ok ? vc[u] : 0.f, acc);
     }
@@ -290,7 +374,15 @@ __global__ void __launch_bounds__(kSpmmThreads)
 
 template <typename Tin, typename Tout, int TT>
 cudaError_t run_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
-                     const float *val, int64_t nnz, int n_seg, float alpha, void *out, cudaStream_t s) {
+                     const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha, int2 *ent,
+                     void *out, cudaStream_t s) {
+  constexpr int M = 128 / (TT * (int)sizeof(Tin));  // staged rows per bank line
+  {
+    const int64_t grid = std::min<int64_t>(cdiv(n_seg, 256 / 32), (int64_t)sm_count() * 8);
+    arrange_kernel<M><<<(unsigned)grid, 256, 0, s>>>(seg_ptr, n_seg, idx, val, perm, nnz, ent);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const size_t smem = (size_t)W_in * TT * sizeof(Tin) + ((size_t)n_seg + 1) * sizeof(int32_t);
   auto k = seg_spmm_kernel<Tin, Tout, TT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -298,32 +390,25 @@ cudaError_t run_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr
   const int64_t tiles = cdiv(T, TT);
   // one CTA per SM: split the segments so that the token tiles fill whole waves
   const dim3 grid((unsigned)tiles, (unsigned)wave_split(tiles, n_seg >= 4 * kSpmmThreads / 32 ? 4 : 1));
-  k<<<grid, kSpmmThreads, smem, s>>>(static_cast<const Tin *>(in), T, W_in, seg_ptr, idx, val, nnz, n_seg,
-                                              alpha, static_cast<Tout *>(out));
+  k<<<grid, kSpmmThreads, smem, s>>>(static_cast<const Tin *>(in), T, W_in, seg_ptr, ent, nnz, n_seg, alpha,
+                                     static_cast<Tout *>(out));
   return cudaGetLastError();
 }
 
 template <typename Tin, typename Tout>
 cudaError_t pick_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
-                      const float *val, int64_t nnz, int n_seg, float alpha, void *out, cudaStream_t s) {
+                      const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha, int2 *ent,
+                      void *out, cudaStream_t s) {
   const size_t row = (size_t)W_in * sizeof(Tin);
   const size_t ptrs = ((size_t)n_seg + 1) * sizeof(int32_t);
   const size_t cap = kSpmmSmemCap > ptrs ? kSpmmSmemCap - ptrs : 0;
   if (row * 16 <= cap)
-    return run_spmm<Tin, Tout, 16>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
+    return run_spmm<Tin, Tout, 16>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
   if (row * 8 <= cap)
-    return run_spmm<Tin, Tout, 8>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
+    return run_spmm<Tin, Tout, 8>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
   if (row * 4 <= cap)
-    return run_spmm<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
+    return run_spmm<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
   return cudaErrorInvalidValue;  // rows too long for one staged token tile
-}
-
-__global__ void permute_kernel(const float *__restrict__ src, const int32_t *__restrict__ perm, int64_t p,
-                               float *__restrict__ dst) {
-  for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < p; q += (int64_t)gridDim.x * blockDim.x) {
-    const int32_t j = perm[q];
-    dst[q] = (uint64_t)j < (uint64_t)p ? src[j] : 0.f;
-  }
 }
 
 // ---------------------------------------------------------------- SDDMM
@@ -517,23 +602,19 @@ __global__ void sddmm_reduce_kernel(const float *__restrict__ partial, int n_chu
 }  // namespace
 
 cudaError_t launch_seg_spmm(qwha_dtype din, qwha_dtype dout, const void *in, int64_t T, int W_in,
-                            const int32_t *seg_ptr, const int32_t *idx, const float *val, int64_t nnz, int n_seg,
-                            float alpha, void *out, cudaStream_t s) {
+                            const int32_t *seg_ptr, const int32_t *idx, const float *val, const int32_t *perm,
+                            int64_t nnz, int n_seg, float alpha, int2 *ent, void *out, cudaStream_t s) {
   if (T <= 0 || n_seg <= 0) return cudaSuccess;
+  if (reinterpret_cast<uintptr_t>(ent) & 7) return cudaErrorMisalignedAddress;
   using bf = __nv_bfloat16;
   if (din == QWHA_BF16) {
-    if (dout == QWHA_BF16) return pick_spmm<bf, bf>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
-    return pick_spmm<bf, float>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
+    if (dout == QWHA_BF16)
+      return pick_spmm<bf, bf>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
+    return pick_spmm<bf, float>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
   }
-  if (dout == QWHA_BF16) return pick_spmm<float, bf>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
-  return pick_spmm<float, float>(in, T, W_in, seg_ptr, idx, val, nnz, n_seg, alpha, out, s);
-}
-
-cudaError_t launch_permute(const float *src, const int32_t *perm, int64_t p, float *dst, cudaStream_t s) {
-  if (p <= 0) return cudaSuccess;
-  const int64_t grid = std::min<int64_t>(cdiv(p, 256), (int64_t)sm_count() * 8);
-  permute_kernel<<<(unsigned)grid, 256, 0, s>>>(src, perm, p, dst);
-  return cudaGetLastError();
+  if (dout == QWHA_BF16)
+    return pick_spmm<float, bf>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
+  return pick_spmm<float, float>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
 }
 
 int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in) {
