@@ -79,3 +79,22 @@ def test_host_checks_of_init_variants_and_refinement():
     assert h.qwha_init_budgets(dummy, 4, 8, 4, 2, 0, dummy, dummy, dummy, 1 << 20, None) == 1  # p < 2 * d_out
     assert h.qwha_init_select(dummy, 4, 96, 64, dummy, dummy, 8, dummy, dummy, None) == 1  # 64 does not divide 96
     assert h.qwha_workspace_size(7, 64, 64, 100, 0, 0) > 0 and h.qwha_workspace_size(6, 64, 64, 100, 0, 0) > 0
+
+
+def test_sparse_forward_needs_entry_workspace():
+    """The sparse products write their (index, value) pairs, ordered for the shared-memory gather, into the caller's
+    workspace (8 bytes per coefficient), so the adapter-only sparse forward needs a workspace too; without one it is
+    refused on the host, before any CUDA call (no GPU needed)."""
+    _ensure_built()
+    import walsh_hadamard_sparse_b200._lib as L
+
+    h = L.lib()
+    d, p, T = 64, 100, 16
+    need = h.qwha_workspace_size(0, d, d, p, T, 0)  # QWHA_OP_FWD, adapter only
+    assert need >= 8 * p
+    assert h.qwha_workspace_size(0, d, d, p, T, 1) >= need + 4 * T * d  # plus the fp32 adapter term
+    assert h.qwha_workspace_size(1, d, d, p, T, 0) >= 8 * p + 4 * T * d  # QWHA_OP_BWD: entries and dZ
+    a = L.QwhaAdapter(d_in=d, d_out=d, had_block=d, algo=0, p=p, row_ptr=4096, col_idx=8192, coef=12288)
+    buf = ctypes.c_void_p(16384)
+    rc = h.qwha_adapter_fwd(ctypes.byref(a), None, 1, buf, T, ctypes.c_float(1.0), buf, buf, None, 0, None)
+    assert rc == 4 and b"workspace" in h.qwha_last_error()
