@@ -445,3 +445,27 @@ def test_dense_rejects_fp32():
     with pytest.raises(W.QwhaError) as ei:
         W.adapter_fwd(a, to_dev(L["X"]), 1.0)
     assert ei.value.status == 3
+
+
+@pytest.mark.parametrize("algo", ["sparse", "dense"])
+def test_token_shards_give_the_same_rows_bitwise(algo):
+    """Token data parallelism hands each rank a slice of the step's tokens. The per-token outputs of a slice (Z, Y, dX)
+    are bit for bit the same rows of the whole call, also for slices that start inside a token tile: the sparse
+    products' entry order depends on E alone and every token is summed in the same order wherever it sits in a tile.
+    Only dc, a sum over tokens, is split across ranks."""
+    import torch
+
+    W = _W()
+    d_in, d_out, n, T = 1024, 768, 1024, 300
+    L = synth_layer(39, d_in, d_out, n, T, d_out * 8, "bf16", bits=4, group=128)
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"], algo=algo)
+    wq = dev_qweight(L)
+    Xd, dYd = dev_act(L["X"], "bf16"), dev_act(L["dY"], "bf16")
+    Z, Y = W.adapter_fwd(a, Xd, 0.8, wq=wq)
+    _, dX = W.adapter_bwd(a, dYd, Z, 0.8, wq=wq, want_dc=False)
+    for lo, hi in ((0, 129), (129, 300)):
+        Zs, Ys = W.adapter_fwd(a, Xd[lo:hi].contiguous(), 0.8, wq=wq)
+        _, dXs = W.adapter_bwd(a, dYd[lo:hi].contiguous(), Zs, 0.8, wq=wq, want_dc=False)
+        torch.cuda.synchronize()
+        for name, part, whole in (("Z", Zs, Z), ("Y", Ys, Y), ("dX", dXs, dX)):
+            assert torch.equal(part.view(torch.int16), whole[lo:hi].view(torch.int16)), (name, lo, hi)
