@@ -65,6 +65,8 @@ def _load():
                 "oracle_init_select_global": [P, i32, i32, i32, i64, i32, ctypes.c_uint64, P, P, P, P],
                 "oracle_refine_values": [P, i32, i32, i32, P, f64, P, P, i32, P, P],
                 "oracle_plan_build": [i32, i32, i64, P, P, P, P, P],
+                "oracle_pattern_stats": [i32, i32, i64, P, P, P, P],
+                "oracle_energy_stats": [P, i32, i32, i32, i64, P],
             }
             for name, args in sig.items():
                 fn = getattr(lib, name)
@@ -281,3 +283,38 @@ def plan_build(row_ptr, col_idx, d_in: int):
     pm = np.empty(p, dtype=np.int32)
     _check(_load().oracle_plan_build(d_out, d_in, p, _p(rp), _p(ci), _p(cp), _p(ri), _p(pm)), "plan_build")
     return cp, ri, pm
+
+
+PATTERN_STATS = ("empty_rows", "empty_cols", "min_row", "max_row", "min_col", "max_col", "rank_bound", "half_rows")
+
+
+def pattern_stats(row_ptr, col_idx, d_in: int) -> dict:
+    """Counts of E by row and column (the rank argument of the pages): dict of PATTERN_STATS plus col_counts."""
+    rp, ci = _i32(row_ptr), _i32(col_idx)
+    d_out = rp.size - 1
+    cc = np.empty(d_in, dtype=np.int32)
+    st = np.empty(8, dtype=np.int64)
+    _check(_load().oracle_pattern_stats(d_out, d_in, ci.size, _p(rp), _p(ci), _p(cc), _p(st)), "pattern_stats")
+    out = {k: int(v) for k, v in zip(PATTERN_STATS, st)}
+    out["col_counts"] = cc
+    return out
+
+
+def numerical_rank(row_ptr, col_idx, coef, d_in: int) -> int:
+    """rank(F) of F = Scatter(c, E) [d_out, d_in] in fp64 (numpy's SVD-based matrix_rank with its default
+    tolerance); for the small shapes of the tests."""
+    rp, ci = _i32(row_ptr), _i32(col_idx)
+    d_out = rp.size - 1
+    F = np.zeros((d_out, d_in), dtype=np.float64)
+    F[np.repeat(np.arange(d_out), np.diff(rp)), ci] = _f64(coef)
+    return int(np.linalg.matrix_rank(F))
+
+
+def energy_stats(dWq, k: int, n: int) -> dict:
+    """Hill exponent eta and cumulative energy of the k largest transform coefficients |dW_Q H| (see
+    oracle_energy_stats): dict(eta, energy, threshold, total)."""
+    w = np.ascontiguousarray(dWq, dtype=np.float32)
+    d_out, d_in = w.shape
+    out = np.empty(4, dtype=np.float64)
+    _check(_load().oracle_energy_stats(_p(w), d_out, d_in, n, int(k), _p(out)), "energy_stats")
+    return dict(eta=float(out[0]), energy=float(out[1]), threshold=float(out[2]), total=float(out[3]))

@@ -607,6 +607,98 @@ int oracle_refine_values(const float *dWq, int32_t d_out, int32_t d_in, int32_t 
   return status;
 }
 
+// Diagnostics of the selection (the pages' argument for AdaAlloc).
+//
+// [P1 设计1]: F = Scatter(c, E) is full rank with high probability once every
+// row and every column holds more than two nonzeros on average, and rank(dW) =
+// rank(F) because H is orthogonal. [P1 设计2; P2 2.2]: choosing E by magnitude
+// over the whole matrix crowds the parameters into the few channels that hold
+// outliers, and F degenerates to low rank. A row or a column of F without any
+// entry cannot add to the rank, so rank(F) <= min(non-empty rows, non-empty
+// columns); the numerical rank itself is computed in the Python wrapper.
+// stats (8 entries):
+//   [0] rows without entries        [1] columns without entries
+//   [2] fewest entries in a row     [3] most entries in a row
+//   [4] fewest entries in a column  [5] most entries in a column
+//   [6] min(d_out - [0], d_in - [1])
+//   [7] the fewest rows that together hold at least ceil(p / 2) entries
+// col_counts [d_in] receives the entries of every column.
+int oracle_pattern_stats(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr, const int32_t *col_idx,
+                         int32_t *col_counts, int64_t *stats) {
+  if (d_out <= 0 || d_in <= 0 || p < 0 || row_ptr[0] != 0 || row_ptr[d_out] != p) return 1;
+  std::vector<int64_t> rows((size_t)d_out);
+  for (int i = 0; i < d_out; ++i) {
+    rows[i] = (int64_t)row_ptr[i + 1] - row_ptr[i];
+    if (rows[i] < 0) return 1;
+  }
+  for (int k = 0; k < d_in; ++k) col_counts[k] = 0;
+  for (int64_t j = 0; j < p; ++j) {
+    if (col_idx[j] < 0 || col_idx[j] >= d_in) return 1;
+    col_counts[col_idx[j]]++;
+  }
+  int64_t empty_r = 0, empty_c = 0;
+  for (int i = 0; i < d_out; ++i) empty_r += rows[i] == 0;
+  for (int k = 0; k < d_in; ++k) empty_c += col_counts[k] == 0;
+  stats[0] = empty_r;
+  stats[1] = empty_c;
+  stats[2] = *std::min_element(rows.begin(), rows.end());
+  stats[3] = *std::max_element(rows.begin(), rows.end());
+  stats[4] = *std::min_element(col_counts, col_counts + d_in);
+  stats[5] = *std::max_element(col_counts, col_counts + d_in);
+  stats[6] = std::min<int64_t>(d_out - empty_r, d_in - empty_c);
+  // the most crowded rows first: how many are needed to reach half the entries
+  std::vector<int64_t> sorted = rows;
+  std::sort(sorted.begin(), sorted.end(), [](int64_t a, int64_t b) { return a > b; });
+  const int64_t half = (p + 1) / 2;
+  int64_t taken = 0, m = 0;
+  while (taken < half) taken += sorted[(size_t)m++];
+  stats[7] = m;
+  return 0;
+}
+
+// Energy concentration of the transform coefficients [P1 设计1, "why the
+// WHT"]: the magnitudes of the coefficients of dW_Q after the transform are
+// fitted with a Pareto law, whose Hill exponent eta measures how steep the
+// tail is (the smaller eta, the more of the error energy sits in few
+// coefficients); with the same number of parameters the transform with the
+// smallest eta reconstructs the most error energy (the cumulative-energy
+// curve). Reading taken (the pages give no formula): a = |V| over all
+// d_out * d_in coefficients, V = dW_Q H_unnormalised (fp64 butterflies, as
+// in AdaAlloc), sorted a_(1) >= a_(2) >= ...; Hill's estimate over the k
+// largest is
+//   xi = (1/k) sum_{i=1..k} ln(a_(i) / a_(k+1)),   eta = 1 / xi
+// (eta is the Pareto tail index; NaN when a_(k+1) = 0 or xi = 0), and the
+// cumulative energy at k is sum_{i<=k} a_(i)^2 / sum_all a^2 (NaN for an
+// all-zero dW_Q). Both are scale-free, so the normalisation of H does not
+// enter. out: [0] eta, [1] energy fraction of the k largest, [2] a_(k+1),
+// [3] sum of all a^2. Requires 1 <= k < d_out * d_in.
+int oracle_energy_stats(const float *dWq, int32_t d_out, int32_t d_in, int32_t n, int64_t k, double *out) {
+  if (!shape_ok(d_in, n) || d_out <= 0) return 1;
+  const int64_t N = (int64_t)d_out * d_in;
+  if (k < 1 || k >= N) return 1;
+  std::vector<double> a((size_t)N);
+  parallel_for(d_out, [&](int64_t i) {
+    double *v = a.data() + i * d_in;
+    for (int c = 0; c < d_in; ++c) v[c] = (double)dWq[i * d_in + c];
+    for (int blk = 0; blk < d_in / n; ++blk) butterflies(v + (int64_t)blk * n, n);
+    for (int c = 0; c < d_in; ++c) v[c] = std::fabs(v[c]);
+  });
+  std::sort(a.begin(), a.end(), [](double x, double y) { return x > y; });
+  const double thr = a[(size_t)k];  // a_(k+1), zero-based
+  double hill = 0.0, top = 0.0, all = 0.0;
+  for (int64_t i = 0; i < k; ++i) {
+    hill += std::log(a[(size_t)i] / thr);
+    top += a[(size_t)i] * a[(size_t)i];
+  }
+  for (int64_t i = 0; i < N; ++i) all += a[(size_t)i] * a[(size_t)i];
+  const double xi = hill / (double)k;
+  out[0] = (thr > 0.0 && xi > 0.0) ? 1.0 / xi : NAN;
+  out[1] = all > 0.0 ? top / all : NAN;
+  out[2] = thr;
+  out[3] = all;
+  return 0;
+}
+
 // Column view of the CSR pattern: for every column k the nonzeros j with
 // col_idx[j] == k, in increasing j: col_ptr [d_in+1], row_idx [p] (their rows),
 // perm [p] (their CSR positions).

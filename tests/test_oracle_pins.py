@@ -439,3 +439,98 @@ def test_refine_never_worse_than_dense_solution():
             r = w[i].astype(np.float64) - x @ H[sel]  # dW_Q[i,:] - (F H^-1)[i,:]
             return r @ S @ r  # || r X^T ||^2
         assert err(got[rp[i]:rp[i + 1]].astype(np.float64)) <= err(e["coef"][rp[i]:rp[i + 1]].astype(np.float64)) + 1e-12
+
+
+# --------------------------------------------------------------------------- selection diagnostics
+
+
+def _csr_from_rows(rows):
+    rp = np.zeros(len(rows) + 1, dtype=np.int32)
+    rp[1:] = np.cumsum([len(r) for r in rows])
+    ci = np.array([k for r in rows for k in r], dtype=np.int32)
+    return rp, ci
+
+
+def test_pattern_stats_golden():
+    """Row and column counts, empty rows and columns, the rank bound and the half-mass row count of a hand-worked
+    pattern; the numerical rank of F with generic coefficients reaches the bound."""
+    g = json.load(open(os.path.join(GOLDEN, "pattern_stats.json")))
+    rp, ci = _csr_from_rows(g["rows"])
+    got = oracle.pattern_stats(rp, ci, g["d_in"])
+    assert list(got["col_counts"]) == g["col_counts"]
+    assert {k: got[k] for k in g["stats"]} == g["stats"]
+    coef = rng_for(80, "pattern-golden").uniform(0.5, 2.0, ci.size)
+    assert oracle.numerical_rank(rp, ci, coef, g["d_in"]) == g["generic_rank"]
+
+
+def test_numerical_rank_of_constructed_patterns():
+    """rank(F) on patterns whose rank is known by construction: a full diagonal, all entries in two rows, two rows
+    with proportional coefficients on the same columns, and a full block with outer-product values (rank 1)."""
+    g = rng_for(81, "rank")
+    d = 12
+    rp, ci = _csr_from_rows([[i] for i in range(d)])
+    assert oracle.numerical_rank(rp, ci, g.uniform(1, 2, d), d) == d
+    rows = [list(range(0, 14, 1)) if i in (2, 7) else [] for i in range(9)]
+    rp, ci = _csr_from_rows(rows)
+    assert oracle.numerical_rank(rp, ci, g.standard_normal(ci.size), 14) == 2
+    base = g.standard_normal(5)
+    rows = [[1, 3, 4, 8, 9], [], [1, 3, 4, 8, 9]]
+    rp, ci = _csr_from_rows(rows)
+    assert oracle.numerical_rank(rp, ci, np.concatenate([base, -2.5 * base]), 10) == 1
+    u, v = g.uniform(1, 2, 4), g.uniform(1, 2, 6)
+    rows = [list(range(6))] * 4
+    rp, ci = _csr_from_rows(rows)
+    assert oracle.numerical_rank(rp, ci, np.outer(u, v).ravel(), 6) == 1
+    # a wide pattern (rows fewer than columns): a transposed scatter would not fit
+    rp, ci = _csr_from_rows([[0, 5], [1, 6], [2, 7]])
+    assert oracle.numerical_rank(rp, ci, np.ones(6), 8) == 3
+
+
+def _spike_rows(d_in, n):
+    """dW_Q whose rows hold one spike each (values 8, 2, 0.5, 0; powers of two, exact in fp32): row r of
+    V = dW_Q H_unnormalised is s_r times a row of the n-point Hadamard block it falls in, so n magnitudes equal |s_r|
+    and the other d_in - n are zero."""
+    w = np.zeros((4, d_in), dtype=np.float32)
+    for r, (s, k) in enumerate(((8.0, 3), (2.0, 10), (0.5, 6), (0.0, 0))):
+        w[r, k] = s
+    return w
+
+
+def test_energy_stats_closed_form():
+    """Hill exponent and cumulative energy where the order statistics are known exactly (spike rows), for the
+    full transform and for a block-diagonal one: eta = k / sum_{i<=k} ln(a_(i)/a_(k+1)), energy = sum of the k
+    largest a^2 over all, NaN for eta when a_(k+1) = 0."""
+    ln4, ln16 = np.log(4.0), np.log(16.0)
+    w = _spike_rows(16, 16)  # magnitudes: 16 x 8, 16 x 2, 16 x 0.5, 16 x 0; total 16 * 68.25 = 1092
+    cases = {
+        16: (1.0 / ln4, 1024.0 / 1092, 2.0),
+        20: (20.0 / (16 * ln4), 1040.0 / 1092, 2.0),
+        40: (40.0 / (16 * ln16 + 16 * ln4), 1090.0 / 1092, 0.5),
+        50: (np.nan, 1092.0 / 1092, 0.0),
+    }
+    for k, (eta, energy, thr) in cases.items():
+        got = oracle.energy_stats(w, k, 16)
+        assert got["threshold"] == thr and got["total"] == 1092.0, k
+        assert np.isclose(got["energy"], energy, rtol=1e-14), k
+        assert (np.isnan(got["eta"]) and np.isnan(eta)) or np.isclose(got["eta"], eta, rtol=1e-14), k
+    # two blocks of 8: each spike fills only its own block (8 magnitudes |s_r|, the other 8 of the row zero)
+    got = oracle.energy_stats(_spike_rows(16, 8), 8, 8)
+    assert got["threshold"] == 2.0 and got["total"] == 8 * 68.25
+    assert np.isclose(got["eta"], 1.0 / ln4, rtol=1e-14) and np.isclose(got["energy"], 64.0 / 68.25, rtol=1e-14)
+
+
+def test_energy_stats_recovers_a_pareto_tail_index():
+    """Coefficients drawn from a Pareto law of tail index 1.5 (random signs), mapped back to dW_Q through the
+    library-independent Hadamard matrix: the Hill exponent over the 2000 largest of 65536 is within a few standard
+    errors (1.5 / sqrt(2000) = 0.034) of 1.5. A reciprocal or a log-base mistake lands far away. The total
+    energy obeys Parseval: sum (dW_Q H_unnormalised)^2 = n ||dW_Q||^2."""
+    from scipy.linalg import hadamard
+
+    n, d_out, alpha = 256, 256, 1.5
+    g = rng_for(82, "pareto")
+    V = (1.0 + g.pareto(alpha, (d_out, n))) * g.choice([-1.0, 1.0], (d_out, n))
+    w = (V @ hadamard(n).astype(np.float64) / n).astype(np.float32)  # V = w H_unnormalised (up to fp32 rounding)
+    got = oracle.energy_stats(w, 2000, n)
+    assert abs(got["eta"] - alpha) < 0.15, got
+    assert np.isclose(got["total"], n * np.sum(w.astype(np.float64) ** 2), rtol=1e-12)
+    assert 0.0 < got["energy"] < 1.0
