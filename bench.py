@@ -119,13 +119,31 @@ def stage_work(stage, spec, T, bits, algo="dense"):
     return w.get(stage)
 
 
-def peak_for(kind, peaks):
+SUSTAINED_AFTER_S = 1.0  # timed regions at least this long are compared with the sustained (power-capped) GEMM peak
+
+
+def fp32_fma_tflops(peaks):
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    return 148 * ALU_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+
+
+def peak_for(kind, peaks, region_s=0.0):
+    """(peak, unit, note) for a kernel whose timed region lasted region_s seconds: the burst cuBLAS bf16 figure for
+    regions shorter than SUSTAINED_AFTER_S, the sustained one (a seconds-long loop under the power cap) otherwise."""
     if kind == "hbm":
         return peaks["hbm_gbs"], "GB/s", "HBM copy bandwidth, " + peaks["_source"]
     if kind == "tensor":
-        return peaks["bf16_tflops_sustained"], "TFLOP/s", "cuBLAS bf16 sustained, " + peaks["_source"]
-    mhz = peaks.get("sm_max_mhz", 1965.0)
-    return 148 * ALU_LANES_PER_SM * 2 * mhz * 1e6 / 1e12, "TFLOP/s", "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock"
+        if region_s >= SUSTAINED_AFTER_S:
+            return (peaks["bf16_tflops_sustained"], "TFLOP/s",
+                    f"cuBLAS bf16 sustained ({region_s:.2f} s timed region), " + peaks["_source"])
+        return (peaks["bf16_tflops"], "TFLOP/s",
+                f"cuBLAS bf16 burst ({region_s:.3f} s timed region), " + peaks["_source"])
+    return fp32_fma_tflops(peaks), "TFLOP/s", "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock (derived)"
+
+
+# the method's own work of a stage that the tensor cores do as a larger dense product: the dense dc GEMM computes
+# all d_out x d_in entries of dY^T Z and keeps the p at E, whose sums (2 p T FLOP) are the SDDMM's work
+METHOD_WORK = {"gemm_dc": lambda spec, T: ("alu", 2.0 * spec.p * T)}
 
 
 # --------------------------------------------------------------------------- clocks
@@ -446,14 +464,11 @@ def main():
         ad, (wf, wb) = adapters[algo], ws[algo]
 
         def step():
-            W.adapter_fwd(ad, X, alpha, wq, Z_out=Z, Y=Y, ws=wf)
             if world > 1:
                 # dc first; its all-reduce (the path's one exchange) overlaps the dX computation
-                W.adapter_bwd(ad, dY, Z, alpha, wq, dc=dc, want_dx=False, ws=wb)
-                work = dist.all_reduce(dc, async_op=True)
-                W.adapter_bwd(ad, dY, Z, alpha, wq, dX=dX, want_dc=False, ws=wb)
-                work.wait()
+                W.dp_step(ad, X, dY, alpha, wq, Z=Z, Y=Y, dc=dc, dX=dX, ws_fwd=wf, ws_bwd=wb)
             else:
+                W.adapter_fwd(ad, X, alpha, wq, Z_out=Z, Y=Y, ws=wf)
                 W.adapter_bwd(ad, dY, Z, alpha, wq, dc=dc, dX=dX, ws=wb)
 
         return step
@@ -483,13 +498,14 @@ def main():
         W.stage_timing(False)
         rep = W.stage_report()
         t_ms = sum(s_.elapsed_time(e_) for s_, e_ in zip(starts, ends))
+        span_ms = starts[0].elapsed_time(ends[-1])  # the whole timed region, L2 flushes included
         if world > 1:
-            tt = torch.tensor([t_ms], device=dev)
+            tt = torch.tensor([t_ms, span_ms], device=dev)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t_ms = float(tt.item())
-        return t_ms, rep, clk
+            t_ms, span_ms = float(tt[0].item()), float(tt[1].item())
+        return t_ms, rep, clk, span_ms
 
-    def kernel_table(rep, K, algo):
+    def kernel_table(rep, K, algo, region_s):
         kernels = {}
         for name, (calls, launches, ms) in rep.items():
             if calls == 0:
@@ -499,10 +515,18 @@ def main():
             wk = stage_work(name, spec, T, spec.bits, algo)
             if wk:
                 kind, amount, nbytes = wk
-                peak, unit, _ = peak_for(kind, peaks)
+                peak, unit, note = peak_for(kind, peaks, region_s)
                 ach = amount / (per / 1e3) / (1e9 if unit == "GB/s" else 1e12)
-                k.update(bound=kind, achieved=ach, peak=peak, unit=unit, frac=ach / peak,
-                         alg_GBps=nbytes / (per / 1e3) / 1e9, alg_bytes=nbytes, traffic=ncu_traffic(algo, name))
+                k.update(bound=kind, work=amount, achieved=ach, peak=peak, unit=unit, frac=ach / peak,
+                         peak_source=note, alg_GBps=nbytes / (per / 1e3) / 1e9, alg_bytes=nbytes,
+                         traffic=ncu_traffic(algo, name))
+                if name in METHOD_WORK:
+                    mkind, mwork = METHOD_WORK[name](spec, T)
+                    mpeak, munit, mnote = peak_for(mkind, peaks, region_s)
+                    mach = mwork / (per / 1e3) / 1e12
+                    k["method"] = {"bound": mkind, "work": mwork, "achieved": mach, "peak": mpeak, "unit": munit,
+                                   "frac": mach / mpeak, "peak_source": mnote,
+                                   "what": "2 p T FLOP of the coefficient gradient, against the FP32 FMA roofline"}
             kernels[name] = k
         tot = sum(v["ms_per_call"] * v["calls"] for v in kernels.values())
         for v in kernels.values():
@@ -512,9 +536,12 @@ def main():
     def roofline_of(kernels, algo):
         dom = max((n for n in kernels if "bound" in kernels[n]), key=lambda n: kernels[n]["share"])
         kd = kernels[dom]
-        _, _, note = peak_for(kd["bound"], peaks)
-        return {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
-                "unit": kd["unit"], "frac": kd["frac"], "traffic": ncu_traffic(algo, dom), "peak_source": note}
+        r = {"kernel": dom, "bound": kd["bound"], "achieved": kd["achieved"], "peak": kd["peak"],
+             "unit": kd["unit"], "frac": kd["frac"], "traffic": ncu_traffic(algo, dom), "peak_source": kd["peak_source"],
+             "work_per_launch": kd["work"], "ms_per_call": kd["ms_per_call"]}
+        if "method" in kd:
+            r["method"] = kd["method"]
+        return r
 
     results = {}
     for algo in ("dense", "sparse"):
@@ -525,8 +552,8 @@ def main():
         if not (torch.isfinite(Y.float()).all() and torch.isfinite(dc).all() and torch.isfinite(dX.float()).all()):
             raise RuntimeError(f"non-finite output ({algo})")
         K = args.steps if algo == "dense" else max(3, min(args.steps, args.sparse_steps))
-        t_ms, rep, clk = timed(step, K, algo == "dense")
-        kernels = kernel_table(rep, K, algo)
+        t_ms, rep, clk, span_ms = timed(step, K, algo == "dense")
+        kernels = kernel_table(rep, K, algo, span_ms / 1e3)
         results[algo] = dict(K=K, t_ms=t_ms, value=world * T * K / (t_ms / 1e3), kernels=kernels,
                              roofline=roofline_of(kernels, algo), launches=sum(v[1] for v in rep.values()), clocks=clk)
     head = results["dense"]
@@ -563,13 +590,10 @@ def main():
                     dYb.copy_(dYh, non_blocking=True)
                     ready[b].record(cs)
                 comp.wait_event(ready[b])
-                W.adapter_fwd(ad, Xb, alpha, wq, Z_out=Z, Y=Y, ws=wf)
                 if world > 1:
-                    W.adapter_bwd(ad, dYb, Z, alpha, wq, dc=dc, want_dx=False, ws=wb)
-                    work = dist.all_reduce(dc, async_op=True)
-                    W.adapter_bwd(ad, dYb, Z, alpha, wq, dX=dX, want_dc=False, ws=wb)
-                    work.wait()
+                    W.dp_step(ad, Xb, dYb, alpha, wq, Z=Z, Y=Y, dc=dc, dX=dX, ws_fwd=wf, ws_bwd=wb)
                 else:
+                    W.adapter_fwd(ad, Xb, alpha, wq, Z_out=Z, Y=Y, ws=wf)
                     W.adapter_bwd(ad, dYb, Z, alpha, wq, dc=dc, dX=dX, ws=wb)
                 free[b].record(comp)
                 dch.copy_(dc, non_blocking=True)

@@ -141,7 +141,9 @@ typedef enum {
   QWHA_OP_FWD_DENSE = 4, /* qwha_adapter_fwd, algo dense */
   QWHA_OP_BWD_DENSE = 5, /* qwha_adapter_bwd, algo dense */
   QWHA_OP_SELECT_GLOBAL = 6, /* qwha_init_select_global */
-  QWHA_OP_REFINE = 7         /* qwha_refine_values */
+  QWHA_OP_REFINE = 7,        /* qwha_refine_values */
+  QWHA_OP_ENERGY = 8,        /* qwha_energy_stats */
+  QWHA_OP_PATTERN = 9        /* qwha_pattern_stats */
 } qwha_op;
 
 /* Z = X H row by row: x and z are [rows, n] of dtype dt (device), each row
@@ -249,6 +251,44 @@ qwha_status qwha_init_select_global(const float *dWq, int32_t d_out, int32_t d_i
                                     int32_t *row_ptr, int32_t *col_idx, float *coef, void *ws,
                                     size_t ws_bytes, void *stream);
 
+/* Selection diagnostics: the two measurements the pages use to argue for
+ * the WHT and for AdaAlloc (papernotes.org 关键设计 1 and 2; gist.science
+ * 2.2). Both compute what the pages describe rather than a step of the
+ * training path.
+ *
+ * qwha_energy_stats: energy concentration of the transform coefficients of
+ * the quantization error. The pages fit the coefficient magnitudes with a
+ * Pareto law and compare transforms by its Hill exponent eta (the smaller,
+ * the steeper the tail and the more error energy a fixed number of
+ * coefficients reconstructs); they give no formula, and this library takes
+ * Hill's estimate over the k largest magnitudes a = |V|, V = dWq
+ * H_unnormalised (fp64, as in qwha_init_alloc), sorted a_(1) >= a_(2) >= ...:
+ *   xi = (1/k) sum_{i=1..k} ln(a_(i) / a_(k+1)),  eta = 1 / xi.
+ * stats (device fp64 [4]): [0] eta (NaN when a_(k+1) = 0 or xi = 0), [1] the
+ * fraction of sum a^2 held by the k largest (the cumulative energy at k; NaN
+ * for an all-zero dWq), [2] a_(k+1) (unnormalised), [3] sum a^2
+ * (= had_block * ||dWq||_F^2). dWq fp32 [d_out, d_in]; 1 <= k < d_out * d_in,
+ * k < 2^31, d_in <= 16384. ws: qwha_workspace_size(QWHA_OP_ENERGY, d_out,
+ * d_in, 0, 0, 0) bytes. Deterministic: a fixed-order reduction.
+ *
+ * qwha_pattern_stats: how E spreads over rows and columns. F is full rank with
+ * high probability once rows and columns average more than two entries, and
+ * an empty row or column cannot add to rank(F); a whole-matrix magnitude
+ * selection crowds the entries into a few channels. From the CSR row_ptr
+ * [d_out+1] and col_idx [p] (device) it writes col_counts (device int32
+ * [d_in], entries per column) and stats (device int64 [8]): [0] rows without
+ * entries, [1] columns without entries, [2] fewest entries in a row, [3] most
+ * in a row, [4] fewest in a column, [5] most in a column, [6] min(d_out - [0],
+ * d_in - [1]), an upper bound on rank(F), [7] the fewest rows that together
+ * hold at least ceil(p / 2) entries. Entries with col_idx outside [0, d_in)
+ * are not counted. ws: qwha_workspace_size(QWHA_OP_PATTERN, d_out, d_in, p,
+ * 0, 0) bytes. Exact (integer arithmetic). */
+qwha_status qwha_energy_stats(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block, int64_t k,
+                              double *stats, void *ws, size_t ws_bytes, void *stream);
+qwha_status qwha_pattern_stats(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr,
+                               const int32_t *col_idx, int32_t *col_counts, int64_t *stats, void *ws,
+                               size_t ws_bytes, void *stream);
+
 /* Calibration Hessian for Value Refinement: S = X^T X, fp32 [d_in, d_in]
  * (device), from calibration rows X bf16 [T, d_in] (device, T >= 1, d_in a
  * multiple of 8), on the tensor cores with fp32 accumulation. */
@@ -297,13 +337,19 @@ qwha_status qwha_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_
  *   dc[j] = alpha * sum_t dY[t, r_j] Z[t, k_j]   fp32 [p], CSR order
  * Same arguments and result as the dc of qwha_adapter_bwd (tile view of `a`
  * required; dX is not computed). The partial sums live in one static array of
- * QWHA_NOALLOC_SCRATCH_BYTES inside the library; a call needing more returns
- * QWHA_ERR_WORKSPACE and launches nothing (the q_proj layer, p = 524288 at
- * 8192 tokens, needs about 10.5 MB). Nothing is allocated. All calls on a
- * device share that array: calls whose work overlaps on the GPU race and must
- * be serialised by the caller; each call clears the partial sums it uses. The
- * first call on a device looks up the array's device address (once, with
- * that device current), so it must come before any stream capture. */
+ * QWHA_NOALLOC_SCRATCH_BYTES inside the library: chunks x p x 4 bytes, where
+ * the number of token chunks is chosen from T, the tile count and the
+ * device's SM count (the q_proj layer, p = 524288 at 8192 tokens, takes 4
+ * chunks, 8.4 MB, on a 148-SM B200). A call needing more returns
+ * QWHA_ERR_WORKSPACE and launches nothing. Nothing is allocated. All calls on
+ * a device share that array: calls whose work overlaps on the GPU race and
+ * must be serialised by the caller; each call clears the partial sums it
+ * uses. The first call in a CUDA context (for runtime users: the first call
+ * on a device) looks up the array's device address with that context
+ * current, so it must come before any stream capture; the lookup is cached
+ * per context, so a context created later, e.g. after cudaDeviceReset, gets
+ * a fresh one. The result is bit for bit the dc of qwha_adapter_bwd with the
+ * sparse algorithm (same kernels, same summation order). */
 qwha_status qwha_coef_grad_noalloc(const qwha_adapter *a, qwha_dtype dt, const void *dY, const void *Z,
                                    int64_t T, float alpha, float *dc, void *stream);
 
@@ -338,6 +384,27 @@ void qwha_stage_timing(int32_t enable);
 int32_t qwha_stage_count(void);
 const char *qwha_stage_name(int32_t i);
 qwha_status qwha_stage_report(int64_t *calls, int64_t *launches, double *ms);
+
+/* Test and fault-injection hooks. They change process-wide state of the
+ * library and exist so that the error paths can be exercised without a GPU
+ * fault; production code does not call them.
+ *
+ * qwha_debug_wait_limit_ns sets the bound, in ns, of the main-loop waits of
+ * the row-transform kernel (the bulk-copy ring that qwha_fwht and the sparse
+ * algorithm's transforms run on) and returns the previous bound (default
+ * 2000000000, i.e. 2 s). A wait that gives up sets the device error word and
+ * its CTA exits after letting its own copies already in flight land (those
+ * drain waits keep the fixed 2 s bound); the call's output is then incomplete
+ * and qwha_check_stream_status reports QWHA_ERR_TIMEOUT. A bound of 0 makes a
+ * wait give up soon after its first unsuccessful poll. Not thread-safe with
+ * respect to calls in flight on other threads.
+ *
+ * qwha_debug_fail_cuda_checks(n) makes the next n checks of a successful CUDA
+ * runtime result inside the library (launches, memsets, copies) report
+ * QWHA_ERR_CUDA with "injected failure" in qwha_last_error(), as though that
+ * call had failed; the work itself was enqueued. n <= 0 disarms it. */
+uint64_t qwha_debug_wait_limit_ns(uint64_t ns);
+void qwha_debug_fail_cuda_checks(int32_t n);
 
 const char *qwha_status_string(qwha_status s);
 const char *qwha_last_error(void);

@@ -98,3 +98,18 @@ def test_sparse_forward_needs_entry_workspace():
     buf = ctypes.c_void_p(16384)
     rc = h.qwha_adapter_fwd(ctypes.byref(a), None, 1, buf, T, ctypes.c_float(1.0), buf, buf, None, 0, None)
     assert rc == 4 and b"workspace" in h.qwha_last_error()
+
+
+def test_debug_hooks_round_trip_on_the_host():
+    """The test hooks only change host-side state: the wait limit is returned on the next set, and arming and
+    disarming the injected failures needs no GPU."""
+    _ensure_built()
+    import walsh_hadamard_sparse_b200._lib as L
+
+    h = L.lib()
+    old = h.qwha_debug_wait_limit_ns(12345)
+    assert old == 2_000_000_000
+    assert h.qwha_debug_wait_limit_ns(old) == 12345
+    h.qwha_debug_fail_cuda_checks(3)
+    h.qwha_debug_fail_cuda_checks(0)
+    assert h.qwha_fwht(0, None, None, 4, 256, 3, None) == 1  # host checks are not CUDA checks: unaffected

@@ -316,6 +316,80 @@ def test_adapter_forward_backward(d_in, d_out, n, T, p, dtype, pattern, algo):
         assert torch.equal(Y3, Y) and torch.equal(dc3, dc) and torch.equal(dX3, dX)
 
 
+def edge_pattern(kind, d_out, d_in, g):
+    """Sparsity patterns with the degenerate rows and columns a real E can have: "rows" mixes empty and full rows
+    into rows of ordinary length; "cols" leaves two thirds of the columns (two of every three 256-column tiles, and
+    a ragged run at the end) without any nonzero."""
+    if kind == "rows":
+        c = g.integers(1, 24, d_out)
+        c[::5] = 0
+        c[1::9] = d_in
+        c[-1] = 0
+        return random_pattern(d_out, d_in, counts=c, rng=g)
+    live = np.array([k for k in range(d_in) if (k // 256) % 3 == 1 and k < d_in - 40])
+    rp, ci, cf = random_pattern(d_out, live.size, p=d_out * 12, rng=g)
+    return rp, live[ci].astype(np.int32), cf
+
+
+EDGE_CASES = [
+    # d_in, d_out, n, T, dtype, pattern
+    (1024, 768, 1024, 1, "bf16", "init"),
+    (1024, 768, 1024, 3, "bf16", "init"),
+    (1024, 768, 1024, 127, "bf16", "init"),
+    (256, 256, 256, 1, "f32", "init"),
+    (256, 256, 256, 3, "f32", "init"),
+    (512, 384, 512, 100, "bf16", "rows"),
+    (512, 384, 256, 100, "f32", "rows"),
+    (1536, 520, 512, 70, "bf16", "cols"),
+]
+
+
+@pytest.mark.parametrize("algo", ["sparse", "dense"])
+@pytest.mark.parametrize("d_in,d_out,n,T,dtype,pattern", EDGE_CASES)
+def test_adapter_edge_cases(d_in, d_out, n, T, dtype, pattern, algo):
+    """Token counts of 1, 3 and 127 (a single token, a few, one short of a 128-row tile) and patterns with empty rows,
+    full rows and empty columns: Z, Y, dX and every dc against the oracle, the adapter alone and with a base weight."""
+    import torch
+
+    if algo == "dense" and dtype != "bf16":
+        pytest.skip("the dense algorithm is bf16 only")
+    W = _W()
+    if pattern == "init":
+        L = synth_layer(42, d_in, d_out, n, T, d_out * 16, dtype)
+    else:
+        L = synth_layer(42, d_in, d_out, n, T, d_out * 4, dtype, pattern="random")
+        L["rp"], L["ci"], L["cf"] = edge_pattern(pattern, d_out, d_in, rng_for(43, "edge", pattern, d_in))
+    rp, ci, cf = L["rp"], L["ci"], L["cf"]
+    if pattern == "rows":
+        cnt = np.diff(rp)
+        assert (cnt == 0).any() and (cnt == d_in).any()
+    if pattern == "cols":
+        assert np.bincount(ci, minlength=d_in)[d_in - 40:].sum() == 0
+    a = device_adapter(d_in, d_out, n, rp, ci, cf, algo=algo)
+    alpha = 0.75
+    Xd, dYd = dev_act(L["X"], dtype), dev_act(L["dY"], dtype)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    Zr, Yr = oracle.adapter_fwd(rp, ci, cf, L["X"], d_out, n, alpha)
+    dXr = oracle.adapter_bwd_dx(rp, ci, cf, L["dY"], d_in, n, alpha)
+    dcr = oracle.adapter_bwd_dc(L["X"], L["dY"], oracle.csr_rows(rp), ci, n, alpha)
+    Z, Y = W.adapter_fwd(a, Xd, alpha)
+    dc, dX = W.adapter_bwd(a, dYd, Z, alpha)
+    torch.cuda.synchronize()
+    errs = dict(Z=rel_fro(host(Z), Zr), Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr), dc=rel_fro(dc.cpu().numpy(), dcr))
+    assert all(v <= tol for v in errs.values()), errs
+    if dtype != "bf16":
+        return
+    wq = dev_qweight(L)
+    Wq = oracle.dequant(L["qweight"], L["scales"], L["zeros"], L["bits"], L["group"], d_out, d_in)
+    _, Yr = oracle.adapter_fwd(rp, ci, cf, L["X"], d_out, n, alpha, Wq, want_z=False)
+    dXr = oracle.adapter_bwd_dx(rp, ci, cf, L["dY"], d_in, n, alpha, Wq)
+    Z, Y = W.adapter_fwd(a, Xd, alpha, wq=wq)
+    dc, dX = W.adapter_bwd(a, dYd, Z, alpha, wq=wq)
+    torch.cuda.synchronize()
+    errs = dict(Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr), dc=rel_fro(dc.cpu().numpy(), dcr))
+    assert all(v <= tol for v in errs.values()), errs
+
+
 GEMM_CASES = [
     (512, 256, 512, 200, 4, 64),  # ragged token tile (200 = 128 + 72)
     (1024, 768, 1024, 300, 3, 128),  # int3 bit stream
@@ -376,6 +450,36 @@ def test_backward_in_two_calls_bitwise(algo):
     assert none_dx is None and none_dc is None
     assert torch.equal(dc1.view(torch.int32), dc2.view(torch.int32))
     assert torch.equal(dX1.view(torch.int16), dX2.view(torch.int16))
+
+
+@pytest.mark.parametrize("algo", ["sparse", "dense"])
+def test_dp_backward_world_size_one_bitwise(algo):
+    """The package's data-parallel backward (dc, its NCCL all-reduce started asynchronously, dX meanwhile) in a
+    one-rank NCCL process group: bit for bit the single call's dc and dX."""
+    import torch
+    import torch.distributed as dist
+
+    W = _W()
+    d_in, d_out, n, T = 1024, 768, 1024, 300
+    L = synth_layer(44, d_in, d_out, n, T, d_out * 8, "bf16", bits=4, group=128)
+    a = device_adapter(d_in, d_out, n, L["rp"], L["ci"], L["cf"], algo=algo)
+    if algo == "dense":
+        a.weff = torch.empty((d_out, d_in), dtype=torch.bfloat16, device="cuda")
+    wq = dev_qweight(L)
+    Xd, dYd = dev_act(L["X"], "bf16"), dev_act(L["dY"], "bf16")
+    Z, _ = W.adapter_fwd(a, Xd, 0.8, wq=wq)
+    dc1, dX1 = W.adapter_bwd(a, dYd, Z, 0.8, wq=wq)
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        dc2, dX2 = W.dp_backward(a, dYd, Z, 0.8, wq=wq)
+        _, Y3, dc3, dX3 = W.dp_step(a, Xd, dYd, 0.8, wq=wq)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    for dc in (dc2, dc3):
+        assert torch.equal(dc1.view(torch.int32), dc.view(torch.int32))
+    for dX in (dX2, dX3):
+        assert torch.equal(dX1.view(torch.int16), dX.view(torch.int16))
 
 
 @pytest.mark.parametrize("d_in,d_out,n,T", [(4096, 512, 4096, 300), (3 * 2048, 384, 2048, 129), (4096, 256, 4096, 8)])

@@ -66,6 +66,76 @@ def test_dp_allreduce_of_dc_matches_single_process():
         assert np.allclose(dX_r, dX_all[r * T_RANK:(r + 1) * T_RANK], rtol=1e-12, atol=1e-12)
 
 
+# --------------------------------------------------------------------------- the package's data-parallel step
+
+
+def _oracle_layer_steps(log):
+    """adapter_fwd / adapter_bwd of the oracle on CPU tensors, with the signatures of the package's functions; every
+    call is appended to `log` so that the test can check the order of the step's parts."""
+    import oracle
+
+    rp, ci, cf, _, _ = _layer()
+
+    def fwd(a, X, alpha, wq, Z_out=None, Y=None, ws=None):
+        log.append("fwd")
+        Zr, Yr = oracle.adapter_fwd(rp, ci, cf, X.numpy(), D_OUT, N, alpha)
+        return torch.from_numpy(Zr), torch.from_numpy(Yr)
+
+    def bwd(a, dY, Z, alpha, wq, dc=None, dX=None, want_dx=True, ws=None, want_dc=True):
+        log.append(("bwd", want_dc, want_dx))
+        out_dc = out_dx = None
+        if want_dc:
+            # the oracle's dc takes X; Z = X H and H is its own inverse, so X = Z H
+            X = oracle.fwht(Z.numpy(), N)
+            out_dc = torch.from_numpy(oracle.adapter_bwd_dc(X, dY.numpy(), oracle.csr_rows(rp), ci, N, alpha))
+        if want_dx:
+            out_dx = torch.from_numpy(oracle.adapter_bwd_dx(rp, ci, cf, dY.numpy(), D_IN, N, alpha))
+        return out_dc, out_dx
+
+    return fwd, bwd
+
+
+def _dp_step_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import oracle
+    from walsh_hadamard_sparse_b200.api import dp_step
+    from workloads import rank_rows
+
+    oracle.set_threads(1)
+    _, _, _, X, dY = _layer()
+    rows = rank_rows(rank, T_RANK)
+    log = []
+    fwd, bwd = _oracle_layer_steps(log)
+    Z, Y, dc, dX = dp_step(None, torch.from_numpy(X[rows]), torch.from_numpy(dY[rows]), 0.7, fwd=fwd, bwd=bwd)
+    out[rank] = (Y.numpy().copy(), dc.numpy().copy(), dX.numpy().copy(), log)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_dp_step_of_the_package_on_two_ranks():
+    """walsh_hadamard_sparse_b200.dp_step on 2 gloo ranks, the oracle's forward and backward injected: every rank
+    ends with the dc of all tokens (one all-reduce) and the Y and dX rows of its own tokens, and the step runs the
+    forward, then dc alone, then dX alone (dc's all-reduce is in flight while dX is computed)."""
+    import oracle
+
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_dp_step_worker, args=(2, port, out), nprocs=2, join=True)
+    rp, ci, cf, X, dY = _layer()
+    _, Y_all = oracle.adapter_fwd(rp, ci, cf, X, D_OUT, N, 0.7)
+    dc_all = oracle.adapter_bwd_dc(X, dY, oracle.csr_rows(rp), ci, N, 0.7)
+    dX_all = oracle.adapter_bwd_dx(rp, ci, cf, dY, D_IN, N, 0.7)
+    for r in range(2):
+        Y_r, dc_r, dX_r, log = out[r]
+        rows = slice(r * T_RANK, (r + 1) * T_RANK)
+        assert log == ["fwd", ("bwd", True, False), ("bwd", False, True)], log
+        assert np.allclose(dc_r, dc_all, rtol=1e-12, atol=1e-12)
+        assert np.allclose(Y_r, Y_all[rows], rtol=1e-12, atol=1e-12)
+        assert np.allclose(dX_r, dX_all[rows], rtol=1e-12, atol=1e-12)
+
+
 # --------------------------------------------------------------------------- sharded AdaAlloc
 
 SH_DOUT, SH_DIN, SH_N, SH_P = 97, 128, 64, 97 * 11 + 5  # odd d_out: uneven shards

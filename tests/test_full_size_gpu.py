@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 from _util import TOL_BF16, bf16_dev, host, rel_fro
-from workloads import CONFIGS, layer_inputs, rng_for
+from workloads import CONFIGS, layer_inputs, pack_codes, rng_for
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -58,6 +58,50 @@ def _check_layer(spec, workload, algos=("dense", "sparse"), rows_n=48, dc_n=48):
         del a, Z, Y, dc, dX
 
 
+def _zero_base(spec, d):
+    """A base weight of the layer's format whose codes all equal their group's zero point, so W_Q = 0 exactly:
+    the dense algorithm then runs its full-size kernels (W_eff from packed codes, the GEMMs with the fused
+    transform) while Y and dX hold the adapter term alone."""
+    import torch
+    import walsh_hadamard_sparse_b200 as W
+
+    codes = np.repeat(d["zeros"], spec.group, axis=1)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    return W.QWeight(spec.bits, spec.group, dev(pack_codes(codes, spec.bits)), dev(d["scales"]), dev(d["zeros"]))
+
+
+def _check_adapter_alone(spec, workload, rows_n=32):
+    """The adapter term alone at full size, where the base term cannot hide an error in it: Z, Y and dX on sampled
+    token rows against the oracle's adapter-only forward and backward (papernotes.org "QWHA", 整体框架: Y_ad =
+    alpha X (F H^-1)^T, with E and c from AdaAlloc of the layer's real quantization error). Sparse algorithm without
+    a base weight; dense algorithm with an all-zero base weight of the layer's bit width."""
+    import torch
+    import walsh_hadamard_sparse_b200 as W
+
+    d, ref, _, X, dY = _device_layer(spec, workload)
+    rp, ci, cf = ref["row_ptr"], ref["col_idx"], ref["coef"]
+    g = rng_for(61, "full-adapter", workload, spec.name)
+    rows = np.sort(g.choice(spec.T, rows_n, replace=False))
+    rows[0], rows[-1] = 0, spec.T - 1  # the first and the last token tile
+    Zr, Yr = oracle.adapter_fwd(rp, ci, cf, d["X"][rows], spec.d_out, spec.had_block, 1.0)
+    dXr = oracle.adapter_bwd_dx(rp, ci, cf, d["dY"][rows], spec.d_in, spec.had_block, 1.0)
+    assert np.linalg.norm(Yr) > 0 and np.linalg.norm(dXr) > 0
+    wq0 = _zero_base(spec, d)
+    dv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    ri = torch.as_tensor(rows).cuda()
+    for algo, wq in (("sparse", None), ("dense", wq0)):
+        a = W.Adapter(spec.d_in, spec.d_out, spec.had_block, spec.p, dv(rp), dv(ci), dv(cf), algo=algo)
+        W.plan_build(a)
+        if algo == "dense":
+            a.weff = torch.empty((spec.d_out, spec.d_in), dtype=torch.bfloat16, device="cuda")
+        Z, Y = W.adapter_fwd(a, X, 1.0, wq)
+        _, dX = W.adapter_bwd(a, dY, Z, 1.0, wq, want_dc=False)
+        torch.cuda.synchronize()
+        errs = {"Z": rel_fro(host(Z[ri]), Zr), "Y": rel_fro(host(Y[ri]), Yr), "dX": rel_fro(host(dX[ri]), dXr)}
+        assert all(v <= TOL_BF16 for v in errs.values()), (algo, errs)
+        del a, Z, Y, dX
+
+
 def test_q_proj_full_size():
     """LLaMA-7B q_proj: 4096 x 4096, 8192 tokens, 4-bit g128, p = 524288."""
     _check_layer(CONFIGS["q_proj"][0], "q_proj")
@@ -69,6 +113,19 @@ def test_llama3_mlp_full_size(name):
     down 14336 -> 4096 whose H is block-diagonal with seven 2048-point blocks."""
     spec = next(s for s in CONFIGS["mlp"] if s.name == name)
     _check_layer(spec, "mlp", rows_n=32, dc_n=24)
+
+
+def test_q_proj_adapter_alone_full_size():
+    """The q_proj layer's adapter term alone (no base term to dominate it), both algorithms."""
+    _check_adapter_alone(CONFIGS["q_proj"][0], "q_proj")
+
+
+@pytest.mark.parametrize("name", ["gate", "down"])
+def test_llama3_mlp_adapter_alone_full_size(name):
+    """The MLP layers' adapter term alone at 16384 tokens: gate (4096 -> 14336) and down (14336 -> 4096, seven
+    2048-point Hadamard blocks), both algorithms."""
+    spec = next(s for s in CONFIGS["mlp"] if s.name == name)
+    _check_adapter_alone(spec, "mlp", rows_n=24)
 
 
 def test_init_sweep_full_size_bitexact():

@@ -12,6 +12,9 @@ from .api import (  # noqa: F401
     adapter_bwd,
     adapter_fwd,
     calib_hessian,
+    dp_backward,
+    dp_step,
+    energy_stats,
     fwht,
     init_alloc,
     init_alloc_sharded,
@@ -19,6 +22,7 @@ from .api import (  # noqa: F401
     init_norms,
     init_select,
     init_select_global,
+    pattern_stats,
     plan_build,
     plan_tiles,
     refine_values,

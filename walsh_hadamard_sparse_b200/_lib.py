@@ -61,6 +61,8 @@ _SIGNATURES = {
     "qwha_init_budgets": (ctypes.c_int, [P, i32, i32, i64, i32, ctypes.c_int, P, P, P, sz, P]),
     "qwha_init_select": (ctypes.c_int, [P, i32, i32, i32, P, P, i64, P, P, P]),
     "qwha_plan_build": (ctypes.c_int, [i32, i32, i64, P, P, P, P, P, P, P, P, P, sz, P]),
+    "qwha_energy_stats": (ctypes.c_int, [P, i32, i32, i32, i64, P, P, sz, P]),
+    "qwha_pattern_stats": (ctypes.c_int, [i32, i32, i64, P, P, P, P, P, sz, P]),
     "qwha_plan_tiles": (i64, [i32, i32]),
     "qwha_workspace_size": (sz, [ctypes.c_int, i32, i32, i64, i64, i32]),
     "qwha_validate_plan": (ctypes.c_int, [ctypes.POINTER(QwhaAdapter), P]),
@@ -69,6 +71,8 @@ _SIGNATURES = {
     "qwha_stage_count": (i32, []),
     "qwha_stage_name": (ctypes.c_char_p, [i32]),
     "qwha_stage_report": (ctypes.c_int, [P, P, P]),
+    "qwha_debug_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
+    "qwha_debug_fail_cuda_checks": (None, [i32]),
     "qwha_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qwha_last_error": (ctypes.c_char_p, []),
     "qwha_version": (ctypes.c_char_p, []),

@@ -16,6 +16,8 @@ from ._lib import QwhaAdapter, QwhaQweight, check, lib
 
 F32, BF16 = 0, 1
 OP_FWD, OP_BWD, OP_INIT, OP_PLAN, OP_FWD_DENSE, OP_BWD_DENSE, OP_SELECT_GLOBAL, OP_REFINE = 0, 1, 2, 3, 4, 5, 6, 7
+OP_ENERGY, OP_PATTERN = 8, 9
+PATTERN_STATS = ("empty_rows", "empty_cols", "min_row", "max_row", "min_col", "max_col", "rank_bound", "half_rows")
 SELECTION = {"magnitude": 0, "random": 1}
 ALGO = {"sparse": 0, "dense": 1}
 REMAINDER = {"fewest": 0, "largest": 1}
@@ -158,6 +160,43 @@ def adapter_bwd(a: Adapter, dY: torch.Tensor, Z: torch.Tensor, alpha: float = 1.
     return (dc if want_dc else None), (dX if want_dx else None)
 
 
+def dp_backward(a: Adapter, dY: torch.Tensor, Z: torch.Tensor, alpha: float = 1.0, wq: QWeight | None = None,
+                dc: torch.Tensor | None = None, dX: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                group=None, bwd=None):
+    """Backward of one adapted layer under token data parallelism: every rank holds its own token rows of dY and Z.
+
+    dc is a sum over tokens, so it is the one quantity the ranks exchange (only c trains: papernotes.org "QWHA",
+    整体框架 and 训练策略); dX of a token needs only that token. The call computes this rank's dc first
+    (qwha_adapter_bwd with dX NULL), starts an asynchronous all-reduce (sum) of it over `group`, computes this
+    rank's dX (dc NULL) while the all-reduce runs, and waits for it. Returns (dc summed over the ranks, dX of this
+    rank's tokens); without an initialised process group it is the single-process backward.
+
+    `bwd` replaces adapter_bwd (same signature); the collective runs on whatever device the tensors live on."""
+    import torch.distributed as dist
+
+    bwd = bwd or adapter_bwd
+    dc, _ = bwd(a, dY, Z, alpha, wq, dc=dc, want_dx=False, ws=ws)
+    work = None
+    if dist.is_available() and dist.is_initialized():
+        work = dist.all_reduce(dc, group=group, async_op=True)
+    _, dX = bwd(a, dY, Z, alpha, wq, dX=dX, want_dc=False, ws=ws)
+    if work is not None:
+        work.wait()
+    return dc, dX
+
+
+def dp_step(a: Adapter, X: torch.Tensor, dY: torch.Tensor, alpha: float = 1.0, wq: QWeight | None = None,
+            Z: torch.Tensor | None = None, Y: torch.Tensor | None = None, dc: torch.Tensor | None = None,
+            dX: torch.Tensor | None = None, ws_fwd: torch.Tensor | None = None, ws_bwd: torch.Tensor | None = None,
+            group=None, fwd=None, bwd=None):
+    """One data-parallel training step of the layer on this rank's tokens: the forward (Z, Y), then dp_backward.
+    Returns (Z, Y, dc summed over the ranks, dX). `fwd` / `bwd` replace adapter_fwd / adapter_bwd."""
+    fwd = fwd or adapter_fwd
+    Z, Y = fwd(a, X, alpha, wq, Z_out=Z, Y=Y, ws=ws_fwd)
+    dc, dX = dp_backward(a, dY, Z, alpha, wq, dc=dc, dX=dX, ws=ws_bwd, group=group, bwd=bwd)
+    return Z, Y, dc, dX
+
+
 def init_alloc(dWq: torch.Tensor, p: int, had_block: int, min_per_row: int = 2, mode: str = "fewest",
                ws: torch.Tensor | None = None) -> dict:
     """AdaAlloc on the device: dict(budgets, row_ptr, col_idx, coef)."""
@@ -199,6 +238,34 @@ def init_select_global(dWq: torch.Tensor, p: int, had_block: int, sel: str = "ma
     check(rc, "qwha_init_select_global")
     out["col_idx"], out["coef"] = out["col_idx"][:p], out["coef"][:p]
     return out
+
+
+def energy_stats(dWq: torch.Tensor, k: int, had_block: int, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Hill exponent eta and cumulative energy of the k largest |dW_Q H| (qwha_energy_stats): fp64 device tensor
+    [eta, energy fraction of the k largest, a_(k+1), sum of all a^2]."""
+    d_out, d_in = dWq.shape
+    out = torch.empty(4, dtype=torch.float64, device=dWq.device)
+    need = workspace_size(OP_ENERGY, d_out, d_in, 0, 0, False)
+    ws = _ws(need, dWq.device) if ws is None else ws
+    check(lib().qwha_energy_stats(_ptr(dWq), d_out, d_in, had_block, int(k), _ptr(out), _ptr(ws),
+                                  0 if ws is None else ws.numel(), _stream()), "qwha_energy_stats")
+    return out
+
+
+def pattern_stats(row_ptr: torch.Tensor, col_idx: torch.Tensor, d_in: int,
+                  ws: torch.Tensor | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """(stats int64 [8] in the order of PATTERN_STATS, col_counts int32 [d_in]) of E (qwha_pattern_stats)."""
+    d_out = row_ptr.numel() - 1
+    p = col_idx.numel()
+    dev = row_ptr.device
+    stats = torch.empty(8, dtype=torch.int64, device=dev)
+    cc = torch.empty(d_in, dtype=torch.int32, device=dev)
+    need = workspace_size(OP_PATTERN, d_out, d_in, p, 0, False)
+    ws = _ws(need, dev) if ws is None else ws
+    check(lib().qwha_pattern_stats(d_out, d_in, p, _ptr(row_ptr), _ptr(col_idx) if p else None, _ptr(cc),
+                                   _ptr(stats), _ptr(ws), 0 if ws is None else ws.numel(), _stream()),
+          "qwha_pattern_stats")
+    return stats, cc
 
 
 def calib_hessian(X: torch.Tensor, S: torch.Tensor | None = None) -> torch.Tensor:

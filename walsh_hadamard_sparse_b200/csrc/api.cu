@@ -5,6 +5,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -25,8 +26,22 @@ qwha_status fail(qwha_status s, const char *fmt, ...) {
   return s;
 }
 
+namespace {
+std::atomic<uint64_t> g_ring_wait_ns{2000000000ull};
+std::atomic<int32_t> g_injected_failures{0};
+}  // namespace
+
+uint64_t ring_wait_ns() { return g_ring_wait_ns.load(std::memory_order_relaxed); }
+
 qwha_status cuda_status(cudaError_t e, const char *what) {
-  if (e == cudaSuccess) return QWHA_OK;
+  if (e == cudaSuccess) {
+    // test hook: report an armed number of successful results as failures
+    int32_t n = g_injected_failures.load();
+    while (n > 0 && !g_injected_failures.compare_exchange_weak(n, n - 1)) {
+    }
+    if (n <= 0) return QWHA_OK;
+    return fail(QWHA_ERR_CUDA, "%s: injected failure (qwha_debug_fail_cuda_checks)", what);
+  }
   return fail(QWHA_ERR_CUDA, "%s: %s (cudaError %d)", what, cudaGetErrorString(e), (int)e);
 }
 
@@ -228,6 +243,10 @@ const char *qwha_status_string(qwha_status s) {
 
 const char *qwha_last_error(void) { return g_msg; }
 
+uint64_t qwha_debug_wait_limit_ns(uint64_t ns) { return g_ring_wait_ns.exchange(ns); }
+
+void qwha_debug_fail_cuda_checks(int32_t n) { g_injected_failures.store(n > 0 ? n : 0); }
+
 const char *qwha_version(void) { return "qwha-b200 0.1 (sm_100a)"; }
 
 qwha_status qwha_fwht(qwha_dtype dt, const void *x, void *z, int64_t rows, int32_t n,
@@ -402,6 +421,8 @@ size_t qwha_workspace_size(qwha_op op, int32_t d_out, int32_t d_in, int64_t p, i
     case QWHA_OP_BWD_DENSE: return bwd_dense_ws(d_out, d_in, T);
     case QWHA_OP_SELECT_GLOBAL: return select_global_workspace(d_out, d_in);
     case QWHA_OP_REFINE: return refine_workspace(d_out, d_in);
+    case QWHA_OP_ENERGY: return energy_stats_workspace(d_out, d_in);
+    case QWHA_OP_PATTERN: return pattern_stats_workspace(d_in);
   }
   return 0;
 }
@@ -667,6 +688,39 @@ qwha_status qwha_init_select_global(const float *dWq, int32_t d_out, int32_t d_i
   return cuda_status(launch_select_global(dWq, d_out, d_in, had_block, p, (int)sel, seed, budgets, row_ptr, col_idx,
                                           coef, ws, (cudaStream_t)stream),
                      "init_select_global");
+}
+
+qwha_status qwha_energy_stats(const float *dWq, int32_t d_out, int32_t d_in, int32_t had_block, int64_t k,
+                              double *stats, void *ws, size_t ws_bytes, void *stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(QWHA_ERR_INVALID_ARG, "d_out %d, d_in %d", d_out, d_in);
+  qwha_status st = check_hadamard(d_in, had_block);
+  if (st != QWHA_OK) return st;
+  if (d_in > init_max_din()) return fail(QWHA_ERR_UNSUPPORTED, "d_in %d above %d", d_in, init_max_din());
+  if (k < 1 || k >= (int64_t)d_in * d_out || k >= 2147483647LL)
+    return fail(QWHA_ERR_INVALID_ARG, "k = %lld outside [1, %lld)", (long long)k, (long long)d_in * d_out);
+  QWHA_CHECK_PTR(dWq, "dWq");
+  QWHA_CHECK_PTR(stats, "stats");
+  if ((st = check_ws(ws, ws_bytes, energy_stats_workspace(d_out, d_in))) != QWHA_OK) return st;
+  StageScope sc(ST_INIT, 20, (cudaStream_t)stream);
+  return cuda_status(launch_energy_stats(dWq, d_out, d_in, had_block, k, stats, ws, (cudaStream_t)stream),
+                     "energy_stats");
+}
+
+qwha_status qwha_pattern_stats(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr, const int32_t *col_idx,
+                               int32_t *col_counts, int64_t *stats, void *ws, size_t ws_bytes, void *stream) {
+  if (d_out <= 0 || d_in <= 0) return fail(QWHA_ERR_INVALID_ARG, "d_out %d, d_in %d", d_out, d_in);
+  if (p < 0 || p > (int64_t)d_in * d_out || p > 2147483647LL)
+    return fail(QWHA_ERR_INVALID_ARG, "p = %lld outside [0, %lld]", (long long)p, (long long)d_in * d_out);
+  QWHA_CHECK_PTR(row_ptr, "row_ptr");
+  if (p > 0) QWHA_CHECK_PTR(col_idx, "col_idx");
+  QWHA_CHECK_PTR(col_counts, "col_counts");
+  QWHA_CHECK_PTR(stats, "stats");
+  qwha_status st = check_ws(ws, ws_bytes, pattern_stats_workspace(d_in));
+  if (st != QWHA_OK) return st;
+  StageScope sc(ST_INIT, 4, (cudaStream_t)stream);
+  return cuda_status(launch_pattern_stats(d_out, d_in, p, row_ptr, col_idx, col_counts, stats, ws,
+                                          (cudaStream_t)stream),
+                     "pattern_stats");
 }
 
 qwha_status qwha_calib_hessian(const void *X, int64_t T, int32_t d_in, float *S, void *stream) {

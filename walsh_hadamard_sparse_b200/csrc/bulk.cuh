@@ -42,15 +42,17 @@ __device__ __forceinline__ bool try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase of the given parity to complete; false after kWaitNs.
-__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of the given parity to complete; false once limit_ns
+// have passed since the first unsuccessful poll (the phase is polled at least
+// 33 times, so a limit of 0 gives up soon after a first miss).
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitNs) {
   if (try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (try_wait(bar, parity)) return true;
-    if (now_ns() - t0 > kWaitNs) return false;
+    if (now_ns() - t0 > limit_ns) return false;
   }
 }
 

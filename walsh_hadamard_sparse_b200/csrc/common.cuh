@@ -32,6 +32,10 @@ int device_slot();  // index of the current device in [0, 64) (0 if unreadable),
 // qwha_check_stream_status). One per device, in __device__ memory.
 unsigned int *device_error_word();
 
+// Limit of the row-transform kernel's main-loop waits, in ns (2 s unless a
+// test lowered it through qwha_debug_wait_limit_ns).
+uint64_t ring_wait_ns();
+
 // ---------------------------------------------------------------- device side
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -67,7 +67,8 @@ struct RingGeo {
 template <int LOGN, int V, typename Tin, typename Tout, int S>
 __global__ void __launch_bounds__(RingGeo<LOGN, V>::RW) fwht_ring_kernel(const Tin *__restrict__ x,
                                                                          Tout *__restrict__ z, int64_t rows,
-                                                                         float scale, unsigned int *err) {
+                                                                         float scale, unsigned int *err,
+                                                                         uint64_t wait_ns) {
   using G = Geo<LOGN, V>;
   using RG = RingGeo<LOGN, V>;
   constexpr int RPW = RG::RPW;
@@ -107,7 +108,9 @@ __global__ void __launch_bounds__(RingGeo<LOGN, V>::RW) fwht_ring_kernel(const T
     const int s = (int)(it % S);
     const int64_t row = first + it * stride + rl;
     const bool active = row < rows;
-    const bool ok = bulk::wait(bulk::saddr(full + s), (uint32_t)((it / S) & 1));
+    // wait_ns bounds this wait (the library's limit, lowered only by a test hook); the drain below always
+    // keeps the fixed limit, so that no copy is still landing in shared memory when the CTA exits
+    const bool ok = bulk::wait(bulk::saddr(full + s), (uint32_t)((it / S) & 1), wait_ns);
     if (tid == 0) bulk::wait_stores_read();  // the last iteration's output copies have read buf
     // every thread has left the previous iteration's output reads of buf
     if (__syncthreads_or(!ok)) {
@@ -796,7 +799,7 @@ cudaError_t run_ring(const Tin *x, Tout *z, int64_t rows, float scale, cudaStrea
   const int64_t need = cdiv(rows, RG::RPW);
   const int64_t cap = (int64_t)sm_count() * occ;
   const int grid = (int)(need < cap ? need : cap);
-  k<<<grid, RG::RW, smem, s>>>(x, z, rows, scale, device_error_word());
+  k<<<grid, RG::RW, smem, s>>>(x, z, rows, scale, device_error_word(), ring_wait_ns());
   return cudaGetLastError();
 }
 

@@ -1163,6 +1163,79 @@ __global__ void __launch_bounds__(kSelThreads)
                sh64);
 }
 
+// ---------------------------------------------------------------- energy concentration (selection diagnostics)
+//
+// Hill's estimate over the k largest coefficient magnitudes a = |V| and the
+// energy they hold, from the (k+1)-th largest magnitude thr = a_(k+1) found by
+// the radix select above (with need = k + 1):
+//   sum_{i<=k} ln(a_(i) / thr) = sum over a > thr of ln(a / thr)   (ties add 0)
+//   sum_{i<=k} a_(i)^2 = sum over a > thr of a^2 + (k - #{a > thr}) thr^2
+// Per-CTA partial sums (fixed thread-to-element map and tree), then one CTA
+// adds them in a fixed order: the result does not depend on scheduling.
+
+constexpr int kEnergyMaxParts = 2048;
+
+struct EnergyPart {
+  double hill, top2, all2;
+  long long gt;
+};
+
+__device__ __forceinline__ double magnitude_of_key(uint64_t key) {
+  return __longlong_as_double((long long)(~key & 0x7fffffffffffffffull));
+}
+
+__global__ void __launch_bounds__(kGselThreads)
+    energy_part_kernel(const double *__restrict__ V, int64_t N, const GselState *st, EnergyPart *__restrict__ part) {
+  __shared__ double shd[33];
+  __shared__ long long shl[33];
+  const double thr = magnitude_of_key(st->prefix);
+  double hill = 0.0, top2 = 0.0, all2 = 0.0;
+  long long gt = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < N; j += stride) {
+    const double a = fabs(V[j]);
+    all2 += a * a;
+    if (a > thr) {
+      if (thr > 0.0) hill += log(a / thr);
+      top2 += a * a;
+      ++gt;
+    }
+  }
+  hill = block_sum(hill, shd);
+  top2 = block_sum(top2, shd);
+  all2 = block_sum(all2, shd);
+  gt = block_sum(gt, shl);
+  if (threadIdx.x == 0) part[blockIdx.x] = EnergyPart{hill, top2, all2, gt};
+}
+
+__global__ void __launch_bounds__(kGselThreads)
+    energy_finish_kernel(const EnergyPart *__restrict__ part, int nparts, int64_t k, const GselState *st,
+                         double *__restrict__ out) {
+  __shared__ double shd[33];
+  __shared__ long long shl[33];
+  double hill = 0.0, top2 = 0.0, all2 = 0.0;
+  long long gt = 0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) {
+    hill += part[i].hill;
+    top2 += part[i].top2;
+    all2 += part[i].all2;
+    gt += part[i].gt;
+  }
+  hill = block_sum(hill, shd);
+  top2 = block_sum(top2, shd);
+  all2 = block_sum(all2, shd);
+  gt = block_sum(gt, shl);
+  if (threadIdx.x == 0) {
+    const double thr = magnitude_of_key(st->prefix);
+    const double top = top2 + (double)(k - gt) * thr * thr;
+    const double xi = hill / (double)k;
+    out[0] = (thr > 0.0 && xi > 0.0) ? 1.0 / xi : __longlong_as_double(0x7ff8000000000000ll);
+    out[1] = all2 > 0.0 ? top / all2 : __longlong_as_double(0x7ff8000000000000ll);
+    out[2] = thr;
+    out[3] = all2;
+  }
+}
+
 }  // namespace
 
 size_t init_workspace(int32_t d_out, int32_t d_in) {
@@ -1245,6 +1318,42 @@ cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, i
   if (p > 0)
     gsel_take_kernel<<<d_out, kSelThreads, smem, s>>>(V, d_in, had_block, sel, seed, st, take, row_ptr, p, col_idx,
                                                       coef);
+  return cudaGetLastError();
+}
+
+size_t energy_stats_workspace(int32_t d_out, int32_t d_in) {
+  return select_global_workspace(d_out, d_in) + align_up((size_t)kEnergyMaxParts * sizeof(EnergyPart), 256);
+}
+
+cudaError_t launch_energy_stats(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t k,
+                                double *out, void *ws, cudaStream_t s) {
+  char *w = static_cast<char *>(ws);
+  double *V = reinterpret_cast<double *>(w);
+  w += align_up((size_t)d_out * d_in * 8, 256);
+  GselState *st = reinterpret_cast<GselState *>(w);
+  w += align_up(sizeof(GselState), 256);
+  w += 3 * align_up((size_t)d_out * 4, 256);
+  unsigned long long *cand = reinterpret_cast<unsigned long long *>(w);
+  w += (size_t)kGselCap * 8;
+  EnergyPart *part = reinterpret_cast<EnergyPart *>(w);
+  const size_t smem = vbytes(d_in);
+  cudaError_t e = cudaFuncSetAttribute(gsel_transform_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t N = (int64_t)d_out * d_in;
+  gsel_transform_kernel<<<d_out, kSelThreads, smem, s>>>(dW, d_in, had_block, V);
+  gsel_init_kernel<<<1, 256, 0, s>>>(st, k + 1);  // the (k+1)-th largest magnitude
+  const int64_t grid = std::min<int64_t>(cdiv(N, (int64_t)kGselThreads), (int64_t)sm_count() * 8);
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    gsel_hist_kernel<<<(unsigned)grid, kGselThreads, 0, s>>>(V, N, 0, 0, shift, st);
+    gsel_pick_kernel<<<1, 32, 0, s>>>(st, shift);
+    if (shift > 0) {
+      gsel_list_kernel<<<(unsigned)grid, kGselThreads, 0, s>>>(V, N, 0, 0, shift, st, cand);
+      gsel_finish_kernel<<<1, 1024, 0, s>>>(st, cand);
+    }
+  }
+  const int parts = (int)std::min<int64_t>(grid, kEnergyMaxParts);
+  energy_part_kernel<<<parts, kGselThreads, 0, s>>>(V, N, st, part);
+  energy_finish_kernel<<<1, kGselThreads, 0, s>>>(part, parts, k, st, out);
   return cudaGetLastError();
 }
 

@@ -67,6 +67,14 @@ size_t select_global_workspace(int32_t d_out, int32_t d_in);
 cudaError_t launch_select_global(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t p, int sel,
                                  uint64_t seed, int32_t *budgets, int32_t *row_ptr, int32_t *col_idx, float *coef,
                                  void *ws, cudaStream_t s);
+// Selection diagnostics (init.cu, diag.cu).
+size_t energy_stats_workspace(int32_t d_out, int32_t d_in);
+cudaError_t launch_energy_stats(const float *dW, int32_t d_out, int32_t d_in, int32_t had_block, int64_t k,
+                                double *out, void *ws, cudaStream_t s);
+size_t pattern_stats_workspace(int32_t d_in);
+cudaError_t launch_pattern_stats(int32_t d_out, int32_t d_in, int64_t p, const int32_t *row_ptr,
+                                 const int32_t *col_idx, int32_t *col_counts, int64_t *stats, void *ws,
+                                 cudaStream_t s);
 cudaError_t launch_init_norms(const float *dW, int32_t rows, int32_t d_in, double *e, cudaStream_t s);
 cudaError_t launch_init_budgets(const double *e, int32_t d_out, int32_t d_in, int64_t p, int32_t min_per_row, int mode,
                                 int32_t *budgets, int32_t *row_ptr, void *ws, cudaStream_t s);

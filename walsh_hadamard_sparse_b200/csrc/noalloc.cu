@@ -18,9 +18,15 @@
 //   * the partial sums are cleared at the start of every call, so nothing
 //     left by an earlier call leaks into the result.
 // In host code the array's name is only a host-side stand-in, so its device
-// address is looked up with cudaGetSymbolAddress, once per device, on the
-// first call made with that device current. That first call must therefore
-// come before any stream capture.
+// address is looked up with cudaGetSymbolAddress, once per CUDA context, on
+// the first call made with that context current (for ordinary runtime users:
+// once per device, in its primary context). That first call must therefore
+// come before any stream capture. The cache is keyed on the context's
+// process-unique id, so a context created later (after cudaDeviceReset, or a
+// driver-API context of the caller's own) gets its own lookup instead of a
+// stale address.
+
+#include <cuda.h>
 
 #include <mutex>
 
@@ -32,24 +38,69 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QWHA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_addr[kMaxDevices] = {nullptr};
+// Driver entry points reached through the runtime, so the library needs no
+// link against libcuda.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
 
-// Device address of the scratch array for the current device (set-up on first use).
+struct CachedAddress {
+  unsigned long long ctx_id;
+  void *addr;
+};
+constexpr int kMaxContexts = 64;
+std::mutex g_mu;
+CachedAddress g_cache[kMaxContexts];
+int g_cached = 0, g_next_evict = 0;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+qwha_status driver_entry_points() {
+  if (g_ctx_get_current && g_ctx_get_id) return QWHA_OK;
+  void *f0 = nullptr, *f1 = nullptr;
+  cudaDriverEntryPointQueryResult q0 = cudaDriverEntryPointSymbolNotFound, q1 = q0;
+  cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &f0, cudaEnableDefault, &q0);
+  if (e != cudaSuccess || q0 != cudaDriverEntryPointSuccess || !f0)
+    return e != cudaSuccess ? cuda_status(e, "cudaGetDriverEntryPoint(cuCtxGetCurrent)")
+                            : fail(QWHA_ERR_CUDA, "cuCtxGetCurrent not found");
+  e = cudaGetDriverEntryPoint("cuCtxGetId", &f1, cudaEnableDefault, &q1);
+  if (e != cudaSuccess || q1 != cudaDriverEntryPointSuccess || !f1)
+    return e != cudaSuccess ? cuda_status(e, "cudaGetDriverEntryPoint(cuCtxGetId)")
+                            : fail(QWHA_ERR_CUDA, "cuCtxGetId not found (driver older than CUDA 12.0)");
+  g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f0);
+  g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f1);
+  return QWHA_OK;
+}
+
+// Device address of the scratch array in the current context (looked up on
+// the first call in that context).
 qwha_status scratch_address(void **out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(QWHA_ERR_UNSUPPORTED, "device ordinal %d", dev);
   std::lock_guard<std::mutex> g(g_mu);
-  if (!g_addr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  qwha_status st = driver_entry_points();
+  if (st != QWHA_OK) return st;
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return fail(QWHA_ERR_CUDA, "cuCtxGetCurrent failed");
+  void *p = nullptr;
+  if (!ctx) {
+    // No context is current yet: the runtime makes the current device's
+    // primary context current on its first call that needs one, this lookup.
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(scratch)");
-    g_addr[dev] = p;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx) return fail(QWHA_ERR_CUDA, "no current CUDA context");
   }
-  *out = g_addr[dev];
+  unsigned long long id = 0;
+  if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return fail(QWHA_ERR_CUDA, "cuCtxGetId failed");
+  for (int i = 0; i < g_cached; ++i)
+    if (g_cache[i].ctx_id == id) {
+      *out = g_cache[i].addr;
+      return QWHA_OK;
+    }
+  if (!p) {
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(scratch)");
+  }
+  const int slot = g_cached < kMaxContexts ? g_cached++ : (g_next_evict++ % kMaxContexts);
+  g_cache[slot] = {id, p};
+  *out = p;
   return QWHA_OK;
 }
 
