@@ -269,26 +269,59 @@ def config_block(spec, n):
 # --------------------------------------------------------------------------- main
 
 
-def run_block(args):
-    """The decoder-block workload (seven LLaMA-3-8B-shaped linears, 32768 tokens, 4-bit g128, r = 64): forward of
-    every layer then backward in reverse order, dense algorithm, with the transform Z = X H shared by the layers
-    that read the same input (q, k, v; gate, up) and, for comparison, computed by every layer. Weights and
-    AdaAlloc as in the tests (host-generated seeded weights, AdaAlloc on the GPU); the activations are drawn on
-    the GPU from a seeded generator with the workload's distribution (N(0, 1), 1% of input channels x20)."""
-    import torch
+# --------------------------------------------------------------------------- the other workloads
 
-    import walsh_hadamard_sparse_b200 as W
+# what the GPU needs of a layer's host-generated weights
+W_KEYS = ("qweight", "scales", "zeros", "dWq")
+
+
+def host_weights(spec, seed, workload, keys=W_KEYS):
+    """The seeded weights of one layer (runs in a worker process): only the arrays the GPU needs."""
+    d = layer_inputs(spec, seed, workload, parts=("W",))
+    return {k: d[k] for k in keys}
+
+
+class WeightPool:
+    """Host generation of the other workloads' weights in spawned worker processes (started before the first GPU
+    call), so that it overlaps the headline measurement instead of adding to the run."""
+
+    def __init__(self, seed, workers):
+        import concurrent.futures
+        import multiprocessing
+
+        self.ex = concurrent.futures.ProcessPoolExecutor(max_workers=workers,
+                                                         mp_context=multiprocessing.get_context("spawn"))
+        self.fut = {}
+        for wl in ("mlp", "block"):
+            for spec in CONFIGS[wl]:
+                self.fut[(wl, spec.name)] = self.ex.submit(host_weights, spec, seed, wl)
+        for spec in CONFIGS["init_sweep"]:
+            key = ("init_sweep", spec.w_stream)
+            if key not in self.fut:
+                self.fut[key] = self.ex.submit(host_weights, spec, seed, "init_sweep", ("dWq",))
+
+    def get(self, wl, name):
+        return self.fut[(wl, name)].result()
+
+    def close(self):
+        self.ex.shutdown(wait=True, cancel_futures=True)
+
+
+def run_stack(W, torch, dev, wl, weights, seed, K, warmup, peaks, compare_unshared=False):
+    """Forward of every layer of workload `wl` in order, then the backward in reverse order (dense algorithm), as one
+    step; the transform Z = X H is shared by the layers that read the same input (z_given). AdaAlloc on the GPU from
+    the host-generated dW_Q; activations drawn on the GPU from a seeded generator with the workload's distribution
+    (N(0, 1), 1% of input channels x20). Returns the timing record (and, with compare_unshared, the same step with
+    every layer computing its own transform)."""
     from workloads.synth import _x_channels
 
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    specs = CONFIGS["block"]
+    specs = CONFIGS[wl]
     T = specs[0].T
     gen = torch.Generator(device=dev)
-    gen.manual_seed(args.seed)
+    gen.manual_seed(seed)
     layers, X, Zb, dY, Y, dX, dc = [], {}, {}, {}, {}, {}, {}
     for spec in specs:
-        d = layer_inputs(spec, args.seed, "block", parts=("W",))
+        d = weights(wl, spec.name)
         dWq = torch.from_numpy(d["dWq"]).to(dev)
         e = W.init_alloc(dWq, spec.p, spec.had_block, spec.min_per_row, spec.remainder)
         del dWq
@@ -300,7 +333,7 @@ def run_block(args):
         layers.append((spec, a, wq))
         if spec.x_stream not in X:
             x = torch.randn((T, spec.d_in), generator=gen, device=dev)
-            ch = torch.from_numpy(_x_channels(spec, args.seed, "block")).to(dev)
+            ch = torch.from_numpy(_x_channels(spec, seed, wl)).to(dev)
             x[:, ch] *= spec.x_outlier_scale
             X[spec.x_stream] = x.to(torch.bfloat16)
             Zb[spec.x_stream] = torch.empty_like(X[spec.x_stream])
@@ -309,41 +342,151 @@ def run_block(args):
         Y[spec.name] = torch.empty((T, spec.d_out), dtype=torch.bfloat16, device=dev)
         dX[spec.name] = torch.empty((T, spec.d_in), dtype=torch.bfloat16, device=dev)
         dc[spec.name] = torch.empty(spec.p, dtype=torch.float32, device=dev)
+    ws = {}
+    for spec, _, _ in layers:
+        for op in (4, 5):
+            n = W.workspace_size(op, spec.d_out, spec.d_in, spec.p, T, True)
+            if n > ws.get(op, torch.empty(0)).numel():
+                ws[op] = torch.empty(n, dtype=torch.uint8, device=dev)
 
     def step(shared):
         seen = set()
         for spec, a, wq in layers:
             given = shared and spec.x_stream in seen
-            W.adapter_fwd(a, X[spec.x_stream], 1.0, wq, Z_out=Zb[spec.x_stream], Y=Y[spec.name], z_given=given)
+            W.adapter_fwd(a, X[spec.x_stream], 1.0, wq, Z_out=Zb[spec.x_stream], Y=Y[spec.name], z_given=given,
+                          ws=ws.get(4))
             seen.add(spec.x_stream)
         for spec, a, wq in reversed(layers):
-            W.adapter_bwd(a, dY[spec.name], Zb[spec.x_stream], 1.0, wq, dc=dc[spec.name], dX=dX[spec.name])
+            W.adapter_bwd(a, dY[spec.name], Zb[spec.x_stream], 1.0, wq, dc=dc[spec.name], dX=dX[spec.name],
+                          ws=ws.get(5))
 
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     res = {}
-    K = max(3, min(args.steps, 10))
-    for shared in (True, False):
-        for _ in range(max(args.warmup, 3)):
+    for shared in ((True, False) if compare_unshared else (True,)):
+        for _ in range(warmup):
             step(shared)
         torch.cuda.synchronize()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        W.stage_report()
+        W.stage_timing(shared)
         for i in range(K):
             flush.fill_(i & 0xFF)
             ev[i][0].record()
             step(shared)
             ev[i][1].record()
         torch.cuda.synchronize()
-        res[shared] = sum(s_.elapsed_time(e_) for s_, e_ in ev) / K
+        W.stage_timing(False)
+        rep = W.stage_report()
+        ms = sum(s_.elapsed_time(e_) for s_, e_ in ev) / K
+        res[shared] = (ms, rep, ev[0][0].elapsed_time(ev[-1][1]) / 1e3)
+    ms, rep, region_s = res[True]
+    # per-stage work of one step: every layer runs every stage once
+    stages = {}
+    for name, (calls, launches, tot_ms) in rep.items():
+        if not calls:
+            continue
+        kinds = [stage_work(name, spec, T, spec.bits, "dense") for spec in specs]
+        if any(k is None for k in kinds):
+            stages[name] = {"ms_per_step": tot_ms / K}
+            continue
+        kind = kinds[0][0]
+        work = sum(k[1] for k in kinds)
+        peak, unit, note = peak_for(kind, peaks, region_s)
+        ach = work / (tot_ms / K / 1e3) / (1e9 if unit == "GB/s" else 1e12)
+        stages[name] = {"ms_per_step": tot_ms / K, "calls_per_step": calls / K, "bound": kind, "achieved": ach,
+                        "unit": unit, "peak": peak, "frac": ach / peak, "peak_source": note}
+    dom = max((n for n in stages if "frac" in stages[n]), key=lambda n: stages[n]["ms_per_step"])
     flops = sum(3 * 2.0 * T * sp.d_in * sp.d_out for sp in specs)
+    out = {"ms_per_step": ms, "value": T / (ms / 1e3), "unit": UNIT, "steps": K, "tokens": T,
+           "gemm_tflops": flops / (ms / 1e3) / 1e12, "stages": stages,
+           "roofline": dict(kernel=dom, **{k: stages[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                                                      "peak_source")})}
+    if compare_unshared:
+        out["without_sharing"] = {"ms_per_step": res[False][0], "value": T / (res[False][0] / 1e3)}
+    del layers, X, Zb, dY, Y, dX, dc, ws, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_init_sweep(W, torch, dev, weights, peaks):
+    """AdaAlloc on the seven LLaMA-3-8B shapes at r = 16, 64, 128 (2-bit g64 error): the median of 3 timed calls
+    per shape, each after a warm call; plus the Hill exponent and cumulative energy of |dW_Q H| at k = p (the
+    selection diagnostics) for every shape and r."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    shapes, tot_ms, tot_bytes, cur = {}, 0.0, 0.0, {}
+    for spec in CONFIGS["init_sweep"]:
+        if spec.w_stream not in cur:
+            cur.clear()
+            cur[spec.w_stream] = torch.from_numpy(weights("init_sweep", spec.w_stream)["dWq"]).to(dev)
+        dWq = cur[spec.w_stream]
+        ws = torch.empty(W.workspace_size(2, spec.d_out, spec.d_in, spec.p, 0, False), dtype=torch.uint8, device=dev)
+        W.init_alloc(dWq, spec.p, spec.had_block, spec.min_per_row, spec.remainder, ws=ws)
+        ts = []
+        for _ in range(3):
+            ev[0].record()
+            W.init_alloc(dWq, spec.p, spec.had_block, spec.min_per_row, spec.remainder, ws=ws)
+            ev[1].record()
+            torch.cuda.synchronize()
+            ts.append(ev[0].elapsed_time(ev[1]))
+        ms = statistics.median(ts)
+        nbytes = 2 * 4.0 * spec.d_out * spec.d_in + 8.0 * spec.p
+        es = W.energy_stats(dWq, spec.p, spec.had_block).cpu().numpy()
+        shapes[spec.name] = {"ms": ms, "alg_GBps": nbytes / (ms / 1e3) / 1e9, "eta": float(es[0]),
+                             "energy_top_p": float(es[1])}
+        tot_ms += ms
+        tot_bytes += nbytes
+    return {"ms_total": tot_ms, "shapes": shapes, "alg_GBps": tot_bytes / (tot_ms / 1e3) / 1e9,
+            "frac_hbm": tot_bytes / (tot_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "what": ("AdaAlloc (norms, budgets, fp64 transform, per-row top-k) on the 21 init-sweep shapes, 2-bit g64 "
+                     "RTN error; eta / energy_top_p: Hill exponent and energy share of the p largest |dW_Q H|")}
+
+
+def run_diagnostics(W, torch, spec, dWq, e, sel_e):
+    """The selection diagnostics of the q_proj layer: Hill exponent and cumulative energy of |dW_Q H| at k = p, and
+    the row/column counts (rank bound) of E under AdaAlloc, whole-matrix magnitude and random selection."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ws = torch.empty(W.workspace_size(8, spec.d_out, spec.d_in, 0, 0, False), dtype=torch.uint8, device=dWq.device)
+    W.energy_stats(dWq, spec.p, spec.had_block, ws=ws)
+    ts = []
+    for _ in range(3):
+        ev[0].record()
+        es = W.energy_stats(dWq, spec.p, spec.had_block, ws=ws)
+        ev[1].record()
+        torch.cuda.synchronize()
+        ts.append(ev[0].elapsed_time(ev[1]))
+    es = es.cpu().numpy()
+    names = W.api.PATTERN_STATS
+    pats = {}
+    for rule, ee in [("adaalloc", e)] + list(sel_e.items()):
+        st, _ = W.pattern_stats(ee["row_ptr"], ee["col_idx"], spec.d_in)
+        pats[rule] = dict(zip(names, st.cpu().numpy().tolist()))
+    return {"eta": float(es[0]), "energy_top_p": float(es[1]), "energy_ms": statistics.median(ts),
+            "pattern": pats,
+            "what": ("eta: Hill exponent of the p largest |dW_Q H| (smaller = error energy more concentrated); "
+                     "pattern: counts of E per rule, rank_bound = min(non-empty rows, non-empty columns) >= rank(F), "
+                     "half_rows = fewest rows holding half of E")}
+
+
+def run_block(args):
+    """`--workload block`: the decoder-block workload alone (seven LLaMA-3-8B-shaped linears, 32768 tokens, 4-bit
+    g128, r = 64), with and without the shared transform, printed as its own JSON line."""
+    import torch
+
+    import walsh_hadamard_sparse_b200 as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    r = run_stack(W, torch, dev, "block", lambda wl, name: host_weights(next(s for s in CONFIGS[wl] if s.name == name),
+                                                                        args.seed, wl),
+                  args.seed, max(3, min(args.steps, 10)), max(args.warmup, 3), load_peaks(), compare_unshared=True)
     line = {
-        "metric": "decoder block (7 adapted linears) fwd+bwd tokens/s", "value": T / (res[True] / 1e3),
-        "unit": "tokens/s", "n_gpus": 1, "steps": K, "ms_per_step": res[True], "higher_is_better": True,
-        "dtype": "bf16", "data": "synthetic (seeded; weights host-generated, activations drawn on the GPU)",
+        "metric": "decoder block (7 adapted linears) fwd+bwd tokens/s", "value": r["value"], "unit": "tokens/s",
+        "n_gpus": 1, "steps": r["steps"], "ms_per_step": r["ms_per_step"], "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic (seeded; weights host-generated, activations drawn on the GPU)",
         "config": {"workload": "block: LLaMA-3-8B q/k/v/o/gate/up/down, T=32768 (8 x 4096), 4-bit g128, r=64",
                    "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write)"},
         "algorithm": "dense; Z = X H shared by q/k/v and by gate/up (z_given)",
-        "gemm_tflops": flops / (res[True] / 1e3) / 1e12,
-        "without_sharing": {"ms_per_step": res[False], "value": T / (res[False] / 1e3)},
+        "gemm_tflops": r["gemm_tflops"], "without_sharing": r["without_sharing"], "roofline": r["roofline"],
     }
     print(json.dumps(line), flush=True)
 
@@ -362,6 +505,8 @@ def main():
                     help="block: time the decoder-block workload (seven linears) instead of the q_proj step")
     ap.add_argument("--no-init-extras", action="store_true",
                     help="skip timing the selection variants and Value Refinement (one-off setup, not the step)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads (MLP pair, decoder block, init sweep) and the diagnostics")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     spec = CONFIGS[WORKLOAD][0]
@@ -369,6 +514,11 @@ def main():
         return run_block(args)
     if args.impl == "reference":
         return run_reference(args, spec)
+    # the other workloads' weights are generated on the host while the GPU measures the headline (one GPU only;
+    # the worker processes are spawned before the first CUDA call)
+    pool = None
+    if not args.no_workloads and int(os.environ.get("WORLD_SIZE", "1")) == 1:
+        pool = WeightPool(args.seed, max(1, min(8, (os.cpu_count() or 2) - 1)))
 
     import torch
     import torch.distributed as dist
@@ -411,10 +561,10 @@ def main():
         torch.cuda.synchronize()
         init_ms.append(ev[0].elapsed_time(ev[1]))
     # the pages' alternatives to AdaAlloc (whole-matrix magnitude top-p, seeded random E), timed the same way
-    sel_ms = {}
+    sel_ms, sel_e = {}, {}
     for sel in (() if args.no_init_extras else ("magnitude", "random")):
         sws = torch.empty(W.workspace_size(6, spec.d_out, spec.d_in, spec.p, 0, False), dtype=torch.uint8, device=dev)
-        W.init_select_global(dWq, spec.p, spec.had_block, sel, 1, ws=sws)
+        sel_e[sel] = W.init_select_global(dWq, spec.p, spec.had_block, sel, 1, ws=sws)
         torch.cuda.synchronize()
         ts = []
         for _ in range(3):
@@ -561,6 +711,13 @@ def main():
     roofline, launches = head["roofline"], head["launches"]
     step = make_step("dense")
 
+    # the host generation of the other workloads' weights is over before the host-link and host-core legs
+    weights = {}
+    if pool is not None:
+        for key, f in pool.fut.items():
+            weights[key] = f.result()
+        pool.close()
+
     # ---- end to end through host buffers: every step copies its X and dY in from pinned host memory and reads
     # its dc back; the copy of step i+1's inputs (on a copy stream, into the other of two device buffers) runs
     # while step i computes, as an input pipeline would.
@@ -632,6 +789,24 @@ def main():
                "sample": f"{toks} tokens of the same layer (Y, dX for them; dc over all {spec.p} coefficients), "
                          f"{dt:.1f} s of host time"}
 
+    # ---- the other workloads (one GPU): the LLaMA-3-8B MLP pair, the decoder block, the init sweep; and the
+    # selection diagnostics of the q_proj layer
+    extra = {}
+    if weights:
+        del Z, Y, dX, ws, adapters, flush
+        torch.cuda.empty_cache()
+        get = lambda wl, name: weights[(wl, name)]  # noqa: E731
+        extra["mlp"] = run_stack(W, torch, dev, "mlp", get, args.seed, 10, 3, peaks)
+        extra["mlp"]["what"] = ("LLaMA-3-8B MLP: gate and up 4096 -> 14336 (one shared Z), down 14336 -> 4096 "
+                                "(seven 2048-point blocks), 16384 tokens, 3-bit g128, r = 64, dense, fwd + bwd")
+        extra["block"] = run_stack(W, torch, dev, "block", get, args.seed, 5, 3, peaks, compare_unshared=True)
+        extra["block"]["what"] = ("LLaMA-3-8B decoder block, 7 adapted linears (q, k, v share Z; gate, up share Z), "
+                                  "32768 tokens, 4-bit g128, r = 64, dense, fwd + bwd")
+        extra["init_sweep"] = run_init_sweep(W, torch, dev, get, peaks)
+        diagnostics = run_diagnostics(W, torch, spec, dWq, e, sel_e) if sel_e else None
+    else:
+        diagnostics = None
+
     init_bytes = 2 * 4.0 * spec.d_in * spec.d_out + 8.0 * spec.p
     init_med = statistics.median(init_ms)
     sp = results["sparse"]
@@ -664,6 +839,8 @@ def main():
                        "roofline": sp["roofline"], "gpu_launches": sp["launches"], "kernels": sp["kernels"],
                        "what": "segment SpMM over CSR, tiled SDDMM, CSC gather on the FMA units; base GEMMs on tcgen05"},
         },
+        "workloads": extra or None,
+        "diagnostics": diagnostics,
         "init": {"ms": init_med, "alg_GBps": init_bytes / (init_med / 1e3) / 1e9,
                  "frac_hbm": init_bytes / (init_med / 1e3) / 1e9 / peaks["hbm_gbs"],
                  "what": "AdaAlloc on dW_Q (4096 x 4096 fp32): norms, budgets, fp64 transform, top-k; one-off per layer",
