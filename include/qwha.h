@@ -395,9 +395,10 @@ qwha_status qwha_stage_report(int64_t *calls, int64_t *launches, double *ms);
  * 2000000000, i.e. 2 s). A wait that gives up sets the device error word and
  * its CTA exits after letting its own copies already in flight land (those
  * drain waits keep the fixed 2 s bound); the call's output is then incomplete
- * and qwha_check_stream_status reports QWHA_ERR_TIMEOUT. A bound of 0 makes a
- * wait give up soon after its first unsuccessful poll. Not thread-safe with
- * respect to calls in flight on other threads.
+ * and qwha_check_stream_status reports QWHA_ERR_TIMEOUT. A bound of 0 makes
+ * every such wait give up at once, without polling, so the give-up path runs
+ * whatever the timing. Not thread-safe with respect to calls in flight on
+ * other threads.
  *
  * qwha_debug_fail_cuda_checks(n) makes the next n checks of a successful CUDA
  * runtime result inside the library (launches, memsets, copies) report

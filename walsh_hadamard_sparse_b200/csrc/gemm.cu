@@ -6,13 +6,19 @@
 // The adapter term rides in the epilogue, so it costs one fp32 read.
 //
 // Structure (persistent; one CTA per SM, or one CTA pair per two SMs):
-//   warp 0, one thread : TMA producer. 2-D tensor copies (128B swizzle, no
+//   warp 0, one thread : TMA producer. Tensor copies (128B swizzle, no
 //                        multicast) of A and B k-blocks of 64 into a shared-
 //                        memory ring, completion counted in bytes on the
 //                        stage's "full" mbarrier. An operand may be K-major
-//                        (one box of rows x 64 K) or MN-major (64 x 64 boxes
-//                        along MN); the UMMA descriptors and the instruction
-//                        descriptor's major bits follow.
+//                        (one 2-D box of rows x 64 K) or MN-major: one 3-D
+//                        box that fills the stage's 64 x 64 slabs along MN
+//                        at once (the operand seen as 64 MN elements x K x
+//                        MN / 64 slabs), or, when MN is not a multiple of
+//                        64, one 2-D box per slab. Fewer, larger copies keep
+//                        the tensor pipe fed: the measured cost of an
+//                        MN-major operand fell from ~10% to nothing. The
+//                        UMMA descriptors and the instruction descriptor's
+//                        major bits follow the layout.
 //   warp 1, one thread : MMA issuer. tcgen05.mma kind::f16 (bf16 x bf16 ->
 //                        fp32), K=16 per instruction, accumulator in TMEM;
 //                        tcgen05.commit frees the stage ("empty") and, after
@@ -50,7 +56,7 @@
 namespace qwha {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64;  // accumulator rows per CTA, tile columns, k-block
+constexpr int BM = 128, BN = 256;  // accumulator rows per CTA, tile columns
 constexpr int kGemmThreads = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int kEpiStride = 33;  // per-warp staging row (floats) of the sampled epilogue
@@ -71,9 +77,21 @@ constexpr size_t z_smem() {
            ((size_t)Geo<kZ, 8>::NP * sizeof(float) + (size_t)(1u << kZ) * sizeof(__nv_bfloat16));
 }
 
+// How an operand's stage is filled (64-wide slabs of 128-byte rows, 128B swizzle):
+enum {
+  kLdK2d = 0,   // K-major, one 2-D box of rows x 64 K per slab of K (BK / 64 copies)
+  kLdMn2d = 1,  // MN-major, one 2-D box of BK x 64 MN per slab of MN
+  kLdMn3d = 2,  // MN-major, one 3-D box (64 MN, BK, slabs): the whole stage in one copy (MN % 64 == 0)
+  kLdK3d = 3    // K-major, one 3-D box (64 K, rows, BK / 64 slabs): the whole stage in one copy (K % 64 == 0)
+};
+__host__ __device__ constexpr bool ld_mn(int mode) { return mode == kLdMn2d || mode == kLdMn3d; }
+
 template <int CG, int kMode = kOutBf16, int kZ = 0>
 struct Cfg {
-  static constexpr int kStages = CG == 1 ? 4 : (kZ ? 5 : 6);
+  // k-block depth: 128 for the CTA pair (half the copies and barrier rounds per MMA of 64), 64 when the fused
+  // transform's buffers or the single CTA's 256-row B leave room for too few 128-deep stages
+  static constexpr int BK = (CG == 2 && kZ == 0) ? 128 : 64;
+  static constexpr int kStages = CG == 1 ? 4 : (kZ ? 5 : 3);
   static constexpr uint32_t kABytes = BM * BK * 2;
   static constexpr int kBRows = BN / CG;  // rows of B this CTA loads
   static constexpr uint32_t kBBytes = kBRows * BK * 2;
@@ -173,6 +191,42 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
   }
 }
 
+// 3-D tensor copy (same rules as tma_load_2d): fills box[0] x box[1] x box[2]
+// elements, the last dimension slowest, in shared memory.
+template <int CG>
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y, int z) {
+  if constexpr (CG == 1) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+  }
+}
+
+// One k-block of an operand into its stage (see the kLd* modes): `rows`
+// M or N rows starting at `row`, K from kb * BK.
+template <int CG, int BK>
+__device__ __forceinline__ void load_stage(uint32_t dst, const CUtensorMap *map, uint32_t bar, int mode, int row,
+                                           int rows, int kb) {
+  if (mode == kLdK3d) {
+    tma_load_3d<CG>(dst, map, bar, 0, row, kb * (BK / 64));
+  } else if (mode == kLdMn3d) {
+    tma_load_3d<CG>(dst, map, bar, 0, kb * BK, row / 64);
+  } else if (mode == kLdMn2d) {
+    for (int h = 0; h < rows / 64; ++h) tma_load_2d<CG>(dst + h * (BK * 128), map, bar, row + 64 * h, kb * BK);
+  } else {
+#pragma unroll
+    for (int s = 0; s < BK / 64; ++s) tma_load_2d<CG>(dst + s * (rows * 128), map, bar, kb * BK + 64 * s, row);
+  }
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -203,12 +257,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+template <int BK>
 __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr) {
-  // MN-major: the stage holds 64(MN) x 64(K) boxes of 8 KB each, rows of 128 B
-  // along MN, one box after the other along MN. LBO = 8 KB (next 64 MN
-  // elements), SBO = 1024 B (next 8 K rows), version 1, SWIZZLE_128B.
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(8192 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+  // MN-major: the stage holds slabs of 64(MN) x BK(K), rows of 128 B along MN,
+  // one slab after the other along MN. LBO = BK x 128 B (next 64 MN elements),
+  // SBO = 1024 B (next 8 K rows), version 1, SWIZZLE_128B.
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((BK * 128) >> 4) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
 template <int CG>
@@ -294,18 +349,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
 }
 
 // kF32Out: write fp32 D (no rounding); otherwise bf16. addend may be NULL.
-// a_mn / b_mn: the operand is MN-major in global memory ([K rows][M or N
-// contiguous]); its stage is then filled by BM/64 or BN/64 boxes of 64 x 64.
+// a_ld / b_ld: how the operand's stage is filled (kLd*): K-major in global
+// memory ([M or N rows][K contiguous]) or MN-major ([K rows][M or N
+// contiguous]); a stage holds slabs of 128-byte rows (64 K per slab along K
+// for K-major, BK K rows per slab of 64 MN for MN-major), filled by one 3-D
+// copy when the slab dimension divides evenly, else by one 2-D copy per slab.
 // k_splits > 1 (sampled output only): each tile's K range is cut into that
-// many parts, each part a separate work unit adding its share into dc.
+// many parts, each part a separate work unit adding its share into dc. Units
+// are numbered part-major (unit = part * tiles + tile), so the units running
+// at the same time read the same part of K and share it in L2.
 template <int kMode, int CG, int kZ>
 __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const float *__restrict__ addend, void *__restrict__ out_v, int M, int N, int K,
-                             int a_mn, int b_mn, int group_m, int k_splits, SampleArgs sa_args, ZArgs za,
+                             int a_ld, int b_ld, int group_m, int k_splits, SampleArgs sa_args, ZArgs za,
                              unsigned int *err) {
   using C = Cfg<CG, kMode, kZ>;
   constexpr int STAGES = C::kStages;
+  constexpr int BK = C::BK;
+  const bool a_mn = ld_mn(a_ld), b_mn = ld_mn(b_ld);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t base = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
@@ -377,7 +439,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     int last_parity[STAGES];
     for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
     for (int unit = group_id; unit < num_units && !*abort_flag; unit += n_groups) {
-      const int tile = unit / k_splits, split = unit % k_splits;
+      const int tile = unit % num_tiles, split = unit / num_tiles;
       int m_blk, n_blk;
       tile_coords(tile, m_blk, n_blk);
       const int a_row = m_blk * TM + (int)rank * BM;
@@ -393,18 +455,8 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         if (leader) mbar_expect_tx(full(stage), C::kStageBytes * CG);
         const uint32_t fb = CG == 2 ? peer_addr(full(stage), 0) : full(stage);
         const uint32_t sa = base + stage * C::kStageBytes, sb = sa + C::kABytes;
-        if (a_mn) {
-#pragma unroll
-          for (int h = 0; h < BM / 64; ++h) tma_load_2d<CG>(sa + h * 8192, &tmA, fb, a_row + 64 * h, kb * BK);
-        } else {
-          tma_load_2d<CG>(sa, &tmA, fb, kb * BK, a_row);
-        }
-        if (b_mn) {
-#pragma unroll
-          for (int h = 0; h < C::kBRows / 64; ++h) tma_load_2d<CG>(sb + h * 8192, &tmB, fb, b_row + 64 * h, kb * BK);
-        } else {
-          tma_load_2d<CG>(sb, &tmB, fb, kb * BK, b_row);
-        }
+        load_stage<CG, BK>(sa, &tmA, fb, a_ld, a_row, BM, kb);
+        load_stage<CG, BK>(sb, &tmB, fb, b_ld, b_row, C::kBRows, kb);
         last_parity[stage] = (int)phase;
         if (++stage == STAGES) {
           stage = 0;
@@ -423,7 +475,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     uint32_t phase = 0;
     int it = 0;
     for (int unit = group_id; unit < num_units && !*abort_flag; unit += n_groups, ++it) {
-      const int split = unit % k_splits;
+      const int split = unit / num_tiles;
       const int kb0 = split * kb_per_split, kb1 = min(k_blocks, kb0 + kb_per_split);
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
@@ -442,14 +494,17 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         }
         tc_fence_after();
         const uint32_t sa = base + stage * C::kStageBytes, sb = sa + C::kABytes;
-        const uint64_t da = a_mn ? sw128_desc_mn(sa) : sw128_desc(sa);
-        const uint64_t db = b_mn ? sw128_desc_mn(sb) : sw128_desc(sb);
-        // next 16 of K: +32 B inside the 128 B rows (K-major), +2 KB = 16 rows (MN-major)
-        const uint64_t sta = a_mn ? 128ull : 2ull, stb = b_mn ? 128ull : 2ull;
         const uint32_t idesc = C::kIdesc | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          umma_bf16<CG>(d_tmem, da + sta * k, db + stb * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < BK / 16; ++k) {
+          // next 16 of K: K-major +32 B inside the 128 B rows, the next slab (rows x 128 B) every 64;
+          // MN-major +2 KB (16 rows of 128 B)
+          const uint64_t da = a_mn ? sw128_desc_mn<BK>(sa) + 128ull * k
+                                   : sw128_desc(sa + (uint32_t)(k >> 2) * (BM * 128)) + 2ull * (k & 3);
+          const uint64_t db = b_mn ? sw128_desc_mn<BK>(sb) + 128ull * k
+                                   : sw128_desc(sb + (uint32_t)(k >> 2) * (C::kBRows * 128)) + 2ull * (k & 3);
+          umma_bf16<CG>(d_tmem, da, db, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+        }
         umma_commit_all<CG>(empty(stage));
         if (++stage == STAGES) {
           stage = 0;
@@ -476,7 +531,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     int it = 0;
     float *my_stage = epi_stage + (warp - 2) * (kMode == kOutSampled ? 32 * kEpiStride : 512);
     for (int unit = group_id; unit < num_units; unit += n_groups, ++it) {
-      const int tile = unit / k_splits;
+      const int tile = unit % num_tiles;
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (*abort_flag) break;
@@ -640,6 +695,36 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, uint3
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A K-major operand [rows, K] seen as a 3-D tensor (64 K elements, rows,
+// K / 64 slabs of 128 B), box (64, box_rows, nslab): one copy fills nslab
+// slabs of box_rows x 128 B, one after the other. Requires K % 64 == 0.
+bool make_map_k3d(CUtensorMap *m, const void *ptr, int64_t rows, int64_t K, uint32_t box_rows, uint32_t nslab) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || K % 64) return false;
+  const cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(K / 64)};
+  const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128u};
+  const cuuint32_t box[3] = {64u, box_rows, nslab};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// An MN-major operand [K, MN] seen as a 3-D tensor (64 MN elements, K rows,
+// MN / 64 slabs of 128 B), box (64, bk, nslab): one copy fills nslab slabs of
+// bk x 128 B (one after the other). Requires MN % 64 == 0.
+bool make_map_mn3d(CUtensorMap *m, const void *ptr, int64_t K, int64_t MN, uint32_t bk, uint32_t nslab) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || MN % 64) return false;
+  const cuuint64_t dims[3] = {64u, (cuuint64_t)K, (cuuint64_t)(MN / 64)};
+  const cuuint64_t strides[2] = {(cuuint64_t)MN * 2, 128u};
+  const cuuint32_t box[3] = {64u, bk, nslab};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Co-resident CTA groups of the CG variant (one CTA per SM; pairs need two SMs
 // of one cluster slot).
 template <int kMode, int CG, int kZ>
@@ -678,9 +763,22 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
                            const ZArgs &za = ZArgs{}) {
   using C = Cfg<CG, kMode, kZ>;
   CUtensorMap ta, tb;
-  const bool ok_a = a_mn ? make_map(&ta, A, K, M, 64) : make_map(&ta, A, M, K, BM);
-  const bool ok_b = b_mn ? make_map(&tb, B, K, N, 64) : make_map(&tb, B, N, K, C::kBRows);
-  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+  constexpr int BK = C::BK;
+  // one 3-D copy per operand and stage where the slab dimension divides evenly, else one 2-D copy per slab
+  auto mode = [&](bool mn, int64_t MN) {
+    if (mn) return MN % 64 == 0 ? (int)kLdMn3d : (int)kLdMn2d;
+    return (BK > 64 && K % 64 == 0) ? (int)kLdK3d : (int)kLdK2d;
+  };
+  const int a_ld = mode(a_mn, M), b_ld = mode(b_mn, N);
+  auto map = [&](CUtensorMap *t, const void *P, int ld, int64_t MN, uint32_t rows) {
+    switch (ld) {
+      case kLdK3d: return make_map_k3d(t, P, MN, K, rows, BK / 64);
+      case kLdMn3d: return make_map_mn3d(t, P, K, MN, BK, rows / 64);
+      case kLdMn2d: return make_map(t, P, K, MN, BK);
+      default: return make_map(t, P, MN, K, rows);
+    }
+  };
+  if (!map(&ta, A, a_ld, M, BM) || !map(&tb, B, b_ld, N, C::kBRows)) return cudaErrorInvalidValue;
   auto kern = gemm_bf16_tcgen05_kernel<kMode, CG, kZ>;
   static bool attr[64] = {};  // per device
   bool &attr_done = attr[device_slot()];
@@ -705,7 +803,7 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
   // wave of groups mostly idle (each dc then receives exactly two additions
   // onto zero, whose result does not depend on their order).
   int k_splits = 1;
-  if (kMode == kOutSampled && cdiv(K, BK) >= 8) {
+  if (kMode == kOutSampled && cdiv(K, BK) >= 4) {
     const double waves1 = (double)tiles / groups, waves2 = 2.0 * tiles / groups;
     const double eff1 = waves1 / std::ceil(waves1), eff2 = waves2 / std::ceil(waves2);
     if (eff2 > eff1 + 0.02) k_splits = 2;
@@ -729,7 +827,7 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = CG > 1 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, addend, out, (int)M, (int)N, (int)K, a_mn ? 1 : 0, b_mn ? 1 : 0,
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, addend, out, (int)M, (int)N, (int)K, a_ld, b_ld,
                             (int)group_m, k_splits, sa, za, device_error_word());
 }
 

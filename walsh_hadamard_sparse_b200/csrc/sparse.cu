@@ -590,6 +590,164 @@ __global__ void __launch_bounds__(kSddmmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- SDDMM, bf16 activations
+//
+// The bf16 path keeps the staged sub-tiles in bf16: 64 tokens (128 B) per row
+// of s[row][token], half the shared bytes per product of a widened fp32 tile,
+// and multiplies with fma.rn.f32.bf16 (bf16 x bf16 -> fp32 accumulate; the
+// product of two bf16 values is exact in fp32, so only the summation order
+// differs from the fp32 kernel). The 16-byte chunk c (tokens 8c .. 8c+7) of
+// row r sits at chunk position c ^ ((r & 3) << 1), which keeps the chunk's
+// parity. Lane q of a slot holds tokens 16q .. 16q+15 (chunks 2q, 2q+1) and
+// reads the chunk of its slot's parity first: the two slots of a quarter warp
+// then meet 8 distinct chunk positions whatever their rows, and so do their
+// second reads. Staging: cp.async copies the sub-tile raw (16-byte pieces,
+// [operand][row chunk][token], zero-filled past the edges); once it has landed
+// every thread transposes its pieces into the swizzled layout (a warp writes
+// 64 contiguous bytes of one row per store), and the copy of the next
+// sub-tile is issued into the raw buffer while this one is multiplied.
+constexpr int kSdd16TT = 64;  // tokens per staged sub-tile (bf16)
+constexpr int kSdd16E = 18;   // entries per slot and pass
+
+constexpr size_t sddmm16_smem() {
+  return 2ull * QWHA_TILE * kSdd16TT * 2 /* transposed dY, Z */ + 2ull * QWHA_TILE * kSdd16TT * 2 /* raw */;
+}
+
+// byte offset of (row r, token t) in a transposed operand
+__device__ __forceinline__ uint32_t sdd16_off(int r, int t) {
+  return (uint32_t)r * (kSdd16TT * 2) + ((uint32_t)((t >> 3) ^ ((r & 3) << 1)) << 4) + (uint32_t)(t & 7) * 2;
+}
+
+__device__ __forceinline__ float dot8_bf16(const uint4 y, const uint4 z, float acc) {
+  acc = fma_bf16_lo(y.x, z.x, acc);
+  acc = fma_bf16_hi(y.x, z.x, acc);
+  acc = fma_bf16_lo(y.y, z.y, acc);
+  acc = fma_bf16_hi(y.y, z.y, acc);
+  acc = fma_bf16_lo(y.z, z.z, acc);
+  acc = fma_bf16_hi(y.z, z.z, acc);
+  acc = fma_bf16_lo(y.w, z.w, acc);
+  acc = fma_bf16_hi(y.w, z.w, acc);
+  return acc;
+}
+
+__global__ void __launch_bounds__(kSddmmThreads, 1)
+    sddmm_bf16_kernel(const __nv_bfloat16 *__restrict__ dY, const __nv_bfloat16 *__restrict__ Z, int64_t T_,
+                      int d_out, int d_in, const int32_t *__restrict__ tile_ptr, const int32_t *__restrict__ tile_pos,
+                      const int32_t *__restrict__ tile_rk, int n_rb, int64_t chunk_tokens, int64_t p,
+                      float *__restrict__ partial) {
+  constexpr int E = kSdd16E;
+  constexpr int kPass = kSddmmSlots * E;
+  constexpr int kRowBytes = kSdd16TT * 2;
+  constexpr int kOpBytes = QWHA_TILE * kRowBytes;      // one transposed operand
+  constexpr int kPieces = QWHA_TILE / 8 * kSdd16TT;    // 16-byte raw pieces per operand
+  constexpr int kItems = 2 * kPieces / kSddmmThreads;  // pieces per thread and sub-tile
+  extern __shared__ __align__(16) unsigned char sdd16_smem[];
+  unsigned char *s_dy = sdd16_smem;
+  unsigned char *s_z = sdd16_smem + kOpBytes;
+  uint4 *raw = reinterpret_cast<uint4 *>(sdd16_smem + 2 * kOpBytes);  // [operand][row chunk][token]
+  const int tile = blockIdx.x;
+  const int rb = tile % n_rb, kb = tile / n_rb;
+  const int r0 = rb * QWHA_TILE, k0 = kb * QWHA_TILE;
+  const int r_len = min(QWHA_TILE, d_out - r0), k_len = min(QWHA_TILE, d_in - k0);
+  int64_t e_begin = tile_ptr[tile], e_end = tile_ptr[tile + 1];
+  if (e_begin < 0) e_begin = 0;
+  if (e_end > p) e_end = p;
+  const int64_t c = blockIdx.y;
+  const int64_t ta = c * chunk_tokens, tb = (ta + chunk_tokens < T_) ? ta + chunk_tokens : T_;
+  float *part = partial + c * p;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = lane & 3, slot = warp * 8 + (lane >> 2);
+  const int par = slot & 1;
+
+  auto copy = [&](int64_t t0) {
+#pragma unroll 2
+    for (int u = 0; u < kItems; ++u) {
+      const int it = threadIdx.x + u * kSddmmThreads;
+      const int which = it >= kPieces;
+      const int w = it - which * kPieces;
+      const int t = w % kSdd16TT, ch = w / kSdd16TT;
+      const int64_t tg = t0 + t;
+      const int len = which ? k_len : r_len;
+      const bool in = tg < tb && ch * 8 < len;
+      const __nv_bfloat16 *src = in ? (which ? Z + tg * d_in + k0 + ch * 8 : dY + tg * d_out + r0 + ch * 8) : dY;
+      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(raw + it));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(in ? 16 : 0)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  auto transpose = [&]() {
+#pragma unroll
+    for (int u = 0; u < kItems; ++u) {
+      const int it = threadIdx.x + u * kSddmmThreads;
+      const int which = it >= kPieces;
+      const int w = it - which * kPieces;
+      const int t = w % kSdd16TT, ch = w / kSdd16TT;
+      const uint4 v = raw[it];
+      unsigned char *dst = which ? s_z : s_dy;
+      const uint32_t h[8] = {v.x & 0xffffu, v.x >> 16, v.y & 0xffffu, v.y >> 16,
+                             v.z & 0xffffu, v.z >> 16, v.w & 0xffffu, v.w >> 16};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) *reinterpret_cast<unsigned short *>(dst + sdd16_off(ch * 8 + i, t)) = (unsigned short)h[i];
+    }
+  };
+
+  for (int64_t eb = e_begin; eb < e_end; eb += kPass) {
+    const int64_t my0 = eb + (int64_t)slot * E;
+    // per entry, fixed over the token range: the byte offsets of this lane's first dY and Z chunks (dY high
+    // half, Z low half; an unused entry reads row 0 and is not stored), whether its column differs from the
+    // previous one's, and whether it is in use
+    uint32_t off[E];
+    uint32_t newcol = 0, valid = 0;
+    float acc[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const int64_t e = my0 + i;
+      const int v = e < e_end ? tile_rk[e] : -1;
+      const int r_ = (v >> 16) & 0xffff, k_ = v & 0xffff;
+      const bool ok = e < e_end && v >= 0 && r_ < r_len && k_ < k_len;
+      const int rr = ok ? r_ : 0, kk = ok ? k_ : 0;
+      const int t_first = 16 * q + 8 * par;
+      off[i] = (sdd16_off(rr, t_first) << 16) | sdd16_off(kk, t_first);
+      if (i == 0 || (off[i] & 0xffffu) != (off[i - 1] & 0xffffu)) newcol |= 1u << i;
+      if (ok) valid |= 1u << i;
+      acc[i] = 0.f;
+    }
+    if (ta < tb) copy(ta);
+    for (int64_t t0 = ta; t0 < tb; t0 += kSdd16TT) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();  // this sub-tile's raw pieces have landed; the previous one is multiplied
+      transpose();
+      __syncthreads();
+      if (t0 + kSdd16TT < tb) copy(t0 + kSdd16TT);  // the raw buffer is free again
+      uint4 z0 = make_uint4(0, 0, 0, 0), z1 = z0;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if (newcol & (1u << i)) {
+          const uint32_t oz = off[i] & 0xffffu;
+          z0 = *reinterpret_cast<const uint4 *>(s_z + oz);
+          z1 = *reinterpret_cast<const uint4 *>(s_z + (oz ^ 16u));  // the lane's other chunk: parity flipped
+        }
+        const uint32_t oy = off[i] >> 16;
+        const uint4 y0 = *reinterpret_cast<const uint4 *>(s_dy + oy);
+        const uint4 y1 = *reinterpret_cast<const uint4 *>(s_dy + (oy ^ 16u));
+        acc[i] = dot8_bf16(y1, z1, dot8_bf16(y0, z0, acc[i]));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      float sum = acc[i];
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      if (q == 0 && (valid & (1u << i))) {
+        const int j = tile_pos[my0 + i];
+        if ((uint64_t)j < (uint64_t)p) part[j] = sum;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 __global__ void sddmm_reduce_kernel(const float *__restrict__ partial, int n_chunks, int64_t p, float alpha,
                                     float *__restrict__ dc) {
   for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < p; j += (int64_t)gridDim.x * blockDim.x) {
@@ -650,17 +808,17 @@ cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T
   const int n_rb = (int)cdiv(d_out, QWHA_TILE);
   const int64_t tiles = n_rb * cdiv(d_in, QWHA_TILE);
   const int n_chunks = sddmm_chunks(T, d_out, d_in);
-  const int64_t chunk_tokens = cdiv(cdiv(T, n_chunks), 32) * 32;
+  const int64_t chunk_tokens = cdiv(cdiv(T, n_chunks), 64) * 64;
   cudaError_t e = cudaMemsetAsync(partial, 0, (size_t)n_chunks * p * sizeof(float), s);
   if (e != cudaSuccess) return e;
   if (T > 0) {
     dim3 grid((unsigned)tiles, (unsigned)n_chunks);
-    const size_t smem = dt == QWHA_BF16 ? sddmm_smem<__nv_bfloat16>() : sddmm_smem<float>();
-    e = cudaFuncSetAttribute(dt == QWHA_BF16 ? (const void *)sddmm_kernel<__nv_bfloat16> : (const void *)sddmm_kernel<float>,
+    const size_t smem = dt == QWHA_BF16 ? sddmm16_smem() : sddmm_smem<float>();
+    e = cudaFuncSetAttribute(dt == QWHA_BF16 ? (const void *)sddmm_bf16_kernel : (const void *)sddmm_kernel<float>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (dt == QWHA_BF16)
-      sddmm_kernel<__nv_bfloat16><<<grid, kSddmmThreads, smem, s>>>(
+      sddmm_bf16_kernel<<<grid, kSddmmThreads, smem, s>>>(
           static_cast<const __nv_bfloat16 *>(dY), static_cast<const __nv_bfloat16 *>(Z), T, d_out, d_in, tile_ptr,
           tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
     else
