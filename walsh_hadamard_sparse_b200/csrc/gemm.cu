@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
   using C = Cfg<CG, kMode, kZ>;
   constexpr int STAGES = C::kStages;
   constexpr int BK = C::BK;
-  const bool a_mn = ld_mn(a_ld), b_mn = ld_mn(b_ld);
+  const bool a_mn = kZ ? false : ld_mn(a_ld), b_mn = kZ ? false : ld_mn(b_ld);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t base = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
@@ -455,8 +455,16 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         if (leader) mbar_expect_tx(full(stage), C::kStageBytes * CG);
         const uint32_t fb = CG == 2 ? peer_addr(full(stage), 0) : full(stage);
         const uint32_t sa = base + stage * C::kStageBytes, sb = sa + C::kABytes;
-        load_stage<CG, BK>(sa, &tmA, fb, a_ld, a_row, BM, kb);
-        load_stage<CG, BK>(sb, &tmB, fb, b_ld, b_row, C::kBRows, kb);
+        if constexpr (kZ != 0) {
+          // The fused forward reads both operands K-major in 64-deep blocks. Its binary holds only
+          // this path: with the generic one compiled in as well, the launch (four warp roles, the
+          // transform's unrolled butterflies among them) ran ~10% slower.
+          tma_load_2d<CG>(sa, &tmA, fb, kb * BK, a_row);
+          tma_load_2d<CG>(sb, &tmB, fb, kb * BK, b_row);
+        } else {
+          load_stage<CG, BK>(sa, &tmA, fb, a_ld, a_row, BM, kb);
+          load_stage<CG, BK>(sb, &tmB, fb, b_ld, b_row, C::kBRows, kb);
+        }
         last_parity[stage] = (int)phase;
         if (++stage == STAGES) {
           stage = 0;
@@ -494,16 +502,18 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         }
         tc_fence_after();
         const uint32_t sa = base + stage * C::kStageBytes, sb = sa + C::kABytes;
+        // The descriptors of the stage once; the k-th MMA adds a constant to the start-address field
+        // (address >> 4, 14 bits: shared addresses stay below 256 KB, so nothing carries out of it):
+        // K-major +32 B per 16 of K inside the 128 B rows and the next slab (rows x 128 B) every 64 of K;
+        // MN-major +2 KB (16 rows of 128 B) per 16 of K.
+        const uint64_t da = a_mn ? sw128_desc_mn<BK>(sa) : sw128_desc(sa);
+        const uint64_t db = b_mn ? sw128_desc_mn<BK>(sb) : sw128_desc(sb);
         const uint32_t idesc = C::kIdesc | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k) {
-          // next 16 of K: K-major +32 B inside the 128 B rows, the next slab (rows x 128 B) every 64;
-          // MN-major +2 KB (16 rows of 128 B)
-          const uint64_t da = a_mn ? sw128_desc_mn<BK>(sa) + 128ull * k
-                                   : sw128_desc(sa + (uint32_t)(k >> 2) * (BM * 128)) + 2ull * (k & 3);
-          const uint64_t db = b_mn ? sw128_desc_mn<BK>(sb) + 128ull * k
-                                   : sw128_desc(sb + (uint32_t)(k >> 2) * (C::kBRows * 128)) + 2ull * (k & 3);
-          umma_bf16<CG>(d_tmem, da, db, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          const uint64_t oa = a_mn ? 128ull * k : (uint64_t)((k >> 2) * (BM * 128 / 16) + 2 * (k & 3));
+          const uint64_t ob = b_mn ? 128ull * k : (uint64_t)((k >> 2) * (C::kBRows * 128 / 16) + 2 * (k & 3));
+          umma_bf16<CG>(d_tmem, da + oa, db + ob, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
         }
         umma_commit_all<CG>(empty(stage));
         if (++stage == STAGES) {
