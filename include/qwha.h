@@ -349,7 +349,10 @@ qwha_status qwha_plan_build(int32_t d_out, int32_t d_in, int64_t p, const int32_
  * current, so it must come before any stream capture; the lookup is cached
  * per context, so a context created later, e.g. after cudaDeviceReset, gets
  * a fresh one. The result is bit for bit the dc of qwha_adapter_bwd with the
- * sparse algorithm (same kernels, same summation order). */
+ * sparse algorithm: for bf16 with 16-byte aligned rows that call feeds its
+ * kernel with transposed copies of dY and Z kept in its workspace, while this
+ * entry point stages and transposes the slices inside its kernel; the two
+ * kernels share the multiply-add code, the tiles, chunks and summation order. */
 qwha_status qwha_coef_grad_noalloc(const qwha_adapter *a, qwha_dtype dt, const void *dY, const void *Z,
                                    int64_t T, float alpha, float *dc, void *stream);
 

@@ -5,6 +5,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -363,9 +364,15 @@ size_t bwd_dense_ws(int32_t d_out, int32_t d_in, int64_t T) {
   return align_up((size_t)d_out * d_in * 2, 256);  // W_eff (unless the adapter carries one)
 }
 
+// The sparse backward's dZ buffer, which first holds the transposed dY and Z
+// of the coefficient gradient (the gather writes dZ after the gradient has run).
+size_t dz_region(int32_t d_out, int32_t d_in, int64_t T) {
+  return std::max(align_up((size_t)T * d_in * 4, 256), sddmm_transposed_bytes(T, d_out, d_in));
+}
+
 size_t bwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
   size_t n = align_up((size_t)kSddmmMaxChunks * (size_t)(p > 0 ? p : 1) * 4, 256);
-  n += align_up((size_t)T * d_in * 4, 256);  // dZ
+  n += dz_region(d_out, d_in, T);  // dZ, and before it the transposed dY and Z of the gradient
   n += ent_bytes(p);  // CSC entries in gather order
   if (base) n += align_up((size_t)T * d_in * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
   return n;
@@ -551,13 +558,13 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   if (dense) return dense_bwd(a, wq, dY, Z, T, alpha, dc, dX, ws, s);
   Carver cv(ws);
   float *partial = static_cast<float *>(cv.take((size_t)kSddmmMaxChunks * (size_t)(a->p > 0 ? a->p : 1) * 4));
-  float *dz = static_cast<float *>(cv.take((size_t)T * a->d_in * 4));
+  float *dz = static_cast<float *>(cv.take(dz_region(a->d_out, a->d_in, T)));
   int2 *ent = static_cast<int2 *>(cv.take(ent_bytes(a->p)));
   cudaError_t e = cudaSuccess;
   if (dc) {
     StageScope sc(ST_SDDMM, 2, s);
     e = launch_sddmm(dt, dY, Z, T, a->d_out, a->d_in, a->tile_ptr, a->tile_pos, a->tile_rk, a->p, alpha, partial, dc,
-                     s);
+                     s, dz);
   }
   if (e != cudaSuccess) return cuda_status(e, "sddmm");
   if (!dX || T == 0) return QWHA_OK;

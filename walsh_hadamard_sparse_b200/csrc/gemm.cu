@@ -886,6 +886,19 @@ cudaError_t launch_gemm_fwd_fused(const void *X, const void *W, void *Y, int64_t
   return launch_gemm_cg<kOutBf16, 2, 11>(X, W, nullptr, Y, T, d_out, d_in, false, false, SampleArgs{}, s, za);
 }
 
+bool make_map_rows(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, int64_t ld, uint32_t box_cols,
+                   uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || (ld * 2) % 16 || (reinterpret_cast<uintptr_t>(ptr) & 15)) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm_sampled(const void *A, bool a_mn, const void *B, bool b_mn, int64_t M, int64_t N, int64_t K,
                                 const int32_t *row_ptr, const int32_t *col_idx, int64_t p, float alpha, float *dc,
                                 cudaStream_t s) {

@@ -2,6 +2,7 @@
 // kernels on `s` and returns the launch status; argument checks live in api.cu.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,11 +37,25 @@ cudaError_t launch_seg_spmm(qwha_dtype din, qwha_dtype dout, const void *in, int
 
 int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in);
 
+// Bytes of the transposed copies of dY and Z that launch_sddmm can use (bf16).
+size_t sddmm_transposed_bytes(int64_t T, int32_t d_out, int32_t d_in);
+
 // dc[j] = alpha * sum_t dY[t, r_j] Z[t, k_j] through the tile view; partial is
-// workspace of sddmm_chunks(...) * p floats.
+// workspace of sddmm_chunks(...) * p floats. tscratch (16-byte aligned, at
+// least sddmm_transposed_bytes(...)) lets bf16 inputs take the path that
+// transposes dY and Z once and feeds the kernel by tensor copies; nullptr, or
+// shapes that path does not take (fp32, d_out or d_in not a multiple of 8),
+// keep the kernel that stages and transposes its own tiles. Both give
+// bitwise the same dc.
 cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T, int32_t d_out, int32_t d_in,
                          const int32_t *tile_ptr, const int32_t *tile_pos, const int32_t *tile_rk, int64_t p,
-                         float alpha, float *partial, float *dc, cudaStream_t s);
+                         float alpha, float *partial, float *dc, cudaStream_t s, void *tscratch = nullptr);
+
+// A tensor map over a bf16 matrix of rows x cols with a row stride of ld
+// elements (ld * 2 a multiple of 16, ptr 16-byte aligned), box box_cols x
+// box_rows, no swizzle (gemm.cu).
+bool make_map_rows(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, int64_t ld, uint32_t box_cols,
+                   uint32_t box_rows);
 
 size_t plan_workspace(int32_t d_out, int32_t d_in);
 int plan_max_row_blocks();

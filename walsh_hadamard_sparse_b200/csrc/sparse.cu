@@ -15,16 +15,19 @@
 //
 // sddmm: partial[c, j] = sum_{t in chunk c} dY[t, r_j] * Z[t, k_j] over the
 //   tile view of E (QWHA_TILE x QWHA_TILE blocks of F). Grid = tiles x token
-//   chunks; a CTA stages dY[:, row block] and Z[:, column block] for TT tokens
-//   at a time, transposed, with the next sub-tile's global loads issued into
-//   registers before the current one is consumed (see sddmm_kernel for the
-//   lane layout).
+//   chunks; a CTA multiplies dY[:, row block] and Z[:, column block] held
+//   transposed in shared memory, 64 (bf16) or 32 (fp32) tokens at a time. For
+//   bf16, sdd_transpose_kernel transposes dY and Z once into the layout the
+//   CTAs read and sddmm_t_kernel feeds itself by tensor copies; the other
+//   kernels stage and transpose their own slices (see Sdd16Slot and
+//   sddmm_kernel for the lane layouts).
 // sddmm_reduce: dc[j] = alpha * sum_c partial[c, j] in increasing c (fixed
 //   order: the result is bitwise reproducible).
 
 #include <algorithm>
 #include <type_traits>
 
+#include "bulk.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -697,6 +700,66 @@ __device__ __forceinline__ float dot8_bf16(const uint4 y, const uint4 z, float a
   return acc;
 }
 
+// The per-slot part of the bf16 coefficient gradient, shared by both kernels
+// below so that they do the same arithmetic in the same order. A slot (4
+// lanes, lane q) owns E consecutive entries of the tile from my0 on and
+// multiplies them over every staged 64-token sub-tile.
+struct Sdd16Slot {
+  uint32_t off[kSdd16E];  // byte offsets of the lane's first dY chunk (high half) and Z chunk (low half)
+  uint32_t newcol = 0;    // bit i: entry i's column differs from entry i-1's
+  uint32_t valid = 0;     // bit i: entry i exists
+  float acc[kSdd16E];
+
+  // per entry, fixed over the token range (an unused entry reads row 0 and is not stored)
+  __device__ __forceinline__ void setup(const int32_t *__restrict__ tile_rk, int64_t my0, int64_t e_end, int r_len,
+                                        int k_len, int q, int par) {
+    newcol = 0;
+    valid = 0;
+#pragma unroll
+    for (int i = 0; i < kSdd16E; ++i) {
+      const int64_t e = my0 + i;
+      const int v = e < e_end ? tile_rk[e] : -1;
+      const int r_ = (v >> 16) & 0xffff, k_ = v & 0xffff;
+      const bool ok = e < e_end && v >= 0 && r_ < r_len && k_ < k_len;
+      const int rr = ok ? r_ : 0, kk = ok ? k_ : 0;
+      const int t_first = 16 * q + 8 * par;
+      off[i] = (sdd16_off(rr, t_first) << 16) | sdd16_off(kk, t_first);
+      if (i == 0 || (off[i] & 0xffffu) != (off[i - 1] & 0xffffu)) newcol |= 1u << i;
+      if (ok) valid |= 1u << i;
+      acc[i] = 0.f;
+    }
+  }
+  // one staged sub-tile: s_dy and s_z hold QWHA_TILE rows of 64 tokens each (layout sdd16_off)
+  __device__ __forceinline__ void mac(const unsigned char *s_dy, const unsigned char *s_z) {
+    uint4 z0 = make_uint4(0, 0, 0, 0), z1 = z0;
+#pragma unroll
+    for (int i = 0; i < kSdd16E; ++i) {
+      if (newcol & (1u << i)) {
+        const uint32_t oz = off[i] & 0xffffu;
+        z0 = *reinterpret_cast<const uint4 *>(s_z + oz);
+        z1 = *reinterpret_cast<const uint4 *>(s_z + (oz ^ 16u));  // the lane's other chunk: parity flipped
+      }
+      const uint32_t oy = off[i] >> 16;
+      const uint4 y0 = *reinterpret_cast<const uint4 *>(s_dy + oy);
+      const uint4 y1 = *reinterpret_cast<const uint4 *>(s_dy + (oy ^ 16u));
+      acc[i] = dot8_bf16(y1, z1, dot8_bf16(y0, z0, acc[i]));
+    }
+  }
+  __device__ __forceinline__ void store(const int32_t *__restrict__ tile_pos, int64_t my0, int64_t p, int q,
+                                        float *__restrict__ part) {
+#pragma unroll
+    for (int i = 0; i < kSdd16E; ++i) {
+      float sum = acc[i];
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      if (q == 0 && (valid & (1u << i))) {
+        const int j = tile_pos[my0 + i];
+        if ((uint64_t)j < (uint64_t)p) part[j] = sum;
+      }
+    }
+  }
+};
+
 __global__ void __launch_bounds__(kSddmmThreads, 1)
     sddmm_bf16_kernel(const __nv_bfloat16 *__restrict__ dY, const __nv_bfloat16 *__restrict__ Z, int64_t T_,
                       int d_out, int d_in, const int32_t *__restrict__ tile_ptr, const int32_t *__restrict__ tile_pos,
@@ -772,25 +835,8 @@ __global__ void __launch_bounds__(kSddmmThreads, 1)
 
   for (int64_t eb = e_begin; eb < e_end; eb += kPass) {
     const int64_t my0 = eb + (int64_t)slot * E;
-    // per entry, fixed over the token range: the byte offsets of this lane's first dY and Z chunks (dY high
-    // half, Z low half; an unused entry reads row 0 and is not stored), whether its column differs from the
-    // previous one's, and whether it is in use
-    uint32_t off[E];
-    uint32_t newcol = 0, valid = 0;
-    float acc[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-      const int64_t e = my0 + i;
-      const int v = e < e_end ? tile_rk[e] : -1;
-      const int r_ = (v >> 16) & 0xffff, k_ = v & 0xffff;
-      const bool ok = e < e_end && v >= 0 && r_ < r_len && k_ < k_len;
-      const int rr = ok ? r_ : 0, kk = ok ? k_ : 0;
-      const int t_first = 16 * q + 8 * par;
-      off[i] = (sdd16_off(rr, t_first) << 16) | sdd16_off(kk, t_first);
-      if (i == 0 || (off[i] & 0xffffu) != (off[i - 1] & 0xffffu)) newcol |= 1u << i;
-      if (ok) valid |= 1u << i;
-      acc[i] = 0.f;
-    }
+    Sdd16Slot sl;
+    sl.setup(tile_rk, my0, e_end, r_len, k_len, q, par);
     if (ta < tb) copy(ta);
     for (int64_t t0 = ta; t0 < tb; t0 += kSdd16TT) {
       asm volatile("cp.async.wait_all;" ::: "memory");
@@ -798,31 +844,158 @@ __global__ void __launch_bounds__(kSddmmThreads, 1)
       transpose();
       __syncthreads();
       if (t0 + kSdd16TT < tb) copy(t0 + kSdd16TT);  // the raw buffer is free again
-      uint4 z0 = make_uint4(0, 0, 0, 0), z1 = z0;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if (newcol & (1u << i)) {
-          const uint32_t oz = off[i] & 0xffffu;
-          z0 = *reinterpret_cast<const uint4 *>(s_z + oz);
-          z1 = *reinterpret_cast<const uint4 *>(s_z + (oz ^ 16u));  // the lane's other chunk: parity flipped
-        }
-        const uint32_t oy = off[i] >> 16;
-        const uint4 y0 = *reinterpret_cast<const uint4 *>(s_dy + oy);
-        const uint4 y1 = *reinterpret_cast<const uint4 *>(s_dy + (oy ^ 16u));
-        acc[i] = dot8_bf16(y1, z1, dot8_bf16(y0, z0, acc[i]));
-      }
+      sl.mac(s_dy, s_z);
     }
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-      float sum = acc[i];
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      if (q == 0 && (valid & (1u << i))) {
-        const int j = tile_pos[my0 + i];
-        if ((uint64_t)j < (uint64_t)p) part[j] = sum;
-      }
-    }
+    sl.store(tile_pos, my0, p, q, part);
     __syncthreads();
+  }
+}
+
+// dY and Z transposed once for the whole gradient: out[f, t] = in[t, f] for
+// f < d and t < ld (ld = T rounded up to 64; zeros past T), with the 16-byte
+// chunks of every 64-token block of a row f permuted as sdd16_off permutes
+// them in shared memory (chunk j at j ^ ((f & 3) << 1)). A plain 2-D tensor
+// copy of QWHA_TILE rows x 64 tokens then lands exactly in the layout the
+// gradient kernel reads. One CTA transposes 64 tokens x 64 features through
+// shared memory: each thread packs the same feature of two adjacent tokens
+// into one word, and word slots are XOR-swizzled so that both the writes and
+// the 16-byte reads of the exchange are free of bank conflicts. Requires
+// d % 8 == 0 and 16-byte aligned rows.
+__device__ __forceinline__ int sdd_xpose_swz(int c) { return 4 * ((c + (c >> 3)) & 7); }
+
+__global__ void __launch_bounds__(256) sdd_transpose_kernel(const __nv_bfloat16 *__restrict__ in, int64_t T_, int d,
+                                                            int64_t ld, __nv_bfloat16 *__restrict__ out) {
+  __shared__ __align__(16) uint32_t sw[64 * 32];  // [feature][token pair], 128 B a feature
+  const int64_t t0 = (int64_t)blockIdx.x * 64;
+  const int f0 = blockIdx.y * 64;
+  const int tid = threadIdx.x;
+  {
+    const int tp = tid >> 3, ch = tid & 7;
+    const int64_t t = t0 + 2 * tp;
+    const int f = f0 + 8 * ch;
+    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    if (f < d) {  // d % 8 == 0: the 8 features are all in range
+      if (t < T_) a = ld_stream(in + t * d + f);
+      if (t + 1 < T_) b = ld_stream(in + (t + 1) * d + f);
+    }
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = 8 * ch + 2 * i;
+      sw[c * 32 + (tp ^ sdd_xpose_swz(c))] = __byte_perm(wa[i], wb[i], 0x5410);
+      sw[(c + 1) * 32 + (tp ^ sdd_xpose_swz(c + 1))] = __byte_perm(wa[i], wb[i], 0x7632);
+    }
+  }
+  __syncthreads();
+  const int c = tid >> 2, g = tid & 3;
+  const int f = f0 + c;
+  if (f < d) {
+    const int z = sdd_xpose_swz(c);
+    const uint4 lo = *reinterpret_cast<const uint4 *>(sw + c * 32 + ((8 * g) ^ z));
+    const uint4 hi = *reinterpret_cast<const uint4 *>(sw + c * 32 + ((8 * g + 4) ^ z));
+    const int pos = (2 * g) ^ ((f & 3) << 1);  // even: the chunk pair stays adjacent
+    __nv_bfloat16 *o = out + (int64_t)f * ld + t0 + 8 * pos;
+    st_stream(o, lo);
+    st_stream(o + 8, hi);
+  }
+}
+
+constexpr int kSddTStages = 3;  // sub-tiles in flight per CTA
+constexpr int kSddTOpBytes = QWHA_TILE * kSdd16TT * 2;
+constexpr size_t sddmm_t_smem() { return (size_t)kSddTStages * 2 * kSddTOpBytes + 1024 + kSddTStages * 8; }
+
+__device__ __forceinline__ void sdd_tma_load(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// The bf16 gradient fed by tensor copies of the transposed operands (layout of
+// sdd_transpose_kernel): the CTA's sub-tiles (dY rows of its row block and Z
+// rows of its column block, 64 tokens each) stream through a ring of
+// kSddTStages slots that one thread refills, one CTA barrier per sub-tile.
+// Same tile, chunk, pass and slot structure, and the same Sdd16Slot
+// arithmetic, as sddmm_bf16_kernel. Every wait is bounded; on a timeout the
+// CTA records 0x800 in the error word, lets the copies it issued land and
+// exits.
+__global__ void __launch_bounds__(kSddmmThreads, 1)
+    sddmm_t_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmZ, int64_t T_,
+                   int d_out, int d_in, const int32_t *__restrict__ tile_ptr, const int32_t *__restrict__ tile_pos,
+                   const int32_t *__restrict__ tile_rk, int n_rb, int64_t chunk_tokens, int64_t p,
+                   float *__restrict__ partial, unsigned int *err) {
+  constexpr int E = kSdd16E;
+  constexpr int kPass = kSddmmSlots * E;
+  constexpr int S = kSddTStages;
+  extern __shared__ unsigned char sddt_smem[];
+  unsigned char *ring = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(sddt_smem) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + S * 2 * kSddTOpBytes);
+  const int tile = blockIdx.x;
+  const int rb = tile % n_rb, kb = tile / n_rb;
+  const int r0 = rb * QWHA_TILE, k0 = kb * QWHA_TILE;
+  const int r_len = min(QWHA_TILE, d_out - r0), k_len = min(QWHA_TILE, d_in - k0);
+  int64_t e_begin = tile_ptr[tile], e_end = tile_ptr[tile + 1];
+  if (e_begin < 0) e_begin = 0;
+  if (e_end > p) e_end = p;
+  const int64_t c = blockIdx.y;
+  const int64_t ta = c * chunk_tokens, tb = (ta + chunk_tokens < T_) ? ta + chunk_tokens : T_;
+  const int64_t n_sub = ta < tb ? (tb - ta + kSdd16TT - 1) / kSdd16TT : 0;
+  const int64_t n_pass = e_end > e_begin ? (e_end - e_begin + kPass - 1) / kPass : 0;
+  const int64_t total = n_sub * n_pass;  // ring steps
+  if (total == 0) return;                // the same for every thread of the CTA
+  float *part = partial + c * p;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int q = lane & 3, slot = warp * 8 + (lane >> 2);
+  const int par = slot & 1;
+
+  auto issue = [&](int64_t g) {  // thread 0: sub-tile g % n_sub into slot g % S
+    const int s = (int)(g % S);
+    const int x = (int)(ta + (g % n_sub) * kSdd16TT);
+    const uint32_t bar = bulk::saddr(full + s);
+    const uint32_t dst = bulk::saddr(ring + s * 2 * kSddTOpBytes);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kSddTOpBytes)
+                 : "memory");
+    sdd_tma_load(dst, &tmY, bar, x, r0);
+    sdd_tma_load(dst + kSddTOpBytes, &tmZ, bar, x, k0);
+  };
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) bulk::init(bulk::saddr(full + s), 1);
+    bulk::fence_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int64_t g = 0; g < S && g < total; ++g) issue(g);
+
+  int64_t g = 0;
+  for (int64_t pass = 0; pass < n_pass; ++pass) {
+    const int64_t my0 = e_begin + pass * kPass + (int64_t)slot * E;
+    Sdd16Slot sl;
+    sl.setup(tile_rk, my0, e_end, r_len, k_len, q, par);
+    for (int64_t sub = 0; sub < n_sub; ++sub, ++g) {
+      const int s = (int)(g % S);
+      const bool ok = bulk::wait(bulk::saddr(full + s), (uint32_t)((g / S) & 1));
+      // also: every thread has finished step g - 1, so its slot can be refilled
+      if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+          atomicOr(err, 0x800u);
+          // issued and not yet consumed: steps g .. S - 1 at the first step, else g .. g + S - 2
+          const int64_t last = g == 0 ? S : g + S - 1;
+          for (int64_t j = g; j < total && j < last; ++j)
+            (void)bulk::wait(bulk::saddr(full + (int)(j % S)), (uint32_t)((j / S) & 1));
+        }
+        return;
+      }
+      if (tid == 0 && g >= 1 && g - 1 + S < total) {
+        bulk::fence_proxy();
+        issue(g - 1 + S);
+      }
+      const unsigned char *st = ring + s * 2 * kSddTOpBytes;
+      sl.mac(st, st + kSddTOpBytes);
+    }
+    sl.store(tile_pos, my0, p, q, part);
   }
 }
 
@@ -879,9 +1052,14 @@ int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in) {
   return (int)want;
 }
 
+size_t sddmm_transposed_bytes(int64_t T, int32_t d_out, int32_t d_in) {
+  const int64_t ld = cdiv(T > 0 ? T : 1, kSdd16TT) * kSdd16TT;
+  return align_up((size_t)d_out * ld * 2, 256) + align_up((size_t)d_in * ld * 2, 256);
+}
+
 cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T, int32_t d_out, int32_t d_in,
                          const int32_t *tile_ptr, const int32_t *tile_pos, const int32_t *tile_rk, int64_t p,
-                         float alpha, float *partial, float *dc, cudaStream_t s) {
+                         float alpha, float *partial, float *dc, cudaStream_t s, void *tscratch) {
   if (p <= 0) return cudaSuccess;
   const int n_rb = (int)cdiv(d_out, QWHA_TILE);
   const int64_t tiles = n_rb * cdiv(d_in, QWHA_TILE);
@@ -891,18 +1069,44 @@ cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T
   if (e != cudaSuccess) return e;
   if (T > 0) {
     dim3 grid((unsigned)tiles, (unsigned)n_chunks);
-    const size_t smem = dt == QWHA_BF16 ? sddmm16_smem() : sddmm_smem<float>();
-    e = cudaFuncSetAttribute(dt == QWHA_BF16 ? (const void *)sddmm_bf16_kernel : (const void *)sddmm_kernel<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    if (dt == QWHA_BF16)
-      sddmm_bf16_kernel<<<grid, kSddmmThreads, smem, s>>>(
-          static_cast<const __nv_bfloat16 *>(dY), static_cast<const __nv_bfloat16 *>(Z), T, d_out, d_in, tile_ptr,
-          tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
-    else
-      sddmm_kernel<float><<<grid, kSddmmThreads, smem, s>>>(static_cast<const float *>(dY),
-                                                         static_cast<const float *>(Z), T, d_out, d_in, tile_ptr,
-                                                         tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
+    const int64_t ld = cdiv(T, kSdd16TT) * kSdd16TT;
+    __nv_bfloat16 *yt = static_cast<__nv_bfloat16 *>(tscratch);
+    __nv_bfloat16 *zt = yt ? yt + align_up((size_t)d_out * ld * 2, 256) / 2 : nullptr;
+    CUtensorMap tmY, tmZ;
+    const bool transposed = dt == QWHA_BF16 && yt && aligned16(yt) && d_out % 8 == 0 && d_in % 8 == 0 &&
+                            aligned16(dY) && aligned16(Z) && ld / kSdd16TT <= 0x7fffffff &&
+                            make_map_rows(&tmY, yt, d_out, ld, ld, kSdd16TT, QWHA_TILE) &&
+                            make_map_rows(&tmZ, zt, d_in, ld, ld, kSdd16TT, QWHA_TILE);
+    if (transposed) {
+      const dim3 gy((unsigned)(ld / 64), (unsigned)cdiv(d_out, 64)), gz((unsigned)(ld / 64), (unsigned)cdiv(d_in, 64));
+      sdd_transpose_kernel<<<gy, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(dY), T, d_out, ld, yt);
+      sdd_transpose_kernel<<<gz, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Z), T, d_in, ld, zt);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      const size_t smem = sddmm_t_smem();
+      static bool attr_done[64] = {};
+      const int slot = device_slot();
+      if (!attr_done[slot]) {
+        e = cudaFuncSetAttribute(sddmm_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_done[slot] = true;
+      }
+      sddmm_t_kernel<<<grid, kSddmmThreads, smem, s>>>(tmY, tmZ, T, d_out, d_in, tile_ptr, tile_pos, tile_rk, n_rb,
+                                                        chunk_tokens, p, partial, device_error_word());
+    } else {
+      const size_t smem = dt == QWHA_BF16 ? sddmm16_smem() : sddmm_smem<float>();
+      e = cudaFuncSetAttribute(dt == QWHA_BF16 ? (const void *)sddmm_bf16_kernel : (const void *)sddmm_kernel<float>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      if (dt == QWHA_BF16)
+        sddmm_bf16_kernel<<<grid, kSddmmThreads, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(dY), static_cast<const __nv_bfloat16 *>(Z), T, d_out, d_in, tile_ptr,
+            tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
+      else
+        sddmm_kernel<float><<<grid, kSddmmThreads, smem, s>>>(static_cast<const float *>(dY),
+                                                           static_cast<const float *>(Z), T, d_out, d_in, tile_ptr,
+                                                           tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
