@@ -347,10 +347,14 @@ qwha_status check_ws(void *ws, size_t ws_bytes, size_t need) {
 }
 
 // packed (index, value) entries of the SpMM in gather order
-size_t ent_bytes(int64_t p) { return align_up((size_t)(p > 0 ? p : 1) * 8, 256); }
+// Scratch of the SpMM for both directions: the forward over rows (segments
+// d_out, width d_in) and the backward gather over columns.
+size_t ent_bytes(int64_t p, int32_t d_out, int32_t d_in) {
+  return std::max(spmm_scratch_bytes(p, d_out, d_in), spmm_scratch_bytes(p, d_in, d_out));
+}
 
 size_t fwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
-  const size_t n = ent_bytes(p);
+  const size_t n = ent_bytes(p, d_out, d_in);
   if (!base) return n;
   return n + align_up((size_t)T * d_out * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
 }
@@ -373,7 +377,7 @@ size_t dz_region(int32_t d_out, int32_t d_in, int64_t T) {
 size_t bwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
   size_t n = align_up((size_t)kSddmmMaxChunks * (size_t)(p > 0 ? p : 1) * 4, 256);
   n += dz_region(d_out, d_in, T);  // dZ, and before it the transposed dY and Z of the gradient
-  n += ent_bytes(p);  // CSC entries in gather order
+  n += ent_bytes(p, d_out, d_in);  // CSC entries in gather order
   if (base) n += align_up((size_t)T * d_in * 4, 256) + align_up(wdeq_bytes(d_out, d_in), 256);
   return n;
 }
@@ -511,19 +515,20 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   }
   if (e != cudaSuccess) return cuda_status(e, "fwht");
   Carver cv(ws);
-  int2 *ent = static_cast<int2 *>(cv.take(ent_bytes(a->p)));
+  const size_t ent_n = ent_bytes(a->p, a->d_out, a->d_in);
+  void *ent = cv.take(ent_n);
   if (!wq) {
-    StageScope sc(ST_SPMM_FWD, 2, s);
+    StageScope sc(ST_SPMM_FWD, 0, s);
     e = launch_seg_spmm(dt, dt, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out, alpha,
-                        ent, Y, s);
+                        ent, ent_n, Y, s, &sc.kernels);
     return cuda_status(e, "spmm");
   }
   float *y_ad = static_cast<float *>(cv.take((size_t)T * a->d_out * 4));
   void *wdeq = cv.take(wdeq_bytes(a->d_out, a->d_in));
   {
-    StageScope sc(ST_SPMM_FWD, 2, s);
+    StageScope sc(ST_SPMM_FWD, 0, s);
     e = launch_seg_spmm(dt, QWHA_F32, Z_out, T, a->d_in, a->row_ptr, a->col_idx, a->coef, nullptr, a->p, a->d_out,
-                        alpha, ent, y_ad, s);
+                        alpha, ent, ent_n, y_ad, s, &sc.kernels);
   }
   if (e != cudaSuccess) return cuda_status(e, "spmm");
   {
@@ -559,19 +564,20 @@ qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
   Carver cv(ws);
   float *partial = static_cast<float *>(cv.take((size_t)kSddmmMaxChunks * (size_t)(a->p > 0 ? a->p : 1) * 4));
   float *dz = static_cast<float *>(cv.take(dz_region(a->d_out, a->d_in, T)));
-  int2 *ent = static_cast<int2 *>(cv.take(ent_bytes(a->p)));
+  const size_t ent_n = ent_bytes(a->p, a->d_out, a->d_in);
+  void *ent = cv.take(ent_n);
   cudaError_t e = cudaSuccess;
   if (dc) {
-    StageScope sc(ST_SDDMM, 2, s);
+    StageScope sc(ST_SDDMM, 0, s);
     e = launch_sddmm(dt, dY, Z, T, a->d_out, a->d_in, a->tile_ptr, a->tile_pos, a->tile_rk, a->p, alpha, partial, dc,
-                     s, dz);
+                     s, dz, &sc.kernels);
   }
   if (e != cudaSuccess) return cuda_status(e, "sddmm");
   if (!dX || T == 0) return QWHA_OK;
   {
-    StageScope sc(ST_GATHER_BWD, 2, s);
+    StageScope sc(ST_GATHER_BWD, 0, s);
     e = launch_seg_spmm(dt, QWHA_F32, dY, T, a->d_out, a->col_ptr, a->row_idx, a->coef, a->perm, a->p, a->d_in, alpha,
-                        ent, dz, s);
+                        ent, ent_n, dz, s, &sc.kernels);
   }
   if (e != cudaSuccess) return cuda_status(e, "gather");
   const int logn = ilog2(a->had_block);

@@ -29,11 +29,15 @@ namespace qwha {
 constexpr int kSddmmMaxChunks = 16;
 
 // out[t, i] = alpha * sum_{j in [seg_ptr[i], seg_ptr[i+1])} v_j * in[t, idx[j]], with
-// v_j = val[perm[j]] when perm is given (the CSC view), else val[j]. ent is
-// scratch for max(nnz, 1) packed (index, value) entries (8-byte aligned).
+// v_j = val[perm[j]] when perm is given (the CSC view), else val[j]. scratch
+// (256-byte aligned) holds the entries in the order the kernel reads them;
+// spmm_scratch_bytes(nnz, n_seg, W_in) bytes always suffice. *launched (if
+// given) receives the number of kernels enqueued.
+size_t spmm_scratch_bytes(int64_t p, int n_seg, int W_in);
 cudaError_t launch_seg_spmm(qwha_dtype din, qwha_dtype dout, const void *in, int64_t T, int W_in,
                             const int32_t *seg_ptr, const int32_t *idx, const float *val, const int32_t *perm,
-                            int64_t nnz, int n_seg, float alpha, int2 *ent, void *out, cudaStream_t s);
+                            int64_t nnz, int n_seg, float alpha, void *scratch, size_t scratch_bytes, void *out,
+                            cudaStream_t s, int *launched = nullptr);
 
 int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in);
 
@@ -46,10 +50,12 @@ size_t sddmm_transposed_bytes(int64_t T, int32_t d_out, int32_t d_in);
 // transposes dY and Z once and feeds the kernel by tensor copies; nullptr, or
 // shapes that path does not take (fp32, d_out or d_in not a multiple of 8),
 // keep the kernel that stages and transposes its own tiles. Both give
-// bitwise the same dc.
+// bitwise the same dc. *launched (if given) receives the number of kernels
+// enqueued.
 cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T, int32_t d_out, int32_t d_in,
                          const int32_t *tile_ptr, const int32_t *tile_pos, const int32_t *tile_rk, int64_t p,
-                         float alpha, float *partial, float *dc, cudaStream_t s, void *tscratch = nullptr);
+                         float alpha, float *partial, float *dc, cudaStream_t s, void *tscratch = nullptr,
+                         int *launched = nullptr);
 
 // A tensor map over a bf16 matrix of rows x cols with a row stride of ld
 // elements (ld * 2 a multiple of 16, ptr 16-byte aligned), box box_cols x

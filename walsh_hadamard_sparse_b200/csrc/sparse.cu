@@ -441,6 +441,350 @@ __global__ void __launch_bounds__(kSpmmThreads)
   }
 }
 
+// ---------------------------------------------------------------- sliced SpMM
+//
+// The same product with one segment per slot. Segments are ranked by length
+// (longest first, ties by index) and cut into groups of NSLOT consecutive
+// ranks; a group's entries are stored step-major, two steps of a slot next
+// to each other: entry step t of the slot s of group g sits at
+//   goff[g] + (t / 2) * 2 * NSLOT + 2 * s + (t & 1),
+// padded with empty entries (offset 0, value 0) to the group's longest
+// segment rounded up to an even count. A slot then runs its own segment
+// start to end with no reduction across lanes, and the warp's steps stay
+// full: on the q_proj pattern the padding is 0.3% of the entries, against 46%
+// for groups of consecutive rows. Inside a segment the entries are ordered
+// round robin over the residues of their column modulo M (the staged rows in
+// one 128-byte bank line), starting at residue s mod M, so that the slots that
+// share one shared-memory wavefront read rows on distinct banks until the
+// smaller classes run out. An entry holds the byte offset of its staged row
+// and the value, as a bf16 pair (v, v) for bf16 input (the products are
+// those of seg_spmm_kernel) or as fp32 bits.
+//
+// Scratch (spmm_scratch_bytes): entries, then srank [n_seg], sseg [groups *
+// NSLOT] (rank -> segment, -1 past the end), goff [groups + 1].
+struct SellLayout {
+  int n_grp;
+  size_t ent_cap;  // entries
+  size_t ent_off, srank_off, sseg_off, goff_off, total;
+};
+
+__host__ __device__ inline SellLayout sell_layout(int64_t p, int n_seg, int W_in, int nslot) {
+  SellLayout L;
+  L.n_grp = (n_seg + nslot - 1) / nslot;
+  // p entries, plus padding: at most nslot times the longest segment (<= W_in) and one step a group
+  L.ent_cap = (size_t)(p > 0 ? p : 0) + (size_t)nslot * ((size_t)W_in + 2) + (size_t)L.n_grp * nslot;
+  auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+  L.ent_off = 0;
+  L.srank_off = up(L.ent_cap * 8);
+  L.sseg_off = L.srank_off + up((size_t)n_seg * 4);
+  L.goff_off = L.sseg_off + up((size_t)L.n_grp * nslot * 4);
+  L.total = L.goff_off + up(((size_t)L.n_grp + 1) * 4);
+  return L;
+}
+
+// Rank of every segment by (length descending, index ascending): the number
+// of segments whose key is smaller, summed over chunks of kRankChunk keys
+// (grid.y) with integer atomics on a zeroed srank, so the result does not
+// depend on the order in which the chunks finish. Keys are unique (the index
+// is part of them), so the ranks are a permutation.
+constexpr int kRankChunk = 1024;
+__device__ __forceinline__ uint32_t sell_key(const int32_t *__restrict__ seg_ptr, int i, int nnz) {
+  int a = seg_ptr[i], b = seg_ptr[i + 1];
+  a = a < 0 ? 0 : (a > nnz ? nnz : a);
+  b = b < a ? a : (b > nnz ? nnz : b);
+  const int len = b - a < 65535 ? b - a : 65535;
+  return ((uint32_t)(65535 - len) << 16) | (uint32_t)i;
+}
+
+__global__ void __launch_bounds__(256)
+    sell_rank_kernel(const int32_t *__restrict__ seg_ptr, int n_seg, int64_t nnz64, int32_t *__restrict__ srank) {
+  __shared__ __align__(16) uint32_t keys[kRankChunk];
+  const int nnz = (int)nnz64;
+  const int c0 = (int)blockIdx.y * kRankChunk;
+  const int n = n_seg - c0 < kRankChunk ? n_seg - c0 : kRankChunk;
+  for (int j = threadIdx.x; j < kRankChunk; j += 256) keys[j] = j < n ? sell_key(seg_ptr, c0 + j, nnz) : 0xffffffffu;
+  __syncthreads();
+  const int i = (int)blockIdx.x * 256 + (int)threadIdx.x;
+  if (i >= n_seg) return;
+  const uint32_t mine = sell_key(seg_ptr, i, nnz);
+  int cnt = 0;
+  const int n4 = (n + 3) / 4;
+  for (int j = 0; j < n4; ++j) {
+    const uint4 k = reinterpret_cast<const uint4 *>(keys)[j];
+    cnt += (k.x < mine) + (k.y < mine) + (k.z < mine) + (k.w < mine);
+  }
+  if (cnt) atomicAdd(srank + i, cnt);
+}
+
+// sseg[srank[i]] = i, and -1 for the positions past n_seg of the last group.
+__global__ void sell_place_kernel(const int32_t *__restrict__ srank, int n_seg, int n_pad,
+                                  int32_t *__restrict__ sseg) {
+  const int i = (int)blockIdx.x * (int)blockDim.x + (int)threadIdx.x;
+  if (i < n_seg) {
+    const int r = srank[i];
+    if ((unsigned)r < (unsigned)n_seg) sseg[r] = i;
+  } else if (i < n_pad) {
+    sseg[i] = -1;
+  }
+}
+
+// goff[g] = nslot * sum over earlier groups of their step count (the length of
+// the group's first, longest, segment, at most W_in, rounded up to even). One
+// CTA.
+__global__ void __launch_bounds__(1024)
+    sell_offsets_kernel(const int32_t *__restrict__ seg_ptr, const int32_t *__restrict__ sseg, int n_grp,
+                        int64_t nnz64, int nslot, int W_in, int32_t *__restrict__ goff) {
+  __shared__ int32_t part[32];
+  __shared__ int32_t carry;
+  const int nnz = (int)nnz64;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int g0 = 0; g0 < n_grp; g0 += 1024) {
+    const int g = g0 + (int)threadIdx.x;
+    int steps = 0;
+    if (g < n_grp) {
+      const int seg = sseg[(size_t)g * nslot];  // the group's first rank: its longest segment
+      int a = seg_ptr[seg], b = seg_ptr[seg + 1];
+      a = a < 0 ? 0 : (a > nnz ? nnz : a);
+      b = b < a ? a : (b > nnz ? nnz : b);
+      // a segment has at most W_in distinct columns; the cap keeps the layout within its scratch
+      // even for a malformed one (whose entries past W_in are then left out)
+      steps = ((b - a < W_in ? b - a : W_in) + 1) & ~1;
+    }
+    int v = steps;  // inclusive scan over the CTA
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += u;
+    }
+    if (lane == 31) part[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      int w = part[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += u;
+      }
+      part[lane] = w;
+    }
+    __syncthreads();
+    const int incl = v + (warp > 0 ? part[warp - 1] : 0) + carry;
+    if (g < n_grp) goff[g] = (incl - steps) * nslot;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) goff[n_grp] = carry * nslot;
+}
+
+// One warp per segment: its entries in the rotated round-robin order at the
+// positions of its slot, then the padding of the group. The slots of the last
+// group past n_seg (ranks n_seg .. n_pad - 1) are written as empty segments.
+template <typename Tin, int TT, int M, int NSLOT>
+__global__ void __launch_bounds__(256)
+    sell_arrange_kernel(const int32_t *__restrict__ seg_ptr, int n_seg, const int32_t *__restrict__ idx,
+                        const float *__restrict__ val, const int32_t *__restrict__ perm, int64_t nnz64, int W_in,
+                        const int32_t *__restrict__ srank, const int32_t *__restrict__ goff, int2 *__restrict__ ent) {
+  static_assert(M >= 1 && M <= 32 && (M & (M - 1)) == 0, "residue classes");
+  const int lane = threadIdx.x & 31;
+  const int nnz = (int)nnz64;
+  const unsigned below = (1u << lane) - 1u;
+  const int warps = (int)gridDim.x * (int)(blockDim.x >> 5);
+  const int n_pad = (n_seg + NSLOT - 1) / NSLOT * NSLOT;
+  for (int seg = (int)blockIdx.x * (int)(blockDim.x >> 5) + (int)(threadIdx.x >> 5); seg < n_pad;
+       seg += warps) {
+    const bool real = seg < n_seg;
+    int s = real ? seg_ptr[seg] : 0, e = real ? seg_ptr[seg + 1] : 0;
+    s = s < 0 ? 0 : (s > nnz ? nnz : s);
+    e = e < s ? s : (e > nnz ? nnz : e);
+    const int rk = real ? srank[seg] : seg;
+    const int g = rk / NSLOT, slot = rk % NSLOT;
+    const int r0 = slot & (M - 1);  // the class this slot starts with
+    const int base = goff[g], steps = (goff[g + 1] - base) / NSLOT;
+    int2 *dst = ent + base + 2 * slot;
+    auto at = [&](int t) { return dst + (t >> 1) * (2 * NSLOT) + (t & 1); };
+    int cnt[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) cnt[m] = 0;
+    for (int j = s + lane; j < e; j += 32) {
+      const int r = (__ldg(idx + j) - r0) & (M - 1);
+#pragma unroll
+      for (int m = 0; m < M; ++m) cnt[m] += r == m ? 1 : 0;
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) cnt[m] += __shfl_xor_sync(0xffffffffu, cnt[m], off);
+    int run[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) run[m] = 0;
+    for (int b = s; b < e; b += 32) {
+      const int j = b + lane;
+      int k = 0, r = -1;
+      float v = 0.f;
+      if (j < e) {
+        k = __ldg(idx + j);
+        r = (k - r0) & (M - 1);
+        if (perm) {
+          const int32_t src = __ldg(perm + j);
+          v = (unsigned)src < (unsigned)nnz ? __ldg(val + src) : 0.f;
+        } else {
+          v = __ldg(val + j);
+        }
+      }
+      int q = 0;
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const unsigned bal = __ballot_sync(0xffffffffu, r == m);
+        if (r == m) q = run[m] + __popc(bal & below);
+        run[m] += __popc(bal);
+      }
+      if (j < e) {
+        int t = 0;
+#pragma unroll
+        for (int m = 0; m < M; ++m) t += (cnt[m] < q ? cnt[m] : q) + (m < r && cnt[m] > q ? 1 : 0);
+        const bool ok = (unsigned)k < (unsigned)W_in && t < steps;
+        int vb;
+        if constexpr (sizeof(Tin) == 2) vb = (int)pack_bf16x2(v, v);
+        else vb = __float_as_int(v);
+        if (t < steps) *at(t) = ok ? make_int2(k * TT * (int)sizeof(Tin), vb) : make_int2(0, 0);
+      }
+    }
+    for (int t = e - s + lane; t < steps; t += 32) *at(t) = make_int2(0, 0);  // none if e - s >= steps
+  }
+}
+
+// acc[i] += v * row[i] for the G tokens a lane holds, v as stored in a sliced entry.
+template <int G>
+__device__ __forceinline__ void mac_sliced(const __nv_bfloat16 *row, int vbits, float *acc) {
+  const uint32_t vv = (uint32_t)vbits;
+  uint32_t w[G / 2];
+  if constexpr (G == 8) {
+    const uint4 t = *reinterpret_cast<const uint4 *>(row);
+    w[0] = t.x, w[1] = t.y, w[2] = t.z, w[3] = t.w;
+  } else {
+    const uint2 t = *reinterpret_cast<const uint2 *>(row);
+    w[0] = t.x, w[1] = t.y;
+  }
+#pragma unroll
+  for (int i = 0; i < G / 2; ++i) {
+    acc[2 * i] = fma_bf16_lo(w[i], vv, acc[2 * i]);
+    acc[2 * i + 1] = fma_bf16_hi(w[i], vv, acc[2 * i + 1]);
+  }
+}
+template <int G>
+__device__ __forceinline__ void mac_sliced(const float *row, int vbits, float *acc) {
+  mac_tokens<G>(row, __int_as_float(vbits), acc);
+}
+
+constexpr int kSellPairs = 4;  // step pairs per load batch (8 entries a slot)
+
+template <typename Tin, typename Tout, int TT>
+__global__ void __launch_bounds__(kSpmmThreads)
+    sell_spmm_kernel(const Tin *__restrict__ in, int64_t T, int W_in, const int4 *__restrict__ ent,
+                     const int32_t *__restrict__ sseg, const int32_t *__restrict__ goff, int n_grp, int n_seg,
+                     float alpha, Tout *__restrict__ out) {
+  static_assert(TT == 4 || TT == 8 || TT == 16, "token tile");
+  constexpr int G = TT < 8 ? TT : 8;  // tokens per lane
+  constexpr int Q = TT / G;           // lanes per slot
+  constexpr int NSLOT = 32 / Q;
+  constexpr int kWarps = kSpmmThreads / 32;
+  constexpr int U = kSellPairs;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Tin *s_in = reinterpret_cast<Tin *>(smem_raw);
+  const int64_t t0 = (int64_t)blockIdx.x * TT;
+  stage_transposed<Tin, TT>(in, T, W_in, t0, 0, W_in, W_in, s_in);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = lane % Q, slot = lane / Q;
+  const unsigned char *s_q = reinterpret_cast<const unsigned char *>(s_in) + (size_t)G * q * sizeof(Tin);
+  // groups (longest first) go to the gridDim.y CTAs of a token tile in turn, and within a CTA to
+  // its warps in snake order (round j: warp w, then warp kWarps - 1 - w), which evens out the
+  // warps' total steps
+  for (int j = 0;; ++j) {
+    const int local = (j & 1) ? kWarps - 1 - warp : warp;
+    const int g = (int)blockIdx.y + (int)gridDim.y * (kWarps * j + local);
+    if (g >= n_grp) break;
+    const int base = goff[g];
+    const int npair = (goff[g + 1] - base) / (2 * NSLOT);
+    // pair i of this slot: ent[(base / 2) + i * NSLOT + slot] as (offset, value) x 2
+    const int4 *e = ent + base / 2 + slot;
+    float acc[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) acc[i] = 0.f;
+    int4 cur[U], nxt[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) cur[u] = u < npair ? __ldg(e + (size_t)u * NSLOT) : make_int4(0, 0, 0, 0);
+    for (int i0 = 0; i0 < npair; i0 += U) {
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        nxt[u] = i0 + U + u < npair ? __ldg(e + (size_t)(i0 + U + u) * NSLOT) : make_int4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (i0 + u >= npair) break;  // warp-uniform
+        mac_sliced<G>(reinterpret_cast<const Tin *>(s_q + cur[u].x), cur[u].y, acc);
+        mac_sliced<G>(reinterpret_cast<const Tin *>(s_q + cur[u].z), cur[u].w, acc);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+    }
+    const int seg = sseg[(size_t)g * NSLOT + slot];
+    if (seg >= 0 && seg < n_seg) {
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        const int64_t t = t0 + G * q + i;
+        if (t < T) io<Tout>::store1(out + t * n_seg + seg, alpha * acc[i]);
+      }
+    }
+  }
+}
+
+template <typename Tin, typename Tout, int TT>
+cudaError_t run_spmm_sliced(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
+                            const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha,
+                            void *scratch, void *out, cudaStream_t s) {
+  constexpr int G = TT < 8 ? TT : 8;
+  constexpr int NSLOT = 32 / (TT / G);
+  constexpr int M = 128 / (TT * (int)sizeof(Tin));  // staged rows per bank line
+  const SellLayout L = sell_layout(nnz, n_seg, W_in, NSLOT);
+  char *base = static_cast<char *>(scratch);
+  int2 *ent = reinterpret_cast<int2 *>(base + L.ent_off);
+  int32_t *srank = reinterpret_cast<int32_t *>(base + L.srank_off);
+  int32_t *sseg = reinterpret_cast<int32_t *>(base + L.sseg_off);
+  int32_t *goff = reinterpret_cast<int32_t *>(base + L.goff_off);
+  const int n_pad = L.n_grp * NSLOT;
+  cudaError_t e = cudaMemsetAsync(srank, 0, (size_t)n_seg * 4, s);
+  if (e != cudaSuccess) return e;
+  sell_rank_kernel<<<dim3((unsigned)cdiv(n_seg, 256), (unsigned)cdiv(n_seg, kRankChunk)), 256, 0, s>>>(seg_ptr, n_seg,
+                                                                                                      nnz, srank);
+  sell_place_kernel<<<(unsigned)cdiv(n_pad, 256), 256, 0, s>>>(srank, n_seg, n_pad, sseg);
+  sell_offsets_kernel<<<1, 1024, 0, s>>>(seg_ptr, sseg, L.n_grp, nnz, NSLOT, W_in, goff);
+  {
+    const int64_t grid = std::min<int64_t>(cdiv(n_pad, 256 / 32), (int64_t)sm_count() * 8);
+    sell_arrange_kernel<Tin, TT, M, NSLOT><<<(unsigned)grid, 256, 0, s>>>(seg_ptr, n_seg, idx, val, perm, nnz, W_in,
+                                                                          srank, goff, ent);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = ((size_t)W_in * TT * sizeof(Tin) + 15) & ~(size_t)15;
+  auto k = sell_spmm_kernel<Tin, Tout, TT>;
+  static bool attr_done[64] = {};
+  const int slot = device_slot();
+  if (!attr_done[slot]) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSpmmSmemCap);
+    if (e != cudaSuccess) return e;
+    attr_done[slot] = true;
+  }
+  const int64_t tiles = cdiv(T, TT);
+  // one CTA per SM: split the groups so that the token tiles fill whole waves
+  const dim3 grid((unsigned)tiles, (unsigned)wave_split(tiles, L.n_grp >= 4 * kSpmmThreads / 32 ? 4 : 1));
+  k<<<grid, kSpmmThreads, smem, s>>>(static_cast<const Tin *>(in), T, W_in, reinterpret_cast<const int4 *>(ent), sseg,
+                                     goff, L.n_grp, n_seg, alpha, static_cast<Tout *>(out));
+  return cudaGetLastError();
+}
+
 template <typename Tin, typename Tout, int TT>
 cudaError_t run_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
                      const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha, int2 *ent,
@@ -465,11 +809,28 @@ cudaError_t run_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr
   return cudaGetLastError();
 }
 
+bool sliced_ok(int64_t nnz, int n_seg, int W_in, int nslot, size_t scratch_bytes) {
+  // 16-bit length and index fields of the rank keys
+  return n_seg <= 65536 && W_in <= 65535 && nnz < ((int64_t)1 << 30) &&
+         sell_layout(nnz, n_seg, W_in, nslot).total <= scratch_bytes;
+}
+
 template <typename Tin, typename Tout>
 cudaError_t pick_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
-                      const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha, int2 *ent,
-                      void *out, cudaStream_t s) {
+                      const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha, void *scratch,
+                      size_t scratch_bytes, void *out, cudaStream_t s, int *launched) {
   const size_t row = (size_t)W_in * sizeof(Tin);
+  // the sliced kernel stages the token tile alone (5 kernels: rank, place, offsets, arrange, product)
+  *launched = 5;
+  if (row * 16 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 16, scratch_bytes))
+    return run_spmm_sliced<Tin, Tout, 16>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
+  if (row * 16 > kSpmmSmemCap && row * 8 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
+    return run_spmm_sliced<Tin, Tout, 8>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
+  if (row * 8 > kSpmmSmemCap && row * 4 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
+    return run_spmm_sliced<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
+  *launched = 2;  // arrange, product
+  if (scratch_bytes < (size_t)(nnz > 0 ? nnz : 1) * 8) return cudaErrorInvalidValue;
+  int2 *ent = static_cast<int2 *>(scratch);
   const size_t ptrs = ((size_t)n_seg + 1) * sizeof(int32_t) + 16;
   const size_t cap = kSpmmSmemCap > ptrs ? kSpmmSmemCap - ptrs : 0;
   if (row * 16 + spmm_obuf_bytes<Tout>(16) <= cap)
@@ -1010,20 +1371,34 @@ __global__ void sddmm_reduce_kernel(const float *__restrict__ partial, int n_chu
 
 }  // namespace
 
+size_t spmm_scratch_bytes(int64_t p, int n_seg, int W_in) {
+  const size_t a = sell_layout(p, n_seg, W_in, 16).total, b = sell_layout(p, n_seg, W_in, 32).total;
+  const size_t c = align_up((size_t)(p > 0 ? p : 1) * 8, 256);
+  return std::max(std::max(a, b), c);
+}
+
 cudaError_t launch_seg_spmm(qwha_dtype din, qwha_dtype dout, const void *in, int64_t T, int W_in,
                             const int32_t *seg_ptr, const int32_t *idx, const float *val, const int32_t *perm,
-                            int64_t nnz, int n_seg, float alpha, int2 *ent, void *out, cudaStream_t s) {
+                            int64_t nnz, int n_seg, float alpha, void *scratch, size_t scratch_bytes, void *out,
+                            cudaStream_t s, int *launched) {
+  int dummy = 0;
+  int *nk = launched ? launched : &dummy;
+  *nk = 0;
   if (T <= 0 || n_seg <= 0) return cudaSuccess;
-  if (reinterpret_cast<uintptr_t>(ent) & 7) return cudaErrorMisalignedAddress;
+  if (reinterpret_cast<uintptr_t>(scratch) & 255) return cudaErrorMisalignedAddress;
   using bf = __nv_bfloat16;
   if (din == QWHA_BF16) {
     if (dout == QWHA_BF16)
-      return pick_spmm<bf, bf>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
-    return pick_spmm<bf, float>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
+      return pick_spmm<bf, bf>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, scratch_bytes, out, s,
+                               nk);
+    return pick_spmm<bf, float>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, scratch_bytes, out,
+                                s, nk);
   }
   if (dout == QWHA_BF16)
-    return pick_spmm<float, bf>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
-  return pick_spmm<float, float>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, ent, out, s);
+    return pick_spmm<float, bf>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, scratch_bytes, out,
+                                s, nk);
+  return pick_spmm<float, float>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, scratch_bytes, out,
+                                 s, nk);
 }
 
 int sddmm_chunks(int64_t T, int32_t d_out, int32_t d_in) {
@@ -1059,7 +1434,10 @@ size_t sddmm_transposed_bytes(int64_t T, int32_t d_out, int32_t d_in) {
 
 cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T, int32_t d_out, int32_t d_in,
                          const int32_t *tile_ptr, const int32_t *tile_pos, const int32_t *tile_rk, int64_t p,
-                         float alpha, float *partial, float *dc, cudaStream_t s, void *tscratch) {
+                         float alpha, float *partial, float *dc, cudaStream_t s, void *tscratch, int *launched) {
+  int dummy = 0;
+  int *nk = launched ? launched : &dummy;
+  *nk = 0;
   if (p <= 0) return cudaSuccess;
   const int n_rb = (int)cdiv(d_out, QWHA_TILE);
   const int64_t tiles = n_rb * cdiv(d_in, QWHA_TILE);
@@ -1093,6 +1471,7 @@ cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T
       }
       sddmm_t_kernel<<<grid, kSddmmThreads, smem, s>>>(tmY, tmZ, T, d_out, d_in, tile_ptr, tile_pos, tile_rk, n_rb,
                                                         chunk_tokens, p, partial, device_error_word());
+      *nk += 3;
     } else {
       const size_t smem = dt == QWHA_BF16 ? sddmm16_smem() : sddmm_smem<float>();
       e = cudaFuncSetAttribute(dt == QWHA_BF16 ? (const void *)sddmm_bf16_kernel : (const void *)sddmm_kernel<float>,
@@ -1106,12 +1485,14 @@ cudaError_t launch_sddmm(qwha_dtype dt, const void *dY, const void *Z, int64_t T
         sddmm_kernel<float><<<grid, kSddmmThreads, smem, s>>>(static_cast<const float *>(dY),
                                                            static_cast<const float *>(Z), T, d_out, d_in, tile_ptr,
                                                            tile_pos, tile_rk, n_rb, chunk_tokens, p, partial);
+      *nk += 1;
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   sddmm_reduce_kernel<<<(unsigned)std::min<int64_t>(cdiv(p, 256), (int64_t)sm_count() * 8), 256, 0, s>>>(partial, n_chunks, p,
                                                                                          alpha, dc);
+  *nk += 1;
   return cudaGetLastError();
 }
 
