@@ -579,6 +579,42 @@ __global__ void __launch_bounds__(1024)
   if (threadIdx.x == 0) goff[n_grp] = carry * nslot;
 }
 
+// Staged row of input column k in the sliced kernel: k with its low log2(M)
+// bits XORed with bits 8 and up. The bank line position of a staged row is
+// its index modulo M, and the columns a segment selects are not spread evenly
+// over k mod M (on q_proj a row's largest residue class holds 34% of its
+// entries, against 30% for random columns); mixing in the higher bits makes
+// the classes as even as random ones (29%), so the round-robin order below
+// meets fewer bank conflicts (CPU model of q_proj: 1.48 -> 1.25 wavefronts per
+// conflict-free one). A bijection within each aligned block of M rows.
+template <int M>
+__host__ __device__ __forceinline__ int sell_row(int k) {
+  return k ^ ((k >> 8) & (M - 1));
+}
+
+// stage_transposed with rows placed by sell_row<M>: s[sell_row(k) * TT + t].
+template <typename T, int TT, int M>
+__device__ __forceinline__ void stage_sliced(const T *__restrict__ in, int64_t T_, int W, int64_t t0, T *s) {
+  constexpr int V = 16 / (int)sizeof(T);
+  static_assert(256 % V == 0 && M <= 256, "the V columns of a chunk share their bits 8 and up");
+  const int chunks = W / V;
+  for (int it = threadIdx.x; it < chunks * TT; it += blockDim.x) {
+    const int t = it % TT;
+    const int c = it / TT;
+    const int64_t tg = t0 + t;
+    float v[V];
+    if (tg < T_) {
+      io<T>::unpack(*reinterpret_cast<const uint4 *>(in + tg * W + c * V), v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < V; ++i) v[i] = 0.f;
+    }
+    const int x = ((c * V) >> 8) & (M - 1);  // the same for the chunk's V columns
+#pragma unroll
+    for (int i = 0; i < V; ++i) io<T>::store1(s + (int64_t)((c * V + i) ^ x) * TT + t, v[i]);
+  }
+}
+
 // One warp per segment: its entries in the rotated round-robin order at the
 // positions of its slot, then the padding of the group. The slots of the last
 // group past n_seg (ranks n_seg .. n_pad - 1) are written as empty segments.
@@ -609,7 +645,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int m = 0; m < M; ++m) cnt[m] = 0;
     for (int j = s + lane; j < e; j += 32) {
-      const int r = (__ldg(idx + j) - r0) & (M - 1);
+      const int r = (sell_row<M>(__ldg(idx + j)) - r0) & (M - 1);
 #pragma unroll
       for (int m = 0; m < M; ++m) cnt[m] += r == m ? 1 : 0;
     }
@@ -626,7 +662,7 @@ __global__ void __launch_bounds__(256)
       float v = 0.f;
       if (j < e) {
         k = __ldg(idx + j);
-        r = (k - r0) & (M - 1);
+        r = (sell_row<M>(k) - r0) & (M - 1);
         if (perm) {
           const int32_t src = __ldg(perm + j);
           v = (unsigned)src < (unsigned)nnz ? __ldg(val + src) : 0.f;
@@ -649,7 +685,7 @@ __global__ void __launch_bounds__(256)
         int vb;
         if constexpr (sizeof(Tin) == 2) vb = (int)pack_bf16x2(v, v);
         else vb = __float_as_int(v);
-        if (t < steps) *at(t) = ok ? make_int2(k * TT * (int)sizeof(Tin), vb) : make_int2(0, 0);
+        if (t < steps) *at(t) = ok ? make_int2(sell_row<M>(k) * TT * (int)sizeof(Tin), vb) : make_int2(0, 0);
       }
     }
     for (int t = e - s + lane; t < steps; t += 32) *at(t) = make_int2(0, 0);  // none if e - s >= steps
@@ -692,10 +728,11 @@ __global__ void __launch_bounds__(kSpmmThreads)
   constexpr int NSLOT = 32 / Q;
   constexpr int kWarps = kSpmmThreads / 32;
   constexpr int U = kSellPairs;
+  constexpr int M = 128 / (TT * (int)sizeof(Tin));
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Tin *s_in = reinterpret_cast<Tin *>(smem_raw);
   const int64_t t0 = (int64_t)blockIdx.x * TT;
-  stage_transposed<Tin, TT>(in, T, W_in, t0, 0, W_in, W_in, s_in);
+  stage_sliced<Tin, TT, M>(in, T, W_in, t0, s_in);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int q = lane % Q, slot = lane / Q;
@@ -768,7 +805,8 @@ cudaError_t run_spmm_sliced(const void *in, int64_t T, int W_in, const int32_t *
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = ((size_t)W_in * TT * sizeof(Tin) + 15) & ~(size_t)15;
+  // rows rounded up to a whole block of M: sell_row may place a column of a partial last block past W_in
+  const size_t smem = (((size_t)W_in + M - 1) / M * M * TT * sizeof(Tin) + 15) & ~(size_t)15;
   auto k = sell_spmm_kernel<Tin, Tout, TT>;
   static bool attr_done[64] = {};
   const int slot = device_slot();
@@ -822,11 +860,12 @@ cudaError_t pick_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_pt
   const size_t row = (size_t)W_in * sizeof(Tin);
   // the sliced kernel stages the token tile alone (5 kernels: rank, place, offsets, arrange, product)
   *launched = 5;
-  if (row * 16 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 16, scratch_bytes))
+  const size_t rowr = ((size_t)W_in + 16) * sizeof(Tin);  // with the rows of a partial last block
+  if (rowr * 16 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 16, scratch_bytes))
     return run_spmm_sliced<Tin, Tout, 16>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
-  if (row * 16 > kSpmmSmemCap && row * 8 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
+  if (rowr * 16 > kSpmmSmemCap && rowr * 8 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
     return run_spmm_sliced<Tin, Tout, 8>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
-  if (row * 8 > kSpmmSmemCap && row * 4 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
+  if (rowr * 8 > kSpmmSmemCap && rowr * 4 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
     return run_spmm_sliced<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
   *launched = 2;  // arrange, product
   if (scratch_bytes < (size_t)(nnz > 0 ? nnz : 1) * 8) return cudaErrorInvalidValue;
