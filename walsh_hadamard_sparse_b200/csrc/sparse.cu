@@ -482,11 +482,13 @@ __host__ __device__ inline SellLayout sell_layout(int64_t p, int n_seg, int W_in
   return L;
 }
 
-// Rank of every segment by (length descending, index ascending): the number
-// of segments whose key is smaller, summed over chunks of kRankChunk keys
-// (grid.y) with integer atomics on a zeroed srank, so the result does not
-// depend on the order in which the chunks finish. Keys are unique (the index
-// is part of them), so the ranks are a permutation.
+// Rank of every segment within its window of ws consecutive segments (ws a
+// power of two and a multiple of the group size): window * ws plus the
+// number of segments of the window whose key (length descending, index
+// ascending) is smaller, summed over chunks of kRankChunk keys (grid.y) with
+// integer atomics on a zeroed srank, so the result does not depend on the
+// order in which the chunks finish. Keys are unique (the index is part of
+// them), so the ranks are a permutation that keeps every window in place.
 constexpr int kRankChunk = 1024;
 __device__ __forceinline__ uint32_t sell_key(const int32_t *__restrict__ seg_ptr, int i, int nnz) {
   int a = seg_ptr[i], b = seg_ptr[i + 1];
@@ -497,7 +499,8 @@ __device__ __forceinline__ uint32_t sell_key(const int32_t *__restrict__ seg_ptr
 }
 
 __global__ void __launch_bounds__(256)
-    sell_rank_kernel(const int32_t *__restrict__ seg_ptr, int n_seg, int64_t nnz64, int32_t *__restrict__ srank) {
+    sell_rank_kernel(const int32_t *__restrict__ seg_ptr, int n_seg, int64_t nnz64, int ws,
+                     int32_t *__restrict__ srank) {
   __shared__ __align__(16) uint32_t keys[kRankChunk];
   const int nnz = (int)nnz64;
   const int c0 = (int)blockIdx.y * kRankChunk;
@@ -506,13 +509,18 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   const int i = (int)blockIdx.x * 256 + (int)threadIdx.x;
   if (i >= n_seg) return;
+  const int w0 = i / ws * ws;  // this segment's window [w0, w0 + ws)
+  const int lo = (w0 > c0 ? w0 : c0) - c0, hi = (w0 + ws < c0 + n ? w0 + ws : c0 + n) - c0;
+  if (lo >= hi) return;  // the window does not meet this chunk
   const uint32_t mine = sell_key(seg_ptr, i, nnz);
   int cnt = 0;
-  const int n4 = (n + 3) / 4;
-  for (int j = 0; j < n4; ++j) {
+  // lo is a multiple of 4; the keys past n up to (hi + 3) / 4 * 4 are padding and compare false
+  for (int j = lo / 4; j < (hi + 3) / 4; ++j) {
     const uint4 k = reinterpret_cast<const uint4 *>(keys)[j];
     cnt += (k.x < mine) + (k.y < mine) + (k.z < mine) + (k.w < mine);
   }
+  // the window's base, added by the chunk that holds the window's start (which always meets it)
+  if (blockIdx.y == (unsigned)(w0 / kRankChunk)) cnt += w0;
   if (cnt) atomicAdd(srank + i, cnt);
 }
 
@@ -717,11 +725,17 @@ __device__ __forceinline__ void mac_sliced(const float *row, int vbits, float *a
 
 constexpr int kSellPairs = 4;  // step pairs per load batch (8 entries a slot)
 
+// Output staging of the sliced kernel: the CTA's window of ws output columns
+// for its TT tokens, fp32, row t at t * ws; a slot's two lanes (tokens t and
+// t + 8) would meet the same bank, so rows with bit 3 of t set have their
+// columns XORed with 16 (whole 16-byte chunks stay in place).
+__device__ __forceinline__ int sell_out_col(int t, int c) { return c ^ (((t >> 3) & 1) << 4); }
+
 template <typename Tin, typename Tout, int TT>
 __global__ void __launch_bounds__(kSpmmThreads)
     sell_spmm_kernel(const Tin *__restrict__ in, int64_t T, int W_in, const int4 *__restrict__ ent,
                      const int32_t *__restrict__ sseg, const int32_t *__restrict__ goff, int n_grp, int n_seg,
-                     float alpha, Tout *__restrict__ out) {
+                     int ws, float alpha, Tout *__restrict__ out) {
   static_assert(TT == 4 || TT == 8 || TT == 16, "token tile");
   constexpr int G = TT < 8 ? TT : 8;  // tokens per lane
   constexpr int Q = TT / G;           // lanes per slot
@@ -731,19 +745,23 @@ __global__ void __launch_bounds__(kSpmmThreads)
   constexpr int M = 128 / (TT * (int)sizeof(Tin));
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Tin *s_in = reinterpret_cast<Tin *>(smem_raw);
+  const size_t in_bytes = ((((size_t)W_in + M - 1) / M * M) * TT * sizeof(Tin) + 15) & ~(size_t)15;
+  float *s_out = reinterpret_cast<float *>(smem_raw + in_bytes);
   const int64_t t0 = (int64_t)blockIdx.x * TT;
+  const int w0 = (int)blockIdx.y * ws;  // this CTA's output columns [w0, w1)
+  const int w1 = w0 + ws < n_seg ? w0 + ws : n_seg;
+  const int g0 = w0 / NSLOT, g1 = (w1 + NSLOT - 1) / NSLOT;
   stage_sliced<Tin, TT, M>(in, T, W_in, t0, s_in);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int q = lane % Q, slot = lane / Q;
   const unsigned char *s_q = reinterpret_cast<const unsigned char *>(s_in) + (size_t)G * q * sizeof(Tin);
-  // groups (longest first) go to the gridDim.y CTAs of a token tile in turn, and within a CTA to
-  // its warps in snake order (round j: warp w, then warp kWarps - 1 - w), which evens out the
-  // warps' total steps
+  // the window's groups (longest first) go to the warps in snake order (round j: warp w, then warp
+  // kWarps - 1 - w), which evens out the warps' total steps
   for (int j = 0;; ++j) {
     const int local = (j & 1) ? kWarps - 1 - warp : warp;
-    const int g = (int)blockIdx.y + (int)gridDim.y * (kWarps * j + local);
-    if (g >= n_grp) break;
+    const int g = g0 + kWarps * j + local;
+    if (g >= g1) break;
     const int base = goff[g];
     const int npair = (goff[g + 1] - base) / (2 * NSLOT);
     // pair i of this slot: ent[(base / 2) + i * NSLOT + slot] as (offset, value) x 2
@@ -768,20 +786,48 @@ __global__ void __launch_bounds__(kSpmmThreads)
       for (int u = 0; u < U; ++u) cur[u] = nxt[u];
     }
     const int seg = sseg[(size_t)g * NSLOT + slot];
-    if (seg >= 0 && seg < n_seg) {
+    if (seg >= w0 && seg < w1) {
+      const int c = seg - w0;
 #pragma unroll
       for (int i = 0; i < G; ++i) {
-        const int64_t t = t0 + G * q + i;
-        if (t < T) io<Tout>::store1(out + t * n_seg + seg, alpha * acc[i]);
+        const int t = G * q + i;
+        s_out[t * ws + sell_out_col(t, c)] = alpha * acc[i];
       }
     }
   }
+  __syncthreads();
+  // the window's rows leave as 16-byte vectors (n_seg and ws are multiples of 8)
+  const int nv = (w1 - w0) / 4;  // 4-column chunks per row
+  for (int it = threadIdx.x; it < TT * nv; it += kSpmmThreads) {
+    const int t = it / nv, c4 = it % nv;
+    const int64_t tg = t0 + t;
+    if (tg >= T) continue;
+    const float4 v = *reinterpret_cast<const float4 *>(s_out + t * ws + sell_out_col(t, 4 * c4));
+    Tout *o = out + tg * n_seg + w0 + 4 * c4;
+    const float f[4] = {v.x, v.y, v.z, v.w};
+    store_vec<Tout, 4>(o, f);
+  }
+}
+
+// Output window of the sliced kernel: the largest power of two ws (>= 32, and
+// not beyond n_seg rounded up to a power of two) whose fp32 staging for TT
+// tokens fits in the shared memory left after the token tile; 0 if none.
+template <typename Tin, int TT>
+int sell_window(int W_in, int n_seg) {
+  constexpr int M = 128 / (TT * (int)sizeof(Tin));
+  const size_t in_bytes = ((((size_t)W_in + M - 1) / M * M) * TT * sizeof(Tin) + 15) & ~(size_t)15;
+  if (in_bytes >= kSpmmSmemCap) return 0;
+  const size_t room = (kSpmmSmemCap - in_bytes) / (TT * sizeof(float));
+  int ws = 32;
+  if ((size_t)ws > room) return 0;
+  while ((size_t)ws * 2 <= room && ws < n_seg) ws *= 2;
+  return ws;
 }
 
 template <typename Tin, typename Tout, int TT>
 cudaError_t run_spmm_sliced(const void *in, int64_t T, int W_in, const int32_t *seg_ptr, const int32_t *idx,
                             const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha,
-                            void *scratch, void *out, cudaStream_t s) {
+                            void *scratch, int ws, void *out, cudaStream_t s) {
   constexpr int G = TT < 8 ? TT : 8;
   constexpr int NSLOT = 32 / (TT / G);
   constexpr int M = 128 / (TT * (int)sizeof(Tin));  // staged rows per bank line
@@ -795,7 +841,7 @@ cudaError_t run_spmm_sliced(const void *in, int64_t T, int W_in, const int32_t *
   cudaError_t e = cudaMemsetAsync(srank, 0, (size_t)n_seg * 4, s);
   if (e != cudaSuccess) return e;
   sell_rank_kernel<<<dim3((unsigned)cdiv(n_seg, 256), (unsigned)cdiv(n_seg, kRankChunk)), 256, 0, s>>>(seg_ptr, n_seg,
-                                                                                                      nnz, srank);
+                                                                                                      nnz, ws, srank);
   sell_place_kernel<<<(unsigned)cdiv(n_pad, 256), 256, 0, s>>>(srank, n_seg, n_pad, sseg);
   sell_offsets_kernel<<<1, 1024, 0, s>>>(seg_ptr, sseg, L.n_grp, nnz, NSLOT, W_in, goff);
   {
@@ -805,8 +851,10 @@ cudaError_t run_spmm_sliced(const void *in, int64_t T, int W_in, const int32_t *
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // rows rounded up to a whole block of M: sell_row may place a column of a partial last block past W_in
-  const size_t smem = (((size_t)W_in + M - 1) / M * M * TT * sizeof(Tin) + 15) & ~(size_t)15;
+  // rows rounded up to a whole block of M (sell_row may place a column of a partial last block past
+  // W_in), then the output window
+  const size_t smem = ((((size_t)W_in + M - 1) / M * M) * TT * sizeof(Tin) + 15 & ~(size_t)15) +
+                      (size_t)TT * ws * sizeof(float);
   auto k = sell_spmm_kernel<Tin, Tout, TT>;
   static bool attr_done[64] = {};
   const int slot = device_slot();
@@ -815,11 +863,9 @@ cudaError_t run_spmm_sliced(const void *in, int64_t T, int W_in, const int32_t *
     if (e != cudaSuccess) return e;
     attr_done[slot] = true;
   }
-  const int64_t tiles = cdiv(T, TT);
-  // one CTA per SM: split the groups so that the token tiles fill whole waves
-  const dim3 grid((unsigned)tiles, (unsigned)wave_split(tiles, L.n_grp >= 4 * kSpmmThreads / 32 ? 4 : 1));
+  const dim3 grid((unsigned)cdiv(T, TT), (unsigned)cdiv(n_seg, ws));
   k<<<grid, kSpmmThreads, smem, s>>>(static_cast<const Tin *>(in), T, W_in, reinterpret_cast<const int4 *>(ent), sseg,
-                                     goff, L.n_grp, n_seg, alpha, static_cast<Tout *>(out));
+                                     goff, L.n_grp, n_seg, ws, alpha, static_cast<Tout *>(out));
   return cudaGetLastError();
 }
 
@@ -858,15 +904,19 @@ cudaError_t pick_spmm(const void *in, int64_t T, int W_in, const int32_t *seg_pt
                       const float *val, const int32_t *perm, int64_t nnz, int n_seg, float alpha, void *scratch,
                       size_t scratch_bytes, void *out, cudaStream_t s, int *launched) {
   const size_t row = (size_t)W_in * sizeof(Tin);
-  // the sliced kernel stages the token tile alone (5 kernels: rank, place, offsets, arrange, product)
+  // the sliced kernel stages the token tile and an output window (5 kernels: rank, place, offsets,
+  // arrange, product); the widest token tile with a window of at least 256 columns (or all of them)
   *launched = 5;
-  const size_t rowr = ((size_t)W_in + 16) * sizeof(Tin);  // with the rows of a partial last block
-  if (rowr * 16 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 16, scratch_bytes))
-    return run_spmm_sliced<Tin, Tout, 16>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
-  if (rowr * 16 > kSpmmSmemCap && rowr * 8 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
-    return run_spmm_sliced<Tin, Tout, 8>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
-  if (rowr * 8 > kSpmmSmemCap && rowr * 4 <= kSpmmSmemCap && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
-    return run_spmm_sliced<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, out, s);
+  auto fits = [&](int ws) { return ws >= 256 || (ws > 0 && ws >= n_seg); };
+  if (const int ws = sell_window<Tin, 16>(W_in, n_seg); fits(ws) && sliced_ok(nnz, n_seg, W_in, 16, scratch_bytes))
+    return run_spmm_sliced<Tin, Tout, 16>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, ws, out,
+                                          s);
+  if (const int ws = sell_window<Tin, 8>(W_in, n_seg); fits(ws) && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
+    return run_spmm_sliced<Tin, Tout, 8>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, ws, out,
+                                         s);
+  if (const int ws = sell_window<Tin, 4>(W_in, n_seg); fits(ws) && sliced_ok(nnz, n_seg, W_in, 32, scratch_bytes))
+    return run_spmm_sliced<Tin, Tout, 4>(in, T, W_in, seg_ptr, idx, val, perm, nnz, n_seg, alpha, scratch, ws, out,
+                                         s);
   *launched = 2;  // arrange, product
   if (scratch_bytes < (size_t)(nnz > 0 ? nnz : 1) * 8) return cudaErrorInvalidValue;
   int2 *ent = static_cast<int2 *>(scratch);
