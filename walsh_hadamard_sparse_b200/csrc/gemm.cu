@@ -60,7 +60,11 @@ constexpr int BM = 128, BN = 256;  // accumulator rows per CTA, tile columns
 constexpr int kGemmThreads = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int kEpiStride = 33;  // per-warp staging row (floats) of the sampled epilogue
-constexpr size_t kEpiSmem = 4 * 32 * kEpiStride * sizeof(float);
+// Columns (relative to the tile) of a row's entries that the sampled epilogue
+// fetches before the tile's accumulator is ready, one byte each per lane.
+constexpr int kSelMax = 16;
+static_assert(BN <= 256, "prefetched columns are bytes relative to the tile");
+constexpr size_t kEpiSmem = 4 * 32 * kEpiStride * sizeof(float) + 4 * 32 * kSelMax;
 // bf16 output: each epilogue warp stages its 32 x 32 block (2 KB) before the coalesced stores
 constexpr size_t kEpiBf16Smem = 4 * 2048;
 
@@ -540,22 +544,24 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int it = 0;
     float *my_stage = epi_stage + (warp - 2) * (kMode == kOutSampled ? 32 * kEpiStride : 512);
+    // this lane's prefetched entry columns (sampled output only)
+    uint8_t *my_sel = reinterpret_cast<uint8_t *>(epi_stage + 4 * 32 * kEpiStride) + ((warp - 2) * 32 + lane) * kSelMax;
     for (int unit = group_id; unit < num_units; unit += n_groups, ++it) {
       const int tile = unit % num_tiles;
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
-      if (*abort_flag) break;
-      if (!mbar_wait(tfull(buf), use & 1)) {
-        give_up(0x20u);
-        break;
-      }
-      tc_fence_after();
       int m_blk, n_blk;
       tile_coords(tile, m_blk, n_blk);
       const int row = m_blk * TM + (int)rank * BM + q * 32 + lane;
-      // sampled output: this row's CSR entries with column in [n0, n0 + BN)
+      // Sampled output: this row's CSR entries with column in [n0, n0 + BN), found while the tile's
+      // MMAs still run (the search and the column loads are dependent global reads): j is the first
+      // of them, and the columns of up to kSelMax of them, relative to n0, go to my_sel (nsel of
+      // them; when all kSelMax fall in the tile, `more` says the ones after are read in the chunk loop).
       int64_t j = 0, j_end = 0;
+      int nsel = 0;
+      bool more = false;
       if (kMode == kOutSampled && row < M) {
+        const int n0 = n_blk * BN;
         j = sa_args.row_ptr[row];
         j_end = sa_args.row_ptr[row + 1];
         if (j < 0) j = 0;
@@ -563,10 +569,27 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         int64_t hi = j_end;  // first entry with column >= n0 (columns ascend within a row)
         while (j < hi) {
           const int64_t mid = (j + hi) >> 1;
-          if (sa_args.col_idx[mid] < n_blk * BN) j = mid + 1;
+          if (sa_args.col_idx[mid] < n0) j = mid + 1;
           else hi = mid;
         }
+        int cols[kSelMax];
+#pragma unroll
+        for (int i = 0; i < kSelMax; ++i) cols[i] = j + i < j_end ? sa_args.col_idx[j + i] - n0 : BN;
+#pragma unroll
+        for (int i = 0; i < kSelMax; ++i) {
+          const bool in = (unsigned)cols[i] < (unsigned)BN;
+          my_sel[i] = in ? (uint8_t)cols[i] : (uint8_t)255;
+          nsel += in ? 1 : 0;
+        }
+        more = nsel == kSelMax;
       }
+      if (*abort_flag) break;
+      if (!mbar_wait(tfull(buf), use & 1)) {
+        give_up(0x20u);
+        break;
+      }
+      tc_fence_after();
+      int sel = 0;  // entries of the row already written: CSR positions j .. j + sel - 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
@@ -575,13 +598,22 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) my_stage[lane * kEpiStride + i] = __uint_as_float(r[i]);
           __syncwarp();
-          for (; j < j_end; ++j) {
-            const int k = sa_args.col_idx[j] - col0;
-            if (k >= 32) break;
-            if (k >= 0) {
-              const float v = sa_args.alpha * my_stage[lane * kEpiStride + k];
-              if (k_splits > 1) atomicAdd(sa_args.dc + j, v);
-              else sa_args.dc[j] = v;
+          const int hi = 32 * (c + 1);  // chunk c covers tile columns [32 c, hi)
+          auto put = [&](int o) {
+            const float v = sa_args.alpha * my_stage[lane * kEpiStride + (o - 32 * c)];
+            if (k_splits > 1) atomicAdd(sa_args.dc + j + sel, v);
+            else sa_args.dc[j + sel] = v;
+          };
+          for (; sel < nsel; ++sel) {
+            const int o = my_sel[sel];
+            if (o >= hi) break;
+            put(o);
+          }
+          if (more && sel >= nsel) {  // past the prefetched entries: the rest from global memory
+            for (; j + sel < j_end; ++sel) {
+              const int o = sa_args.col_idx[j + sel] - n_blk * BN;
+              if (o >= hi) break;
+              put(o);
             }
           }
           __syncwarp();

@@ -489,7 +489,7 @@ __host__ __device__ inline SellLayout sell_layout(int64_t p, int n_seg, int W_in
 // integer atomics on a zeroed srank, so the result does not depend on the
 // order in which the chunks finish. Keys are unique (the index is part of
 // them), so the ranks are a permutation that keeps every window in place.
-constexpr int kRankChunk = 1024;
+constexpr int kRankChunk = 256;  // keys per chunk: 4096 segments in 1024-wide windows give 64 busy CTAs
 __device__ __forceinline__ uint32_t sell_key(const int32_t *__restrict__ seg_ptr, int i, int nnz) {
   int a = seg_ptr[i], b = seg_ptr[i + 1];
   a = a < 0 ? 0 : (a > nnz ? nnz : a);
