@@ -59,12 +59,11 @@ namespace {
 constexpr int BM = 128, BN = 256;  // accumulator rows per CTA, tile columns
 constexpr int kGemmThreads = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
-constexpr int kEpiStride = 33;  // per-warp staging row (floats) of the sampled epilogue
 // Columns (relative to the tile) of a row's entries that the sampled epilogue
-// fetches before the tile's accumulator is ready, one byte each per lane.
+// fetches before the tile's accumulator is ready: one byte each, packed in
+// registers.
 constexpr int kSelMax = 16;
 static_assert(BN <= 256, "prefetched columns are bytes relative to the tile");
-constexpr size_t kEpiSmem = 4 * 32 * kEpiStride * sizeof(float) + 4 * 32 * kSelMax;
 // bf16 output: each epilogue warp stages its 32 x 32 block (2 KB) before the coalesced stores
 constexpr size_t kEpiBf16Smem = 4 * 2048;
 
@@ -100,7 +99,7 @@ struct Cfg {
   static constexpr int kBRows = BN / CG;  // rows of B this CTA loads
   static constexpr uint32_t kBBytes = kBRows * BK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr size_t kEpiBytes = kMode == kOutSampled ? kEpiSmem : (kMode == kOutBf16 ? kEpiBf16Smem : 0);
+  static constexpr size_t kEpiBytes = kMode == kOutBf16 ? kEpiBf16Smem : 0;
   static constexpr size_t kZOffset = (size_t)kStages * kStageBytes + 256 + kEpiBytes;  // from the aligned base
   static constexpr size_t kSmem = kZOffset + 1024 + z_smem<kZ>();
   static constexpr int kThreads = kGemmThreads + (kZ ? kZThreads : 0);
@@ -362,6 +361,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
 // many parts, each part a separate work unit adding its share into dc. Units
 // are numbered part-major (unit = part * tiles + tile), so the units running
 // at the same time read the same part of K and share it in L2.
+// r[k] for a run-time k in [0, 32): a tree of selects over the index bits, so
+// the registers are only indexed at compile time (no local or shared memory).
+__device__ __forceinline__ uint32_t pick32(const uint32_t (&r)[32], int k) {
+  uint32_t a[16], b[8], c[4], d[2];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a[i] = (k & 1) ? r[2 * i + 1] : r[2 * i];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = (k & 2) ? a[2 * i + 1] : a[2 * i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = (k & 4) ? b[2 * i + 1] : b[2 * i];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) d[i] = (k & 8) ? c[2 * i + 1] : c[2 * i];
+  return (k & 16) ? d[1] : d[0];
+}
+
 template <int kMode, int CG, int kZ>
 __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -543,9 +557,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     // ------------------------------------------------ epilogue (every CTA)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int it = 0;
-    float *my_stage = epi_stage + (warp - 2) * (kMode == kOutSampled ? 32 * kEpiStride : 512);
-    // this lane's prefetched entry columns (sampled output only)
-    uint8_t *my_sel = reinterpret_cast<uint8_t *>(epi_stage + 4 * 32 * kEpiStride) + ((warp - 2) * 32 + lane) * kSelMax;
+    float *my_stage = epi_stage + (warp - 2) * 512;
     for (int unit = group_id; unit < num_units; unit += n_groups, ++it) {
       const int tile = unit % num_tiles;
       const int buf = it & 1;
@@ -555,11 +567,14 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
       const int row = m_blk * TM + (int)rank * BM + q * 32 + lane;
       // Sampled output: this row's CSR entries with column in [n0, n0 + BN), found while the tile's
       // MMAs still run (the search and the column loads are dependent global reads): j is the first
-      // of them, and the columns of up to kSelMax of them, relative to n0, go to my_sel (nsel of
-      // them; when all kSelMax fall in the tile, `more` says the ones after are read in the chunk loop).
+      // of them, and the columns of up to kSelMax of them, relative to n0, are packed four to a
+      // register in selw (nsel of them; when all kSelMax fall in the tile, `more` says the ones after
+      // are read in the chunk loop). The epilogue then touches no shared memory, whose bandwidth the
+      // copies and the MMAs of the next tile are using.
       int64_t j = 0, j_end = 0;
       int nsel = 0;
       bool more = false;
+      uint32_t selw[kSelMax / 4] = {};
       if (kMode == kOutSampled && row < M) {
         const int n0 = n_blk * BN;
         j = sa_args.row_ptr[row];
@@ -578,7 +593,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kSelMax; ++i) {
           const bool in = (unsigned)cols[i] < (unsigned)BN;
-          my_sel[i] = in ? (uint8_t)cols[i] : (uint8_t)255;
+          selw[i / 4] |= (in ? (uint32_t)cols[i] : 255u) << (8 * (i % 4));
           nsel += in ? 1 : 0;
         }
         more = nsel == kSelMax;
@@ -595,17 +610,15 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
         const int col0 = n_blk * BN + c * 32;
         if (kMode == kOutSampled) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) my_stage[lane * kEpiStride + i] = __uint_as_float(r[i]);
-          __syncwarp();
           const int hi = 32 * (c + 1);  // chunk c covers tile columns [32 c, hi)
           auto put = [&](int o) {
-            const float v = sa_args.alpha * my_stage[lane * kEpiStride + (o - 32 * c)];
+            const float v = sa_args.alpha * __uint_as_float(pick32(r, o & 31));
             if (k_splits > 1) atomicAdd(sa_args.dc + j + sel, v);
             else sa_args.dc[j + sel] = v;
           };
           for (; sel < nsel; ++sel) {
-            const int o = my_sel[sel];
+            const uint32_t w = sel < 8 ? (sel < 4 ? selw[0] : selw[1]) : (sel < 12 ? selw[2] : selw[3]);
+            const int o = (int)((w >> (8 * (sel & 3))) & 255u);
             if (o >= hi) break;
             put(o);
           }
@@ -616,7 +629,6 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
               put(o);
             }
           }
-          __syncwarp();
           continue;
         }
         if (kMode == kOutBf16 && !addend && col0 + 32 <= N) {
