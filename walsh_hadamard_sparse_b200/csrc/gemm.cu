@@ -57,7 +57,6 @@ namespace qwha {
 namespace {
 
 constexpr int BM = 128, BN = 256;  // accumulator rows per CTA, tile columns
-constexpr int kGemmThreads = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 // Columns (relative to the tile) of a row's entries that the sampled epilogue
 // fetches before the tile's accumulator is ready: one byte each, packed in
@@ -68,6 +67,14 @@ static_assert(BN <= 256, "prefetched columns are bytes relative to the tile");
 constexpr size_t kEpiBf16Smem = 4 * 2048;
 
 enum { kOutBf16 = 0, kOutF32 = 1, kOutSampled = 2 };
+
+// Epilogue warps per CTA: one per TMEM lane quarter, or, for the sampled
+// output, two, each draining half of the tile's columns (its per-entry work
+// makes its epilogue the longest, and the last tile's is hidden behind no MMA:
+// 186.8 -> 182.6 us on q_proj). Two per quarter slowed the other outputs (the
+// fused forward by 3 us; the bf16 output with an fp32 addend by 18 us).
+template <int kMode>
+constexpr int epi_warps() { return kMode == kOutSampled ? 8 : 4; }
 
 // Extra warps of the fused forward: they transform rows of X (Z = X H, bf16,
 // blocks of 2^kZ) while the other warps run the GEMM.
@@ -102,6 +109,8 @@ struct Cfg {
   static constexpr size_t kEpiBytes = kMode == kOutBf16 ? kEpiBf16Smem : 0;
   static constexpr size_t kZOffset = (size_t)kStages * kStageBytes + 256 + kEpiBytes;  // from the aligned base
   static constexpr size_t kSmem = kZOffset + 1024 + z_smem<kZ>();
+  static constexpr int kEpiWarps = epi_warps<kMode>();
+  static constexpr int kGemmThreads = 64 + 32 * kEpiWarps;  // producer warp, MMA warp, epilogue warps
   static constexpr int kThreads = kGemmThreads + (kZ ? kZThreads : 0);
   // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (7-9 = 1),
   // B bf16 (10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
@@ -351,16 +360,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// kF32Out: write fp32 D (no rounding); otherwise bf16. addend may be NULL.
-// a_ld / b_ld: how the operand's stage is filled (kLd*): K-major in global
-// memory ([M or N rows][K contiguous]) or MN-major ([K rows][M or N
-// contiguous]); a stage holds slabs of 128-byte rows (64 K per slab along K
-// for K-major, BK K rows per slab of 64 MN for MN-major), filled by one 3-D
-// copy when the slab dimension divides evenly, else by one 2-D copy per slab.
-// k_splits > 1 (sampled output only): each tile's K range is cut into that
-// many parts, each part a separate work unit adding its share into dc. Units
-// are numbered part-major (unit = part * tiles + tile), so the units running
-// at the same time read the same part of K and share it in L2.
 // r[k] for a run-time k in [0, 32): a tree of selects over the index bits, so
 // the registers are only indexed at compile time (no local or shared memory).
 __device__ __forceinline__ uint32_t pick32(const uint32_t (&r)[32], int k) {
@@ -376,6 +375,16 @@ __device__ __forceinline__ uint32_t pick32(const uint32_t (&r)[32], int k) {
   return (k & 16) ? d[1] : d[0];
 }
 
+// kF32Out: write fp32 D (no rounding); otherwise bf16. addend may be NULL.
+// a_ld / b_ld: how the operand's stage is filled (kLd*): K-major in global
+// memory ([M or N rows][K contiguous]) or MN-major ([K rows][M or N
+// contiguous]); a stage holds slabs of 128-byte rows (64 K per slab along K
+// for K-major, BK K rows per slab of 64 MN for MN-major), filled by one 3-D
+// copy when the slab dimension divides evenly, else by one 2-D copy per slab.
+// k_splits > 1 (sampled output only): each tile's K range is cut into that
+// many parts, each part a separate work unit adding its share into dc. Units
+// are numbered part-major (unit = part * tiles + tile), so the units running
+// at the same time read the same part of K and share it in L2.
 template <int kMode, int CG, int kZ>
 __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -412,7 +421,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull(b), 1);
-      mbar_init(tempty(b), 4 * CG);  // the epilogue warps of every CTA of the group
+      mbar_init(tempty(b), C::kEpiWarps * CG);  // the epilogue warps of every CTA of the group
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -545,17 +554,21 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
     // drain: all issued MMAs complete before TMEM is released
     umma_commit_local<CG>(done_bar);
     if (!mbar_wait(done_bar, 0)) give_up(0x10u);
-  } else if (kZ && warp >= 6) {
+  } else if (kZ && warp >= C::kGemmThreads / 32) {
     // ------------------------------------------------ fused transform Z = X H (every CTA)
     if constexpr (kZ != 0) {
       float *zs = reinterpret_cast<float *>(smem + C::kZOffset);
       fwht_rows_body<kZ, 8, __nv_bfloat16, __nv_bfloat16, kZThreads>(
-          za.x, za.z, za.rows, za.scale, zs, (int)threadIdx.x - kGemmThreads, blockIdx.x, gridDim.x,
+          za.x, za.z, za.rows, za.scale, zs, (int)threadIdx.x - C::kGemmThreads, blockIdx.x, gridDim.x,
           [] { asm volatile("bar.sync 1, %0;" ::"n"(kZThreads) : "memory"); });
     }
   } else if (warp >= 2) {
     // ------------------------------------------------ epilogue (every CTA)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // which half of the tile's columns this warp drains (warps 2-5 and 6-9 cover the four quarters)
+    const int half = (warp - 2) / 4;
+    constexpr int kChunks = BN / 32 / (C::kEpiWarps / 4);  // 32-column chunks per warp
+    static_assert(C::kEpiWarps == 4 || C::kEpiWarps == 8, "one or two warps per lane quarter");
     int it = 0;
     float *my_stage = epi_stage + (warp - 2) * 512;
     for (int unit = group_id; unit < num_units; unit += n_groups, ++it) {
@@ -576,15 +589,16 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
       bool more = false;
       uint32_t selw[kSelMax / 4] = {};
       if (kMode == kOutSampled && row < M) {
-        const int n0 = n_blk * BN;
+        const int n0 = n_blk * BN;                 // offsets stay relative to the tile
+        const int c0 = half * kChunks * 32;        // this warp's columns: [n0 + c0, n0 + c0 + 32 kChunks)
         j = sa_args.row_ptr[row];
         j_end = sa_args.row_ptr[row + 1];
         if (j < 0) j = 0;
         if (j_end > sa_args.p) j_end = sa_args.p;
-        int64_t hi = j_end;  // first entry with column >= n0 (columns ascend within a row)
+        int64_t hi = j_end;  // first entry with column >= n0 + c0 (columns ascend within a row)
         while (j < hi) {
           const int64_t mid = (j + hi) >> 1;
-          if (sa_args.col_idx[mid] < n0) j = mid + 1;
+          if (sa_args.col_idx[mid] < n0 + c0) j = mid + 1;
           else hi = mid;
         }
         int cols[kSelMax];
@@ -592,7 +606,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         for (int i = 0; i < kSelMax; ++i) cols[i] = j + i < j_end ? sa_args.col_idx[j + i] - n0 : BN;
 #pragma unroll
         for (int i = 0; i < kSelMax; ++i) {
-          const bool in = (unsigned)cols[i] < (unsigned)BN;
+          const bool in = (unsigned)(cols[i] - c0) < (unsigned)(32 * kChunks);
           selw[i / 4] |= (in ? (uint32_t)cols[i] : 255u) << (8 * (i % 4));
           nsel += in ? 1 : 0;
         }
@@ -605,7 +619,7 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
       }
       tc_fence_after();
       int sel = 0;  // entries of the row already written: CSR positions j .. j + sel - 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
         const int col0 = n_blk * BN + c * 32;
