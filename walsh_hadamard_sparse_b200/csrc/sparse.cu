@@ -1,17 +1,21 @@
 // Sparse products of the adapter with F = Scatter(c, E) ("QWHA",
 // papernotes.org 整体框架; gist.science 2.1).
 //
-// seg_spmm: out[t, i] = alpha * sum_{j in segment i} val[j] * in[t, idx[j]].
+// SpMM: out[t, i] = alpha * sum_{j in segment i} val[j] * in[t, idx[j]].
 //   Forward (segments = rows of F, CSR):  Y_ad = alpha Z F^T.
 //   Backward (segments = columns of F, CSC, val through perm): dZ = alpha dY F.
-//   One CTA owns TT tokens: their input rows are staged transposed in shared
-//   memory as s_in[k][TT] (a column of the tile is TT contiguous values), then
-//   each warp runs one segment at a time (see seg_spmm_kernel). The segment
-//   entries stream from L2 once per token tile, as packed (index, value)
-//   words that arrange_kernel writes first: it orders each segment so that
-//   the rows one shared-memory wavefront gathers sit on distinct banks as far
-//   as the indices allow, and for the backward applies the CSC permutation
-//   to the coefficients.
+//   A CTA owns TT tokens: their input rows are staged transposed in shared
+//   memory (a column of the tile is TT contiguous values). The segment
+//   entries stream from L2 once per token tile, as packed (staged-row,
+//   value) words that a preparation kernel writes first, ordered so that the
+//   rows one shared-memory wavefront gathers sit on distinct banks as far as
+//   the indices allow, with the CSC permutation applied to the coefficients
+//   for the backward.
+//   sell_spmm_kernel (the sliced layout, see the section that defines it): a
+//   slot owns a whole segment; segments are ranked by length within windows
+//   of output columns, whose results the CTA writes as whole rows.
+//   seg_spmm_kernel (shapes the sliced layout does not take): a warp spreads
+//   one segment at a time over its slots and reduces across them at the end.
 //
 // sddmm: partial[c, j] = sum_{t in chunk c} dY[t, r_j] * Z[t, k_j] over the
 //   tile view of E (QWHA_TILE x QWHA_TILE blocks of F). Grid = tiles x token
