@@ -573,3 +573,52 @@ def test_token_shards_give_the_same_rows_bitwise(algo):
         torch.cuda.synchronize()
         for name, part, whole in (("Z", Zs, Z), ("Y", Ys, Y), ("dX", dXs, dX)):
             assert torch.equal(part.view(torch.int16), whole[lo:hi].view(torch.int16)), (name, lo, hi)
+
+
+# Shapes for the sliced SpMM's layouts (sparse algorithm): the 8-token tile (rows too wide for 16
+# tokens: 8192 bf16 or 4096 fp32 columns) and output windows whose last one is partial (the kernel
+# ranks segments within windows of 1024 or 2048 output columns, 32- or 16-segment groups).
+SLICED_CASES = [
+    # d_in, d_out, n, T, p per row, dtype
+    (8192, 2600, 4096, 50, 20, "bf16"),  # forward: 8-token tile, windows 2048 + 552; gather: 4 windows
+    (4096, 4616, 4096, 40, 24, "bf16"),  # forward: 16-token tile, windows 4 x 1024 + 520
+    (4096, 3000, 2048, 30, 16, "f32"),  # fp32 forward: 8-token tile, windows 2048 + 952
+]
+
+
+@pytest.mark.parametrize("d_in,d_out,n,T,per_row,dtype", SLICED_CASES)
+def test_sliced_spmm_tiles_and_windows(d_in, d_out, n, T, per_row, dtype):
+    """Y, dX (the SpMM and the CSC gather) and dc of the sparse algorithm against the oracle at shapes that reach
+    the 8-token tile and partial output windows, with rows of uneven length (so that the length ranking and
+    the group padding matter) and a few empty and full rows."""
+    import torch
+
+    W = _W()
+    g = rng_for(37, "sliced", d_in, d_out, T, dtype)
+    counts = g.integers(per_row // 4, 2 * per_row, d_out)
+    counts[::97] = 0
+    counts[5] = d_in
+    rp, ci, cf = random_pattern(d_out, d_in, counts=counts, rng=g)
+    X = g.standard_normal((T, d_in)).astype(np.float32)
+    dY = g.standard_normal((T, d_out)).astype(np.float32)
+    if dtype == "bf16":
+        X, dY = bf16_bits_to_f32(f32_to_bf16_bits(X)), bf16_bits_to_f32(f32_to_bf16_bits(dY))
+    a = device_adapter(d_in, d_out, n, rp, ci, cf)
+    alpha = 0.7
+    Xd, dYd = dev_act(X, dtype), dev_act(dY, dtype)
+    Z, Y = W.adapter_fwd(a, Xd, alpha)
+    dc, dX = W.adapter_bwd(a, dYd, Z, alpha)
+    torch.cuda.synchronize()
+    _, Yr = oracle.adapter_fwd(rp, ci, cf, X, d_out, n, alpha, want_z=False)
+    dXr = oracle.adapter_bwd_dx(rp, ci, cf, dY, d_in, n, alpha)
+    rows = oracle.csr_rows(rp)
+    sel = np.sort(rng_for(38, "sliced-dc").choice(ci.size, min(ci.size, 3000), replace=False))
+    dcr = oracle.adapter_bwd_dc(X, dY, rows[sel], ci[sel], n, alpha)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    errs = dict(Y=rel_fro(host(Y), Yr), dX=rel_fro(host(dX), dXr), dc=rel_fro(dc.cpu().numpy()[sel], dcr))
+    assert all(v <= tol for v in errs.values()), errs
+    # every output column, the empty rows' zeros included, against the oracle column by column
+    Yh = host(Y)
+    assert np.abs(Yh[:, counts == 0]).max() == 0.0
+    col_err = np.abs(Yh - Yr).max(axis=0) / (np.abs(Yr).max() + 1e-30)
+    assert col_err.max() <= (1e-5 if dtype == "f32" else 4e-2), (int(col_err.argmax()), float(col_err.max()))
