@@ -77,8 +77,11 @@ template <int kMode>
 constexpr int epi_warps() { return kMode == kOutSampled ? 8 : 4; }
 
 // Extra warps of the fused forward: they transform rows of X (Z = X H, bf16,
-// blocks of 2^kZ) while the other warps run the GEMM.
-constexpr int kZThreads = 128;
+// blocks of 2^kZ) while the other warps run the GEMM. Two warps (one 4096-point
+// row at a time) keep up with the GEMM on q_proj and leave room for three
+// 128-deep stages: 182.8 us against 184.9 us with four warps and five 64-deep
+// stages (two 128-deep stages with four warps: 225 us).
+constexpr int kZThreads = 64;
 template <int kZ>
 constexpr size_t z_smem() {
   if constexpr (kZ == 0) return 0;
@@ -98,10 +101,10 @@ __host__ __device__ constexpr bool ld_mn(int mode) { return mode == kLdMn2d || m
 
 template <int CG, int kMode = kOutBf16, int kZ = 0>
 struct Cfg {
-  // k-block depth: 128 for the CTA pair (half the copies and barrier rounds per MMA of 64), 64 when the fused
-  // transform's buffers or the single CTA's 256-row B leave room for too few 128-deep stages
-  static constexpr int BK = (CG == 2 && kZ == 0) ? 128 : 64;
-  static constexpr int kStages = CG == 1 ? 4 : (kZ ? 5 : 3);
+  // k-block depth: 128 for the CTA pair (half the copies and barrier rounds per MMA of 64), 64 when the single
+  // CTA's 256-row B leaves room for too few 128-deep stages
+  static constexpr int BK = CG == 2 ? 128 : 64;
+  static constexpr int kStages = CG == 1 ? 4 : 3;
   static constexpr uint32_t kABytes = BM * BK * 2;
   static constexpr int kBRows = BN / CG;  // rows of B this CTA loads
   static constexpr uint32_t kBBytes = kBRows * BK * 2;
@@ -483,11 +486,11 @@ __global__ void __launch_bounds__(Cfg<CG, kMode, kZ>::kThreads, 1)
         const uint32_t fb = CG == 2 ? peer_addr(full(stage), 0) : full(stage);
         const uint32_t sa = base + stage * C::kStageBytes, sb = sa + C::kABytes;
         if constexpr (kZ != 0) {
-          // The fused forward reads both operands K-major in 64-deep blocks. Its binary holds only
-          // this path: with the generic one compiled in as well, the launch (four warp roles, the
-          // transform's unrolled butterflies among them) ran ~10% slower.
-          tma_load_2d<CG>(sa, &tmA, fb, kb * BK, a_row);
-          tma_load_2d<CG>(sb, &tmB, fb, kb * BK, b_row);
+          // The fused forward reads both operands K-major, each stage in one 3-D copy. Its binary
+          // holds only this path: with the generic one compiled in as well, the launch (four warp
+          // roles, the transform's unrolled butterflies among them) ran ~10% slower.
+          tma_load_3d<CG>(sa, &tmA, fb, 0, a_row, kb * (BK / 64));
+          tma_load_3d<CG>(sb, &tmB, fb, 0, b_row, kb * (BK / 64));
         } else {
           load_stage<CG, BK>(sa, &tmA, fb, a_ld, a_row, BM, kb);
           load_stage<CG, BK>(sb, &tmB, fb, b_ld, b_row, C::kBRows, kb);
@@ -846,6 +849,9 @@ cudaError_t launch_gemm_cg(const void *A, const void *B, const float *addend, vo
       default: return make_map(t, P, MN, K, rows);
     }
   };
+  // the fused forward's producer issues only 3-D K-major copies (its K, d_in, is a whole number of 2048-point
+  // blocks)
+  if (kZ && (a_ld != kLdK3d || b_ld != kLdK3d)) return cudaErrorNotSupported;
   if (!map(&ta, A, a_ld, M, BM) || !map(&tb, B, b_ld, N, C::kBRows)) return cudaErrorInvalidValue;
   auto kern = gemm_bf16_tcgen05_kernel<kMode, CG, kZ>;
   static bool attr[64] = {};  // per device
