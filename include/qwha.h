@@ -162,10 +162,11 @@ qwha_status qwha_fwht(qwha_dtype dt, const void *x, void *z, int64_t rows, int32
  * a->algo == QWHA_ALGO_DENSE, dt must be QWHA_BF16. X, Z_out, Y are device
  * buffers; a->row_ptr/col_idx/coef are required, the other views are not
  * read. T >= 0 (T = 0 does nothing). ws: qwha_workspace_size(QWHA_OP_FWD,
- * ...) bytes for the sparse algorithm (it holds the entries of E ordered for
- * the gather, 8 bytes each, and with wq the fp32 adapter term and the
- * dequantized weight), QWHA_OP_FWD_DENSE for the dense one (W_eff, unless
- * a->weff is given). */
+ * ...) bytes for the sparse algorithm (it holds the entries of E in the order
+ * the SpMM reads them, 8 bytes each with the padding of the groups of
+ * segments, the segments' ranking by length, and with wq the fp32 adapter
+ * term and the dequantized weight), QWHA_OP_FWD_DENSE for the dense one
+ * (W_eff, unless a->weff is given). */
 qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt,
                              const void *X, int64_t T, float alpha, void *Z_out, void *Y,
                              void *ws, size_t ws_bytes, void *stream);
@@ -179,7 +180,9 @@ qwha_status qwha_adapter_fwd(const qwha_adapter *a, const qwha_qweight *wq, qwha
  * data-parallel caller computes dc first, starts its all-reduce, then dX; the
  * results are the same as from one call). Every reduction runs in a fixed
  * order: results are bitwise reproducible. ws: qwha_workspace_size(QWHA_OP_BWD
- * or QWHA_OP_BWD_DENSE, ...) bytes. */
+ * or QWHA_OP_BWD_DENSE, ...) bytes (for the sparse algorithm: the partial sums
+ * of dc, the transposed dY and Z of the coefficient gradient, which dZ reuses
+ * afterwards, and the gather's entries). */
 qwha_status qwha_adapter_bwd(const qwha_adapter *a, const qwha_qweight *wq, qwha_dtype dt,
                              const void *dY, const void *Z, int64_t T, float alpha, float *dc,
                              void *dX, void *ws, size_t ws_bytes, void *stream);
