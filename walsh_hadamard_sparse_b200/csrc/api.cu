@@ -288,7 +288,6 @@ struct Carver {  // hands out 256-byte aligned slices of the caller's workspace
   }
 };
 
-size_t esize(qwha_dtype d) { return d == QWHA_F32 ? 4 : 2; }
 
 qwha_status check_adapter_shape(const qwha_adapter *a) {
   if (!a) return fail(QWHA_ERR_INVALID_ARG, "adapter is NULL");
@@ -361,7 +360,6 @@ size_t fwd_ws(int32_t d_out, int32_t d_in, int64_t p, int64_t T, bool base) {
 
 size_t fwd_dense_ws(int32_t d_out, int32_t d_in) { return align_up((size_t)d_out * d_in * 2, 256); }
 
-int64_t pad8(int64_t v) { return (v + 7) / 8 * 8; }
 
 size_t bwd_dense_ws(int32_t d_out, int32_t d_in, int64_t T) {
   (void)T;
