@@ -82,9 +82,10 @@ def test_host_checks_of_init_variants_and_refinement():
 
 
 def test_sparse_forward_needs_entry_workspace():
-    """The sparse products write their (index, value) pairs, ordered for the shared-memory gather, into the caller's
-    workspace (8 bytes per coefficient), so the adapter-only sparse forward needs a workspace too; without one it is
-    refused on the host, before any CUDA call (no GPU needed)."""
+    """The sparse products write their (staged-row, value) pairs, ordered for the shared-memory gather, into the
+    caller's workspace (8 bytes per coefficient, plus the padding of the groups of segments), so the adapter-only
+    sparse forward needs a workspace too; without one it is refused on the host, before any CUDA call (no GPU
+    needed)."""
     _ensure_built()
     import walsh_hadamard_sparse_b200._lib as L
 
@@ -113,3 +114,24 @@ def test_debug_hooks_round_trip_on_the_host():
     h.qwha_debug_fail_cuda_checks(3)
     h.qwha_debug_fail_cuda_checks(0)
     assert h.qwha_fwht(0, None, None, 4, 256, 3, None) == 1  # host checks are not CUDA checks: unaffected
+
+
+def test_sparse_workspace_covers_the_sliced_layout_and_the_transposes():
+    """The sizes qwha_workspace_size reports cover the worst case of what the sparse kernels place there (no GPU):
+    the sliced SpMM's entries (every group of 16 or 32 segments padded to its longest segment, at most the
+    coefficients plus 32 entries per column of the row width, plus one step a group) and ranking tables, and in the
+    backward the transposed dY and Z of the coefficient gradient (bf16, tokens rounded up to 64), which share a
+    region with dZ."""
+    _ensure_built()
+    import walsh_hadamard_sparse_b200._lib as L
+
+    h = L.lib()
+    for d_out, d_in, p, T in ((2600, 8192, 65100, 50), (4616, 4096, 125296, 40), (64, 4096, 3, 1), (4096, 64, 4096, 129)):
+        fwd = h.qwha_workspace_size(0, d_out, d_in, p, T, 0)
+        bwd = h.qwha_workspace_size(1, d_out, d_in, p, T, 0)
+        ent_fwd = 8 * (p + 32 * (d_in + 2) + 32 * ((d_out + 15) // 16))  # forward: segments are rows, width d_in
+        ent_bwd = 8 * (p + 32 * (d_out + 2) + 32 * ((d_in + 15) // 16))  # gather: segments are columns, width d_out
+        assert fwd >= max(ent_fwd, ent_bwd), (d_out, d_in)
+        t64 = (T + 63) // 64 * 64
+        region = max(4 * T * d_in, 2 * (d_out + d_in) * t64)  # dZ, or before it the transposed dY and Z
+        assert bwd >= 16 * p * 4 + region + max(ent_fwd, ent_bwd), (d_out, d_in)
